@@ -1,0 +1,386 @@
+"""fp64 CPU oracle for the fused attention forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU
+baseline and ``--impl reference`` arm) may import this module. The library
+never calls it; the two share no code.
+
+What it computes is the plain definition, two passes per query row, no
+tiling, no online recurrence:
+
+  S      = scale * Q K^T                       (CANN "flash_attn", 计算公式;
+                                                MindSpore "sparse_flash_attention",
+                                                formula; ``scale_value``)
+  M      = max_{j visible} S_j
+  m      = max(sink, M)     if a sink is given (CANN "flash_attn", 计算公式,
+                                                the sink variant)
+  O      = sum_j e^{S_j - m} V_j / (sum_j e^{S_j - m} + e^{sink - m})
+  LSE    = M + ln sum_j e^{S_j - M}            (CANN "flash_attn", 计算公式,
+                                                the softmax_lse definition, and
+                                                the ``softmax_lse`` output note)
+
+Readings taken where the pages are silent or ambiguous:
+
+* LSE excludes the sink: the softmax_lse formula is written over S alone.
+* The causal mask is bottom-right aligned (MindSpore "sparse_flash_attention",
+  ``sparse_mode=3`` "rightDownCausal"): with delta = L_k - L_q, key j is
+  visible to query i iff j <= i + delta.
+* A sliding window (left, right) keeps i+delta-left <= j <= i+delta+right,
+  bounds inclusive, -1 = unbounded (MindSpore Lite "flash_attention",
+  ``window_size=(-1, -1)``; MindSpore "sparse_flash_attention",
+  ``pre_tokens`` / ``next_tokens``). causal is the same as right = 0.
+* GQA: query head h reads KV head floor(h / (H_q / H_kv)) (contiguous groups).
+* A row that sees no key gives O = 0 and LSE = -inf, with or without a sink.
+* FP8 inputs are decoded exactly and multiplied by their fp32 descale of
+  shape (B, H_kv) (MATE "Attention", FMHA dtype notes).
+* MLA: the 576-wide row is [512 latent | 64 rope] and V is its first 512
+  entries (MindSpore "sparse_flash_attention", ``attention_mode=2``; MATE
+  "Attention", MLA example with ``head_dim_v=512``).
+* Sparse: the visible set is the listed logical positions that are
+  >= 0 and < cache_seqlens[b]; others are skipped.
+* Combine (MATE "Attention", FMHA notes on ``flash_attn_combine``; no formula
+  is printed): LSE = ln sum_s e^{LSE_s}, O = sum_s e^{LSE_s - LSE} O_s for
+  sink-free partials; the sink is applied once afterwards as
+  O <- O / (1 + e^{sink - LSE}).
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against
+library routines (torch's fp64 scaled_dot_product_attention, logsumexp,
+tril/triu, float8 conversions), closed forms and invariants.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+NEG_INF = -math.inf
+
+
+# ---------------------------------------------------------------------------
+# Number formats, decoded from their definitions
+# ---------------------------------------------------------------------------
+
+def decode_bf16(bits: np.ndarray) -> np.ndarray:
+    """bfloat16 is the upper half of an IEEE-754 binary32: widen the 16 bits
+    into the high half of a 32-bit word and read it as binary32."""
+    b = np.asarray(bits).astype(np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def decode_fp16(bits: np.ndarray) -> np.ndarray:
+    """IEEE-754 binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits."""
+    b = np.asarray(bits).astype(np.uint16).astype(np.int64)
+    sign = np.where(b >> 15, -1.0, 1.0)
+    e = (b >> 10) & 0x1F
+    f = (b & 0x3FF).astype(np.float64)
+    normal = sign * np.ldexp(1.0 + f / 1024.0, (e - 15).astype(np.int64))
+    sub = sign * np.ldexp(f / 1024.0, -14)
+    special = np.where(f == 0, sign * np.inf, np.nan)
+    return np.where(e == 0, sub, np.where(e == 31, special, normal))
+
+
+def decode_e4m3(bits: np.ndarray) -> np.ndarray:
+    """OCP 8-bit E4M3 ("fn"): 1 sign, 4 exponent bits (bias 7), 3 mantissa
+    bits; no infinities; S.1111.111 is NaN; largest finite value 448;
+    exponent field 0 encodes subnormals m/8 * 2^-6."""
+    b = np.asarray(bits).astype(np.uint8).astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    normal = sign * np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64))
+    sub = sign * np.ldexp(m / 8.0, -6)
+    val = np.where(e == 0, sub, normal)
+    return np.where((e == 15) & ((b & 0x7) == 7), np.nan, val)
+
+
+def decode_e5m2(bits: np.ndarray) -> np.ndarray:
+    """OCP 8-bit E5M2: 1 sign, 5 exponent bits (bias 15), 2 mantissa bits,
+    IEEE-style infinities and NaNs at exponent 31."""
+    b = np.asarray(bits).astype(np.uint8).astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 2) & 0x1F
+    m = (b & 0x3).astype(np.float64)
+    normal = sign * np.ldexp(1.0 + m / 4.0, (e - 15).astype(np.int64))
+    sub = sign * np.ldexp(m / 4.0, -14)
+    special = np.where(m == 0, sign * np.inf, np.nan)
+    return np.where(e == 0, sub, np.where(e == 31, special, normal))
+
+
+_DECODERS = {"bf16": decode_bf16, "fp16": decode_fp16, "e4m3": decode_e4m3, "e5m2": decode_e5m2}
+
+
+def decode(bits: np.ndarray, fmt: str) -> np.ndarray:
+    """Raw storage bits (uint16 for bf16/fp16, uint8 for FP8) -> float64."""
+    return _DECODERS[fmt](bits)
+
+
+# ---------------------------------------------------------------------------
+# Visibility (masks)
+# ---------------------------------------------------------------------------
+
+def visible_range(i: int, len_q: int, len_k: int, causal: bool, window_left: int,
+                  window_right: int) -> Tuple[int, int]:
+    """Inclusive [lo, hi] of keys visible to query row i (empty if lo > hi).
+
+    delta = len_k - len_q aligns the last query with the last key (bottom
+    right). causal caps the right edge at i + delta; a window bound of -1 is
+    unbounded."""
+    delta = len_k - len_q
+    lo = 0
+    hi = len_k - 1
+    if causal:
+        hi = min(hi, i + delta)
+    if window_right >= 0:
+        hi = min(hi, i + delta + window_right)
+    if window_left >= 0:
+        lo = max(lo, i + delta - window_left)
+    return lo, hi
+
+
+def visible_mask(len_q: int, len_k: int, causal: bool = False, window_left: int = -1,
+                 window_right: int = -1) -> np.ndarray:
+    """Boolean (len_q, len_k) matrix of visible (query, key) pairs."""
+    mask = np.zeros((len_q, len_k), dtype=bool)
+    for i in range(len_q):
+        lo, hi = visible_range(i, len_q, len_k, causal, window_left, window_right)
+        if lo <= hi:
+            mask[i, lo:hi + 1] = True
+    return mask
+
+
+# ---------------------------------------------------------------------------
+# The definition, per query row
+# ---------------------------------------------------------------------------
+
+def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                   vis: np.ndarray, sink=None) -> Tuple[np.ndarray, np.ndarray]:
+    """Attention for a block of query rows against one key/value set.
+
+    q (R, D_qk), k (L, D_qk), v (L, D_v), vis (R, L) bool; sink is None, a
+    scalar, or an array (R,) of per-row sink logits. Returns O (R, D_v) and the
+    keys-only LSE (R,), all float64."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    R = q.shape[0]
+    out = np.zeros((R, v.shape[1]), dtype=np.float64)
+    lse = np.full((R,), NEG_INF, dtype=np.float64)
+    if R == 0 or k.shape[0] == 0:
+        return out, lse
+    s = scale * (q @ k.T)
+    sinks = None
+    if sink is not None:
+        sinks = np.broadcast_to(np.asarray(sink, dtype=np.float64), (R,))
+    for r in range(R):
+        J = np.nonzero(vis[r])[0]
+        if J.size == 0:
+            continue
+        sj = s[r, J]
+        M = sj.max()
+        m = M if sinks is None else max(M, sinks[r])
+        e = np.exp(sj - m)
+        Z = e.sum()
+        if sinks is not None:
+            Z += math.exp(sinks[r] - m)
+        out[r] = (e @ v[J]) / Z
+        lse[r] = M + math.log(np.exp(sj - M).sum())
+    return out, lse
+
+
+def _kv_head(h: int, num_heads_q: int, num_heads_kv: int) -> int:
+    return h // (num_heads_q // num_heads_kv)
+
+
+# ---------------------------------------------------------------------------
+# Dense / varlen prefill
+# ---------------------------------------------------------------------------
+
+def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal=False,
+                     window=(-1, -1), sink=None, q_descale=None, k_descale=None,
+                     v_descale=None, rows: Optional[Iterable[Tuple[int, int, int]]] = None):
+    """Packed (TND) layout: q (T_q, H_q, D), k/v (T_k, H_kv, D) as float64,
+    cu_seqlens int arrays (B+1). Returns out (T_q, H_q, D_v) and lse (H_q, T_q).
+
+    ``rows`` optionally restricts the work to (b, i, h) triples; the other
+    entries of out/lse are left at 0 / -inf."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    cu_q = [int(x) for x in cu_seqlens_q]
+    cu_k = [int(x) for x in cu_seqlens_k]
+    B = len(cu_q) - 1
+    Hq, Hkv = q.shape[1], k.shape[1]
+    out = np.zeros((q.shape[0], Hq, v.shape[2]), np.float64)
+    lse = np.full((Hq, q.shape[0]), NEG_INF, np.float64)
+    want = None
+    if rows is not None:
+        want = {}
+        for (b, i, h) in rows:
+            want.setdefault((b, h), []).append(i)
+    for b in range(B):
+        Lq, Lk = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        for h in range(Hq):
+            if want is not None and (b, h) not in want:
+                continue
+            g = _kv_head(h, Hq, Hkv)
+            ii = np.arange(Lq) if want is None else np.array(sorted(set(want[(b, h)])))
+            qs = q[cu_q[b] + ii, h, :]
+            ks = k[cu_k[b]:cu_k[b + 1], g, :]
+            vs = v[cu_k[b]:cu_k[b + 1], g, :]
+            if q_descale is not None:
+                qs = qs * float(q_descale[b][g])
+                ks = ks * float(k_descale[b][g])
+                vs = vs * float(v_descale[b][g])
+            vis = np.zeros((len(ii), Lk), dtype=bool)
+            for r, i in enumerate(ii):
+                lo, hi = visible_range(int(i), Lq, Lk, causal, window[0], window[1])
+                if lo <= hi:
+                    vis[r, lo:hi + 1] = True
+            o, l = attention_rows(qs, ks, vs, scale, vis,
+                                  None if sink is None else float(sink[h]))
+            out[cu_q[b] + ii, h, :] = o
+            lse[h, cu_q[b] + ii] = l
+    return out, lse
+
+
+def attention_padded(q, k, v, scale, causal=False, window=(-1, -1), sink=None,
+                     q_descale=None, k_descale=None, v_descale=None, rows=None):
+    """Padded (BSHD) layout: q (B, S_q, H_q, D), k/v (B, S_k, H_kv, D).
+    Returns out (B, S_q, H_q, D_v) and lse (B, H_q, S_q)."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, Sq, Hq, _ = q.shape
+    Sk = k.shape[1]
+    cu_q = np.arange(B + 1) * Sq
+    cu_k = np.arange(B + 1) * Sk
+    o, l = attention_varlen(q.reshape(B * Sq, Hq, -1), k.reshape(B * Sk, k.shape[2], -1),
+                            v.reshape(B * Sk, v.shape[2], -1), cu_q, cu_k, scale, causal,
+                            window, sink, q_descale, k_descale, v_descale, rows)
+    return o.reshape(B, Sq, Hq, -1), l.reshape(Hq, B, Sq).transpose(1, 0, 2)
+
+
+# ---------------------------------------------------------------------------
+# Paged KV cache decode
+# ---------------------------------------------------------------------------
+
+def gather_pages(cache: np.ndarray, block_table_row: Sequence[int], length: int) -> np.ndarray:
+    """Logical rows 0..length-1 of one sequence: row t lives in physical page
+    block_table_row[t // page_size] at offset t % page_size."""
+    page = cache.shape[1]
+    idx = np.arange(length)
+    blocks = np.asarray(block_table_row, dtype=np.int64)[idx // page]
+    return cache[blocks, idx % page]
+
+
+def attention_paged(q, k_cache, v_cache, block_table, cache_seqlens, scale, causal=False,
+                    window=(-1, -1), sink=None, rows=None):
+    """q (B, s_q, H_q, D); caches (num_blocks, page_size, H_kv, D) float64;
+    block_table (B, max_pages); cache_seqlens (B,). The s_q query rows are the
+    last s_q positions of the sequence (bottom-right alignment).
+    Returns out (B, s_q, H_q, D_v) and lse (B, H_q, s_q)."""
+    q = np.asarray(q, np.float64)
+    B, Sq, Hq, _ = q.shape
+    Hkv = k_cache.shape[2]
+    out = np.zeros((B, Sq, Hq, v_cache.shape[3]), np.float64)
+    lse = np.full((B, Hq, Sq), NEG_INF, np.float64)
+    want = None
+    if rows is not None:
+        want = {}
+        for (b, i, h) in rows:
+            want.setdefault(b, set()).add((i, h))
+    for b in range(B):
+        if want is not None and b not in want:
+            continue
+        L = int(cache_seqlens[b])
+        ks = gather_pages(k_cache, block_table[b], L)
+        vs = gather_pages(v_cache, block_table[b], L)
+        for h in range(Hq):
+            ii = [i for i in range(Sq) if want is None or (i, h) in want[b]]
+            if not ii:
+                continue
+            g = _kv_head(h, Hq, Hkv)
+            vis = np.zeros((len(ii), L), dtype=bool)
+            for r, i in enumerate(ii):
+                lo, hi = visible_range(i, Sq, L, causal, window[0], window[1])
+                if lo <= hi:
+                    vis[r, lo:hi + 1] = True
+            o, l = attention_rows(q[b, ii, h, :], ks[:, g, :], vs[:, g, :], scale, vis,
+                                  None if sink is None else float(sink[h]))
+            out[b, ii, h, :] = o
+            lse[b, h, ii] = l
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Split-KV combine
+# ---------------------------------------------------------------------------
+
+def combine(out_partial: np.ndarray, lse_partial: np.ndarray, sink=None):
+    """Merge sink-free partial results over disjoint key splits.
+
+    out_partial (n_splits, ..., D_v), lse_partial (n_splits, ...). A split with
+    LSE = -inf carries weight 0; if every split is -inf the result is O = 0,
+    LSE = -inf. ``sink`` (broadcastable to lse_partial[0]) is applied once
+    after the merge. Returns (out, lse)."""
+    O = np.asarray(out_partial, np.float64)
+    Ls = np.asarray(lse_partial, np.float64)
+    Mx = Ls.max(axis=0)
+    finite = np.isfinite(Mx)
+    Msafe = np.where(finite, Mx, 0.0)
+    w = np.where(np.isfinite(Ls), np.exp(Ls - Msafe[None]), 0.0)
+    tot = w.sum(axis=0)
+    lse = np.where(finite, Msafe + np.log(np.where(finite, tot, 1.0)), NEG_INF)
+    wn = np.where(finite[None], w / np.where(finite, tot, 1.0)[None], 0.0)
+    out = (wn[..., None] * O).sum(axis=0)
+    if sink is not None:
+        sk = np.broadcast_to(np.asarray(sink, np.float64), lse.shape)
+        factor = np.where(finite, 1.0 / (1.0 + np.exp(sk - np.where(finite, lse, 0.0))), 0.0)
+        out = out * factor[..., None]
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# MLA-absorbed decode (dense and top-k sparse)
+# ---------------------------------------------------------------------------
+
+def mla_paged(q, kv_cache, block_table, cache_seqlens, head_dim_v, scale, causal=False,
+              rows=None):
+    """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, 1, 576). K is the
+    whole row, V its first head_dim_v entries."""
+    kv = np.asarray(kv_cache, np.float64)
+    return attention_paged(q, kv, kv[..., :head_dim_v], block_table, cache_seqlens, scale,
+                           causal, (-1, -1), None, rows)
+
+
+def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, scale,
+               rows=None):
+    """q (B, s_q, H_q, 576); indices (B, s_q, 1, topk) logical positions. Query
+    token (b, i) attends to the listed positions p with 0 <= p < L_b (each
+    listed occurrence counts once); the others are skipped.
+    Returns out (B, s_q, H_q, D_v) and lse (B, H_q, s_q)."""
+    q = np.asarray(q, np.float64)
+    kv = np.asarray(kv_cache, np.float64)
+    B, Sq, Hq, _ = q.shape
+    page = kv.shape[1]
+    out = np.zeros((B, Sq, Hq, head_dim_v), np.float64)
+    lse = np.full((B, Hq, Sq), NEG_INF, np.float64)
+    want = None
+    if rows is not None:
+        want = {}
+        for (b, i, h) in rows:
+            want.setdefault((b, i), []).append(h)
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        for i in range(Sq):
+            if want is not None and (b, i) not in want:
+                continue
+            hs = list(range(Hq)) if want is None else sorted(set(want[(b, i)]))
+            idx = np.asarray(indices[b, i, 0], dtype=np.int64)
+            idx = idx[(idx >= 0) & (idx < L)]
+            rows_kv = kv[np.asarray(block_table[b], np.int64)[idx // page], idx % page, 0, :]
+            vis = np.ones((len(hs), idx.size), dtype=bool)
+            o, l = attention_rows(q[b, i, hs, :], rows_kv, rows_kv[:, :head_dim_v], scale, vis)
+            out[b, i, hs, :] = o
+            lse[b, hs, i] = l
+    return out, lse

@@ -1,0 +1,374 @@
+"""Pins for the fp64 oracle, checked on the CPU.
+
+The oracle is compared with things other than itself: torch's own fp64
+routines (scaled_dot_product_attention, logsumexp, tril/triu, the float8 /
+bfloat16 / float16 conversions), closed forms and invariants that follow from
+the pages' formulas, and brute force on tiny inputs. Each test names what it
+guards against.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from oracle import attention as orc
+
+RNG = np.random.default_rng(1234)
+
+
+def _sdpa(q, k, v, scale, mask=None):
+    """torch fp64 SDPA on (H, L, D) arrays; mask (Lq, Lk) bool, True = visible."""
+    tq = torch.as_tensor(q, dtype=torch.float64)[None]
+    tk = torch.as_tensor(k, dtype=torch.float64)[None]
+    tv = torch.as_tensor(v, dtype=torch.float64)[None]
+    m = None if mask is None else torch.as_tensor(mask)[None, None]
+    gqa = tq.shape[1] != tk.shape[1]
+    return F.scaled_dot_product_attention(tq, tk, tv, attn_mask=m, scale=scale,
+                                          enable_gqa=gqa)[0].numpy()
+
+
+# --------------------------------------------------------------------------
+# number formats: every code against torch's conversion
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt,tdt,nbits", [
+    ("bf16", torch.bfloat16, 16), ("fp16", torch.float16, 16),
+    ("e4m3", torch.float8_e4m3fn, 8), ("e5m2", torch.float8_e5m2, 8)])
+def test_decode_all_codes_match_torch(fmt, tdt, nbits):
+    if nbits == 16:
+        codes = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+        ref = torch.from_numpy(codes.view(np.int16).copy()).view(tdt).to(torch.float64).numpy()
+    else:
+        codes = np.arange(256, dtype=np.uint8)
+        ref = torch.from_numpy(codes.copy()).view(tdt).to(torch.float64).numpy()
+    got = oracle.decode(codes, fmt)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+
+
+def test_e4m3_format_landmarks():
+    d = orc.decode_e4m3(np.array([0x7E, 0x08, 0x01, 0x38, 0xB8, 0x7F, 0xFF], np.uint8))
+    assert d[0] == 448.0                      # largest finite
+    assert d[1] == 2.0 ** -6                  # smallest normal
+    assert d[2] == 2.0 ** -9                  # smallest subnormal
+    assert d[3] == 1.0 and d[4] == -1.0
+    assert np.isnan(d[5]) and np.isnan(d[6])  # S.1111.111
+
+
+# --------------------------------------------------------------------------
+# masks
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lq,lk", [(5, 5), (3, 7), (7, 3), (1, 9), (6, 1)])
+def test_causal_mask_is_bottom_right_tril(lq, lk):
+    ref = torch.ones(lq, lk, dtype=torch.bool).tril(diagonal=lk - lq).numpy()
+    assert np.array_equal(oracle.visible_mask(lq, lk, causal=True), ref)
+
+
+@pytest.mark.parametrize("lq,lk,left,right", [(9, 9, 2, 0), (9, 9, 3, 1), (4, 10, 2, -1),
+                                              (10, 4, -1, 2), (6, 6, 0, 0)])
+def test_window_mask_is_band(lq, lk, left, right):
+    d = lk - lq
+    band = torch.ones(lq, lk, dtype=torch.bool)
+    if right >= 0:
+        band = band.tril(diagonal=d + right)
+    if left >= 0:
+        band = band.triu(diagonal=d - left)
+    assert np.array_equal(oracle.visible_mask(lq, lk, False, left, right), band.numpy())
+    # inclusive bounds: a square window (left, 0) keeps min(i, left) + 1 keys
+    if lq == lk and right == 0:
+        counts = oracle.visible_mask(lq, lk, False, left, right).sum(1)
+        assert list(counts) == [min(i, left) + 1 for i in range(lq)]
+
+
+def test_mask_special_cases():
+    assert oracle.visible_mask(5, 8).all()                                     # (-1,-1): full
+    assert oracle.visible_mask(1, 8, causal=True).all()                        # decode row
+    assert np.array_equal(oracle.visible_mask(6, 6, True, 100, -1),
+                          oracle.visible_mask(6, 6, True))                     # huge window
+    assert np.array_equal(oracle.visible_mask(6, 6, False, -1, 0),
+                          oracle.visible_mask(6, 6, True))                     # causal == right 0
+
+
+# --------------------------------------------------------------------------
+# the per-row definition
+# --------------------------------------------------------------------------
+
+def test_rows_match_torch_sdpa_and_logsumexp():
+    R, L, D, Dv = 6, 11, 8, 5
+    q, k, v = RNG.normal(size=(R, D)), RNG.normal(size=(L, D)), RNG.normal(size=(L, Dv))
+    vis = RNG.random((R, L)) < 0.6
+    vis[:, 0] = True
+    scale = 0.37
+    o, lse = oracle.attention_rows(q, k, v, scale, vis)
+    ref = _sdpa(q[None], k[None], v[None], scale, vis)[0]
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-12)
+    s = torch.as_tensor(scale * q @ k.T).masked_fill(~torch.as_tensor(vis), -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=1).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_rows_single_key_and_identical_values():
+    q, k = RNG.normal(size=(3, 4)), RNG.normal(size=(5, 4))
+    v = RNG.normal(size=(5, 3))
+    vis = np.zeros((3, 5), bool)
+    vis[0, 2] = vis[1, 4] = vis[2, 0] = True
+    o, lse = oracle.attention_rows(q, k, v, 0.5, vis)
+    for r, j in enumerate([2, 4, 0]):
+        np.testing.assert_allclose(o[r], v[j], rtol=0, atol=1e-15)
+        assert abs(lse[r] - 0.5 * q[r] @ k[j]) < 1e-14
+    vv = np.tile(RNG.normal(size=(1, 3)), (5, 1))
+    o2, _ = oracle.attention_rows(q, k, vv, 0.5, np.ones((3, 5), bool))
+    np.testing.assert_allclose(o2, np.tile(vv[:1], (3, 1)), rtol=1e-13)
+
+
+def test_rows_shift_invariance_and_lse_identity():
+    q, k, v = RNG.normal(size=(4, 6)), RNG.normal(size=(9, 6)), RNG.normal(size=(9, 2))
+    vis = np.ones((4, 9), bool)
+    o, lse = oracle.attention_rows(q, k, v, 1.0, vis)
+    # adding c to every score (append a constant feature) moves LSE by c only
+    c = 3.25
+    q2 = np.hstack([q, np.ones((4, 1))])
+    k2 = np.hstack([k, np.full((9, 1), c)])
+    o2, lse2 = oracle.attention_rows(q2, k2, v, 1.0, vis)
+    np.testing.assert_allclose(o2, o, rtol=1e-12)
+    np.testing.assert_allclose(lse2, lse + c, rtol=1e-12)
+    # sum_j e^{s_j - LSE} = 1 and O = sum_j e^{s_j - LSE} v_j
+    w = np.exp(q @ k.T - lse[:, None])
+    np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-12)
+    np.testing.assert_allclose(w @ v, o, rtol=1e-12)
+
+
+def test_sink_closed_forms():
+    q, k, v = RNG.normal(size=(5, 4)), RNG.normal(size=(7, 4)), RNG.normal(size=(7, 3))
+    vis = np.ones((5, 7), bool)
+    vis[1, 3:] = False
+    sink = RNG.normal(size=5) * 2
+    o0, lse0 = oracle.attention_rows(q, k, v, 0.8, vis)
+    o1, lse1 = oracle.attention_rows(q, k, v, 0.8, vis, sink)
+    sig = 1.0 / (1.0 + np.exp(sink - lse0))          # O_sink = O * sigma(LSE - sink)
+    np.testing.assert_allclose(o1, o0 * sig[:, None], rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(lse1, lse0, rtol=0, atol=0)  # keys-only LSE
+    o2, _ = oracle.attention_rows(q, k, v, 0.8, vis, np.full(5, -1e4))
+    np.testing.assert_allclose(o2, o0, rtol=1e-14)    # sink -> -inf: no sink
+    # one key whose score equals the sink: half the weight goes to the sink
+    s = 0.8 * q[0] @ k[0]
+    o3, _ = oracle.attention_rows(q[:1], k[:1], v[:1], 0.8, np.ones((1, 1), bool), s)
+    np.testing.assert_allclose(o3[0], v[0] / 2, rtol=1e-14)
+
+
+def test_rows_without_visible_keys():
+    o, lse = oracle.attention_rows(np.ones((2, 3)), np.ones((4, 3)), np.ones((4, 2)), 1.0,
+                                   np.zeros((2, 4), bool), 0.5)
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+
+
+# --------------------------------------------------------------------------
+# layouts: varlen, padded, GQA, FP8 descale
+# --------------------------------------------------------------------------
+
+def _varlen_case(lens_q, lens_k, Hq, Hkv, D):
+    tq, tk = sum(lens_q), sum(lens_k)
+    q = RNG.normal(size=(tq, Hq, D))
+    k = RNG.normal(size=(tk, Hkv, D))
+    v = RNG.normal(size=(tk, Hkv, D))
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)])
+    cu_k = np.concatenate([[0], np.cumsum(lens_k)])
+    return q, k, v, cu_q, cu_k
+
+
+@pytest.mark.parametrize("causal,window", [(False, (-1, -1)), (True, (-1, -1)), (True, (3, 0)),
+                                           (False, (2, 1))])
+def test_varlen_gqa_matches_sdpa(causal, window):
+    lens_q, lens_k = [5, 1, 9], [7, 4, 9]
+    Hq, Hkv, D = 6, 2, 4
+    q, k, v, cu_q, cu_k = _varlen_case(lens_q, lens_k, Hq, Hkv, D)
+    out, lse = oracle.attention_varlen(q, k, v, cu_q, cu_k, 0.6, causal, window)
+    for b in range(3):
+        sq = slice(cu_q[b], cu_q[b + 1])
+        sk = slice(cu_k[b], cu_k[b + 1])
+        mask = torch.ones(lens_q[b], lens_k[b], dtype=torch.bool)
+        d = lens_k[b] - lens_q[b]
+        if causal or window[1] >= 0:
+            mask = mask.tril(diagonal=d + (0 if causal else window[1]))
+        if window[0] >= 0:
+            mask = mask.triu(diagonal=d - window[0])
+        ref = _sdpa(q[sq].transpose(1, 0, 2), k[sk].transpose(1, 0, 2), v[sk].transpose(1, 0, 2),
+                    0.6, mask.numpy()).transpose(1, 0, 2)
+        rows = mask.any(1).numpy()
+        np.testing.assert_allclose(out[sq][rows], ref[rows], rtol=1e-11, atol=1e-12)
+        assert np.all(out[sq][~rows] == 0) and np.all(np.isneginf(lse[:, sq][:, ~rows]))
+
+
+def test_gqa_equals_repeated_heads_and_padded_equals_varlen():
+    B, S, Hq, Hkv, D = 2, 6, 4, 2, 3
+    q, k, v = (RNG.normal(size=(B, S, Hq, D)), RNG.normal(size=(B, S, Hkv, D)),
+               RNG.normal(size=(B, S, Hkv, D)))
+    o, l = oracle.attention_padded(q, k, v, 0.7, causal=True)
+    kr, vr = np.repeat(k, Hq // Hkv, axis=2), np.repeat(v, Hq // Hkv, axis=2)
+    o2, l2 = oracle.attention_padded(q, kr, vr, 0.7, causal=True)
+    np.testing.assert_allclose(o, o2, rtol=1e-14)
+    np.testing.assert_allclose(l, l2, rtol=1e-14)
+    cu = np.arange(B + 1) * S
+    o3, l3 = oracle.attention_varlen(q.reshape(B * S, Hq, D), k.reshape(B * S, Hkv, D),
+                                     v.reshape(B * S, Hkv, D), cu, cu, 0.7, True)
+    np.testing.assert_allclose(o, o3.reshape(B, S, Hq, D), rtol=1e-14)
+    np.testing.assert_allclose(l, l3.reshape(Hq, B, S).transpose(1, 0, 2), rtol=1e-14)
+
+
+def test_row_subset_equals_full():
+    q, k, v, cu_q, cu_k = _varlen_case([4, 6], [4, 8], 4, 2, 3)
+    out, lse = oracle.attention_varlen(q, k, v, cu_q, cu_k, 0.5, True, (2, 0), np.ones(4))
+    rows = [(1, 5, 3), (0, 0, 0), (1, 2, 1)]
+    o2, l2 = oracle.attention_varlen(q, k, v, cu_q, cu_k, 0.5, True, (2, 0), np.ones(4), rows=rows)
+    for b, i, h in rows:
+        t = cu_q[b] + i
+        np.testing.assert_array_equal(o2[t, h], out[t, h])
+        assert l2[h, t] == lse[h, t]
+
+
+def test_fp8_descale_equals_prescaled_inputs():
+    q, k, v, cu_q, cu_k = _varlen_case([3, 5], [3, 5], 4, 2, 4)
+    qd, kd, vd = (RNG.uniform(0.5, 2, size=(2, 2)) for _ in range(3))
+    out, lse = oracle.attention_varlen(q, k, v, cu_q, cu_k, 0.5, True, q_descale=qd,
+                                       k_descale=kd, v_descale=vd)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for b in range(2):
+        for g in range(2):
+            q2[cu_q[b]:cu_q[b + 1], 2 * g:2 * g + 2] *= qd[b, g]
+            k2[cu_k[b]:cu_k[b + 1], g] *= kd[b, g]
+            v2[cu_k[b]:cu_k[b + 1], g] *= vd[b, g]
+    o2, l2 = oracle.attention_varlen(q2, k2, v2, cu_q, cu_k, 0.5, True)
+    np.testing.assert_allclose(out, o2, rtol=1e-13)
+    np.testing.assert_allclose(lse, l2, rtol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# paged cache
+# --------------------------------------------------------------------------
+
+def _paged_case(lens, page, Hkv, D, table):
+    pages = [max(1, -(-L // page)) for L in lens]
+    total = sum(pages)
+    cache_k = RNG.normal(size=(total, page, Hkv, D))
+    cache_v = RNG.normal(size=(total, page, Hkv, D))
+    perm = np.arange(total) if table == "identity" else RNG.permutation(total)
+    bt = np.zeros((len(lens), max(pages)), np.int64)
+    off = 0
+    for b, n in enumerate(pages):
+        bt[b, :n] = perm[off:off + n]
+        off += n
+    return cache_k, cache_v, bt
+
+
+def test_gather_pages_brute_force():
+    cache = RNG.normal(size=(5, 4, 1, 2))
+    bt = [3, 0, 4]
+    got = oracle.gather_pages(cache, bt, 10)
+    want = np.stack([cache[bt[t // 4], t % 4] for t in range(10)])
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("table", ["identity", "permuted"])
+def test_paged_equals_contiguous(table):
+    lens, page, Hq, Hkv, D, sq = [9, 16, 3], 4, 4, 2, 5, 2
+    ck, cv, bt = _paged_case(lens, page, Hkv, D, table)
+    q = RNG.normal(size=(3, sq, Hq, D))
+    sink = RNG.normal(size=Hq)
+    out, lse = oracle.attention_paged(q, ck, cv, bt, lens, 0.4, causal=True, sink=sink)
+    for b, L in enumerate(lens):
+        kk = oracle.gather_pages(ck, bt[b], L)
+        vv = oracle.gather_pages(cv, bt[b], L)
+        cu_q, cu_k = np.array([0, sq]), np.array([0, L])
+        o2, l2 = oracle.attention_varlen(q[b], kk, vv, cu_q, cu_k, 0.4, True, sink=sink)
+        np.testing.assert_allclose(out[b], o2, rtol=1e-13)
+        np.testing.assert_allclose(lse[b], l2, rtol=1e-13)
+
+
+def test_paged_aliased_table_repeats_one_page():
+    page, L = 4, 10
+    ck = RNG.normal(size=(1, page, 1, 3))
+    cv = RNG.normal(size=(1, page, 1, 3))
+    q = RNG.normal(size=(1, 1, 2, 3))
+    out, lse = oracle.attention_paged(q, ck, cv, np.zeros((1, 3), np.int64), [L], 1.0)
+    kk = np.concatenate([ck[0]] * 3)[:L]
+    vv = np.concatenate([cv[0]] * 3)[:L]
+    ref = _sdpa(q[0].transpose(1, 0, 2), np.repeat(kk.transpose(1, 0, 2), 2, 0),
+                np.repeat(vv.transpose(1, 0, 2), 2, 0), 1.0)
+    np.testing.assert_allclose(out[0], ref.transpose(1, 0, 2), rtol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# combine
+# --------------------------------------------------------------------------
+
+def test_split_then_combine_equals_unsplit():
+    L, D = 23, 4
+    q, k, v = RNG.normal(size=(3, D)), RNG.normal(size=(L, D)), RNG.normal(size=(L, D))
+    vis = np.ones((3, L), bool)
+    vis[2, 10:] = False
+    o, lse = oracle.attention_rows(q, k, v, 0.5, vis)
+    cuts = [0, 5, 5, 12, 23]            # includes an empty split
+    parts = [oracle.attention_rows(q, k[a:b], v[a:b], 0.5, vis[:, a:b]) for a, b in
+             zip(cuts[:-1], cuts[1:])]
+    oc, lc = oracle.combine(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    np.testing.assert_allclose(oc, o, rtol=1e-12)
+    np.testing.assert_allclose(lc, lse, rtol=1e-12)
+    sink = np.array([0.3, -1.0, 2.0])
+    o_s, _ = oracle.attention_rows(q, k, v, 0.5, vis, sink)
+    oc2, lc2 = oracle.combine(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]),
+                              sink)
+    np.testing.assert_allclose(oc2, o_s, rtol=1e-12)      # sink applied once
+    np.testing.assert_allclose(lc2, lse, rtol=1e-12)
+
+
+def test_combine_all_empty():
+    oc, lc = oracle.combine(np.ones((3, 2, 4)), np.full((3, 2), -np.inf), np.zeros(2))
+    assert np.all(oc == 0) and np.all(np.isneginf(lc))
+
+
+# --------------------------------------------------------------------------
+# MLA
+# --------------------------------------------------------------------------
+
+def test_mla_dense_equals_sdpa_with_latent_values():
+    lens, page, Hq, D, Dv = [7, 12], 4, 3, 10, 6
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    q = RNG.normal(size=(2, 2, Hq, D))
+    out, lse = oracle.mla_paged(q, ck, bt, lens, Dv, 0.3)
+    for b, L in enumerate(lens):
+        kk = oracle.gather_pages(ck, bt[b], L)[:, 0, :]
+        for i in range(2):
+            ref = _sdpa(q[b, i][:, None, :], np.repeat(kk[None], Hq, 0),
+                        np.repeat(kk[None, :, :Dv], Hq, 0), 0.3)[:, 0, :]
+            np.testing.assert_allclose(out[b, i], ref, rtol=1e-12)
+
+
+def test_mla_sparse_all_positions_equals_dense_and_skips_invalid():
+    lens, page, Hq, D, Dv, topk = [7, 12], 4, 3, 10, 6, 16
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    q = RNG.normal(size=(2, 2, Hq, D))
+    idx = np.full((2, 2, 1, topk), -1, np.int64)
+    for b, L in enumerate(lens):
+        idx[b, :, 0, :L] = np.arange(L)
+    idx[0, 1, 0, 10] = 99                       # beyond the cache length: skipped
+    o_s, l_s = oracle.mla_sparse(q, ck, bt, lens, idx, Dv, 0.3)
+    o_d, l_d = oracle.mla_paged(q, ck, bt, lens, Dv, 0.3)
+    np.testing.assert_allclose(o_s, o_d, rtol=1e-12)
+    np.testing.assert_allclose(l_s, l_d, rtol=1e-12)
+
+
+def test_mla_sparse_subset_matches_sdpa_on_gathered_rows():
+    lens, page, Hq, D, Dv, topk = [20], 4, 2, 8, 5, 6
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    q = RNG.normal(size=(1, 1, Hq, D))
+    sel = np.array([1, 4, 5, 11, 17, 19])
+    idx = sel.reshape(1, 1, 1, topk)
+    out, _ = oracle.mla_sparse(q, ck, bt, lens, idx, Dv, 0.5)
+    kk = oracle.gather_pages(ck, bt[0], 20)[sel, 0, :]
+    ref = _sdpa(q[0, 0][:, None, :], np.repeat(kk[None], Hq, 0),
+                np.repeat(kk[None, :, :Dv], Hq, 0), 0.5)[:, 0, :]
+    np.testing.assert_allclose(out[0, 0], ref, rtol=1e-12)
