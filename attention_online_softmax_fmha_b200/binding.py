@@ -1,0 +1,224 @@
+"""Thin Python binding of libattn (ctypes).
+
+Argument marshalling only: torch tensors supply device pointers, shapes and
+strides; every step of the computation runs in libattn's CUDA kernels. There
+is no fallback: if libattn.so is missing or a call fails, an exception is
+raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+c_i32, c_i64, c_f32, c_vp, c_sz = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                   ctypes.c_void_p, ctypes.c_size_t)
+
+# status codes and enums (include/libattn.h)
+OK, INVALID_ARG, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA_ERROR, DEVICE_ERROR = range(6)
+DTYPE_BF16, DTYPE_FP16, DTYPE_E4M3, DTYPE_E5M2, DTYPE_FP32 = range(5)
+SCHED_MHA, SCHED_MLA, SCHED_MLA_SPARSE = range(3)
+DEVERR_TIMEOUT, DEVERR_META_MISMATCH = 1, 2
+
+_TORCH_DTYPE = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16,
+                torch.float8_e4m3fn: DTYPE_E4M3, torch.float8_e5m2: DTYPE_E5M2}
+
+
+class VarlenArgs(ctypes.Structure):
+    _fields_ = [("q", c_vp), ("k", c_vp), ("v", c_vp), ("out", c_vp), ("lse", c_vp),
+                ("cu_seqlens_q", c_vp), ("cu_seqlens_k", c_vp),
+                ("batch", c_i32), ("max_seqlen_q", c_i32), ("max_seqlen_k", c_i32),
+                ("total_q", c_i32), ("total_k", c_i32), ("num_heads_q", c_i32),
+                ("num_heads_kv", c_i32), ("head_dim_qk", c_i32), ("head_dim_v", c_i32),
+                ("q_stride_b", c_i64), ("q_stride_s", c_i64), ("q_stride_h", c_i64),
+                ("k_stride_b", c_i64), ("k_stride_s", c_i64), ("k_stride_h", c_i64),
+                ("v_stride_b", c_i64), ("v_stride_s", c_i64), ("v_stride_h", c_i64),
+                ("o_stride_b", c_i64), ("o_stride_s", c_i64), ("o_stride_h", c_i64),
+                ("lse_stride_b", c_i64), ("lse_stride_h", c_i64),
+                ("dtype", c_i32), ("scale", c_f32), ("causal", c_i32),
+                ("window_left", c_i32), ("window_right", c_i32),
+                ("sink", c_vp), ("q_descale", c_vp), ("k_descale", c_vp), ("v_descale", c_vp)]
+
+
+class SchedArgs(ctypes.Structure):
+    _fields_ = [("cache_seqlens", c_vp), ("batch", c_i32), ("seqlen_q", c_i32),
+                ("num_heads_q", c_i32), ("num_heads_kv", c_i32), ("head_dim_qk", c_i32),
+                ("head_dim_v", c_i32), ("page_size", c_i32), ("mode", c_i32), ("topk", c_i32),
+                ("num_ctas", c_i32), ("meta", c_vp), ("meta_bytes", c_sz)]
+
+
+class PagedArgs(ctypes.Structure):
+    _fields_ = [("q", c_vp), ("k_cache", c_vp), ("v_cache", c_vp), ("block_table", c_vp),
+                ("cache_seqlens", c_vp), ("out", c_vp), ("lse", c_vp),
+                ("batch", c_i32), ("seqlen_q", c_i32), ("num_heads_q", c_i32),
+                ("num_heads_kv", c_i32), ("head_dim", c_i32), ("page_size", c_i32),
+                ("num_blocks", c_i32), ("max_pages_per_seq", c_i32),
+                ("block_table_stride", c_i64),
+                ("q_stride_b", c_i64), ("q_stride_s", c_i64), ("q_stride_h", c_i64),
+                ("kc_stride_blk", c_i64), ("kc_stride_tok", c_i64), ("kc_stride_h", c_i64),
+                ("vc_stride_blk", c_i64), ("vc_stride_tok", c_i64), ("vc_stride_h", c_i64),
+                ("o_stride_b", c_i64), ("o_stride_s", c_i64), ("o_stride_h", c_i64),
+                ("dtype", c_i32), ("scale", c_f32), ("causal", c_i32),
+                ("window_left", c_i32), ("window_right", c_i32), ("sink", c_vp),
+                ("meta", c_vp), ("meta_bytes", c_sz), ("workspace", c_vp),
+                ("workspace_bytes", c_sz)]
+
+
+class CombineArgs(ctypes.Structure):
+    _fields_ = [("out_partial", c_vp), ("lse_partial", c_vp), ("out", c_vp), ("lse", c_vp),
+                ("num_splits_per_seq", c_vp), ("sink", c_vp), ("num_splits", c_i32),
+                ("batch", c_i32), ("seqlen_q", c_i32), ("num_heads", c_i32),
+                ("head_dim_v", c_i32), ("o_stride_b", c_i64), ("o_stride_s", c_i64),
+                ("o_stride_h", c_i64), ("out_dtype", c_i32)]
+
+
+class MlaArgs(ctypes.Structure):
+    _fields_ = [("q", c_vp), ("kv_cache", c_vp), ("block_table", c_vp), ("cache_seqlens", c_vp),
+                ("indices", c_vp), ("out", c_vp), ("lse", c_vp),
+                ("batch", c_i32), ("seqlen_q", c_i32), ("num_heads_q", c_i32),
+                ("num_heads_kv", c_i32), ("head_dim_qk", c_i32), ("head_dim_v", c_i32),
+                ("page_size", c_i32), ("num_blocks", c_i32), ("max_pages_per_seq", c_i32),
+                ("topk", c_i32), ("block_table_stride", c_i64),
+                ("q_stride_b", c_i64), ("q_stride_s", c_i64), ("q_stride_h", c_i64),
+                ("kv_stride_blk", c_i64), ("kv_stride_tok", c_i64),
+                ("o_stride_b", c_i64), ("o_stride_s", c_i64), ("o_stride_h", c_i64),
+                ("idx_stride_b", c_i64), ("idx_stride_s", c_i64),
+                ("scale", c_f32), ("causal", c_i32), ("meta", c_vp), ("meta_bytes", c_sz),
+                ("workspace", c_vp), ("workspace_bytes", c_sz)]
+
+
+ARG_STRUCTS = {0: VarlenArgs, 1: SchedArgs, 2: PagedArgs, 3: CombineArgs, 4: MlaArgs}
+
+EXPORTS = ["attn_fwd_varlen", "attn_sched_metadata_size", "attn_sched_metadata",
+           "attn_paged_workspace_size", "attn_fwd_paged_kvcache", "attn_combine",
+           "mla_workspace_size", "mla_fwd_paged", "mla_sparse_fwd", "attn_get_device_error",
+           "attn_status_str", "attn_args_sizeof"]
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_str(status)} (status {status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libattn.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"libattn.so not built at {LIB_PATH}; run "
+                          "`python -m attention_online_softmax_fmha_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name in ["attn_fwd_varlen", "attn_sched_metadata", "attn_fwd_paged_kvcache",
+                     "attn_combine", "mla_fwd_paged", "mla_sparse_fwd"]:
+            getattr(L, name).argtypes = [c_vp, c_vp]
+            getattr(L, name).restype = c_i32
+        for name in ["attn_sched_metadata_size"]:
+            getattr(L, name).argtypes = [c_vp]
+            getattr(L, name).restype = c_sz
+        for name in ["attn_paged_workspace_size", "mla_workspace_size"]:
+            getattr(L, name).argtypes = [c_vp, c_vp]
+            getattr(L, name).restype = c_sz
+        L.attn_get_device_error.argtypes = [c_vp, c_vp]
+        L.attn_get_device_error.restype = c_i32
+        L.attn_status_str.argtypes = [c_i32]
+        L.attn_status_str.restype = ctypes.c_char_p
+        L.attn_args_sizeof.argtypes = [c_i32]
+        L.attn_args_sizeof.restype = c_sz
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().attn_status_str(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(fn: str, status: int):
+    if status != OK:
+        raise AttnError(fn, status)
+
+
+def device_error(stream=None) -> int:
+    """Read and clear the device error word (synchronises the stream)."""
+    code = c_i32(0)
+    st = lib().attn_get_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (OK, DEVICE_ERROR):
+        raise AttnError("attn_get_device_error", st)
+    return code.value
+
+
+def out_dtype_for(dtype: torch.dtype) -> torch.dtype:
+    """FP8 and bf16 inputs give bf16 outputs; fp16 gives fp16."""
+    return torch.float16 if dtype == torch.float16 else torch.bfloat16
+
+
+# ---------------------------------------------------------------------------
+# attn_fwd_varlen
+# ---------------------------------------------------------------------------
+
+def varlen_args(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None,
+                max_seqlen_k=None, scale=None, causal=False, window=(-1, -1), sink=None,
+                q_descale=None, k_descale=None, v_descale=None, out=None, lse=None):
+    """Build the argument struct (and allocate out/lse if not given)."""
+    varlen = cu_seqlens_q is not None
+    Hq, D = q.shape[-2], q.shape[-1]
+    Hkv, Dv = k.shape[-2], v.shape[-1]
+    if varlen:
+        B = cu_seqlens_q.numel() - 1
+        assert max_seqlen_q is not None and max_seqlen_k is not None, "varlen needs max lengths"
+        if out is None:
+            out = torch.empty(q.shape[0], Hq, Dv, device=q.device, dtype=out_dtype_for(q.dtype))
+        if lse is None:
+            lse = torch.empty(Hq, q.shape[0], device=q.device, dtype=torch.float32)
+        qsb = ksb = vsb = osb = 0
+        qss, qsh = q.stride(0), q.stride(1)
+        kss, ksh = k.stride(0), k.stride(1)
+        vss, vsh = v.stride(0), v.stride(1)
+        oss, osh = out.stride(0), out.stride(1)
+        lsb, lsh = 0, lse.stride(0)
+        sq, sk = int(max_seqlen_q), int(max_seqlen_k)
+    else:
+        B, sq, sk = q.shape[0], q.shape[1], k.shape[1]
+        if out is None:
+            out = torch.empty(B, sq, Hq, Dv, device=q.device, dtype=out_dtype_for(q.dtype))
+        if lse is None:
+            lse = torch.empty(B, Hq, sq, device=q.device, dtype=torch.float32)
+        qsb, qss, qsh = q.stride(0), q.stride(1), q.stride(2)
+        ksb, kss, ksh = k.stride(0), k.stride(1), k.stride(2)
+        vsb, vss, vsh = v.stride(0), v.stride(1), v.stride(2)
+        osb, oss, osh = out.stride(0), out.stride(1), out.stride(2)
+        lsb, lsh = lse.stride(0), lse.stride(1)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    a = VarlenArgs(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+        B, sq, sk, q.shape[0] if varlen else 0, k.shape[0] if varlen else 0, Hq, Hkv, D, Dv,
+        qsb, qss, qsh, ksb, kss, ksh, vsb, vss, vsh, osb, oss, osh, lsb, lsh,
+        _TORCH_DTYPE.get(q.dtype, -1), float(scale), int(bool(causal)), int(window[0]),
+        int(window[1]), _ptr(sink), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale))
+    return a, out, lse
+
+
+def fwd_varlen(q, k, v, *, stream=None, **kw):
+    """Attention forward (attn_fwd_varlen). Returns (out, lse)."""
+    a, out, lse = varlen_args(q, k, v, **kw)
+    _check("attn_fwd_varlen", lib().attn_fwd_varlen(ctypes.byref(a), _stream(stream)))
+    return out, lse

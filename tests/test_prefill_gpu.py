@@ -1,0 +1,120 @@
+"""attn_fwd_varlen on the GPU against the fp64 oracle, element by element.
+
+Tolerances: max-abs 1e-2 on bf16/fp16 outputs (N(0,1) inputs), 1e-3 on the
+fp32 LSE, and the -inf pattern of the LSE must match exactly."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_online_softmax_fmha_b200 import binding as B
+from attention_online_softmax_fmha_b200 import build as BUILD
+from attention_online_softmax_fmha_b200 import workloads as W
+from tests._util import assert_close_lse, assert_close_out, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    BUILD.build()
+    B.lib()
+
+
+def run_and_check(inp, atol=1e-2, with_lse=True):
+    kw = dict(scale=inp.scale, causal=inp.causal, window=inp.window, sink=inp.sink,
+              q_descale=inp.q_descale, k_descale=inp.k_descale, v_descale=inp.v_descale)
+    if inp.varlen:
+        kw.update(cu_seqlens_q=inp.cu_seqlens_q, cu_seqlens_k=inp.cu_seqlens_k,
+                  max_seqlen_q=max(inp.seqlens_q), max_seqlen_k=max(inp.seqlens_k))
+    out, lse = B.fwd_varlen(inp.q, inp.k, inp.v, **kw)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    q, k, v = to_f64(inp.q), to_f64(inp.k), to_f64(inp.v)
+    sink = None if inp.sink is None else inp.sink.cpu().numpy()
+    desc = {}
+    if inp.q_descale is not None:
+        desc = dict(q_descale=inp.q_descale.cpu().numpy(), k_descale=inp.k_descale.cpu().numpy(),
+                    v_descale=inp.v_descale.cpu().numpy())
+    if inp.varlen:
+        ro, rl = oracle.attention_varlen(q, k, v, inp.cu_seqlens_q.cpu().numpy(),
+                                         inp.cu_seqlens_k.cpu().numpy(), inp.scale, inp.causal,
+                                         inp.window, sink, **desc)
+    else:
+        ro, rl = oracle.attention_padded(q, k, v, inp.scale, inp.causal, inp.window, sink, **desc)
+    e_o = assert_close_out(to_f64(out), ro, atol)
+    e_l = assert_close_lse(lse.cpu().numpy(), rl) if with_lse else 0.0
+    return e_o, e_l
+
+
+def test_tiny_dense_mha_full_config():
+    # B=1, H=2, S=128, D=64, non-causal, scale 1/8: the whole workload.
+    inp = W.build_config("tiny_dense_mha", seed=0, device="cuda")
+    run_and_check(inp)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_varlen_causal_gqa_edge_lengths(D):
+    lens = [1, 63, 64, 65, 127, 128, 129, 300]
+    inp = W.make_prefill(seqlens_q=lens, num_heads_q=4, num_heads_kv=2, head_dim=D, varlen=True,
+                         causal=True, seed=1, device="cuda")
+    run_and_check(inp)
+
+
+def test_padded_window_sink():
+    inp = W.make_prefill(seqlens_q=[700] * 2, num_heads_q=4, num_heads_kv=4, head_dim=128,
+                         varlen=False, causal=True, window=(100, 0), sink=True, seed=2,
+                         device="cuda")
+    run_and_check(inp)
+
+
+@pytest.mark.parametrize("lq,lk", [([5, 130, 200], [300, 140, 200]), ([200, 33], [50, 1])])
+def test_varlen_causal_unequal_lengths(lq, lk):
+    # bottom-right alignment: L_k > L_q shifts the diagonal right; L_k < L_q
+    # leaves the first L_q - L_k rows with no visible key (O = 0, LSE = -inf).
+    inp = W.make_prefill(seqlens_q=lq, seqlens_k=lk, num_heads_q=2, num_heads_kv=1,
+                         head_dim=128, varlen=True, causal=True, sink=False, seed=3,
+                         device="cuda")
+    run_and_check(inp)
+
+
+def test_two_sided_window_and_window_wider_than_sequence():
+    inp = W.make_prefill(seqlens_q=[333, 90], num_heads_q=2, num_heads_kv=2, head_dim=64,
+                         varlen=True, causal=False, window=(64, 32), seed=4, device="cuda")
+    run_and_check(inp)
+    inp = W.make_prefill(seqlens_q=[200] * 2, num_heads_q=2, num_heads_kv=2, head_dim=128,
+                         varlen=False, causal=True, window=(5000, 0), sink=True, seed=5,
+                         device="cuda")
+    run_and_check(inp)
+
+
+def test_fp16_and_no_lse():
+    inp = W.make_prefill(seqlens_q=[257] * 2, num_heads_q=4, num_heads_kv=1, head_dim=64,
+                         varlen=False, causal=False, dtype="fp16", seed=6, device="cuda")
+    run_and_check(inp)
+    out, lse = B.fwd_varlen(inp.q, inp.k, inp.v, scale=inp.scale, lse=None)
+    a, out2, _ = B.varlen_args(inp.q, inp.k, inp.v, scale=inp.scale)
+    a.lse = None
+    import ctypes
+    assert B.lib().attn_fwd_varlen(ctypes.byref(a), B._stream(None)) == B.OK
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+def test_many_tiles_per_cta():
+    # more work tiles than SMs: every CTA runs several tiles back to back
+    inp = W.make_prefill(seqlens_q=[1024] * 2, num_heads_q=64, num_heads_kv=8, head_dim=128,
+                         varlen=False, causal=True, seed=7, device="cuda")
+    kw = dict(scale=inp.scale, causal=True)
+    out, lse = B.fwd_varlen(inp.q, inp.k, inp.v, **kw)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    # check a sample of rows with the oracle
+    rows = [(b, i, h) for b in range(2) for i in (0, 127, 128, 511, 1023) for h in (0, 9, 63)]
+    ro, rl = oracle.attention_padded(to_f64(inp.q), to_f64(inp.k), to_f64(inp.v), inp.scale, True,
+                                     rows=rows)
+    o = to_f64(out)
+    l = lse.cpu().numpy()
+    for b, i, h in rows:
+        assert_close_out(o[b, i, h], ro[b, i, h], 1e-2)
+        assert abs(l[b, h, i] - rl[b, h, i]) <= 1e-3
