@@ -66,7 +66,7 @@ class PagedArgs(ctypes.Structure):
                 ("o_stride_b", c_i64), ("o_stride_s", c_i64), ("o_stride_h", c_i64),
                 ("dtype", c_i32), ("scale", c_f32), ("causal", c_i32),
                 ("window_left", c_i32), ("window_right", c_i32), ("sink", c_vp),
-                ("meta", c_vp), ("meta_bytes", c_sz), ("workspace", c_vp),
+                ("meta", c_vp), ("meta_bytes", c_sz), ("num_ctas", c_i32), ("workspace", c_vp),
                 ("workspace_bytes", c_sz)]
 
 
@@ -90,7 +90,7 @@ class MlaArgs(ctypes.Structure):
                 ("o_stride_b", c_i64), ("o_stride_s", c_i64), ("o_stride_h", c_i64),
                 ("idx_stride_b", c_i64), ("idx_stride_s", c_i64),
                 ("scale", c_f32), ("causal", c_i32), ("meta", c_vp), ("meta_bytes", c_sz),
-                ("workspace", c_vp), ("workspace_bytes", c_sz)]
+                ("num_ctas", c_i32), ("workspace", c_vp), ("workspace_bytes", c_sz)]
 
 
 ARG_STRUCTS = {0: VarlenArgs, 1: SchedArgs, 2: PagedArgs, 3: CombineArgs, 4: MlaArgs}
@@ -125,7 +125,7 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).argtypes = [c_vp]
             getattr(L, name).restype = c_sz
         for name in ["attn_paged_workspace_size", "mla_workspace_size"]:
-            getattr(L, name).argtypes = [c_vp, c_vp]
+            getattr(L, name).argtypes = [c_vp]
             getattr(L, name).restype = c_sz
         L.attn_get_device_error.argtypes = [c_vp, c_vp]
         L.attn_get_device_error.restype = c_i32
@@ -221,4 +221,93 @@ def fwd_varlen(q, k, v, *, stream=None, **kw):
     """Attention forward (attn_fwd_varlen). Returns (out, lse)."""
     a, out, lse = varlen_args(q, k, v, **kw)
     _check("attn_fwd_varlen", lib().attn_fwd_varlen(ctypes.byref(a), _stream(stream)))
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# attn_sched_metadata
+# ---------------------------------------------------------------------------
+
+def sched_args(cache_seqlens, *, batch, seqlen_q, num_heads_q, num_heads_kv, head_dim_qk,
+               head_dim_v, page_size, mode=SCHED_MHA, topk=0, num_ctas=0):
+    return SchedArgs(_ptr(cache_seqlens), batch, seqlen_q, num_heads_q, num_heads_kv, head_dim_qk,
+                     head_dim_v, page_size, mode, topk, num_ctas, None, 0)
+
+
+def sched_metadata_size(a: SchedArgs) -> int:
+    return int(lib().attn_sched_metadata_size(ctypes.byref(a)))
+
+
+def sched_metadata(cache_seqlens, *, stream=None, meta=None, **kw) -> torch.Tensor:
+    """Scheduler metadata (attn_sched_metadata); returns the int32 buffer."""
+    a = sched_args(cache_seqlens, **kw)
+    nbytes = sched_metadata_size(a)
+    if nbytes == 0:
+        raise AttnError("attn_sched_metadata_size", INVALID_ARG)
+    if meta is None:
+        meta = torch.empty(nbytes // 4, dtype=torch.int32, device=cache_seqlens.device)
+    a.meta = meta.data_ptr()
+    a.meta_bytes = meta.numel() * 4
+    _check("attn_sched_metadata", lib().attn_sched_metadata(ctypes.byref(a), _stream(stream)))
+    return meta
+
+
+# ---------------------------------------------------------------------------
+# attn_fwd_paged_kvcache
+# ---------------------------------------------------------------------------
+
+def paged_args(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, causal=False,
+               window=(-1, -1), sink=None, meta=None, num_ctas=0, workspace=None, out=None,
+               lse=None):
+    B, sq, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    if out is None:
+        out = torch.empty(B, sq, Hq, D, device=q.device, dtype=out_dtype_for(q.dtype))
+    if lse is None:
+        lse = torch.empty(B, Hq, sq, device=q.device, dtype=torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    a = PagedArgs(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(out),
+        _ptr(lse), B, sq, Hq, Hkv, D, k_cache.shape[1], k_cache.shape[0], block_table.shape[1],
+        block_table.stride(0), q.stride(0), q.stride(1), q.stride(2), k_cache.stride(0),
+        k_cache.stride(1), k_cache.stride(2), v_cache.stride(0), v_cache.stride(1),
+        v_cache.stride(2), out.stride(0), out.stride(1), out.stride(2),
+        _TORCH_DTYPE.get(q.dtype, -1), float(scale), int(bool(causal)), int(window[0]),
+        int(window[1]), _ptr(sink), _ptr(meta), 0 if meta is None else meta.numel() * 4,
+        int(num_ctas), None, 0)
+    if meta is not None:
+        nbytes = int(lib().attn_paged_workspace_size(ctypes.byref(a)))
+        if workspace is None:
+            workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        a.workspace = workspace.data_ptr()
+        a.workspace_bytes = workspace.numel()
+    return a, out, lse, workspace
+
+
+def fwd_paged_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, *, stream=None, **kw):
+    """Paged-KV decode (attn_fwd_paged_kvcache, combine included). Returns (out, lse)."""
+    a, out, lse, ws = paged_args(q, k_cache, v_cache, block_table, cache_seqlens, **kw)
+    _check("attn_fwd_paged_kvcache", lib().attn_fwd_paged_kvcache(ctypes.byref(a),
+                                                                 _stream(stream)))
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# attn_combine
+# ---------------------------------------------------------------------------
+
+def combine(out_partial, lse_partial, *, num_splits_per_seq=None, sink=None, out=None, lse=None,
+            out_dtype=torch.bfloat16, stream=None):
+    """Merge split partials: out_partial fp32 (n, B, S, H, Dv), lse_partial fp32
+    (n, B, H, S). Returns (out (B, S, H, Dv), lse (B, H, S))."""
+    n, B, S, H, Dv = out_partial.shape
+    if out is None:
+        out = torch.empty(B, S, H, Dv, device=out_partial.device, dtype=out_dtype)
+    if lse is None:
+        lse = torch.empty(B, H, S, device=out_partial.device, dtype=torch.float32)
+    a = CombineArgs(_ptr(out_partial), _ptr(lse_partial), _ptr(out), _ptr(lse),
+                    _ptr(num_splits_per_seq), _ptr(sink), n, B, S, H, Dv, out.stride(0),
+                    out.stride(1), out.stride(2), _TORCH_DTYPE[out.dtype])
+    _check("attn_combine", lib().attn_combine(ctypes.byref(a), _stream(stream)))
     return out, lse

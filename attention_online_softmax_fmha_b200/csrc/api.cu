@@ -10,8 +10,11 @@
 #include <mutex>
 
 #include "../../include/libattn.h"
+#include "combine.cuh"
 #include "common.cuh"
+#include "decode_paged.cuh"
 #include "prefill_sm100.cuh"
+#include "sched.cuh"
 
 namespace attn {
 namespace {
@@ -171,6 +174,143 @@ attn_status_t check_varlen(const attn_varlen_args* a) {
   return ATTN_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Scheduler metadata / paged decode / combine
+// ---------------------------------------------------------------------------
+bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+// Segments and units of a decode problem (see sched.cuh).
+struct DecodeShape {
+  SchedShape sh;
+  int group = 0, rows = 0, n_rsub = 0, S = 0, G = 0;
+};
+
+attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int heads_kv,
+                           int topk, int num_ctas, DecodeShape& ds) {
+  if (batch <= 0 || seqlen_q <= 0 || heads_q <= 0 || heads_kv <= 0 || heads_q % heads_kv)
+    return ATTN_ERR_INVALID_ARG;
+  ds.sh.mode = mode;
+  ds.sh.topk = topk;
+  if (mode == ATTN_SCHED_MHA) {
+    ds.group = heads_q / heads_kv;
+    ds.rows = seqlen_q * ds.group;
+    ds.n_rsub = (ds.rows + kDecRows - 1) / kDecRows;
+    ds.sh.segs_per_seq = heads_kv * ds.n_rsub;
+    ds.sh.unit_keys = kDecTileKeys;
+  } else {
+    return ATTN_ERR_UNSUPPORTED;
+  }
+  const int64_t S = (int64_t)batch * ds.sh.segs_per_seq;
+  if (S > (1 << 24)) return ATTN_ERR_UNSUPPORTED;
+  ds.S = (int)S;
+  ds.G = num_ctas > 0 ? num_ctas : device_sm_count();
+  if (ds.G <= 0 || ds.G > 65536) return num_ctas < 0 ? ATTN_ERR_INVALID_ARG : ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+size_t meta_bytes_for(const DecodeShape& ds) {
+  return (size_t)MetaLayout(ds.G, ds.S).words * sizeof(int32_t);
+}
+
+attn_status_t check_paged(const attn_paged_args* a) {
+  if (!a) return ATTN_ERR_INVALID_ARG;
+  if (!a->q || !a->k_cache || !a->v_cache || !a->block_table || !a->cache_seqlens || !a->out)
+    return ATTN_ERR_INVALID_ARG;
+  if (a->batch <= 0 || a->seqlen_q <= 0 || a->num_heads_q <= 0 || a->num_heads_kv <= 0 ||
+      a->num_heads_q % a->num_heads_kv != 0 || a->head_dim <= 0 || a->num_blocks <= 0 ||
+      a->max_pages_per_seq <= 0 || a->page_size <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (a->block_table_stride < a->max_pages_per_seq) return ATTN_ERR_INVALID_ARG;
+  if (!(a->scale > 0.f) || !std::isfinite(a->scale)) return ATTN_ERR_INVALID_ARG;
+  if (a->window_left < -1 || a->window_right < -1 || a->num_ctas < 0) return ATTN_ERR_INVALID_ARG;
+  if (a->dtype < ATTN_DTYPE_BF16 || a->dtype > ATTN_DTYPE_E5M2) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k_cache) || !aligned16(a->v_cache) || !aligned16(a->out))
+    return ATTN_ERR_INVALID_ARG;
+  const int es = (a->dtype == ATTN_DTYPE_E4M3 || a->dtype == ATTN_DTYPE_E5M2) ? 1 : 2;
+  if (!stride_ok(a->q_stride_b, es) || !stride_ok(a->q_stride_s, es) ||
+      !stride_ok(a->q_stride_h, es) || !stride_ok(a->kc_stride_blk, es) ||
+      !stride_ok(a->kc_stride_tok, es) || !stride_ok(a->kc_stride_h, es) ||
+      !stride_ok(a->vc_stride_blk, es) || !stride_ok(a->vc_stride_tok, es) ||
+      !stride_ok(a->vc_stride_h, es) || !stride_ok(a->o_stride_b, 2) ||
+      !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
+    return ATTN_ERR_INVALID_ARG;
+  if (a->dtype != ATTN_DTYPE_BF16 && a->dtype != ATTN_DTYPE_FP16) return ATTN_ERR_UNSUPPORTED;
+  if (a->head_dim != 64 && a->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!pow2_in(a->page_size, 16, 256)) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+size_t paged_ws_bytes(const attn_paged_args* a, const DecodeShape& ds) {
+  const size_t slots = (size_t)ds.S + ds.G;
+  return slots * kDecRows * a->head_dim * sizeof(float) + slots * kDecRows * sizeof(float) + 256;
+}
+
+template <int D, bool kFp16>
+attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaStream_t stream) {
+  using C = DecodeCfg<D>;
+  const CUtensorMapDataType dt =
+      kFp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint32_t box_rows = a.page_size >= kDecTileKeys ? kDecTileKeys : a.page_size;
+  CUtensorMap mk, mv;
+  if (!encode_4d(&mk, a.k_cache, dt, 2, D, a.num_heads_kv, a.page_size, a.num_blocks,
+                 a.kc_stride_h, a.kc_stride_tok, a.kc_stride_blk, 64, 1, box_rows, 1) ||
+      !encode_4d(&mv, a.v_cache, dt, 2, D, a.num_heads_kv, a.page_size, a.num_blocks,
+                 a.vc_stride_h, a.vc_stride_tok, a.vc_stride_blk, 64, 1, box_rows, 1))
+    return ATTN_ERR_INVALID_ARG;
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = a.q;
+  p.out = a.out;
+  p.lse = a.lse;
+  p.block_table = a.block_table;
+  p.cache_seqlens = a.cache_seqlens;
+  p.meta = a.meta;
+  p.sink = a.sink;
+  p.bt_stride = a.block_table_stride;
+  p.q_sb = a.q_stride_b;
+  p.q_ss = a.q_stride_s;
+  p.q_sh = a.q_stride_h;
+  p.o_sb = a.o_stride_b;
+  p.o_ss = a.o_stride_s;
+  p.o_sh = a.o_stride_h;
+  p.batch = a.batch;
+  p.seqlen_q = a.seqlen_q;
+  p.heads_q = a.num_heads_q;
+  p.heads_kv = a.num_heads_kv;
+  p.group = ds.group;
+  p.rows = ds.rows;
+  p.n_rsub = ds.n_rsub;
+  p.segs_per_seq = ds.sh.segs_per_seq;
+  p.num_segs = ds.S;
+  p.page_size = a.page_size;
+  p.num_ctas = ds.G;
+  p.scale_log2 = a.scale * kLog2e;
+  p.causal = a.causal;
+  p.window_left = a.window_left;
+  p.window_right = a.window_right;
+  if (a.meta) {
+    const size_t slots = (size_t)ds.S + ds.G;
+    p.ws_o = reinterpret_cast<float*>(a.workspace);
+    p.ws_lse = p.ws_o + slots * kDecRows * D;
+  }
+  auto kernel = decode_kernel<D, kFp16>;
+  static bool configured = false;
+  if (!configured) {
+    if (set_smem(kernel, C::kSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
+    configured = true;
+  }
+  const int grid = a.meta ? ds.G : ds.S;
+  kernel<<<grid, 160, C::kSmemBytes, stream>>>(mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (a.meta) {
+    const int64_t warps = (int64_t)ds.S * kDecRows;
+    const int blocks = (int)((warps + 7) / 8);
+    decode_combine_kernel<D, kFp16><<<blocks, 256, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
 }  // namespace
 }  // namespace attn
 
@@ -193,18 +333,111 @@ attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream) {
   }
 }
 
-size_t attn_sched_metadata_size(const attn_sched_args*) { return 0; }
-attn_status_t attn_sched_metadata(const attn_sched_args* a, void*) {
-  return a ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+size_t attn_sched_metadata_size(const attn_sched_args* a) {
+  if (!a) return 0;
+  DecodeShape ds;
+  if (decode_shape(a->mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv, a->topk,
+                   a->num_ctas, ds) != ATTN_OK)
+    return 0;
+  return meta_bytes_for(ds);
 }
-size_t attn_paged_workspace_size(const attn_paged_args*, const attn_sched_args*) { return 0; }
-attn_status_t attn_fwd_paged_kvcache(const attn_paged_args* a, void*) {
-  return a ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+
+attn_status_t attn_sched_metadata(const attn_sched_args* a, void* stream) {
+  if (!a || !a->cache_seqlens || !a->meta) return ATTN_ERR_INVALID_ARG;
+  if (a->page_size <= 0 || a->head_dim_qk <= 0 || a->head_dim_v <= 0 || a->num_ctas < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (a->mode < ATTN_SCHED_MHA || a->mode > ATTN_SCHED_MLA_SPARSE) return ATTN_ERR_INVALID_ARG;
+  DecodeShape ds;
+  const attn_status_t st = decode_shape(a->mode, a->batch, a->seqlen_q, a->num_heads_q,
+                                        a->num_heads_kv, a->topk, a->num_ctas, ds);
+  if (st != ATTN_OK) return st;
+  if (a->meta_bytes < meta_bytes_for(ds)) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+  SchedParams p;
+  memset(&p, 0, sizeof(p));
+  p.cache_seqlens = a->cache_seqlens;
+  p.meta = a->meta;
+  p.sh = ds.sh;
+  p.batch = a->batch;
+  p.seqlen_q = a->seqlen_q;
+  p.heads_q = a->num_heads_q;
+  p.heads_kv = a->num_heads_kv;
+  p.page_size = a->page_size;
+  p.G = ds.G;
+  p.S = ds.S;
+  p.dim_qk = a->head_dim_qk;
+  p.dim_v = a->head_dim_v;
+  sched_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return launch_status(cudaGetLastError());
 }
-attn_status_t attn_combine(const attn_combine_args* a, void*) {
-  return a ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+
+size_t attn_paged_workspace_size(const attn_paged_args* a) {
+  if (!a || !a->meta || check_paged(a) != ATTN_OK) return 0;
+  DecodeShape ds;
+  if (decode_shape(ATTN_SCHED_MHA, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv, 0,
+                   a->num_ctas, ds) != ATTN_OK)
+    return 0;
+  return paged_ws_bytes(a, ds);
 }
-size_t mla_workspace_size(const mla_args*, const attn_sched_args*) { return 0; }
+
+attn_status_t attn_fwd_paged_kvcache(const attn_paged_args* a, void* stream) {
+  attn_status_t st = check_paged(a);
+  if (st != ATTN_OK) return st;
+  DecodeShape ds;
+  st = decode_shape(ATTN_SCHED_MHA, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv, 0,
+                    a->num_ctas, ds);
+  if (st != ATTN_OK) return st;
+  if (a->meta) {
+    if (a->meta_bytes < meta_bytes_for(ds)) return ATTN_ERR_INVALID_ARG;
+    if (!a->workspace || a->workspace_bytes < paged_ws_bytes(a, ds))
+      return ATTN_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(a->workspace)) return ATTN_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool f16 = a->dtype == ATTN_DTYPE_FP16;
+  if (a->head_dim == 64)
+    return f16 ? run_decode<64, true>(*a, ds, s) : run_decode<64, false>(*a, ds, s);
+  return f16 ? run_decode<128, true>(*a, ds, s) : run_decode<128, false>(*a, ds, s);
+}
+
+attn_status_t attn_combine(const attn_combine_args* a, void* stream) {
+  if (!a || !a->out_partial || !a->lse_partial || !a->out) return ATTN_ERR_INVALID_ARG;
+  if (a->num_splits <= 0 || a->batch <= 0 || a->seqlen_q <= 0 || a->num_heads <= 0 ||
+      a->head_dim_v <= 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (a->out_dtype != ATTN_DTYPE_BF16 && a->out_dtype != ATTN_DTYPE_FP16)
+    return ATTN_ERR_INVALID_ARG;
+  if (a->num_splits > kCombineMaxSplits || a->head_dim_v % 8 || a->head_dim_v > 1024)
+    return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(a->out_partial) || !aligned16(a->out)) return ATTN_ERR_INVALID_ARG;
+  if (!stride_ok(a->o_stride_b, 2) || !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
+    return ATTN_ERR_INVALID_ARG;
+  CombineParams p;
+  p.o_part = a->out_partial;
+  p.lse_part = a->lse_partial;
+  p.out = a->out;
+  p.lse = a->lse;
+  p.nsplit_per_seq = a->num_splits_per_seq;
+  p.sink = a->sink;
+  p.num_splits = a->num_splits;
+  p.batch = a->batch;
+  p.seqlen_q = a->seqlen_q;
+  p.heads = a->num_heads;
+  p.dv = a->head_dim_v;
+  p.o_sb = a->o_stride_b;
+  p.o_ss = a->o_stride_s;
+  p.o_sh = a->o_stride_h;
+  const int64_t rows = (int64_t)a->batch * a->seqlen_q * a->num_heads;
+  const int64_t blocks = (rows + 7) / 8;
+  if (blocks > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->out_dtype == ATTN_DTYPE_FP16)
+    combine_kernel<true><<<(int)blocks, 256, 0, s>>>(p);
+  else
+    combine_kernel<false><<<(int)blocks, 256, 0, s>>>(p);
+  return launch_status(cudaGetLastError());
+}
+
+size_t mla_workspace_size(const mla_args*) { return 0; }
 attn_status_t mla_fwd_paged(const mla_args* a, void*) {
   return a ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
 }

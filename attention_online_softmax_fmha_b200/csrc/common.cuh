@@ -308,6 +308,9 @@ DEVI float sum2(uint32_t packed) {
   return __uint_as_float(packed << 16) + __uint_as_float(packed & 0xffff0000u);
 }
 
+DEVI void store_out(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+DEVI void store_out(__half* p, float v) { *p = __float2half_rn(v); }
+
 DEVI int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace attn

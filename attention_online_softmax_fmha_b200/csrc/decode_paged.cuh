@@ -1,0 +1,538 @@
+// Decode against a paged KV cache, split over persistent CTAs (MATE
+// "Attention", FMHA: flash_attn_with_kvcache with scheduler metadata and
+// flash_attn_combine; MindSpore "sparse_flash_attention": PA_BSND cache of
+// (block_num, block_size, N, D) with a block table).
+//
+// One segment = (sequence b, KV head g, block of <= 16 query rows that read
+// g: (query token, head) pairs). Its KV stream is cut into 64-key tiles;
+// logical key t lives in row t % page_size of physical page
+// block_table[b][t / page_size].
+//
+// The work is HBM-bound (about 4 flop per KV byte at s_q = 1, H_q/H_kv = 4),
+// so the design goal is a full memory pipe, not tensor throughput:
+//   warp 4      producer: reads the block-table entries 32 at a time and
+//               issues one TMA box per (page, 64-column chunk) for K and V,
+//               128-byte swizzled, into a 6-stage ring (32 KB per stage).
+//   warps 0-3   consumers: warp w owns keys [16w, 16w + 16) of every tile and
+//               keeps its own online-softmax state (running max, sums, O in
+//               registers). S = Q K^T and O += P V use mma.sync m16n8k16 with
+//               fp32 accumulation; their cost is far below the tile's load
+//               time. At the end of a segment piece the four warp states are
+//               merged through shared memory.
+// A piece that is the whole segment writes O (bf16) and LSE directly; a piece
+// of a split segment writes a sink-free partial (O / l, LSE) to the workspace
+// for the combine kernel.
+#pragma once
+
+#include "common.cuh"
+#include "sched.cuh"
+
+namespace attn {
+
+constexpr int kDecTileKeys = 64;
+constexpr int kDecRows = 16;       // query rows per segment (mma M)
+constexpr int kDecStages = 6;
+
+struct DecodeParams {
+  const void* q;
+  void* out;
+  float* lse;
+  const int32_t* block_table;
+  const int32_t* cache_seqlens;
+  const int32_t* meta;       // nullptr: one CTA per segment, no split
+  float* ws_o;               // [slot][kDecRows][D]
+  float* ws_lse;             // [slot][kDecRows]
+  const float* sink;
+  int64_t bt_stride;
+  int64_t q_sb, q_ss, q_sh;
+  int64_t o_sb, o_ss, o_sh;
+  int32_t batch, seqlen_q, heads_q, heads_kv, group, rows, n_rsub, segs_per_seq, num_segs;
+  int32_t page_size;
+  int32_t num_ctas;          // grid size with metadata
+  float scale_log2;
+  int32_t causal, window_left, window_right;
+};
+
+template <int D>
+struct DecodeCfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kDecTileKeys * D * 2;  // K or V tile
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kQStride = D * 2 + 16;               // padded Q row (bytes)
+  static constexpr int kStageOff = 0;
+  static constexpr int kQOff = kDecStages * kStageBytes;
+  static constexpr int kRedOff = kQOff + kDecRows * kQStride;  // merge buffers
+  static constexpr int kRedBytes = kDecRows * D * 4 + 4 * kDecRows * 4 * 3;
+  static constexpr int kBarOff = kRedOff + kRedBytes;
+  static constexpr int kSmemBytes = kBarOff + 2 * kDecStages * 8 + 64 + 1024;
+};
+
+struct DecodeSeg {
+  int b, g, rsub, len;
+  int t0, t1;  // visible tile range of the segment
+};
+
+DEVI void decode_seg(const DecodeParams& p, int s, DecodeSeg& sg) {
+  sg.b = s / p.segs_per_seq;
+  const int rem = s - sg.b * p.segs_per_seq;
+  sg.g = rem / p.n_rsub;
+  sg.rsub = rem - sg.g * p.n_rsub;
+  sg.len = p.cache_seqlens[sg.b];
+  // union of the rows' visible ranges (row i = 0 has the smallest left edge,
+  // i = s_q - 1 the largest right edge)
+  const int delta = sg.len - p.seqlen_q;
+  int lo = 0, hi = sg.len - 1;
+  if (p.window_left >= 0) lo = max(lo, delta - p.window_left);
+  if (p.causal) hi = min(hi, p.seqlen_q - 1 + delta);
+  if (p.window_right >= 0) hi = min(hi, p.seqlen_q - 1 + delta + p.window_right);
+  if (hi < lo) {
+    sg.t0 = sg.t1 = 0;
+  } else {
+    sg.t0 = lo / kDecTileKeys;
+    sg.t1 = hi / kDecTileKeys + 1;
+  }
+}
+
+// ---- mma.sync / ldmatrix helpers -------------------------------------------
+DEVI void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+DEVI void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+template <bool kFp16>
+DEVI void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  if (kFp16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+DEVI void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Address of the 16-byte chunk holding (row, col..col+7) of a 128-byte-
+// swizzled tile made of 64-column chunks of `rows` rows each.
+DEVI uint32_t sw128_addr(uint32_t base, int rows, int row, int col) {
+  const int chunk = col >> 6;
+  const int c16 = (col & 63) >> 3;
+  return base + chunk * rows * 128 + row * 128 + ((c16 ^ (row & 7)) << 4);
+}
+
+// ---------------------------------------------------------------------------
+template <int D>
+DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CUtensorMap* mv,
+                          uint8_t* smem, uint64_t* full, uint64_t* empty, volatile int* abort,
+                          int seg_begin_units, int seg_end_units, int first_seg,
+                          const int32_t* seg_prefix) {
+  using C = DecodeCfg<D>;
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) {
+    tma_prefetch_desc(mk);
+    tma_prefetch_desc(mv);
+  }
+  int it = 0;
+  const int P = p.page_size;
+  const int loads_per_tile = P >= kDecTileKeys ? 1 : kDecTileKeys / P;
+  const int box_rows = P >= kDecTileKeys ? kDecTileKeys : P;
+  int u = seg_begin_units, s = first_seg;
+  while (u < seg_end_units) {
+    // segment s covers units [seg_prefix(s), seg_prefix(s+1)) (or all of
+    // one segment without metadata)
+    int sb, se;
+    if (seg_prefix) {
+      sb = seg_prefix[s];
+      se = seg_prefix[s + 1];
+      if (se <= u) { ++s; continue; }
+    } else {
+      sb = u;
+      se = seg_end_units;
+    }
+    DecodeSeg sg;
+    decode_seg(p, s, sg);
+    const int a = u - sb, e = min(seg_end_units, se) - sb;  // tiles [a, e) of this segment
+    const int32_t* bt = p.block_table + (int64_t)sg.b * p.bt_stride;
+    const int npages_seq = (sg.len + P - 1) / P;
+    // A window of 32 block-table entries lives in the lanes' registers
+    // (lane x holds entry win0 + x) and is refilled when a tile leaves it.
+    int win0 = -(1 << 30), win_val = 0;
+    for (int t = a; t < e; ++t) {
+      if (t < sg.t0 || t >= sg.t1) continue;  // no visible key: skipped by all roles
+      const int st = it % kDecStages;
+      const int first_page = (t * kDecTileKeys) / P;
+      const int nload = min(loads_per_tile, npages_seq - first_page);
+      if (first_page < win0 || first_page + nload > win0 + 32) {
+        win0 = first_page;
+        win_val = (win0 + lane < npages_seq) ? bt[win0 + lane] : 0;
+      }
+      const int row_in_page = (t * kDecTileKeys) % P;  // 0 unless P > 64
+      if (it >= kDecStages) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&empty[st], ((it / kDecStages) - 1) & 1, abort, 31);
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
+      }
+      if (lane == 0)
+        mbar_expect_tx(&full[st], 2u * nload * box_rows * D * 2);
+      __syncwarp();
+      uint8_t* kdst = smem + C::kStageOff + st * C::kStageBytes;
+      uint8_t* vdst = kdst + C::kTileBytes;
+      for (int j = 0; j < nload; ++j) {
+        const int page = __shfl_sync(0xffffffffu, win_val, first_page + j - win0);
+        if (lane == 0) {
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c) {
+            tma_load_4d(kdst + c * kDecTileKeys * 128 + j * box_rows * 128, mk, &full[st],
+                        c * 64, sg.g, row_in_page, page);
+            tma_load_4d(vdst + c * kDecTileKeys * 128 + j * box_rows * 128, mv, &full[st],
+                        c * 64, sg.g, row_in_page, page);
+          }
+        }
+      }
+      ++it;
+    }
+    u = min(seg_end_units, se);
+    ++s;
+  }
+  // drain: the last stages' copies must land before the CTA exits
+  if (lane == 0) {
+    int zero = 0;
+    for (int i = max(0, it - kDecStages); i < it; ++i)
+      mbar_wait(&full[i % kDecStages], (i / kDecStages) & 1, &zero, 32);
+  }
+}
+
+// ---------------------------------------------------------------------------
+template <int D, bool kFp16>
+DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, uint64_t* empty,
+                          volatile int* abort, int seg_begin_units, int seg_end_units,
+                          int first_seg, const int32_t* seg_prefix) {
+  using C = DecodeCfg<D>;
+  using InT = typename std::conditional<kFp16, __half, __nv_bfloat16>::type;
+  const int tid = threadIdx.x;  // 0..127
+  const int warp = tid >> 5, lane = tid & 31;
+  const int qr = lane >> 2;          // fragment row (and row + 8)
+  const int qc = (lane & 3) * 2;     // fragment column pair
+  uint8_t* qs = smem + C::kQOff;
+  float* red_o = reinterpret_cast<float*>(smem + C::kRedOff);  // [16][D]
+  float* red_m = red_o + kDecRows * D;                          // [4 warps][16]
+  float* red_l = red_m + 4 * kDecRows;
+  float* red_r = red_l + 4 * kDecRows;
+  const int32_t* meta = p.meta;
+  const MetaLayout ml(p.num_ctas, p.num_segs);
+  int it = 0;
+  int u = seg_begin_units, s = first_seg;
+  while (u < seg_end_units) {
+    int sb, se;
+    if (seg_prefix) {
+      sb = seg_prefix[s];
+      se = seg_prefix[s + 1];
+      if (se <= u) { ++s; continue; }
+    } else {
+      sb = u;
+      se = seg_end_units;
+    }
+    DecodeSeg sg;
+    decode_seg(p, s, sg);
+    const int a = u - sb, e = min(seg_end_units, se) - sb;
+    const int row0 = sg.rsub * kDecRows;
+    const int nrows = min(kDecRows, p.rows - row0);
+
+    // --- Q rows of the segment -> shared memory (bf16, zero padded) ---
+    named_barrier(1, 128);  // previous piece finished with qs / red
+    for (int x = tid; x < kDecRows * (D / 8); x += 128) {
+      const int r = x / (D / 8), c8 = x % (D / 8);
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (r < nrows) {
+        const int rr = row0 + r;
+        const int i = rr / p.group, h = sg.g * p.group + rr % p.group;
+        const InT* src = reinterpret_cast<const InT*>(p.q) + sg.b * p.q_sb + i * p.q_ss +
+                         h * p.q_sh + c8 * 8;
+        v = *reinterpret_cast<const uint4*>(src);
+      }
+      *reinterpret_cast<uint4*>(qs + r * C::kQStride + c8 * 16) = v;
+    }
+    named_barrier(1, 128);
+    uint32_t qa[D / 16][4];
+    {
+      const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int cofs = (lane >> 4) * 8;
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k)
+        ldsm_x4(smem_u32(qs + r * C::kQStride + (k * 16 + cofs) * 2), qa[k]);
+    }
+    // per-row visible key range (rows qr and qr + 8)
+    int lo[2], hi[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int rr = row0 + qr + h2 * 8;
+      const int i = min(rr, p.rows - 1) / p.group;
+      const int delta = sg.len - p.seqlen_q;
+      lo[h2] = 0;
+      hi[h2] = sg.len - 1;
+      if (p.window_left >= 0) lo[h2] = max(lo[h2], i + delta - p.window_left);
+      if (p.causal) hi[h2] = min(hi[h2], i + delta);
+      if (p.window_right >= 0) hi[h2] = min(hi[h2], i + delta + p.window_right);
+    }
+    float o[D / 8][4];
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f}, l_rnd[2] = {0.f, 0.f};
+    const float sl2 = p.scale_log2;
+
+    for (int t = a; t < e; ++t) {
+      if (t < sg.t0 || t >= sg.t1) continue;
+      const int st = it % kDecStages;
+      if (!warp_wait(&full[st], (it / kDecStages) & 1, abort, 33)) return;
+      const uint32_t kbase = smem_u32(smem + C::kStageOff + st * C::kStageBytes);
+      const uint32_t vbase = kbase + C::kTileBytes;
+      const int key0 = t * kDecTileKeys + warp * 16;  // this warp's first key
+      // Keys past the end of the sequence hold whatever the page has there:
+      // zero their V rows so that P = 0 never meets a NaN.
+      if (key0 + 16 > sg.len) {
+        for (int x = lane; x < 16 * (D / 8); x += 32) {
+          const int kr = x / (D / 8), c8 = x % (D / 8);
+          if (key0 + kr >= sg.len) {
+            const uint32_t ad = sw128_addr(vbase, kDecTileKeys, warp * 16 + kr, c8 * 8);
+            asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(ad), "r"(0) : "memory");
+          }
+        }
+        __syncwarp();
+      }
+      // S = Q K^T for this warp's 16 keys: two n-tiles of 8 keys
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int kr = warp * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int cofs = ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          uint32_t b[4];
+          ldsm_x4(sw128_addr(kbase, kDecTileKeys, kr, k * 16 + cofs), b);
+          mma16816<kFp16>(sacc[0], qa[k], b[0], b[1]);
+          mma16816<kFp16>(sacc[1], qa[k], b[2], b[3]);
+        }
+      }
+      // mask, running max (rows qr, qr+8 across the 4 lanes of a quad)
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const int key = key0 + nt * 8 + qc + (x & 1);
+          const int h2 = x >> 1;
+          if (key < lo[h2] || key > hi[h2]) sacc[nt][x] = -INFINITY;
+          mx[h2] = fmaxf(mx[h2], sacc[nt][x]);
+        }
+      float alpha[2], m_use[2];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 1));
+        mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 2));
+        const float mn = fmaxf(m_run[h2], mx[h2] * sl2);
+        alpha[h2] = (m_run[h2] == -INFINITY) ? 1.f : ex2(m_run[h2] - mn);
+        m_run[h2] = mn;
+        m_use[h2] = (mn == -INFINITY) ? 0.f : mn;
+        l_run[h2] *= alpha[h2];
+        l_rnd[h2] *= alpha[h2];
+      }
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        o[n][0] *= alpha[0];
+        o[n][1] *= alpha[0];
+        o[n][2] *= alpha[1];
+        o[n][3] *= alpha[1];
+      }
+      // P (rounded to the input type) as the A operand of P V
+      uint32_t pa[4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const float p0 = ex2(fmaf(sacc[nt][2 * h2], sl2, -m_use[h2]));
+          const float p1 = ex2(fmaf(sacc[nt][2 * h2 + 1], sl2, -m_use[h2]));
+          const uint32_t pk = pack2<kFp16>(p0, p1);
+          pa[nt * 2 + h2] = pk;
+          l_run[h2] += p0 + p1;
+          l_rnd[h2] += sum2<kFp16>(pk);
+        }
+      // O += P V over this warp's 16 keys: 16 d-tiles of 8
+      {
+        const int kr = warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int cofs = (lane >> 4) * 8;
+#pragma unroll
+        for (int n2 = 0; n2 < D / 16; ++n2) {
+          uint32_t b[4];
+          ldsm_x4_t(sw128_addr(vbase, kDecTileKeys, kr, n2 * 16 + cofs), b);
+          mma16816<kFp16>(o[2 * n2], pa, b[0], b[1]);
+          mma16816<kFp16>(o[2 * n2 + 1], pa, b[2], b[3]);
+        }
+      }
+      // this warp is done with the stage (zeroed rows included)
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      ++it;
+    }
+
+    // --- merge the four warps' states -----------------------------------
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      l_run[h2] += __shfl_xor_sync(0xffffffffu, l_run[h2], 1);
+      l_run[h2] += __shfl_xor_sync(0xffffffffu, l_run[h2], 2);
+      l_rnd[h2] += __shfl_xor_sync(0xffffffffu, l_rnd[h2], 1);
+      l_rnd[h2] += __shfl_xor_sync(0xffffffffu, l_rnd[h2], 2);
+    }
+    if ((lane & 3) == 0) {
+      red_m[warp * kDecRows + qr] = m_run[0];
+      red_m[warp * kDecRows + qr + 8] = m_run[1];
+    }
+    for (int x = tid; x < kDecRows * D; x += 128) red_o[x] = 0.f;
+    named_barrier(1, 128);
+    float scale_w[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int r = qr + h2 * 8;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w * kDecRows + r]);
+      scale_w[h2] = (m_run[h2] == -INFINITY) ? 0.f : ex2(m_run[h2] - M);
+      if ((lane & 3) == 0) {
+        red_l[warp * kDecRows + r] = l_run[h2] * scale_w[h2];
+        red_r[warp * kDecRows + r] = l_rnd[h2] * scale_w[h2];
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      const int c = n * 8 + qc;
+      atomicAdd(&red_o[qr * D + c], o[n][0] * scale_w[0]);
+      atomicAdd(&red_o[qr * D + c + 1], o[n][1] * scale_w[0]);
+      atomicAdd(&red_o[(qr + 8) * D + c], o[n][2] * scale_w[1]);
+      atomicAdd(&red_o[(qr + 8) * D + c + 1], o[n][3] * scale_w[1]);
+    }
+    named_barrier(1, 128);
+
+    // --- write: thread -> (row, 16 columns) --------------------------------
+    {
+      int nsplit = 1, slot = -1;
+      if (meta) {
+        nsplit = meta[ml.seg_nsplit + s];
+        if (nsplit > 1) slot = meta[ml.seg_slot + s] + (blockIdx.x - meta[ml.seg_first + s]);
+      }
+      constexpr int kPer = D / 8;  // columns per thread (8 threads per row)
+      const int r = tid >> 3, c0 = (tid & 7) * kPer;
+      if (r < nrows) {
+        float M = -INFINITY, L = 0.f, LR = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          M = fmaxf(M, red_m[w * kDecRows + r]);
+          L += red_l[w * kDecRows + r];
+          LR += red_r[w * kDecRows + r];
+        }
+        const float m_use = (M == -INFINITY) ? 0.f : M;
+        const float lse2 = L > 0.f ? m_use + log2f(L) : -INFINITY;
+        const int rr = row0 + r;
+        const int i = rr / p.group, h = sg.g * p.group + rr % p.group;
+        if (slot < 0) {
+          float denom = LR;
+          if (p.sink) denom += ex2(p.sink[h] * kLog2e - m_use);
+          const float inv = denom > 0.f ? 1.f / denom : 0.f;
+          InT* dst = reinterpret_cast<InT*>(p.out) + sg.b * p.o_sb + i * p.o_ss + h * p.o_sh + c0;
+#pragma unroll
+          for (int c = 0; c < kPer; c += 8) {
+            uint4 w;
+            w.x = pack2<kFp16>(red_o[r * D + c0 + c] * inv, red_o[r * D + c0 + c + 1] * inv);
+            w.y = pack2<kFp16>(red_o[r * D + c0 + c + 2] * inv, red_o[r * D + c0 + c + 3] * inv);
+            w.z = pack2<kFp16>(red_o[r * D + c0 + c + 4] * inv, red_o[r * D + c0 + c + 5] * inv);
+            w.w = pack2<kFp16>(red_o[r * D + c0 + c + 6] * inv, red_o[r * D + c0 + c + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + c) = w;
+          }
+          if (p.lse && (tid & 7) == 0)
+            p.lse[((int64_t)sg.b * p.heads_q + h) * p.seqlen_q + i] = lse2 * kLn2;
+        } else {
+          const float inv = LR > 0.f ? 1.f / LR : 0.f;
+          float* dst = p.ws_o + ((int64_t)slot * kDecRows + r) * D + c0;
+#pragma unroll
+          for (int c = 0; c < kPer; c += 4)
+            *reinterpret_cast<float4*>(dst + c) =
+                make_float4(red_o[r * D + c0 + c] * inv, red_o[r * D + c0 + c + 1] * inv,
+                            red_o[r * D + c0 + c + 2] * inv, red_o[r * D + c0 + c + 3] * inv);
+          if ((tid & 7) == 0) p.ws_lse[(int64_t)slot * kDecRows + r] = lse2 * kLn2;
+        }
+      }
+    }
+    u = min(seg_end_units, se);
+    ++s;
+  }
+}
+
+template <int D, bool kFp16>
+__global__ void __launch_bounds__(160, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap map_k,
+                  const __grid_constant__ CUtensorMap map_v, const DecodeParams p) {
+  using C = DecodeCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* empty = full + kDecStages;
+  int* abort = reinterpret_cast<int*>(empty + kDecStages);
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDecStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);
+    }
+    *abort = 0;
+    s_bad = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // This CTA's unit range and first segment.
+  int ub, ue, s0;
+  const int32_t* seg_prefix = nullptr;
+  if (p.meta) {
+    const MetaLayout ml(p.num_ctas, p.num_segs);
+    if (threadIdx.x == 0 &&
+        !(meta_matches(p.meta, ATTN_SCHED_MHA, p.batch, p.seqlen_q, p.heads_q, p.heads_kv,
+                       p.page_size, p.num_segs, kDecTileKeys, D, D) &&
+          p.meta[kMetaNumCtas] == p.num_ctas)) {
+      raise_error(ATTN_DEVERR_META_MISMATCH, 40);
+      s_bad = 1;
+    }
+    __syncthreads();
+    if (s_bad) return;
+    ub = p.meta[ml.cta_begin + blockIdx.x];
+    ue = p.meta[ml.cta_begin + blockIdx.x + 1];
+    s0 = p.meta[ml.cta_seg + blockIdx.x];
+    seg_prefix = p.meta + ml.seg_begin;
+  } else {
+    // one CTA per segment: all of its tiles
+    s0 = blockIdx.x;
+    const int b = s0 / p.segs_per_seq;
+    const int len = p.cache_seqlens[b];
+    ub = 0;
+    ue = len > 0 ? (len + kDecTileKeys - 1) / kDecTileKeys : 0;
+    if (ue == 0) ue = 1;  // still write O = 0, LSE = -inf for an empty sequence
+  }
+  if (threadIdx.x >= 128) {
+    decode_producer<D>(p, &map_k, &map_v, smem, full, empty, abort, ub, ue, s0, seg_prefix);
+  } else {
+    decode_consumer<D, kFp16>(p, smem, full, empty, abort, ub, ue, s0, seg_prefix);
+  }
+}
+
+}  // namespace attn

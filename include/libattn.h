@@ -196,7 +196,8 @@ attn_status_t attn_sched_metadata(const attn_sched_args* args, void* stream);
 /* meta: from attn_sched_metadata(mode=ATTN_SCHED_MHA, same args), or NULL   */
 /*   for one CTA per (sequence, KV head) and no splitting.                   */
 /* workspace: device buffer of attn_paged_workspace_size() bytes (partial   */
-/*   O and LSE of the splits); may be NULL when meta is NULL.                */
+/*   O and LSE of the splits); may be NULL when meta is NULL. The combine    */
+/*   step runs inside this call.                                             */
 /* Supported now: bf16, D in {64, 128}, page_size in {16, 32, 64, 128, 256}, */
 /*   s_q * H_q / H_kv <= 16.                                                 */
 /* ------------------------------------------------------------------------ */
@@ -229,11 +230,13 @@ typedef struct {
   const float* sink;
   const int32_t* meta;
   size_t meta_bytes;
+  int32_t num_ctas;       /* the num_ctas given to attn_sched_metadata (0 = SMs) */
   void* workspace;
   size_t workspace_bytes;
 } attn_paged_args;
 
-size_t attn_paged_workspace_size(const attn_paged_args* args, const attn_sched_args* sched);
+/* Bytes of workspace for these arguments (host only; 0 when meta is NULL).  */
+size_t attn_paged_workspace_size(const attn_paged_args* args);
 attn_status_t attn_fwd_paged_kvcache(const attn_paged_args* args, void* stream);
 
 /* ------------------------------------------------------------------------ */
@@ -314,11 +317,13 @@ typedef struct {
   int32_t causal;
   const int32_t* meta;
   size_t meta_bytes;
+  int32_t num_ctas;           /* the num_ctas given to attn_sched_metadata    */
   void* workspace;
   size_t workspace_bytes;
 } mla_args;
 
-size_t mla_workspace_size(const mla_args* args, const attn_sched_args* sched);
+/* Bytes of workspace for these arguments (host only; 0 when meta is NULL).  */
+size_t mla_workspace_size(const mla_args* args);
 attn_status_t mla_fwd_paged(const mla_args* args, void* stream);
 
 /* ------------------------------------------------------------------------ */
