@@ -117,13 +117,13 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   p.batch = a.batch;
   p.seqlen_q = a.max_seqlen_q;
   p.seqlen_k = a.max_seqlen_k;
-  p.num_q_tiles = (a.max_seqlen_q + kPrefillBM - 1) / kPrefillBM;
+  p.num_units_q = (a.max_seqlen_q + kPrefillUnit - 1) / kPrefillUnit;
   p.num_heads_q = a.num_heads_q;
   p.num_heads_kv = a.num_heads_kv;
   p.group = a.num_heads_q / a.num_heads_kv;
-  const int64_t total = (int64_t)p.num_q_tiles * a.batch * a.num_heads_q;
+  const int64_t total = (int64_t)p.num_units_q * a.batch * a.num_heads_q;
   if (total > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
-  p.total_tiles = (int32_t)total;
+  p.total_units = (int32_t)total;
   p.scale_log2 = a.scale * kLog2e;
   p.causal = a.causal;
   p.window_left = a.window_left;
@@ -132,13 +132,18 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   auto kernel = prefill_kernel<D, kFp16>;
   static bool configured = false;
   if (!configured) {
+    // The warpgroups trade registers with setmaxnreg out of the block's
+    // launch allocation; that split is only valid at exactly this count.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (fa.numRegs != kPrefillLaunchRegs) return ATTN_ERR_UNSUPPORTED;
     if (set_smem(kernel, C::kSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
     configured = true;
   }
   const int sms = device_sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(total, sms);
-  kernel<<<grid, 192, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+  kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
   return launch_status(cudaGetLastError());
 }
 

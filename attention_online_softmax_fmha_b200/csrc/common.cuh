@@ -314,3 +314,146 @@ DEVI void store_out(__half* p, float v) { *p = __float2half_rn(v); }
 DEVI int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace attn
+
+namespace attn {
+
+// ---------------------------------------------------------------------------
+// Packed fp32x2 arithmetic (sm_100: two fp32 lanes per instruction)
+// ---------------------------------------------------------------------------
+DEVI uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+DEVI void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+DEVI uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+DEVI uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+DEVI uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// The two 16-bit floats of a packed word, widened to fp32 (exact).
+template <bool kFp16>
+DEVI uint64_t widen2(uint32_t packed) {
+  if (kFp16) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&packed));
+    return f2pack(f.x, f.y);
+  }
+  return f2pack(__uint_as_float(packed << 16), __uint_as_float(packed & 0xffff0000u));
+}
+
+// Register reallocation between warpgroups (all warps of a warpgroup execute it).
+template <uint32_t N>
+DEVI void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <uint32_t N>
+DEVI void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
+// 32 lanes x 128 columns of 32 bits in one load (outputs valid on return).
+DEVI void tmem_load128(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
+      "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
+      "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127},"
+      " [%128];\n\ttcgen05.wait::ld.sync.aligned;"
+      : ATTN_R16(0), ATTN_R16(16), ATTN_R16(32), ATTN_R16(48), ATTN_R16(64), ATTN_R16(80),
+        ATTN_R16(96), ATTN_R16(112)
+      : "r"(taddr)
+      : "memory");
+}
+
+}  // namespace attn
+
+namespace attn {
+
+// 2^x for a pair of fp32 values on the FMA pipe (no MUFU), for x <= 64.
+// Range reduction x = j + f with j = rint(x) (adding 1.5 * 2^23 rounds to an
+// integer in the low mantissa bits), f in [-0.5, 0.5]; 2^f by a degree-3
+// polynomial whose coefficients minimise the maximum relative error on
+// [-0.5, 0.5] (a linear-programming minimax fit, max relative error 7.5e-5);
+// 2^j is added to the exponent field with an integer multiply-add. Inputs
+// below -126 are clamped: the result is then a tiny positive number
+// (<= 2^-125), not 0.
+DEVI uint64_t exp2_poly_x2(float x0, float x1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = add2(x, f2pack(kMagic, kMagic));
+  const uint64_t jf = add2(t, f2pack(-kMagic, -kMagic));
+  const uint64_t f = fma2(jf, f2pack(-1.f, -1.f), x);
+  uint64_t p = fma2(f2pack(0.05517222f, 0.05517222f), f, f2pack(0.24261115f, 0.24261115f));
+  p = fma2(p, f, f2pack(0.69326085f, 0.69326085f));
+  p = fma2(p, f, f2pack(0.99992806f, 0.99992806f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  uint32_t r0, r1;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r0) : "r"(__float_as_uint(t0)), "r"(__float_as_uint(p0)));
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r1) : "r"(__float_as_uint(t1)), "r"(__float_as_uint(p1)));
+  return f2pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
+}  // namespace attn
+
+namespace attn {
+
+// Warp-wide forms of the MMA issue: the whole warp runs the issuing loop (its
+// values stay warp-uniform, so descriptors live in uniform registers) and
+// one elected lane issues each tcgen05 instruction.
+DEVI void mma_f16_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+DEVI void mma_f16_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+DEVI void mma_f8_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                      uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+DEVI void mma_f8_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                      uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+DEVI void tc_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+}  // namespace attn

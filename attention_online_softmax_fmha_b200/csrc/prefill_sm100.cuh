@@ -8,19 +8,25 @@
 // "flash_attention": causal, window_size; MindSpore "sparse_flash_attention":
 // sparse_mode=3 "rightDownCausal").
 //
-// Design (one CTA per SM, persistent over (q-tile, batch, head) work tiles,
-// heaviest q tiles first):
-//   warp 4      TMA producer: Q tile (128 rows) and a ring of K/V tiles of
-//               128 keys, 128-byte swizzled, one head per box.
-//   warp 5      TMEM owner and MMA issuer (one thread): S = Q K^T into one of
-//               two TMEM S buffers (128 x 128 fp32), then O += P V with P read
-//               from TMEM (bf16, written over its S buffer) and V from smem.
-//   warps 0-3   softmax: thread r owns query row r (= TMEM lane r). Online
-//               softmax in the log2 domain: running max m, running sum l;
-//               O in TMEM is rescaled only when the max grows by more than
-//               2^8 (exact after the final division by l).
-// Every mbarrier wait is bounded; a timeout raises ATTN_DEVERR_TIMEOUT, the
-// roles unwind, in-flight copies and MMAs are drained and TMEM is freed.
+// Design: one CTA per SM, persistent over work units of 256 query rows (two
+// 128-row tiles Q0, Q1 of one sequence and head; heaviest units first). Both
+// tiles stream the same K/V tiles of 128 keys.
+//   warpgroup 0, 1   softmax of Q0 / Q1: thread r owns query row r of its
+//                    tile (= TMEM lane r). Online softmax in the log2 domain;
+//                    O in TMEM is rescaled only when a row's max grows by more
+//                    than 2^8 (exact after the final division).
+//   warp 8           TMA producer: Q0, Q1 and a ring of K/V tiles, 128-byte
+//                    swizzled, one head per box.
+//   warp 9           TMEM owner and MMA issuer (one thread), in the order
+//                    S0_j, PV1_{j-1}, S1_j, PV0_j, ... so that the tensor core
+//                    works on one tile while the other tile's softmax runs.
+//                    S_w = Q_w K^T lands in TMEM; P_w (bf16) overwrites it and
+//                    is the TMEM A operand of O_w += P_w V.
+//   warps 10, 11     idle (they complete the register warpgroup).
+// Registers move from warpgroup 2 to the softmax warpgroups with setmaxnreg;
+// the host checks the kernel's register count before launching.
+// Every mbarrier wait is bounded; a timeout raises ATTN_DEVERR_TIMEOUT and the
+// roles unwind, draining in-flight copies and MMAs before TMEM is freed.
 #pragma once
 
 #include "common.cuh"
@@ -41,47 +47,61 @@ struct PrefillParams {
   int32_t batch;
   int32_t seqlen_q;     // padded S_q (unused for varlen)
   int32_t seqlen_k;
-  int32_t num_q_tiles;  // ceil(max_seqlen_q / 128)
+  int32_t num_units_q;  // ceil(max_seqlen_q / 256)
   int32_t num_heads_q;
   int32_t num_heads_kv;
   int32_t group;        // H_q / H_kv
-  int32_t total_tiles;
+  int32_t total_units;
   float scale_log2;     // scale * log2(e)
   int32_t causal;
   int32_t window_left;
   int32_t window_right;
 };
 
-constexpr int kPrefillBM = 128;   // query rows per tile
-constexpr int kPrefillBN = 128;   // keys per tile
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kPrefillBM = 128;               // query rows per tile
+constexpr int kPrefillUnit = 2 * kPrefillBM;  // query rows per work unit
+constexpr int kPrefillBN = 128;               // keys per tile
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
+// Of every 16 P pairs, this many are exponentiated on the FMA pipe (a
+// polynomial) and the rest on the MUFU pipe, to balance the two.
+constexpr int kEmuPairs = 4;
+constexpr int kPrefillThreads = 384;
+constexpr int kPrefillLaunchRegs = 168;       // 65536 / 384, rounded down to 8
+constexpr int kPrefillSoftmaxRegs = 208;
+constexpr int kPrefillOtherRegs = 88;
+static_assert(2 * 128 * kPrefillSoftmaxRegs + 128 * kPrefillOtherRegs <=
+                  kPrefillThreads * kPrefillLaunchRegs,
+              "register split exceeds the launch allocation");
 
 template <int D>
 struct PrefillCfg {
   static constexpr int kChunks = D / 64;                 // 128-byte column chunks
-  static constexpr int kStages = (D == 64) ? 4 : 3;
+  // K and V tiles have separate rings: K is released as soon as both S MMAs
+  // have read it, V after both P V MMAs.
+  static constexpr int kKStages = (D == 64) ? 4 : 3;
+  static constexpr int kVStages = (D == 64) ? 4 : 2;
   static constexpr int kChunkBytes = 128 * 128;          // 128 rows x 128 bytes
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  static constexpr int kQOff = 0;                        // Q0, Q1
+  static constexpr int kKOff = 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers, + alignment slack
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128;
+  static constexpr uint32_t kTmemO0 = 256, kTmemO1 = 256 + D;
 };
 
 struct PrefillBarriers {
   uint64_t q_full, q_empty;
-  uint64_t k_full[4], v_full[4], kv_empty[4];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_full, o_empty;
+  uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
   int32_t abort;
 };
 
-struct PrefillTile {
+struct PrefillUnit {
   int b, h, m;
   int len_q, len_k;
   int row_q, row_k;  // first packed row of this sequence (0 for padded)
@@ -89,41 +109,41 @@ struct PrefillTile {
   int kt0, kt1;      // key tiles [kt0, kt1)
 };
 
-// Maps a linear work index to a tile; returns false for tiles past the end
-// of their sequence. Every role calls this with the same t and gets the same
-// answer, so all roles skip the same tiles.
-DEVI bool prefill_tile(const PrefillParams& p, int t, PrefillTile& ti) {
+// Maps a linear work index to a unit; returns false for units past the end
+// of their sequence. Every role calls this with the same index and gets the
+// same answer, so all roles skip the same units.
+DEVI bool prefill_unit(const PrefillParams& p, int t, PrefillUnit& u) {
   const int bh = p.batch * p.num_heads_q;
   const int mr = t / bh;
   const int rem = t - mr * bh;
-  ti.b = rem / p.num_heads_q;
-  ti.h = rem - ti.b * p.num_heads_q;
-  ti.m = p.num_q_tiles - 1 - mr;
+  u.b = rem / p.num_heads_q;
+  u.h = rem - u.b * p.num_heads_q;
+  u.m = p.num_units_q - 1 - mr;
   if (p.cu_q != nullptr) {
-    ti.row_q = p.cu_q[ti.b];
-    ti.len_q = p.cu_q[ti.b + 1] - ti.row_q;
-    ti.row_k = p.cu_k[ti.b];
-    ti.len_k = p.cu_k[ti.b + 1] - ti.row_k;
-    ti.bcoord = 0;
+    u.row_q = p.cu_q[u.b];
+    u.len_q = p.cu_q[u.b + 1] - u.row_q;
+    u.row_k = p.cu_k[u.b];
+    u.len_k = p.cu_k[u.b + 1] - u.row_k;
+    u.bcoord = 0;
   } else {
-    ti.row_q = ti.row_k = 0;
-    ti.len_q = p.seqlen_q;
-    ti.len_k = p.seqlen_k;
-    ti.bcoord = ti.b;
+    u.row_q = u.row_k = 0;
+    u.len_q = p.seqlen_q;
+    u.len_k = p.seqlen_k;
+    u.bcoord = u.b;
   }
-  const int q0 = ti.m * kPrefillBM;
-  if (q0 >= ti.len_q) return false;
-  const int q1 = min(q0 + kPrefillBM, ti.len_q) - 1;
-  const int delta = ti.len_k - ti.len_q;
-  int lo = 0, hi = ti.len_k - 1;
+  const int q0 = u.m * kPrefillUnit;
+  if (q0 >= u.len_q) return false;
+  const int q1 = min(q0 + kPrefillUnit, u.len_q) - 1;
+  const int delta = u.len_k - u.len_q;
+  int lo = 0, hi = u.len_k - 1;
   if (p.window_left >= 0) lo = max(lo, q0 + delta - p.window_left);
   if (p.causal) hi = min(hi, q1 + delta);
   if (p.window_right >= 0) hi = min(hi, q1 + delta + p.window_right);
   if (hi < lo) {
-    ti.kt0 = ti.kt1 = 0;
+    u.kt0 = u.kt1 = 0;
   } else {
-    ti.kt0 = lo / kPrefillBN;
-    ti.kt1 = hi / kPrefillBN + 1;
+    u.kt0 = lo / kPrefillBN;
+    u.kt1 = hi / kPrefillBN + 1;
   }
   return true;
 }
@@ -150,35 +170,40 @@ DEVI void prefill_producer(const PrefillParams& p, const CUtensorMap* mq, const 
   tma_prefetch_desc(mk);
   tma_prefetch_desc(mv);
   int it = 0, nq = 0;
-  for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
-    PrefillTile ti;
-    if (!prefill_tile(p, t, ti)) continue;
-    const int n = ti.kt1 - ti.kt0;
+  for (int t = blockIdx.x; t < p.total_units; t += gridDim.x) {
+    PrefillUnit u;
+    if (!prefill_unit(p, t, u)) continue;
+    const int n = u.kt1 - u.kt0;
     if (n <= 0) continue;
-    const int hk = ti.h / p.group;
+    const int hk = u.h / p.group;
     if (nq > 0 && !mbar_wait(&bars->q_empty, (nq - 1) & 1, abort, 1)) goto drain;
-    mbar_expect_tx(&bars->q_full, C::kTileBytes);
+    mbar_expect_tx(&bars->q_full, 2 * C::kTileBytes);
 #pragma unroll
-    for (int c = 0; c < C::kChunks; ++c)
-      tma_load_4d(smem + C::kQOff + c * C::kChunkBytes, mq, &bars->q_full, c * 64, ti.h,
-                  ti.row_q + ti.m * kPrefillBM, ti.bcoord);
+    for (int w = 0; w < 2; ++w)
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_4d(smem + C::kQOff + w * C::kTileBytes + c * C::kChunkBytes, mq, &bars->q_full,
+                    c * 64, u.h, u.row_q + u.m * kPrefillUnit + w * kPrefillBM, u.bcoord);
     ++nq;
     for (int j = 0; j < n; ++j, ++it) {
-      const int s = it % C::kStages;
-      if (it >= C::kStages &&
-          !mbar_wait(&bars->kv_empty[s], ((it / C::kStages) - 1) & 1, abort, 2))
+      const int row = u.row_k + (u.kt0 + j) * kPrefillBN;
+      const int sk = it % C::kKStages, sv = it % C::kVStages;
+      if (it >= C::kKStages &&
+          !mbar_wait(&bars->k_empty[sk], ((it / C::kKStages) - 1) & 1, abort, 2))
         goto drain;
-      const int row = ti.row_k + (ti.kt0 + j) * kPrefillBN;
-      mbar_expect_tx(&bars->k_full[s], C::kTileBytes);
+      mbar_expect_tx(&bars->k_full[sk], C::kTileBytes);
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c)
-        tma_load_4d(smem + C::kKOff + s * C::kTileBytes + c * C::kChunkBytes, mk,
-                    &bars->k_full[s], c * 64, hk, row, ti.bcoord);
-      mbar_expect_tx(&bars->v_full[s], C::kTileBytes);
+        tma_load_4d(smem + C::kKOff + sk * C::kTileBytes + c * C::kChunkBytes, mk,
+                    &bars->k_full[sk], c * 64, hk, row, u.bcoord);
+      if (it >= C::kVStages &&
+          !mbar_wait(&bars->v_empty[sv], ((it / C::kVStages) - 1) & 1, abort, 4))
+        goto drain;
+      mbar_expect_tx(&bars->v_full[sv], C::kTileBytes);
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c)
-        tma_load_4d(smem + C::kVOff + s * C::kTileBytes + c * C::kChunkBytes, mv,
-                    &bars->v_full[s], c * 64, hk, row, ti.bcoord);
+        tma_load_4d(smem + C::kVOff + sv * C::kTileBytes + c * C::kChunkBytes, mv,
+                    &bars->v_full[sv], c * 64, hk, row, u.bcoord);
     }
   }
 drain:
@@ -187,16 +212,37 @@ drain:
   {
     int zero = 0;
     if (nq > 0) mbar_wait(&bars->q_full, (nq - 1) & 1, &zero, 3);
-    for (int i = max(0, it - C::kStages); i < it; ++i) {
-      mbar_wait(&bars->k_full[i % C::kStages], (i / C::kStages) & 1, &zero, 3);
-      mbar_wait(&bars->v_full[i % C::kStages], (i / C::kStages) & 1, &zero, 3);
-    }
+    for (int i = max(0, it - C::kKStages); i < it; ++i)
+      mbar_wait(&bars->k_full[i % C::kKStages], (i / C::kKStages) & 1, &zero, 3);
+    for (int i = max(0, it - C::kVStages); i < it; ++i)
+      mbar_wait(&bars->v_full[i % C::kVStages], (i / C::kVStages) & 1, &zero, 3);
   }
 }
 
 // ---------------------------------------------------------------------------
 // MMA warp (one thread issues)
 // ---------------------------------------------------------------------------
+// Descriptors are built once; a K step or a stage moves the start address,
+// which is the low 14-bit field (in 16-byte units) of the descriptor, so an
+// integer add of the offset in 16-byte units advances it (shared memory is
+// below 256 KB, the field never carries).
+template <int D>
+DEVI void prefill_issue_s(uint32_t d_tmem, uint64_t dq, uint64_t dk, uint32_t idesc) {
+  using C = PrefillCfg<D>;
+#pragma unroll
+  for (int k = 0; k < D / 16; ++k) {
+    const uint32_t off16 = (k >> 2) * (C::kChunkBytes >> 4) + (k & 3) * 2;
+    mma_f16_ss_w(d_tmem, dq + off16, dk + off16, idesc, k > 0 ? 1u : 0u);
+  }
+}
+DEVI void prefill_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t dv, uint32_t idesc,
+                           bool first) {
+#pragma unroll
+  for (int kk = 0; kk < kPrefillBN / 16; ++kk)
+    mma_f16_ts_w(d_tmem, a_tmem + kk * 8, dv + kk * (16 * 128 >> 4), idesc,
+               (!first || kk > 0) ? 1u : 0u);
+}
+
 template <int D, bool kFp16>
 DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* bars,
                       uint32_t tmem) {
@@ -204,97 +250,101 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
   volatile int* abort = &bars->abort;
   constexpr int fmt = kFp16 ? 0 : 1;
   constexpr uint32_t idesc_qk = make_idesc(128, kPrefillBN, fmt, 0, 0);
-  constexpr uint32_t idesc_pv = make_idesc(128, 64, fmt, 0, 1);
-  const uint32_t q_base = smem_u32(smem + C::kQOff);
-  const uint32_t k_base = smem_u32(smem + C::kKOff);
-  const uint32_t v_base = smem_u32(smem + C::kVOff);
-  int it = 0, sj = 0, nq = 0, o_tiles = 0;
+  // V is MN-major (d contiguous): one MMA covers all D columns; the 64-column
+  // chunks of the tile are kChunkBytes apart (leading byte offset), groups
+  // of 8 keys are 1024 bytes apart (stride byte offset).
+  constexpr uint32_t idesc_pv = make_idesc(128, D, fmt, 0, 1);
+  const uint64_t dq0 = sdesc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+  const uint64_t dq1 = dq0 + (C::kTileBytes >> 4);
+  const uint64_t dk_base = sdesc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
+  const uint64_t dv_base = sdesc_sw128(smem_u32(smem + C::kVOff), C::kChunkBytes, 1024);
+  const uint32_t tS0 = tmem + C::kTmemS0, tS1 = tmem + C::kTmemS1;
+  const uint32_t tO0 = tmem + C::kTmemO0, tO1 = tmem + C::kTmemO1;
+  int it = 0, nq = 0, units = 0;
 
-  auto issue_pv = [&](int jj, int tile_it, int tile_sj) -> bool {
-    const int b = (tile_sj + jj) & 1;
-    const int s = (tile_it + jj) % C::kStages;
-    if (!mbar_wait(&bars->p_full[b], ((tile_sj + jj) >> 1) & 1, abort, 11)) return false;
-    if (!mbar_wait(&bars->v_full[s], ((tile_it + jj) / C::kStages) & 1, abort, 12)) return false;
-    if (jj == 0 && o_tiles > 0 &&
-        !mbar_wait(&bars->o_empty, (o_tiles - 1) & 1, abort, 13))
-      return false;
-    tc_fence_after();
-    const uint32_t s_tmem = tmem + (b ? C::kTmemS1 : C::kTmemS0);
-    const uint32_t vs = v_base + s * C::kTileBytes;
-#pragma unroll
-    for (int kk = 0; kk < kPrefillBN / 16; ++kk) {
-#pragma unroll
-      for (int dc = 0; dc < C::kChunks; ++dc) {
-        const uint64_t bdesc = sdesc_sw128(vs + dc * C::kChunkBytes + kk * 16 * 128, 1024, 1024);
-        mma_f16_ts(tmem + C::kTmemO + dc * 64, s_tmem + kk * 8, bdesc, idesc_pv,
-                   (jj > 0 || kk > 0) ? 1u : 0u);
-      }
-    }
-    tc_commit(&bars->o_full);
-    tc_commit(&bars->kv_empty[s]);
-    return true;
-  };
-
-  for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
-    PrefillTile ti;
-    if (!prefill_tile(p, t, ti)) continue;
-    const int n = ti.kt1 - ti.kt0;
+  for (int t = blockIdx.x; t < p.total_units; t += gridDim.x) {
+    PrefillUnit u;
+    if (!prefill_unit(p, t, u)) continue;
+    const int n = u.kt1 - u.kt0;
     if (n <= 0) continue;
-    if (!mbar_wait(&bars->q_full, nq & 1, abort, 10)) goto drain;
+    if (!warp_wait(&bars->q_full, nq & 1, abort, 10)) goto drain;
     ++nq;
-    for (int j = 0; j < n; ++j) {
-      const int s = (it + j) % C::kStages;
-      const int b = (sj + j) & 1;
-      if (!mbar_wait(&bars->k_full[s], ((it + j) / C::kStages) & 1, abort, 14)) goto drain;
-      tc_fence_after();
-      const uint32_t s_tmem = tmem + (b ? C::kTmemS1 : C::kTmemS0);
-      const uint32_t ks = k_base + s * C::kTileBytes;
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t off = (k >> 2) * C::kChunkBytes + (k & 3) * 32;
-        mma_f16_ss(s_tmem, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(ks + off, 16, 1024),
-                   idesc_qk, k > 0 ? 1u : 0u);
+    // Order per key tile j: PV0_{j-1}, S0_j, PV1_{j-1}, S1_j. S_w needs the
+    // S_w/P_w buffer that PV_w_{j-1} reads; the tensor pipe runs in order.
+    for (int j = 0; j <= n; ++j) {
+      const int g = it + j;
+      const int s = g % C::kKStages;
+      const int sp = (g - 1) % C::kVStages;
+      if (j < n) {
+        if (!warp_wait(&bars->k_full[s], (g / C::kKStages) & 1, abort, 14)) goto drain;
       }
-      tc_commit(&bars->s_full[b]);
-      if (j == n - 1) tc_commit(&bars->q_empty);
-      if (j > 0 && !issue_pv(j - 1, it, sj)) goto drain;
+      if (j > 0) {
+        if (!warp_wait(&bars->p_full[0], (g - 1) & 1, abort, 11)) goto drain;
+        if (!warp_wait(&bars->v_full[sp], ((g - 1) / C::kVStages) & 1, abort, 12)) goto drain;
+        if (j == 1 && units > 0 && !warp_wait(&bars->o_empty[0], (units - 1) & 1, abort, 13))
+          goto drain;
+        tc_fence_after();
+        prefill_issue_pv(tO0, tS0, dv_base + sp * (C::kTileBytes >> 4), idesc_pv, j == 1);
+        if (j == n) tc_commit_w(&bars->o_full[0]);
+      } else {
+        tc_fence_after();
+      }
+      if (j < n) {
+        prefill_issue_s<D>(tS0, dq0, dk_base + s * (C::kTileBytes >> 4), idesc_qk);
+        tc_commit_w(&bars->s_full[0]);
+      }
+      if (j > 0) {
+        if (!warp_wait(&bars->p_full[1], (g - 1) & 1, abort, 11)) goto drain;
+        if (j == 1 && units > 0 && !warp_wait(&bars->o_empty[1], (units - 1) & 1, abort, 13))
+          goto drain;
+        tc_fence_after();
+        prefill_issue_pv(tO1, tS1, dv_base + sp * (C::kTileBytes >> 4), idesc_pv, j == 1);
+        if (j == n) tc_commit_w(&bars->o_full[1]);
+        tc_commit_w(&bars->v_empty[sp]);
+      }
+      if (j < n) {
+        prefill_issue_s<D>(tS1, dq1, dk_base + s * (C::kTileBytes >> 4), idesc_qk);
+        tc_commit_w(&bars->s_full[1]);
+        tc_commit_w(&bars->k_empty[s]);
+        if (j == n - 1) tc_commit_w(&bars->q_empty);
+      }
     }
-    if (!issue_pv(n - 1, it, sj)) goto drain;
     it += n;
-    sj += n;
-    ++o_tiles;
+    ++units;
   }
 drain : {
   // All issued MMAs must finish before TMEM is released.
   int zero = 0;
-  tc_commit(&bars->mma_drain);
-  mbar_wait(&bars->mma_drain, 0, &zero, 15);
+  tc_commit_w(&bars->mma_drain);
+  warp_wait(&bars->mma_drain, 0, &zero, 15);
 }
 }
 
 // ---------------------------------------------------------------------------
-// Softmax warpgroup (warps 0-3): one query row per thread
+// Softmax warpgroups: warpgroup w owns tile Q_w, one query row per thread
 // ---------------------------------------------------------------------------
 template <int D, bool kFp16>
-DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_t tmem) {
+DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_t tmem, int w) {
   using C = PrefillCfg<D>;
+  using OutT = typename std::conditional<kFp16, __half, __nv_bfloat16>::type;
   volatile int* abort = &bars->abort;
-  const int r = threadIdx.x;  // 0..127
+  const int r = threadIdx.x & 127;
   const uint32_t lane = (uint32_t)(r & ~31) << 16;
-  int sj = 0, pv = 0;
-  for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
-    PrefillTile ti;
-    if (!prefill_tile(p, t, ti)) continue;
-    const int n = ti.kt1 - ti.kt0;
-    const int i = ti.m * kPrefillBM + r;
-    const bool valid = i < ti.len_q;
-    using OutT = typename std::conditional<kFp16, __half, __nv_bfloat16>::type;
-    OutT* orow = reinterpret_cast<OutT*>(p.out) + ti.bcoord * p.o_sb +
-                 (int64_t)(ti.row_q + i) * p.o_ss + (int64_t)ti.h * p.o_sh;
-    float* lrow = p.lse ? p.lse + ti.b * p.lse_sb + ti.h * p.lse_sh + (ti.row_q + i) : nullptr;
+  const uint32_t s_tmem = tmem + (w ? C::kTmemS1 : C::kTmemS0) + lane;
+  const uint32_t o_tmem = tmem + (w ? C::kTmemO1 : C::kTmemO0) + lane;
+  int sj = 0, units = 0;
+  for (int t = blockIdx.x; t < p.total_units; t += gridDim.x) {
+    PrefillUnit u;
+    if (!prefill_unit(p, t, u)) continue;
+    const int n = u.kt1 - u.kt0;
+    const int i = u.m * kPrefillUnit + w * kPrefillBM + r;
+    const bool valid = i < u.len_q;
+    OutT* orow = reinterpret_cast<OutT*>(p.out) + u.bcoord * p.o_sb +
+                 (int64_t)(u.row_q + i) * p.o_ss + (int64_t)u.h * p.o_sh;
+    float* lrow = p.lse ? p.lse + u.b * p.lse_sb + u.h * p.lse_sh + (u.row_q + i) : nullptr;
     if (n <= 0) {
       if (valid) {
-        uint4 z = make_uint4(0, 0, 0, 0);
+        const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
         if (lrow) *lrow = -INFINITY;
@@ -302,44 +352,46 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
       continue;
     }
     int lo_i, hi_i;
-    row_key_range(p, i, ti.len_q, ti.len_k, lo_i, hi_i);
+    row_key_range(p, i, u.len_q, u.len_k, lo_i, hi_i);
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2pack(sl2, sl2);
     const bool has_sink = p.sink != nullptr;
-    const float sink2 = has_sink ? p.sink[ti.h] * kLog2e : -INFINITY;
+    const float sink2 = has_sink ? p.sink[u.h] * kLog2e : -INFINITY;
     float m_run = sink2;
     float l_run = 0.f;  // sum of the fp32 P (for the LSE)
     float l_rnd = 0.f;  // sum of the rounded P the MMA consumes (for O)
+    bool seen = false;  // some key of this row is visible
 
-    for (int j = 0; j < n; ++j) {
-      const int b = (sj + j) & 1;
-      if (!warp_wait(&bars->s_full[b], ((sj + j) >> 1) & 1, abort, 20)) return;
+    for (int j = 0; j < n; ++j, ++sj) {
+      if (!warp_wait(&bars->s_full[w], sj & 1, abort, 20 + w)) return;
       tc_fence_after();
-      const uint32_t s_tmem = tmem + (b ? C::kTmemS1 : C::kTmemS0) + lane;
       uint32_t s[kPrefillBN];
-#pragma unroll
-      for (int c = 0; c < kPrefillBN; c += 32) tmem_load<32>(s_tmem + c, s + c);
-      const int k0 = (ti.kt0 + j) * kPrefillBN;
+      tmem_load128(s_tmem, s);
+      const int k0 = (u.kt0 + j) * kPrefillBN;
       if (!(k0 >= lo_i && k0 + kPrefillBN - 1 <= hi_i)) {
 #pragma unroll
         for (int c = 0; c < kPrefillBN; ++c) {
           const bool vis = (k0 + c >= lo_i) && (k0 + c <= hi_i);
-          if (!vis) s[c] = __float_as_uint(-INFINITY);
+          s[c] = vis ? s[c] : __float_as_uint(-INFINITY);
         }
       }
-      float tmax = -INFINITY;
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < kPrefillBN; ++c) tmax = fmaxf(tmax, __uint_as_float(s[c]));
+      for (int x = 0; x < 8; ++x) mx8[x] = __uint_as_float(s[x]);
+#pragma unroll
+      for (int c = 8; c < kPrefillBN; c += 8)
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], __uint_as_float(s[c + x]));
+      const float tmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float mx = tmax * sl2;
-      if (j > 0) {
-        if (!warp_wait(&bars->o_full, pv & 1, abort, 21)) return;
-        ++pv;
-        tc_fence_after();
-      }
-      // Raise the running max only when it grows by more than 2^8; O is then
-      // rescaled in TMEM. tcgen05.ld/st are warp-collective, so the warp
-      // rescales together, each thread with its own factor (1 if unchanged).
-      // On the first tile the max is set exactly (so the row's largest P is
-      // exactly 1 when it is not the sink).
+      seen |= tmax != -INFINITY;
+      // The first tile sets the max exactly (the row's largest P is then 1
+      // unless the sink is larger); later tiles raise it only when it grows by
+      // more than 2^8, and then O is rescaled in TMEM. The previous P V of
+      // this tile has completed: it was issued before this S.
+      // tcgen05.ld/st are warp-collective, so the warp rescales together, each
+      // thread with its own factor (1 if unchanged).
       float alpha = 1.f;
       const bool grow = (j == 0) ? (mx > m_run) : (mx > m_run + kRescaleThreshold);
       if (grow) {
@@ -349,60 +401,108 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
         l_rnd *= alpha;
       }
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
-          tmem_load<32>(tmem + C::kTmemO + lane + c, o);
+          tmem_load<32>(o_tmem + c, o);
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-          tmem_store<32>(tmem + C::kTmemO + lane + c, o);
+          for (int x = 0; x < 32; x += 2) {
+            const uint64_t v =
+                mul2(f2pack(__uint_as_float(o[x]), __uint_as_float(o[x + 1])), a2);
+            float a, b;
+            f2unpack(v, a, b);
+            o[x] = __float_as_uint(a);
+            o[x + 1] = __float_as_uint(b);
+          }
+          tmem_store<32>(o_tmem + c, o);
         }
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float lsum = 0.f, lsum_rnd = 0.f;
-      uint32_t pk[kPrefillBN / 2];
+      const uint64_t negm = f2pack(-m_use, -m_use);
+      // P = 2^(s * scale * log2e - m), converted to the input type. O is
+      // normalised by the sum of the rounded P the MMA consumes (the weights
+      // then stay a convex combination and the rounding error scales with the
+      // spread of V, not with |O|); the LSE uses the fp32 sum.
+      // P is written to TMEM 32 columns (16 packed words) at a time, so only
+      // one chunk of packed values is live next to S.
+      uint64_t acc_e[4], acc_r[4];
 #pragma unroll
-      for (int c = 0; c < kPrefillBN / 2; ++c) {
-        const float p0 = ex2(fmaf(__uint_as_float(s[2 * c]), sl2, -m_use));
-        const float p1 = ex2(fmaf(__uint_as_float(s[2 * c + 1]), sl2, -m_use));
-        pk[c] = pack2<kFp16>(p0, p1);
-        // O is normalised by the sum of the rounded P that the MMA consumes:
-        // the weights then stay a convex combination and the rounding error
-        // scales with the spread of V, not with |O|. The LSE uses the fp32 sum.
-        lsum += p0 + p1;
-        lsum_rnd += sum2<kFp16>(pk[c]);
+      for (int x = 0; x < 4; ++x) acc_e[x] = acc_r[x] = 0ull;
+#pragma unroll
+      for (int ch = 0; ch < kPrefillBN / 32; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int e = ch * 32 + 2 * c;
+          const uint64_t arg =
+              fma2(f2pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2x2, negm);
+          float a0, a1;
+          f2unpack(arg, a0, a1);
+          float p0, p1;
+          if (c >= 16 - kEmuPairs) {
+            f2unpack(exp2_poly_x2(a0, a1), p0, p1);
+          } else {
+            p0 = ex2(a0);
+            p1 = ex2(a1);
+          }
+          acc_e[c & 3] = add2(acc_e[c & 3], f2pack(p0, p1));
+          if constexpr (kFp16) {
+            pk[c] = pack_f16x2(p0, p1);
+            acc_r[c & 3] = add2(acc_r[c & 3], widen2<true>(pk[c]));
+          } else {
+            // bf16 by truncation (keep the top 16 bits) on the integer pipe.
+            // Normalising O by the sum of these same values cancels their
+            // common bias; what remains is of the size of a rounding error.
+            const uint32_t r0 = __float_as_uint(p0), r1 = __float_as_uint(p1);
+            pk[c] = __byte_perm(r0, r1, 0x7632);
+            acc_r[c & 3] = add2(acc_r[c & 3], f2pack(__uint_as_float(r0 & 0xffff0000u),
+                                                     __uint_as_float(r1 & 0xffff0000u)));
+          }
+        }
+        tmem_store<16>(s_tmem + ch * 16, pk);
       }
-      l_run += lsum;
-      l_rnd += lsum_rnd;
-      const uint32_t p_tmem = tmem + (b ? C::kTmemS1 : C::kTmemS0) + lane;
-      tmem_store<32>(p_tmem, pk);
-      tmem_store<32>(p_tmem + 32, pk + 32);
+      {
+        const uint64_t e = add2(add2(acc_e[0], acc_e[1]), add2(acc_e[2], acc_e[3]));
+        const uint64_t q = add2(add2(acc_r[0], acc_r[1]), add2(acc_r[2], acc_r[3]));
+        float e0, e1, q0, q1;
+        f2unpack(e, e0, e1);
+        f2unpack(q, q0, q1);
+        l_run += e0 + e1;
+        l_rnd += q0 + q1;
+      }
       tmem_store_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[b]);
+      mbar_arrive(&bars->p_full[w]);
     }
-    sj += n;
     // Epilogue: wait for the last P V, read O, release O, normalise, store.
-    if (!warp_wait(&bars->o_full, pv & 1, abort, 22)) return;
-    ++pv;
+    if (!warp_wait(&bars->o_full[w], units & 1, abort, 22 + w)) return;
+    ++units;
     tc_fence_after();
     uint32_t o[D];
+    if constexpr (D == 128) {
+      tmem_load128(o_tmem, o);
+    } else {
 #pragma unroll
-    for (int c = 0; c < D; c += 32) tmem_load<32>(tmem + C::kTmemO + lane + c, o + c);
+      for (int c = 0; c < D; c += 32) tmem_load<32>(o_tmem + c, o + c);
+    }
     tc_fence_before();
-    mbar_arrive(&bars->o_empty);
+    mbar_arrive(&bars->o_empty[w]);
+    // A row that saw no key: O = 0, LSE = -inf (polynomial exponentials of
+    // masked scores are tiny but not 0, so the sums alone cannot tell).
+    if (!seen) l_run = l_rnd = 0.f;
     const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
     const float denom = l_rnd + (has_sink ? ex2(sink2 - m_use) : 0.f);
-    const float inv = denom > 0.f ? 1.f / denom : 0.f;
+    const float inv = (denom > 0.f && seen) ? 1.f / denom : 0.f;
     if (valid) {
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
-        uint4 w;
-        w.x = pack2<kFp16>(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-        w.y = pack2<kFp16>(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-        w.z = pack2<kFp16>(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-        w.w = pack2<kFp16>(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-        reinterpret_cast<uint4*>(orow)[c] = w;
+        uint4 v;
+        v.x = pack2<kFp16>(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
+        v.y = pack2<kFp16>(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
+        v.z = pack2<kFp16>(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
+        v.w = pack2<kFp16>(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
+        reinterpret_cast<uint4*>(orow)[c] = v;
       }
       if (lrow) *lrow = l_run > 0.f ? (m_use + log2f(l_run)) * kLn2 : -INFINITY;
     }
@@ -410,7 +510,7 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
 }
 
 template <int D, bool kFp16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
@@ -424,22 +524,25 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], 128);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&bars->s_full[w], 1);
+      mbar_init(&bars->p_full[w], 128);
+      mbar_init(&bars->o_full[w], 1);
+      mbar_init(&bars->o_empty[w], 128);
     }
-    mbar_init(&bars->o_full, 1);
-    mbar_init(&bars->o_empty, 128);
     mbar_init(&bars->mma_drain, 1);
     bars->abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&bars->tmem_base, C::kTmemCols);
     tmem_relinquish();
   }
@@ -448,17 +551,21 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp < 4) {
-    prefill_softmax<D, kFp16>(p, bars, tmem);
-  } else if (warp == 4) {
-    if (elect_lane0()) prefill_producer<D>(p, &map_q, &map_k, &map_v, smem, bars);
+  if (warp < 8) {
+    regs_inc<kPrefillSoftmaxRegs>();
+    prefill_softmax<D, kFp16>(p, bars, tmem, warp >> 2);
   } else {
-    if (elect_lane0()) prefill_mma<D, kFp16>(p, smem, bars, tmem);
+    regs_dec<kPrefillOtherRegs>();
+    if (warp == 8) {
+      if (elect_lane0()) prefill_producer<D>(p, &map_q, &map_k, &map_v, smem, bars);
+    } else if (warp == 9) {
+      prefill_mma<D, kFp16>(p, smem, bars, tmem);  // whole warp, one lane issues
+    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

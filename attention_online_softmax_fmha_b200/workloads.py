@@ -285,6 +285,10 @@ CONFIGS = {
                             window=(1024, 0), sink=True, dtype="e4m3"),
     "paged_decode": dict(kind="paged", lengths=(64, 1024, 32768), seqlen_q=1, num_heads_q=32,
                          num_heads_kv=8, head_dim=128, page_size=64),
+    # the same decode with 16 sequences (about 1.1 GB of cache), for profiler
+    # captures that must stay small
+    "paged_decode_small": dict(kind="paged", lengths=(16, 1024, 32768), seqlen_q=1,
+                               num_heads_q=32, num_heads_kv=8, head_dim=128, page_size=64),
     "mla_dense": dict(kind="mla", lengths=(64, 4096, 65536), seqlen_q=2, num_heads_q=128,
                       page_size=64),
     "mla_sparse": dict(kind="mla", lengths=(64, 4096, 65536), seqlen_q=2, num_heads_q=128,

@@ -103,6 +103,11 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def wait_first(self, timeout: float):
+        t0 = time.perf_counter()
+        while self.proc is not None and not self.lines and time.perf_counter() - t0 < timeout:
+            time.sleep(0.02)
+
     def __exit__(self, *exc):
         if self.proc is not None:
             self.proc.terminate()
@@ -205,10 +210,68 @@ def prefill_workload(name: str, seed: int, device):
                 f"{pairs} visible pairs per head")
 
 
+def paged_workload(name: str, seed: int, device):
+    inp = W.build_config(name, seed=seed, device=device)
+    D, Hq, Hkv, B_ = inp.head_dim, inp.num_heads_q, inp.num_heads_kv, inp.batch
+    sq = inp.q.shape[1]
+    import ctypes
+    L = B.lib()
+    sa = B.sched_args(inp.cache_seqlens, batch=B_, seqlen_q=sq, num_heads_q=Hq,
+                      num_heads_kv=Hkv, head_dim_qk=D, head_dim_v=D, page_size=inp.page_size)
+    meta = torch.empty(B.sched_metadata_size(sa) // 4, dtype=torch.int32, device=device)
+    sa.meta = meta.data_ptr()
+    sa.meta_bytes = meta.numel() * 4
+    pa, out, lse, ws = B.paged_args(inp.q, inp.k_cache, inp.v_cache, inp.block_table,
+                                    inp.cache_seqlens, scale=inp.scale, causal=inp.causal,
+                                    window=inp.window, sink=inp.sink, meta=meta)
+    # algorithmic bytes: every visible K and V row once per KV head, Q, O, LSE,
+    # the used block-table entries and cache_seqlens
+    kv_rows = sum(inp.seqlens)
+    pages = sum(-(-x // inp.page_size) for x in inp.seqlens)
+    nbytes = (kv_rows * Hkv * 2 * D * 2 + inp.q.numel() * 2 + out.numel() * 2 + lse.numel() * 4
+              + pages * 4 + B_ * 4)
+
+    def step(stream):
+        st = L.attn_sched_metadata(ctypes.byref(sa), stream.cuda_stream)
+        if st != B.OK:
+            raise B.AttnError("attn_sched_metadata", st)
+        st = L.attn_fwd_paged_kvcache(ctypes.byref(pa), stream.cuda_stream)
+        if st != B.OK:
+            raise B.AttnError("attn_fwd_paged_kvcache", st)
+
+    # e2e: the step's inputs are the new query rows, the block table and the
+    # cache lengths (the KV cache is resident state); out and LSE come back.
+    small = [inp.q, inp.block_table, inp.cache_seqlens]
+    host_small = [t.cpu().pin_memory() for t in small]
+    host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                torch.empty(lse.shape, dtype=lse.dtype).pin_memory()]
+
+    def e2e_step(stream):
+        for h, d in zip(host_small, small):
+            d.copy_(h, non_blocking=True)
+        step(stream)
+        host_out[0].copy_(out, non_blocking=True)
+        host_out[1].copy_(lse, non_blocking=True)
+
+    cfg = {"workload": name, "batch": B_, "seqlen_q": sq, "num_heads_q": Hq,
+           "num_heads_kv": Hkv, "head_dim": D, "page_size": inp.page_size,
+           "cache_seqlens": "uniform[1024,32768]", "block_table": "seeded permutation",
+           "kv_tokens": kv_rows, "dtype": inp.dtype}
+    return dict(step=step, e2e_step=e2e_step, work=nbytes / 1e9, unit="GB/s", bound="hbm",
+                kernel="decode_kernel<128>", launches_per_step=3,
+                h2d=sum(t.numel() * t.element_size() for t in host_small),
+                d2h=sum(t.numel() * t.element_size() for t in host_out), cfg=cfg,
+                dtype=inp.dtype, inp=inp, keep=(meta, ws, out, lse),
+                per_unit=f"(D_k + D_v) * 2 B per cached token per KV head + Q/O/LSE/table; "
+                f"{nbytes} B per step")
+
+
 WORKLOADS = {
     "tiny_dense_mha": prefill_workload,
     "varlen_causal_gqa": prefill_workload,
     "window_sink": prefill_workload,
+    "paged_decode": paged_workload,
+    "paged_decode_small": paged_workload,
 }
 
 
@@ -268,6 +331,16 @@ def cpu_baseline(name: str, seed: int, budget_s: float = 15.0):
 # timing
 # ---------------------------------------------------------------------------
 
+def load_for(fn, stream, seconds: float):
+    """Untimed repetitions of a step for about `seconds`."""
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        while time.perf_counter() - t0 < seconds:
+            for _ in range(8):
+                fn(stream)
+            stream.synchronize()
+
+
 def time_steps(fn, steps: int, warmup: int, stream, flush):
     for _ in range(warmup):
         fn(stream)
@@ -290,7 +363,7 @@ def run_ours(args, rank, world, device):
     peaks, peak_kind = load_peaks()
     traffic = load_traffic()
     shash = source_hash()
-    names = list(WORKLOADS) if args.all else [args.workload]
+    names = (args.only or list(WORKLOADS)) if args.all else [args.workload]
     if args.workload not in names:
         names.insert(0, args.workload)
     results = {}
@@ -300,7 +373,15 @@ def run_ours(args, rank, world, device):
             torch.distributed.barrier()
         torch.cuda.synchronize()
         with ClockSampler(torch.cuda.current_device()) as clk:
+            # The timed region is milliseconds long, shorter than the sampling
+            # period: keep the GPU busy with the same step for a short window
+            # on both sides so the samples describe the clocks it ran at.
+            if args.clock_window > 0:
+                clk.wait_first(3.0)
+                load_for(wl["step"], stream, args.clock_window)
             times = time_steps(wl["step"], args.steps, args.warmup, stream, flush)
+            if args.clock_window > 0:
+                load_for(wl["step"], stream, args.clock_window / 2)
         torch.cuda.synchronize()
         if world > 1:
             torch.distributed.barrier()
@@ -351,9 +432,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
+    ap.add_argument("--only", nargs="*", default=None, help="with --all: a subset of workloads")
     ap.add_argument("--all", action="store_true", help="also run every other workload")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-window", type=float, default=0.5,
+                    help="seconds of untimed load around the timed region while clocks are "
+                         "sampled (0: none, e.g. under a profiler)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
     if args.warmup < 3:
