@@ -81,12 +81,15 @@ attn_status_t launch_status(cudaError_t e) {
 // ---------------------------------------------------------------------------
 // attn_fwd_varlen
 // ---------------------------------------------------------------------------
-template <int D, bool kFp16>
+template <int D, int kType>
 attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
-  using C = PrefillCfg<D>;
+  using C = PrefillCfg<D, kType>;
   const bool varlen = a.cu_seqlens_q != nullptr;
-  const CUtensorMapDataType dt =
-      kFp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapDataType dt = kType == 2   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : kType == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int es = C::kInBytes;
+  const uint32_t bx = C::kChunkElems;
   const uint64_t rows_q = varlen ? (uint64_t)a.total_q : (uint64_t)a.max_seqlen_q;
   const uint64_t rows_k = varlen ? (uint64_t)a.total_k : (uint64_t)a.max_seqlen_k;
   const uint64_t nb = varlen ? 1 : (uint64_t)a.batch;
@@ -94,12 +97,12 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   const uint64_t ksb = varlen ? rows_k * a.k_stride_s : a.k_stride_b;
   const uint64_t vsb = varlen ? rows_k * a.v_stride_s : a.v_stride_b;
   CUtensorMap mq, mk, mv;
-  if (!encode_4d(&mq, a.q, dt, 2, D, a.num_heads_q, rows_q, nb, a.q_stride_h, a.q_stride_s, qsb,
-                 64, 1, 128, 1) ||
-      !encode_4d(&mk, a.k, dt, 2, D, a.num_heads_kv, rows_k, nb, a.k_stride_h, a.k_stride_s, ksb,
-                 64, 1, 128, 1) ||
-      !encode_4d(&mv, a.v, dt, 2, D, a.num_heads_kv, rows_k, nb, a.v_stride_h, a.v_stride_s, vsb,
-                 64, 1, 128, 1))
+  if (!encode_4d(&mq, a.q, dt, es, D, a.num_heads_q, rows_q, nb, a.q_stride_h, a.q_stride_s, qsb,
+                 bx, 1, 128, 1) ||
+      !encode_4d(&mk, a.k, dt, es, D, a.num_heads_kv, rows_k, nb, a.k_stride_h, a.k_stride_s, ksb,
+                 bx, 1, 128, 1) ||
+      !encode_4d(&mv, a.v, dt, es, D, a.num_heads_kv, rows_k, nb, a.v_stride_h, a.v_stride_s, vsb,
+                 bx, 1, 128, 1))
     return ATTN_ERR_INVALID_ARG;
 
   PrefillParams p;
@@ -109,6 +112,9 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   p.cu_q = a.cu_seqlens_q;
   p.cu_k = a.cu_seqlens_k;
   p.sink = a.sink;
+  p.q_descale = a.q_descale;
+  p.k_descale = a.k_descale;
+  p.v_descale = a.v_descale;
   p.o_sb = a.o_stride_b;
   p.o_ss = a.o_stride_s;
   p.o_sh = a.o_stride_h;
@@ -129,7 +135,7 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   p.window_left = a.window_left;
   p.window_right = a.window_right;
 
-  auto kernel = prefill_kernel<D, kFp16>;
+  auto kernel = prefill_kernel<D, kType>;
   static bool configured = false;
   if (!configured) {
     // The warpgroups trade registers with setmaxnreg out of the block's
@@ -176,6 +182,7 @@ attn_status_t check_varlen(const attn_varlen_args* a) {
   if (a->head_dim_qk != a->head_dim_v) return ATTN_ERR_UNSUPPORTED;
   if (a->head_dim_qk != 64 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
   if (a->dtype == ATTN_DTYPE_E5M2) return ATTN_ERR_UNSUPPORTED;
+  if (a->dtype == ATTN_DTYPE_E4M3 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
@@ -330,9 +337,11 @@ attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream) {
   const int D = args->head_dim_qk;
   switch (args->dtype) {
     case ATTN_DTYPE_BF16:
-      return D == 64 ? run_prefill<64, false>(*args, s) : run_prefill<128, false>(*args, s);
+      return D == 64 ? run_prefill<64, 0>(*args, s) : run_prefill<128, 0>(*args, s);
     case ATTN_DTYPE_FP16:
-      return D == 64 ? run_prefill<64, true>(*args, s) : run_prefill<128, true>(*args, s);
+      return D == 64 ? run_prefill<64, 1>(*args, s) : run_prefill<128, 1>(*args, s);
+    case ATTN_DTYPE_E4M3:
+      return run_prefill<128, 2>(*args, s);
     default:
       return ATTN_ERR_UNSUPPORTED;
   }

@@ -22,7 +22,8 @@
 //                    works on one tile while the other tile's softmax runs.
 //                    S_w = Q_w K^T lands in TMEM; P_w (bf16) overwrites it and
 //                    is the TMEM A operand of O_w += P_w V.
-//   warps 10, 11     idle (they complete the register warpgroup).
+//   warps 10, 11     FP8 only: convert each e4m3 V tile to fp16 for P V;
+//                    otherwise idle (they complete the register warpgroup).
 // Registers move from warpgroup 2 to the softmax warpgroups with setmaxnreg;
 // the host checks the kernel's register count before launching.
 // Every mbarrier wait is bounded; a timeout raises ATTN_DEVERR_TIMEOUT and the
@@ -73,19 +74,30 @@ static_assert(2 * 128 * kPrefillSoftmaxRegs + 128 * kPrefillOtherRegs <=
                   kPrefillThreads * kPrefillLaunchRegs,
               "register split exceeds the launch allocation");
 
-template <int D>
+// Input types: 0 = bf16, 1 = fp16, 2 = FP8 E4M3.
+// With FP8 inputs S = Q K^T runs as an e4m3 MMA; P is kept in fp16 (e4m3 has
+// too few mantissa bits for P: rows with few visible keys would miss the
+// accuracy bound), so V is converted to fp16 in shared memory (exact: every
+// e4m3 value is an fp16 value) for the fp16 P V MMA.
+template <int D, int kType>
 struct PrefillCfg {
-  static constexpr int kChunks = D / 64;                 // 128-byte column chunks
+  static constexpr bool kFp8 = kType == 2;
+  static constexpr int kInBytes = kFp8 ? 1 : 2;
+  static constexpr int kChunkElems = 128 / kInBytes;     // elements per 128-byte row chunk
+  static constexpr int kChunks = D * kInBytes / 128;     // 128-byte column chunks
   // K and V tiles have separate rings: K is released as soon as both S MMAs
-  // have read it, V after both P V MMAs.
-  static constexpr int kKStages = (D == 64) ? 4 : 3;
+  // have read it, V after both P V MMAs (FP8: after the conversion).
+  static constexpr int kKStages = kFp8 ? 4 : ((D == 64) ? 4 : 3);
   static constexpr int kVStages = (D == 64) ? 4 : 2;
+  static constexpr int kVHStages = kFp8 ? 2 : 0;         // fp16 copies of V (FP8)
   static constexpr int kChunkBytes = 128 * 128;          // 128 rows x 128 bytes
   static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kVHBytes = (D / 64) * kChunkBytes;
   static constexpr int kQOff = 0;                        // Q0, Q1
   static constexpr int kKOff = 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kVStages * kTileBytes;
+  static constexpr int kVHOff = kVOff + kVStages * kTileBytes;
+  static constexpr int kBarOff = kVHOff + kVHStages * kVHBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers, + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128;
@@ -95,6 +107,7 @@ struct PrefillCfg {
 struct PrefillBarriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
+  uint64_t vh_full[4], vh_empty[4];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
@@ -161,10 +174,10 @@ DEVI void row_key_range(const PrefillParams& p, int i, int len_q, int len_k, int
 // ---------------------------------------------------------------------------
 // Producer warp (one thread)
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int kType>
 DEVI void prefill_producer(const PrefillParams& p, const CUtensorMap* mq, const CUtensorMap* mk,
                            const CUtensorMap* mv, uint8_t* smem, PrefillBarriers* bars) {
-  using C = PrefillCfg<D>;
+  using C = PrefillCfg<D, kType>;
   volatile int* abort = &bars->abort;
   tma_prefetch_desc(mq);
   tma_prefetch_desc(mk);
@@ -183,7 +196,8 @@ DEVI void prefill_producer(const PrefillParams& p, const CUtensorMap* mq, const 
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c)
         tma_load_4d(smem + C::kQOff + w * C::kTileBytes + c * C::kChunkBytes, mq, &bars->q_full,
-                    c * 64, u.h, u.row_q + u.m * kPrefillUnit + w * kPrefillBM, u.bcoord);
+                    c * C::kChunkElems, u.h, u.row_q + u.m * kPrefillUnit + w * kPrefillBM,
+                    u.bcoord);
     ++nq;
     for (int j = 0; j < n; ++j, ++it) {
       const int row = u.row_k + (u.kt0 + j) * kPrefillBN;
@@ -195,7 +209,7 @@ DEVI void prefill_producer(const PrefillParams& p, const CUtensorMap* mq, const 
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c)
         tma_load_4d(smem + C::kKOff + sk * C::kTileBytes + c * C::kChunkBytes, mk,
-                    &bars->k_full[sk], c * 64, hk, row, u.bcoord);
+                    &bars->k_full[sk], c * C::kChunkElems, hk, row, u.bcoord);
       if (it >= C::kVStages &&
           !mbar_wait(&bars->v_empty[sv], ((it / C::kVStages) - 1) & 1, abort, 4))
         goto drain;
@@ -203,7 +217,7 @@ DEVI void prefill_producer(const PrefillParams& p, const CUtensorMap* mq, const 
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c)
         tma_load_4d(smem + C::kVOff + sv * C::kTileBytes + c * C::kChunkBytes, mv,
-                    &bars->v_full[sv], c * 64, hk, row, u.bcoord);
+                    &bars->v_full[sv], c * C::kChunkElems, hk, row, u.bcoord);
     }
   }
 drain:
@@ -226,13 +240,17 @@ drain:
 // which is the low 14-bit field (in 16-byte units) of the descriptor, so an
 // integer add of the offset in 16-byte units advances it (shared memory is
 // below 256 KB, the field never carries).
-template <int D>
+// One MMA consumes 32 bytes of K (16 bf16/fp16 or 32 FP8 elements).
+template <int D, int kType>
 DEVI void prefill_issue_s(uint32_t d_tmem, uint64_t dq, uint64_t dk, uint32_t idesc) {
-  using C = PrefillCfg<D>;
+  using C = PrefillCfg<D, kType>;
 #pragma unroll
-  for (int k = 0; k < D / 16; ++k) {
+  for (int k = 0; k < D * C::kInBytes / 32; ++k) {
     const uint32_t off16 = (k >> 2) * (C::kChunkBytes >> 4) + (k & 3) * 2;
-    mma_f16_ss_w(d_tmem, dq + off16, dk + off16, idesc, k > 0 ? 1u : 0u);
+    if constexpr (C::kFp8)
+      mma_f8_ss_w(d_tmem, dq + off16, dk + off16, idesc, k > 0 ? 1u : 0u);
+    else
+      mma_f16_ss_w(d_tmem, dq + off16, dk + off16, idesc, k > 0 ? 1u : 0u);
   }
 }
 DEVI void prefill_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t dv, uint32_t idesc,
@@ -243,21 +261,29 @@ DEVI void prefill_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t dv, uint32
                (!first || kk > 0) ? 1u : 0u);
 }
 
-template <int D, bool kFp16>
+template <int D, int kType>
 DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* bars,
                       uint32_t tmem) {
-  using C = PrefillCfg<D>;
+  using C = PrefillCfg<D, kType>;
   volatile int* abort = &bars->abort;
-  constexpr int fmt = kFp16 ? 0 : 1;
-  constexpr uint32_t idesc_qk = make_idesc(128, kPrefillBN, fmt, 0, 0);
+  // kind::f16 formats: 0 = fp16, 1 = bf16; kind::f8f6f4: 0 = e4m3. P V runs
+  // in fp16 for FP8 inputs.
+  constexpr int fmt_qk = kType == 0 ? 1 : 0;
+  constexpr int fmt_pv = kType == 0 ? 1 : 0;
+  constexpr uint32_t idesc_qk = make_idesc(128, kPrefillBN, fmt_qk, 0, 0);
   // V is MN-major (d contiguous): one MMA covers all D columns; the 64-column
   // chunks of the tile are kChunkBytes apart (leading byte offset), groups
   // of 8 keys are 1024 bytes apart (stride byte offset).
-  constexpr uint32_t idesc_pv = make_idesc(128, D, fmt, 0, 1);
+  constexpr uint32_t idesc_pv = make_idesc(128, D, fmt_pv, 0, 1);
+  constexpr int kPVStages = C::kFp8 ? C::kVHStages : C::kVStages;
+  constexpr int kPVBytes = C::kFp8 ? C::kVHBytes : C::kTileBytes;
+  uint64_t* pv_full = C::kFp8 ? bars->vh_full : bars->v_full;
+  uint64_t* pv_empty = C::kFp8 ? bars->vh_empty : bars->v_empty;
   const uint64_t dq0 = sdesc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
   const uint64_t dq1 = dq0 + (C::kTileBytes >> 4);
   const uint64_t dk_base = sdesc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
-  const uint64_t dv_base = sdesc_sw128(smem_u32(smem + C::kVOff), C::kChunkBytes, 1024);
+  const uint64_t dv_base =
+      sdesc_sw128(smem_u32(smem + (C::kFp8 ? C::kVHOff : C::kVOff)), C::kChunkBytes, 1024);
   const uint32_t tS0 = tmem + C::kTmemS0, tS1 = tmem + C::kTmemS1;
   const uint32_t tO0 = tmem + C::kTmemO0, tO1 = tmem + C::kTmemO1;
   int it = 0, nq = 0, units = 0;
@@ -274,23 +300,23 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
     for (int j = 0; j <= n; ++j) {
       const int g = it + j;
       const int s = g % C::kKStages;
-      const int sp = (g - 1) % C::kVStages;
+      const int sp = (g - 1) % kPVStages;
       if (j < n) {
         if (!warp_wait(&bars->k_full[s], (g / C::kKStages) & 1, abort, 14)) goto drain;
       }
       if (j > 0) {
         if (!warp_wait(&bars->p_full[0], (g - 1) & 1, abort, 11)) goto drain;
-        if (!warp_wait(&bars->v_full[sp], ((g - 1) / C::kVStages) & 1, abort, 12)) goto drain;
+        if (!warp_wait(&pv_full[sp], ((g - 1) / kPVStages) & 1, abort, 12)) goto drain;
         if (j == 1 && units > 0 && !warp_wait(&bars->o_empty[0], (units - 1) & 1, abort, 13))
           goto drain;
         tc_fence_after();
-        prefill_issue_pv(tO0, tS0, dv_base + sp * (C::kTileBytes >> 4), idesc_pv, j == 1);
+        prefill_issue_pv(tO0, tS0, dv_base + sp * (kPVBytes >> 4), idesc_pv, j == 1);
         if (j == n) tc_commit_w(&bars->o_full[0]);
       } else {
         tc_fence_after();
       }
       if (j < n) {
-        prefill_issue_s<D>(tS0, dq0, dk_base + s * (C::kTileBytes >> 4), idesc_qk);
+        prefill_issue_s<D, kType>(tS0, dq0, dk_base + s * (C::kTileBytes >> 4), idesc_qk);
         tc_commit_w(&bars->s_full[0]);
       }
       if (j > 0) {
@@ -298,12 +324,12 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
         if (j == 1 && units > 0 && !warp_wait(&bars->o_empty[1], (units - 1) & 1, abort, 13))
           goto drain;
         tc_fence_after();
-        prefill_issue_pv(tO1, tS1, dv_base + sp * (C::kTileBytes >> 4), idesc_pv, j == 1);
+        prefill_issue_pv(tO1, tS1, dv_base + sp * (kPVBytes >> 4), idesc_pv, j == 1);
         if (j == n) tc_commit_w(&bars->o_full[1]);
-        tc_commit_w(&bars->v_empty[sp]);
+        tc_commit_w(&pv_empty[sp]);
       }
       if (j < n) {
-        prefill_issue_s<D>(tS1, dq1, dk_base + s * (C::kTileBytes >> 4), idesc_qk);
+        prefill_issue_s<D, kType>(tS1, dq1, dk_base + s * (C::kTileBytes >> 4), idesc_qk);
         tc_commit_w(&bars->s_full[1]);
         tc_commit_w(&bars->k_empty[s]);
         if (j == n - 1) tc_commit_w(&bars->q_empty);
@@ -321,12 +347,62 @@ drain : {
 }
 
 // ---------------------------------------------------------------------------
+// FP8 only: V conversion warps (warps 10, 11). Each e4m3 V tile (128-byte
+// swizzled rows of 128 elements) is rewritten as an fp16 tile in the layout
+// the P V MMA reads (two 64-column chunks, 128-byte swizzled); the e4m3 stage
+// is then released to the producer and the fp16 stage handed to the MMA.
+// ---------------------------------------------------------------------------
+template <int D, int kType>
+DEVI void prefill_convert(const PrefillParams& p, uint8_t* smem, PrefillBarriers* bars) {
+  using C = PrefillCfg<D, kType>;
+  static_assert(D == 128, "FP8 prefill is built for D = 128");
+  volatile int* abort = &bars->abort;
+  const int t = threadIdx.x - 320;  // 0..63
+  int it = 0;
+  for (int wu = blockIdx.x; wu < p.total_units; wu += gridDim.x) {
+    PrefillUnit u;
+    if (!prefill_unit(p, wu, u)) continue;
+    const int n = u.kt1 - u.kt0;
+    for (int j = 0; j < n; ++j, ++it) {
+      const int sv = it % C::kVStages, sh = it % C::kVHStages;
+      if (!mbar_wait(&bars->v_full[sv], (it / C::kVStages) & 1, abort, 50)) return;
+      if (it >= C::kVHStages &&
+          !mbar_wait(&bars->vh_empty[sh], ((it / C::kVHStages) - 1) & 1, abort, 51))
+        return;
+      const uint8_t* src = smem + C::kVOff + sv * C::kTileBytes;
+      uint8_t* dst = smem + C::kVHOff + sh * C::kVHBytes;
+#pragma unroll 4
+      for (int x = t; x < 128 * 8; x += 64) {
+        const int row = x >> 3, unit = x & 7;  // 16 e4m3 values = d 16*unit .. +15
+        const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + ((unit ^ (row & 7)) << 4));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * q]) : "h"((unsigned short)(w[q] & 0xffff)));
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * q + 1]) : "h"((unsigned short)(w[q] >> 16)));
+        }
+        const int chunk = unit >> 2, u16 = (unit & 3) * 2;
+        uint8_t* drow = dst + chunk * C::kChunkBytes + row * 128;
+        *reinterpret_cast<uint4*>(drow + ((u16 ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(drow + (((u16 + 1) ^ (row & 7)) << 4)) =
+            make_uint4(h[4], h[5], h[6], h[7]);
+      }
+      fence_proxy_async_smem();  // the fp16 tile is read by the tensor core
+      mbar_arrive(&bars->vh_full[sh]);
+      mbar_arrive(&bars->v_empty[sv]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Softmax warpgroups: warpgroup w owns tile Q_w, one query row per thread
 // ---------------------------------------------------------------------------
-template <int D, bool kFp16>
+template <int D, int kType>
 DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_t tmem, int w) {
-  using C = PrefillCfg<D>;
-  using OutT = typename std::conditional<kFp16, __half, __nv_bfloat16>::type;
+  using C = PrefillCfg<D, kType>;
+  constexpr bool kFp16 = kType != 0;  // P in fp16 (fp16 and FP8 inputs)
+  using OutT = typename std::conditional<kType == 1, __half, __nv_bfloat16>::type;
   volatile int* abort = &bars->abort;
   const int r = threadIdx.x & 127;
   const uint32_t lane = (uint32_t)(r & ~31) << 16;
@@ -353,7 +429,15 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
     }
     int lo_i, hi_i;
     row_key_range(p, i, u.len_q, u.len_k, lo_i, hi_i);
-    const float sl2 = p.scale_log2;
+    float sl2 = p.scale_log2;
+    float v_scale = 1.f;
+    if constexpr (C::kFp8) {
+      // S and O use the dequantised inputs: q * q_descale, k * k_descale,
+      // v * v_descale, per (sequence, KV head) (MATE FMHA dtype notes).
+      const int dk = u.b * p.num_heads_kv + u.h / p.group;
+      sl2 *= p.q_descale[dk] * p.k_descale[dk];
+      v_scale = p.v_descale[dk];
+    }
     const uint64_t sl2x2 = f2pack(sl2, sl2);
     const bool has_sink = p.sink != nullptr;
     const float sink2 = has_sink ? p.sink[u.h] * kLog2e : -INFINITY;
@@ -493,15 +577,16 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
     if (!seen) l_run = l_rnd = 0.f;
     const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
     const float denom = l_rnd + (has_sink ? ex2(sink2 - m_use) : 0.f);
-    const float inv = (denom > 0.f && seen) ? 1.f / denom : 0.f;
+    const float inv = (denom > 0.f && seen) ? v_scale / denom : 0.f;
     if (valid) {
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
         uint4 v;
-        v.x = pack2<kFp16>(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-        v.y = pack2<kFp16>(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-        v.z = pack2<kFp16>(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-        v.w = pack2<kFp16>(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
+        constexpr bool kOutF16 = kType == 1;
+        v.x = pack2<kOutF16>(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
+        v.y = pack2<kOutF16>(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
+        v.z = pack2<kOutF16>(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
+        v.w = pack2<kOutF16>(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
         reinterpret_cast<uint4*>(orow)[c] = v;
       }
       if (lrow) *lrow = l_run > 0.f ? (m_use + log2f(l_run)) * kLn2 : -INFINITY;
@@ -509,12 +594,12 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
   }
 }
 
-template <int D, bool kFp16>
+template <int D, int kType>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
-  using C = PrefillCfg<D>;
+  using C = PrefillCfg<D, kType>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -530,7 +615,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     for (int s = 0; s < C::kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->v_empty[s], C::kFp8 ? 64 : 1);  // FP8: released by the 64 converters
+    }
+    for (int s = 0; s < C::kVHStages; ++s) {
+      mbar_init(&bars->vh_full[s], 64);
+      mbar_init(&bars->vh_empty[s], 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
@@ -553,13 +642,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   if (warp < 8) {
     regs_inc<kPrefillSoftmaxRegs>();
-    prefill_softmax<D, kFp16>(p, bars, tmem, warp >> 2);
+    prefill_softmax<D, kType>(p, bars, tmem, warp >> 2);
   } else {
     regs_dec<kPrefillOtherRegs>();
     if (warp == 8) {
-      if (elect_lane0()) prefill_producer<D>(p, &map_q, &map_k, &map_v, smem, bars);
+      if (elect_lane0()) prefill_producer<D, kType>(p, &map_q, &map_k, &map_v, smem, bars);
     } else if (warp == 9) {
-      prefill_mma<D, kFp16>(p, smem, bars, tmem);  // whole warp, one lane issues
+      prefill_mma<D, kType>(p, smem, bars, tmem);  // whole warp, one lane issues
+    } else if constexpr (C::kFp8) {
+      prefill_convert<D, kType>(p, smem, bars);
     }
   }
 

@@ -182,6 +182,7 @@ def prefill_workload(name: str, seed: int, device):
 
     # e2e: pinned host copies of the step's inputs; H2D, the call, D2H of out/lse
     host_in = [t.cpu().pin_memory() for t in (inp.q, inp.k, inp.v)]
+    # (FP8 tensors are copied as raw bytes)
     host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),
                 torch.empty(lse.shape, dtype=lse.dtype).pin_memory()]
     dev_in = [inp.q, inp.k, inp.v]
@@ -205,7 +206,7 @@ def prefill_workload(name: str, seed: int, device):
            "sink": inp.sink is not None, "dtype": inp.dtype, "total_q_tokens": sum(inp.seqlens_q),
            "visible_pairs_per_head": pairs}
     return dict(step=step, e2e_step=e2e_step, work=flops / 1e12, unit="TFLOP/s", bound=bound,
-                kernel=f"prefill_kernel<{D}>", launches_per_step=1, h2d=h2d, d2h=d2h, cfg=cfg,
+                kernel=f"prefill_kernel<{D},{ {'bf16': 0, 'fp16': 1, 'e4m3': 2}[inp.dtype] }>", launches_per_step=1, h2d=h2d, d2h=d2h, cfg=cfg,
                 dtype=inp.dtype, inp=inp, per_unit=f"2*(D_qk+D_v)*H_q FLOP per visible pair, "
                 f"{pairs} visible pairs per head")
 
@@ -270,6 +271,7 @@ WORKLOADS = {
     "tiny_dense_mha": prefill_workload,
     "varlen_causal_gqa": prefill_workload,
     "window_sink": prefill_workload,
+    "window_sink_fp8": prefill_workload,
     "paged_decode": paged_workload,
     "paged_decode_small": paged_workload,
 }

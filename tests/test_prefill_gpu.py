@@ -118,3 +118,44 @@ def test_many_tiles_per_cta():
     for b, i, h in rows:
         assert_close_out(o[b, i, h], ro[b, i, h], 1e-2)
         assert abs(l[b, h, i] - rl[b, h, i]) <= 1e-3
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 inputs with fp32 descales (B, H_kv), bf16 output: max-abs 5e-2.
+# ---------------------------------------------------------------------------
+
+def test_fp8_padded_window_sink():
+    inp = W.make_prefill(seqlens_q=[700] * 2, num_heads_q=4, num_heads_kv=2, head_dim=128,
+                         varlen=False, causal=True, window=(100, 0), sink=True, dtype="e4m3",
+                         seed=11, device="cuda")
+    run_and_check(inp, atol=5e-2)
+
+
+def test_fp8_varlen_causal_gqa_edge_lengths():
+    lens = [1, 2, 63, 64, 65, 129, 300, 513]
+    inp = W.make_prefill(seqlens_q=lens, num_heads_q=8, num_heads_kv=2, head_dim=128,
+                         varlen=True, causal=True, dtype="e4m3", seed=12, device="cuda")
+    run_and_check(inp, atol=5e-2)
+
+
+def test_fp8_full_size_window_sink_sampled():
+    """The FP8 window + sink workload at full size (B=4, S=8192, H=32, D=128,
+    window (1024, 0), sink, descales U[0.5, 2]); rows sampled for the oracle."""
+    inp = W.build_config("window_sink_fp8", seed=0, device="cuda")
+    out, lse = B.fwd_varlen(inp.q, inp.k, inp.v, scale=inp.scale, causal=True,
+                            window=inp.window, sink=inp.sink, q_descale=inp.q_descale,
+                            k_descale=inp.k_descale, v_descale=inp.v_descale)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    rows = [(b, i, h) for b in (0, 3) for i in (0, 1, 2, 700, 1024, 1025, 4095, 8191)
+            for h in (0, 17, 31)]
+    q, k, v = to_f64(inp.q), to_f64(inp.k), to_f64(inp.v)
+    ro, rl = oracle.attention_padded(q, k, v, inp.scale, True, inp.window,
+                                     inp.sink.cpu().numpy(), inp.q_descale.cpu().numpy(),
+                                     inp.k_descale.cpu().numpy(), inp.v_descale.cpu().numpy(),
+                                     rows=rows)
+    o = to_f64(out)
+    l = lse.cpu().numpy()
+    for b, i, h in rows:
+        assert_close_out(o[b, i, h], ro[b, i, h], 5e-2)
+        assert abs(l[b, h, i] - rl[b, h, i]) <= 1e-3
