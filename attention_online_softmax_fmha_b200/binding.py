@@ -311,3 +311,59 @@ def combine(out_partial, lse_partial, *, num_splits_per_seq=None, sink=None, out
                     out.stride(1), out.stride(2), _TORCH_DTYPE[out.dtype])
     _check("attn_combine", lib().attn_combine(ctypes.byref(a), _stream(stream)))
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# mla_fwd_paged / mla_sparse_fwd
+# ---------------------------------------------------------------------------
+
+def mla_args(q, kv_cache, block_table, cache_seqlens, *, head_dim_v=512, scale=None,
+             causal=False, indices=None, meta=None, num_ctas=0, workspace=None, out=None,
+             lse=None):
+    B, sq, Hq, Dqk = q.shape
+    if out is None:
+        out = torch.empty(B, sq, Hq, head_dim_v, device=q.device, dtype=torch.bfloat16)
+    if lse is None:
+        lse = torch.empty(B, Hq, sq, device=q.device, dtype=torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dqk)
+    topk = 0 if indices is None else indices.shape[-1]
+    a = MlaArgs(
+        _ptr(q), _ptr(kv_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(indices),
+        _ptr(out), _ptr(lse), B, sq, Hq, kv_cache.shape[2], Dqk, head_dim_v, kv_cache.shape[1],
+        kv_cache.shape[0], block_table.shape[1], topk, block_table.stride(0), q.stride(0),
+        q.stride(1), q.stride(2), kv_cache.stride(0), kv_cache.stride(1), out.stride(0),
+        out.stride(1), out.stride(2), 0 if indices is None else indices.stride(0),
+        0 if indices is None else indices.stride(1), float(scale), int(bool(causal)), _ptr(meta),
+        0 if meta is None else meta.numel() * 4, int(num_ctas), None, 0)
+    if meta is not None:
+        nbytes = int(lib().mla_workspace_size(ctypes.byref(a)))
+        if workspace is None:
+            workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        a.workspace = workspace.data_ptr()
+        a.workspace_bytes = workspace.numel()
+    return a, out, lse, workspace
+
+
+def mla_fwd_paged(q, kv_cache, block_table, cache_seqlens, *, stream=None, **kw):
+    """MLA-absorbed decode over a paged latent cache. Returns (out, lse)."""
+    a, out, lse, ws = mla_args(q, kv_cache, block_table, cache_seqlens, **kw)
+    _check("mla_fwd_paged", lib().mla_fwd_paged(ctypes.byref(a), _stream(stream)))
+    return out, lse
+
+
+def mla_sparse_fwd(q, kv_cache, block_table, cache_seqlens, indices, *, stream=None, **kw):
+    """MLA decode over top-k index sets. Returns (out, lse)."""
+    a, out, lse, ws = mla_args(q, kv_cache, block_table, cache_seqlens, indices=indices, **kw)
+    _check("mla_sparse_fwd", lib().mla_sparse_fwd(ctypes.byref(a), _stream(stream)))
+    return out, lse
+
+
+def mla_metadata(inp_cache_seqlens, *, batch, seqlen_q, num_heads_q, page_size, topk=0,
+                 num_ctas=0, stream=None):
+    """Scheduler metadata for mla_fwd_paged (topk = 0) or mla_sparse_fwd."""
+    return sched_metadata(inp_cache_seqlens, batch=batch, seqlen_q=seqlen_q,
+                          num_heads_q=num_heads_q, num_heads_kv=1, head_dim_qk=576,
+                          head_dim_v=512, page_size=page_size,
+                          mode=SCHED_MLA_SPARSE if topk else SCHED_MLA, topk=topk,
+                          num_ctas=num_ctas, stream=stream)

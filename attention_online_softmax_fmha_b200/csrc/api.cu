@@ -13,6 +13,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "decode_paged.cuh"
+#include "mla_sm100.cuh"
 #include "prefill_sm100.cuh"
 #include "sched.cuh"
 
@@ -195,7 +196,15 @@ bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1))
 struct DecodeShape {
   SchedShape sh;
   int group = 0, rows = 0, n_rsub = 0, S = 0, G = 0;
+  int tiles_per_token = 1, tokens_per_tile = 1, row_tiles = 0;  // MLA
 };
+
+// MLA row tiles of 128 (token, head) rows: heads_q a power of two up to 128
+// (tiles hold 128 / heads_q tokens) or a multiple of 128.
+bool mla_heads_ok(int heads_q) {
+  return heads_q > 0 && ((heads_q <= kMlaRows && (heads_q & (heads_q - 1)) == 0) ||
+                         heads_q % kMlaRows == 0);
+}
 
 attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int heads_kv,
                            int topk, int num_ctas, DecodeShape& ds) {
@@ -210,7 +219,17 @@ attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int h
     ds.sh.segs_per_seq = heads_kv * ds.n_rsub;
     ds.sh.unit_keys = kDecTileKeys;
   } else {
-    return ATTN_ERR_UNSUPPORTED;
+    if (heads_kv != 1 || !mla_heads_ok(heads_q)) return ATTN_ERR_UNSUPPORTED;
+    if (mode == ATTN_SCHED_MLA_SPARSE && topk <= 0) return ATTN_ERR_INVALID_ARG;
+    if (heads_q >= kMlaRows) {
+      ds.tiles_per_token = heads_q / kMlaRows;
+      ds.row_tiles = seqlen_q * ds.tiles_per_token;
+    } else {
+      ds.tokens_per_tile = mode == ATTN_SCHED_MLA_SPARSE ? 1 : kMlaRows / heads_q;
+      ds.row_tiles = (seqlen_q + ds.tokens_per_tile - 1) / ds.tokens_per_tile;
+    }
+    ds.sh.segs_per_seq = ds.row_tiles * 2;  // x two V halves
+    ds.sh.unit_keys = kMlaBN;
   }
   const int64_t S = (int64_t)batch * ds.sh.segs_per_seq;
   if (S > (1 << 24)) return ATTN_ERR_UNSUPPORTED;
@@ -321,6 +340,124 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// MLA decode (dense and sparse)
+// ---------------------------------------------------------------------------
+attn_status_t check_mla(const mla_args* a, bool sparse) {
+  if (!a) return ATTN_ERR_INVALID_ARG;
+  if (!a->q || !a->kv_cache || !a->block_table || !a->cache_seqlens || !a->out)
+    return ATTN_ERR_INVALID_ARG;
+  if (sparse && (!a->indices || a->topk <= 0)) return ATTN_ERR_INVALID_ARG;
+  if (a->batch <= 0 || a->seqlen_q <= 0 || a->num_heads_q <= 0 || a->num_heads_kv <= 0 ||
+      a->head_dim_qk <= 0 || a->head_dim_v <= 0 || a->page_size <= 0 || a->num_blocks <= 0 ||
+      a->max_pages_per_seq <= 0 || a->num_ctas < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (a->block_table_stride < a->max_pages_per_seq) return ATTN_ERR_INVALID_ARG;
+  if (!(a->scale > 0.f) || !std::isfinite(a->scale)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->kv_cache) || !aligned16(a->out)) return ATTN_ERR_INVALID_ARG;
+  if (!stride_ok(a->q_stride_b, 2) || !stride_ok(a->q_stride_s, 2) ||
+      !stride_ok(a->q_stride_h, 2) || !stride_ok(a->kv_stride_blk, 2) ||
+      !stride_ok(a->kv_stride_tok, 2) || !stride_ok(a->o_stride_b, 2) ||
+      !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
+    return ATTN_ERR_INVALID_ARG;
+  if (sparse && (a->idx_stride_b <= 0 || a->idx_stride_s <= 0)) return ATTN_ERR_INVALID_ARG;
+  if (a->head_dim_qk != kMlaDqk || a->head_dim_v != kMlaDv) return ATTN_ERR_UNSUPPORTED;
+  if (a->num_heads_kv != 1 || !mla_heads_ok(a->num_heads_q)) return ATTN_ERR_UNSUPPORTED;
+  if (!pow2_in(a->page_size, 16, 256)) return ATTN_ERR_UNSUPPORTED;
+  if (sparse && a->causal) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+size_t mla_ws_bytes(const DecodeShape& ds) {
+  const size_t slots = (size_t)ds.S + ds.G;
+  return slots * kMlaRows * kMlaDvHalf * sizeof(float) + slots * kMlaRows * sizeof(float) + 256;
+}
+
+template <bool kSparse>
+attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t stream) {
+  const int box_h = a.num_heads_q >= kMlaRows ? kMlaRows : a.num_heads_q;
+  const int box_t = a.num_heads_q >= kMlaRows ? 1 : ds.tokens_per_tile;
+  CUtensorMap mq, mkv;
+  if (!encode_4d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk, a.num_heads_q,
+                 a.seqlen_q, a.batch, a.q_stride_h, a.q_stride_s, a.q_stride_b, 64, box_h, box_t,
+                 1) ||
+      !encode_4d(&mkv, a.kv_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk, a.page_size,
+                 a.num_blocks, 1, a.kv_stride_tok, a.kv_stride_blk,
+                 a.kv_stride_blk * (uint64_t)a.num_blocks, 64,
+                 a.page_size >= kMlaBN ? kMlaBN : a.page_size, 1, 1))
+    return ATTN_ERR_INVALID_ARG;
+  MlaParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = a.q;
+  p.out = a.out;
+  p.lse = a.lse;
+  p.block_table = a.block_table;
+  p.cache_seqlens = a.cache_seqlens;
+  p.indices = a.indices;
+  p.meta = a.meta;
+  p.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv_cache);
+  p.bt_stride = a.block_table_stride;
+  p.q_sb = a.q_stride_b;
+  p.q_ss = a.q_stride_s;
+  p.q_sh = a.q_stride_h;
+  p.o_sb = a.o_stride_b;
+  p.o_ss = a.o_stride_s;
+  p.o_sh = a.o_stride_h;
+  p.kv_sblk = a.kv_stride_blk;
+  p.kv_stok = a.kv_stride_tok;
+  p.idx_sb = a.idx_stride_b;
+  p.idx_ss = a.idx_stride_s;
+  p.batch = a.batch;
+  p.seqlen_q = a.seqlen_q;
+  p.heads_q = a.num_heads_q;
+  p.page_size = a.page_size;
+  p.topk = a.topk;
+  p.tiles_per_token = ds.tiles_per_token;
+  p.tokens_per_tile = ds.tokens_per_tile;
+  p.row_tiles = ds.row_tiles;
+  p.segs_per_seq = ds.sh.segs_per_seq;
+  p.num_segs = ds.S;
+  p.num_ctas = ds.G;
+  p.scale_log2 = a.scale * kLog2e;
+  p.causal = a.causal;
+  if (a.meta) {
+    const size_t slots = (size_t)ds.S + ds.G;
+    p.ws_o = reinterpret_cast<float*>(a.workspace);
+    p.ws_lse = p.ws_o + slots * kMlaRows * kMlaDvHalf;
+  }
+  auto kernel = mla_kernel<kSparse>;
+  static bool configured = false;
+  if (!configured) {
+    if (set_smem(kernel, kMlaSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
+    configured = true;
+  }
+  kernel<<<a.meta ? ds.G : ds.S, 192, kMlaSmemBytes, stream>>>(mq, mkv, p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (a.meta) {
+    const int64_t warps = (int64_t)ds.S * kMlaRows;
+    mla_combine_kernel<kSparse><<<(int)((warps + 7) / 8), 256, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+attn_status_t mla_entry(const mla_args* a, void* stream, bool sparse) {
+  attn_status_t st = check_mla(a, sparse);
+  if (st != ATTN_OK) return st;
+  DecodeShape ds;
+  st = decode_shape(sparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA, a->batch, a->seqlen_q,
+                    a->num_heads_q, a->num_heads_kv, a->topk, a->num_ctas, ds);
+  if (st != ATTN_OK) return st;
+  if (a->meta) {
+    if (a->meta_bytes < meta_bytes_for(ds)) return ATTN_ERR_INVALID_ARG;
+    if (!a->workspace || a->workspace_bytes < mla_ws_bytes(ds))
+      return ATTN_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(a->workspace)) return ATTN_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return sparse ? run_mla<true>(*a, ds, s) : run_mla<false>(*a, ds, s);
 }
 
 }  // namespace
@@ -451,12 +588,22 @@ attn_status_t attn_combine(const attn_combine_args* a, void* stream) {
   return launch_status(cudaGetLastError());
 }
 
-size_t mla_workspace_size(const mla_args*) { return 0; }
-attn_status_t mla_fwd_paged(const mla_args* a, void*) {
-  return a ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+size_t mla_workspace_size(const mla_args* a) {
+  if (!a || !a->meta) return 0;
+  const bool sparse = a->indices != nullptr;
+  if (check_mla(a, sparse) != ATTN_OK) return 0;
+  DecodeShape ds;
+  if (decode_shape(sparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA, a->batch, a->seqlen_q,
+                   a->num_heads_q, a->num_heads_kv, a->topk, a->num_ctas, ds) != ATTN_OK)
+    return 0;
+  return mla_ws_bytes(ds);
 }
-attn_status_t mla_sparse_fwd(const mla_args* a, void*) {
-  return a ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+attn_status_t mla_fwd_paged(const mla_args* a, void* stream) {
+  if (a && a->indices) return ATTN_ERR_INVALID_ARG;  // indices belong to mla_sparse_fwd
+  return mla_entry(a, stream, false);
+}
+attn_status_t mla_sparse_fwd(const mla_args* a, void* stream) {
+  return mla_entry(a, stream, true);
 }
 
 attn_status_t attn_get_device_error(int32_t* code, void* stream) {

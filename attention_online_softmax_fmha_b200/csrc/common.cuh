@@ -17,6 +17,11 @@ namespace attn {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// Online softmax: after the first key tile, the running max of a row is
+// raised (and O rescaled) only when it grows by more than this many log2
+// units; P then stays below 2^8 and the result is exact after the final
+// division by the row sum.
+constexpr float kRescaleThreshold = 8.0f;
 
 // ---------------------------------------------------------------------------
 // Device error word: the first error wins. Low 8 bits = ATTN_DEVERR_* code,

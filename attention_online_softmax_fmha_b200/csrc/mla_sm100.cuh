@@ -1,0 +1,668 @@
+// MLA-absorbed decode on sm_100a, dense (paged) and top-k sparse.
+//
+// MATE "Attention", MLA (flash_mla_with_kvcache: 576-wide rows, head_dim_v =
+// 512; flash_mla_sparse_fwd); MindSpore "sparse_flash_attention"
+// (attention_mode=2: the 512 latent ("nope") and 64 rope parts concatenated
+// along D; sparse_indices of logical positions; PA_BSND cache + block table).
+// One KV head: every query row (token i, head h) scores against the whole
+// 576-wide cached row; V is the row's first 512 entries.
+//
+// Work decomposition. An fp32 accumulator for 128 query rows x 512 V columns
+// would fill all of TMEM, so a CTA owns 128 query rows and one half of the V
+// columns (256); the two halves of a row tile are separate segments (both
+// compute S = Q K^T). Segments are split over persistent CTAs by the
+// scheduler metadata; split segments go through the combine kernel.
+//   dense : segment = (sequence, 128-row tile of (token, head) rows, V half),
+//           keys 0 .. L-1 in tiles of 32 (causal: key j visible to token i iff
+//           j <= i + L - s_q).
+//   sparse: segment = (sequence, token, head tile, V half), keys = that
+//           token's listed positions in tiles of 32 entries; entries outside
+//           [0, L) are skipped.
+//
+// Roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r (= TMEM lane r).
+//   warp 4     producer: Q tile (TMA, 144 KB resident), K/V tiles of 32
+//              keys x 576 into a 2-stage ring: dense by TMA boxes through the
+//              block table; sparse by per-lane 16-byte async copies of the
+//              gathered rows (each lane one key, zeros for skipped keys),
+//              completed and fenced before the stage is handed over.
+//   warp 5     TMEM owner and MMA issuer (whole warp, one elected lane):
+//              S_j = Q K_j^T (M=128, N=32, K=576) into one of two TMEM S
+//              buffers; O += P_j V_j (M=128, N=256, K=32) with P from TMEM.
+#pragma once
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "sched.cuh"
+
+namespace attn {
+
+constexpr int kMlaDqk = 576;
+constexpr int kMlaDv = 512;
+constexpr int kMlaDvHalf = 256;
+constexpr int kMlaBN = 32;         // keys per tile
+constexpr int kMlaRows = 128;      // query rows per CTA
+constexpr int kMlaStages = 2;
+constexpr int kMlaChunks = kMlaDqk / 64;                       // 9 column chunks
+constexpr int kMlaQChunkBytes = kMlaRows * 128;                // 16 KB
+constexpr int kMlaKVChunkBytes = kMlaBN * 128;                 // 4 KB
+constexpr int kMlaQBytes = kMlaChunks * kMlaQChunkBytes;       // 144 KB
+constexpr int kMlaKVBytes = kMlaChunks * kMlaKVChunkBytes;     // 36 KB
+constexpr int kMlaQOff = 0;
+constexpr int kMlaKVOff = kMlaQBytes;
+constexpr int kMlaBarOff = kMlaKVOff + kMlaStages * kMlaKVBytes;
+constexpr int kMlaSmemBytes = kMlaBarOff + 256 + 1024;
+constexpr uint32_t kMlaTmemCols = 512;
+constexpr uint32_t kMlaTmemS = 0;      // two S buffers of 32 columns
+constexpr uint32_t kMlaTmemO = 256;    // 256 columns of O
+
+struct MlaParams {
+  const void* q;
+  void* out;
+  float* lse;
+  const int32_t* block_table;
+  const int32_t* cache_seqlens;
+  const int32_t* indices;
+  const int32_t* meta;
+  float* ws_o;    // [slot][128][256]
+  float* ws_lse;  // [slot][128]
+  const __nv_bfloat16* kv;
+  int64_t bt_stride;
+  int64_t q_sb, q_ss, q_sh;
+  int64_t o_sb, o_ss, o_sh;
+  int64_t kv_sblk, kv_stok;
+  int64_t idx_sb, idx_ss;
+  int32_t batch, seqlen_q, heads_q, page_size, topk;
+  int32_t tiles_per_token;  // heads_q >= 128: heads_q / 128 (else 1)
+  int32_t tokens_per_tile;  // heads_q < 128: 128 / heads_q (else 1)
+  int32_t row_tiles;        // dense: row tiles per sequence
+  int32_t segs_per_seq, num_segs, num_ctas;
+  float scale_log2;
+  int32_t causal;
+};
+
+struct MlaBarriers {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[kMlaStages], kv_empty[kMlaStages];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full, o_empty;
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+// A segment and its rows.
+struct MlaSeg {
+  int b, vh, len;
+  int tok0, head0;   // first (token, head) of the row tile
+  int rows_valid;    // rows of the tile that exist (the rest are padding)
+  int units;         // KV tiles of the segment
+};
+
+template <bool kSparse>
+DEVI void mla_seg(const MlaParams& p, int s, MlaSeg& g) {
+  g.b = s / p.segs_per_seq;
+  const int rem = s - g.b * p.segs_per_seq;
+  g.vh = rem & 1;
+  const int rt = rem >> 1;  // row tile index within the sequence
+  g.len = p.cache_seqlens[g.b];
+  if (p.heads_q >= kMlaRows) {
+    g.tok0 = rt / p.tiles_per_token;
+    g.head0 = (rt % p.tiles_per_token) * kMlaRows;
+    g.rows_valid = kMlaRows;
+  } else {
+    g.tok0 = kSparse ? rt : rt * p.tokens_per_tile;
+    g.head0 = 0;
+    g.rows_valid = kSparse ? p.heads_q : min(kMlaRows, (p.seqlen_q - g.tok0) * p.heads_q);
+  }
+  if (kSparse)
+    g.units = (p.topk + kMlaBN - 1) / kMlaBN;
+  else
+    g.units = g.len > 0 ? (g.len + kMlaBN - 1) / kMlaBN : 0;
+}
+
+// Token and head of tile row x.
+DEVI void mla_row(const MlaParams& p, const MlaSeg& g, int x, int& tok, int& head) {
+  if (p.heads_q >= kMlaRows) {
+    tok = g.tok0;
+    head = g.head0 + x;
+  } else {
+    tok = g.tok0 + x / p.heads_q;
+    head = x % p.heads_q;
+  }
+}
+
+// The CTA's unit range [ub, ue) and first segment (metadata or one segment
+// per CTA).
+template <bool kSparse>
+DEVI void mla_range(const MlaParams& p, int& ub, int& ue, int& s0, const int32_t*& prefix) {
+  if (p.meta) {
+    const MetaLayout ml(p.num_ctas, p.num_segs);
+    ub = p.meta[ml.cta_begin + blockIdx.x];
+    ue = p.meta[ml.cta_begin + blockIdx.x + 1];
+    s0 = p.meta[ml.cta_seg + blockIdx.x];
+    prefix = p.meta + ml.seg_begin;
+  } else {
+    MlaSeg g;
+    mla_seg<kSparse>(p, blockIdx.x, g);
+    s0 = blockIdx.x;
+    ub = 0;
+    ue = g.units;  // an empty sequence: the softmax warps write O = 0, LSE = -inf
+    prefix = nullptr;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Producer warp
+// ---------------------------------------------------------------------------
+template <bool kSparse>
+DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensorMap* mkv,
+                       uint8_t* smem, MlaBarriers* bars) {
+  volatile int* abort = &bars->abort;
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) {
+    tma_prefetch_desc(mq);
+    if (!kSparse) tma_prefetch_desc(mkv);
+  }
+  int ub, ue, s;
+  const int32_t* prefix;
+  mla_range<kSparse>(p, ub, ue, s, prefix);
+  int it = 0, nq = 0;
+  const int P = p.page_size;
+  int u = ub;
+  while (u < ue) {
+    int sb, se;
+    if (prefix) {
+      sb = prefix[s];
+      se = prefix[s + 1];
+      if (se <= u) { ++s; continue; }
+    } else {
+      sb = u;
+      se = ue;
+    }
+    MlaSeg g;
+    mla_seg<kSparse>(p, s, g);
+    const int a = u - sb, e = min(ue, se) - sb;
+    if (e <= a) {
+      u = min(ue, se);
+      ++s;
+      continue;
+    }
+    // Q tile of the segment
+    if (lane == 0) {
+      bool ok = nq == 0 || mbar_wait(&bars->q_empty, (nq - 1) & 1, abort, 60);
+      if (ok) {
+        const int box_rows = p.heads_q >= kMlaRows ? kMlaRows : p.heads_q * (kSparse ? 1 : p.tokens_per_tile);
+        mbar_expect_tx(&bars->q_full, kMlaChunks * box_rows * 128);
+        for (int c = 0; c < kMlaChunks; ++c)
+          tma_load_4d(smem + kMlaQOff + c * kMlaQChunkBytes, mq, &bars->q_full, c * 64, g.head0,
+                      g.tok0, g.b);
+      }
+    }
+    if (!__shfl_sync(0xffffffffu, (int)(*abort == 0), 0)) return;
+    ++nq;
+    const int32_t* bt = p.block_table + (int64_t)g.b * p.bt_stride;
+    for (int t = a; t < e; ++t, ++it) {
+      const int st = it % kMlaStages;
+      uint8_t* dst = smem + kMlaKVOff + st * kMlaKVBytes;
+      bool ok = true;
+      if (lane == 0 && it >= kMlaStages)
+        ok = mbar_wait(&bars->kv_empty[st], ((it / kMlaStages) - 1) & 1, abort, 61);
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
+      if constexpr (!kSparse) {
+        // keys [32t, 32t + 32): pages of the block table, one TMA box per
+        // (page, 64-column chunk)
+        const int key0 = t * kMlaBN;
+        const int npages = (g.len + P - 1) / P;
+        const int box = P >= kMlaBN ? kMlaBN : P;
+        const int nload = P >= kMlaBN ? 1 : min(kMlaBN / P, npages - key0 / P);
+        int page = 0;
+        if (lane < nload) page = bt[key0 / P + lane];
+        if (lane == 0) {
+          mbar_expect_tx(&bars->kv_full[st], kMlaChunks * nload * box * 128);
+        }
+        for (int j = 0; j < nload; ++j) {
+          const int pg = __shfl_sync(0xffffffffu, page, j);
+          if (lane == 0)
+            for (int c = 0; c < kMlaChunks; ++c)
+              tma_load_4d(dst + c * kMlaKVChunkBytes + j * box * 128, mkv, &bars->kv_full[st],
+                          c * 64, key0 % P, pg, 0);
+        }
+      } else {
+        // lane k gathers key t*32 + k: 72 async copies of 16 bytes into the
+        // 128-byte-swizzled layout, or zeros if the entry is skipped.
+        const int e_idx = t * kMlaBN + lane;
+        int pos = -1;
+        if (e_idx < p.topk) pos = p.indices[g.b * p.idx_sb + g.tok0 * p.idx_ss + e_idx];
+        const bool valid = pos >= 0 && pos < g.len;
+        const __nv_bfloat16* src = nullptr;
+        if (valid) src = p.kv + (int64_t)bt[pos / P] * p.kv_sblk + (int64_t)(pos % P) * p.kv_stok;
+        const uint32_t dbase = smem_u32(dst) + lane * 128;
+        for (int c = 0; c < kMlaChunks; ++c) {
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const uint32_t d = dbase + c * kMlaKVChunkBytes + ((x ^ (lane & 7)) << 4);
+            if (valid) {
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d),
+                           "l"(src + c * 64 + x * 8)
+                           : "memory");
+            } else {
+              asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(d), "r"(0) : "memory");
+            }
+          }
+        }
+        // Wait for this lane's copies, make them visible to the tensor core
+        // (async proxy) and signal the stage. (With two stages the stage must
+        // be complete before the next one is claimed: releasing stage s needs
+        // the P V two tiles back, which the MMA issues after the S of the
+        // tile loaded here.)
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->kv_full[st]);
+      }
+    }
+    u = min(ue, se);
+    ++s;
+  }
+  if constexpr (!kSparse) {
+    if (lane == 0) {  // the last stages' copies must land before the CTA exits
+      int zero = 0;
+      for (int i = max(0, it - kMlaStages); i < it; ++i)
+        mbar_wait(&bars->kv_full[i % kMlaStages], (i / kMlaStages) & 1, &zero, 62);
+    }
+  }
+  if (lane == 0 && nq > 0) {
+    int zero = 0;
+    mbar_wait(&bars->q_full, (nq - 1) & 1, &zero, 63);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MMA warp (whole warp; one elected lane issues)
+// ---------------------------------------------------------------------------
+template <bool kSparse>
+DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem) {
+  volatile int* abort = &bars->abort;
+  constexpr uint32_t idesc_s = make_idesc(128, kMlaBN, 1, 0, 0);
+  constexpr uint32_t idesc_pv = make_idesc(128, kMlaDvHalf, 1, 0, 1);
+  const uint64_t dq = sdesc_sw128(smem_u32(smem + kMlaQOff), 16, 1024);
+  const uint64_t dkv = sdesc_sw128(smem_u32(smem + kMlaKVOff), 16, 1024);
+  // V half vh: chunks 4vh .. 4vh+3 of the KV tile, MN-major (leading byte
+  // offset = chunk stride, stride byte offset = 8 keys x 128 bytes).
+  const uint64_t dv = sdesc_sw128(smem_u32(smem + kMlaKVOff), kMlaKVChunkBytes, 1024);
+  int ub, ue, s;
+  const int32_t* prefix;
+  mla_range<kSparse>(p, ub, ue, s, prefix);
+  int it = 0, nq = 0, pieces = 0;
+  int u = ub;
+  while (u < ue) {
+    int sb, se;
+    if (prefix) {
+      sb = prefix[s];
+      se = prefix[s + 1];
+      if (se <= u) { ++s; continue; }
+    } else {
+      sb = u;
+      se = ue;
+    }
+    MlaSeg g;
+    mla_seg<kSparse>(p, s, g);
+    const int a = u - sb, e = min(ue, se) - sb;
+    const int n = max(0, e - a);
+    if (n == 0) {  // empty sequence without metadata: the softmax writes O = 0
+      u = min(ue, se);
+      ++s;
+      continue;
+    }
+    if (!warp_wait(&bars->q_full, nq & 1, abort, 70)) goto drain;
+    ++nq;
+    for (int j = 0; j <= n; ++j) {
+      const int gi = it + j;
+      const int st = gi % kMlaStages;
+      if (j < n) {
+        if (!warp_wait(&bars->kv_full[st], (gi / kMlaStages) & 1, abort, 71)) goto drain;
+        tc_fence_after();
+        // S_j into buffer gi & 1 (its previous P was read by PV_{j-2}, issued
+        // before this in the in-order tensor pipe)
+        const uint32_t sbuf = tmem + kMlaTmemS + (gi & 1) * kMlaBN;
+        const uint64_t kst = dkv + st * (kMlaKVBytes >> 4);
+#pragma unroll
+        for (int k = 0; k < kMlaDqk / 16; ++k) {
+          const uint32_t qo = (k >> 2) * (kMlaQChunkBytes >> 4) + (k & 3) * 2;
+          const uint32_t ko = (k >> 2) * (kMlaKVChunkBytes >> 4) + (k & 3) * 2;
+          mma_f16_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
+        }
+        tc_commit_w(&bars->s_full[gi & 1]);
+        if (j == n - 1) tc_commit_w(&bars->q_empty);
+      }
+      if (j > 0) {
+        const int gp = gi - 1, sp = gp % kMlaStages;
+        if (!warp_wait(&bars->p_full[gp & 1], (gp >> 1) & 1, abort, 72)) goto drain;
+        if (j == 1 && pieces > 0 && !warp_wait(&bars->o_empty, (pieces - 1) & 1, abort, 73))
+          goto drain;
+        tc_fence_after();
+        const uint32_t pbuf = tmem + kMlaTmemS + (gp & 1) * kMlaBN;
+        const uint64_t vst = dv + sp * (kMlaKVBytes >> 4) + g.vh * 4 * (kMlaKVChunkBytes >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kMlaBN / 16; ++kk)
+          mma_f16_ts_w(tmem + kMlaTmemO, pbuf + kk * 8, vst + kk * (16 * 128 >> 4), idesc_pv,
+                       (j > 1 || kk > 0) ? 1u : 0u);
+        tc_commit_w(&bars->kv_empty[sp]);
+        tc_commit_w(&bars->o_full);  // the softmax waits for every P V in order
+      }
+    }
+    it += n;
+    ++pieces;
+    u = min(ue, se);
+    ++s;
+  }
+drain : {
+  int zero = 0;
+  tc_commit_w(&bars->mma_drain);
+  warp_wait(&bars->mma_drain, 0, &zero, 74);
+}
+}
+
+// ---------------------------------------------------------------------------
+// Softmax warpgroup
+// ---------------------------------------------------------------------------
+template <bool kSparse>
+DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem) {
+  volatile int* abort = &bars->abort;
+  const int r = threadIdx.x;  // 0..127
+  const uint32_t lane = (uint32_t)(r & ~31) << 16;
+  const uint32_t o_tmem = tmem + kMlaTmemO + lane;
+  const MetaLayout ml(p.num_ctas, p.num_segs);
+  int ub, ue, s;
+  const int32_t* prefix;
+  mla_range<kSparse>(p, ub, ue, s, prefix);
+  int it = 0, pv = 0;
+  const float sl2 = p.scale_log2;
+  if (!p.meta && ue == 0) {
+    // empty sequence without metadata: O = 0, LSE = -inf
+    MlaSeg g;
+    mla_seg<kSparse>(p, blockIdx.x, g);
+    int tok, head;
+    mla_row(p, g, r, tok, head);
+    if (r < g.rows_valid && tok < p.seqlen_q) {
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + g.b * p.o_sb +
+                            (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + g.vh * kMlaDvHalf;
+      for (int c = 0; c < kMlaDvHalf; c += 8)
+        *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+      if (p.lse && g.vh == 0) p.lse[((int64_t)g.b * p.heads_q + head) * p.seqlen_q + tok] = -INFINITY;
+    }
+    return;
+  }
+  int u = ub;
+  while (u < ue) {
+    int sb, se;
+    if (prefix) {
+      sb = prefix[s];
+      se = prefix[s + 1];
+      if (se <= u) { ++s; continue; }
+    } else {
+      sb = u;
+      se = ue;
+    }
+    MlaSeg g;
+    mla_seg<kSparse>(p, s, g);
+    const int a = u - sb, e = min(ue, se) - sb;
+    const int n = max(0, e - a);
+    int tok, head;
+    mla_row(p, g, r, tok, head);
+    const bool valid_row = r < g.rows_valid && tok < p.seqlen_q;
+    // dense: visible keys [0, hi]; causal aligns the last token with the last key
+    int hi = g.len - 1;
+    if (!kSparse && p.causal) hi = min(hi, tok + g.len - p.seqlen_q);
+    float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
+    bool seen = false;
+    for (int j = 0; j < n; ++j) {
+      const int gi = it + j;
+      const int t = a + j;
+      if (!warp_wait(&bars->s_full[gi & 1], (gi >> 1) & 1, abort, 80)) return;
+      tc_fence_after();
+      const uint32_t s_tmem = tmem + kMlaTmemS + (gi & 1) * kMlaBN + lane;
+      uint32_t sv[kMlaBN];
+      tmem_load<32>(s_tmem, sv);
+      if constexpr (kSparse) {
+        const int* idx = p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss + t * kMlaBN;
+#pragma unroll
+        for (int c = 0; c < kMlaBN; ++c) {
+          const int pos = (t * kMlaBN + c < p.topk && valid_row) ? __ldg(idx + c) : -1;
+          if (!(pos >= 0 && pos < g.len)) sv[c] = __float_as_uint(-INFINITY);
+        }
+      } else {
+        const int k0 = t * kMlaBN;
+        if (k0 + kMlaBN - 1 > hi) {
+#pragma unroll
+          for (int c = 0; c < kMlaBN; ++c)
+            if (k0 + c > hi) sv[c] = __float_as_uint(-INFINITY);
+        }
+        // Rows of the tile past the end of the cache hold whatever the page
+        // has there: zero this V half of them so P = 0 never meets a NaN. S
+        // of this tile has been computed already.
+        const int nvalid = g.len - k0;
+        if (nvalid < kMlaBN) {
+          uint8_t* kvs = smem + kMlaKVOff + (gi % kMlaStages) * kMlaKVBytes;
+          const int bad = kMlaBN - nvalid;
+          for (int x = r; x < 4 * bad * 8; x += 128) {
+            const int c = x / (bad * 8), rem = x % (bad * 8);
+            const int row = nvalid + rem / 8, u16 = rem % 8;
+            *reinterpret_cast<uint4*>(kvs + (g.vh * 4 + c) * kMlaKVChunkBytes + row * 128 +
+                                      u16 * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kMlaBN; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+      seen |= mx != -INFINITY;
+      mx *= sl2;
+      // P V of the previous tile must be complete before O may be rescaled
+      // (waited at every tile so the barrier phases stay in step).
+      if (j > 0) {
+        if (!warp_wait(&bars->o_full, pv & 1, abort, 81)) return;
+        ++pv;
+        tc_fence_after();
+      }
+      float alpha = 1.f;
+      const bool grow = (j == 0) ? (mx > m_run) : (mx > m_run + kRescaleThreshold);
+      if (grow) {
+        if (j > 0 && m_run != -INFINITY) alpha = ex2(m_run - mx);
+        m_run = mx;
+        l_run *= alpha;
+        l_rnd *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < kMlaDvHalf; c += 32) {
+          uint32_t o[32];
+          tmem_load<32>(o_tmem + c, o);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+          tmem_store<32>(o_tmem + c, o);
+        }
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      uint32_t pk[kMlaBN / 2];
+      float le = 0.f, lr = 0.f;
+#pragma unroll
+      for (int c = 0; c < kMlaBN / 2; ++c) {
+        const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), sl2, -m_use));
+        const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -m_use));
+        // bf16 P rounded to nearest (ties away from zero; P >= 0); O is
+        // normalised by the sum of the same rounded values
+        const uint32_t r0 = __float_as_uint(p0) + 0x8000u, r1 = __float_as_uint(p1) + 0x8000u;
+        pk[c] = __byte_perm(r0, r1, 0x7632);
+        le += p0 + p1;
+        lr += __uint_as_float(r0 & 0xffff0000u) + __uint_as_float(r1 & 0xffff0000u);
+      }
+      l_run += le;
+      l_rnd += lr;
+      tmem_store<16>(s_tmem, pk);
+      tmem_store_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[gi & 1]);
+    }
+    it += n;
+
+    // --- epilogue: O / l (or a sink-free partial for the combine step) -------
+    int slot = -1;
+    if (p.meta && n > 0) {
+      const int ns = p.meta[ml.seg_nsplit + s];
+      if (ns > 1) slot = p.meta[ml.seg_slot + s] + (blockIdx.x - p.meta[ml.seg_first + s]);
+    }
+    if (n > 0) {
+      if (!warp_wait(&bars->o_full, pv & 1, abort, 82)) return;
+      ++pv;
+      tc_fence_after();
+    }
+    if (!seen) l_run = l_rnd = 0.f;
+    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+    const float inv = (l_rnd > 0.f && seen) ? 1.f / l_rnd : 0.f;
+    const float lse = (l_run > 0.f && seen) ? (m_use + log2f(l_run)) * kLn2 : -INFINITY;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + g.b * p.o_sb +
+                          (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + g.vh * kMlaDvHalf;
+    float* wrow = slot >= 0 ? p.ws_o + ((int64_t)slot * kMlaRows + r) * kMlaDvHalf : nullptr;
+#pragma unroll 1
+    for (int c = 0; c < kMlaDvHalf; c += 32) {
+      uint32_t o[32];
+      if (n > 0) {
+        tmem_load<32>(o_tmem + c, o);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) o[x] = 0u;
+      }
+      if (valid_row) {
+        if (slot < 0) {
+#pragma unroll
+          for (int x = 0; x < 32; x += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[x + 0]) * inv, __uint_as_float(o[x + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(o[x + 2]) * inv, __uint_as_float(o[x + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(o[x + 4]) * inv, __uint_as_float(o[x + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(o[x + 6]) * inv, __uint_as_float(o[x + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c + x) = v;
+          }
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(wrow + c + x) =
+                make_float4(__uint_as_float(o[x]) * inv, __uint_as_float(o[x + 1]) * inv,
+                            __uint_as_float(o[x + 2]) * inv, __uint_as_float(o[x + 3]) * inv);
+        }
+      }
+    }
+    if (n > 0) {
+      tc_fence_before();
+      mbar_arrive(&bars->o_empty);
+    }
+    if (valid_row) {
+      if (slot >= 0)
+        p.ws_lse[(int64_t)slot * kMlaRows + r] = lse;
+      else if (p.lse && g.vh == 0)
+        p.lse[((int64_t)g.b * p.heads_q + head) * p.seqlen_q + tok] = lse;
+    }
+    u = min(ue, se);
+    ++s;
+  }
+}
+
+template <bool kSparse>
+__global__ void __launch_bounds__(192, 1)
+    mla_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
+               const MlaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  MlaBarriers* bars = reinterpret_cast<MlaBarriers*>(smem + kMlaBarOff);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int i = 0; i < kMlaStages; ++i) {
+      mbar_init(&bars->kv_full[i], kSparse ? 32 : 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+    }
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->o_empty, 128);
+    mbar_init(&bars->mma_drain, 1);
+    bars->abort = 0;
+    fence_barrier_init();
+  }
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) {
+    s_bad = 0;
+    if (p.meta) {
+      const int mode = kSparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
+      if (!(meta_matches(p.meta, mode, p.batch, p.seqlen_q, p.heads_q, 1, p.page_size,
+                         p.num_segs, kMlaBN, kMlaDqk, kMlaDv) &&
+            p.meta[kMetaNumCtas] == p.num_ctas && (!kSparse || p.meta[kMetaTopk] == p.topk))) {
+        raise_error(ATTN_DEVERR_META_MISMATCH, 90);
+        s_bad = 1;
+      }
+    }
+  }
+  if (warp == 5) {
+    tmem_alloc(&bars->tmem_base, kMlaTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  if (!s_bad) {
+    if (warp < 4)
+      mla_softmax<kSparse>(p, smem, bars, tmem);
+    else if (warp == 4)
+      mla_producer<kSparse>(p, &map_q, &map_kv, smem, bars);
+    else
+      mla_mma<kSparse>(p, smem, bars, tmem);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kMlaTmemCols);
+  }
+}
+
+// Merges split MLA segments: one warp per (segment, row); each segment covers
+// 256 of the 512 output columns (its V half); the V-half-0 segment writes LSE.
+template <bool kSparse>
+__global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int s = gw / kMlaRows, r = gw % kMlaRows;
+  if (s >= p.num_segs) return;
+  const int mode = kSparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
+  if (!(meta_matches(p.meta, mode, p.batch, p.seqlen_q, p.heads_q, 1, p.page_size, p.num_segs,
+                     kMlaBN, kMlaDqk, kMlaDv) &&
+        p.meta[kMetaNumCtas] == p.num_ctas))
+    return;
+  const MetaLayout ml(p.num_ctas, p.num_segs);
+  const int ns = p.meta[ml.seg_nsplit + s];
+  if (ns == 1) return;
+  MlaSeg g;
+  mla_seg<kSparse>(p, s, g);
+  int tok, head;
+  mla_row(p, g, r, tok, head);
+  if (r >= g.rows_valid || tok >= p.seqlen_q) return;
+  const int slot0 = ns > 1 ? p.meta[ml.seg_slot + s] : 0;
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + g.b * p.o_sb +
+                       (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + g.vh * kMlaDvHalf;
+  const float lse = combine_row(
+      ns, kMlaDvHalf, 0.f, false,
+      [&](int k) { return p.ws_lse[(int64_t)(slot0 + k) * kMlaRows + r]; },
+      [&](int k) { return p.ws_o + ((int64_t)(slot0 + k) * kMlaRows + r) * kMlaDvHalf; },
+      [&](int c, float v) { store_out(dst + c, v); });
+  if (p.lse && g.vh == 0 && (threadIdx.x & 31) == 0)
+    p.lse[((int64_t)g.b * p.heads_q + head) * p.seqlen_q + tok] = lse;
+}
+
+}  // namespace attn

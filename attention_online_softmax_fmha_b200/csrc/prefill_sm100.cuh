@@ -62,7 +62,7 @@ struct PrefillParams {
 constexpr int kPrefillBM = 128;               // query rows per tile
 constexpr int kPrefillUnit = 2 * kPrefillBM;  // query rows per work unit
 constexpr int kPrefillBN = 128;               // keys per tile
-constexpr float kRescaleThreshold = 8.0f;     // log2 units
+
 // Of every 16 P pairs, this many are exponentiated on the FMA pipe (a
 // polynomial) and the rest on the MUFU pipe, to balance the two.
 constexpr int kEmuPairs = 4;
@@ -535,10 +535,10 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
             pk[c] = pack_f16x2(p0, p1);
             acc_r[c & 3] = add2(acc_r[c & 3], widen2<true>(pk[c]));
           } else {
-            // bf16 by truncation (keep the top 16 bits) on the integer pipe.
-            // Normalising O by the sum of these same values cancels their
-            // common bias; what remains is of the size of a rounding error.
-            const uint32_t r0 = __float_as_uint(p0), r1 = __float_as_uint(p1);
+            // bf16 rounding on the integer pipe (P >= 0: add half an ulp of
+            // bf16, keep the top 16 bits: to nearest, ties away from zero).
+            const uint32_t r0 = __float_as_uint(p0) + 0x8000u;
+            const uint32_t r1 = __float_as_uint(p1) + 0x8000u;
             pk[c] = __byte_perm(r0, r1, 0x7632);
             acc_r[c & 3] = add2(acc_r[c & 3], f2pack(__uint_as_float(r0 & 0xffff0000u),
                                                      __uint_as_float(r1 & 0xffff0000u)));

@@ -267,6 +267,67 @@ def paged_workload(name: str, seed: int, device):
                 f"{nbytes} B per step")
 
 
+def mla_workload(name: str, seed: int, device):
+    inp = W.build_config(name, seed=seed, device=device)
+    import ctypes
+    L = B.lib()
+    sparse = inp.indices is not None
+    sq, Hq = inp.q.shape[1], inp.num_heads_q
+    topk = inp.topk if sparse else 0
+    sa = B.sched_args(inp.cache_seqlens, batch=inp.batch, seqlen_q=sq, num_heads_q=Hq,
+                      num_heads_kv=1, head_dim_qk=576, head_dim_v=512, page_size=inp.page_size,
+                      mode=B.SCHED_MLA_SPARSE if sparse else B.SCHED_MLA, topk=topk)
+    meta = torch.empty(B.sched_metadata_size(sa) // 4, dtype=torch.int32, device=device)
+    sa.meta = meta.data_ptr()
+    sa.meta_bytes = meta.numel() * 4
+    ma, out, lse, ws = B.mla_args(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens,
+                                  scale=inp.scale, causal=inp.causal, indices=inp.indices,
+                                  meta=meta)
+    fn = L.mla_sparse_fwd if sparse else L.mla_fwd_paged
+    if sparse:
+        idx = inp.indices.cpu()
+        lens = torch.tensor(inp.seqlens).view(-1, 1, 1, 1)
+        pairs_tok = int(((idx >= 0) & (idx < lens)).sum())   # visible keys over all tokens
+        kv_rows = pairs_tok
+    else:
+        pairs_tok = sum(inp.seqlens) * sq
+        kv_rows = sum(inp.seqlens)
+    flops = 2.0 * (576 + 512) * Hq * pairs_tok
+    nbytes = kv_rows * 576 * 2 + inp.q.numel() * 2 + out.numel() * 2 + lse.numel() * 4
+
+    def step(stream):
+        st = L.attn_sched_metadata(ctypes.byref(sa), stream.cuda_stream)
+        if st != B.OK:
+            raise B.AttnError("attn_sched_metadata", st)
+        st = fn(ctypes.byref(ma), stream.cuda_stream)
+        if st != B.OK:
+            raise B.AttnError(name, st)
+
+    small = [inp.q, inp.block_table, inp.cache_seqlens] + ([inp.indices] if sparse else [])
+    host_small = [t.cpu().pin_memory() for t in small]
+    host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                torch.empty(lse.shape, dtype=lse.dtype).pin_memory()]
+
+    def e2e_step(stream):
+        for h, d in zip(host_small, small):
+            d.copy_(h, non_blocking=True)
+        step(stream)
+        host_out[0].copy_(out, non_blocking=True)
+        host_out[1].copy_(lse, non_blocking=True)
+
+    cfg = {"workload": name, "batch": inp.batch, "seqlen_q": sq, "num_heads_q": Hq,
+           "num_heads_kv": 1, "head_dim_qk": 576, "head_dim_v": 512, "page_size": inp.page_size,
+           "cache_seqlens": "uniform[4096,65536]", "topk": topk or None, "dtype": "bf16",
+           "kv_bytes_per_step": nbytes}
+    return dict(step=step, e2e_step=e2e_step, work=flops / 1e12, unit="TFLOP/s", bound="tensor",
+                kernel=f"mla_kernel<{int(sparse)}>", launches_per_step=3,
+                h2d=sum(t.numel() * t.element_size() for t in host_small),
+                d2h=sum(t.numel() * t.element_size() for t in host_out), cfg=cfg, dtype="bf16",
+                inp=inp, keep=(meta, ws, out, lse), gbytes=nbytes / 1e9,
+                per_unit=f"2*(576+512)*H_q FLOP per visible (token, key) pair; "
+                f"{pairs_tok} pairs, {nbytes} bytes per step")
+
+
 WORKLOADS = {
     "tiny_dense_mha": prefill_workload,
     "varlen_causal_gqa": prefill_workload,
@@ -274,6 +335,8 @@ WORKLOADS = {
     "window_sink_fp8": prefill_workload,
     "paged_decode": paged_workload,
     "paged_decode_small": paged_workload,
+    "mla_dense": mla_workload,
+    "mla_sparse": mla_workload,
 }
 
 
@@ -422,6 +485,9 @@ def run_ours(args, rank, world, device):
             "gpu_launches": wl["launches_per_step"] * args.steps,
             "work_per_step": wl["work"], "per_unit": wl["per_unit"],
         }
+        if "gbytes" in wl:
+            results[name]["gbytes_per_s"] = wl["gbytes"] / per_launch
+            results[name]["hbm_frac"] = wl["gbytes"] / per_launch / peaks["hbm_gbs"]
         del wl
         torch.cuda.empty_cache()
     return results

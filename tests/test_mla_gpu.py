@@ -1,0 +1,142 @@
+"""MLA-absorbed decode (mla_fwd_paged) and its top-k sparse variant
+(mla_sparse_fwd) on the GPU against the fp64 oracle: bf16 outputs within
+1e-2 max-abs, LSE within 1e-3."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_online_softmax_fmha_b200 import binding as B
+from attention_online_softmax_fmha_b200 import build as BUILD
+from attention_online_softmax_fmha_b200 import workloads as W
+from tests._util import assert_close_lse, assert_close_out, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    BUILD.build()
+    B.lib()
+
+
+def run(inp, use_meta=True, num_ctas=0):
+    meta = None
+    topk = inp.topk if inp.indices is not None else 0
+    if use_meta:
+        meta = B.mla_metadata(inp.cache_seqlens, batch=inp.batch, seqlen_q=inp.q.shape[1],
+                              num_heads_q=inp.num_heads_q, page_size=inp.page_size, topk=topk,
+                              num_ctas=num_ctas)
+    kw = dict(scale=inp.scale, causal=inp.causal, meta=meta, num_ctas=num_ctas)
+    if inp.indices is None:
+        out, lse = B.mla_fwd_paged(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, **kw)
+    else:
+        out, lse = B.mla_sparse_fwd(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens,
+                                    inp.indices, **kw)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    return out, lse
+
+
+def check(inp, **kw):
+    out, lse = run(inp, **kw)
+    q, kv = to_f64(inp.q), to_f64(inp.kv_cache)
+    bt = inp.block_table.cpu().numpy()
+    if inp.indices is None:
+        ro, rl = oracle.mla_paged(q, kv, bt, inp.seqlens, 512, inp.scale, inp.causal)
+    else:
+        ro, rl = oracle.mla_sparse(q, kv, bt, inp.seqlens, inp.indices.cpu().numpy(), 512,
+                                   inp.scale)
+    assert_close_out(to_f64(out), ro, 1e-2)
+    assert_close_lse(lse.cpu().numpy(), rl)
+
+
+LENS = [1, 31, 32, 33, 200, 1000]
+
+
+@pytest.mark.parametrize("num_ctas", [1, 5, 0])
+def test_dense_split_counts(num_ctas):
+    inp = W.make_mla(seqlens=LENS, seqlen_q=2, num_heads_q=128, page_size=64, seed=0,
+                     device="cuda")
+    check(inp, num_ctas=num_ctas)
+
+
+def test_dense_without_metadata_causal_and_page16():
+    inp = W.make_mla(seqlens=[5, 77, 300], seqlen_q=2, num_heads_q=128, page_size=16,
+                     causal=True, seed=1, device="cuda")
+    check(inp, use_meta=False)
+    check(inp, num_ctas=4)
+
+
+def test_mate_example_shapes():
+    # The MATE MLA example: q (1, 32, 8, 576), a 4-page cache of 16-token
+    # pages, block_table all zeros, cache_seqlens [32], head_dim_v 512. Its
+    # cache has 2 KV heads, which is rejected; with one KV head it runs (the
+    # all-zero table repeats page 0).
+    g = torch.Generator(device="cuda").manual_seed(0)
+    q = torch.randn(1, 32, 8, 576, generator=g, device="cuda").to(torch.bfloat16)
+    bt = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
+    cs = torch.tensor([32], dtype=torch.int32, device="cuda")
+    kv2 = torch.randn(4, 16, 2, 576, generator=g, device="cuda").to(torch.bfloat16)
+    with pytest.raises(B.AttnError) as e:
+        B.mla_fwd_paged(q, kv2, bt, cs, head_dim_v=512)
+    assert e.value.status == B.UNSUPPORTED
+    kv1 = kv2[:, :, :1].contiguous()
+    out, lse = B.mla_fwd_paged(q, kv1, bt, cs, head_dim_v=512)
+    torch.cuda.synchronize()
+    ro, rl = oracle.mla_paged(to_f64(q), to_f64(kv1), bt.cpu().numpy(), [32], 512, 1 / 24.0)
+    assert_close_out(to_f64(out), ro, 1e-2)
+    assert_close_lse(lse.cpu().numpy(), rl)
+
+
+@pytest.mark.parametrize("num_ctas", [3, 0])
+def test_sparse_against_oracle(num_ctas):
+    inp = W.make_mla(seqlens=[20, 300, 3000], seqlen_q=2, num_heads_q=128, page_size=64,
+                     topk=256, seed=2, device="cuda")
+    inp.indices[0, 1, 0, 5] = 19999       # beyond the cache: skipped
+    inp.indices[2, 0, 0, 7] = -5          # negative: skipped
+    check(inp, num_ctas=num_ctas)
+    check(inp, use_meta=False)
+
+
+def test_sparse_all_positions_equals_dense():
+    inp = W.make_mla(seqlens=[64, 100], seqlen_q=1, num_heads_q=128, page_size=32, topk=128,
+                     index_kind="all", seed=3, device="cuda")
+    out_s, lse_s = run(inp, num_ctas=2)
+    dense = W.MlaInputs(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, inp.seqlens,
+                        inp.page_size, inp.num_heads_q, 512, False, inp.scale, None, 0)
+    out_d, lse_d = run(dense, num_ctas=2)
+    assert (to_f64(out_s) - to_f64(out_d)).__abs__().max() <= 2e-2
+    assert np.abs(lse_s.cpu().numpy() - lse_d.cpu().numpy()).max() <= 1e-3
+    check(inp, num_ctas=2)
+
+
+def _sampled(name, topk):
+    inp = W.build_config(name, seed=0, device="cuda")
+    out, lse = run(inp)
+    o, l = to_f64(out), lse.cpu().numpy()
+    order = np.argsort(inp.seqlens)
+    for b in [int(order[0]), int(order[-1]), 9]:
+        L = inp.seqlens[b]
+        npg = -(-L // inp.page_size)
+        pages = inp.block_table[b, :npg].long()
+        kv = to_f64(inp.kv_cache[pages])
+        q = to_f64(inp.q[b:b + 1])
+        if topk:
+            ro, rl = oracle.mla_sparse(q, kv, np.arange(npg)[None], [L],
+                                       inp.indices[b:b + 1].cpu().numpy(), 512, inp.scale)
+        else:
+            ro, rl = oracle.mla_paged(q, kv, np.arange(npg)[None], [L], 512, inp.scale)
+        assert_close_out(o[b:b + 1], ro, 1e-2)
+        assert_close_lse(l[b:b + 1], rl)
+
+
+def test_full_size_dense_sampled():
+    """MLA dense decode at full size (64 sequences, L ~ U[4096, 65536], 2
+    tokens x 128 heads, pages of 64, permuted table); 3 sequences checked."""
+    _sampled("mla_dense", 0)
+
+
+def test_full_size_sparse_sampled():
+    """The top-2048 sparse variant at full size; 3 sequences checked."""
+    _sampled("mla_sparse", 2048)
