@@ -406,6 +406,21 @@ def load_for(fn, stream, seconds: float):
             stream.synchronize()
 
 
+def reduce_max_over_ranks(values_ms, world: int, device) -> list:
+    """Max of each timing over all ranks (every rank gets the result)."""
+    if world <= 1:
+        return [float(v) for v in values_ms]
+    t = torch.tensor([float(v) for v in values_ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_rate(work_per_step: float, steps: int, world: int, total_ms: float) -> float:
+    """Work done by all ranks (weak scaling: each rank runs `steps` steps of
+    its own batch) divided by the slowest rank's time."""
+    return work_per_step * steps * world / (total_ms / 1e3)
+
+
 def time_steps(fn, steps: int, warmup: int, stream, flush):
     for _ in range(warmup):
         fn(stream)
@@ -454,15 +469,9 @@ def run_ours(args, rank, world, device):
         if err:
             raise RuntimeError(f"{name}: device error word {err:#x}")
         e2e_times = time_steps(wl["e2e_step"], max(2, args.steps // 2), 2, stream, flush)
-        tot = sum(times)
-        e2e_tot = sum(e2e_times)
-        if world > 1:
-            t = torch.tensor([tot, e2e_tot], dtype=torch.float64, device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            tot, e2e_tot = float(t[0]), float(t[1])
-        work = wl["work"] * args.steps * world
-        value = work / (tot / 1e3)
-        e2e_value = wl["work"] * len(e2e_times) * world / (e2e_tot / 1e3)
+        tot, e2e_tot = reduce_max_over_ranks([sum(times), sum(e2e_times)], world, device)
+        value = whole_job_rate(wl["work"], args.steps, world, tot)
+        e2e_value = whole_job_rate(wl["work"], len(e2e_times), world, e2e_tot)
         per_launch = tot / args.steps / 1e3  # s, one kernel sequence
         achieved = wl["work"] / per_launch
         if wl["bound"] == "tensor":
