@@ -98,7 +98,7 @@ ARG_STRUCTS = {0: VarlenArgs, 1: SchedArgs, 2: PagedArgs, 3: CombineArgs, 4: Mla
 EXPORTS = ["attn_fwd_varlen", "attn_sched_metadata_size", "attn_sched_metadata",
            "attn_paged_workspace_size", "attn_fwd_paged_kvcache", "attn_combine",
            "mla_workspace_size", "mla_fwd_paged", "mla_sparse_fwd", "attn_get_device_error",
-           "attn_status_str", "attn_args_sizeof"]
+           "attn_status_str", "attn_args_sizeof", "attn_fwd_paged_kvcache_static"]
 
 _lib = None
 
@@ -118,7 +118,8 @@ def lib() -> ctypes.CDLL:
                           "`python -m attention_online_softmax_fmha_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
         for name in ["attn_fwd_varlen", "attn_sched_metadata", "attn_fwd_paged_kvcache",
-                     "attn_combine", "mla_fwd_paged", "mla_sparse_fwd"]:
+                     "attn_combine", "mla_fwd_paged", "mla_sparse_fwd",
+                     "attn_fwd_paged_kvcache_static"]:
             getattr(L, name).argtypes = [c_vp, c_vp]
             getattr(L, name).restype = c_i32
         for name in ["attn_sched_metadata_size"]:
@@ -290,6 +291,18 @@ def fwd_paged_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, *, stream
     a, out, lse, ws = paged_args(q, k_cache, v_cache, block_table, cache_seqlens, **kw)
     _check("attn_fwd_paged_kvcache", lib().attn_fwd_paged_kvcache(ctypes.byref(a),
                                                                  _stream(stream)))
+    return out, lse
+
+
+def fwd_paged_kvcache_static(q, k_cache, v_cache, block_table, cache_seqlens, *, stream=None,
+                             num_ctas=0, **kw):
+    """Paged-KV decode with the library's built-in scratch
+    (attn_fwd_paged_kvcache_static): for callers that cannot allocate the
+    metadata and workspace buffers. Returns (out, lse)."""
+    a, out, lse, _ = paged_args(q, k_cache, v_cache, block_table, cache_seqlens,
+                                num_ctas=num_ctas, **kw)
+    _check("attn_fwd_paged_kvcache_static",
+           lib().attn_fwd_paged_kvcache_static(ctypes.byref(a), _stream(stream)))
     return out, lse
 
 

@@ -644,3 +644,83 @@ size_t attn_args_sizeof(int32_t which) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attn_fwd_paged_kvcache_static: the paged decode with built-in scratch.
+//
+// The regular entry point needs two caller-provided device buffers (the
+// scheduler metadata and the split-KV partials). This variant keeps both in
+// one file-scope device array instead, so a caller that cannot allocate
+// device memory can still run the split-KV decode. The array is part of the
+// library image: every GPU on which the library is used holds it until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_paged_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once
+// per device; host code must not use the array's name as an address).
+void* static_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress((void**)&ptr, g_paged_scratch) != cudaSuccess) return nullptr;
+    g_scratch_addr[dev] = ptr;
+  }
+  return g_scratch_addr[dev];
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_fwd_paged_kvcache_static(const attn_paged_args* args,
+                                                       void* stream) {
+  if (!args) return ATTN_ERR_INVALID_ARG;
+  // This entry point brings its own scratch; caller buffers are a usage error.
+  if (args->meta != nullptr || args->workspace != nullptr) return ATTN_ERR_INVALID_ARG;
+  attn_status_t st = check_paged(args);
+  if (st != ATTN_OK) return st;
+  DecodeShape ds;
+  st = decode_shape(ATTN_SCHED_MHA, args->batch, args->seqlen_q, args->num_heads_q,
+                    args->num_heads_kv, 0, args->num_ctas, ds);
+  if (st != ATTN_OK) return st;
+  // metadata first (256-byte aligned), the split-KV partials after it
+  const size_t meta_bytes = (meta_bytes_for(ds) + 255) & ~size_t(255);
+  const size_t ws_bytes = paged_ws_bytes(args, ds);
+  if (meta_bytes + ws_bytes > kStaticScratchBytes) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+  unsigned char* base = static_cast<unsigned char*>(static_scratch_address());
+  if (base == nullptr) return ATTN_ERR_CUDA;
+
+  // Nothing in the scratch has to start at zero: the metadata kernel writes
+  // every word the decode and combine kernels read, and every partial slot the
+  // combine reads is written by the decode kernel first.
+  attn_sched_args sa;
+  memset(&sa, 0, sizeof(sa));
+  sa.cache_seqlens = args->cache_seqlens;
+  sa.batch = args->batch;
+  sa.seqlen_q = args->seqlen_q;
+  sa.num_heads_q = args->num_heads_q;
+  sa.num_heads_kv = args->num_heads_kv;
+  sa.head_dim_qk = args->head_dim;
+  sa.head_dim_v = args->head_dim;
+  sa.page_size = args->page_size;
+  sa.mode = ATTN_SCHED_MHA;
+  sa.num_ctas = args->num_ctas;
+  sa.meta = reinterpret_cast<int32_t*>(base);
+  sa.meta_bytes = meta_bytes;
+  st = attn_sched_metadata(&sa, stream);
+  if (st != ATTN_OK) return st;
+  attn_paged_args a = *args;
+  a.meta = reinterpret_cast<const int32_t*>(base);
+  a.meta_bytes = meta_bytes;
+  a.workspace = base + meta_bytes;
+  a.workspace_bytes = ws_bytes;
+  return attn_fwd_paged_kvcache(&a, stream);
+}

@@ -240,6 +240,35 @@ size_t attn_paged_workspace_size(const attn_paged_args* args);
 attn_status_t attn_fwd_paged_kvcache(const attn_paged_args* args, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* attn_fwd_paged_kvcache_static: the same paged split-KV decode, with no    */
+/* caller-provided scratch. The pages have no counterpart of this entry      */
+/* point; it exists for callers that cannot allocate device memory when      */
+/* they run the decode -- for example code that runs inside a host callback  */
+/* or a plugin interface that hands it only its inputs and outputs, or a     */
+/* runtime whose device memory is fully reserved up front -- so they cannot  */
+/* provide the metadata and workspace buffers attn_fwd_paged_kvcache needs.  */
+/*                                                                          */
+/* Arguments as attn_fwd_paged_kvcache, except that meta and workspace must  */
+/* be NULL (ATTN_ERR_INVALID_ARG otherwise): the scheduler metadata and the  */
+/* split partials live in one 16 MiB array inside the library image, which   */
+/* every GPU that uses the library holds until the process exits. The call   */
+/* computes the metadata itself (num_ctas as given, 0 = SM count), then runs */
+/* the decode and the combine. Problems whose metadata plus partials exceed  */
+/* 16 MiB (about S + G slots of 16 x D x 4 bytes, S = batch x H_kv x         */
+/* ceil(s_q x H_q / H_kv / 16), G = num_ctas) return                         */
+/* ATTN_ERR_WORKSPACE_TOO_SMALL and launch nothing. No device memory is     */
+/* allocated or freed.                                                       */
+/*                                                                          */
+/* The first call on a device looks up the array's device address (a        */
+/* runtime call); make that first call before any stream capture. All calls */
+/* share the one array and it keeps the last call's contents: calls that may */
+/* overlap on the GPU (other streams, other host threads) race on it and     */
+/* must be serialised by the caller. Nothing in the array needs to start at */
+/* zero.                                                                     */
+/* ------------------------------------------------------------------------ */
+attn_status_t attn_fwd_paged_kvcache_static(const attn_paged_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* attn_combine: merge split partial results.                                */
 /*                                                                          */
 /* MATE "Attention", FMHA notes (flash_attn_combine merges partial outputs   */
