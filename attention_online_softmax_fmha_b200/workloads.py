@@ -293,6 +293,11 @@ CONFIGS = {
                       page_size=64),
     "mla_sparse": dict(kind="mla", lengths=(64, 4096, 65536), seqlen_q=2, num_heads_q=128,
                        page_size=64, topk=2048),
+    # 8-sequence versions of the MLA workloads, for profiler captures
+    "mla_dense_small": dict(kind="mla", lengths=(8, 4096, 65536), seqlen_q=2, num_heads_q=128,
+                            page_size=64),
+    "mla_sparse_small": dict(kind="mla", lengths=(8, 4096, 65536), seqlen_q=2,
+                             num_heads_q=128, page_size=64, topk=2048),
 }
 
 

@@ -337,6 +337,8 @@ WORKLOADS = {
     "paged_decode_small": paged_workload,
     "mla_dense": mla_workload,
     "mla_sparse": mla_workload,
+    "mla_dense_small": mla_workload,
+    "mla_sparse_small": mla_workload,
 }
 
 
