@@ -349,6 +349,28 @@ DEVI uint64_t mul2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// max(a, b, c) in one instruction (sm_100).
+DEVI float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Adds the two 16-bit floats of a packed word to two fp32 accumulators with
+// the sm_100 mixed-precision add (the 16-bit operand is widened exactly).
+template <bool kFp16>
+DEVI void acc_packed(float& lo, float& hi, uint32_t packed) {
+  if constexpr (kFp16) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.f16 %0, l, %0;\n\tadd.rn.f32.f16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi) : "r"(packed));
+  } else {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi) : "r"(packed));
+  }
+}
+
 // The two 16-bit floats of a packed word, widened to fp32 (exact).
 template <bool kFp16>
 DEVI uint64_t widen2(uint32_t packed) {
@@ -364,6 +386,25 @@ template <uint32_t N>
 DEVI void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 template <uint32_t N>
 DEVI void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
+// 32 lanes x 64 columns of 32 bits in one load (outputs valid on return).
+DEVI void tmem_load64(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : ATTN_R16(0), ATTN_R16(16), ATTN_R16(32), ATTN_R16(48)
+      : "r"(taddr)
+      : "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32).
+DEVI void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 // 32 lanes x 128 columns of 32 bits in one load (outputs valid on return).
 DEVI void tmem_load128(uint32_t taddr, uint32_t* r) {

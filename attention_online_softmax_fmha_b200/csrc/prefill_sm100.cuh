@@ -18,10 +18,11 @@
 //   warp 8           TMA producer: Q0, Q1 and a ring of K/V tiles, 128-byte
 //                    swizzled, one head per box.
 //   warp 9           TMEM owner and MMA issuer (one thread), in the order
-//                    S0_j, PV1_{j-1}, S1_j, PV0_j, ... so that the tensor core
-//                    works on one tile while the other tile's softmax runs.
-//                    S_w = Q_w K^T lands in TMEM; P_w (bf16) overwrites it and
-//                    is the TMEM A operand of O_w += P_w V.
+//                    PV0_{j-1}, S0_j, PV1_{j-1}, S1_j, ... so that the tensor
+//                    core works on one tile while the other tile's softmax
+//                    runs. S_w = Q_w K^T lands in TMEM; P_w (bf16) overwrites
+//                    it and is the TMEM A operand of O_w += P_w V, started on
+//                    the first 96 keys while the last 32 are exponentiated.
 //   warps 10, 11     FP8 only: convert each e4m3 V tile to fp16 for P V;
 //                    otherwise idle (they complete the register warpgroup).
 // Registers move from warpgroup 2 to the softmax warpgroups with setmaxnreg;
@@ -65,7 +66,13 @@ constexpr int kPrefillBN = 128;               // keys per tile
 
 // Of every 16 P pairs, this many are exponentiated on the FMA pipe (a
 // polynomial) and the rest on the MUFU pipe, to balance the two.
-constexpr int kEmuPairs = 4;
+constexpr int kEmuPairs = 0;
+// The softmax hands P to the MMA warp in two parts: the first kSplitKeys keys
+// (p_head), then the rest (p_full), so that the P V MMA starts on the head
+// while the tail is exponentiated.
+constexpr int kSplitKeys = 96;
+static_assert(kSplitKeys % 32 == 0 && kSplitKeys > 0 && kSplitKeys < kPrefillBN,
+              "split on a 32-key chunk");
 constexpr int kPrefillThreads = 384;
 constexpr int kPrefillLaunchRegs = 168;       // 65536 / 384, rounded down to 8
 constexpr int kPrefillSoftmaxRegs = 208;
@@ -98,7 +105,10 @@ struct PrefillCfg {
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kVHOff = kVOff + kVStages * kTileBytes;
   static constexpr int kBarOff = kVHOff + kVHStages * kVHBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers, + alignment slack
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmemBytes = kBarOff + kBarBytes;
+  // The dynamic shared memory base is 1024-byte aligned (the kernel checks).
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128;
   static constexpr uint32_t kTmemO0 = 256, kTmemO1 = 256 + D;
@@ -108,11 +118,12 @@ struct PrefillBarriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t vh_full[4], vh_empty[4];
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t s_full[2], p_head[2], p_full[2], o_full[2], o_empty[2];
   uint64_t mma_drain;
   uint32_t tmem_base;
   int32_t abort;
 };
+static_assert(sizeof(PrefillBarriers) <= 512, "barrier block");
 
 struct PrefillUnit {
   int b, h, m;
@@ -253,12 +264,30 @@ DEVI void prefill_issue_s(uint32_t d_tmem, uint64_t dq, uint64_t dk, uint32_t id
       mma_f16_ss_w(d_tmem, dq + off16, dk + off16, idesc, k > 0 ? 1u : 0u);
   }
 }
+template <int kK0, int kK1>
 DEVI void prefill_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t dv, uint32_t idesc,
                            bool first) {
 #pragma unroll
-  for (int kk = 0; kk < kPrefillBN / 16; ++kk)
+  for (int kk = kK0; kk < kK1; ++kk)
     mma_f16_ts_w(d_tmem, a_tmem + kk * 8, dv + kk * (16 * 128 >> 4), idesc,
                (!first || kk > 0) ? 1u : 0u);
+}
+
+// O_w += P_w V for the key tile with global index g: the head of P as soon as
+// the softmax has released it, then the tail.
+DEVI bool prefill_pv(PrefillBarriers* bars, int w, int g, uint32_t t_o, uint32_t t_p, uint64_t dv,
+                     uint32_t idesc, bool first) {
+  volatile int* abort = &bars->abort;
+  constexpr int kHead = kSplitKeys / 16;
+  if constexpr (kHead > 0) {
+    if (!warp_wait(&bars->p_head[w], g & 1, abort, 16)) return false;
+    tc_fence_after();
+    prefill_issue_pv<0, kHead>(t_o, t_p, dv, idesc, first);
+  }
+  if (!warp_wait(&bars->p_full[w], g & 1, abort, 11)) return false;
+  tc_fence_after();
+  prefill_issue_pv<kHead, kPrefillBN / 16>(t_o, t_p, dv, idesc, first);
+  return true;
 }
 
 template <int D, int kType>
@@ -305,12 +334,12 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
         if (!warp_wait(&bars->k_full[s], (g / C::kKStages) & 1, abort, 14)) goto drain;
       }
       if (j > 0) {
-        if (!warp_wait(&bars->p_full[0], (g - 1) & 1, abort, 11)) goto drain;
         if (!warp_wait(&pv_full[sp], ((g - 1) / kPVStages) & 1, abort, 12)) goto drain;
         if (j == 1 && units > 0 && !warp_wait(&bars->o_empty[0], (units - 1) & 1, abort, 13))
           goto drain;
-        tc_fence_after();
-        prefill_issue_pv(tO0, tS0, dv_base + sp * (kPVBytes >> 4), idesc_pv, j == 1);
+        if (!prefill_pv(bars, 0, g - 1, tO0, tS0, dv_base + sp * (kPVBytes >> 4), idesc_pv,
+                        j == 1))
+          goto drain;
         if (j == n) tc_commit_w(&bars->o_full[0]);
       } else {
         tc_fence_after();
@@ -320,11 +349,11 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
         tc_commit_w(&bars->s_full[0]);
       }
       if (j > 0) {
-        if (!warp_wait(&bars->p_full[1], (g - 1) & 1, abort, 11)) goto drain;
         if (j == 1 && units > 0 && !warp_wait(&bars->o_empty[1], (units - 1) & 1, abort, 13))
           goto drain;
-        tc_fence_after();
-        prefill_issue_pv(tO1, tS1, dv_base + sp * (kPVBytes >> 4), idesc_pv, j == 1);
+        if (!prefill_pv(bars, 1, g - 1, tO1, tS1, dv_base + sp * (kPVBytes >> 4), idesc_pv,
+                        j == 1))
+          goto drain;
         if (j == n) tc_commit_w(&bars->o_full[1]);
         tc_commit_w(&pv_empty[sp]);
       }
@@ -396,12 +425,143 @@ DEVI void prefill_convert(const PrefillParams& p, uint8_t* smem, PrefillBarriers
 }
 
 // ---------------------------------------------------------------------------
-// Softmax warpgroups: warpgroup w owns tile Q_w, one query row per thread
+// Softmax warpgroups: warpgroup w owns tile Q_w, thread r query row r of it
+// (= TMEM lane r). The two warpgroups run offset by about half a tile, so one
+// exponentiates while the other waits for its next S.
 // ---------------------------------------------------------------------------
+struct PrefillRow {
+  float m_run;  // running max (log2 domain, includes the sink)
+  float l_run;  // sum of the fp32 P (for the LSE)
+  float l_rnd;  // sum of the rounded P the MMA consumes (for O)
+  int lo, hi;   // visible key range
+  bool seen;    // some key of this row is visible
+};
+
+// One S tile of keys [k0, k0 + 128) of this thread's row: mask, row max,
+// lazy O rescale, P = 2^(s * scale * log2e - m) written over S (head first),
+// row sums. Returns false if a wait gave up.
+template <int D, int kType>
+DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t o_tmem, int w,
+                               int j, int g, int k0, float sl2, PrefillRow& row) {
+  constexpr bool kFp16 = kType != 0;  // P in fp16 (fp16 and FP8 inputs)
+  volatile int* abort = &bars->abort;
+  if (!warp_wait(&bars->s_full[w], g & 1, abort, 20 + w)) return false;
+  tc_fence_after();
+  uint32_t s[kPrefillBN];
+  tmem_load128(s_tmem, s);
+  if (!(k0 >= row.lo && k0 + kPrefillBN - 1 <= row.hi)) {
+#pragma unroll
+    for (int c = 0; c < kPrefillBN; ++c) {
+      const bool vis = (k0 + c >= row.lo) && (k0 + c <= row.hi);
+      s[c] = vis ? s[c] : __float_as_uint(-INFINITY);
+    }
+  }
+  // Row max: four independent chains of three-input maxima.
+  float mx4[4];
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+    mx4[x] = fmax3(__uint_as_float(s[x]), __uint_as_float(s[4 + x]), __uint_as_float(s[8 + x]));
+#pragma unroll
+  for (int c = 12; c + 8 <= kPrefillBN; c += 8)
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+      mx4[x] = fmax3(mx4[x], __uint_as_float(s[c + x]), __uint_as_float(s[c + 4 + x]));
+#pragma unroll
+  for (int x = 0; x < 4; ++x) mx4[x] = fmaxf(mx4[x], __uint_as_float(s[kPrefillBN - 4 + x]));
+  const float tmax = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
+  const float mx = tmax * sl2;
+  row.seen |= tmax != -INFINITY;
+  // The first tile sets the max exactly (the row's largest P is then 1
+  // unless the sink is larger); later tiles raise it only when it grows by
+  // more than 2^8, and then O is rescaled in TMEM. The previous P V of this
+  // tile has completed: it was issued before this S. tcgen05.ld/st are
+  // warp-collective, so the warp rescales together, each thread with its own
+  // factor (1 if unchanged).
+  float alpha = 1.f;
+  const bool grow = (j == 0) ? (mx > row.m_run) : (mx > row.m_run + kRescaleThreshold);
+  if (grow) {
+    if (j > 0 && row.m_run != -INFINITY) alpha = ex2(row.m_run - mx);
+    row.m_run = mx;
+    row.l_run *= alpha;
+    row.l_rnd *= alpha;
+  }
+  if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+    const uint64_t a2 = f2pack(alpha, alpha);
+#pragma unroll
+    for (int c = 0; c < D; c += 32) {
+      uint32_t o[32];
+      tmem_load<32>(o_tmem + c, o);
+#pragma unroll
+      for (int x = 0; x < 32; x += 2) {
+        const uint64_t v = mul2(f2pack(__uint_as_float(o[x]), __uint_as_float(o[x + 1])), a2);
+        float a, b;
+        f2unpack(v, a, b);
+        o[x] = __float_as_uint(a);
+        o[x + 1] = __float_as_uint(b);
+      }
+      tmem_store<32>(o_tmem + c, o);
+    }
+  }
+  const float m_use = (row.m_run == -INFINITY) ? 0.f : row.m_run;
+  const uint64_t negm = f2pack(-m_use, -m_use);
+  const uint64_t sl2x2 = f2pack(sl2, sl2);
+  // P rounded to the MMA's input type (to nearest even), written over S 32
+  // keys (16 packed words) at a time. O is normalised by the sum of the
+  // rounded P the MMA consumes (the weights then stay a convex combination
+  // and the rounding error scales with the spread of V, not with |O|); the
+  // LSE uses the fp32 sum.
+  uint64_t acc_e[4];
+  float acc_r[4];
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    acc_e[x] = 0ull;
+    acc_r[x] = 0.f;
+  }
+#pragma unroll
+  for (int ch = 0; ch < kPrefillBN / 32; ++ch) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int e = ch * 32 + 2 * c;
+      const uint64_t arg =
+          fma2(f2pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2x2, negm);
+      float a0, a1;
+      f2unpack(arg, a0, a1);
+      float p0, p1;
+      if (c >= 16 - kEmuPairs) {
+        f2unpack(exp2_poly_x2(a0, a1), p0, p1);
+      } else {
+        p0 = ex2(a0);
+        p1 = ex2(a1);
+      }
+      acc_e[c & 3] = add2(acc_e[c & 3], f2pack(p0, p1));
+      pk[c] = pack2<kFp16>(p0, p1);
+      acc_packed<kFp16>(acc_r[c & 1], acc_r[2 + (c & 1)], pk[c]);
+    }
+    tmem_store<16>(s_tmem + ch * 16, pk);
+    if (ch == kSplitKeys / 32 - 1) {
+      // The head of P: the P V MMA starts on it.
+      tmem_store_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_head[w]);
+    }
+  }
+  {
+    const uint64_t e = add2(add2(acc_e[0], acc_e[1]), add2(acc_e[2], acc_e[3]));
+    float e0, e1;
+    f2unpack(e, e0, e1);
+    row.l_run += e0 + e1;
+    row.l_rnd += (acc_r[0] + acc_r[1]) + (acc_r[2] + acc_r[3]);
+  }
+  tmem_store_wait();
+  tc_fence_before();
+  mbar_arrive(&bars->p_full[w]);
+  return true;
+}
+
 template <int D, int kType>
 DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_t tmem, int w) {
   using C = PrefillCfg<D, kType>;
-  constexpr bool kFp16 = kType != 0;  // P in fp16 (fp16 and FP8 inputs)
   using OutT = typename std::conditional<kType == 1, __half, __nv_bfloat16>::type;
   volatile int* abort = &bars->abort;
   const int r = threadIdx.x & 127;
@@ -427,8 +587,6 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
       }
       continue;
     }
-    int lo_i, hi_i;
-    row_key_range(p, i, u.len_q, u.len_k, lo_i, hi_i);
     float sl2 = p.scale_log2;
     float v_scale = 1.f;
     if constexpr (C::kFp8) {
@@ -438,127 +596,17 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
       sl2 *= p.q_descale[dk] * p.k_descale[dk];
       v_scale = p.v_descale[dk];
     }
-    const uint64_t sl2x2 = f2pack(sl2, sl2);
     const bool has_sink = p.sink != nullptr;
     const float sink2 = has_sink ? p.sink[u.h] * kLog2e : -INFINITY;
-    float m_run = sink2;
-    float l_run = 0.f;  // sum of the fp32 P (for the LSE)
-    float l_rnd = 0.f;  // sum of the rounded P the MMA consumes (for O)
-    bool seen = false;  // some key of this row is visible
-
-    for (int j = 0; j < n; ++j, ++sj) {
-      if (!warp_wait(&bars->s_full[w], sj & 1, abort, 20 + w)) return;
-      tc_fence_after();
-      uint32_t s[kPrefillBN];
-      tmem_load128(s_tmem, s);
-      const int k0 = (u.kt0 + j) * kPrefillBN;
-      if (!(k0 >= lo_i && k0 + kPrefillBN - 1 <= hi_i)) {
-#pragma unroll
-        for (int c = 0; c < kPrefillBN; ++c) {
-          const bool vis = (k0 + c >= lo_i) && (k0 + c <= hi_i);
-          s[c] = vis ? s[c] : __float_as_uint(-INFINITY);
-        }
-      }
-      float mx8[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) mx8[x] = __uint_as_float(s[x]);
-#pragma unroll
-      for (int c = 8; c < kPrefillBN; c += 8)
-#pragma unroll
-        for (int x = 0; x < 8; ++x) mx8[x] = fmaxf(mx8[x], __uint_as_float(s[c + x]));
-      const float tmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float mx = tmax * sl2;
-      seen |= tmax != -INFINITY;
-      // The first tile sets the max exactly (the row's largest P is then 1
-      // unless the sink is larger); later tiles raise it only when it grows by
-      // more than 2^8, and then O is rescaled in TMEM. The previous P V of
-      // this tile has completed: it was issued before this S.
-      // tcgen05.ld/st are warp-collective, so the warp rescales together, each
-      // thread with its own factor (1 if unchanged).
-      float alpha = 1.f;
-      const bool grow = (j == 0) ? (mx > m_run) : (mx > m_run + kRescaleThreshold);
-      if (grow) {
-        if (j > 0 && m_run != -INFINITY) alpha = ex2(m_run - mx);
-        m_run = mx;
-        l_run *= alpha;
-        l_rnd *= alpha;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        const uint64_t a2 = f2pack(alpha, alpha);
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-          tmem_load<32>(o_tmem + c, o);
-#pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            const uint64_t v =
-                mul2(f2pack(__uint_as_float(o[x]), __uint_as_float(o[x + 1])), a2);
-            float a, b;
-            f2unpack(v, a, b);
-            o[x] = __float_as_uint(a);
-            o[x + 1] = __float_as_uint(b);
-          }
-          tmem_store<32>(o_tmem + c, o);
-        }
-      }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      const uint64_t negm = f2pack(-m_use, -m_use);
-      // P = 2^(s * scale * log2e - m), converted to the input type. O is
-      // normalised by the sum of the rounded P the MMA consumes (the weights
-      // then stay a convex combination and the rounding error scales with the
-      // spread of V, not with |O|); the LSE uses the fp32 sum.
-      // P is written to TMEM 32 columns (16 packed words) at a time, so only
-      // one chunk of packed values is live next to S.
-      uint64_t acc_e[4], acc_r[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) acc_e[x] = acc_r[x] = 0ull;
-#pragma unroll
-      for (int ch = 0; ch < kPrefillBN / 32; ++ch) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int e = ch * 32 + 2 * c;
-          const uint64_t arg =
-              fma2(f2pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2x2, negm);
-          float a0, a1;
-          f2unpack(arg, a0, a1);
-          float p0, p1;
-          if (c >= 16 - kEmuPairs) {
-            f2unpack(exp2_poly_x2(a0, a1), p0, p1);
-          } else {
-            p0 = ex2(a0);
-            p1 = ex2(a1);
-          }
-          acc_e[c & 3] = add2(acc_e[c & 3], f2pack(p0, p1));
-          if constexpr (kFp16) {
-            pk[c] = pack_f16x2(p0, p1);
-            acc_r[c & 3] = add2(acc_r[c & 3], widen2<true>(pk[c]));
-          } else {
-            // bf16 rounding on the integer pipe (P >= 0: add half an ulp of
-            // bf16, keep the top 16 bits: to nearest, ties away from zero).
-            const uint32_t r0 = __float_as_uint(p0) + 0x8000u;
-            const uint32_t r1 = __float_as_uint(p1) + 0x8000u;
-            pk[c] = __byte_perm(r0, r1, 0x7632);
-            acc_r[c & 3] = add2(acc_r[c & 3], f2pack(__uint_as_float(r0 & 0xffff0000u),
-                                                     __uint_as_float(r1 & 0xffff0000u)));
-          }
-        }
-        tmem_store<16>(s_tmem + ch * 16, pk);
-      }
-      {
-        const uint64_t e = add2(add2(acc_e[0], acc_e[1]), add2(acc_e[2], acc_e[3]));
-        const uint64_t q = add2(add2(acc_r[0], acc_r[1]), add2(acc_r[2], acc_r[3]));
-        float e0, e1, q0, q1;
-        f2unpack(e, e0, e1);
-        f2unpack(q, q0, q1);
-        l_run += e0 + e1;
-        l_rnd += q0 + q1;
-      }
-      tmem_store_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[w]);
-    }
+    PrefillRow row;
+    row_key_range(p, i, u.len_q, u.len_k, row.lo, row.hi);
+    row.m_run = sink2;
+    row.l_run = row.l_rnd = 0.f;
+    row.seen = false;
+    for (int j = 0; j < n; ++j, ++sj)
+      if (!prefill_softmax_tile<D, kType>(bars, s_tmem, o_tmem, w, j, sj,
+                                          (u.kt0 + j) * kPrefillBN, sl2, row))
+        return;
     // Epilogue: wait for the last P V, read O, release O, normalise, store.
     if (!warp_wait(&bars->o_full[w], units & 1, abort, 22 + w)) return;
     ++units;
@@ -574,10 +622,10 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
     mbar_arrive(&bars->o_empty[w]);
     // A row that saw no key: O = 0, LSE = -inf (polynomial exponentials of
     // masked scores are tiny but not 0, so the sums alone cannot tell).
-    if (!seen) l_run = l_rnd = 0.f;
-    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-    const float denom = l_rnd + (has_sink ? ex2(sink2 - m_use) : 0.f);
-    const float inv = (denom > 0.f && seen) ? v_scale / denom : 0.f;
+    if (!row.seen) row.l_run = row.l_rnd = 0.f;
+    const float m_use = (row.m_run == -INFINITY) ? 0.f : row.m_run;
+    const float denom = row.l_rnd + (has_sink ? ex2(sink2 - m_use) : 0.f);
+    const float inv = (denom > 0.f && row.seen) ? v_scale / denom : 0.f;
     if (valid) {
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
@@ -589,7 +637,7 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
         v.w = pack2<kOutF16>(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
         reinterpret_cast<uint4*>(orow)[c] = v;
       }
-      if (lrow) *lrow = l_run > 0.f ? (m_use + log2f(l_run)) * kLn2 : -INFINITY;
+      if (lrow) *lrow = row.l_run > 0.f ? (m_use + log2f(row.l_run)) * kLn2 : -INFINITY;
     }
   }
 }
@@ -600,9 +648,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                    const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
   using C = PrefillCfg<D, kType>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 128-byte swizzled TMA tiles need 1024-byte aligned shared memory. The
+  // layout leaves no slack for aligning at run time (the tiles take 224 KB),
+  // so a misaligned base is reported and the CTA exits before any barrier.
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) raise_error(ATTN_DEVERR_SMEM_ALIGN, 1);
+    return;
+  }
   PrefillBarriers* bars = reinterpret_cast<PrefillBarriers*>(smem + C::kBarOff);
   const int warp = threadIdx.x >> 5;
 
@@ -623,6 +676,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&bars->s_full[w], 1);
+      mbar_init(&bars->p_head[w], 128);
       mbar_init(&bars->p_full[w], 128);
       mbar_init(&bars->o_full[w], 1);
       mbar_init(&bars->o_empty[w], 128);

@@ -69,7 +69,8 @@ typedef enum {
 enum {
   ATTN_DEVERR_NONE = 0,
   ATTN_DEVERR_TIMEOUT = 1,        /* a bounded pipeline wait gave up            */
-  ATTN_DEVERR_META_MISMATCH = 2   /* scheduler metadata built for other args    */
+  ATTN_DEVERR_META_MISMATCH = 2,  /* scheduler metadata built for other args    */
+  ATTN_DEVERR_SMEM_ALIGN = 3      /* dynamic shared memory not 1024-byte aligned */
 };
 
 typedef enum {
