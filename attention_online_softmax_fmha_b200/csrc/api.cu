@@ -101,9 +101,9 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   if (!encode_4d(&mq, a.q, dt, es, D, a.num_heads_q, rows_q, nb, a.q_stride_h, a.q_stride_s, qsb,
                  bx, 1, 128, 1) ||
       !encode_4d(&mk, a.k, dt, es, D, a.num_heads_kv, rows_k, nb, a.k_stride_h, a.k_stride_s, ksb,
-                 bx, 1, 128, 1) ||
+                 bx, 1, kPrefillBN, 1) ||
       !encode_4d(&mv, a.v, dt, es, D, a.num_heads_kv, rows_k, nb, a.v_stride_h, a.v_stride_s, vsb,
-                 bx, 1, 128, 1))
+                 bx, 1, kPrefillBN, 1))
     return ATTN_ERR_INVALID_ARG;
 
   PrefillParams p;

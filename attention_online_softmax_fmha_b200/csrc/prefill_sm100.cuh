@@ -75,8 +75,8 @@ static_assert(kSplitKeys % 32 == 0 && kSplitKeys > 0 && kSplitKeys < kPrefillBN,
               "split on a 32-key chunk");
 constexpr int kPrefillThreads = 384;
 constexpr int kPrefillLaunchRegs = 168;       // 65536 / 384, rounded down to 8
-constexpr int kPrefillSoftmaxRegs = 208;
-constexpr int kPrefillOtherRegs = 88;
+constexpr int kPrefillSoftmaxRegs = 216;
+constexpr int kPrefillOtherRegs = 72;
 static_assert(2 * 128 * kPrefillSoftmaxRegs + 128 * kPrefillOtherRegs <=
                   kPrefillThreads * kPrefillLaunchRegs,
               "register split exceeds the launch allocation");
@@ -437,19 +437,77 @@ struct PrefillRow {
   bool seen;    // some key of this row is visible
 };
 
+// P = 2^(s * scale * log2e - m) rounded to the MMA's input type (to nearest
+// even), written over S 32 keys (16 packed words) at a time, the head
+// released first; the row sums (kRnd: also the sum of the rounded P).
+template <int kType, bool kRnd>
+DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float sl2,
+                           const uint32_t* s, PrefillRow& row) {
+  constexpr bool kFp16 = kType != 0;  // P in fp16 (fp16 and FP8 inputs)
+  const float m_use = (row.m_run == -INFINITY) ? 0.f : row.m_run;
+  const uint64_t negm = f2pack(-m_use, -m_use);
+  const uint64_t sl2x2 = f2pack(sl2, sl2);
+  uint64_t acc_e[4];
+  float acc_r[4];
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    acc_e[x] = 0ull;
+    acc_r[x] = 0.f;
+  }
+#pragma unroll
+  for (int ch = 0; ch < kPrefillBN / 32; ++ch) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int e = ch * 32 + 2 * c;
+      const uint64_t arg =
+          fma2(f2pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2x2, negm);
+      float a0, a1;
+      f2unpack(arg, a0, a1);
+      float p0, p1;
+      if (c >= 16 - kEmuPairs) {
+        f2unpack(exp2_poly_x2(a0, a1), p0, p1);
+      } else {
+        p0 = ex2(a0);
+        p1 = ex2(a1);
+      }
+      acc_e[c & 3] = add2(acc_e[c & 3], f2pack(p0, p1));
+      pk[c] = pack2<kFp16>(p0, p1);
+      if constexpr (kRnd) acc_packed<kFp16>(acc_r[c & 1], acc_r[2 + (c & 1)], pk[c]);
+    }
+    tmem_store<16>(s_tmem + ch * 16, pk);
+    if (ch == kSplitKeys / 32 - 1) {
+      // The head of P: the P V MMA starts on it.
+      tmem_store_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_head[w]);
+    }
+  }
+  {
+    const uint64_t e = add2(add2(acc_e[0], acc_e[1]), add2(acc_e[2], acc_e[3]));
+    float e0, e1;
+    f2unpack(e, e0, e1);
+    row.l_run += e0 + e1;
+    row.l_rnd += kRnd ? (acc_r[0] + acc_r[1]) + (acc_r[2] + acc_r[3]) : e0 + e1;
+  }
+  tmem_store_wait();
+  tc_fence_before();
+  mbar_arrive(&bars->p_full[w]);
+}
+
 // One S tile of keys [k0, k0 + 128) of this thread's row: mask, row max,
 // lazy O rescale, P = 2^(s * scale * log2e - m) written over S (head first),
 // row sums. Returns false if a wait gave up.
 template <int D, int kType>
 DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t o_tmem, int w,
                                int j, int g, int k0, float sl2, PrefillRow& row) {
-  constexpr bool kFp16 = kType != 0;  // P in fp16 (fp16 and FP8 inputs)
   volatile int* abort = &bars->abort;
   if (!warp_wait(&bars->s_full[w], g & 1, abort, 20 + w)) return false;
   tc_fence_after();
   uint32_t s[kPrefillBN];
   tmem_load128(s_tmem, s);
-  if (!(k0 >= row.lo && k0 + kPrefillBN - 1 <= row.hi)) {
+  const bool partial = !(k0 >= row.lo && k0 + kPrefillBN - 1 <= row.hi);
+  if (partial) {
 #pragma unroll
     for (int c = 0; c < kPrefillBN; ++c) {
       const bool vis = (k0 + c >= row.lo) && (k0 + c <= row.hi);
@@ -502,60 +560,16 @@ DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t 
       tmem_store<32>(o_tmem + c, o);
     }
   }
-  const float m_use = (row.m_run == -INFINITY) ? 0.f : row.m_run;
-  const uint64_t negm = f2pack(-m_use, -m_use);
-  const uint64_t sl2x2 = f2pack(sl2, sl2);
-  // P rounded to the MMA's input type (to nearest even), written over S 32
-  // keys (16 packed words) at a time. O is normalised by the sum of the
-  // rounded P the MMA consumes (the weights then stay a convex combination
-  // and the rounding error scales with the spread of V, not with |O|); the
-  // LSE uses the fp32 sum.
-  uint64_t acc_e[4];
-  float acc_r[4];
-#pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    acc_e[x] = 0ull;
-    acc_r[x] = 0.f;
-  }
-#pragma unroll
-  for (int ch = 0; ch < kPrefillBN / 32; ++ch) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const int e = ch * 32 + 2 * c;
-      const uint64_t arg =
-          fma2(f2pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sl2x2, negm);
-      float a0, a1;
-      f2unpack(arg, a0, a1);
-      float p0, p1;
-      if (c >= 16 - kEmuPairs) {
-        f2unpack(exp2_poly_x2(a0, a1), p0, p1);
-      } else {
-        p0 = ex2(a0);
-        p1 = ex2(a1);
-      }
-      acc_e[c & 3] = add2(acc_e[c & 3], f2pack(p0, p1));
-      pk[c] = pack2<kFp16>(p0, p1);
-      acc_packed<kFp16>(acc_r[c & 1], acc_r[2 + (c & 1)], pk[c]);
-    }
-    tmem_store<16>(s_tmem + ch * 16, pk);
-    if (ch == kSplitKeys / 32 - 1) {
-      // The head of P: the P V MMA starts on it.
-      tmem_store_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->p_head[w]);
-    }
-  }
-  {
-    const uint64_t e = add2(add2(acc_e[0], acc_e[1]), add2(acc_e[2], acc_e[3]));
-    float e0, e1;
-    f2unpack(e, e0, e1);
-    row.l_run += e0 + e1;
-    row.l_rnd += (acc_r[0] + acc_r[1]) + (acc_r[2] + acc_r[3]);
-  }
-  tmem_store_wait();
-  tc_fence_before();
-  mbar_arrive(&bars->p_full[w]);
+  // O is normalised by the sum of the rounded P the MMA consumes (the
+  // weights then stay a convex combination and the rounding error scales
+  // with the spread of V, not with |O|); the LSE uses the fp32 sum. The
+  // difference matters only for rows with few visible keys, whose keys all
+  // lie in first or partially masked tiles; other tiles add their fp32 sum to
+  // both (their rounding errors average out over the row's many keys).
+  if (j == 0 || __any_sync(0xffffffffu, partial))
+    prefill_exp_tile<kType, true>(bars, s_tmem, w, sl2, s, row);
+  else
+    prefill_exp_tile<kType, false>(bars, s_tmem, w, sl2, s, row);
   return true;
 }
 
