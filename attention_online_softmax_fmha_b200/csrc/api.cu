@@ -228,7 +228,7 @@ attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int h
       ds.tokens_per_tile = mode == ATTN_SCHED_MLA_SPARSE ? 1 : kMlaRows / heads_q;
       ds.row_tiles = (seqlen_q + ds.tokens_per_tile - 1) / ds.tokens_per_tile;
     }
-    ds.sh.segs_per_seq = ds.row_tiles * 2;  // x two V halves
+    ds.sh.segs_per_seq = ds.row_tiles;  // both V halves: one cluster of two CTAs
     ds.sh.unit_keys = kMlaBN;
   }
   const int64_t S = (int64_t)batch * ds.sh.segs_per_seq;
@@ -236,6 +236,8 @@ attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int h
   ds.S = (int)S;
   ds.G = num_ctas > 0 ? num_ctas : device_sm_count();
   if (ds.G <= 0 || ds.G > 65536) return num_ctas < 0 ? ATTN_ERR_INVALID_ARG : ATTN_ERR_CUDA;
+  // MLA work goes to clusters of two CTAs: the scheduler's slots are clusters.
+  if (mode != ATTN_SCHED_MHA) ds.G = std::max(1, ds.G / 2);
   return ATTN_OK;
 }
 
@@ -370,9 +372,11 @@ attn_status_t check_mla(const mla_args* a, bool sparse) {
   return ATTN_OK;
 }
 
+// Split partials: per slot, both V halves of O (fp32) and the LSE.
 size_t mla_ws_bytes(const DecodeShape& ds) {
   const size_t slots = (size_t)ds.S + ds.G;
-  return slots * kMlaRows * kMlaDvHalf * sizeof(float) + slots * kMlaRows * sizeof(float) + 256;
+  return slots * 2 * kMlaRows * kMlaDvHalf * sizeof(float) + slots * kMlaRows * sizeof(float) +
+         256;
 }
 
 template <bool kSparse>
@@ -425,7 +429,7 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   if (a.meta) {
     const size_t slots = (size_t)ds.S + ds.G;
     p.ws_o = reinterpret_cast<float*>(a.workspace);
-    p.ws_lse = p.ws_o + slots * kMlaRows * kMlaDvHalf;
+    p.ws_lse = p.ws_o + slots * 2 * kMlaRows * kMlaDvHalf;
   }
   auto kernel = mla_kernel<kSparse>;
   static bool configured = false;
@@ -433,10 +437,12 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
     if (set_smem(kernel, kMlaSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
     configured = true;
   }
-  kernel<<<a.meta ? ds.G : ds.S, 192, kMlaSmemBytes, stream>>>(mq, mkv, p);
+  // Clusters of two CTAs (the kernel's __cluster_dims__): one per segment, or
+  // one per metadata slot.
+  kernel<<<2 * (a.meta ? ds.G : ds.S), 192, kMlaSmemBytes, stream>>>(mq, mkv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (a.meta) {
-    const int64_t warps = (int64_t)ds.S * kMlaRows;
+    const int64_t warps = (int64_t)ds.S * 2 * kMlaRows;
     mla_combine_kernel<kSparse><<<(int)((warps + 7) / 8), 256, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }

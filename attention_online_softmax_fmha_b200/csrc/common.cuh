@@ -401,6 +401,72 @@ DEVI void tmem_load64(uint32_t taddr, uint32_t* r) {
       : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Thread-block clusters: rank, distributed shared memory, remote mbarriers
+// ---------------------------------------------------------------------------
+DEVI uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared-memory offset in CTA `rank`.
+DEVI uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+DEVI void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b),
+               "r"(c), "r"(d)
+               : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster, ordering this thread's
+// earlier (distributed) shared-memory writes before the arrival.
+DEVI void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+DEVI bool mbar_test_cluster(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// As warp_wait, with cluster-scope acquire (the arrivals come from another
+// CTA of the cluster).
+DEVI bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
+  const uint32_t a = smem_u32(bar);
+  bool ok = mbar_test_cluster(a, parity);
+  if (!ok) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_test_cluster(a, parity)) {
+        ok = true;
+        break;
+      }
+      if ((it & 255u) == 0) {
+        if (*abort) break;
+        if (globaltimer() - t0 > kWaitTimeoutNs) {
+          raise_error(ATTN_DEVERR_TIMEOUT, site);
+          *abort = 1;
+          break;
+        }
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+// All threads of every CTA of the cluster.
+DEVI void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
 // Named barrier over `count` threads (a multiple of 32).
 DEVI void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

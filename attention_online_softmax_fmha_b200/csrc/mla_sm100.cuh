@@ -7,28 +7,34 @@
 // One KV head: every query row (token i, head h) scores against the whole
 // 576-wide cached row; V is the row's first 512 entries.
 //
-// Work decomposition. An fp32 accumulator for 128 query rows x 512 V columns
-// would fill all of TMEM, so a CTA owns 128 query rows and one half of the V
-// columns (256); the two halves of a row tile are separate segments (both
-// compute S = Q K^T). Segments are split over persistent CTAs by the
-// scheduler metadata; split segments go through the combine kernel.
-//   dense : segment = (sequence, 128-row tile of (token, head) rows, V half),
-//           keys 0 .. L-1 in tiles of 32 (causal: key j visible to token i iff
-//           j <= i + L - s_q).
-//   sparse: segment = (sequence, token, head tile, V half), keys = that
-//           token's listed positions in tiles of 32 entries; entries outside
-//           [0, L) are skipped.
+// Work decomposition. A cluster of two CTAs owns 128 query rows ("row tile")
+// and streams the keys once for both V halves: CTA rank r holds the score
+// dimensions of its V half (rank 0: nope 0..255 and the 64 rope dimensions,
+// rank 1: nope 256..511) of Q and of every key, computes the partial scores
+// S_r = Q_r K_r^T on its tensor core, and the two halves swap partials through
+// distributed shared memory, so both see S = S_0 + S_1 (the same sum in the
+// same order: identical P). Each CTA then accumulates O for its 256 V columns
+// (its first four 64-column chunks). Half of Q and of each key row per CTA
+// leaves room for a five-stage key ring, and the cache is read once per row
+// tile instead of once per V half.
+//   dense : segment = (sequence, row tile), keys 0 .. L-1 in tiles of 32
+//           (causal: key j visible to token i iff j <= i + L - s_q).
+//   sparse: segment = (sequence, token, head tile), keys = that token's
+//           listed positions in tiles of 32 entries; entries outside [0, L)
+//           are skipped.
+// Segments are split over persistent clusters by the scheduler metadata (a
+// metadata "CTA" is a cluster); split segments go through the combine kernel.
 //
-// Roles (192 threads):
+// Roles (192 threads per CTA):
 //   warps 0-3  softmax: thread r owns query row r (= TMEM lane r).
-//   warp 4     producer: Q tile (TMA, 144 KB resident), K/V tiles of 32
-//              keys x 576 into a 2-stage ring: dense by TMA boxes through the
-//              block table; sparse by per-lane 16-byte async copies of the
-//              gathered rows (each lane one key, zeros for skipped keys),
-//              completed and fenced before the stage is handed over.
+//   warp 4     producer: Q tile (TMA, resident), key tiles of 32 keys into a
+//              5-stage ring: dense by TMA boxes through the block table;
+//              sparse by per-lane 16-byte async copies of the gathered rows
+//              (each lane one key, zeros for skipped keys), completed and
+//              fenced before the stage is handed over.
 //   warp 5     TMEM owner and MMA issuer (whole warp, one elected lane):
-//              S_j = Q K_j^T (M=128, N=32, K=576) into one of two TMEM S
-//              buffers; O += P_j V_j (M=128, N=256, K=32) with P from TMEM.
+//              S_j = Q K_j^T (M=128, N=32) into one of two TMEM S buffers;
+//              O += P_j V_j (M=128, N=256, K=32) with P from TMEM.
 #pragma once
 
 #include "combine.cuh"
@@ -41,20 +47,27 @@ constexpr int kMlaDqk = 576;
 constexpr int kMlaDv = 512;
 constexpr int kMlaDvHalf = 256;
 constexpr int kMlaBN = 32;         // keys per tile
-constexpr int kMlaRows = 128;      // query rows per CTA
-constexpr int kMlaStages = 2;
-constexpr int kMlaChunks = kMlaDqk / 64;                       // 9 column chunks
+constexpr int kMlaRows = 128;      // query rows per row tile
+constexpr int kMlaStages = 5;
+constexpr int kMlaMaxChunks = 5;   // 64-column chunks per CTA (rank 0: 5, rank 1: 4)
 constexpr int kMlaQChunkBytes = kMlaRows * 128;                // 16 KB
 constexpr int kMlaKVChunkBytes = kMlaBN * 128;                 // 4 KB
-constexpr int kMlaQBytes = kMlaChunks * kMlaQChunkBytes;       // 144 KB
-constexpr int kMlaKVBytes = kMlaChunks * kMlaKVChunkBytes;     // 36 KB
+constexpr int kMlaQBytes = kMlaMaxChunks * kMlaQChunkBytes;    // 80 KB
+constexpr int kMlaKVBytes = kMlaMaxChunks * kMlaKVChunkBytes;  // 20 KB
+constexpr int kMlaXsBytes = kMlaRows * kMlaBN * 4;             // one partial S tile, 16 KB
 constexpr int kMlaQOff = 0;
-constexpr int kMlaKVOff = kMlaQBytes;
+constexpr int kMlaXsOff = kMlaQOff + kMlaQBytes;               // two partial-S buffers
+constexpr int kMlaKVOff = kMlaXsOff + 2 * kMlaXsBytes;
 constexpr int kMlaBarOff = kMlaKVOff + kMlaStages * kMlaKVBytes;
-constexpr int kMlaSmemBytes = kMlaBarOff + 256 + 1024;
+constexpr int kMlaSmemBytes = kMlaBarOff + 256;
+static_assert(kMlaSmemBytes <= 232448, "shared memory per CTA");
 constexpr uint32_t kMlaTmemCols = 512;
 constexpr uint32_t kMlaTmemS = 0;      // two S buffers of 32 columns
 constexpr uint32_t kMlaTmemO = 256;    // 256 columns of O
+
+// Global 64-column chunk of the 576-wide row held in local chunk c of rank r.
+DEVI int mla_chunk(int rank, int c) { return rank == 0 ? (c < 4 ? c : 8) : 4 + c; }
+DEVI int mla_nchunks(int rank) { return rank == 0 ? 5 : 4; }
 
 struct MlaParams {
   const void* q;
@@ -64,7 +77,7 @@ struct MlaParams {
   const int32_t* cache_seqlens;
   const int32_t* indices;
   const int32_t* meta;
-  float* ws_o;    // [slot][128][256]
+  float* ws_o;    // [slot][V half][128][256]
   float* ws_lse;  // [slot][128]
   const __nv_bfloat16* kv;
   int64_t bt_stride;
@@ -76,7 +89,7 @@ struct MlaParams {
   int32_t tiles_per_token;  // heads_q >= 128: heads_q / 128 (else 1)
   int32_t tokens_per_tile;  // heads_q < 128: 128 / heads_q (else 1)
   int32_t row_tiles;        // dense: row tiles per sequence
-  int32_t segs_per_seq, num_segs, num_ctas;
+  int32_t segs_per_seq, num_segs, num_ctas;  // num_ctas: clusters (metadata slots)
   float scale_log2;
   int32_t causal;
 };
@@ -85,15 +98,17 @@ struct MlaBarriers {
   uint64_t q_full, q_empty;
   uint64_t kv_full[kMlaStages], kv_empty[kMlaStages];
   uint64_t s_full[2], p_full[2];
+  uint64_t xs_full[2];  // the other CTA's partial S tile has landed here
   uint64_t o_full, o_empty;
   uint64_t mma_drain;
   uint32_t tmem_base;
   int32_t abort;
 };
+static_assert(sizeof(MlaBarriers) <= 256, "barrier block");
 
 // A segment and its rows.
 struct MlaSeg {
-  int b, vh, len;
+  int b, len;
   int tok0, head0;   // first (token, head) of the row tile
   int rows_valid;    // rows of the tile that exist (the rest are padding)
   int units;         // KV tiles of the segment
@@ -102,9 +117,7 @@ struct MlaSeg {
 template <bool kSparse>
 DEVI void mla_seg(const MlaParams& p, int s, MlaSeg& g) {
   g.b = s / p.segs_per_seq;
-  const int rem = s - g.b * p.segs_per_seq;
-  g.vh = rem & 1;
-  const int rt = rem >> 1;  // row tile index within the sequence
+  const int rt = s - g.b * p.segs_per_seq;  // row tile index within the sequence
   g.len = p.cache_seqlens[g.b];
   if (p.heads_q >= kMlaRows) {
     g.tok0 = rt / p.tiles_per_token;
@@ -132,20 +145,21 @@ DEVI void mla_row(const MlaParams& p, const MlaSeg& g, int x, int& tok, int& hea
   }
 }
 
-// The CTA's unit range [ub, ue) and first segment (metadata or one segment
-// per CTA).
+// The cluster's unit range [ub, ue) and first segment (metadata, or one
+// segment per cluster).
 template <bool kSparse>
 DEVI void mla_range(const MlaParams& p, int& ub, int& ue, int& s0, const int32_t*& prefix) {
+  const int cl = blockIdx.x >> 1;
   if (p.meta) {
     const MetaLayout ml(p.num_ctas, p.num_segs);
-    ub = p.meta[ml.cta_begin + blockIdx.x];
-    ue = p.meta[ml.cta_begin + blockIdx.x + 1];
-    s0 = p.meta[ml.cta_seg + blockIdx.x];
+    ub = p.meta[ml.cta_begin + cl];
+    ue = p.meta[ml.cta_begin + cl + 1];
+    s0 = p.meta[ml.cta_seg + cl];
     prefix = p.meta + ml.seg_begin;
   } else {
     MlaSeg g;
-    mla_seg<kSparse>(p, blockIdx.x, g);
-    s0 = blockIdx.x;
+    mla_seg<kSparse>(p, cl, g);
+    s0 = cl;
     ub = 0;
     ue = g.units;  // an empty sequence: the softmax warps write O = 0, LSE = -inf
     prefix = nullptr;
@@ -157,9 +171,10 @@ DEVI void mla_range(const MlaParams& p, int& ub, int& ue, int& s0, const int32_t
 // ---------------------------------------------------------------------------
 template <bool kSparse>
 DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensorMap* mkv,
-                       uint8_t* smem, MlaBarriers* bars) {
+                       uint8_t* smem, MlaBarriers* bars, int rank) {
   volatile int* abort = &bars->abort;
   const int lane = threadIdx.x & 31;
+  const int nch = mla_nchunks(rank);
   if (lane == 0) {
     tma_prefetch_desc(mq);
     if (!kSparse) tma_prefetch_desc(mkv);
@@ -188,15 +203,15 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       ++s;
       continue;
     }
-    // Q tile of the segment
+    // Q tile of the segment: this CTA's chunks of the 576 columns
     if (lane == 0) {
       bool ok = nq == 0 || mbar_wait(&bars->q_empty, (nq - 1) & 1, abort, 60);
       if (ok) {
         const int box_rows = p.heads_q >= kMlaRows ? kMlaRows : p.heads_q * (kSparse ? 1 : p.tokens_per_tile);
-        mbar_expect_tx(&bars->q_full, kMlaChunks * box_rows * 128);
-        for (int c = 0; c < kMlaChunks; ++c)
-          tma_load_4d(smem + kMlaQOff + c * kMlaQChunkBytes, mq, &bars->q_full, c * 64, g.head0,
-                      g.tok0, g.b);
+        mbar_expect_tx(&bars->q_full, nch * box_rows * 128);
+        for (int c = 0; c < nch; ++c)
+          tma_load_4d(smem + kMlaQOff + c * kMlaQChunkBytes, mq, &bars->q_full,
+                      mla_chunk(rank, c) * 64, g.head0, g.tok0, g.b);
       }
     }
     if (!__shfl_sync(0xffffffffu, (int)(*abort == 0), 0)) return;
@@ -219,18 +234,18 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
         int page = 0;
         if (lane < nload) page = bt[key0 / P + lane];
         if (lane == 0) {
-          mbar_expect_tx(&bars->kv_full[st], kMlaChunks * nload * box * 128);
+          mbar_expect_tx(&bars->kv_full[st], nch * nload * box * 128);
         }
         for (int j = 0; j < nload; ++j) {
           const int pg = __shfl_sync(0xffffffffu, page, j);
           if (lane == 0)
-            for (int c = 0; c < kMlaChunks; ++c)
+            for (int c = 0; c < nch; ++c)
               tma_load_4d(dst + c * kMlaKVChunkBytes + j * box * 128, mkv, &bars->kv_full[st],
-                          c * 64, key0 % P, pg, 0);
+                          mla_chunk(rank, c) * 64, key0 % P, pg, 0);
         }
       } else {
-        // lane k gathers key t*32 + k: 72 async copies of 16 bytes into the
-        // 128-byte-swizzled layout, or zeros if the entry is skipped.
+        // lane k gathers key t*32 + k: 8 async copies of 16 bytes per chunk
+        // into the 128-byte-swizzled layout, or zeros if the entry is skipped.
         const int e_idx = t * kMlaBN + lane;
         int pos = -1;
         if (e_idx < p.topk) pos = p.indices[g.b * p.idx_sb + g.tok0 * p.idx_ss + e_idx];
@@ -238,13 +253,14 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
         const __nv_bfloat16* src = nullptr;
         if (valid) src = p.kv + (int64_t)bt[pos / P] * p.kv_sblk + (int64_t)(pos % P) * p.kv_stok;
         const uint32_t dbase = smem_u32(dst) + lane * 128;
-        for (int c = 0; c < kMlaChunks; ++c) {
+        for (int c = 0; c < nch; ++c) {
+          const int gc = mla_chunk(rank, c);
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
             const uint32_t d = dbase + c * kMlaKVChunkBytes + ((x ^ (lane & 7)) << 4);
             if (valid) {
               asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d),
-                           "l"(src + c * 64 + x * 8)
+                           "l"(src + gc * 64 + x * 8)
                            : "memory");
             } else {
               asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(d), "r"(0) : "memory");
@@ -252,10 +268,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
           }
         }
         // Wait for this lane's copies, make them visible to the tensor core
-        // (async proxy) and signal the stage. (With two stages the stage must
-        // be complete before the next one is claimed: releasing stage s needs
-        // the P V two tiles back, which the MMA issues after the S of the
-        // tile loaded here.)
+        // (async proxy) and signal the stage.
         asm volatile("cp.async.commit_group;" ::: "memory");
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         fence_proxy_async_smem();
@@ -282,14 +295,15 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
 // MMA warp (whole warp; one elected lane issues)
 // ---------------------------------------------------------------------------
 template <bool kSparse>
-DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem) {
+DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem, int rank) {
   volatile int* abort = &bars->abort;
+  const int nk = mla_nchunks(rank) * 4;  // 16-column K steps of the partial score
   constexpr uint32_t idesc_s = make_idesc(128, kMlaBN, 1, 0, 0);
   constexpr uint32_t idesc_pv = make_idesc(128, kMlaDvHalf, 1, 0, 1);
   const uint64_t dq = sdesc_sw128(smem_u32(smem + kMlaQOff), 16, 1024);
   const uint64_t dkv = sdesc_sw128(smem_u32(smem + kMlaKVOff), 16, 1024);
-  // V half vh: chunks 4vh .. 4vh+3 of the KV tile, MN-major (leading byte
-  // offset = chunk stride, stride byte offset = 8 keys x 128 bytes).
+  // This CTA's V half: local chunks 0..3 of the key tile, MN-major (leading
+  // byte offset = chunk stride, stride byte offset = 8 keys x 128 bytes).
   const uint64_t dv = sdesc_sw128(smem_u32(smem + kMlaKVOff), kMlaKVChunkBytes, 1024);
   int ub, ue, s;
   const int32_t* prefix;
@@ -327,8 +341,8 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
         // before this in the in-order tensor pipe)
         const uint32_t sbuf = tmem + kMlaTmemS + (gi & 1) * kMlaBN;
         const uint64_t kst = dkv + st * (kMlaKVBytes >> 4);
-#pragma unroll
-        for (int k = 0; k < kMlaDqk / 16; ++k) {
+#pragma unroll 4
+        for (int k = 0; k < nk; ++k) {
           const uint32_t qo = (k >> 2) * (kMlaQChunkBytes >> 4) + (k & 3) * 2;
           const uint32_t ko = (k >> 2) * (kMlaKVChunkBytes >> 4) + (k & 3) * 2;
           mma_f16_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
@@ -343,7 +357,7 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
           goto drain;
         tc_fence_after();
         const uint32_t pbuf = tmem + kMlaTmemS + (gp & 1) * kMlaBN;
-        const uint64_t vst = dv + sp * (kMlaKVBytes >> 4) + g.vh * 4 * (kMlaKVChunkBytes >> 4);
+        const uint64_t vst = dv + sp * (kMlaKVBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < kMlaBN / 16; ++kk)
           mma_f16_ts_w(tmem + kMlaTmemO, pbuf + kk * 8, vst + kk * (16 * 128 >> 4), idesc_pv,
@@ -368,7 +382,8 @@ drain : {
 // Softmax warpgroup
 // ---------------------------------------------------------------------------
 template <bool kSparse>
-DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem) {
+DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem,
+                      int rank) {
   volatile int* abort = &bars->abort;
   const int r = threadIdx.x;  // 0..127
   const uint32_t lane = (uint32_t)(r & ~31) << 16;
@@ -377,20 +392,20 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
   int ub, ue, s;
   const int32_t* prefix;
   mla_range<kSparse>(p, ub, ue, s, prefix);
-  int it = 0, pv = 0;
+  int it = 0;
   const float sl2 = p.scale_log2;
   if (!p.meta && ue == 0) {
     // empty sequence without metadata: O = 0, LSE = -inf
     MlaSeg g;
-    mla_seg<kSparse>(p, blockIdx.x, g);
+    mla_seg<kSparse>(p, blockIdx.x >> 1, g);
     int tok, head;
     mla_row(p, g, r, tok, head);
     if (r < g.rows_valid && tok < p.seqlen_q) {
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + g.b * p.o_sb +
-                            (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + g.vh * kMlaDvHalf;
+                            (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + rank * kMlaDvHalf;
       for (int c = 0; c < kMlaDvHalf; c += 8)
         *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-      if (p.lse && g.vh == 0) p.lse[((int64_t)g.b * p.heads_q + head) * p.seqlen_q + tok] = -INFINITY;
+      if (p.lse && rank == 0) p.lse[((int64_t)g.b * p.heads_q + head) * p.seqlen_q + tok] = -INFINITY;
     }
     return;
   }
@@ -425,6 +440,31 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       const uint32_t s_tmem = tmem + kMlaTmemS + (gi & 1) * kMlaBN + lane;
       uint32_t sv[kMlaBN];
       tmem_load<32>(s_tmem, sv);
+      {
+        // Swap the partial scores with the other CTA of the cluster: each
+        // row's 32 partials go to the other CTA's buffer (16-byte pieces
+        // permuted by row to spread the banks), then the other CTA's land
+        // here. Buffer b is written again two tiles later, by which time this
+        // CTA has read it (the other CTA needs this CTA's next partials first).
+        const int b = gi & 1;
+        const uint32_t mine = smem_u32(smem + kMlaXsOff + b * kMlaXsBytes) + r * 128;
+        const uint32_t theirs = mapa_shared(mine, rank ^ 1);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          st_cluster_v4(theirs + ((k ^ (r & 7)) << 4), sv[4 * k], sv[4 * k + 1], sv[4 * k + 2],
+                        sv[4 * k + 3]);
+        mbar_arrive_remote(mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1));
+        if (!warp_wait_cluster(&bars->xs_full[b], (gi >> 1) & 1, abort, 83)) return;
+        const uint8_t* src = smem + kMlaXsOff + b * kMlaXsBytes + r * 128;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + ((k ^ (r & 7)) << 4));
+          sv[4 * k] = __float_as_uint(__uint_as_float(sv[4 * k]) + __uint_as_float(v.x));
+          sv[4 * k + 1] = __float_as_uint(__uint_as_float(sv[4 * k + 1]) + __uint_as_float(v.y));
+          sv[4 * k + 2] = __float_as_uint(__uint_as_float(sv[4 * k + 2]) + __uint_as_float(v.z));
+          sv[4 * k + 3] = __float_as_uint(__uint_as_float(sv[4 * k + 3]) + __uint_as_float(v.w));
+        }
+      }
       if constexpr (kSparse) {
         const int* idx = p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss + t * kMlaBN;
 #pragma unroll
@@ -449,7 +489,7 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
           for (int x = r; x < 4 * bad * 8; x += 128) {
             const int c = x / (bad * 8), rem = x % (bad * 8);
             const int row = nvalid + rem / 8, u16 = rem % 8;
-            *reinterpret_cast<uint4*>(kvs + (g.vh * 4 + c) * kMlaKVChunkBytes + row * 128 +
+            *reinterpret_cast<uint4*>(kvs + c * kMlaKVChunkBytes + row * 128 +
                                       u16 * 16) = make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
@@ -460,13 +500,6 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       for (int c = 0; c < kMlaBN; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
       seen |= mx != -INFINITY;
       mx *= sl2;
-      // P V of the previous tile must be complete before O may be rescaled
-      // (waited at every tile so the barrier phases stay in step).
-      if (j > 0) {
-        if (!warp_wait(&bars->o_full, pv & 1, abort, 81)) return;
-        ++pv;
-        tc_fence_after();
-      }
       float alpha = 1.f;
       const bool grow = (j == 0) ? (mx > m_run) : (mx > m_run + kRescaleThreshold);
       if (grow) {
@@ -476,6 +509,12 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
         l_rnd *= alpha;
       }
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O may be rescaled once P V of the previous tile (global index
+        // gi - 1) has landed. o_full completes once per P V; P V gi - 2 has
+        // completed (S gi was issued after it) and P V gi is issued only after
+        // this tile's P, so the barrier is at most this one phase behind.
+        if (!warp_wait(&bars->o_full, (gi - 1) & 1, abort, 81)) return;
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < kMlaDvHalf; c += 32) {
           uint32_t o[32];
@@ -512,11 +551,11 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     int slot = -1;
     if (p.meta && n > 0) {
       const int ns = p.meta[ml.seg_nsplit + s];
-      if (ns > 1) slot = p.meta[ml.seg_slot + s] + (blockIdx.x - p.meta[ml.seg_first + s]);
+      if (ns > 1) slot = p.meta[ml.seg_slot + s] + ((blockIdx.x >> 1) - p.meta[ml.seg_first + s]);
     }
     if (n > 0) {
-      if (!warp_wait(&bars->o_full, pv & 1, abort, 82)) return;
-      ++pv;
+      // the segment's last P V (global index it + n - 1; it now counts it)
+      if (!warp_wait(&bars->o_full, (it - 1) & 1, abort, 82)) return;
       tc_fence_after();
     }
     if (!seen) l_run = l_rnd = 0.f;
@@ -524,8 +563,9 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     const float inv = (l_rnd > 0.f && seen) ? 1.f / l_rnd : 0.f;
     const float lse = (l_run > 0.f && seen) ? (m_use + log2f(l_run)) * kLn2 : -INFINITY;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + g.b * p.o_sb +
-                          (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + g.vh * kMlaDvHalf;
-    float* wrow = slot >= 0 ? p.ws_o + ((int64_t)slot * kMlaRows + r) * kMlaDvHalf : nullptr;
+                          (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + rank * kMlaDvHalf;
+    float* wrow =
+        slot >= 0 ? p.ws_o + (((int64_t)slot * 2 + rank) * kMlaRows + r) * kMlaDvHalf : nullptr;
 #pragma unroll 1
     for (int c = 0; c < kMlaDvHalf; c += 32) {
       uint32_t o[32];
@@ -560,9 +600,9 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       mbar_arrive(&bars->o_empty);
     }
     if (valid_row) {
-      if (slot >= 0)
-        p.ws_lse[(int64_t)slot * kMlaRows + r] = lse;
-      else if (p.lse && g.vh == 0)
+      if (slot >= 0) {
+        if (rank == 0) p.ws_lse[(int64_t)slot * kMlaRows + r] = lse;
+      } else if (p.lse && rank == 0)
         p.lse[((int64_t)g.b * p.heads_q + head) * p.seqlen_q + tok] = lse;
     }
     u = min(ue, se);
@@ -571,14 +611,19 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
 }
 
 template <bool kSparse>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     mla_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
                const MlaParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 128-byte swizzled TMA tiles need 1024-byte aligned shared memory; both
+  // CTAs of the cluster share the layout, so both leave here or neither.
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) raise_error(ATTN_DEVERR_SMEM_ALIGN, 2);
+    return;
+  }
   MlaBarriers* bars = reinterpret_cast<MlaBarriers*>(smem + kMlaBarOff);
   const int warp = threadIdx.x >> 5;
+  const int rank = (int)cluster_ctarank();
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
@@ -589,6 +634,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->xs_full[i], 128);  // the other CTA's 128 softmax threads
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_empty, 128);
@@ -616,29 +662,34 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The other CTA's barriers are initialised before any remote arrival.
+  cluster_sync();
   const uint32_t tmem = bars->tmem_base;
   if (!s_bad) {
     if (warp < 4)
-      mla_softmax<kSparse>(p, smem, bars, tmem);
+      mla_softmax<kSparse>(p, smem, bars, tmem, rank);
     else if (warp == 4)
-      mla_producer<kSparse>(p, &map_q, &map_kv, smem, bars);
+      mla_producer<kSparse>(p, &map_q, &map_kv, smem, bars, rank);
     else
-      mla_mma<kSparse>(p, smem, bars, tmem);
+      mla_mma<kSparse>(p, smem, bars, tmem, rank);
   }
   tc_fence_before();
   __syncthreads();
+  // No remote arrival or store into this CTA's shared memory after this.
+  cluster_sync();
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, kMlaTmemCols);
   }
 }
 
-// Merges split MLA segments: one warp per (segment, row); each segment covers
-// 256 of the 512 output columns (its V half); the V-half-0 segment writes LSE.
+// Merges split MLA segments: one warp per (segment, V half, row); each half
+// covers 256 of the 512 output columns; half 0 writes the LSE.
 template <bool kSparse>
 __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int s = gw / kMlaRows, r = gw % kMlaRows;
+  const int s = gw / (2 * kMlaRows);
+  const int vh = (gw / kMlaRows) & 1, r = gw % kMlaRows;
   if (s >= p.num_segs) return;
   const int mode = kSparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
   if (!(meta_matches(p.meta, mode, p.batch, p.seqlen_q, p.heads_q, 1, p.page_size, p.num_segs,
@@ -655,13 +706,13 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
   if (r >= g.rows_valid || tok >= p.seqlen_q) return;
   const int slot0 = ns > 1 ? p.meta[ml.seg_slot + s] : 0;
   __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + g.b * p.o_sb +
-                       (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + g.vh * kMlaDvHalf;
+                       (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + vh * kMlaDvHalf;
   const float lse = combine_row(
       ns, kMlaDvHalf, 0.f, false,
       [&](int k) { return p.ws_lse[(int64_t)(slot0 + k) * kMlaRows + r]; },
-      [&](int k) { return p.ws_o + ((int64_t)(slot0 + k) * kMlaRows + r) * kMlaDvHalf; },
+      [&](int k) { return p.ws_o + (((int64_t)(slot0 + k) * 2 + vh) * kMlaRows + r) * kMlaDvHalf; },
       [&](int c, float v) { store_out(dst + c, v); });
-  if (p.lse && g.vh == 0 && (threadIdx.x & 31) == 0)
+  if (p.lse && vh == 0 && (threadIdx.x & 31) == 0)
     p.lse[((int64_t)g.b * p.heads_q + head) * p.seqlen_q + tok] = lse;
 }
 

@@ -154,7 +154,9 @@ attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream);
 /* step uses. One small kernel on `stream`.                                  */
 /* mode: ATTN_SCHED_MHA (attn_fwd_paged_kvcache), ATTN_SCHED_MLA             */
 /* (mla_fwd_paged), ATTN_SCHED_MLA_SPARSE (mla_sparse_fwd; uses topk).       */
-/* num_ctas = 0 picks the device's SM count.                                 */
+/* num_ctas = 0 picks the device's SM count. The MLA modes schedule over     */
+/* clusters of two CTAs: their slots number max(1, num_ctas / 2), and the    */
+/* MLA kernels launch two CTAs per slot.                                     */
 /* ------------------------------------------------------------------------ */
 enum { ATTN_SCHED_MHA = 0, ATTN_SCHED_MLA = 1, ATTN_SCHED_MLA_SPARSE = 2 };
 
