@@ -33,8 +33,9 @@
 //              (each lane one key, zeros for skipped keys), completed and
 //              fenced before the stage is handed over.
 //   warp 5     TMEM owner and MMA issuer (whole warp, one elected lane):
-//              S_j = Q K_j^T (M=128, N=32) into one of two TMEM S buffers;
-//              O += P_j V_j (M=128, N=256, K=32) with P from TMEM.
+//              S_j = Q K_j^T (M=128, N=32) into one of three TMEM S buffers
+//              (issued three tiles ahead); O += P_j V_j (M=128, N=256, K=32)
+//              with P from TMEM.
 #pragma once
 
 #include "combine.cuh"
@@ -49,6 +50,8 @@ constexpr int kMlaDvHalf = 256;
 constexpr int kMlaBN = 32;         // keys per tile
 constexpr int kMlaRows = 128;      // query rows per row tile
 constexpr int kMlaStages = 5;
+constexpr int kMlaSBufs = 3;       // S buffers in TMEM
+constexpr int kMlaXsBufs = 2;      // partial-S exchange buffers in shared memory
 constexpr int kMlaMaxChunks = 5;   // 64-column chunks per CTA (rank 0: 5, rank 1: 4)
 constexpr int kMlaQChunkBytes = kMlaRows * 128;                // 16 KB
 constexpr int kMlaKVChunkBytes = kMlaBN * 128;                 // 4 KB
@@ -56,13 +59,13 @@ constexpr int kMlaQBytes = kMlaMaxChunks * kMlaQChunkBytes;    // 80 KB
 constexpr int kMlaKVBytes = kMlaMaxChunks * kMlaKVChunkBytes;  // 20 KB
 constexpr int kMlaXsBytes = kMlaRows * kMlaBN * 4;             // one partial S tile, 16 KB
 constexpr int kMlaQOff = 0;
-constexpr int kMlaXsOff = kMlaQOff + kMlaQBytes;               // two partial-S buffers
-constexpr int kMlaKVOff = kMlaXsOff + 2 * kMlaXsBytes;
+constexpr int kMlaXsOff = kMlaQOff + kMlaQBytes;               // partial-S buffers
+constexpr int kMlaKVOff = kMlaXsOff + kMlaXsBufs * kMlaXsBytes;
 constexpr int kMlaBarOff = kMlaKVOff + kMlaStages * kMlaKVBytes;
 constexpr int kMlaSmemBytes = kMlaBarOff + 256;
 static_assert(kMlaSmemBytes <= 232448, "shared memory per CTA");
 constexpr uint32_t kMlaTmemCols = 512;
-constexpr uint32_t kMlaTmemS = 0;      // two S buffers of 32 columns
+constexpr uint32_t kMlaTmemS = 0;      // three S buffers of 32 columns
 constexpr uint32_t kMlaTmemO = 256;    // 256 columns of O
 
 // Global 64-column chunk of the 576-wide row held in local chunk c of rank r.
@@ -97,8 +100,8 @@ struct MlaParams {
 struct MlaBarriers {
   uint64_t q_full, q_empty;
   uint64_t kv_full[kMlaStages], kv_empty[kMlaStages];
-  uint64_t s_full[2], p_full[2];
-  uint64_t xs_full[2];  // the other CTA's partial S tile has landed here
+  uint64_t s_full[kMlaSBufs], p_full[2];
+  uint64_t xs_full[kMlaXsBufs];  // the other CTA's partial S tile has landed here
   uint64_t o_full, o_empty;
   uint64_t mma_drain;
   uint32_t tmem_base;
@@ -294,11 +297,31 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
 // ---------------------------------------------------------------------------
 // MMA warp (whole warp; one elected lane issues)
 // ---------------------------------------------------------------------------
+// S of the tile with global index g (this CTA's partial scores): waits for
+// its key stage, writes S buffer g % 3; after the segment's last S, releases Q.
+DEVI bool mla_issue_s(MlaBarriers* bars, int g, uint64_t dq, uint64_t dkv, uint32_t tmem, int nk,
+                      bool last) {
+  constexpr uint32_t idesc_s = make_idesc(128, kMlaBN, 1, 0, 0);
+  const int st = g % kMlaStages;
+  if (!warp_wait(&bars->kv_full[st], (g / kMlaStages) & 1, &bars->abort, 71)) return false;
+  tc_fence_after();
+  const uint32_t sbuf = tmem + kMlaTmemS + (g % kMlaSBufs) * kMlaBN;
+  const uint64_t kst = dkv + st * (kMlaKVBytes >> 4);
+#pragma unroll 4
+  for (int k = 0; k < nk; ++k) {
+    const uint32_t qo = (k >> 2) * (kMlaQChunkBytes >> 4) + (k & 3) * 2;
+    const uint32_t ko = (k >> 2) * (kMlaKVChunkBytes >> 4) + (k & 3) * 2;
+    mma_f16_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
+  }
+  tc_commit_w(&bars->s_full[g % kMlaSBufs]);
+  if (last) tc_commit_w(&bars->q_empty);
+  return true;
+}
+
 template <bool kSparse>
 DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem, int rank) {
   volatile int* abort = &bars->abort;
   const int nk = mla_nchunks(rank) * 4;  // 16-column K steps of the partial score
-  constexpr uint32_t idesc_s = make_idesc(128, kMlaBN, 1, 0, 0);
   constexpr uint32_t idesc_pv = make_idesc(128, kMlaDvHalf, 1, 0, 1);
   const uint64_t dq = sdesc_sw128(smem_u32(smem + kMlaQOff), 16, 1024);
   const uint64_t dkv = sdesc_sw128(smem_u32(smem + kMlaKVOff), 16, 1024);
@@ -331,40 +354,29 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
     }
     if (!warp_wait(&bars->q_full, nq & 1, abort, 70)) goto drain;
     ++nq;
-    for (int j = 0; j <= n; ++j) {
-      const int gi = it + j;
-      const int st = gi % kMlaStages;
-      if (j < n) {
-        if (!warp_wait(&bars->kv_full[st], (gi / kMlaStages) & 1, abort, 71)) goto drain;
-        tc_fence_after();
-        // S_j into buffer gi & 1 (its previous P was read by PV_{j-2}, issued
-        // before this in the in-order tensor pipe)
-        const uint32_t sbuf = tmem + kMlaTmemS + (gi & 1) * kMlaBN;
-        const uint64_t kst = dkv + st * (kMlaKVBytes >> 4);
-#pragma unroll 4
-        for (int k = 0; k < nk; ++k) {
-          const uint32_t qo = (k >> 2) * (kMlaQChunkBytes >> 4) + (k & 3) * 2;
-          const uint32_t ko = (k >> 2) * (kMlaKVChunkBytes >> 4) + (k & 3) * 2;
-          mma_f16_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
-        }
-        tc_commit_w(&bars->s_full[gi & 1]);
-        if (j == n - 1) tc_commit_w(&bars->q_empty);
-      }
-      if (j > 0) {
-        const int gp = gi - 1, sp = gp % kMlaStages;
-        if (!warp_wait(&bars->p_full[gp & 1], (gp >> 1) & 1, abort, 72)) goto drain;
-        if (j == 1 && pieces > 0 && !warp_wait(&bars->o_empty, (pieces - 1) & 1, abort, 73))
-          goto drain;
-        tc_fence_after();
-        const uint32_t pbuf = tmem + kMlaTmemS + (gp & 1) * kMlaBN;
-        const uint64_t vst = dv + sp * (kMlaKVBytes >> 4);
+    // S of the first three tiles, then per tile g: PV_g, S_{g+3} (S_{g+3}
+    // reuses S_g's buffer, whose P the tensor core has read in PV_g just
+    // before: the pipe runs in order). The softmax thus finds S_{g+1} ready
+    // while it finishes tile g.
+    for (int j = 0; j < kMlaSBufs && j < n; ++j)
+      if (!mla_issue_s(bars, it + j, dq, dkv, tmem, nk, j == n - 1)) goto drain;
+    for (int j = 0; j < n; ++j) {
+      const int gi = it + j, sp = gi % kMlaStages;
+      if (!warp_wait(&bars->p_full[gi & 1], (gi >> 1) & 1, abort, 72)) goto drain;
+      if (j == 0 && pieces > 0 && !warp_wait(&bars->o_empty, (pieces - 1) & 1, abort, 73))
+        goto drain;
+      tc_fence_after();
+      const uint32_t pbuf = tmem + kMlaTmemS + (gi % kMlaSBufs) * kMlaBN;
+      const uint64_t vst = dv + sp * (kMlaKVBytes >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kMlaBN / 16; ++kk)
-          mma_f16_ts_w(tmem + kMlaTmemO, pbuf + kk * 8, vst + kk * (16 * 128 >> 4), idesc_pv,
-                       (j > 1 || kk > 0) ? 1u : 0u);
-        tc_commit_w(&bars->kv_empty[sp]);
-        tc_commit_w(&bars->o_full);  // the softmax waits for every P V in order
-      }
+      for (int kk = 0; kk < kMlaBN / 16; ++kk)
+        mma_f16_ts_w(tmem + kMlaTmemO, pbuf + kk * 8, vst + kk * (16 * 128 >> 4), idesc_pv,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+      tc_commit_w(&bars->kv_empty[sp]);
+      tc_commit_w(&bars->o_full);
+      if (j + kMlaSBufs < n &&
+          !mla_issue_s(bars, gi + kMlaSBufs, dq, dkv, tmem, nk, j + kMlaSBufs == n - 1))
+        goto drain;
     }
     it += n;
     ++pieces;
@@ -381,6 +393,29 @@ drain : {
 // ---------------------------------------------------------------------------
 // Softmax warpgroup
 // ---------------------------------------------------------------------------
+// Loads this CTA's partial scores of the tile with global index g into sv
+// and sends them to the other CTA of the cluster: 16-byte pieces permuted by
+// row (to spread the banks) into its buffer g % 2, then one arrival per row
+// on its barrier. This CTA sends tile g only after it has received the other
+// CTA's tile g - 1, which the other CTA sent after reading its tile g - 2
+// (the buffer's last use there), so the buffer is free; and the barrier is at
+// most one phase ahead of its waiter.
+DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint32_t lane, int r,
+                           int rank, int g, uint32_t* sv) {
+  const int sb = g % kMlaSBufs, b = g % kMlaXsBufs;
+  if (!warp_wait(&bars->s_full[sb], (g / kMlaSBufs) & 1, &bars->abort, 80)) return false;
+  tc_fence_after();
+  tmem_load<32>(tmem + kMlaTmemS + sb * kMlaBN + lane, sv);
+  const uint32_t mine = smem_u32(smem + kMlaXsOff + b * kMlaXsBytes) + r * 128;
+  const uint32_t theirs = mapa_shared(mine, rank ^ 1);
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    st_cluster_v4(theirs + ((k ^ (r & 7)) << 4), sv[4 * k], sv[4 * k + 1], sv[4 * k + 2],
+                  sv[4 * k + 3]);
+  mbar_arrive_remote(mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1));
+  return true;
+}
+
 template <bool kSparse>
 DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem,
                       int rank) {
@@ -432,29 +467,19 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     if (!kSparse && p.causal) hi = min(hi, tok + g.len - p.seqlen_q);
     float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
     bool seen = false;
+    // The partial scores of tile g + 1 go to the other CTA as soon as those of
+    // tile g have arrived here: they are in flight while tile g is
+    // exponentiated.
+    uint32_t sv[kMlaBN];
+    if (n > 0 && !mla_send_partial(bars, smem, tmem, lane, r, rank, it, sv)) return;
     for (int j = 0; j < n; ++j) {
       const int gi = it + j;
       const int t = a + j;
-      if (!warp_wait(&bars->s_full[gi & 1], (gi >> 1) & 1, abort, 80)) return;
-      tc_fence_after();
-      const uint32_t s_tmem = tmem + kMlaTmemS + (gi & 1) * kMlaBN + lane;
-      uint32_t sv[kMlaBN];
-      tmem_load<32>(s_tmem, sv);
+      uint32_t sv_next[kMlaBN];
       {
-        // Swap the partial scores with the other CTA of the cluster: each
-        // row's 32 partials go to the other CTA's buffer (16-byte pieces
-        // permuted by row to spread the banks), then the other CTA's land
-        // here. Buffer b is written again two tiles later, by which time this
-        // CTA has read it (the other CTA needs this CTA's next partials first).
-        const int b = gi & 1;
-        const uint32_t mine = smem_u32(smem + kMlaXsOff + b * kMlaXsBytes) + r * 128;
-        const uint32_t theirs = mapa_shared(mine, rank ^ 1);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          st_cluster_v4(theirs + ((k ^ (r & 7)) << 4), sv[4 * k], sv[4 * k + 1], sv[4 * k + 2],
-                        sv[4 * k + 3]);
-        mbar_arrive_remote(mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1));
-        if (!warp_wait_cluster(&bars->xs_full[b], (gi >> 1) & 1, abort, 83)) return;
+        // The other CTA's partials of this tile.
+        const int b = gi % kMlaXsBufs;
+        if (!warp_wait_cluster(&bars->xs_full[b], (gi / kMlaXsBufs) & 1, abort, 83)) return;
         const uint8_t* src = smem + kMlaXsOff + b * kMlaXsBytes + r * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -465,6 +490,7 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
           sv[4 * k + 3] = __float_as_uint(__uint_as_float(sv[4 * k + 3]) + __uint_as_float(v.w));
         }
       }
+      if (j + 1 < n && !mla_send_partial(bars, smem, tmem, lane, r, rank, gi + 1, sv_next)) return;
       if constexpr (kSparse) {
         const int* idx = p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss + t * kMlaBN;
 #pragma unroll
@@ -540,10 +566,12 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       }
       l_run += le;
       l_rnd += lr;
-      tmem_store<16>(s_tmem, pk);
+      tmem_store<16>(tmem + kMlaTmemS + (gi % kMlaSBufs) * kMlaBN + lane, pk);
       tmem_store_wait();
       tc_fence_before();
       mbar_arrive(&bars->p_full[gi & 1]);
+#pragma unroll
+      for (int c = 0; c < kMlaBN; ++c) sv[c] = sv_next[c];
     }
     it += n;
 
@@ -631,11 +659,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_init(&bars->kv_full[i], kSparse ? 32 : 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
+    for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->s_full[i], 1);
+    for (int i = 0; i < kMlaXsBufs; ++i)
       mbar_init(&bars->xs_full[i], 128);  // the other CTA's 128 softmax threads
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(&bars->p_full[i], 128);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_empty, 128);
     mbar_init(&bars->mma_drain, 1);
