@@ -86,7 +86,7 @@ template <int D, int kType>
 attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   using C = PrefillCfg<D, kType>;
   const bool varlen = a.cu_seqlens_q != nullptr;
-  const CUtensorMapDataType dt = kType == 2   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+  const CUtensorMapDataType dt = kType >= 2   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                  : kType == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int es = C::kInBytes;
@@ -182,8 +182,7 @@ attn_status_t check_varlen(const attn_varlen_args* a) {
     return ATTN_ERR_INVALID_ARG;
   if (a->head_dim_qk != a->head_dim_v) return ATTN_ERR_UNSUPPORTED;
   if (a->head_dim_qk != 64 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
-  if (a->dtype == ATTN_DTYPE_E5M2) return ATTN_ERR_UNSUPPORTED;
-  if (a->dtype == ATTN_DTYPE_E4M3 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
+  if (fp8 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
@@ -485,6 +484,8 @@ attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream) {
       return D == 64 ? run_prefill<64, 1>(*args, s) : run_prefill<128, 1>(*args, s);
     case ATTN_DTYPE_E4M3:
       return run_prefill<128, 2>(*args, s);
+    case ATTN_DTYPE_E5M2:
+      return run_prefill<128, 3>(*args, s);
     default:
       return ATTN_ERR_UNSUPPORTED;
   }

@@ -81,14 +81,14 @@ static_assert(2 * 128 * kPrefillSoftmaxRegs + 128 * kPrefillOtherRegs <=
                   kPrefillThreads * kPrefillLaunchRegs,
               "register split exceeds the launch allocation");
 
-// Input types: 0 = bf16, 1 = fp16, 2 = FP8 E4M3.
-// With FP8 inputs S = Q K^T runs as an e4m3 MMA; P is kept in fp16 (e4m3 has
+// Input types: 0 = bf16, 1 = fp16, 2 = FP8 E4M3, 3 = FP8 E5M2.
+// With FP8 inputs S = Q K^T runs as an FP8 MMA; P is kept in fp16 (FP8 has
 // too few mantissa bits for P: rows with few visible keys would miss the
 // accuracy bound), so V is converted to fp16 in shared memory (exact: every
-// e4m3 value is an fp16 value) for the fp16 P V MMA.
+// e4m3 and every e5m2 value is an fp16 value) for the fp16 P V MMA.
 template <int D, int kType>
 struct PrefillCfg {
-  static constexpr bool kFp8 = kType == 2;
+  static constexpr bool kFp8 = kType == 2 || kType == 3;
   static constexpr int kInBytes = kFp8 ? 1 : 2;
   static constexpr int kChunkElems = 128 / kInBytes;     // elements per 128-byte row chunk
   static constexpr int kChunks = D * kInBytes / 128;     // 128-byte column chunks
@@ -295,9 +295,9 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
                       uint32_t tmem) {
   using C = PrefillCfg<D, kType>;
   volatile int* abort = &bars->abort;
-  // kind::f16 formats: 0 = fp16, 1 = bf16; kind::f8f6f4: 0 = e4m3. P V runs
-  // in fp16 for FP8 inputs.
-  constexpr int fmt_qk = kType == 0 ? 1 : 0;
+  // Operand formats: kind::f16 0 = fp16, 1 = bf16; kind::f8f6f4 0 = e4m3,
+  // 1 = e5m2. P V runs in fp16 for FP8 inputs.
+  constexpr int fmt_qk = (kType == 0 || kType == 3) ? 1 : 0;
   constexpr int fmt_pv = kType == 0 ? 1 : 0;
   constexpr uint32_t idesc_qk = make_idesc(128, kPrefillBN, fmt_qk, 0, 0);
   // V is MN-major (d contiguous): one MMA covers all D columns; the 64-column
@@ -381,6 +381,17 @@ drain : {
 // the P V MMA reads (two 64-column chunks, 128-byte swizzled); the e4m3 stage
 // is then released to the producer and the fp16 stage handed to the MMA.
 // ---------------------------------------------------------------------------
+// Two FP8 values (low byte first) to two fp16 values, exactly.
+template <int kType>
+DEVI uint32_t fp8x2_to_f16x2(unsigned short v) {
+  uint32_t h;
+  if constexpr (kType == 3)
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(v));
+  else
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  return h;
+}
+
 template <int D, int kType>
 DEVI void prefill_convert(const PrefillParams& p, uint8_t* smem, PrefillBarriers* bars) {
   using C = PrefillCfg<D, kType>;
@@ -408,8 +419,8 @@ DEVI void prefill_convert(const PrefillParams& p, uint8_t* smem, PrefillBarriers
         uint32_t h[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * q]) : "h"((unsigned short)(w[q] & 0xffff)));
-          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * q + 1]) : "h"((unsigned short)(w[q] >> 16)));
+          h[2 * q] = fp8x2_to_f16x2<kType>((unsigned short)(w[q] & 0xffff));
+          h[2 * q + 1] = fp8x2_to_f16x2<kType>((unsigned short)(w[q] >> 16));
         }
         const int chunk = unit >> 2, u16 = (unit & 3) * 2;
         uint8_t* drow = dst + chunk * C::kChunkBytes + row * 128;

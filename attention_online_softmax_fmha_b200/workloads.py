@@ -283,6 +283,10 @@ CONFIGS = {
     "window_sink_fp8": dict(kind="prefill", seqlens_q=[8192] * 4, num_heads_q=32,
                             num_heads_kv=32, head_dim=128, varlen=False, causal=True,
                             window=(1024, 0), sink=True, dtype="e4m3"),
+    # the same with e5m2 inputs (MATE FMHA dtype list)
+    "window_sink_e5m2": dict(kind="prefill", seqlens_q=[8192] * 4, num_heads_q=32,
+                             num_heads_kv=32, head_dim=128, varlen=False, causal=True,
+                             window=(1024, 0), sink=True, dtype="e5m2"),
     "paged_decode": dict(kind="paged", lengths=(64, 1024, 32768), seqlen_q=1, num_heads_q=32,
                          num_heads_kv=8, head_dim=128, page_size=64),
     # the same decode with 16 sequences (about 1.1 GB of cache), for profiler

@@ -206,7 +206,7 @@ def prefill_workload(name: str, seed: int, device):
            "sink": inp.sink is not None, "dtype": inp.dtype, "total_q_tokens": sum(inp.seqlens_q),
            "visible_pairs_per_head": pairs}
     return dict(step=step, e2e_step=e2e_step, work=flops / 1e12, unit="TFLOP/s", bound=bound,
-                kernel=f"prefill_kernel<{D},{ {'bf16': 0, 'fp16': 1, 'e4m3': 2}[inp.dtype] }>", launches_per_step=1, h2d=h2d, d2h=d2h, cfg=cfg,
+                kernel=f"prefill_kernel<{D},{ {'bf16': 0, 'fp16': 1, 'e4m3': 2, 'e5m2': 3}[inp.dtype] }>", launches_per_step=1, h2d=h2d, d2h=d2h, cfg=cfg,
                 dtype=inp.dtype, inp=inp, per_unit=f"2*(D_qk+D_v)*H_q FLOP per visible pair, "
                 f"{pairs} visible pairs per head")
 
@@ -333,6 +333,7 @@ WORKLOADS = {
     "varlen_causal_gqa": prefill_workload,
     "window_sink": prefill_workload,
     "window_sink_fp8": prefill_workload,
+    "window_sink_e5m2": prefill_workload,
     "paged_decode": paged_workload,
     "paged_decode_small": paged_workload,
     "mla_dense": mla_workload,

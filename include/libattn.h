@@ -103,7 +103,7 @@ typedef enum {
 /*   ignored otherwise; S uses q*q_descale and k*k_descale, O uses           */
 /*   v*v_descale (MATE FMHA dtype notes).                                    */
 /* sink: fp32 (H_q,) per-head logit, nullable.                               */
-/* Supported now: D_qk = D_v in {64, 128}; e5m2 returns UNSUPPORTED.         */
+/* Supported now: D_qk = D_v in {64, 128}; FP8 (e4m3, e5m2) with D = 128.   */
 /* ------------------------------------------------------------------------ */
 typedef struct {
   const void* q;

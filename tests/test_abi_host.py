@@ -76,7 +76,8 @@ def _varlen(**over):
     (dict(q_stride_s=8 * 128 + 1), B.INVALID_ARG),  # row start not 16-byte aligned
     (dict(dtype=9), B.INVALID_ARG),
     (dict(dtype=B.DTYPE_E4M3), B.INVALID_ARG),      # FP8 without descales
-    (dict(dtype=B.DTYPE_E5M2, q_descale=8, k_descale=8, v_descale=8), B.UNSUPPORTED),
+    (dict(dtype=B.DTYPE_E5M2, q_descale=8, k_descale=8, v_descale=8, head_dim_qk=64,
+          head_dim_v=64), B.UNSUPPORTED),            # FP8 is built for D = 128
     (dict(head_dim_qk=96, head_dim_v=96), B.UNSUPPORTED),
     (dict(head_dim_v=64), B.UNSUPPORTED),
     (dict(cu_seqlens_q=0x5000), B.INVALID_ARG),     # cu_seqlens_k missing

@@ -138,6 +138,22 @@ def test_fp8_varlen_causal_gqa_edge_lengths():
     run_and_check(inp, atol=5e-2)
 
 
+@pytest.mark.parametrize("fmt", ["e5m2"])
+def test_fp8_e5m2_padded_window_sink(fmt):
+    # e5m2 inputs (MATE FMHA dtype list): S as an e5m2 MMA, V exactly to fp16.
+    inp = W.make_prefill(seqlens_q=[700] * 2, num_heads_q=4, num_heads_kv=2, head_dim=128,
+                         varlen=False, causal=True, window=(100, 0), sink=True, dtype=fmt,
+                         seed=13, device="cuda")
+    run_and_check(inp, atol=5e-2)
+
+
+def test_fp8_e5m2_varlen_causal_gqa_edge_lengths():
+    lens = [1, 2, 63, 64, 65, 129, 300, 513]
+    inp = W.make_prefill(seqlens_q=lens, num_heads_q=8, num_heads_kv=2, head_dim=128,
+                         varlen=True, causal=True, dtype="e5m2", seed=14, device="cuda")
+    run_and_check(inp, atol=5e-2)
+
+
 def test_fp8_full_size_window_sink_sampled():
     """The FP8 window + sink workload at full size (B=4, S=8192, H=32, D=128,
     window (1024, 0), sink, descales U[0.5, 2]); rows sampled for the oracle."""
