@@ -153,12 +153,15 @@ def visible_mask(len_q: int, len_k: int, causal: bool = False, window_left: int 
 # ---------------------------------------------------------------------------
 
 def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
-                   vis: np.ndarray, sink=None) -> Tuple[np.ndarray, np.ndarray]:
+                   vis: np.ndarray, sink=None, bias=None) -> Tuple[np.ndarray, np.ndarray]:
     """Attention for a block of query rows against one key/value set.
 
     q (R, D_qk), k (L, D_qk), v (L, D_v), vis (R, L) bool; sink is None, a
-    scalar, or an array (R,) of per-row sink logits. Returns O (R, D_v) and the
-    keys-only LSE (R,), all float64."""
+    scalar, or an array (R,) of per-row sink logits; bias is None or an
+    additive score mask (R, L) added after the scale (Mojo
+    "flash_attention_split_kv": input_mask_fn loads additive mask values), a
+    key with bias -inf being left out like an invisible one. Returns O (R, D_v)
+    and the keys-only LSE (R,), all float64."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -168,6 +171,9 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
     if R == 0 or k.shape[0] == 0:
         return out, lse
     s = scale * (q @ k.T)
+    if bias is not None:
+        s = s + np.asarray(bias, dtype=np.float64)
+        vis = np.logical_and(vis, s > NEG_INF)
     sinks = None
     if sink is not None:
         sinks = np.broadcast_to(np.asarray(sink, dtype=np.float64), (R,))
@@ -197,19 +203,35 @@ def _kv_head(h: int, num_heads_q: int, num_heads_kv: int) -> int:
 
 def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal=False,
                      window=(-1, -1), sink=None, q_descale=None, k_descale=None,
-                     v_descale=None, rows: Optional[Iterable[Tuple[int, int, int]]] = None):
+                     v_descale=None, rows: Optional[Iterable[Tuple[int, int, int]]] = None,
+                     mask=None):
     """Packed (TND) layout: q (T_q, H_q, D), k/v (T_k, H_kv, D) as float64,
     cu_seqlens int arrays (B+1). Returns out (T_q, H_q, D_v) and lse (H_q, T_q).
 
     ``rows`` optionally restricts the work to (b, i, h) triples; the other
-    entries of out/lse are left at 0 / -inf."""
-    q = np.asarray(q, np.float64)
-    k = np.asarray(k, np.float64)
-    v = np.asarray(v, np.float64)
+    entries of out/lse are left at 0 / -inf. ``mask`` is None or an additive
+    score mask indexed [b, h, i, j] by sequence, query head, and the row and
+    key positions within the sequence (broadcastable numpy array)."""
     cu_q = [int(x) for x in cu_seqlens_q]
     cu_k = [int(x) for x in cu_seqlens_k]
     B = len(cu_q) - 1
+    return _attention_segments(q, k, v, cu_q[:B], [cu_q[b + 1] - cu_q[b] for b in range(B)],
+                               cu_k[:B], [cu_k[b + 1] - cu_k[b] for b in range(B)], scale,
+                               causal, window, sink, q_descale, k_descale, v_descale, rows,
+                               mask)
+
+
+def _attention_segments(q, k, v, start_q, len_q, start_k, len_k, scale, causal, window, sink,
+                        q_descale, k_descale, v_descale, rows, mask):
+    """Sequence b: query rows start_q[b] .. + len_q[b] of q (T_q, H_q, D), keys
+    start_k[b] .. + len_k[b] of k/v (T_k, H_kv, D)."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B = len(start_q)
     Hq, Hkv = q.shape[1], k.shape[1]
+    if mask is not None:
+        mask = np.asarray(mask, np.float64)
     out = np.zeros((q.shape[0], Hq, v.shape[2]), np.float64)
     lse = np.full((Hq, q.shape[0]), NEG_INF, np.float64)
     want = None
@@ -218,15 +240,16 @@ def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal=False,
         for (b, i, h) in rows:
             want.setdefault((b, h), []).append(i)
     for b in range(B):
-        Lq, Lk = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        Lq, Lk = int(len_q[b]), int(len_k[b])
+        q0, k0 = int(start_q[b]), int(start_k[b])
         for h in range(Hq):
             if want is not None and (b, h) not in want:
                 continue
             g = _kv_head(h, Hq, Hkv)
             ii = np.arange(Lq) if want is None else np.array(sorted(set(want[(b, h)])))
-            qs = q[cu_q[b] + ii, h, :]
-            ks = k[cu_k[b]:cu_k[b + 1], g, :]
-            vs = v[cu_k[b]:cu_k[b + 1], g, :]
+            qs = q[q0 + ii, h, :]
+            ks = k[k0:k0 + Lk, g, :]
+            vs = v[k0:k0 + Lk, g, :]
             if q_descale is not None:
                 qs = qs * float(q_descale[b][g])
                 ks = ks * float(k_descale[b][g])
@@ -236,27 +259,40 @@ def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, scale, causal=False,
                 lo, hi = visible_range(int(i), Lq, Lk, causal, window[0], window[1])
                 if lo <= hi:
                     vis[r, lo:hi + 1] = True
+            bias = None
+            if mask is not None:
+                mb = mask[b if mask.shape[0] > 1 else 0, h if mask.shape[1] > 1 else 0]
+                rows_b = mb[ii] if mb.shape[0] > 1 else np.repeat(mb[:1], len(ii), 0)
+                bias = rows_b[:, :Lk] if rows_b.shape[1] > 1 else np.repeat(rows_b, Lk, 1)
             o, l = attention_rows(qs, ks, vs, scale, vis,
-                                  None if sink is None else float(sink[h]))
-            out[cu_q[b] + ii, h, :] = o
-            lse[h, cu_q[b] + ii] = l
+                                  None if sink is None else float(sink[h]), bias)
+            out[q0 + ii, h, :] = o
+            lse[h, q0 + ii] = l
     return out, lse
 
 
 def attention_padded(q, k, v, scale, causal=False, window=(-1, -1), sink=None,
-                     q_descale=None, k_descale=None, v_descale=None, rows=None):
+                     q_descale=None, k_descale=None, v_descale=None, rows=None, mask=None,
+                     seqused_q=None, seqused_k=None):
     """Padded (BSHD) layout: q (B, S_q, H_q, D), k/v (B, S_k, H_kv, D).
-    Returns out (B, S_q, H_q, D_v) and lse (B, H_q, S_q)."""
+    Returns out (B, S_q, H_q, D_v) and lse (B, H_q, S_q).
+
+    seqused_q / seqused_k (CANN "flash_attn": seqused_q, seqused_kv) are None
+    or per-sequence counts of the rows / keys in use (<= S_q / S_k): sequence b
+    is then its first seqused_q[b] rows against its first seqused_k[b] keys
+    (bottom-right causal alignment uses those lengths); rows past it stay
+    0 / -inf. ``mask`` as in attention_varlen."""
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
     B, Sq, Hq, _ = q.shape
     Sk = k.shape[1]
-    cu_q = np.arange(B + 1) * Sq
-    cu_k = np.arange(B + 1) * Sk
-    o, l = attention_varlen(q.reshape(B * Sq, Hq, -1), k.reshape(B * Sk, k.shape[2], -1),
-                            v.reshape(B * Sk, v.shape[2], -1), cu_q, cu_k, scale, causal,
-                            window, sink, q_descale, k_descale, v_descale, rows)
+    len_q = [Sq] * B if seqused_q is None else [int(x) for x in seqused_q]
+    len_k = [Sk] * B if seqused_k is None else [int(x) for x in seqused_k]
+    o, l = _attention_segments(q.reshape(B * Sq, Hq, -1), k.reshape(B * Sk, k.shape[2], -1),
+                               v.reshape(B * Sk, v.shape[2], -1), [b * Sq for b in range(B)],
+                               len_q, [b * Sk for b in range(B)], len_k, scale, causal, window,
+                               sink, q_descale, k_descale, v_descale, rows, mask)
     return o.reshape(B, Sq, Hq, -1), l.reshape(Hq, B, Sq).transpose(1, 0, 2)
 
 

@@ -372,3 +372,70 @@ def test_mla_sparse_subset_matches_sdpa_on_gathered_rows():
     ref = _sdpa(q[0, 0][:, None, :], np.repeat(kk[None], Hq, 0),
                 np.repeat(kk[None, :, :Dv], Hq, 0), 0.5)[:, 0, :]
     np.testing.assert_allclose(out[0, 0], ref, rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Additive score mask and seqused (padded layout)
+# ---------------------------------------------------------------------------
+
+def test_additive_mask_zero_and_constant_shift():
+    """A zero mask changes nothing; a mask constant over a row's keys leaves O
+    unchanged (softmax is shift-invariant) and adds the constant to the LSE."""
+    B, S, Hq, Hkv, D = 2, 9, 4, 2, 8
+    q = RNG.normal(size=(B, S, Hq, D))
+    k = RNG.normal(size=(B, S, Hkv, D))
+    v = RNG.normal(size=(B, S, Hkv, D))
+    o0, l0 = oracle.attention_padded(q, k, v, 0.3, causal=True)
+    oz, lz = oracle.attention_padded(q, k, v, 0.3, causal=True, mask=np.zeros((1, 1, S, S)))
+    np.testing.assert_array_equal(oz, o0)
+    np.testing.assert_array_equal(lz, l0)
+    c = RNG.normal(size=(B, Hq, S, 1))
+    oc, lc = oracle.attention_padded(q, k, v, 0.3, causal=True, mask=np.repeat(c, S, 3))
+    np.testing.assert_allclose(oc, o0, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lc, l0 + c[..., 0], rtol=1e-12)
+
+
+def test_additive_mask_minus_inf_removes_keys_and_bias_matches_sdpa():
+    """-inf entries drop those keys (compared with the attention over the
+    remaining keys only); a finite bias matches torch SDPA with an additive
+    float mask on the same rows."""
+    S, Hq, D = 11, 3, 6
+    q = RNG.normal(size=(1, S, Hq, D))
+    k = RNG.normal(size=(1, S, Hq, D))
+    v = RNG.normal(size=(1, S, Hq, D))
+    drop = np.zeros((1, 1, S, S))
+    keep = np.array([0, 2, 3, 7, 10])
+    drop[..., np.setdiff1d(np.arange(S), keep)] = -np.inf
+    o, l = oracle.attention_padded(q, k, v, 0.4, mask=drop)
+    ref_o, ref_l = oracle.attention_padded(q, k[:, keep], v[:, keep], 0.4)
+    np.testing.assert_allclose(o, ref_o, rtol=1e-12)
+    np.testing.assert_allclose(l, ref_l, rtol=1e-12)
+    bias = RNG.normal(size=(1, Hq, S, S))
+    ob, _ = oracle.attention_padded(q, k, v, 0.4, mask=bias)
+    qt = torch.tensor(q[0].transpose(1, 0, 2))
+    kt = torch.tensor(k[0].transpose(1, 0, 2))
+    vt = torch.tensor(v[0].transpose(1, 0, 2))
+    ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=torch.tensor(bias[0]),
+                                         scale=0.4).numpy().transpose(1, 0, 2)
+    np.testing.assert_allclose(ob[0], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_seqused_equals_varlen_of_the_used_rows():
+    """Padded q/k/v with seqused_q/k = the packed (varlen) attention of each
+    sequence's first seqused rows and keys; rows past seqused stay 0 / -inf."""
+    B, Sq, Sk, Hq, Hkv, D = 3, 10, 13, 4, 2, 8
+    q = RNG.normal(size=(B, Sq, Hq, D))
+    k = RNG.normal(size=(B, Sk, Hkv, D))
+    v = RNG.normal(size=(B, Sk, Hkv, D))
+    uq, uk = [10, 4, 7], [13, 9, 1]
+    o, l = oracle.attention_padded(q, k, v, 0.35, causal=True, window=(5, 0),
+                                   seqused_q=uq, seqused_k=uk)
+    qp = np.concatenate([q[b, :uq[b]] for b in range(B)])
+    kp = np.concatenate([k[b, :uk[b]] for b in range(B)])
+    vp = np.concatenate([v[b, :uk[b]] for b in range(B)])
+    cq, ck = np.concatenate([[0], np.cumsum(uq)]), np.concatenate([[0], np.cumsum(uk)])
+    ov, lv = oracle.attention_varlen(qp, kp, vp, cq, ck, 0.35, True, (5, 0))
+    for b in range(B):
+        np.testing.assert_array_equal(o[b, :uq[b]], ov[cq[b]:cq[b + 1]])
+        np.testing.assert_array_equal(l[b, :, :uq[b]], lv[:, cq[b]:cq[b + 1]])
+        assert np.all(o[b, uq[b]:] == 0) and np.all(np.isneginf(l[b, :, uq[b]:]))
