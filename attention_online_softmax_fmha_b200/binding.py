@@ -43,7 +43,9 @@ class VarlenArgs(ctypes.Structure):
                 ("lse_stride_b", c_i64), ("lse_stride_h", c_i64),
                 ("dtype", c_i32), ("scale", c_f32), ("causal", c_i32),
                 ("window_left", c_i32), ("window_right", c_i32),
-                ("sink", c_vp), ("q_descale", c_vp), ("k_descale", c_vp), ("v_descale", c_vp)]
+                ("sink", c_vp), ("q_descale", c_vp), ("k_descale", c_vp), ("v_descale", c_vp),
+                ("seqused_q", c_vp), ("seqused_k", c_vp), ("mask", c_vp),
+                ("mask_stride_b", c_i64), ("mask_stride_h", c_i64), ("mask_stride_s", c_i64)]
 
 
 class SchedArgs(ctypes.Structure):
@@ -177,8 +179,12 @@ def out_dtype_for(dtype: torch.dtype) -> torch.dtype:
 
 def varlen_args(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None,
                 max_seqlen_k=None, scale=None, causal=False, window=(-1, -1), sink=None,
-                q_descale=None, k_descale=None, v_descale=None, out=None, lse=None):
-    """Build the argument struct (and allocate out/lse if not given)."""
+                q_descale=None, k_descale=None, v_descale=None, out=None, lse=None,
+                seqused_q=None, seqused_k=None, mask=None):
+    """Build the argument struct (and allocate out/lse if not given).
+
+    mask: fp32 tensor indexed [b, h, i, j] (a 4-D view; size-1 axes broadcast
+    with stride 0); seqused_q/k: int32 (B,) for the padded layout."""
     varlen = cu_seqlens_q is not None
     Hq, D = q.shape[-2], q.shape[-1]
     Hkv, Dv = k.shape[-2], v.shape[-1]
@@ -209,12 +215,18 @@ def varlen_args(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=N
         lsb, lsh = lse.stride(0), lse.stride(1)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    msb = msh = mss = 0
+    if mask is not None:
+        assert mask.dim() == 4 and mask.dtype == torch.float32, "mask: fp32 [b, h, i, j]"
+        assert mask.stride(3) == 1, "mask rows must be contiguous"
+        msb, msh, mss = (mask.stride(d) if mask.shape[d] > 1 else 0 for d in range(3))
     a = VarlenArgs(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
         B, sq, sk, q.shape[0] if varlen else 0, k.shape[0] if varlen else 0, Hq, Hkv, D, Dv,
         qsb, qss, qsh, ksb, kss, ksh, vsb, vss, vsh, osb, oss, osh, lsb, lsh,
         _TORCH_DTYPE.get(q.dtype, -1), float(scale), int(bool(causal)), int(window[0]),
-        int(window[1]), _ptr(sink), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale))
+        int(window[1]), _ptr(sink), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
+        _ptr(seqused_q), _ptr(seqused_k), _ptr(mask), msb, msh, mss)
     return a, out, lse
 
 

@@ -82,6 +82,25 @@ attn_status_t launch_status(cudaError_t e) {
 // ---------------------------------------------------------------------------
 // attn_fwd_varlen
 // ---------------------------------------------------------------------------
+template <int D, int kType, bool kMask>
+attn_status_t launch_prefill(int grid, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mv, const PrefillParams& p, cudaStream_t stream) {
+  using C = PrefillCfg<D, kType>;
+  auto kernel = prefill_kernel<D, kType, kMask>;
+  static bool configured = false;
+  if (!configured) {
+    // The warpgroups trade registers with setmaxnreg out of the block's
+    // launch allocation; that split is only valid at exactly this count.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (fa.numRegs != kPrefillLaunchRegs) return ATTN_ERR_UNSUPPORTED;
+    if (set_smem(kernel, C::kSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
+    configured = true;
+  }
+  kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+  return launch_status(cudaGetLastError());
+}
+
 template <int D, int kType>
 attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   using C = PrefillCfg<D, kType>;
@@ -113,6 +132,12 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   p.cu_q = a.cu_seqlens_q;
   p.cu_k = a.cu_seqlens_k;
   p.sink = a.sink;
+  p.seqused_q = a.seqused_q;
+  p.seqused_k = a.seqused_k;
+  p.mask = a.mask;
+  p.m_sb = a.mask_stride_b;
+  p.m_sh = a.mask_stride_h;
+  p.m_ss = a.mask_stride_s;
   p.q_descale = a.q_descale;
   p.k_descale = a.k_descale;
   p.v_descale = a.v_descale;
@@ -136,22 +161,13 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   p.window_left = a.window_left;
   p.window_right = a.window_right;
 
-  auto kernel = prefill_kernel<D, kType>;
-  static bool configured = false;
-  if (!configured) {
-    // The warpgroups trade registers with setmaxnreg out of the block's
-    // launch allocation; that split is only valid at exactly this count.
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
-    if (fa.numRegs != kPrefillLaunchRegs) return ATTN_ERR_UNSUPPORTED;
-    if (set_smem(kernel, C::kSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
-    configured = true;
-  }
   const int sms = device_sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(total, sms);
-  kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
-  return launch_status(cudaGetLastError());
+  // The additive-mask path is a separate instantiation, so the common path
+  // carries none of its registers.
+  return a.mask ? launch_prefill<D, kType, true>(grid, mq, mk, mv, p, stream)
+                : launch_prefill<D, kType, false>(grid, mq, mk, mv, p, stream);
 }
 
 attn_status_t check_varlen(const attn_varlen_args* a) {
@@ -183,6 +199,15 @@ attn_status_t check_varlen(const attn_varlen_args* a) {
   if (a->head_dim_qk != a->head_dim_v) return ATTN_ERR_UNSUPPORTED;
   if (a->head_dim_qk != 64 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
   if (fp8 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
+  if (varlen && (a->seqused_q || a->seqused_k)) return ATTN_ERR_INVALID_ARG;  // padded only
+  if (a->mask) {
+    if (a->mask_stride_b < 0 || a->mask_stride_h < 0 || a->mask_stride_s < 0)
+      return ATTN_ERR_INVALID_ARG;
+    // mask rows are read as 16-byte vectors
+    if (!aligned16(a->mask) || a->mask_stride_s % 4 || a->mask_stride_h % 4 ||
+        a->mask_stride_b % 4)
+      return ATTN_ERR_INVALID_ARG;
+  }
   return ATTN_OK;
 }
 

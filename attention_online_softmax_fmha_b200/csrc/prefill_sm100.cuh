@@ -40,6 +40,10 @@ struct PrefillParams {
   float* lse;
   const int32_t* cu_q;
   const int32_t* cu_k;
+  const int32_t* seqused_q;  // padded layout: rows / keys in use per sequence
+  const int32_t* seqused_k;
+  const float* mask;         // additive score mask [b, h, i, j] (strides in elements)
+  int64_t m_sb, m_sh, m_ss;
   const float* sink;
   const float* q_descale;
   const float* k_descale;
@@ -151,8 +155,8 @@ DEVI bool prefill_unit(const PrefillParams& p, int t, PrefillUnit& u) {
     u.bcoord = 0;
   } else {
     u.row_q = u.row_k = 0;
-    u.len_q = p.seqlen_q;
-    u.len_k = p.seqlen_k;
+    u.len_q = p.seqused_q ? p.seqused_q[u.b] : p.seqlen_q;
+    u.len_k = p.seqused_k ? p.seqused_k[u.b] : p.seqlen_k;
     u.bcoord = u.b;
   }
   const int q0 = u.m * kPrefillUnit;
@@ -509,14 +513,39 @@ DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float 
 // One S tile of keys [k0, k0 + 128) of this thread's row: mask, row max,
 // lazy O rescale, P = 2^(s * scale * log2e - m) written over S (head first),
 // row sums. Returns false if a wait gave up.
-template <int D, int kType>
+template <int D, int kType, bool kMask>
 DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t o_tmem, int w,
-                               int j, int g, int k0, float sl2, PrefillRow& row) {
+                               int j, int g, int k0, float sl2, PrefillRow& row,
+                               const float* mrow, int len_k) {
   volatile int* abort = &bars->abort;
   if (!warp_wait(&bars->s_full[w], g & 1, abort, 20 + w)) return false;
   tc_fence_after();
   uint32_t s[kPrefillBN];
   tmem_load128(s_tmem, s);
+  if constexpr (kMask) {
+    // Additive mask: scores become log2-domain s * scale * log2e + mask *
+    // log2e here (keys past the sequence end read nothing; they are masked
+    // below), and the rest of the tile uses a unit scale.
+#pragma unroll
+    for (int c = 0; c < kPrefillBN; c += 4) {
+      const int key = k0 + c;
+      float4 mv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (mrow != nullptr) {
+        if (key + 3 < len_k) {
+          mv = __ldg(reinterpret_cast<const float4*>(mrow + key));
+        } else {
+          if (key < len_k) mv.x = __ldg(mrow + key);
+          if (key + 1 < len_k) mv.y = __ldg(mrow + key + 1);
+          if (key + 2 < len_k) mv.z = __ldg(mrow + key + 2);
+        }
+      }
+      s[c] = __float_as_uint(fmaf(__uint_as_float(s[c]), sl2, mv.x * kLog2e));
+      s[c + 1] = __float_as_uint(fmaf(__uint_as_float(s[c + 1]), sl2, mv.y * kLog2e));
+      s[c + 2] = __float_as_uint(fmaf(__uint_as_float(s[c + 2]), sl2, mv.z * kLog2e));
+      s[c + 3] = __float_as_uint(fmaf(__uint_as_float(s[c + 3]), sl2, mv.w * kLog2e));
+    }
+    sl2 = 1.f;
+  }
   const bool partial = !(k0 >= row.lo && k0 + kPrefillBN - 1 <= row.hi);
   if (partial) {
 #pragma unroll
@@ -577,14 +606,14 @@ DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t 
   // difference matters only for rows with few visible keys, whose keys all
   // lie in first or partially masked tiles; other tiles add their fp32 sum to
   // both (their rounding errors average out over the row's many keys).
-  if (j == 0 || __any_sync(0xffffffffu, partial))
+  if (j == 0 || kMask || __any_sync(0xffffffffu, partial))
     prefill_exp_tile<kType, true>(bars, s_tmem, w, sl2, s, row);
   else
     prefill_exp_tile<kType, false>(bars, s_tmem, w, sl2, s, row);
   return true;
 }
 
-template <int D, int kType>
+template <int D, int kType, bool kMask>
 DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_t tmem, int w) {
   using C = PrefillCfg<D, kType>;
   using OutT = typename std::conditional<kType == 1, __half, __nv_bfloat16>::type;
@@ -628,9 +657,12 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
     row.m_run = sink2;
     row.l_run = row.l_rnd = 0.f;
     row.seen = false;
+    const float* mrow =
+        (kMask && valid) ? p.mask + u.b * p.m_sb + u.h * p.m_sh + (int64_t)i * p.m_ss : nullptr;
     for (int j = 0; j < n; ++j, ++sj)
-      if (!prefill_softmax_tile<D, kType>(bars, s_tmem, o_tmem, w, j, sj,
-                                          (u.kt0 + j) * kPrefillBN, sl2, row))
+      if (!prefill_softmax_tile<D, kType, kMask>(bars, s_tmem, o_tmem, w, j, sj,
+                                                 (u.kt0 + j) * kPrefillBN, sl2, row, mrow,
+                                                 u.len_k))
         return;
     // Epilogue: wait for the last P V, read O, release O, normalise, store.
     if (!warp_wait(&bars->o_full[w], units & 1, abort, 22 + w)) return;
@@ -667,7 +699,7 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
   }
 }
 
-template <int D, int kType>
+template <int D, int kType, bool kMask>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_k,
@@ -721,7 +753,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   if (warp < 8) {
     regs_inc<kPrefillSoftmaxRegs>();
-    prefill_softmax<D, kType>(p, bars, tmem, warp >> 2);
+    prefill_softmax<D, kType, kMask>(p, bars, tmem, warp >> 2);
   } else {
     regs_dec<kPrefillOtherRegs>();
     if (warp == 8) {

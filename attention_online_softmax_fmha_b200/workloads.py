@@ -84,6 +84,9 @@ class PrefillInputs:
     k_descale: Optional[torch.Tensor]
     v_descale: Optional[torch.Tensor]
     dtype: str
+    # additive score mask fp32 [b, 1, i, j] (broadcast over heads), rows padded
+    # to a multiple of 4 floats in storage; None = no mask
+    mask: Optional[torch.Tensor] = None
 
     @property
     def batch(self) -> int:
@@ -98,10 +101,11 @@ def make_prefill(*, seqlens_q: Sequence[int], seqlens_k: Optional[Sequence[int]]
                  num_heads_q: int, num_heads_kv: int, head_dim: int, varlen: bool,
                  causal: bool = False, window=(-1, -1), sink: bool = False,
                  dtype: str = "bf16", scale: Optional[float] = None, seed: int = 0,
-                 device="cpu") -> PrefillInputs:
+                 mask: bool = False, device="cpu") -> PrefillInputs:
     """Prefill inputs. ``varlen`` packs the sequences back to back (TND with
     cu_seqlens); otherwise all sequences must share one length and the tensors
-    are padded BSHD."""
+    are padded BSHD. ``mask``: an additive fp32 score mask N(0, 1) per
+    (sequence, row, key), shared by the heads."""
     seqlens_q = [int(x) for x in seqlens_q]
     seqlens_k = [int(x) for x in (seqlens_k if seqlens_k is not None else seqlens_q)]
     B = len(seqlens_q)
@@ -134,9 +138,15 @@ def make_prefill(*, seqlens_q: Sequence[int], seqlens_k: Optional[Sequence[int]]
         vd = torch.rand(B, num_heads_kv, generator=g, device=device) * 1.5 + 0.5
     if scale is None:
         scale = 1.0 / math.sqrt(head_dim)
+    mask_t = None
+    if mask:
+        lq, lk = max(seqlens_q), max(seqlens_k)
+        store = torch.randn(B, 1, lq, (lk + 3) // 4 * 4, generator=g, device=device,
+                            dtype=torch.float32)
+        mask_t = store[..., :lk]
     return PrefillInputs(q, k, v, cu_q, cu_k, seqlens_q, seqlens_k, num_heads_q, num_heads_kv,
                          head_dim, bool(causal), tuple(window), float(scale), sink_t, qd, kd, vd,
-                         dtype)
+                         dtype, mask_t)
 
 
 @dataclasses.dataclass
@@ -287,6 +297,10 @@ CONFIGS = {
     "window_sink_e5m2": dict(kind="prefill", seqlens_q=[8192] * 4, num_heads_q=32,
                              num_heads_kv=32, head_dim=128, varlen=False, causal=True,
                              window=(1024, 0), sink=True, dtype="e5m2"),
+    # an additive score mask on a causal padded prefill (B4 S4096 H32/8 D128;
+    # the mask is 4 x 4096 x 4096 fp32, shared by the heads)
+    "dense_mask": dict(kind="prefill", seqlens_q=[4096] * 4, num_heads_q=32, num_heads_kv=8,
+                       head_dim=128, varlen=False, causal=True, mask=True),
     "paged_decode": dict(kind="paged", lengths=(64, 1024, 32768), seqlen_q=1, num_heads_q=32,
                          num_heads_kv=8, head_dim=128, page_size=64),
     # the same decode with 16 sequences (about 1.1 GB of cache), for profiler

@@ -167,7 +167,8 @@ def prefill_workload(name: str, seed: int, device):
                 for a, b in zip(inp.seqlens_q, inp.seqlens_k))
     flops = 2.0 * (D + D) * inp.num_heads_q * pairs
     kw = dict(scale=inp.scale, causal=inp.causal, window=inp.window, sink=inp.sink,
-              q_descale=inp.q_descale, k_descale=inp.k_descale, v_descale=inp.v_descale)
+              q_descale=inp.q_descale, k_descale=inp.k_descale, v_descale=inp.v_descale,
+              mask=inp.mask)
     if inp.varlen:
         kw.update(cu_seqlens_q=inp.cu_seqlens_q, cu_seqlens_k=inp.cu_seqlens_k,
                   max_seqlen_q=max(inp.seqlens_q), max_seqlen_k=max(inp.seqlens_k))
@@ -188,6 +189,9 @@ def prefill_workload(name: str, seed: int, device):
     dev_in = [inp.q, inp.k, inp.v]
     small = [t for t in (inp.cu_seqlens_q, inp.cu_seqlens_k, inp.sink, inp.q_descale,
                          inp.k_descale, inp.v_descale) if t is not None]
+    if inp.mask is not None:  # the mask's storage (rows padded to 4 floats)
+        small.append(inp.mask.as_strided((inp.mask.numel() // inp.mask.shape[-1] *
+                                           inp.mask.stride(2),), (1,)))
     host_small = [t.cpu().pin_memory() for t in small]
 
     def e2e_step(stream):
@@ -204,7 +208,7 @@ def prefill_workload(name: str, seed: int, device):
            else inp.seqlens_q[0], "num_heads_q": inp.num_heads_q, "num_heads_kv": inp.num_heads_kv,
            "head_dim": D, "causal": inp.causal, "window": list(inp.window),
            "sink": inp.sink is not None, "dtype": inp.dtype, "total_q_tokens": sum(inp.seqlens_q),
-           "visible_pairs_per_head": pairs}
+           "visible_pairs_per_head": pairs, "additive_mask": inp.mask is not None}
     return dict(step=step, e2e_step=e2e_step, work=flops / 1e12, unit="TFLOP/s", bound=bound,
                 kernel=f"prefill_kernel<{D},{ {'bf16': 0, 'fp16': 1, 'e4m3': 2, 'e5m2': 3}[inp.dtype] }>", launches_per_step=1, h2d=h2d, d2h=d2h, cfg=cfg,
                 dtype=inp.dtype, inp=inp, per_unit=f"2*(D_qk+D_v)*H_q FLOP per visible pair, "
@@ -334,6 +338,7 @@ WORKLOADS = {
     "window_sink": prefill_workload,
     "window_sink_fp8": prefill_workload,
     "window_sink_e5m2": prefill_workload,
+    "dense_mask": prefill_workload,
     "paged_decode": paged_workload,
     "paged_decode_small": paged_workload,
     "mla_dense": mla_workload,

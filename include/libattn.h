@@ -103,6 +103,20 @@ typedef enum {
 /*   ignored otherwise; S uses q*q_descale and k*k_descale, O uses           */
 /*   v*v_descale (MATE FMHA dtype notes).                                    */
 /* sink: fp32 (H_q,) per-head logit, nullable.                               */
+/* seqused_q / seqused_k (CANN "flash_attn": seqused_q, seqused_kv): padded  */
+/*   layout only, nullable, device int32 (batch): the rows of q and the keys */
+/*   of k/v in use per sequence (<= max_seqlen_q / max_seqlen_k; values are  */
+/*   not checked). Sequence b is its first seqused_q[b] rows against its     */
+/*   first seqused_k[b] keys (bottom-right causal alignment on those); rows  */
+/*   past seqused_q[b] are not written.                                      */
+/* mask (Mojo "flash_attention_split_kv": input_mask_fn, additive mask       */
+/*   values): nullable device fp32, added to scale * q.k before the softmax; */
+/*   element (b, h, i, j) for sequence b, query head h, row i and key j of   */
+/*   the sequence at b*mask_stride_b + h*mask_stride_h + i*mask_stride_s + j */
+/*   (strides in elements, >= 0, 0 broadcasts; rows 16-byte aligned: base    */
+/*   and mask_stride_s multiples of 4 elements). -inf leaves a key out. The  */
+/*   causal/window masks still apply. Each row reads its mask row once per   */
+/*   key tile, so the mask adds S_q x S_k x 4 bytes per (sequence, head).    */
 /* Supported now: D_qk = D_v in {64, 128}; FP8 (e4m3, e5m2) with D = 128.   */
 /* ------------------------------------------------------------------------ */
 typedef struct {
@@ -136,6 +150,10 @@ typedef struct {
   const float* q_descale;
   const float* k_descale;
   const float* v_descale;
+  const int32_t* seqused_q;  /* padded layout only; nullable                  */
+  const int32_t* seqused_k;  /* padded layout only; nullable                  */
+  const float* mask;         /* additive score mask; nullable                 */
+  int64_t mask_stride_b, mask_stride_h, mask_stride_s;
 } attn_varlen_args;
 
 attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream);

@@ -175,3 +175,81 @@ def test_fp8_full_size_window_sink_sampled():
     for b, i, h in rows:
         assert_close_out(o[b, i, h], ro[b, i, h], 5e-2)
         assert abs(l[b, h, i] - rl[b, h, i]) <= 1e-3
+
+
+# ---------------------------------------------------------------------------
+# seqused (padded layout) and the additive score mask
+# ---------------------------------------------------------------------------
+
+def _padded_case(B, Sq, Sk, Hq, Hkv, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Sq, Hq, D, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(B, Sk, Hkv, D, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(B, Sk, Hkv, D, generator=g).to(torch.bfloat16).cuda()
+    return q, k, v
+
+
+def test_padded_seqused_causal_window_gqa():
+    """Padded q/k/v with seqused_q/k (CANN flash_attn seqused_q, seqused_kv):
+    each sequence is its first seqused rows against its first seqused keys."""
+    B, Sq, Sk, Hq, Hkv, D = 3, 300, 400, 4, 2, 128
+    q, k, v = _padded_case(B, Sq, Sk, Hq, Hkv, D, 21)
+    uq, uk = [300, 17, 129], [400, 5, 250]
+    out = torch.zeros(B, Sq, Hq, D, dtype=torch.bfloat16, device="cuda")
+    out, lse = B_fwd(q, k, v, scale=D ** -0.5, causal=True, window=(100, 0), out=out,
+                     seqused_q=torch.tensor(uq, dtype=torch.int32, device="cuda"),
+                     seqused_k=torch.tensor(uk, dtype=torch.int32, device="cuda"))
+    ro, rl = oracle.attention_padded(to_f64(q), to_f64(k), to_f64(v), D ** -0.5, True, (100, 0),
+                                     seqused_q=uq, seqused_k=uk)
+    o = to_f64(out)
+    for b in range(B):
+        assert_close_out(o[b, :uq[b]], ro[b, :uq[b]], 1e-2)
+        assert_close_lse(lse.cpu().numpy()[b, :, :uq[b]], rl[b, :, :uq[b]])
+        assert np.all(o[b, uq[b]:] == 0), "rows past seqused_q are not written"
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_additive_mask_padded(D):
+    """Additive fp32 score mask (Mojo flash_attention_split_kv input_mask_fn)
+    per (b, h, i, j), with -inf entries, on top of a causal mask; mask rows
+    padded to a multiple of 4 floats."""
+    B, S, Hq, Hkv = 2, 333, 4, 2
+    q, k, v = _padded_case(B, S, S, Hq, Hkv, D, 22 + D)
+    g = torch.Generator().manual_seed(7)
+    store = torch.randn(B, Hq, S, 336, generator=g, dtype=torch.float32)
+    store[torch.rand(B, Hq, S, 336, generator=g) < 0.1] = -float("inf")
+    mask = store.cuda()[..., :S]
+    out, lse = B_fwd(q, k, v, scale=D ** -0.5, causal=True, mask=mask)
+    ro, rl = oracle.attention_padded(to_f64(q), to_f64(k), to_f64(v), D ** -0.5, True,
+                                     mask=store[..., :S].double().numpy())
+    assert_close_out(to_f64(out), ro, 1e-2)
+    assert_close_lse(lse.cpu().numpy(), rl)
+
+
+def test_additive_mask_varlen_broadcast_over_heads():
+    """Varlen rows index the mask by position within the sequence; a size-1
+    head axis broadcasts (stride 0)."""
+    lens = [1, 70, 200, 129]
+    inp = W.make_prefill(seqlens_q=lens, num_heads_q=4, num_heads_kv=1, head_dim=128, varlen=True,
+                         causal=False, seed=23, device="cuda")
+    L = max(lens)
+    g = torch.Generator().manual_seed(8)
+    store = torch.randn(len(lens), 1, L, 200, generator=g, dtype=torch.float32) * 2
+    mask = store.cuda()
+    out, lse = B.fwd_varlen(inp.q, inp.k, inp.v, scale=inp.scale, cu_seqlens_q=inp.cu_seqlens_q,
+                            cu_seqlens_k=inp.cu_seqlens_k, max_seqlen_q=L, max_seqlen_k=L,
+                            mask=mask)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    ro, rl = oracle.attention_varlen(to_f64(inp.q), to_f64(inp.k), to_f64(inp.v),
+                                     inp.cu_seqlens_q.cpu().numpy(), inp.cu_seqlens_k.cpu().numpy(),
+                                     inp.scale, mask=store.double().numpy())
+    assert_close_out(to_f64(out), ro, 1e-2)
+    assert_close_lse(lse.cpu().numpy(), rl)
+
+
+def B_fwd(q, k, v, **kw):
+    out, lse = B.fwd_varlen(q, k, v, **kw)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    return out, lse
