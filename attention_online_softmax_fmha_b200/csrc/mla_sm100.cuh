@@ -12,7 +12,8 @@
 // dimensions of its V half (rank 0: nope 0..255 and the 64 rope dimensions,
 // rank 1: nope 256..511) of Q and of every key, computes the partial scores
 // S_r = Q_r K_r^T on its tensor core, and the two halves swap partials through
-// distributed shared memory, so both see S = S_0 + S_1 (the same sum in the
+// distributed shared memory (one bulk copy per warp into the other CTA,
+// completing on its barrier), so both see S = S_0 + S_1 (the same sum in the
 // same order: identical P). Each CTA then accumulates O for its 256 V columns
 // (its first four 64-column chunks). Half of Q and of each key row per CTA
 // leaves room for a five-stage key ring, and the cache is read once per row
@@ -28,7 +29,7 @@
 // Roles (192 threads per CTA):
 //   warps 0-3  softmax: thread r owns query row r (= TMEM lane r).
 //   warp 4     producer: Q tile (TMA, resident), key tiles of 32 keys into a
-//              5-stage ring: dense by TMA boxes through the block table;
+//              4-stage ring: dense by TMA boxes through the block table;
 //              sparse by per-lane 16-byte async copies of the gathered rows
 //              (each lane one key, zeros for skipped keys), completed and
 //              fenced before the stage is handed over.
@@ -49,8 +50,14 @@ constexpr int kMlaDv = 512;
 constexpr int kMlaDvHalf = 256;
 constexpr int kMlaBN = 32;         // keys per tile
 constexpr int kMlaRows = 128;      // query rows per row tile
-constexpr int kMlaStages = 5;
+constexpr int kMlaStages = 4;
 constexpr int kMlaSBufs = 3;       // S buffers in TMEM
+// S of tile g + kMlaSAhead is issued after P V of tile g. The softmax needs
+// S one tile ahead (it sends tile g + 1's partials before finishing tile g),
+// so at least 2; each tile further ahead keeps one more key stage busy and
+// leaves one tile less of slack for the loads.
+constexpr int kMlaSAhead = 3;
+static_assert(kMlaSAhead >= 2 && kMlaSAhead <= kMlaSBufs, "S lookahead");
 constexpr int kMlaXsBufs = 2;      // partial-S exchange buffers in shared memory
 constexpr int kMlaMaxChunks = 5;   // 64-column chunks per CTA (rank 0: 5, rank 1: 4)
 constexpr int kMlaQChunkBytes = kMlaRows * 128;                // 16 KB
@@ -59,8 +66,9 @@ constexpr int kMlaQBytes = kMlaMaxChunks * kMlaQChunkBytes;    // 80 KB
 constexpr int kMlaKVBytes = kMlaMaxChunks * kMlaKVChunkBytes;  // 20 KB
 constexpr int kMlaXsBytes = kMlaRows * kMlaBN * 4;             // one partial S tile, 16 KB
 constexpr int kMlaQOff = 0;
-constexpr int kMlaXsOff = kMlaQOff + kMlaQBytes;               // partial-S buffers
-constexpr int kMlaKVOff = kMlaXsOff + kMlaXsBufs * kMlaXsBytes;
+constexpr int kMlaXsOff = kMlaQOff + kMlaQBytes;               // partial S received here
+constexpr int kMlaXoOff = kMlaXsOff + kMlaXsBufs * kMlaXsBytes;  // and staged here to send
+constexpr int kMlaKVOff = kMlaXoOff + kMlaXsBufs * kMlaXsBytes;
 constexpr int kMlaBarOff = kMlaKVOff + kMlaStages * kMlaKVBytes;
 constexpr int kMlaSmemBytes = kMlaBarOff + 256;
 static_assert(kMlaSmemBytes <= 232448, "shared memory per CTA");
@@ -354,11 +362,11 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
     }
     if (!warp_wait(&bars->q_full, nq & 1, abort, 70)) goto drain;
     ++nq;
-    // S of the first three tiles, then per tile g: PV_g, S_{g+3} (S_{g+3}
-    // reuses S_g's buffer, whose P the tensor core has read in PV_g just
-    // before: the pipe runs in order). The softmax thus finds S_{g+1} ready
-    // while it finishes tile g.
-    for (int j = 0; j < kMlaSBufs && j < n; ++j)
+    // S of the first kMlaSAhead tiles, then per tile g: PV_g, S_{g+kMlaSAhead}
+    // (into buffer (g + kMlaSAhead) % 3, whose last P the tensor core has read
+    // in an earlier P V: the pipe runs in order). The softmax thus finds
+    // S_{g+1} ready while it finishes tile g.
+    for (int j = 0; j < kMlaSAhead && j < n; ++j)
       if (!mla_issue_s(bars, it + j, dq, dkv, tmem, nk, j == n - 1)) goto drain;
     for (int j = 0; j < n; ++j) {
       const int gi = it + j, sp = gi % kMlaStages;
@@ -374,8 +382,8 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
                      (j > 0 || kk > 0) ? 1u : 0u);
       tc_commit_w(&bars->kv_empty[sp]);
       tc_commit_w(&bars->o_full);
-      if (j + kMlaSBufs < n &&
-          !mla_issue_s(bars, gi + kMlaSBufs, dq, dkv, tmem, nk, j + kMlaSBufs == n - 1))
+      if (j + kMlaSAhead < n &&
+          !mla_issue_s(bars, gi + kMlaSAhead, dq, dkv, tmem, nk, j + kMlaSAhead == n - 1))
         goto drain;
     }
     it += n;
@@ -406,13 +414,29 @@ DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint
   if (!warp_wait(&bars->s_full[sb], (g / kMlaSBufs) & 1, &bars->abort, 80)) return false;
   tc_fence_after();
   tmem_load<32>(tmem + kMlaTmemS + sb * kMlaBN + lane, sv);
-  const uint32_t mine = smem_u32(smem + kMlaXsOff + b * kMlaXsBytes) + r * 128;
-  const uint32_t theirs = mapa_shared(mine, rank ^ 1);
+  // Stage this warp's 32 rows (16-byte pieces permuted by row to spread the
+  // banks) and send them with one bulk copy into the other CTA's buffer b,
+  // completing on its barrier. Staging buffer b was last the source of the
+  // copy two tiles ago: that copy must have read it.
+  const int warp_row0 = r & ~31;
+  const bool leader = (threadIdx.x & 31) == 0;
+  if (leader) bulk_wait_read<1>();
+  __syncwarp();
+  uint8_t* stage = smem + kMlaXoOff + b * kMlaXsBytes + r * 128;
 #pragma unroll
   for (int k = 0; k < 8; ++k)
-    st_cluster_v4(theirs + ((k ^ (r & 7)) << 4), sv[4 * k], sv[4 * k + 1], sv[4 * k + 2],
-                  sv[4 * k + 3]);
-  mbar_arrive_remote(mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1));
+    *reinterpret_cast<uint4*>(stage + ((k ^ (r & 7)) << 4)) =
+        make_uint4(sv[4 * k], sv[4 * k + 1], sv[4 * k + 2], sv[4 * k + 3]);
+  fence_proxy_async_smem();  // the copy reads through the async proxy
+  __syncwarp();
+  if (leader) {
+    const uint32_t bar = mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1);
+    const uint32_t off = b * kMlaXsBytes + warp_row0 * 128;
+    mbar_arrive_expect_tx_remote(bar, 32 * 128);
+    bulk_copy_to_cluster(mapa_shared(smem_u32(smem + kMlaXsOff + off), rank ^ 1),
+                         smem_u32(smem + kMlaXoOff + off), 32 * 128, bar);
+    bulk_commit();
+  }
   return true;
 }
 
@@ -661,7 +685,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->s_full[i], 1);
     for (int i = 0; i < kMlaXsBufs; ++i)
-      mbar_init(&bars->xs_full[i], 128);  // the other CTA's 128 softmax threads
+      mbar_init(&bars->xs_full[i], 4);  // one bulk copy from each softmax warp of the other CTA
     for (int i = 0; i < 2; ++i) mbar_init(&bars->p_full[i], 128);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_empty, 128);
@@ -700,6 +724,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     else
       mla_mma<kSparse>(p, smem, bars, tmem, rank);
   }
+  // The partial-score copies this CTA sent have landed in the other CTA.
+  if (warp < 4 && (threadIdx.x & 31) == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   // No remote arrival or store into this CTA's shared memory after this.
