@@ -16,7 +16,7 @@
 // completing on its barrier), so both see S = S_0 + S_1 (the same sum in the
 // same order: identical P). Each CTA then accumulates O for its 256 V columns
 // (its first four 64-column chunks). Half of Q and of each key row per CTA
-// leaves room for a five-stage key ring, and the cache is read once per row
+// leaves room for a four-stage key ring, and the cache is read once per row
 // tile instead of once per V half.
 //   dense : segment = (sequence, row tile), keys 0 .. L-1 in tiles of 32
 //           (causal: key j visible to token i iff j <= i + L - s_q).
