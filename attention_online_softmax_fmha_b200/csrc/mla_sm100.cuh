@@ -60,6 +60,8 @@ constexpr int kMlaSAhead = 3;
 static_assert(kMlaSAhead >= 2 && kMlaSAhead <= kMlaSBufs, "S lookahead");
 constexpr int kMlaXsBufs = 2;      // partial-S exchange buffers in shared memory
 constexpr int kMlaMaxChunks = 5;   // 64-column chunks per CTA (rank 0: 5, rank 1: 4)
+constexpr int kGatherLag = 1;      // sparse: tiles of gathers in flight before a stage is signalled
+static_assert(kGatherLag < kMlaStages, "gather lag");
 constexpr int kMlaQChunkBytes = kMlaRows * 128;                // 16 KB
 constexpr int kMlaKVChunkBytes = kMlaBN * 128;                 // 4 KB
 constexpr int kMlaQBytes = kMlaMaxChunks * kMlaQChunkBytes;    // 80 KB
@@ -195,6 +197,13 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
   mla_range<kSparse>(p, ub, ue, s, prefix);
   int it = 0, nq = 0;
   const int P = p.page_size;
+  // Sparse gathers issued and not yet signalled: tiles it - pend .. it - 1.
+  int pend = 0;
+  auto flush_gathers = [&]() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    fence_proxy_async_smem();
+    for (; pend > 0; --pend) mbar_arrive(&bars->kv_full[(it - pend) % kMlaStages]);
+  };
   int u = ub;
   while (u < ue) {
     int sb, se;
@@ -232,9 +241,20 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       const int st = it % kMlaStages;
       uint8_t* dst = smem + kMlaKVOff + st * kMlaKVBytes;
       bool ok = true;
-      if (lane == 0 && it >= kMlaStages)
-        ok = mbar_wait(&bars->kv_empty[st], ((it / kMlaStages) - 1) & 1, abort, 61);
-      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
+      if (it >= kMlaStages) {
+        const uint32_t parity = ((it / kMlaStages) - 1) & 1;
+        if constexpr (kSparse) {
+          // About to block on a stage: signal every gathered tile first (the
+          // MMA warp may need them to free that stage).
+          const bool free_now = lane == 0 && mbar_test(smem_u32(&bars->kv_empty[st]), parity);
+          if (!__shfl_sync(0xffffffffu, free_now ? 1 : 0, 0)) flush_gathers();
+        }
+        if (lane == 0) ok = mbar_wait(&bars->kv_empty[st], parity, abort, 61);
+      }
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+        if constexpr (kSparse) flush_gathers();
+        return;
+      }
       if constexpr (!kSparse) {
         // keys [32t, 32t + 32): pages of the block table, one TMA box per
         // (page, 64-column chunk)
@@ -278,14 +298,21 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
             }
           }
         }
-        // Wait for this lane's copies, make them visible to the tensor core
-        // (async proxy) and signal the stage.
+        // The stage is signalled kGatherLag tiles later, once this lane's
+        // copies of it have landed (made visible to the tensor core, the async
+        // proxy), so the gathers of several tiles are in flight at once.
         asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->kv_full[st]);
+        ++pend;
+        if (pend > kGatherLag) {
+          asm volatile("cp.async.wait_group %0;" ::"n"(kGatherLag) : "memory");
+          fence_proxy_async_smem();
+          mbar_arrive(&bars->kv_full[(it - kGatherLag) % kMlaStages]);
+          --pend;
+        }
       }
     }
+    // The segment's last S needs its last tiles before Q may be replaced.
+    if constexpr (kSparse) flush_gathers();
     u = min(ue, se);
     ++s;
   }
