@@ -390,10 +390,14 @@ def mla_paged(q, kv_cache, block_table, cache_seqlens, head_dim_v, scale, causal
 
 
 def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, scale,
-               rows=None):
+               rows=None, block_size=1):
     """q (B, s_q, H_q, 576); indices (B, s_q, 1, topk) logical positions. Query
     token (b, i) attends to the listed positions p with 0 <= p < L_b (each
     listed occurrence counts once); the others are skipped.
+    block_size > 1 (MindSpore "sparse_flash_attention": sparse_block_size, a
+    power of two up to 128): each index k >= 0 lists the block of positions
+    k * block_size .. k * block_size + block_size - 1 (reading: the index
+    counts blocks); negative indices are skipped.
     Returns out (B, s_q, H_q, D_v) and lse (B, H_q, s_q)."""
     q = np.asarray(q, np.float64)
     kv = np.asarray(kv_cache, np.float64)
@@ -413,6 +417,9 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
                 continue
             hs = list(range(Hq)) if want is None else sorted(set(want[(b, i)]))
             idx = np.asarray(indices[b, i, 0], dtype=np.int64)
+            if block_size > 1:
+                idx = idx[idx >= 0]
+                idx = (idx[:, None] * block_size + np.arange(block_size)[None, :]).reshape(-1)
             idx = idx[(idx >= 0) & (idx < L)]
             rows_kv = kv[np.asarray(block_table[b], np.int64)[idx // page], idx % page, 0, :]
             vis = np.ones((len(hs), idx.size), dtype=bool)

@@ -439,3 +439,26 @@ def test_seqused_equals_varlen_of_the_used_rows():
         np.testing.assert_array_equal(o[b, :uq[b]], ov[cq[b]:cq[b + 1]])
         np.testing.assert_array_equal(l[b, :, :uq[b]], lv[:, cq[b]:cq[b + 1]])
         assert np.all(o[b, uq[b]:] == 0) and np.all(np.isneginf(l[b, :, uq[b]:]))
+
+
+def test_mla_sparse_blocks_covering_the_cache_equal_dense():
+    """Block indices 0 .. L/bs - 1 with block size bs list every position once:
+    the result is the dense MLA attention; a -1 entry and a block reaching past
+    the cache end only drop positions."""
+    lens, page, Hq, D, Dv, bs = [16, 11], 4, 2, 10, 6, 4
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    q = RNG.normal(size=(2, 2, Hq, D))
+    idx = np.full((2, 2, 1, 5), -1, np.int64)
+    for b, L in enumerate(lens):
+        nb = (L + bs - 1) // bs                 # the last block of sequence 1 runs past L
+        idx[b, :, 0, :nb] = np.arange(nb)
+    o_s, l_s = oracle.mla_sparse(q, ck, bt, lens, idx, Dv, 0.3, block_size=bs)
+    o_d, l_d = oracle.mla_paged(q, ck, bt, lens, Dv, 0.3)
+    np.testing.assert_allclose(o_s, o_d, rtol=1e-12)
+    np.testing.assert_allclose(l_s, l_d, rtol=1e-12)
+    # one block of 4: the same as listing its 4 positions with block size 1
+    sel = np.array([[[[2, -1]]]])
+    o_b, _ = oracle.mla_sparse(q[:1, :1], ck, bt[:1], lens[:1], sel, Dv, 0.3, block_size=4)
+    o_1, _ = oracle.mla_sparse(q[:1, :1], ck, bt[:1], lens[:1],
+                               np.array([[[[8, 9, 10, 11]]]]), Dv, 0.3)
+    np.testing.assert_allclose(o_b, o_1, rtol=1e-12)
