@@ -52,7 +52,8 @@ class SchedArgs(ctypes.Structure):
     _fields_ = [("cache_seqlens", c_vp), ("batch", c_i32), ("seqlen_q", c_i32),
                 ("num_heads_q", c_i32), ("num_heads_kv", c_i32), ("head_dim_qk", c_i32),
                 ("head_dim_v", c_i32), ("page_size", c_i32), ("mode", c_i32), ("topk", c_i32),
-                ("num_ctas", c_i32), ("meta", c_vp), ("meta_bytes", c_sz)]
+                ("num_ctas", c_i32), ("meta", c_vp), ("meta_bytes", c_sz),
+                ("sparse_block_size", c_i32)]
 
 
 class PagedArgs(ctypes.Structure):
@@ -92,7 +93,8 @@ class MlaArgs(ctypes.Structure):
                 ("o_stride_b", c_i64), ("o_stride_s", c_i64), ("o_stride_h", c_i64),
                 ("idx_stride_b", c_i64), ("idx_stride_s", c_i64),
                 ("scale", c_f32), ("causal", c_i32), ("meta", c_vp), ("meta_bytes", c_sz),
-                ("num_ctas", c_i32), ("workspace", c_vp), ("workspace_bytes", c_sz)]
+                ("num_ctas", c_i32), ("workspace", c_vp), ("workspace_bytes", c_sz),
+                ("sparse_block_size", c_i32)]
 
 
 ARG_STRUCTS = {0: VarlenArgs, 1: SchedArgs, 2: PagedArgs, 3: CombineArgs, 4: MlaArgs}
@@ -242,9 +244,9 @@ def fwd_varlen(q, k, v, *, stream=None, **kw):
 # ---------------------------------------------------------------------------
 
 def sched_args(cache_seqlens, *, batch, seqlen_q, num_heads_q, num_heads_kv, head_dim_qk,
-               head_dim_v, page_size, mode=SCHED_MHA, topk=0, num_ctas=0):
+               head_dim_v, page_size, mode=SCHED_MHA, topk=0, num_ctas=0, sparse_block_size=0):
     return SchedArgs(_ptr(cache_seqlens), batch, seqlen_q, num_heads_q, num_heads_kv, head_dim_qk,
-                     head_dim_v, page_size, mode, topk, num_ctas, None, 0)
+                     head_dim_v, page_size, mode, topk, num_ctas, None, 0, sparse_block_size)
 
 
 def sched_metadata_size(a: SchedArgs) -> int:
@@ -344,7 +346,7 @@ def combine(out_partial, lse_partial, *, num_splits_per_seq=None, sink=None, out
 
 def mla_args(q, kv_cache, block_table, cache_seqlens, *, head_dim_v=512, scale=None,
              causal=False, indices=None, meta=None, num_ctas=0, workspace=None, out=None,
-             lse=None):
+             lse=None, sparse_block_size=0):
     B, sq, Hq, Dqk = q.shape
     if out is None:
         out = torch.empty(B, sq, Hq, head_dim_v, device=q.device, dtype=torch.bfloat16)
@@ -360,7 +362,7 @@ def mla_args(q, kv_cache, block_table, cache_seqlens, *, head_dim_v=512, scale=N
         q.stride(1), q.stride(2), kv_cache.stride(0), kv_cache.stride(1), out.stride(0),
         out.stride(1), out.stride(2), 0 if indices is None else indices.stride(0),
         0 if indices is None else indices.stride(1), float(scale), int(bool(causal)), _ptr(meta),
-        0 if meta is None else meta.numel() * 4, int(num_ctas), None, 0)
+        0 if meta is None else meta.numel() * 4, int(num_ctas), None, 0, int(sparse_block_size))
     if meta is not None:
         nbytes = int(lib().mla_workspace_size(ctypes.byref(a)))
         if workspace is None:
@@ -385,10 +387,10 @@ def mla_sparse_fwd(q, kv_cache, block_table, cache_seqlens, indices, *, stream=N
 
 
 def mla_metadata(inp_cache_seqlens, *, batch, seqlen_q, num_heads_q, page_size, topk=0,
-                 num_ctas=0, stream=None):
+                 num_ctas=0, stream=None, sparse_block_size=0):
     """Scheduler metadata for mla_fwd_paged (topk = 0) or mla_sparse_fwd."""
     return sched_metadata(inp_cache_seqlens, batch=batch, seqlen_q=seqlen_q,
                           num_heads_q=num_heads_q, num_heads_kv=1, head_dim_qk=576,
                           head_dim_v=512, page_size=page_size,
                           mode=SCHED_MLA_SPARSE if topk else SCHED_MLA, topk=topk,
-                          num_ctas=num_ctas, stream=stream)
+                          num_ctas=num_ctas, stream=stream, sparse_block_size=sparse_block_size)

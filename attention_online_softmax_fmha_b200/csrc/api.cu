@@ -230,6 +230,14 @@ bool mla_heads_ok(int heads_q) {
                          heads_q % kMlaRows == 0);
 }
 
+// sparse_block_size: 0 or 1 (one position per index) or a power of two up to
+// 128 (MindSpore sparse_flash_attention range).
+bool sbs_ok(int bs) { return bs == 0 || pow2_in(bs, 1, 128); }
+// Key positions per token of a sparse MLA problem (topk indices of bs keys).
+int sparse_positions(int mode, int topk, int bs) {
+  return mode == ATTN_SCHED_MLA_SPARSE ? topk * (bs > 1 ? bs : 1) : topk;
+}
+
 attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int heads_kv,
                            int topk, int num_ctas, DecodeShape& ds) {
   if (batch <= 0 || seqlen_q <= 0 || heads_q <= 0 || heads_kv <= 0 || heads_q % heads_kv)
@@ -393,6 +401,8 @@ attn_status_t check_mla(const mla_args* a, bool sparse) {
   if (a->num_heads_kv != 1 || !mla_heads_ok(a->num_heads_q)) return ATTN_ERR_UNSUPPORTED;
   if (!pow2_in(a->page_size, 16, 256)) return ATTN_ERR_UNSUPPORTED;
   if (sparse && a->causal) return ATTN_ERR_UNSUPPORTED;
+  if (!sbs_ok(a->sparse_block_size) || (!sparse && a->sparse_block_size > 1))
+    return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
 }
 
@@ -442,6 +452,7 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   p.heads_q = a.num_heads_q;
   p.page_size = a.page_size;
   p.topk = a.topk;
+  p.sbs = a.sparse_block_size > 1 ? a.sparse_block_size : 1;
   p.tiles_per_token = ds.tiles_per_token;
   p.tokens_per_tile = ds.tokens_per_tile;
   p.row_tiles = ds.row_tiles;
@@ -477,8 +488,9 @@ attn_status_t mla_entry(const mla_args* a, void* stream, bool sparse) {
   attn_status_t st = check_mla(a, sparse);
   if (st != ATTN_OK) return st;
   DecodeShape ds;
-  st = decode_shape(sparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA, a->batch, a->seqlen_q,
-                    a->num_heads_q, a->num_heads_kv, a->topk, a->num_ctas, ds);
+  const int mode = sparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
+  st = decode_shape(mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv,
+                    sparse_positions(mode, a->topk, a->sparse_block_size), a->num_ctas, ds);
   if (st != ATTN_OK) return st;
   if (a->meta) {
     if (a->meta_bytes < meta_bytes_for(ds)) return ATTN_ERR_INVALID_ARG;
@@ -519,7 +531,9 @@ attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream) {
 size_t attn_sched_metadata_size(const attn_sched_args* a) {
   if (!a) return 0;
   DecodeShape ds;
-  if (decode_shape(a->mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv, a->topk,
+  if (!sbs_ok(a->sparse_block_size)) return 0;
+  if (decode_shape(a->mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv,
+                   sparse_positions(a->mode, a->topk, a->sparse_block_size),
                    a->num_ctas, ds) != ATTN_OK)
     return 0;
   return meta_bytes_for(ds);
@@ -530,9 +544,11 @@ attn_status_t attn_sched_metadata(const attn_sched_args* a, void* stream) {
   if (a->page_size <= 0 || a->head_dim_qk <= 0 || a->head_dim_v <= 0 || a->num_ctas < 0)
     return ATTN_ERR_INVALID_ARG;
   if (a->mode < ATTN_SCHED_MHA || a->mode > ATTN_SCHED_MLA_SPARSE) return ATTN_ERR_INVALID_ARG;
+  if (!sbs_ok(a->sparse_block_size)) return ATTN_ERR_INVALID_ARG;
   DecodeShape ds;
-  const attn_status_t st = decode_shape(a->mode, a->batch, a->seqlen_q, a->num_heads_q,
-                                        a->num_heads_kv, a->topk, a->num_ctas, ds);
+  const attn_status_t st =
+      decode_shape(a->mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv,
+                   sparse_positions(a->mode, a->topk, a->sparse_block_size), a->num_ctas, ds);
   if (st != ATTN_OK) return st;
   if (a->meta_bytes < meta_bytes_for(ds)) return ATTN_ERR_WORKSPACE_TOO_SMALL;
   SchedParams p;
@@ -625,8 +641,10 @@ size_t mla_workspace_size(const mla_args* a) {
   const bool sparse = a->indices != nullptr;
   if (check_mla(a, sparse) != ATTN_OK) return 0;
   DecodeShape ds;
-  if (decode_shape(sparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA, a->batch, a->seqlen_q,
-                   a->num_heads_q, a->num_heads_kv, a->topk, a->num_ctas, ds) != ATTN_OK)
+  const int mode = sparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
+  if (decode_shape(mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv,
+                   sparse_positions(mode, a->topk, a->sparse_block_size), a->num_ctas,
+                   ds) != ATTN_OK)
     return 0;
   return mla_ws_bytes(ds);
 }

@@ -99,6 +99,7 @@ struct MlaParams {
   int64_t kv_sblk, kv_stok;
   int64_t idx_sb, idx_ss;
   int32_t batch, seqlen_q, heads_q, page_size, topk;
+  int32_t sbs;              // sparse: positions per index (sparse_block_size, >= 1)
   int32_t tiles_per_token;  // heads_q >= 128: heads_q / 128 (else 1)
   int32_t tokens_per_tile;  // heads_q < 128: 128 / heads_q (else 1)
   int32_t row_tiles;        // dense: row tiles per sequence
@@ -142,9 +143,18 @@ DEVI void mla_seg(const MlaParams& p, int s, MlaSeg& g) {
     g.rows_valid = kSparse ? p.heads_q : min(kMlaRows, (p.seqlen_q - g.tok0) * p.heads_q);
   }
   if (kSparse)
-    g.units = (p.topk + kMlaBN - 1) / kMlaBN;
+    g.units = (p.topk * p.sbs + kMlaBN - 1) / kMlaBN;
   else
     g.units = g.len > 0 ? (g.len + kMlaBN - 1) / kMlaBN : 0;
+}
+
+// Key position of entry e of token tok's sparse list (-1: skipped): with
+// sparse_block_size bs, index k >= 0 lists positions k*bs .. k*bs + bs - 1.
+DEVI int mla_sparse_pos(const MlaParams& p, int b, int tok, int e) {
+  if (e >= p.topk * p.sbs) return -1;
+  const int blk = e / p.sbs;
+  const int k = __ldg(p.indices + b * p.idx_sb + (int64_t)tok * p.idx_ss + blk);
+  return k >= 0 ? k * p.sbs + (e - blk * p.sbs) : -1;
 }
 
 // Token and head of tile row x.
@@ -277,9 +287,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       } else {
         // lane k gathers key t*32 + k: 8 async copies of 16 bytes per chunk
         // into the 128-byte-swizzled layout, or zeros if the entry is skipped.
-        const int e_idx = t * kMlaBN + lane;
-        int pos = -1;
-        if (e_idx < p.topk) pos = p.indices[g.b * p.idx_sb + g.tok0 * p.idx_ss + e_idx];
+        const int pos = mla_sparse_pos(p, g.b, g.tok0, t * kMlaBN + lane);
         const bool valid = pos >= 0 && pos < g.len;
         const __nv_bfloat16* src = nullptr;
         if (valid) src = p.kv + (int64_t)bt[pos / P] * p.kv_sblk + (int64_t)(pos % P) * p.kv_stok;
@@ -543,10 +551,9 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       }
       if (j + 1 < n && !mla_send_partial(bars, smem, tmem, lane, r, rank, gi + 1, sv_next)) return;
       if constexpr (kSparse) {
-        const int* idx = p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss + t * kMlaBN;
 #pragma unroll
         for (int c = 0; c < kMlaBN; ++c) {
-          const int pos = (t * kMlaBN + c < p.topk && valid_row) ? __ldg(idx + c) : -1;
+          const int pos = valid_row ? mla_sparse_pos(p, g.b, tok, t * kMlaBN + c) : -1;
           if (!(pos >= 0 && pos < g.len)) sv[c] = __float_as_uint(-INFINITY);
         }
       } else {
@@ -727,7 +734,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const int mode = kSparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
       if (!(meta_matches(p.meta, mode, p.batch, p.seqlen_q, p.heads_q, 1, p.page_size,
                          p.num_segs, kMlaBN, kMlaDqk, kMlaDv) &&
-            p.meta[kMetaNumCtas] == p.num_ctas && (!kSparse || p.meta[kMetaTopk] == p.topk))) {
+            p.meta[kMetaNumCtas] == p.num_ctas &&
+            (!kSparse || p.meta[kMetaTopk] == p.topk * p.sbs))) {
         raise_error(ATTN_DEVERR_META_MISMATCH, 90);
         s_bad = 1;
       }

@@ -192,6 +192,7 @@ typedef struct {
   int32_t num_ctas;
   int32_t* meta;
   size_t meta_bytes;
+  int32_t sparse_block_size;  /* ATTN_SCHED_MLA_SPARSE: as in mla_args          */
 } attn_sched_args;
 
 /* Bytes of `meta` needed for these arguments (host only, no device access). */
@@ -370,6 +371,11 @@ typedef struct {
   int32_t num_ctas;           /* the num_ctas given to attn_sched_metadata    */
   void* workspace;
   size_t workspace_bytes;
+  int32_t sparse_block_size;  /* mla_sparse_fwd: 0 or 1 = each index is one     */
+                              /* position; a power of two up to 128 = each     */
+                              /* index k >= 0 lists positions k*bs .. k*bs+bs-1 */
+                              /* (MindSpore sparse_flash_attention             */
+                              /* sparse_block_size); dense: must be 0 or 1     */
 } mla_args;
 
 /* Bytes of workspace for these arguments (host only; 0 when meta is NULL).  */

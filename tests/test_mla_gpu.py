@@ -140,3 +140,32 @@ def test_full_size_dense_sampled():
 def test_full_size_sparse_sampled():
     """The top-2048 sparse variant at full size; 3 sequences checked."""
     _sampled("mla_sparse", 2048)
+
+
+@pytest.mark.parametrize("bs,num_ctas", [(4, 3), (64, 0)])
+def test_sparse_block_indices(bs, num_ctas):
+    """sparse_block_size > 1 (MindSpore sparse_flash_attention): index k lists
+    positions k*bs .. k*bs + bs - 1; -1 entries and positions past the cache
+    end are skipped."""
+    lens, topk = [20, 300, 3000], 64
+    inp = W.make_mla(seqlens=lens, seqlen_q=2, num_heads_q=128, page_size=64, topk=topk,
+                     seed=5, device="cuda")
+    g = torch.Generator().manual_seed(bs)
+    idx = torch.full((3, 2, 1, topk), -1, dtype=torch.int32)
+    for b, L in enumerate(lens):
+        nb = -(-L // bs)
+        for i in range(2):
+            n = min(nb, topk - 3)
+            idx[b, i, 0, :n] = torch.randperm(nb, generator=g)[:n].sort().values.int()
+    inp.indices = idx.cuda()
+    meta = B.mla_metadata(inp.cache_seqlens, batch=3, seqlen_q=2, num_heads_q=128, page_size=64,
+                          topk=topk, num_ctas=num_ctas, sparse_block_size=bs)
+    out, lse = B.mla_sparse_fwd(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens,
+                                inp.indices, scale=inp.scale, meta=meta, num_ctas=num_ctas,
+                                sparse_block_size=bs)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    ro, rl = oracle.mla_sparse(to_f64(inp.q), to_f64(inp.kv_cache), inp.block_table.cpu().numpy(),
+                               lens, idx.numpy(), 512, inp.scale, block_size=bs)
+    assert_close_out(to_f64(out), ro, 1e-2)
+    assert_close_lse(lse.cpu().numpy(), rl)
