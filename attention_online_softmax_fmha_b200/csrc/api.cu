@@ -400,7 +400,6 @@ attn_status_t check_mla(const mla_args* a, bool sparse) {
   if (a->head_dim_qk != kMlaDqk || a->head_dim_v != kMlaDv) return ATTN_ERR_UNSUPPORTED;
   if (a->num_heads_kv != 1 || !mla_heads_ok(a->num_heads_q)) return ATTN_ERR_UNSUPPORTED;
   if (!pow2_in(a->page_size, 16, 256)) return ATTN_ERR_UNSUPPORTED;
-  if (sparse && a->causal) return ATTN_ERR_UNSUPPORTED;
   if (!sbs_ok(a->sparse_block_size) || (!sparse && a->sparse_block_size > 1))
     return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;

@@ -22,7 +22,8 @@
 //           (causal: key j visible to token i iff j <= i + L - s_q).
 //   sparse: segment = (sequence, token, head tile), keys = that token's
 //           listed positions in tiles of 32 entries; entries outside [0, L)
-//           are skipped.
+//           are skipped, and with causal (sparse_mode=3) those past
+//           i + L - s_q too.
 // Segments are split over persistent clusters by the scheduler metadata (a
 // metadata "CTA" is a cluster); split segments go through the combine kernel.
 //
@@ -523,7 +524,7 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     const bool valid_row = r < g.rows_valid && tok < p.seqlen_q;
     // dense: visible keys [0, hi]; causal aligns the last token with the last key
     int hi = g.len - 1;
-    if (!kSparse && p.causal) hi = min(hi, tok + g.len - p.seqlen_q);
+    if (p.causal) hi = min(hi, tok + g.len - p.seqlen_q);
     float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
     bool seen = false;
     // The partial scores of tile g + 1 go to the other CTA as soon as those of
@@ -554,7 +555,9 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
 #pragma unroll
         for (int c = 0; c < kMlaBN; ++c) {
           const int pos = valid_row ? mla_sparse_pos(p, g.b, tok, t * kMlaBN + c) : -1;
-          if (!(pos >= 0 && pos < g.len)) sv[c] = __float_as_uint(-INFINITY);
+          // sparse_mode=3 ("rightDownCausal"): also pos <= tok + L - s_q
+          if (!(pos >= 0 && pos < g.len && (!p.causal || pos <= hi)))
+            sv[c] = __float_as_uint(-INFINITY);
         }
       } else {
         const int k0 = t * kMlaBN;

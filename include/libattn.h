@@ -392,7 +392,8 @@ attn_status_t mla_fwd_paged(const mla_args* args, void* stream);
 /* As mla_fwd_paged, plus indices int32 (B, s_q, 1, topk): query token       */
 /* (b, i) attends to the listed logical positions p with                     */
 /* 0 <= p < cache_seqlens[b]; other entries (e.g. -1 padding) are skipped.   */
-/* No mask beyond the index set (sparse_mode=0).                             */
+/* causal = 0: no mask beyond the index set (sparse_mode=0); causal = 1:    */
+/* also p <= i + cache_seqlens[b] - s_q (sparse_mode=3, "rightDownCausal").   */
 /* meta from attn_sched_metadata(mode=ATTN_SCHED_MLA_SPARSE) or NULL.        */
 /* ------------------------------------------------------------------------ */
 attn_status_t mla_sparse_fwd(const mla_args* args, void* stream);

@@ -390,7 +390,7 @@ def mla_paged(q, kv_cache, block_table, cache_seqlens, head_dim_v, scale, causal
 
 
 def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, scale,
-               rows=None, block_size=1):
+               rows=None, block_size=1, causal=False):
     """q (B, s_q, H_q, 576); indices (B, s_q, 1, topk) logical positions. Query
     token (b, i) attends to the listed positions p with 0 <= p < L_b (each
     listed occurrence counts once); the others are skipped.
@@ -398,6 +398,8 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
     power of two up to 128): each index k >= 0 lists the block of positions
     k * block_size .. k * block_size + block_size - 1 (reading: the index
     counts blocks); negative indices are skipped.
+    causal (sparse_mode=3, "rightDownCausal"): a listed position p is also
+    required to satisfy p <= i + L_b - s_q (bottom-right alignment).
     Returns out (B, s_q, H_q, D_v) and lse (B, H_q, s_q)."""
     q = np.asarray(q, np.float64)
     kv = np.asarray(kv_cache, np.float64)
@@ -421,6 +423,8 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
                 idx = idx[idx >= 0]
                 idx = (idx[:, None] * block_size + np.arange(block_size)[None, :]).reshape(-1)
             idx = idx[(idx >= 0) & (idx < L)]
+            if causal:
+                idx = idx[idx <= i + L - Sq]
             rows_kv = kv[np.asarray(block_table[b], np.int64)[idx // page], idx % page, 0, :]
             vis = np.ones((len(hs), idx.size), dtype=bool)
             o, l = attention_rows(q[b, i, hs, :], rows_kv, rows_kv[:, :head_dim_v], scale, vis)

@@ -169,3 +169,24 @@ def test_sparse_block_indices(bs, num_ctas):
                                lens, idx.numpy(), 512, inp.scale, block_size=bs)
     assert_close_out(to_f64(out), ro, 1e-2)
     assert_close_lse(lse.cpu().numpy(), rl)
+
+
+def test_sparse_causal_right_down():
+    """sparse_mode=3 ("rightDownCausal"): listed positions past i + L - s_q are
+    skipped as well."""
+    lens = [40, 300, 3000]
+    inp = W.make_mla(seqlens=lens, seqlen_q=3, num_heads_q=128, page_size=64, topk=128,
+                     seed=6, device="cuda")
+    # make sure the last positions are listed, so the causal cut removes some
+    for b, L in enumerate(lens):
+        inp.indices[b, :, 0, -3:] = torch.tensor([L - 3, L - 2, L - 1], dtype=torch.int32)
+    meta = B.mla_metadata(inp.cache_seqlens, batch=3, seqlen_q=3, num_heads_q=128, page_size=64,
+                          topk=128)
+    out, lse = B.mla_sparse_fwd(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens,
+                                inp.indices, scale=inp.scale, meta=meta, causal=True)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    ro, rl = oracle.mla_sparse(to_f64(inp.q), to_f64(inp.kv_cache), inp.block_table.cpu().numpy(),
+                               lens, inp.indices.cpu().numpy(), 512, inp.scale, causal=True)
+    assert_close_out(to_f64(out), ro, 1e-2)
+    assert_close_lse(lse.cpu().numpy(), rl)

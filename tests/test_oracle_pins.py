@@ -462,3 +462,18 @@ def test_mla_sparse_blocks_covering_the_cache_equal_dense():
     o_1, _ = oracle.mla_sparse(q[:1, :1], ck, bt[:1], lens[:1],
                                np.array([[[[8, 9, 10, 11]]]]), Dv, 0.3)
     np.testing.assert_allclose(o_b, o_1, rtol=1e-12)
+
+
+def test_mla_sparse_causal_all_positions_equals_dense_causal():
+    """sparse_mode=3 (rightDownCausal) over the list of all positions is the
+    dense MLA attention with the bottom-right causal mask."""
+    lens, page, Hq, D, Dv = [9, 14], 4, 2, 10, 6
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    q = RNG.normal(size=(2, 3, Hq, D))
+    idx = np.full((2, 3, 1, 16), -1, np.int64)
+    for b, L in enumerate(lens):
+        idx[b, :, 0, :L] = np.arange(L)
+    o_s, l_s = oracle.mla_sparse(q, ck, bt, lens, idx, Dv, 0.3, causal=True)
+    o_d, l_d = oracle.mla_paged(q, ck, bt, lens, Dv, 0.3, causal=True)
+    np.testing.assert_allclose(o_s, o_d, rtol=1e-12)
+    np.testing.assert_allclose(l_s, l_d, rtol=1e-12)
