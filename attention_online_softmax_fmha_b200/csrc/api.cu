@@ -452,6 +452,8 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   p.page_size = a.page_size;
   p.topk = a.topk;
   p.sbs = a.sparse_block_size > 1 ? a.sparse_block_size : 1;
+  p.sbs_log2 = 0;
+  while ((1 << p.sbs_log2) < p.sbs) ++p.sbs_log2;
   p.tiles_per_token = ds.tiles_per_token;
   p.tokens_per_tile = ds.tokens_per_tile;
   p.row_tiles = ds.row_tiles;

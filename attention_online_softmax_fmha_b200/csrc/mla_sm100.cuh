@@ -101,6 +101,7 @@ struct MlaParams {
   int64_t idx_sb, idx_ss;
   int32_t batch, seqlen_q, heads_q, page_size, topk;
   int32_t sbs;              // sparse: positions per index (sparse_block_size, >= 1)
+  int32_t sbs_log2;         // log2(sbs) (sbs is a power of two)
   int32_t tiles_per_token;  // heads_q >= 128: heads_q / 128 (else 1)
   int32_t tokens_per_tile;  // heads_q < 128: 128 / heads_q (else 1)
   int32_t row_tiles;        // dense: row tiles per sequence
@@ -152,10 +153,10 @@ DEVI void mla_seg(const MlaParams& p, int s, MlaSeg& g) {
 // Key position of entry e of token tok's sparse list (-1: skipped): with
 // sparse_block_size bs, index k >= 0 lists positions k*bs .. k*bs + bs - 1.
 DEVI int mla_sparse_pos(const MlaParams& p, int b, int tok, int e) {
-  if (e >= p.topk * p.sbs) return -1;
-  const int blk = e / p.sbs;
+  if (e >= (p.topk << p.sbs_log2)) return -1;
+  const int blk = e >> p.sbs_log2;
   const int k = __ldg(p.indices + b * p.idx_sb + (int64_t)tok * p.idx_ss + blk);
-  return k >= 0 ? k * p.sbs + (e - blk * p.sbs) : -1;
+  return k >= 0 ? (k << p.sbs_log2) + (e & (p.sbs - 1)) : -1;
 }
 
 // Token and head of tile row x.
@@ -288,7 +289,13 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       } else {
         // lane k gathers key t*32 + k: 8 async copies of 16 bytes per chunk
         // into the 128-byte-swizzled layout, or zeros if the entry is skipped.
-        const int pos = mla_sparse_pos(p, g.b, g.tok0, t * kMlaBN + lane);
+        int pos = -1;
+        if (p.sbs_log2 == 0) {  // one key per index: the index itself
+          const int e_idx = t * kMlaBN + lane;
+          if (e_idx < p.topk) pos = p.indices[g.b * p.idx_sb + g.tok0 * p.idx_ss + e_idx];
+        } else {
+          pos = mla_sparse_pos(p, g.b, g.tok0, t * kMlaBN + lane);
+        }
         const bool valid = pos >= 0 && pos < g.len;
         const __nv_bfloat16* src = nullptr;
         if (valid) src = p.kv + (int64_t)bt[pos / P] * p.kv_sblk + (int64_t)(pos % P) * p.kv_stok;
@@ -525,6 +532,8 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     // dense: visible keys [0, hi]; causal aligns the last token with the last key
     int hi = g.len - 1;
     if (p.causal) hi = min(hi, tok + g.len - p.seqlen_q);
+    const int* idx_row =
+        kSparse ? p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss : nullptr;
     float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
     bool seen = false;
     // The partial scores of tile g + 1 go to the other CTA as soon as those of
@@ -554,10 +563,21 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       if constexpr (kSparse) {
 #pragma unroll
         for (int c = 0; c < kMlaBN; ++c) {
-          const int pos = valid_row ? mla_sparse_pos(p, g.b, tok, t * kMlaBN + c) : -1;
+          // Key position of entry e (see mla_sparse_pos); the index row of this
+          // token is read with contiguous loads when each index is one key.
+          const int e = t * kMlaBN + c;
+          int pos = -1;
+          if (valid_row && e < (p.topk << p.sbs_log2)) {
+            if (p.sbs_log2 == 0) {
+              pos = __ldg(idx_row + e);
+            } else {
+              const int k = __ldg(idx_row + (e >> p.sbs_log2));
+              pos = k >= 0 ? (k << p.sbs_log2) + (e & (p.sbs - 1)) : -1;
+            }
+          }
           // sparse_mode=3 ("rightDownCausal"): also pos <= tok + L - s_q
-          if (!(pos >= 0 && pos < g.len && (!p.causal || pos <= hi)))
-            sv[c] = __float_as_uint(-INFINITY);
+          // (hi = L - 1 without it)
+          if (!(pos >= 0 && pos <= hi)) sv[c] = __float_as_uint(-INFINITY);
         }
       } else {
         const int k0 = t * kMlaBN;
