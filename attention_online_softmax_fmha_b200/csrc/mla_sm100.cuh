@@ -561,23 +561,29 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       }
       if (j + 1 < n && !mla_send_partial(bars, smem, tmem, lane, r, rank, gi + 1, sv_next)) return;
       if constexpr (kSparse) {
+        // Key position of entry e (see mla_sparse_pos); visible iff
+        // 0 <= pos <= hi (hi = L - 1, or with sparse_mode=3, "rightDownCausal",
+        // also tok + L - s_q). One key per index: the index row is read with
+        // contiguous loads.
+        const int n_e = valid_row ? (p.topk << p.sbs_log2) : 0;
+        if (p.sbs_log2 == 0) {
+          const int* idx = idx_row + t * kMlaBN;
 #pragma unroll
-        for (int c = 0; c < kMlaBN; ++c) {
-          // Key position of entry e (see mla_sparse_pos); the index row of this
-          // token is read with contiguous loads when each index is one key.
-          const int e = t * kMlaBN + c;
-          int pos = -1;
-          if (valid_row && e < (p.topk << p.sbs_log2)) {
-            if (p.sbs_log2 == 0) {
-              pos = __ldg(idx_row + e);
-            } else {
+          for (int c = 0; c < kMlaBN; ++c) {
+            const int pos = (t * kMlaBN + c < n_e) ? __ldg(idx + c) : -1;
+            if (!(pos >= 0 && pos <= hi)) sv[c] = __float_as_uint(-INFINITY);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kMlaBN; ++c) {
+            const int e = t * kMlaBN + c;
+            int pos = -1;
+            if (e < n_e) {
               const int k = __ldg(idx_row + (e >> p.sbs_log2));
               pos = k >= 0 ? (k << p.sbs_log2) + (e & (p.sbs - 1)) : -1;
             }
+            if (!(pos >= 0 && pos <= hi)) sv[c] = __float_as_uint(-INFINITY);
           }
-          // sparse_mode=3 ("rightDownCausal"): also pos <= tok + L - s_q
-          // (hi = L - 1 without it)
-          if (!(pos >= 0 && pos <= hi)) sv[c] = __float_as_uint(-INFINITY);
         }
       } else {
         const int k0 = t * kMlaBN;
