@@ -65,14 +65,33 @@ def load_traffic():
         return json.load(f)
 
 
-def source_hash() -> str:
+# The source files each kernel family is built from (its own header, the
+# shared helpers, the host launch code and the C header).
+_FAMILY_SOURCES = {
+    "prefill_kernel": ["prefill_sm100.cuh"],
+    "decode_kernel": ["decode_paged.cuh", "sched.cuh", "combine.cuh"],
+    "mla_kernel": ["mla_sm100.cuh", "sched.cuh", "combine.cuh"],
+}
+
+
+def source_hash(kernel: str = None) -> str:
+    """Hash of the sources a kernel is built from (all kernel sources when
+    `kernel` is None); keys the committed ncu traffic figures."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "attention_online_softmax_fmha_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    family = None
+    if kernel is not None:
+        family = _FAMILY_SOURCES.get(kernel.split("<")[0])
+    names = sorted(os.listdir(csrc)) if family is None else sorted(
+        family + ["common.cuh", "api.cu"])
+    for name in names:
         if name.endswith((".cu", ".cuh")):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
+    if family is not None:
+        with open(os.path.join(ROOT, "include", "libattn.h"), "rb") as f:
+            h.update(b"libattn.h" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -450,7 +469,6 @@ def run_ours(args, rank, world, device):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
     peaks, peak_kind = load_peaks()
     traffic = load_traffic()
-    shash = source_hash()
     names = (args.only or list(WORKLOADS)) if args.all else [args.workload]
     if args.workload not in names:
         names.insert(0, args.workload)
@@ -489,7 +507,8 @@ def run_ours(args, rank, world, device):
             peak = peaks["hbm_gbs"]
             runit = "GB/s"
         tr = traffic.get(wl["kernel"])
-        tr_val = tr["bytes_per_launch"] if tr and tr.get("source_hash") == shash else None
+        tr_val = (tr["bytes_per_launch"]
+                  if tr and tr.get("source_hash") == source_hash(wl["kernel"]) else None)
         results[name] = {
             "value": value, "unit": wl["unit"], "ms_per_step": tot / args.steps,
             "roofline": {"bound": wl["bound"], "achieved": achieved, "peak": peak, "unit": runit,
