@@ -13,208 +13,17 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "decode_paged.cuh"
+#include "host.cuh"
 #include "mla_sm100.cuh"
-#include "prefill_sm100.cuh"
+#include "prefill_host.cuh"
 #include "sched.cuh"
 
 namespace attn {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Driver entry point for cuTensorMapEncodeTiled (fetched through the runtime
-// so the library does not link libcuda directly).
-// ---------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// A 4-D tiled map over (dim0 = D contiguous, dim1, dim2, dim3) with strides
-// in bytes for dims 1..3, a box of (box0, box1, box2, box3) and 128-byte
-// swizzle. Out-of-range elements of a box read as zero.
-bool encode_4d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize,
-               uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3, uint64_t s1, uint64_t s2,
-               uint64_t s3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {d0, d1, d2, d3};
-  cuuint64_t strides[3] = {s1 * esize, s2 * esize, s3 * esize};
-  cuuint32_t box[4] = {b0, b1, b2, b3};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int device_sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool stride_ok(int64_t s, int esize) { return s > 0 && ((s * esize) % 16) == 0; }
-
-template <typename K>
-cudaError_t set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-}
-
-attn_status_t launch_status(cudaError_t e) {
-  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
-}
-
-// ---------------------------------------------------------------------------
-// attn_fwd_varlen
-// ---------------------------------------------------------------------------
-template <int D, int kType, bool kMask>
-attn_status_t launch_prefill(int grid, const CUtensorMap& mq, const CUtensorMap& mk,
-                             const CUtensorMap& mv, const PrefillParams& p, cudaStream_t stream) {
-  using C = PrefillCfg<D, kType>;
-  auto kernel = prefill_kernel<D, kType, kMask>;
-  static bool configured = false;
-  if (!configured) {
-    // The warpgroups trade registers with setmaxnreg out of the block's
-    // launch allocation; that split is only valid at exactly this count.
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
-    if (fa.numRegs != kPrefillLaunchRegs) return ATTN_ERR_UNSUPPORTED;
-    if (set_smem(kernel, C::kSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
-    configured = true;
-  }
-  kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
-  return launch_status(cudaGetLastError());
-}
-
-template <int D, int kType>
-attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
-  using C = PrefillCfg<D, kType>;
-  const bool varlen = a.cu_seqlens_q != nullptr;
-  const CUtensorMapDataType dt = kType >= 2   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
-                                 : kType == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                              : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const int es = C::kInBytes;
-  const uint32_t bx = C::kChunkElems;
-  const uint64_t rows_q = varlen ? (uint64_t)a.total_q : (uint64_t)a.max_seqlen_q;
-  const uint64_t rows_k = varlen ? (uint64_t)a.total_k : (uint64_t)a.max_seqlen_k;
-  const uint64_t nb = varlen ? 1 : (uint64_t)a.batch;
-  const uint64_t qsb = varlen ? rows_q * a.q_stride_s : a.q_stride_b;
-  const uint64_t ksb = varlen ? rows_k * a.k_stride_s : a.k_stride_b;
-  const uint64_t vsb = varlen ? rows_k * a.v_stride_s : a.v_stride_b;
-  CUtensorMap mq, mk, mv;
-  if (!encode_4d(&mq, a.q, dt, es, D, a.num_heads_q, rows_q, nb, a.q_stride_h, a.q_stride_s, qsb,
-                 bx, 1, 128, 1) ||
-      !encode_4d(&mk, a.k, dt, es, D, a.num_heads_kv, rows_k, nb, a.k_stride_h, a.k_stride_s, ksb,
-                 bx, 1, kPrefillBN, 1) ||
-      !encode_4d(&mv, a.v, dt, es, D, a.num_heads_kv, rows_k, nb, a.v_stride_h, a.v_stride_s, vsb,
-                 bx, 1, kPrefillBN, 1))
-    return ATTN_ERR_INVALID_ARG;
-
-  PrefillParams p;
-  memset(&p, 0, sizeof(p));
-  p.out = a.out;
-  p.lse = a.lse;
-  p.cu_q = a.cu_seqlens_q;
-  p.cu_k = a.cu_seqlens_k;
-  p.sink = a.sink;
-  p.seqused_q = a.seqused_q;
-  p.seqused_k = a.seqused_k;
-  p.mask = a.mask;
-  p.m_sb = a.mask_stride_b;
-  p.m_sh = a.mask_stride_h;
-  p.m_ss = a.mask_stride_s;
-  p.q_descale = a.q_descale;
-  p.k_descale = a.k_descale;
-  p.v_descale = a.v_descale;
-  p.o_sb = a.o_stride_b;
-  p.o_ss = a.o_stride_s;
-  p.o_sh = a.o_stride_h;
-  p.lse_sb = varlen ? 0 : a.lse_stride_b;
-  p.lse_sh = a.lse_stride_h;
-  p.batch = a.batch;
-  p.seqlen_q = a.max_seqlen_q;
-  p.seqlen_k = a.max_seqlen_k;
-  p.num_units_q = (a.max_seqlen_q + kPrefillUnit - 1) / kPrefillUnit;
-  p.num_heads_q = a.num_heads_q;
-  p.num_heads_kv = a.num_heads_kv;
-  p.group = a.num_heads_q / a.num_heads_kv;
-  const int64_t total = (int64_t)p.num_units_q * a.batch * a.num_heads_q;
-  if (total > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
-  p.total_units = (int32_t)total;
-  p.scale_log2 = a.scale * kLog2e;
-  p.causal = a.causal;
-  p.window_left = a.window_left;
-  p.window_right = a.window_right;
-
-  const int sms = device_sm_count();
-  if (sms <= 0) return ATTN_ERR_CUDA;
-  const int grid = (int)std::min<int64_t>(total, sms);
-  // The additive-mask path is a separate instantiation, so the common path
-  // carries none of its registers.
-  return a.mask ? launch_prefill<D, kType, true>(grid, mq, mk, mv, p, stream)
-                : launch_prefill<D, kType, false>(grid, mq, mk, mv, p, stream);
-}
-
-attn_status_t check_varlen(const attn_varlen_args* a) {
-  if (!a) return ATTN_ERR_INVALID_ARG;
-  if (!a->q || !a->k || !a->v || !a->out) return ATTN_ERR_INVALID_ARG;
-  const bool varlen = a->cu_seqlens_q != nullptr;
-  if (varlen != (a->cu_seqlens_k != nullptr)) return ATTN_ERR_INVALID_ARG;
-  if (a->batch <= 0 || a->max_seqlen_q <= 0 || a->max_seqlen_k <= 0) return ATTN_ERR_INVALID_ARG;
-  if (varlen && (a->total_q <= 0 || a->total_k <= 0)) return ATTN_ERR_INVALID_ARG;
-  if (a->num_heads_q <= 0 || a->num_heads_kv <= 0 || a->num_heads_q % a->num_heads_kv != 0)
-    return ATTN_ERR_INVALID_ARG;
-  if (a->head_dim_qk <= 0 || a->head_dim_v <= 0) return ATTN_ERR_INVALID_ARG;
-  if (!(a->scale > 0.f) || !std::isfinite(a->scale)) return ATTN_ERR_INVALID_ARG;
-  if (a->window_left < -1 || a->window_right < -1) return ATTN_ERR_INVALID_ARG;
-  if (a->dtype < ATTN_DTYPE_BF16 || a->dtype > ATTN_DTYPE_E5M2) return ATTN_ERR_INVALID_ARG;
-  const bool fp8 = a->dtype == ATTN_DTYPE_E4M3 || a->dtype == ATTN_DTYPE_E5M2;
-  if (fp8 && (!a->q_descale || !a->k_descale || !a->v_descale)) return ATTN_ERR_INVALID_ARG;
-  const int es = fp8 ? 1 : 2;
-  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
-    return ATTN_ERR_INVALID_ARG;
-  if (!stride_ok(a->q_stride_s, es) || !stride_ok(a->q_stride_h, es) ||
-      !stride_ok(a->k_stride_s, es) || !stride_ok(a->k_stride_h, es) ||
-      !stride_ok(a->v_stride_s, es) || !stride_ok(a->v_stride_h, es) ||
-      !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
-    return ATTN_ERR_INVALID_ARG;
-  if (!varlen && (!stride_ok(a->q_stride_b, es) || !stride_ok(a->k_stride_b, es) ||
-                  !stride_ok(a->v_stride_b, es) || !stride_ok(a->o_stride_b, 2)))
-    return ATTN_ERR_INVALID_ARG;
-  if (a->head_dim_qk != a->head_dim_v) return ATTN_ERR_UNSUPPORTED;
-  if (a->head_dim_qk != 64 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
-  if (fp8 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
-  if (varlen && (a->seqused_q || a->seqused_k)) return ATTN_ERR_INVALID_ARG;  // padded only
-  if (a->mask) {
-    if (a->mask_stride_b < 0 || a->mask_stride_h < 0 || a->mask_stride_s < 0)
-      return ATTN_ERR_INVALID_ARG;
-    // mask rows are read as 16-byte vectors
-    if (!aligned16(a->mask) || a->mask_stride_s % 4 || a->mask_stride_h % 4 ||
-        a->mask_stride_b % 4)
-      return ATTN_ERR_INVALID_ARG;
-  }
-  return ATTN_OK;
-}
-
-// ---------------------------------------------------------------------------
 // Scheduler metadata / paged decode / combine
 // ---------------------------------------------------------------------------
-bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
 
 // Segments and units of a decode problem (see sched.cuh).
 struct DecodeShape {
@@ -511,22 +320,7 @@ using namespace attn;
 extern "C" {
 
 attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream) {
-  const attn_status_t st = check_varlen(args);
-  if (st != ATTN_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int D = args->head_dim_qk;
-  switch (args->dtype) {
-    case ATTN_DTYPE_BF16:
-      return D == 64 ? run_prefill<64, 0>(*args, s) : run_prefill<128, 0>(*args, s);
-    case ATTN_DTYPE_FP16:
-      return D == 64 ? run_prefill<64, 1>(*args, s) : run_prefill<128, 1>(*args, s);
-    case ATTN_DTYPE_E4M3:
-      return run_prefill<128, 2>(*args, s);
-    case ATTN_DTYPE_E5M2:
-      return run_prefill<128, 3>(*args, s);
-    default:
-      return ATTN_ERR_UNSUPPORTED;
-  }
+  return varlen_entry(args, stream);
 }
 
 size_t attn_sched_metadata_size(const attn_sched_args* a) {

@@ -65,12 +65,12 @@ def load_traffic():
         return json.load(f)
 
 
-# The source files each kernel family is built from (its own header, the
-# shared helpers, the host launch code and the C header).
+# The sources each kernel family is built from: its device code, its
+# launch code and the shared device and host helpers.
 _FAMILY_SOURCES = {
-    "prefill_kernel": ["prefill_sm100.cuh"],
-    "decode_kernel": ["decode_paged.cuh", "sched.cuh", "combine.cuh"],
-    "mla_kernel": ["mla_sm100.cuh", "sched.cuh", "combine.cuh"],
+    "prefill_kernel": ["prefill_sm100.cuh", "prefill_host.cuh"],
+    "decode_kernel": ["decode_paged.cuh", "sched.cuh", "combine.cuh", "api.cu"],
+    "mla_kernel": ["mla_sm100.cuh", "sched.cuh", "combine.cuh", "api.cu"],
 }
 
 
@@ -84,14 +84,11 @@ def source_hash(kernel: str = None) -> str:
     if kernel is not None:
         family = _FAMILY_SOURCES.get(kernel.split("<")[0])
     names = sorted(os.listdir(csrc)) if family is None else sorted(
-        family + ["common.cuh", "api.cu"])
+        family + ["common.cuh", "host.cuh"])
     for name in names:
         if name.endswith((".cu", ".cuh")):
             with open(os.path.join(csrc, name), "rb") as f:
                 h.update(name.encode() + f.read())
-    if family is not None:
-        with open(os.path.join(ROOT, "include", "libattn.h"), "rb") as f:
-            h.update(b"libattn.h" + f.read())
     return h.hexdigest()[:16]
 
 
