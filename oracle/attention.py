@@ -310,10 +310,14 @@ def gather_pages(cache: np.ndarray, block_table_row: Sequence[int], length: int)
 
 
 def attention_paged(q, k_cache, v_cache, block_table, cache_seqlens, scale, causal=False,
-                    window=(-1, -1), sink=None, rows=None):
+                    window=(-1, -1), sink=None, rows=None, q_descale=None, k_descale=None,
+                    v_descale=None):
     """q (B, s_q, H_q, D); caches (num_blocks, page_size, H_kv, D) float64;
     block_table (B, max_pages); cache_seqlens (B,). The s_q query rows are the
     last s_q positions of the sequence (bottom-right alignment).
+    FP8 (MATE "Attention", FMHA FP8 paragraph, which covers the KV-cache call
+    too): q, k and v of sequence b and KV head g are multiplied by their
+    descale [b, g] (all three given or none).
     Returns out (B, s_q, H_q, D_v) and lse (B, H_q, s_q)."""
     q = np.asarray(q, np.float64)
     B, Sq, Hq, _ = q.shape
@@ -341,7 +345,12 @@ def attention_paged(q, k_cache, v_cache, block_table, cache_seqlens, scale, caus
                 lo, hi = visible_range(i, Sq, L, causal, window[0], window[1])
                 if lo <= hi:
                     vis[r, lo:hi + 1] = True
-            o, l = attention_rows(q[b, ii, h, :], ks[:, g, :], vs[:, g, :], scale, vis,
+            qh, kh, vh = q[b, ii, h, :], ks[:, g, :], vs[:, g, :]
+            if q_descale is not None:
+                qh = qh * float(q_descale[b][g])
+                kh = kh * float(k_descale[b][g])
+                vh = vh * float(v_descale[b][g])
+            o, l = attention_rows(qh, kh, vh, scale, vis,
                                   None if sink is None else float(sink[h]))
             out[b, ii, h, :] = o
             lse[b, h, ii] = l

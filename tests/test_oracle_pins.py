@@ -288,6 +288,28 @@ def test_paged_equals_contiguous(table):
         np.testing.assert_allclose(lse[b], l2, rtol=1e-13)
 
 
+def test_paged_descale_equals_varlen_descale_on_gathered_rows():
+    # the paged FP8 path scales per (sequence, KV head) exactly as the
+    # contiguous one does
+    lens, page, Hq, Hkv, D, sq = [7, 12], 4, 4, 2, 3, 2
+    ck, cv, bt = _paged_case(lens, page, Hkv, D, "permuted")
+    q = RNG.normal(size=(2, sq, Hq, D))
+    qd, kd, vd = (RNG.uniform(0.5, 2, size=(2, Hkv)) for _ in range(3))
+    out, lse = oracle.attention_paged(q, ck, cv, bt, lens, 0.6, causal=True, q_descale=qd,
+                                      k_descale=kd, v_descale=vd)
+    plain, _ = oracle.attention_paged(q, ck, cv, bt, lens, 0.6, causal=True)
+    assert np.abs(out - plain).max() > 1e-3  # the descales matter
+    for b, L in enumerate(lens):
+        kk = oracle.gather_pages(ck, bt[b], L)
+        vv = oracle.gather_pages(cv, bt[b], L)
+        cu_q, cu_k = np.array([0, sq]), np.array([0, L])
+        o2, l2 = oracle.attention_varlen(q[b], kk, vv, cu_q, cu_k, 0.6, True,
+                                         q_descale=qd[b:b + 1], k_descale=kd[b:b + 1],
+                                         v_descale=vd[b:b + 1])
+        np.testing.assert_allclose(out[b], o2, rtol=1e-13)
+        np.testing.assert_allclose(lse[b], l2, rtol=1e-13)
+
+
 def test_paged_aliased_table_repeats_one_page():
     page, L = 4, 10
     ck = RNG.normal(size=(1, page, 1, 3))
