@@ -70,7 +70,8 @@ class PagedArgs(ctypes.Structure):
                 ("dtype", c_i32), ("scale", c_f32), ("causal", c_i32),
                 ("window_left", c_i32), ("window_right", c_i32), ("sink", c_vp),
                 ("meta", c_vp), ("meta_bytes", c_sz), ("num_ctas", c_i32), ("workspace", c_vp),
-                ("workspace_bytes", c_sz)]
+                ("workspace_bytes", c_sz), ("q_descale", c_vp), ("k_descale", c_vp),
+                ("v_descale", c_vp)]
 
 
 class CombineArgs(ctypes.Structure):
@@ -273,7 +274,9 @@ def sched_metadata(cache_seqlens, *, stream=None, meta=None, **kw) -> torch.Tens
 
 def paged_args(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, causal=False,
                window=(-1, -1), sink=None, meta=None, num_ctas=0, workspace=None, out=None,
-               lse=None):
+               lse=None, q_descale=None, k_descale=None, v_descale=None):
+    """FP8 (float8_e4m3fn / float8_e5m2 q and caches, D = 128) takes
+    q/k/v_descale as contiguous fp32 (B, H_kv) device tensors."""
     B, sq, Hq, D = q.shape
     Hkv = k_cache.shape[2]
     if out is None:
@@ -290,7 +293,7 @@ def paged_args(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, c
         v_cache.stride(2), out.stride(0), out.stride(1), out.stride(2),
         _TORCH_DTYPE.get(q.dtype, -1), float(scale), int(bool(causal)), int(window[0]),
         int(window[1]), _ptr(sink), _ptr(meta), 0 if meta is None else meta.numel() * 4,
-        int(num_ctas), None, 0)
+        int(num_ctas), None, 0, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale))
     if meta is not None:
         nbytes = int(lib().attn_paged_workspace_size(ctypes.byref(a)))
         if workspace is None:

@@ -100,7 +100,9 @@ attn_status_t check_paged(const attn_paged_args* a) {
   if (a->dtype < ATTN_DTYPE_BF16 || a->dtype > ATTN_DTYPE_E5M2) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(a->q) || !aligned16(a->k_cache) || !aligned16(a->v_cache) || !aligned16(a->out))
     return ATTN_ERR_INVALID_ARG;
-  const int es = (a->dtype == ATTN_DTYPE_E4M3 || a->dtype == ATTN_DTYPE_E5M2) ? 1 : 2;
+  const bool fp8 = a->dtype == ATTN_DTYPE_E4M3 || a->dtype == ATTN_DTYPE_E5M2;
+  if (fp8 && (!a->q_descale || !a->k_descale || !a->v_descale)) return ATTN_ERR_INVALID_ARG;
+  const int es = fp8 ? 1 : 2;
   if (!stride_ok(a->q_stride_b, es) || !stride_ok(a->q_stride_s, es) ||
       !stride_ok(a->q_stride_h, es) || !stride_ok(a->kc_stride_blk, es) ||
       !stride_ok(a->kc_stride_tok, es) || !stride_ok(a->kc_stride_h, es) ||
@@ -108,8 +110,8 @@ attn_status_t check_paged(const attn_paged_args* a) {
       !stride_ok(a->vc_stride_h, es) || !stride_ok(a->o_stride_b, 2) ||
       !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
     return ATTN_ERR_INVALID_ARG;
-  if (a->dtype != ATTN_DTYPE_BF16 && a->dtype != ATTN_DTYPE_FP16) return ATTN_ERR_UNSUPPORTED;
   if (a->head_dim != 64 && a->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
+  if (fp8 && a->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
   if (!pow2_in(a->page_size, 16, 256)) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
@@ -119,17 +121,21 @@ size_t paged_ws_bytes(const attn_paged_args* a, const DecodeShape& ds) {
   return slots * kDecRows * a->head_dim * sizeof(float) + slots * kDecRows * sizeof(float) + 256;
 }
 
-template <int D, bool kFp16>
+// kType: 0 bf16, 1 fp16, 2 e4m3, 3 e5m2 (q and both caches).
+template <int D, int kType>
 attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaStream_t stream) {
-  using C = DecodeCfg<D>;
-  const CUtensorMapDataType dt =
-      kFp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  using C = DecodeCfg<D, (kType >= 2)>;
+  const CUtensorMapDataType dt = kType >= 2   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : kType == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const uint32_t box_rows = a.page_size >= kDecTileKeys ? kDecTileKeys : a.page_size;
   CUtensorMap mk, mv;
-  if (!encode_4d(&mk, a.k_cache, dt, 2, D, a.num_heads_kv, a.page_size, a.num_blocks,
-                 a.kc_stride_h, a.kc_stride_tok, a.kc_stride_blk, 64, 1, box_rows, 1) ||
-      !encode_4d(&mv, a.v_cache, dt, 2, D, a.num_heads_kv, a.page_size, a.num_blocks,
-                 a.vc_stride_h, a.vc_stride_tok, a.vc_stride_blk, 64, 1, box_rows, 1))
+  if (!encode_4d(&mk, a.k_cache, dt, C::kElt, D, a.num_heads_kv, a.page_size, a.num_blocks,
+                 a.kc_stride_h, a.kc_stride_tok, a.kc_stride_blk, C::kChunkCols, 1, box_rows,
+                 1) ||
+      !encode_4d(&mv, a.v_cache, dt, C::kElt, D, a.num_heads_kv, a.page_size, a.num_blocks,
+                 a.vc_stride_h, a.vc_stride_tok, a.vc_stride_blk, C::kChunkCols, 1, box_rows,
+                 1))
     return ATTN_ERR_INVALID_ARG;
   DecodeParams p;
   memset(&p, 0, sizeof(p));
@@ -140,6 +146,9 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
   p.cache_seqlens = a.cache_seqlens;
   p.meta = a.meta;
   p.sink = a.sink;
+  p.q_descale = a.q_descale;
+  p.k_descale = a.k_descale;
+  p.v_descale = a.v_descale;
   p.bt_stride = a.block_table_stride;
   p.q_sb = a.q_stride_b;
   p.q_ss = a.q_stride_s;
@@ -167,7 +176,7 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
     p.ws_o = reinterpret_cast<float*>(a.workspace);
     p.ws_lse = p.ws_o + slots * kDecRows * D;
   }
-  auto kernel = decode_kernel<D, kFp16>;
+  auto kernel = decode_kernel<D, kType>;
   static bool configured = false;
   if (!configured) {
     if (set_smem(kernel, C::kSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -179,7 +188,7 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
   if (a.meta) {
     const int64_t warps = (int64_t)ds.S * kDecRows;
     const int blocks = (int)((warps + 7) / 8);
-    decode_combine_kernel<D, kFp16><<<blocks, 256, 0, stream>>>(p);
+    decode_combine_kernel<D, kType == 1><<<blocks, 256, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
@@ -387,10 +396,18 @@ attn_status_t attn_fwd_paged_kvcache(const attn_paged_args* a, void* stream) {
     if (!aligned16(a->workspace)) return ATTN_ERR_INVALID_ARG;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool f16 = a->dtype == ATTN_DTYPE_FP16;
-  if (a->head_dim == 64)
-    return f16 ? run_decode<64, true>(*a, ds, s) : run_decode<64, false>(*a, ds, s);
-  return f16 ? run_decode<128, true>(*a, ds, s) : run_decode<128, false>(*a, ds, s);
+  switch (a->dtype) {
+    case ATTN_DTYPE_BF16:
+      return a->head_dim == 64 ? run_decode<64, 0>(*a, ds, s) : run_decode<128, 0>(*a, ds, s);
+    case ATTN_DTYPE_FP16:
+      return a->head_dim == 64 ? run_decode<64, 1>(*a, ds, s) : run_decode<128, 1>(*a, ds, s);
+    case ATTN_DTYPE_E4M3:
+      return run_decode<128, 2>(*a, ds, s);
+    case ATTN_DTYPE_E5M2:
+      return run_decode<128, 3>(*a, ds, s);
+    default:
+      return ATTN_ERR_UNSUPPORTED;
+  }
 }
 
 attn_status_t attn_combine(const attn_combine_args* a, void* stream) {

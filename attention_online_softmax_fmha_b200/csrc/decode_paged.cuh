@@ -19,6 +19,11 @@
 //               fp32 accumulation; their cost is far below the tile's load
 //               time. At the end of a segment piece the four warp states are
 //               merged through shared memory.
+// FP8 caches (e4m3 / e5m2, D = 128) arrive as 128-byte rows; each warp
+// rewrites its 16 keys of K and V as fp16 (exact for both formats) in a
+// private staging tile, releases the stage and runs the fp16 MMAs from
+// there. The q/k descales fold into the score scale and the v descale into
+// the output scale.
 // A piece that is the whole segment writes O (bf16) and LSE directly; a piece
 // of a split segment writes a sink-free partial (O / l, LSE) to the workspace
 // for the combine kernel.
@@ -43,6 +48,9 @@ struct DecodeParams {
   float* ws_o;               // [slot][kDecRows][D]
   float* ws_lse;             // [slot][kDecRows]
   const float* sink;
+  const float* q_descale;    // FP8: (B, H_kv) fp32, else unused
+  const float* k_descale;
+  const float* v_descale;
   int64_t bt_stride;
   int64_t q_sb, q_ss, q_sh;
   int64_t o_sb, o_ss, o_sh;
@@ -53,15 +61,21 @@ struct DecodeParams {
   int32_t causal, window_left, window_right;
 };
 
-template <int D>
+template <int D, bool kFp8>
 struct DecodeCfg {
-  static constexpr int kChunks = D / 64;
-  static constexpr int kTileBytes = kDecTileKeys * D * 2;  // K or V tile
+  static_assert(!kFp8 || D == 128, "FP8 caches: D = 128 (one 128-byte chunk per row)");
+  static constexpr int kElt = kFp8 ? 1 : 2;                    // bytes per cached element
+  static constexpr int kChunkCols = 128 / kElt;                // columns per 128-byte chunk
+  static constexpr int kChunks = D / kChunkCols;
+  static constexpr int kTileBytes = kDecTileKeys * D * kElt;  // K or V tile
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kQStride = D * 2 + 16;               // padded Q row (bytes)
+  static constexpr int kQStride = D * 2 + 16;                  // padded 16-bit Q row (bytes)
   static constexpr int kStageOff = 0;
   static constexpr int kQOff = kDecStages * kStageBytes;
-  static constexpr int kRedOff = kQOff + kDecRows * kQStride;  // merge buffers
+  // FP8: each consumer warp's fp16 copy of its 16 keys of K, then of V
+  static constexpr int kStgWarpBytes = kFp8 ? 2 * 16 * D * 2 : 0;
+  static constexpr int kStgOff = kQOff + kDecRows * kQStride;
+  static constexpr int kRedOff = kStgOff + 4 * kStgWarpBytes;  // merge buffers
   static constexpr int kRedBytes = kDecRows * D * 4 + 4 * kDecRows * 4 * 3;
   static constexpr int kBarOff = kRedOff + kRedBytes;
   static constexpr int kSmemBytes = kBarOff + 2 * kDecStages * 8 + 64 + 1024;
@@ -132,13 +146,37 @@ DEVI uint32_t sw128_addr(uint32_t base, int rows, int row, int col) {
   return base + chunk * rows * 128 + row * 128 + ((c16 ^ (row & 7)) << 4);
 }
 
+// Sixteen FP8 values (one 16-byte unit of a cached row) as fp16 into columns
+// col .. col + 15 of `row` of a 128-byte-swizzled fp16 tile of 16 rows.
+template <int kType>
+DEVI void fp8x16_to_f16_tile(uint32_t tile, int row, int col, uint4 w) {
+  const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+  uint32_t h[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const unsigned short lo = (unsigned short)(in[i] & 0xffffu);
+    const unsigned short hi = (unsigned short)(in[i] >> 16);
+    if constexpr (kType == 3) {
+      asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h[2 * i]) : "h"(lo));
+      asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h[2 * i + 1]) : "h"(hi));
+    } else {
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * i]) : "h"(lo));
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2 * i + 1]) : "h"(hi));
+    }
+  }
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sw128_addr(tile, 16, row, col)),
+               "r"(h[0]), "r"(h[1]), "r"(h[2]), "r"(h[3]) : "memory");
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(sw128_addr(tile, 16, row, col + 8)),
+               "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7]) : "memory");
+}
+
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool kFp8>
 DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CUtensorMap* mv,
                           uint8_t* smem, uint64_t* full, uint64_t* empty, volatile int* abort,
                           int seg_begin_units, int seg_end_units, int first_seg,
                           const int32_t* seg_prefix) {
-  using C = DecodeCfg<D>;
+  using C = DecodeCfg<D, kFp8>;
   const int lane = threadIdx.x & 31;
   if (lane == 0) {
     tma_prefetch_desc(mk);
@@ -185,7 +223,7 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
         if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
       }
       if (lane == 0)
-        mbar_expect_tx(&full[st], 2u * nload * box_rows * D * 2);
+        mbar_expect_tx(&full[st], 2u * nload * box_rows * D * C::kElt);
       __syncwarp();
       uint8_t* kdst = smem + C::kStageOff + st * C::kStageBytes;
       uint8_t* vdst = kdst + C::kTileBytes;
@@ -195,9 +233,9 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c) {
             tma_load_4d(kdst + c * kDecTileKeys * 128 + j * box_rows * 128, mk, &full[st],
-                        c * 64, sg.g, row_in_page, page);
+                        c * C::kChunkCols, sg.g, row_in_page, page);
             tma_load_4d(vdst + c * kDecTileKeys * 128 + j * box_rows * 128, mv, &full[st],
-                        c * 64, sg.g, row_in_page, page);
+                        c * C::kChunkCols, sg.g, row_in_page, page);
           }
         }
       }
@@ -215,12 +253,16 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
 }
 
 // ---------------------------------------------------------------------------
-template <int D, bool kFp16>
+// kType: 0 bf16, 1 fp16, 2 e4m3, 3 e5m2.
+template <int D, int kType>
 DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, uint64_t* empty,
                           volatile int* abort, int seg_begin_units, int seg_end_units,
                           int first_seg, const int32_t* seg_prefix) {
-  using C = DecodeCfg<D>;
-  using InT = typename std::conditional<kFp16, __half, __nv_bfloat16>::type;
+  constexpr bool kFp8 = kType >= 2;
+  constexpr bool kFp16 = kType != 0;      // MMA operand type: fp16 unless bf16
+  constexpr bool kOutF16 = kType == 1;    // output: fp16 for fp16 input, else bf16
+  using C = DecodeCfg<D, kFp8>;
+  using InT = typename std::conditional<kOutF16, __half, __nv_bfloat16>::type;
   const int tid = threadIdx.x;  // 0..127
   const int warp = tid >> 5, lane = tid & 31;
   const int qr = lane >> 2;          // fragment row (and row + 8)
@@ -258,9 +300,23 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       if (r < nrows) {
         const int rr = row0 + r;
         const int i = rr / p.group, h = sg.g * p.group + rr % p.group;
-        const InT* src = reinterpret_cast<const InT*>(p.q) + sg.b * p.q_sb + i * p.q_ss +
-                         h * p.q_sh + c8 * 8;
-        v = *reinterpret_cast<const uint4*>(src);
+        const int64_t off = sg.b * p.q_sb + i * p.q_ss + h * p.q_sh + c8 * 8;
+        if constexpr (kFp8) {
+          const uint2 w = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(p.q) +
+                                                          off);
+          const unsigned short* b2 = reinterpret_cast<const unsigned short*>(&w);
+          uint32_t h4[4];
+#pragma unroll
+          for (int x2 = 0; x2 < 4; ++x2) {
+            if constexpr (kType == 3)
+              asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h4[x2]) : "h"(b2[x2]));
+            else
+              asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h4[x2]) : "h"(b2[x2]));
+          }
+          v = make_uint4(h4[0], h4[1], h4[2], h4[3]);
+        } else {
+          v = *reinterpret_cast<const uint4*>(reinterpret_cast<const InT*>(p.q) + off);
+        }
       }
       *reinterpret_cast<uint4*>(qs + r * C::kQStride + c8 * 16) = v;
     }
@@ -291,7 +347,15 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
     for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_run[2] = {0.f, 0.f}, l_rnd[2] = {0.f, 0.f};
-    const float sl2 = p.scale_log2;
+    float sl2 = p.scale_log2, vscale = 1.f;
+    if constexpr (kFp8) {
+      const int di = sg.b * p.heads_kv + sg.g;
+      sl2 *= p.q_descale[di] * p.k_descale[di];
+      vscale = p.v_descale[di];
+    }
+    // FP8: this warp's fp16 K and V tiles (16 keys each)
+    const uint32_t kstg = smem_u32(smem + C::kStgOff + warp * C::kStgWarpBytes);
+    const uint32_t vstg = kstg + 16 * D * 2;
 
     for (int t = a; t < e; ++t) {
       if (t < sg.t0 || t >= sg.t1) continue;
@@ -300,9 +364,30 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       const uint32_t kbase = smem_u32(smem + C::kStageOff + st * C::kStageBytes);
       const uint32_t vbase = kbase + C::kTileBytes;
       const int key0 = t * kDecTileKeys + warp * 16;  // this warp's first key
-      // Keys past the end of the sequence hold whatever the page has there:
-      // zero their V rows so that P = 0 never meets a NaN.
-      if (key0 + 16 > sg.len) {
+      if constexpr (kFp8) {
+        // FP8 -> fp16 staging of this warp's 16 keys; V rows past the end of
+        // the sequence become zeros (P = 0 must not meet a NaN there).
+        __syncwarp();  // the previous tile's reads of the staging are done
+        const uint8_t* kt = smem + C::kStageOff + st * C::kStageBytes;
+        const uint8_t* vt = kt + C::kTileBytes;
+#pragma unroll
+        for (int x = lane; x < 16 * (D / 16); x += 32) {
+          const int kr = x / (D / 16), u = x % (D / 16);
+          const int row = warp * 16 + kr;
+          const int so = row * 128 + ((u ^ (row & 7)) << 4);
+          const uint4 kw = *reinterpret_cast<const uint4*>(kt + so);
+          uint4 vw = *reinterpret_cast<const uint4*>(vt + so);
+          if (key0 + kr >= sg.len) vw = make_uint4(0, 0, 0, 0);
+          fp8x16_to_f16_tile<kType>(kstg, kr, u * 16, kw);
+          fp8x16_to_f16_tile<kType>(vstg, kr, u * 16, vw);
+        }
+        // the stage is no longer read by this warp
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      } else if (key0 + 16 > sg.len) {
+        // Keys past the end of the sequence hold whatever the page has there:
+        // zero their V rows so that P = 0 never meets a NaN.
         for (int x = lane; x < 16 * (D / 8); x += 32) {
           const int kr = x / (D / 8), c8 = x % (D / 8);
           if (key0 + kr >= sg.len) {
@@ -312,15 +397,20 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         }
         __syncwarp();
       }
+      // The MMA operands: the stage itself, or for FP8 this warp's staging.
+      const uint32_t kop = kFp8 ? kstg : kbase;
+      const uint32_t vop = kFp8 ? vstg : vbase;
+      constexpr int kOpRows = kFp8 ? 16 : kDecTileKeys;
+      const int row0w = kFp8 ? 0 : warp * 16;
       // S = Q K^T for this warp's 16 keys: two n-tiles of 8 keys
       float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       {
-        const int kr = warp * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int kr = row0w + (lane & 7) + ((lane >> 4) << 3);
         const int cofs = ((lane >> 3) & 1) * 8;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           uint32_t b[4];
-          ldsm_x4(sw128_addr(kbase, kDecTileKeys, kr, k * 16 + cofs), b);
+          ldsm_x4(sw128_addr(kop, kOpRows, kr, k * 16 + cofs), b);
           mma16816<kFp16>(sacc[0], qa[k], b[0], b[1]);
           mma16816<kFp16>(sacc[1], qa[k], b[2], b[3]);
         }
@@ -370,20 +460,22 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         }
       // O += P V over this warp's 16 keys: 16 d-tiles of 8
       {
-        const int kr = warp * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int kr = row0w + (lane & 7) + (((lane >> 3) & 1) << 3);
         const int cofs = (lane >> 4) * 8;
 #pragma unroll
         for (int n2 = 0; n2 < D / 16; ++n2) {
           uint32_t b[4];
-          ldsm_x4_t(sw128_addr(vbase, kDecTileKeys, kr, n2 * 16 + cofs), b);
+          ldsm_x4_t(sw128_addr(vop, kOpRows, kr, n2 * 16 + cofs), b);
           mma16816<kFp16>(o[2 * n2], pa, b[0], b[1]);
           mma16816<kFp16>(o[2 * n2 + 1], pa, b[2], b[3]);
         }
       }
-      // this warp is done with the stage (zeroed rows included)
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
+      if constexpr (!kFp8) {
+        // this warp is done with the stage (zeroed rows included)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
       ++it;
     }
 
@@ -448,21 +540,21 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         if (slot < 0) {
           float denom = LR;
           if (p.sink) denom += ex2(p.sink[h] * kLog2e - m_use);
-          const float inv = denom > 0.f ? 1.f / denom : 0.f;
+          const float inv = denom > 0.f ? vscale / denom : 0.f;
           InT* dst = reinterpret_cast<InT*>(p.out) + sg.b * p.o_sb + i * p.o_ss + h * p.o_sh + c0;
 #pragma unroll
           for (int c = 0; c < kPer; c += 8) {
             uint4 w;
-            w.x = pack2<kFp16>(red_o[r * D + c0 + c] * inv, red_o[r * D + c0 + c + 1] * inv);
-            w.y = pack2<kFp16>(red_o[r * D + c0 + c + 2] * inv, red_o[r * D + c0 + c + 3] * inv);
-            w.z = pack2<kFp16>(red_o[r * D + c0 + c + 4] * inv, red_o[r * D + c0 + c + 5] * inv);
-            w.w = pack2<kFp16>(red_o[r * D + c0 + c + 6] * inv, red_o[r * D + c0 + c + 7] * inv);
+            w.x = pack2<kOutF16>(red_o[r * D + c0 + c] * inv, red_o[r * D + c0 + c + 1] * inv);
+            w.y = pack2<kOutF16>(red_o[r * D + c0 + c + 2] * inv, red_o[r * D + c0 + c + 3] * inv);
+            w.z = pack2<kOutF16>(red_o[r * D + c0 + c + 4] * inv, red_o[r * D + c0 + c + 5] * inv);
+            w.w = pack2<kOutF16>(red_o[r * D + c0 + c + 6] * inv, red_o[r * D + c0 + c + 7] * inv);
             *reinterpret_cast<uint4*>(dst + c) = w;
           }
           if (p.lse && (tid & 7) == 0)
             p.lse[((int64_t)sg.b * p.heads_q + h) * p.seqlen_q + i] = lse2 * kLn2;
         } else {
-          const float inv = LR > 0.f ? 1.f / LR : 0.f;
+          const float inv = LR > 0.f ? vscale / LR : 0.f;
           float* dst = p.ws_o + ((int64_t)slot * kDecRows + r) * D + c0;
 #pragma unroll
           for (int c = 0; c < kPer; c += 4)
@@ -478,11 +570,12 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
   }
 }
 
-template <int D, bool kFp16>
+template <int D, int kType>
 __global__ void __launch_bounds__(160, 1)
     decode_kernel(const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v, const DecodeParams p) {
-  using C = DecodeCfg<D>;
+  constexpr bool kFp8 = kType >= 2;
+  using C = DecodeCfg<D, kFp8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -529,9 +622,10 @@ __global__ void __launch_bounds__(160, 1)
     if (ue == 0) ue = 1;  // still write O = 0, LSE = -inf for an empty sequence
   }
   if (threadIdx.x >= 128) {
-    decode_producer<D>(p, &map_k, &map_v, smem, full, empty, abort, ub, ue, s0, seg_prefix);
+    decode_producer<D, kFp8>(p, &map_k, &map_v, smem, full, empty, abort, ub, ue, s0,
+                             seg_prefix);
   } else {
-    decode_consumer<D, kFp16>(p, smem, full, empty, abort, ub, ue, s0, seg_prefix);
+    decode_consumer<D, kType>(p, smem, full, empty, abort, ub, ue, s0, seg_prefix);
   }
 }
 

@@ -167,6 +167,9 @@ class PagedInputs:
     scale: float
     sink: Optional[torch.Tensor]
     dtype: str
+    q_descale: Optional[torch.Tensor] = None   # FP8: fp32 (B, H_kv) in [0.5, 2]
+    k_descale: Optional[torch.Tensor] = None
+    v_descale: Optional[torch.Tensor] = None
 
     @property
     def batch(self) -> int:
@@ -212,11 +215,15 @@ def make_paged(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, num_h
     vc = _values((nblocks, page_size, num_heads_kv, head_dim), dtype, g, device)
     sink_t = (torch.randn(num_heads_q, generator=g, device=device, dtype=torch.float32)
               if sink else None)
+    desc = [None, None, None]
+    if dtype in _FP8:
+        desc = [torch.rand(B, num_heads_kv, generator=g, device=device) * 1.5 + 0.5
+                for _ in range(3)]
     if scale is None:
         scale = 1.0 / math.sqrt(head_dim)
     return PagedInputs(q, kc, vc, bt.to(device), torch.tensor(seqlens, dtype=torch.int32,
                        device=device), seqlens, page_size, num_heads_q, num_heads_kv, head_dim,
-                       bool(causal), tuple(window), float(scale), sink_t, dtype)
+                       bool(causal), tuple(window), float(scale), sink_t, dtype, *desc)
 
 
 @dataclasses.dataclass
@@ -303,6 +310,10 @@ CONFIGS = {
                        head_dim=128, varlen=False, causal=True, mask=True),
     "paged_decode": dict(kind="paged", lengths=(64, 1024, 32768), seqlen_q=1, num_heads_q=32,
                          num_heads_kv=8, head_dim=128, page_size=64),
+    # the same decode against an e4m3 cache with per-(sequence, KV head) descales
+    "paged_decode_fp8": dict(kind="paged", lengths=(64, 1024, 32768), seqlen_q=1,
+                             num_heads_q=32, num_heads_kv=8, head_dim=128, page_size=64,
+                             dtype="e4m3"),
     # the same decode with 16 sequences (about 1.1 GB of cache), for profiler
     # captures that must stay small
     "paged_decode_small": dict(kind="paged", lengths=(16, 1024, 32768), seqlen_q=1,

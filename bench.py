@@ -244,13 +244,18 @@ def paged_workload(name: str, seed: int, device):
     sa.meta_bytes = meta.numel() * 4
     pa, out, lse, ws = B.paged_args(inp.q, inp.k_cache, inp.v_cache, inp.block_table,
                                     inp.cache_seqlens, scale=inp.scale, causal=inp.causal,
-                                    window=inp.window, sink=inp.sink, meta=meta)
+                                    window=inp.window, sink=inp.sink, meta=meta,
+                                    q_descale=inp.q_descale, k_descale=inp.k_descale,
+                                    v_descale=inp.v_descale)
     # algorithmic bytes: every visible K and V row once per KV head, Q, O, LSE,
-    # the used block-table entries and cache_seqlens
+    # the used block-table entries and cache_seqlens (and the FP8 descales)
     kv_rows = sum(inp.seqlens)
     pages = sum(-(-x // inp.page_size) for x in inp.seqlens)
-    nbytes = (kv_rows * Hkv * 2 * D * 2 + inp.q.numel() * 2 + out.numel() * 2 + lse.numel() * 4
-              + pages * 4 + B_ * 4)
+    es = inp.k_cache.element_size()
+    fp8 = inp.q_descale is not None
+    nbytes = (kv_rows * Hkv * 2 * D * es + inp.q.numel() * inp.q.element_size()
+              + out.numel() * 2 + lse.numel() * 4 + pages * 4 + B_ * 4
+              + (3 * B_ * Hkv * 4 if fp8 else 0))
 
     def step(stream):
         st = L.attn_sched_metadata(ctypes.byref(sa), stream.cuda_stream)
@@ -279,11 +284,11 @@ def paged_workload(name: str, seed: int, device):
            "cache_seqlens": "uniform[1024,32768]", "block_table": "seeded permutation",
            "kv_tokens": kv_rows, "dtype": inp.dtype}
     return dict(step=step, e2e_step=e2e_step, work=nbytes / 1e9, unit="GB/s", bound="hbm",
-                kernel="decode_kernel<128>", launches_per_step=3,
+                kernel="decode_kernel<128,%d>" % (2 if fp8 else 0), launches_per_step=3,
                 h2d=sum(t.numel() * t.element_size() for t in host_small),
                 d2h=sum(t.numel() * t.element_size() for t in host_out), cfg=cfg,
                 dtype=inp.dtype, inp=inp, keep=(meta, ws, out, lse),
-                per_unit=f"(D_k + D_v) * 2 B per cached token per KV head + Q/O/LSE/table; "
+                per_unit=f"(D_k + D_v) * {es} B per cached token per KV head + Q/O/LSE/table; "
                 f"{nbytes} B per step")
 
 
@@ -357,6 +362,7 @@ WORKLOADS = {
     "dense_mask": prefill_workload,
     "paged_decode": paged_workload,
     "paged_decode_small": paged_workload,
+    "paged_decode_fp8": paged_workload,
     "mla_dense": mla_workload,
     "mla_sparse": mla_workload,
     "mla_dense_small": mla_workload,

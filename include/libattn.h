@@ -215,13 +215,21 @@ attn_status_t attn_sched_metadata(const attn_sched_args* args, void* stream);
 /* (B,) = L_b; the s_q query rows are the last s_q positions (delta =        */
 /* L_b - s_q). out (B, s_q, H_q, D) bf16 (fp16 for fp16 input); lse (B, H_q, */
 /* s_q) fp32, nullable.                                                     */
+/* FP8 (dtype e4m3 or e5m2; q and both caches in that format, D = 128):     */
+/*   q_descale, k_descale, v_descale fp32 (B, H_kv), all required: the      */
+/*   values of sequence b and KV head g are the stored codes times their     */
+/*   descale [b][g] (MATE "Attention", FMHA FP8 paragraph). out is bf16.     */
+/*   The descales are ignored for bf16 and fp16 input.                      */
 /* meta: from attn_sched_metadata(mode=ATTN_SCHED_MHA, same args), or NULL   */
 /*   for one CTA per (sequence, KV head) and no splitting.                   */
 /* workspace: device buffer of attn_paged_workspace_size() bytes (partial   */
 /*   O and LSE of the splits); may be NULL when meta is NULL. The combine    */
 /*   step runs inside this call.                                             */
-/* Supported now: bf16, D in {64, 128}, page_size in {16, 32, 64, 128, 256}, */
-/*   s_q * H_q / H_kv <= 16.                                                 */
+/* Supported now: bf16 and fp16 with D in {64, 128}; e4m3 and e5m2 with     */
+/*   D = 128; page_size in {16, 32, 64, 128, 256}; s_q * H_q / H_kv <= 16.  */
+/* Errors: INVALID_ARG for NULL required pointers (the descales included    */
+/*   for FP8), bad sizes or misaligned strides; UNSUPPORTED outside the     */
+/*   supported shapes above.                                                 */
 /* ------------------------------------------------------------------------ */
 typedef struct {
   const void* q;
@@ -255,6 +263,9 @@ typedef struct {
   int32_t num_ctas;       /* the num_ctas given to attn_sched_metadata (0 = SMs) */
   void* workspace;
   size_t workspace_bytes;
+  const float* q_descale; /* FP8 only: (B, H_kv) fp32 */
+  const float* k_descale;
+  const float* v_descale;
 } attn_paged_args;
 
 /* Bytes of workspace for these arguments (host only; 0 when meta is NULL).  */

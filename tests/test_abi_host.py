@@ -88,6 +88,38 @@ def test_varlen_rejects_bad_arguments(L, over, want):
     assert L.attn_fwd_varlen(ctypes.byref(a), None) == want
 
 
+def _paged(**over):
+    a = B.PagedArgs()
+    base = dict(q=0x1000, k_cache=0x2000, v_cache=0x3000, block_table=0x4000,
+                cache_seqlens=0x5000, out=0x6000, batch=2, seqlen_q=1, num_heads_q=8,
+                num_heads_kv=2, head_dim=128, page_size=64, num_blocks=16, max_pages_per_seq=8,
+                block_table_stride=8, q_stride_b=8 * 128, q_stride_s=8 * 128, q_stride_h=128,
+                kc_stride_blk=64 * 2 * 128, kc_stride_tok=2 * 128, kc_stride_h=128,
+                vc_stride_blk=64 * 2 * 128, vc_stride_tok=2 * 128, vc_stride_h=128,
+                o_stride_b=8 * 128, o_stride_s=8 * 128, o_stride_h=128, dtype=B.DTYPE_BF16,
+                scale=0.1, window_left=-1, window_right=-1)
+    base.update(over)
+    for k, v in base.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("over,want", [
+    (dict(k_cache=None), B.INVALID_ARG),
+    (dict(num_heads_kv=3), B.INVALID_ARG),
+    (dict(block_table_stride=4), B.INVALID_ARG),    # shorter than a table row
+    (dict(dtype=B.DTYPE_E4M3), B.INVALID_ARG),      # FP8 without descales
+    (dict(dtype=B.DTYPE_E5M2, q_descale=8, k_descale=8), B.INVALID_ARG),
+    (dict(dtype=B.DTYPE_E4M3, q_descale=8, k_descale=8, v_descale=8, head_dim=64),
+     B.UNSUPPORTED),                                # FP8 is built for D = 128
+    (dict(head_dim=96), B.UNSUPPORTED),
+    (dict(page_size=8), B.UNSUPPORTED),
+])
+def test_paged_rejects_bad_arguments(L, over, want):
+    a = _paged(**over)
+    assert L.attn_fwd_paged_kvcache(ctypes.byref(a), None) == want
+
+
 def test_null_struct_is_invalid(L):
     for fn in ["attn_fwd_varlen", "attn_sched_metadata", "attn_fwd_paged_kvcache",
                "attn_combine", "mla_fwd_paged", "mla_sparse_fwd"]:

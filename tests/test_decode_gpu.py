@@ -21,11 +21,15 @@ def _lib():
     B.lib()
 
 
+def _np(t):
+    return None if t is None else t.cpu().double().numpy()
+
+
 def oracle_paged(inp, rows=None):
-    sink = None if inp.sink is None else inp.sink.cpu().numpy()
     return oracle.attention_paged(to_f64(inp.q), to_f64(inp.k_cache), to_f64(inp.v_cache),
                                   inp.block_table.cpu().numpy(), inp.seqlens, inp.scale,
-                                  inp.causal, inp.window, sink, rows)
+                                  inp.causal, inp.window, _np(inp.sink), rows,
+                                  _np(inp.q_descale), _np(inp.k_descale), _np(inp.v_descale))
 
 
 def run_paged(inp, use_meta=True, num_ctas=0):
@@ -38,16 +42,17 @@ def run_paged(inp, use_meta=True, num_ctas=0):
     out, lse = B.fwd_paged_kvcache(inp.q, inp.k_cache, inp.v_cache, inp.block_table,
                                    inp.cache_seqlens, scale=inp.scale, causal=inp.causal,
                                    window=inp.window, sink=inp.sink, meta=meta,
-                                   num_ctas=num_ctas)
+                                   num_ctas=num_ctas, q_descale=inp.q_descale,
+                                   k_descale=inp.k_descale, v_descale=inp.v_descale)
     torch.cuda.synchronize()
     assert B.device_error() == 0
     return out, lse, meta
 
 
-def check(inp, **kw):
+def check(inp, atol=1e-2, **kw):
     out, lse, _ = run_paged(inp, **kw)
     ro, rl = oracle_paged(inp)
-    assert_close_out(to_f64(out), ro, 1e-2)
+    assert_close_out(to_f64(out), ro, atol)
     assert_close_lse(lse.cpu().numpy(), rl)
 
 
@@ -88,6 +93,25 @@ def test_aliased_block_table_and_empty_sequence():
                        head_dim=128, page_size=16, table="aliased", seed=4, device="cuda")
     check(inp, num_ctas=4)
     check(inp, use_meta=False)
+
+
+# FP8 caches (e4m3 / e5m2, D = 128) with fp32 descales (B, H_kv), bf16 out:
+# max-abs 5e-2 (the FP8 bound), LSE 1e-3.
+@pytest.mark.parametrize("dtype", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("page", [32, 64, 128])
+def test_fp8_cache_split(dtype, page):
+    inp = W.make_paged(seqlens=LENS, seqlen_q=1, num_heads_q=8, num_heads_kv=2, head_dim=128,
+                       page_size=page, dtype=dtype, seed=20, device="cuda")
+    assert inp.k_cache.dtype != torch.bfloat16 and inp.q_descale is not None
+    check(inp, atol=5e-2, num_ctas=7)
+
+
+def test_fp8_cache_multi_token_causal_window_sink_no_metadata():
+    inp = W.make_paged(seqlens=[4, 90, 513, 0], seqlen_q=4, num_heads_q=16, num_heads_kv=2,
+                       head_dim=128, page_size=16, causal=True, window=(200, 0), sink=True,
+                       dtype="e4m3", seed=21, device="cuda")
+    check(inp, atol=5e-2, num_ctas=6)
+    check(inp, atol=5e-2, use_meta=False)
 
 
 @pytest.mark.parametrize("lens,G", [([0, 1, 64, 65, 4000, 12, 9000], 9),
