@@ -19,11 +19,11 @@
 //               fp32 accumulation; their cost is far below the tile's load
 //               time. At the end of a segment piece the four warp states are
 //               merged through shared memory.
-// FP8 caches (e4m3 / e5m2, D = 128) arrive as 128-byte rows; each warp
-// rewrites its 16 keys of K and V as fp16 (exact for both formats) in a
-// private staging tile, releases the stage and runs the fp16 MMAs from
-// there. The q/k descales fold into the score scale and the v descale into
-// the output scale.
+// FP8 caches (e4m3 / e5m2, D = 128) arrive as 128-byte rows. S = Q K^T runs
+// on the FP8 codes directly (mma.sync m16n8k32, Q kept in FP8); each warp
+// rewrites its 16 V rows as fp16 (exact for both formats) in a private
+// tile, and O += P V runs in fp16 from there. The q/k descales fold into the
+// score scale and the v descale into the output scale.
 // A piece that is the whole segment writes O (bf16) and LSE directly; a piece
 // of a split segment writes a sink-free partial (O / l, LSE) to the workspace
 // for the combine kernel.
@@ -72,8 +72,8 @@ struct DecodeCfg {
   static constexpr int kQStride = D * 2 + 16;                  // padded 16-bit Q row (bytes)
   static constexpr int kStageOff = 0;
   static constexpr int kQOff = kDecStages * kStageBytes;
-  // FP8: each consumer warp's fp16 copy of its 16 keys of K, then of V
-  static constexpr int kStgWarpBytes = kFp8 ? 2 * 16 * D * 2 : 0;
+  // FP8: each consumer warp's fp16 copy of its 16 V rows
+  static constexpr int kStgWarpBytes = kFp8 ? 16 * D * 2 : 0;
   static constexpr int kStgOff = kQOff + kDecRows * kQStride;
   static constexpr int kRedOff = kStgOff + 4 * kStgWarpBytes;  // merge buffers
   static constexpr int kRedBytes = kDecRows * D * 4 + 4 * kDecRows * 4 * 3;
@@ -129,6 +129,23 @@ DEVI void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
   } else {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+// FP8 x FP8 -> fp32, m16n8k32 (kType 3 = e5m2, otherwise e4m3).
+template <int kType>
+DEVI void mma16832_fp8(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  if constexpr (kType == 3) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e5m2.e5m2.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -292,41 +309,34 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
     const int row0 = sg.rsub * kDecRows;
     const int nrows = min(kDecRows, p.rows - row0);
 
-    // --- Q rows of the segment -> shared memory (bf16, zero padded) ---
+    // --- Q rows of the segment -> shared memory (16-bit, or the FP8 codes
+    //     as they are; zero padded) ---
     named_barrier(1, 128);  // previous piece finished with qs / red
-    for (int x = tid; x < kDecRows * (D / 8); x += 128) {
-      const int r = x / (D / 8), c8 = x % (D / 8);
+    constexpr int kQUnit = kFp8 ? 16 : 8;  // elements per 16-byte unit
+    for (int x = tid; x < kDecRows * (D / kQUnit); x += 128) {
+      const int r = x / (D / kQUnit), cu = x % (D / kQUnit);
       uint4 v = make_uint4(0, 0, 0, 0);
       if (r < nrows) {
         const int rr = row0 + r;
         const int i = rr / p.group, h = sg.g * p.group + rr % p.group;
-        const int64_t off = sg.b * p.q_sb + i * p.q_ss + h * p.q_sh + c8 * 8;
-        if constexpr (kFp8) {
-          const uint2 w = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint8_t*>(p.q) +
-                                                          off);
-          const unsigned short* b2 = reinterpret_cast<const unsigned short*>(&w);
-          uint32_t h4[4];
-#pragma unroll
-          for (int x2 = 0; x2 < 4; ++x2) {
-            if constexpr (kType == 3)
-              asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h4[x2]) : "h"(b2[x2]));
-            else
-              asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h4[x2]) : "h"(b2[x2]));
-          }
-          v = make_uint4(h4[0], h4[1], h4[2], h4[3]);
-        } else {
+        const int64_t off = sg.b * p.q_sb + i * p.q_ss + h * p.q_sh + cu * kQUnit;
+        if constexpr (kFp8)
+          v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.q) + off);
+        else
           v = *reinterpret_cast<const uint4*>(reinterpret_cast<const InT*>(p.q) + off);
-        }
       }
-      *reinterpret_cast<uint4*>(qs + r * C::kQStride + c8 * 16) = v;
+      *reinterpret_cast<uint4*>(qs + r * C::kQStride + cu * 16) = v;
     }
     named_barrier(1, 128);
-    uint32_t qa[D / 16][4];
+    // A fragments of Q: one per 32-byte k-step (16 bf16/fp16 values, or 32
+    // FP8 codes read through the same 16-bit ldmatrix view)
+    constexpr int kKSteps = D * C::kElt / 32;
+    uint32_t qa[kKSteps][4];
     {
       const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
       const int cofs = (lane >> 4) * 8;
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
+      for (int k = 0; k < kKSteps; ++k)
         ldsm_x4(smem_u32(qs + r * C::kQStride + (k * 16 + cofs) * 2), qa[k]);
     }
     // per-row visible key range (rows qr and qr + 8)
@@ -353,9 +363,8 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       sl2 *= p.q_descale[di] * p.k_descale[di];
       vscale = p.v_descale[di];
     }
-    // FP8: this warp's fp16 K and V tiles (16 keys each)
-    const uint32_t kstg = smem_u32(smem + C::kStgOff + warp * C::kStgWarpBytes);
-    const uint32_t vstg = kstg + 16 * D * 2;
+    // FP8: this warp's fp16 V tile (16 keys)
+    const uint32_t vstg = smem_u32(smem + C::kStgOff + warp * C::kStgWarpBytes);
 
     for (int t = a; t < e; ++t) {
       if (t < sg.t0 || t >= sg.t1) continue;
@@ -365,26 +374,18 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       const uint32_t vbase = kbase + C::kTileBytes;
       const int key0 = t * kDecTileKeys + warp * 16;  // this warp's first key
       if constexpr (kFp8) {
-        // FP8 -> fp16 staging of this warp's 16 keys; V rows past the end of
-        // the sequence become zeros (P = 0 must not meet a NaN there).
-        __syncwarp();  // the previous tile's reads of the staging are done
-        const uint8_t* kt = smem + C::kStageOff + st * C::kStageBytes;
-        const uint8_t* vt = kt + C::kTileBytes;
+        // FP8 -> fp16 copy of this warp's 16 V rows; rows past the end of the
+        // sequence become zeros (P = 0 must not meet a NaN there).
+        __syncwarp();  // the previous tile's reads of the copy are done
+        const uint8_t* vt = smem + C::kStageOff + st * C::kStageBytes + C::kTileBytes;
 #pragma unroll
         for (int x = lane; x < 16 * (D / 16); x += 32) {
           const int kr = x / (D / 16), u = x % (D / 16);
           const int row = warp * 16 + kr;
-          const int so = row * 128 + ((u ^ (row & 7)) << 4);
-          const uint4 kw = *reinterpret_cast<const uint4*>(kt + so);
-          uint4 vw = *reinterpret_cast<const uint4*>(vt + so);
+          uint4 vw = *reinterpret_cast<const uint4*>(vt + row * 128 + ((u ^ (row & 7)) << 4));
           if (key0 + kr >= sg.len) vw = make_uint4(0, 0, 0, 0);
-          fp8x16_to_f16_tile<kType>(kstg, kr, u * 16, kw);
           fp8x16_to_f16_tile<kType>(vstg, kr, u * 16, vw);
         }
-        // the stage is no longer read by this warp
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
       } else if (key0 + 16 > sg.len) {
         // Keys past the end of the sequence hold whatever the page has there:
         // zero their V rows so that P = 0 never meets a NaN.
@@ -397,24 +398,35 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         }
         __syncwarp();
       }
-      // The MMA operands: the stage itself, or for FP8 this warp's staging.
-      const uint32_t kop = kFp8 ? kstg : kbase;
+      // S = Q K^T for this warp's 16 keys: two n-tiles of 8 keys. K is read
+      // from the stage (FP8 rows through the same 16-bit ldmatrix view).
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int kr = warp * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int cofs = ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int k = 0; k < kKSteps; ++k) {
+          uint32_t b[4];
+          ldsm_x4(sw128_addr(kbase, kDecTileKeys, kr, k * 16 + cofs), b);
+          if constexpr (kFp8) {
+            mma16832_fp8<kType>(sacc[0], qa[k], b[0], b[1]);
+            mma16832_fp8<kType>(sacc[1], qa[k], b[2], b[3]);
+          } else {
+            mma16816<kFp16>(sacc[0], qa[k], b[0], b[1]);
+            mma16816<kFp16>(sacc[1], qa[k], b[2], b[3]);
+          }
+        }
+      }
+      if constexpr (kFp8) {
+        // this warp no longer reads the stage (K above, V in the copy)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+      }
+      // the P V operand: the stage's V tile, or for FP8 this warp's copy
       const uint32_t vop = kFp8 ? vstg : vbase;
       constexpr int kOpRows = kFp8 ? 16 : kDecTileKeys;
       const int row0w = kFp8 ? 0 : warp * 16;
-      // S = Q K^T for this warp's 16 keys: two n-tiles of 8 keys
-      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      {
-        const int kr = row0w + (lane & 7) + ((lane >> 4) << 3);
-        const int cofs = ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          uint32_t b[4];
-          ldsm_x4(sw128_addr(kop, kOpRows, kr, k * 16 + cofs), b);
-          mma16816<kFp16>(sacc[0], qa[k], b[0], b[1]);
-          mma16816<kFp16>(sacc[1], qa[k], b[2], b[3]);
-        }
-      }
       // mask, running max (rows qr, qr+8 across the 4 lanes of a quad)
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
