@@ -311,13 +311,18 @@ def gather_pages(cache: np.ndarray, block_table_row: Sequence[int], length: int)
 
 def attention_paged(q, k_cache, v_cache, block_table, cache_seqlens, scale, causal=False,
                     window=(-1, -1), sink=None, rows=None, q_descale=None, k_descale=None,
-                    v_descale=None):
+                    v_descale=None, k_new=None, v_new=None):
     """q (B, s_q, H_q, D); caches (num_blocks, page_size, H_kv, D) float64;
     block_table (B, max_pages); cache_seqlens (B,). The s_q query rows are the
     last s_q positions of the sequence (bottom-right alignment).
     FP8 (MATE "Attention", FMHA FP8 paragraph, which covers the KV-cache call
     too): q, k and v of sequence b and KV head g are multiplied by their
     descale [b, g] (all three given or none).
+    Appended keys (Mojo "flash_attention_split_kv": the previous keys come
+    from the cache and the current ones from separate k and v tensors, read
+    as one concatenated sequence): k_new, v_new (B, s_new, H_kv, D) follow
+    the cache_seqlens[b] cached rows of sequence b, so the sequence has
+    cache_seqlens[b] + s_new keys; the cache itself is not changed.
     Returns out (B, s_q, H_q, D_v) and lse (B, H_q, s_q)."""
     q = np.asarray(q, np.float64)
     B, Sq, Hq, _ = q.shape
@@ -335,6 +340,10 @@ def attention_paged(q, k_cache, v_cache, block_table, cache_seqlens, scale, caus
         L = int(cache_seqlens[b])
         ks = gather_pages(k_cache, block_table[b], L)
         vs = gather_pages(v_cache, block_table[b], L)
+        if k_new is not None:
+            ks = np.concatenate([ks, np.asarray(k_new[b], np.float64)])
+            vs = np.concatenate([vs, np.asarray(v_new[b], np.float64)])
+            L = ks.shape[0]
         for h in range(Hq):
             ii = [i for i in range(Sq) if want is None or (i, h) in want[b]]
             if not ii:

@@ -310,6 +310,34 @@ def test_paged_descale_equals_varlen_descale_on_gathered_rows():
         np.testing.assert_allclose(lse[b], l2, rtol=1e-13)
 
 
+@pytest.mark.parametrize("lens", [[0, 5], [8, 13]])
+def test_paged_append_equals_contiguous_concat_and_cache_written_in_place(lens):
+    # appended keys read as one sequence: equal to (a) the varlen oracle on
+    # [gathered cache | new rows] and (b) the paged oracle on a cache that
+    # holds the new rows at positions L .. L + s_new - 1 with lengths L + s_new
+    page, Hq, Hkv, D, sq, sn = 4, 4, 2, 3, 3, 3
+    ck, cv, bt = _paged_case([L + sn for L in lens], page, Hkv, D, "permuted")
+    q = RNG.normal(size=(2, sq, Hq, D))
+    kn, vn = RNG.normal(size=(2, sn, Hkv, D)), RNG.normal(size=(2, sn, Hkv, D))
+    out, lse = oracle.attention_paged(q, ck, cv, bt, lens, 0.7, causal=True, window=(4, 0),
+                                      k_new=kn, v_new=vn)
+    ck2, cv2 = ck.copy(), cv.copy()
+    for b, L in enumerate(lens):
+        for t in range(sn):
+            ck2[bt[b][(L + t) // page], (L + t) % page] = kn[b, t]
+            cv2[bt[b][(L + t) // page], (L + t) % page] = vn[b, t]
+        kk = np.concatenate([oracle.gather_pages(ck, bt[b], L), kn[b]])
+        vv = np.concatenate([oracle.gather_pages(cv, bt[b], L), vn[b]])
+        cu_q, cu_k = np.array([0, sq]), np.array([0, L + sn])
+        o2, l2 = oracle.attention_varlen(q[b], kk, vv, cu_q, cu_k, 0.7, True, (4, 0))
+        np.testing.assert_allclose(out[b], o2, rtol=1e-13)
+        np.testing.assert_allclose(lse[b], l2, rtol=1e-13)
+    o3, l3 = oracle.attention_paged(q, ck2, cv2, bt, [L + sn for L in lens], 0.7, causal=True,
+                                    window=(4, 0))
+    np.testing.assert_allclose(out, o3, rtol=1e-13)
+    np.testing.assert_allclose(lse, l3, rtol=1e-13)
+
+
 def test_paged_aliased_table_repeats_one_page():
     page, L = 4, 10
     ck = RNG.normal(size=(1, page, 1, 3))
