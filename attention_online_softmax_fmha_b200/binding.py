@@ -53,7 +53,7 @@ class SchedArgs(ctypes.Structure):
                 ("num_heads_q", c_i32), ("num_heads_kv", c_i32), ("head_dim_qk", c_i32),
                 ("head_dim_v", c_i32), ("page_size", c_i32), ("mode", c_i32), ("topk", c_i32),
                 ("num_ctas", c_i32), ("meta", c_vp), ("meta_bytes", c_sz),
-                ("sparse_block_size", c_i32)]
+                ("sparse_block_size", c_i32), ("seqlen_new", c_i32)]
 
 
 class PagedArgs(ctypes.Structure):
@@ -71,7 +71,9 @@ class PagedArgs(ctypes.Structure):
                 ("window_left", c_i32), ("window_right", c_i32), ("sink", c_vp),
                 ("meta", c_vp), ("meta_bytes", c_sz), ("num_ctas", c_i32), ("workspace", c_vp),
                 ("workspace_bytes", c_sz), ("q_descale", c_vp), ("k_descale", c_vp),
-                ("v_descale", c_vp)]
+                ("v_descale", c_vp), ("k_new", c_vp), ("v_new", c_vp), ("seqlen_new", c_i32),
+                ("kn_stride_b", c_i64), ("kn_stride_s", c_i64), ("kn_stride_h", c_i64),
+                ("vn_stride_b", c_i64), ("vn_stride_s", c_i64), ("vn_stride_h", c_i64)]
 
 
 class CombineArgs(ctypes.Structure):
@@ -245,9 +247,11 @@ def fwd_varlen(q, k, v, *, stream=None, **kw):
 # ---------------------------------------------------------------------------
 
 def sched_args(cache_seqlens, *, batch, seqlen_q, num_heads_q, num_heads_kv, head_dim_qk,
-               head_dim_v, page_size, mode=SCHED_MHA, topk=0, num_ctas=0, sparse_block_size=0):
+               head_dim_v, page_size, mode=SCHED_MHA, topk=0, num_ctas=0, sparse_block_size=0,
+               seqlen_new=0):
     return SchedArgs(_ptr(cache_seqlens), batch, seqlen_q, num_heads_q, num_heads_kv, head_dim_qk,
-                     head_dim_v, page_size, mode, topk, num_ctas, None, 0, sparse_block_size)
+                     head_dim_v, page_size, mode, topk, num_ctas, None, 0, sparse_block_size,
+                     seqlen_new)
 
 
 def sched_metadata_size(a: SchedArgs) -> int:
@@ -274,9 +278,12 @@ def sched_metadata(cache_seqlens, *, stream=None, meta=None, **kw) -> torch.Tens
 
 def paged_args(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, causal=False,
                window=(-1, -1), sink=None, meta=None, num_ctas=0, workspace=None, out=None,
-               lse=None, q_descale=None, k_descale=None, v_descale=None):
+               lse=None, q_descale=None, k_descale=None, v_descale=None, k_new=None,
+               v_new=None):
     """FP8 (float8_e4m3fn / float8_e5m2 q and caches, D = 128) takes
-    q/k/v_descale as contiguous fp32 (B, H_kv) device tensors."""
+    q/k/v_descale as contiguous fp32 (B, H_kv) device tensors. k_new, v_new
+    (B, s_new, H_kv, D) are keys read after each sequence's cached ones (the
+    metadata must then be made with seqlen_new=s_new)."""
     B, sq, Hq, D = q.shape
     Hkv = k_cache.shape[2]
     if out is None:
@@ -293,7 +300,10 @@ def paged_args(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, c
         v_cache.stride(2), out.stride(0), out.stride(1), out.stride(2),
         _TORCH_DTYPE.get(q.dtype, -1), float(scale), int(bool(causal)), int(window[0]),
         int(window[1]), _ptr(sink), _ptr(meta), 0 if meta is None else meta.numel() * 4,
-        int(num_ctas), None, 0, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale))
+        int(num_ctas), None, 0, _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
+        _ptr(k_new), _ptr(v_new), 0 if k_new is None else k_new.shape[1],
+        *((0, 0, 0) if k_new is None else k_new.stride()[:3]),
+        *((0, 0, 0) if v_new is None else v_new.stride()[:3]))
     if meta is not None:
         nbytes = int(lib().attn_paged_workspace_size(ctypes.byref(a)))
         if workspace is None:

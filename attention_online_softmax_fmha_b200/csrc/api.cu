@@ -53,6 +53,7 @@ attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int h
     return ATTN_ERR_INVALID_ARG;
   ds.sh.mode = mode;
   ds.sh.topk = topk;
+  ds.sh.new_keys = 0;
   if (mode == ATTN_SCHED_MHA) {
     ds.group = heads_q / heads_kv;
     ds.rows = seqlen_q * ds.group;
@@ -110,6 +111,17 @@ attn_status_t check_paged(const attn_paged_args* a) {
       !stride_ok(a->vc_stride_h, es) || !stride_ok(a->o_stride_b, 2) ||
       !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
     return ATTN_ERR_INVALID_ARG;
+  if ((a->k_new == nullptr) != (a->v_new == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (a->k_new) {
+    if (a->seqlen_new < 1 || !aligned16(a->k_new) || !aligned16(a->v_new))
+      return ATTN_ERR_INVALID_ARG;
+    if (!stride_ok(a->kn_stride_b, es) || !stride_ok(a->kn_stride_s, es) ||
+        !stride_ok(a->kn_stride_h, es) || !stride_ok(a->vn_stride_b, es) ||
+        !stride_ok(a->vn_stride_s, es) || !stride_ok(a->vn_stride_h, es))
+      return ATTN_ERR_INVALID_ARG;
+  } else if (a->seqlen_new != 0) {
+    return ATTN_ERR_INVALID_ARG;
+  }
   if (a->head_dim != 64 && a->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
   if (fp8 && a->head_dim != 128) return ATTN_ERR_UNSUPPORTED;
   if (!pow2_in(a->page_size, 16, 256)) return ATTN_ERR_UNSUPPORTED;
@@ -136,6 +148,17 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
       !encode_4d(&mv, a.v_cache, dt, C::kElt, D, a.num_heads_kv, a.page_size, a.num_blocks,
                  a.vc_stride_h, a.vc_stride_tok, a.vc_stride_blk, C::kChunkCols, 1, box_rows,
                  1))
+    return ATTN_ERR_INVALID_ARG;
+  // appended keys: (D, H_kv, seqlen_new, B) with 64-row boxes; without them
+  // the kernel never reads these maps and gets the cache maps in their place
+  CUtensorMap mkn = mk, mvn = mv;
+  if (a.k_new &&
+      (!encode_4d(&mkn, a.k_new, dt, C::kElt, D, a.num_heads_kv, a.seqlen_new, a.batch,
+                  a.kn_stride_h, a.kn_stride_s, a.kn_stride_b, C::kChunkCols, 1, kDecTileKeys,
+                  1) ||
+       !encode_4d(&mvn, a.v_new, dt, C::kElt, D, a.num_heads_kv, a.seqlen_new, a.batch,
+                  a.vn_stride_h, a.vn_stride_s, a.vn_stride_b, C::kChunkCols, 1, kDecTileKeys,
+                  1)))
     return ATTN_ERR_INVALID_ARG;
   DecodeParams p;
   memset(&p, 0, sizeof(p));
@@ -171,6 +194,7 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
   p.causal = a.causal;
   p.window_left = a.window_left;
   p.window_right = a.window_right;
+  p.seqlen_new = a.k_new ? a.seqlen_new : 0;
   if (a.meta) {
     const size_t slots = (size_t)ds.S + ds.G;
     p.ws_o = reinterpret_cast<float*>(a.workspace);
@@ -183,7 +207,7 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
     configured = true;
   }
   const int grid = a.meta ? ds.G : ds.S;
-  kernel<<<grid, 160, C::kSmemBytes, stream>>>(mk, mv, p);
+  kernel<<<grid, 160, C::kSmemBytes, stream>>>(mk, mv, mkn, mvn, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (a.meta) {
     const int64_t warps = (int64_t)ds.S * kDecRows;
@@ -349,11 +373,15 @@ attn_status_t attn_sched_metadata(const attn_sched_args* a, void* stream) {
     return ATTN_ERR_INVALID_ARG;
   if (a->mode < ATTN_SCHED_MHA || a->mode > ATTN_SCHED_MLA_SPARSE) return ATTN_ERR_INVALID_ARG;
   if (!sbs_ok(a->sparse_block_size)) return ATTN_ERR_INVALID_ARG;
+  // appended keys exist for the GQA decode only
+  if (a->seqlen_new < 0 || (a->seqlen_new > 0 && a->mode != ATTN_SCHED_MHA))
+    return ATTN_ERR_INVALID_ARG;
   DecodeShape ds;
   const attn_status_t st =
       decode_shape(a->mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv,
                    sparse_positions(a->mode, a->topk, a->sparse_block_size), a->num_ctas, ds);
   if (st != ATTN_OK) return st;
+  ds.sh.new_keys = a->seqlen_new;
   if (a->meta_bytes < meta_bytes_for(ds)) return ATTN_ERR_WORKSPACE_TOO_SMALL;
   SchedParams p;
   memset(&p, 0, sizeof(p));
@@ -575,6 +603,7 @@ extern "C" attn_status_t attn_fwd_paged_kvcache_static(const attn_paged_args* ar
   sa.page_size = args->page_size;
   sa.mode = ATTN_SCHED_MHA;
   sa.num_ctas = args->num_ctas;
+  sa.seqlen_new = args->k_new ? args->seqlen_new : 0;
   sa.meta = reinterpret_cast<int32_t*>(base);
   sa.meta_bytes = meta_bytes;
   st = attn_sched_metadata(&sa, stream);

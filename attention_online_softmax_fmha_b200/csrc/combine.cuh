@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeParams 
   if (s >= p.num_segs) return;
   if (!(meta_matches(p.meta, ATTN_SCHED_MHA, p.batch, p.seqlen_q, p.heads_q, p.heads_kv,
                      p.page_size, p.num_segs, kDecTileKeys, D, D) &&
-        p.meta[kMetaNumCtas] == p.num_ctas))
+        p.meta[kMetaNumCtas] == p.num_ctas && p.meta[kMetaNewKeys] == p.seqlen_new))
     return;  // the decode kernel has reported the mismatch
   const MetaLayout ml(p.num_ctas, p.num_segs);
   const int ns = p.meta[ml.seg_nsplit + s];

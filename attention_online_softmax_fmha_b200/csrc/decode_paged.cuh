@@ -27,6 +27,11 @@
 // A piece that is the whole segment writes O (bf16) and LSE directly; a piece
 // of a split segment writes a sink-free partial (O / l, LSE) to the workspace
 // for the combine kernel.
+// Appended keys (Mojo "flash_attention_split_kv": the current k and v are read
+// in place after the cached ones, as one sequence) come from their own
+// (B, s_new, H_kv, D) tensors through a second pair of tensor maps. They
+// start a tile of their own after the cache's last tile, so no tile mixes the
+// two sources; rows past s_new read as zeros.
 #pragma once
 
 #include "common.cuh"
@@ -59,6 +64,7 @@ struct DecodeParams {
   int32_t num_ctas;          // grid size with metadata
   float scale_log2;
   int32_t causal, window_left, window_right;
+  int32_t seqlen_new;        // appended keys per sequence (0: none)
 };
 
 template <int D, bool kFp8>
@@ -82,8 +88,17 @@ struct DecodeCfg {
 };
 
 struct DecodeSeg {
-  int b, g, rsub, len;
-  int t0, t1;  // visible tile range of the segment
+  int b, g, rsub;
+  int len;     // cached keys
+  int ltot;    // cached + appended keys
+  int nct;     // tiles of the cache; appended keys start at tile nct
+  int t0, t1;  // visible cache tiles [t0, t1)
+  int tn0, tn1;  // visible appended tiles [tn0, tn1)
+  DEVI bool visible(int t) const { return (t >= t0 && t < t1) || (t >= tn0 && t < tn1); }
+  // position in the sequence of row 0 of tile t, and the end of the valid
+  // positions of that tile's source
+  DEVI int pos0(int t) const { return t < nct ? t * kDecTileKeys : len + (t - nct) * kDecTileKeys; }
+  DEVI int pend(int t) const { return t < nct ? len : ltot; }
 };
 
 DEVI void decode_seg(const DecodeParams& p, int s, DecodeSeg& sg) {
@@ -92,18 +107,28 @@ DEVI void decode_seg(const DecodeParams& p, int s, DecodeSeg& sg) {
   sg.g = rem / p.n_rsub;
   sg.rsub = rem - sg.g * p.n_rsub;
   sg.len = p.cache_seqlens[sg.b];
+  sg.ltot = sg.len + p.seqlen_new;
+  sg.nct = sg.len > 0 ? (sg.len + kDecTileKeys - 1) / kDecTileKeys : 0;
   // union of the rows' visible ranges (row i = 0 has the smallest left edge,
   // i = s_q - 1 the largest right edge)
-  const int delta = sg.len - p.seqlen_q;
-  int lo = 0, hi = sg.len - 1;
+  const int delta = sg.ltot - p.seqlen_q;
+  int lo = 0, hi = sg.ltot - 1;
   if (p.window_left >= 0) lo = max(lo, delta - p.window_left);
   if (p.causal) hi = min(hi, p.seqlen_q - 1 + delta);
   if (p.window_right >= 0) hi = min(hi, p.seqlen_q - 1 + delta + p.window_right);
-  if (hi < lo) {
+  const int chi = min(hi, sg.len - 1);  // cached part
+  if (chi < lo) {
     sg.t0 = sg.t1 = 0;
   } else {
     sg.t0 = lo / kDecTileKeys;
-    sg.t1 = hi / kDecTileKeys + 1;
+    sg.t1 = chi / kDecTileKeys + 1;
+  }
+  const int nlo = max(lo, sg.len);      // appended part
+  if (hi < nlo) {
+    sg.tn0 = sg.tn1 = 0;
+  } else {
+    sg.tn0 = sg.nct + (nlo - sg.len) / kDecTileKeys;
+    sg.tn1 = sg.nct + (hi - sg.len) / kDecTileKeys + 1;
   }
 }
 
@@ -190,7 +215,8 @@ DEVI void fp8x16_to_f16_tile(uint32_t tile, int row, int col, uint4 w) {
 // ---------------------------------------------------------------------------
 template <int D, bool kFp8>
 DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CUtensorMap* mv,
-                          uint8_t* smem, uint64_t* full, uint64_t* empty, volatile int* abort,
+                          const CUtensorMap* mkn, const CUtensorMap* mvn, uint8_t* smem,
+                          uint64_t* full, uint64_t* empty, volatile int* abort,
                           int seg_begin_units, int seg_end_units, int first_seg,
                           const int32_t* seg_prefix) {
   using C = DecodeCfg<D, kFp8>;
@@ -198,6 +224,10 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
   if (lane == 0) {
     tma_prefetch_desc(mk);
     tma_prefetch_desc(mv);
+    if (p.seqlen_new > 0) {
+      tma_prefetch_desc(mkn);
+      tma_prefetch_desc(mvn);
+    }
   }
   int it = 0;
   const int P = p.page_size;
@@ -225,8 +255,33 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
     // (lane x holds entry win0 + x) and is refilled when a tile leaves it.
     int win0 = -(1 << 30), win_val = 0;
     for (int t = a; t < e; ++t) {
-      if (t < sg.t0 || t >= sg.t1) continue;  // no visible key: skipped by all roles
+      if (!sg.visible(t)) continue;  // no visible key: skipped by all roles
       const int st = it % kDecStages;
+      if (it >= kDecStages) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&empty[st], ((it / kDecStages) - 1) & 1, abort, 31);
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
+      }
+      if (t >= sg.nct) {
+        // appended keys: one 64-row box of the new k / v per 128-byte chunk
+        // (rows past s_new are outside the tensor and read as zeros)
+        if (lane == 0) {
+          mbar_expect_tx(&full[st], 2u * kDecTileKeys * D * C::kElt);
+          uint8_t* kdst = smem + C::kStageOff + st * C::kStageBytes;
+          uint8_t* vdst = kdst + C::kTileBytes;
+          const int row = (t - sg.nct) * kDecTileKeys;
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c) {
+            tma_load_4d(kdst + c * kDecTileKeys * 128, mkn, &full[st], c * C::kChunkCols, sg.g,
+                        row, sg.b);
+            tma_load_4d(vdst + c * kDecTileKeys * 128, mvn, &full[st], c * C::kChunkCols, sg.g,
+                        row, sg.b);
+          }
+        }
+        __syncwarp();
+        ++it;
+        continue;
+      }
       const int first_page = (t * kDecTileKeys) / P;
       const int nload = min(loads_per_tile, npages_seq - first_page);
       if (first_page < win0 || first_page + nload > win0 + 32) {
@@ -234,11 +289,6 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
         win_val = (win0 + lane < npages_seq) ? bt[win0 + lane] : 0;
       }
       const int row_in_page = (t * kDecTileKeys) % P;  // 0 unless P > 64
-      if (it >= kDecStages) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(&empty[st], ((it / kDecStages) - 1) & 1, abort, 31);
-        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
-      }
       if (lane == 0)
         mbar_expect_tx(&full[st], 2u * nload * box_rows * D * C::kElt);
       __syncwarp();
@@ -345,9 +395,9 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
     for (int h2 = 0; h2 < 2; ++h2) {
       const int rr = row0 + qr + h2 * 8;
       const int i = min(rr, p.rows - 1) / p.group;
-      const int delta = sg.len - p.seqlen_q;
+      const int delta = sg.ltot - p.seqlen_q;
       lo[h2] = 0;
-      hi[h2] = sg.len - 1;
+      hi[h2] = sg.ltot - 1;
       if (p.window_left >= 0) lo[h2] = max(lo[h2], i + delta - p.window_left);
       if (p.causal) hi[h2] = min(hi[h2], i + delta);
       if (p.window_right >= 0) hi[h2] = min(hi[h2], i + delta + p.window_right);
@@ -367,12 +417,15 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
     const uint32_t vstg = smem_u32(smem + C::kStgOff + warp * C::kStgWarpBytes);
 
     for (int t = a; t < e; ++t) {
-      if (t < sg.t0 || t >= sg.t1) continue;
+      if (!sg.visible(t)) continue;
       const int st = it % kDecStages;
       if (!warp_wait(&full[st], (it / kDecStages) & 1, abort, 33)) return;
       const uint32_t kbase = smem_u32(smem + C::kStageOff + st * C::kStageBytes);
       const uint32_t vbase = kbase + C::kTileBytes;
-      const int key0 = t * kDecTileKeys + warp * 16;  // this warp's first key
+      // sequence position of this warp's first key, and the end of the valid
+      // rows of the tile's source (the cache, or the appended keys)
+      const int key0 = sg.pos0(t) + warp * 16;
+      const int kend = sg.pend(t);
       if constexpr (kFp8) {
         // FP8 -> fp16 copy of this warp's 16 V rows; rows past the end of the
         // sequence become zeros (P = 0 must not meet a NaN there).
@@ -383,15 +436,15 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
           const int kr = x / (D / 16), u = x % (D / 16);
           const int row = warp * 16 + kr;
           uint4 vw = *reinterpret_cast<const uint4*>(vt + row * 128 + ((u ^ (row & 7)) << 4));
-          if (key0 + kr >= sg.len) vw = make_uint4(0, 0, 0, 0);
+          if (key0 + kr >= kend) vw = make_uint4(0, 0, 0, 0);
           fp8x16_to_f16_tile<kType>(vstg, kr, u * 16, vw);
         }
-      } else if (key0 + 16 > sg.len) {
+      } else if (key0 + 16 > kend) {
         // Keys past the end of the sequence hold whatever the page has there:
         // zero their V rows so that P = 0 never meets a NaN.
         for (int x = lane; x < 16 * (D / 8); x += 32) {
           const int kr = x / (D / 8), c8 = x % (D / 8);
-          if (key0 + kr >= sg.len) {
+          if (key0 + kr >= kend) {
             const uint32_t ad = sw128_addr(vbase, kDecTileKeys, warp * 16 + kr, c8 * 8);
             asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(ad), "r"(0) : "memory");
           }
@@ -435,7 +488,7 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         for (int x = 0; x < 4; ++x) {
           const int key = key0 + nt * 8 + qc + (x & 1);
           const int h2 = x >> 1;
-          if (key < lo[h2] || key > hi[h2]) sacc[nt][x] = -INFINITY;
+          if (key >= kend || key < lo[h2] || key > hi[h2]) sacc[nt][x] = -INFINITY;
           mx[h2] = fmaxf(mx[h2], sacc[nt][x]);
         }
       float alpha[2], m_use[2];
@@ -585,7 +638,9 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
 template <int D, int kType>
 __global__ void __launch_bounds__(160, 1)
     decode_kernel(const __grid_constant__ CUtensorMap map_k,
-                  const __grid_constant__ CUtensorMap map_v, const DecodeParams p) {
+                  const __grid_constant__ CUtensorMap map_v,
+                  const __grid_constant__ CUtensorMap map_kn,
+                  const __grid_constant__ CUtensorMap map_vn, const DecodeParams p) {
   constexpr bool kFp8 = kType >= 2;
   using C = DecodeCfg<D, kFp8>;
   extern __shared__ uint8_t smem_raw[];
@@ -614,7 +669,7 @@ __global__ void __launch_bounds__(160, 1)
     if (threadIdx.x == 0 &&
         !(meta_matches(p.meta, ATTN_SCHED_MHA, p.batch, p.seqlen_q, p.heads_q, p.heads_kv,
                        p.page_size, p.num_segs, kDecTileKeys, D, D) &&
-          p.meta[kMetaNumCtas] == p.num_ctas)) {
+          p.meta[kMetaNumCtas] == p.num_ctas && p.meta[kMetaNewKeys] == p.seqlen_new)) {
       raise_error(ATTN_DEVERR_META_MISMATCH, 40);
       s_bad = 1;
     }
@@ -630,12 +685,13 @@ __global__ void __launch_bounds__(160, 1)
     const int b = s0 / p.segs_per_seq;
     const int len = p.cache_seqlens[b];
     ub = 0;
-    ue = len > 0 ? (len + kDecTileKeys - 1) / kDecTileKeys : 0;
+    ue = (len > 0 ? (len + kDecTileKeys - 1) / kDecTileKeys : 0) +
+         (p.seqlen_new + kDecTileKeys - 1) / kDecTileKeys;
     if (ue == 0) ue = 1;  // still write O = 0, LSE = -inf for an empty sequence
   }
   if (threadIdx.x >= 128) {
-    decode_producer<D, kFp8>(p, &map_k, &map_v, smem, full, empty, abort, ub, ue, s0,
-                             seg_prefix);
+    decode_producer<D, kFp8>(p, &map_k, &map_v, &map_kn, &map_vn, smem, full, empty, abort, ub,
+                             ue, s0, seg_prefix);
   } else {
     decode_consumer<D, kType>(p, smem, full, empty, abort, ub, ue, s0, seg_prefix);
   }

@@ -35,6 +35,7 @@ enum MetaHeader {
   kMetaDimV,
   kMetaTotalSlots,  // written by the device
   kMetaSegsPerSeq,
+  kMetaNewKeys,  // keys appended after each sequence's cache (GQA decode)
   kMetaHeaderWords = 16
 };
 constexpr int32_t kMetaMagicValue = 0x4154544d;  // "MTTA"
@@ -59,12 +60,16 @@ struct SchedShape {
   int32_t unit_keys;     // keys per unit (dense modes)
   int32_t mode;
   int32_t topk;
+  int32_t new_keys;      // GQA decode: keys appended after the cache (own tiles)
 };
 
-// Units (KV tiles) of one segment of a sequence with `len` cached keys.
+// Units (KV tiles) of one segment of a sequence with `len` cached keys. The
+// appended keys of GQA decode start a tile of their own after the cache's
+// last (partial) tile.
 DEVI int32_t sched_units(const SchedShape& sh, int32_t len) {
   if (sh.mode == ATTN_SCHED_MLA_SPARSE) return (sh.topk + sh.unit_keys - 1) / sh.unit_keys;
-  return len > 0 ? (len + sh.unit_keys - 1) / sh.unit_keys : 0;
+  const int32_t cached = len > 0 ? (len + sh.unit_keys - 1) / sh.unit_keys : 0;
+  return cached + (sh.new_keys + sh.unit_keys - 1) / sh.unit_keys;
 }
 
 struct SchedParams {
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(1024, 1) sched_kernel(const SchedParams p) {
     h[kMetaDimV] = p.dim_v;
     h[kMetaTotalSlots] = slots;
     h[kMetaSegsPerSeq] = p.sh.segs_per_seq;
-    h[15] = 0;
+    h[kMetaNewKeys] = p.sh.new_keys;
   }
 }
 

@@ -170,6 +170,8 @@ class PagedInputs:
     q_descale: Optional[torch.Tensor] = None   # FP8: fp32 (B, H_kv) in [0.5, 2]
     k_descale: Optional[torch.Tensor] = None
     v_descale: Optional[torch.Tensor] = None
+    k_new: Optional[torch.Tensor] = None       # appended keys (B, s_new, H_kv, D)
+    v_new: Optional[torch.Tensor] = None
 
     @property
     def batch(self) -> int:
@@ -204,7 +206,8 @@ def _block_table(seqlens: Sequence[int], page_size: int, layout: str, g_cpu: tor
 def make_paged(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, num_heads_kv: int,
                head_dim: int, page_size: int = 64, table: str = "permuted", causal: bool = False,
                window=(-1, -1), sink: bool = False, dtype: str = "bf16",
-               scale: Optional[float] = None, seed: int = 0, device="cpu") -> PagedInputs:
+               scale: Optional[float] = None, seqlen_new: int = 0, seed: int = 0,
+               device="cpu") -> PagedInputs:
     seqlens = [int(x) for x in seqlens]
     g_cpu = _gen(seed + 7919, "cpu")
     bt, nblocks = _block_table(seqlens, page_size, table, g_cpu)
@@ -219,11 +222,15 @@ def make_paged(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, num_h
     if dtype in _FP8:
         desc = [torch.rand(B, num_heads_kv, generator=g, device=device) * 1.5 + 0.5
                 for _ in range(3)]
+    new = [None, None]
+    if seqlen_new > 0:
+        new = [_values((B, seqlen_new, num_heads_kv, head_dim), dtype, g, device)
+               for _ in range(2)]
     if scale is None:
         scale = 1.0 / math.sqrt(head_dim)
     return PagedInputs(q, kc, vc, bt.to(device), torch.tensor(seqlens, dtype=torch.int32,
                        device=device), seqlens, page_size, num_heads_q, num_heads_kv, head_dim,
-                       bool(causal), tuple(window), float(scale), sink_t, dtype, *desc)
+                       bool(causal), tuple(window), float(scale), sink_t, dtype, *desc, *new)
 
 
 @dataclasses.dataclass

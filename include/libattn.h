@@ -193,6 +193,7 @@ typedef struct {
   int32_t* meta;
   size_t meta_bytes;
   int32_t sparse_block_size;  /* ATTN_SCHED_MLA_SPARSE: as in mla_args          */
+  int32_t seqlen_new;  /* ATTN_SCHED_MHA: the seqlen_new of the paged call (0) */
 } attn_sched_args;
 
 /* Bytes of `meta` needed for these arguments (host only, no device access). */
@@ -220,6 +221,14 @@ attn_status_t attn_sched_metadata(const attn_sched_args* args, void* stream);
 /*   values of sequence b and KV head g are the stored codes times their     */
 /*   descale [b][g] (MATE "Attention", FMHA FP8 paragraph). out is bf16.     */
 /*   The descales are ignored for bf16 and fp16 input.                      */
+/* Appended keys (Mojo "flash_attention_split_kv": the previous keys come    */
+/*   from the cache and the current ones from separate k and v tensors, in  */
+/*   one concatenated sequence): k_new, v_new (B, seqlen_new, H_kv, D) of    */
+/*   the cache's dtype, with strides in elements, or both NULL. Sequence b   */
+/*   then has L_b + seqlen_new keys, the new ones after its cached L_b, and  */
+/*   the query rows are its last s_q positions. The cache is not written.    */
+/*   The metadata must come from attn_sched_metadata with the same          */
+/*   seqlen_new (checked on the device: ATTN_DEVERR_META_MISMATCH).         */
 /* meta: from attn_sched_metadata(mode=ATTN_SCHED_MHA, same args), or NULL   */
 /*   for one CTA per (sequence, KV head) and no splitting.                   */
 /* workspace: device buffer of attn_paged_workspace_size() bytes (partial   */
@@ -228,8 +237,9 @@ attn_status_t attn_sched_metadata(const attn_sched_args* args, void* stream);
 /* Supported now: bf16 and fp16 with D in {64, 128}; e4m3 and e5m2 with     */
 /*   D = 128; page_size in {16, 32, 64, 128, 256}; s_q * H_q / H_kv <= 16.  */
 /* Errors: INVALID_ARG for NULL required pointers (the descales included    */
-/*   for FP8), bad sizes or misaligned strides; UNSUPPORTED outside the     */
-/*   supported shapes above.                                                 */
+/*   for FP8), only one of k_new / v_new, seqlen_new < 1 with them, bad      */
+/*   sizes or misaligned strides; UNSUPPORTED outside the supported shapes   */
+/*   above.                                                                  */
 /* ------------------------------------------------------------------------ */
 typedef struct {
   const void* q;
@@ -266,6 +276,11 @@ typedef struct {
   const float* q_descale; /* FP8 only: (B, H_kv) fp32 */
   const float* k_descale;
   const float* v_descale;
+  const void* k_new;      /* appended keys (B, seqlen_new, H_kv, D), or NULL */
+  const void* v_new;
+  int32_t seqlen_new;
+  int64_t kn_stride_b, kn_stride_s, kn_stride_h;
+  int64_t vn_stride_b, vn_stride_s, vn_stride_h;
 } attn_paged_args;
 
 /* Bytes of workspace for these arguments (host only; 0 when meta is NULL).  */

@@ -114,10 +114,23 @@ def _paged(**over):
      B.UNSUPPORTED),                                # FP8 is built for D = 128
     (dict(head_dim=96), B.UNSUPPORTED),
     (dict(page_size=8), B.UNSUPPORTED),
+    (dict(k_new=0x7000, seqlen_new=2, kn_stride_b=2 * 256, kn_stride_s=256, kn_stride_h=128),
+     B.INVALID_ARG),                                # v_new missing
+    (dict(seqlen_new=2), B.INVALID_ARG),            # seqlen_new without k_new / v_new
+    (dict(k_new=0x7000, v_new=0x8000, seqlen_new=0, kn_stride_b=256, kn_stride_s=256,
+          kn_stride_h=128, vn_stride_b=256, vn_stride_s=256, vn_stride_h=128), B.INVALID_ARG),
 ])
 def test_paged_rejects_bad_arguments(L, over, want):
     a = _paged(**over)
     assert L.attn_fwd_paged_kvcache(ctypes.byref(a), None) == want
+
+
+def test_sched_rejects_appended_keys_outside_gqa_decode(L):
+    a = B.SchedArgs(0x1000, 2, 1, 128, 1, 576, 512, 64, B.SCHED_MLA, 0, 0, 0x2000, 1 << 20, 0, 4)
+    assert L.attn_sched_metadata(ctypes.byref(a), None) == B.INVALID_ARG
+    a.mode, a.num_heads_kv, a.num_heads_q, a.head_dim_qk, a.head_dim_v = B.SCHED_MHA, 2, 8, 128, 128
+    a.seqlen_new = -1
+    assert L.attn_sched_metadata(ctypes.byref(a), None) == B.INVALID_ARG
 
 
 def test_null_struct_is_invalid(L):

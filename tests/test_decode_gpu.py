@@ -26,10 +26,13 @@ def _np(t):
 
 
 def oracle_paged(inp, rows=None):
+    kn = None if inp.k_new is None else to_f64(inp.k_new)
+    vn = None if inp.v_new is None else to_f64(inp.v_new)
     return oracle.attention_paged(to_f64(inp.q), to_f64(inp.k_cache), to_f64(inp.v_cache),
                                   inp.block_table.cpu().numpy(), inp.seqlens, inp.scale,
                                   inp.causal, inp.window, _np(inp.sink), rows,
-                                  _np(inp.q_descale), _np(inp.k_descale), _np(inp.v_descale))
+                                  _np(inp.q_descale), _np(inp.k_descale), _np(inp.v_descale),
+                                  kn, vn)
 
 
 def run_paged(inp, use_meta=True, num_ctas=0):
@@ -38,12 +41,14 @@ def run_paged(inp, use_meta=True, num_ctas=0):
         meta = B.sched_metadata(inp.cache_seqlens, batch=inp.batch, seqlen_q=inp.q.shape[1],
                                 num_heads_q=inp.num_heads_q, num_heads_kv=inp.num_heads_kv,
                                 head_dim_qk=inp.head_dim, head_dim_v=inp.head_dim,
-                                page_size=inp.page_size, num_ctas=num_ctas)
+                                page_size=inp.page_size, num_ctas=num_ctas,
+                                seqlen_new=0 if inp.k_new is None else inp.k_new.shape[1])
     out, lse = B.fwd_paged_kvcache(inp.q, inp.k_cache, inp.v_cache, inp.block_table,
                                    inp.cache_seqlens, scale=inp.scale, causal=inp.causal,
                                    window=inp.window, sink=inp.sink, meta=meta,
                                    num_ctas=num_ctas, q_descale=inp.q_descale,
-                                   k_descale=inp.k_descale, v_descale=inp.v_descale)
+                                   k_descale=inp.k_descale, v_descale=inp.v_descale,
+                                   k_new=inp.k_new, v_new=inp.v_new)
     torch.cuda.synchronize()
     assert B.device_error() == 0
     return out, lse, meta
@@ -112,6 +117,46 @@ def test_fp8_cache_multi_token_causal_window_sink_no_metadata():
                        dtype="e4m3", seed=21, device="cuda")
     check(inp, atol=5e-2, num_ctas=6)
     check(inp, atol=5e-2, use_meta=False)
+
+
+# Appended keys (k_new / v_new read after the cached keys, the cache left
+# untouched), against the oracle on the concatenated sequence.
+def test_append_new_tokens_causal_split_and_unsplit():
+    inp = W.make_paged(seqlens=[0, 1, 63, 64, 65, 700], seqlen_q=3, num_heads_q=8,
+                       num_heads_kv=2, head_dim=128, page_size=32, causal=True, seqlen_new=3,
+                       seed=30, device="cuda")
+    before = inp.k_cache.clone()
+    check(inp, num_ctas=7)
+    check(inp, use_meta=False)
+    assert torch.equal(inp.k_cache, before)
+
+
+def test_append_two_tiles_of_new_keys_window_d64():
+    inp = W.make_paged(seqlens=[5, 129, 300], seqlen_q=1, num_heads_q=4, num_heads_kv=4,
+                       head_dim=64, page_size=64, window=(100, 0), causal=True, seqlen_new=70,
+                       seed=31, device="cuda")
+    check(inp, num_ctas=5)
+
+
+def test_append_fp8_with_sink():
+    inp = W.make_paged(seqlens=[17, 400], seqlen_q=2, num_heads_q=8, num_heads_kv=2,
+                       head_dim=128, page_size=64, causal=True, sink=True, seqlen_new=2,
+                       dtype="e4m3", seed=32, device="cuda")
+    check(inp, atol=5e-2, num_ctas=3)
+
+
+def test_append_metadata_without_new_keys_is_reported():
+    inp = W.make_paged(seqlens=[40, 90], seqlen_q=1, num_heads_q=4, num_heads_kv=1,
+                       head_dim=128, page_size=32, seqlen_new=1, seed=33, device="cuda")
+    meta = B.sched_metadata(inp.cache_seqlens, batch=2, seqlen_q=1, num_heads_q=4,
+                            num_heads_kv=1, head_dim_qk=128, head_dim_v=128, page_size=32,
+                            num_ctas=3)  # made for seqlen_new = 0
+    B.fwd_paged_kvcache(inp.q, inp.k_cache, inp.v_cache, inp.block_table, inp.cache_seqlens,
+                        scale=inp.scale, meta=meta, num_ctas=3, k_new=inp.k_new,
+                        v_new=inp.v_new)
+    torch.cuda.synchronize()
+    assert B.device_error() & 0xff == B.DEVERR_META_MISMATCH
+    assert B.device_error() == 0
 
 
 @pytest.mark.parametrize("lens,G", [([0, 1, 64, 65, 4000, 12, 9000], 9),
