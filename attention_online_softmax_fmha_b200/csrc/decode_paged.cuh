@@ -16,9 +16,10 @@
 //   warps 0-3   consumers: warp w owns keys [16w, 16w + 16) of every tile and
 //               keeps its own online-softmax state (running max, sums, O in
 //               registers). S = Q K^T and O += P V use mma.sync m16n8k16 with
-//               fp32 accumulation; their cost is far below the tile's load
-//               time. At the end of a segment piece the four warp states are
-//               merged through shared memory.
+//               fp32 accumulation. With one consumer warp per SM
+//               sub-partition, a 64-key tile takes about as long to consume
+//               as a bf16 tile takes to load. At the end of a segment piece
+//               the four warp states are merged through shared memory.
 // FP8 caches (e4m3 / e5m2, D = 128) arrive as 128-byte rows. S = Q K^T runs
 // on the FP8 codes directly (mma.sync m16n8k32, Q kept in FP8); each warp
 // rewrites its 16 V rows as fp16 (exact for both formats) in a private
