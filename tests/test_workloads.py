@@ -54,3 +54,16 @@ def test_sparse_indices_distinct_sorted_below_length():
             valid = row[row >= 0]
             assert valid.numel() == min(L, 256)
             assert torch.all(valid[1:] > valid[:-1]) and int(valid.max()) < L
+
+
+def test_paged_fp8_descales_and_appended_keys():
+    p = W.make_paged(seqlens=[30, 70], seqlen_q=2, num_heads_q=4, num_heads_kv=2, head_dim=16,
+                     page_size=16, dtype="e5m2", seqlen_new=3, seed=5)
+    assert p.k_cache.dtype == torch.float8_e5m2 and p.q.dtype == torch.float8_e5m2
+    for t in (p.q_descale, p.k_descale, p.v_descale):
+        assert t.shape == (2, 2) and float(t.min()) >= 0.5 and float(t.max()) <= 2.0
+    assert p.k_new.shape == (2, 3, 2, 16) and p.k_new.dtype == torch.float8_e5m2
+    assert not torch.equal(p.k_new.float(), p.v_new.float())
+    plain = W.make_paged(seqlens=[30, 70], seqlen_q=2, num_heads_q=4, num_heads_kv=2,
+                         head_dim=16, page_size=16, seed=5)
+    assert plain.k_new is None and plain.q_descale is None
