@@ -153,6 +153,34 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _rows(**tensors):
+    """The C structs carry element strides of the outer axes only: the last
+    axis of every tensor must be contiguous."""
+    for name, t in tensors.items():
+        if t is not None and t.numel() > 1 and t.stride(-1) != 1:
+            raise ValueError(f"{name}: the last axis must be contiguous (stride 1)")
+
+
+def _dense(**tensors):
+    """Tensors the C side indexes as plain contiguous arrays."""
+    for name, t in tensors.items():
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def _same_dtype(q, **tensors):
+    """The C structs carry one input dtype for q and every K/V operand."""
+    for name, t in tensors.items():
+        if t is not None and t.dtype != q.dtype:
+            raise ValueError(f"{name}: dtype {t.dtype} differs from q's {q.dtype}")
+
+
+def _int32(**tensors):
+    for name, t in tensors.items():
+        if t is not None and t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+
+
 def _stream(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -191,6 +219,13 @@ def varlen_args(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=N
     mask: fp32 tensor indexed [b, h, i, j] (a 4-D view; size-1 axes broadcast
     with stride 0); seqused_q/k: int32 (B,) for the padded layout."""
     varlen = cu_seqlens_q is not None
+    _rows(q=q, k=k, v=v, out=out, lse=lse)
+    _same_dtype(q, k=k, v=v)
+    _dense(cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k, seqused_q=seqused_q,
+           seqused_k=seqused_k, sink=sink, q_descale=q_descale, k_descale=k_descale,
+           v_descale=v_descale)
+    _int32(cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k, seqused_q=seqused_q,
+           seqused_k=seqused_k)
     Hq, D = q.shape[-2], q.shape[-1]
     Hkv, Dv = k.shape[-2], v.shape[-1]
     if varlen:
@@ -284,6 +319,14 @@ def paged_args(q, k_cache, v_cache, block_table, cache_seqlens, *, scale=None, c
     q/k/v_descale as contiguous fp32 (B, H_kv) device tensors. k_new, v_new
     (B, s_new, H_kv, D) are keys read after each sequence's cached ones (the
     metadata must then be made with seqlen_new=s_new)."""
+    _rows(q=q, k_cache=k_cache, v_cache=v_cache, out=out, block_table=block_table, k_new=k_new,
+          v_new=v_new)
+    _same_dtype(q, k_cache=k_cache, v_cache=v_cache, k_new=k_new, v_new=v_new)
+    _dense(cache_seqlens=cache_seqlens, lse=lse, sink=sink, q_descale=q_descale,
+           k_descale=k_descale, v_descale=v_descale)
+    _int32(block_table=block_table, cache_seqlens=cache_seqlens)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
     B, sq, Hq, D = q.shape
     Hkv = k_cache.shape[2]
     if out is None:
@@ -360,6 +403,10 @@ def combine(out_partial, lse_partial, *, num_splits_per_seq=None, sink=None, out
 def mla_args(q, kv_cache, block_table, cache_seqlens, *, head_dim_v=512, scale=None,
              causal=False, indices=None, meta=None, num_ctas=0, workspace=None, out=None,
              lse=None, sparse_block_size=0):
+    _rows(q=q, kv_cache=kv_cache, out=out, block_table=block_table, indices=indices)
+    _same_dtype(q, kv_cache=kv_cache)
+    _dense(cache_seqlens=cache_seqlens, lse=lse)
+    _int32(block_table=block_table, cache_seqlens=cache_seqlens, indices=indices)
     B, sq, Hq, Dqk = q.shape
     if out is None:
         out = torch.empty(B, sq, Hq, head_dim_v, device=q.device, dtype=torch.bfloat16)
