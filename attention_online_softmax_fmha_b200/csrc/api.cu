@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -24,6 +25,21 @@ namespace {
 // ---------------------------------------------------------------------------
 // Scheduler metadata / paged decode / combine
 // ---------------------------------------------------------------------------
+
+// Runs `configure` (a kernel's function attributes) once per device: the
+// attributes belong to the current device's context, so every device needs
+// its own call. Devices past 63 configure on every launch. Safe under
+// concurrent callers (a repeated call is harmless).
+template <typename F>
+attn_status_t configure_per_device(std::atomic<uint64_t>& done, F&& configure) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const uint64_t bit = dev < 64 ? uint64_t(1) << dev : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return ATTN_OK;
+  const attn_status_t st = configure();
+  if (st == ATTN_OK && bit) done.fetch_or(bit, std::memory_order_release);
+  return st;
+}
 
 // Segments and units of a decode problem (see sched.cuh).
 struct DecodeShape {
@@ -201,11 +217,11 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
     p.ws_lse = p.ws_o + slots * kDecRows * D;
   }
   auto kernel = decode_kernel<D, kType>;
-  static bool configured = false;
-  if (!configured) {
-    if (set_smem(kernel, C::kSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  const attn_status_t cst = configure_per_device(configured, [&] {
+    return launch_status(set_smem(kernel, C::kSmemBytes));
+  });
+  if (cst != ATTN_OK) return cst;
   const int grid = a.meta ? ds.G : ds.S;
   kernel<<<grid, 160, C::kSmemBytes, stream>>>(mk, mv, mkn, mvn, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -310,11 +326,11 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
     p.ws_lse = p.ws_o + slots * 2 * kMlaRows * kMlaDvHalf;
   }
   auto kernel = mla_kernel<kSparse>;
-  static bool configured = false;
-  if (!configured) {
-    if (set_smem(kernel, kMlaSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
-    configured = true;
-  }
+  static std::atomic<uint64_t> configured{0};
+  const attn_status_t cst = configure_per_device(configured, [&] {
+    return launch_status(set_smem(kernel, kMlaSmemBytes));
+  });
+  if (cst != ATTN_OK) return cst;
   // Clusters of two CTAs (the kernel's __cluster_dims__): one per segment, or
   // one per metadata slot.
   kernel<<<2 * (a.meta ? ds.G : ds.S), 192, kMlaSmemBytes, stream>>>(mq, mkv, p);
