@@ -25,6 +25,7 @@ OK, INVALID_ARG, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA_ERROR, DEVICE_ERROR = ra
 DTYPE_BF16, DTYPE_FP16, DTYPE_E4M3, DTYPE_E5M2, DTYPE_FP32 = range(5)
 SCHED_MHA, SCHED_MLA, SCHED_MLA_SPARSE = range(3)
 DEVERR_TIMEOUT, DEVERR_META_MISMATCH, DEVERR_SMEM_ALIGN = 1, 2, 3
+SELFTEST_SITE = 200
 
 _TORCH_DTYPE = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16,
                 torch.float8_e4m3fn: DTYPE_E4M3, torch.float8_e5m2: DTYPE_E5M2}
@@ -105,7 +106,8 @@ ARG_STRUCTS = {0: VarlenArgs, 1: SchedArgs, 2: PagedArgs, 3: CombineArgs, 4: Mla
 EXPORTS = ["attn_fwd_varlen", "attn_sched_metadata_size", "attn_sched_metadata",
            "attn_paged_workspace_size", "attn_fwd_paged_kvcache", "attn_combine",
            "mla_workspace_size", "mla_fwd_paged", "mla_sparse_fwd", "attn_get_device_error",
-           "attn_status_str", "attn_args_sizeof", "attn_fwd_paged_kvcache_static"]
+           "attn_status_str", "attn_args_sizeof", "attn_fwd_paged_kvcache_static",
+           "attn_selftest_wait_timeout"]
 
 _lib = None
 
@@ -141,6 +143,8 @@ def lib() -> ctypes.CDLL:
         L.attn_status_str.restype = ctypes.c_char_p
         L.attn_args_sizeof.argtypes = [c_i32]
         L.attn_args_sizeof.restype = c_sz
+        L.attn_selftest_wait_timeout.argtypes = [c_vp]
+        L.attn_selftest_wait_timeout.restype = c_i32
         _lib = L
     return _lib
 
@@ -199,6 +203,13 @@ def device_error(stream=None) -> int:
     if st not in (OK, DEVICE_ERROR):
         raise AttnError("attn_get_device_error", st)
     return code.value
+
+
+def selftest_wait_timeout(stream=None):
+    """Run the failure-detection self-test (attn_selftest_wait_timeout): a
+    bounded wait that nothing satisfies runs out and reports
+    DEVERR_TIMEOUT at SELFTEST_SITE. Read it with device_error()."""
+    _check("attn_selftest_wait_timeout", lib().attn_selftest_wait_timeout(_stream(stream)))
 
 
 def out_dtype_for(dtype: torch.dtype) -> torch.dtype:

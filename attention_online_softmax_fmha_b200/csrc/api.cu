@@ -41,6 +41,21 @@ attn_status_t configure_per_device(std::atomic<uint64_t>& done, F&& configure) {
   return st;
 }
 
+// The failure-detection self-test: one thread waits, with the kernels' own
+// bounded wait, on a barrier nothing arrives on (phase 0 never completes),
+// so the wait runs out, raises ATTN_DEVERR_TIMEOUT and the kernel returns.
+__global__ void __launch_bounds__(32, 1) selftest_wait_timeout_kernel() {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, ATTN_SELFTEST_SITE);
+}
+
 // Segments and units of a decode problem (see sched.cuh).
 struct DecodeShape {
   SchedShape sh;
@@ -510,6 +525,11 @@ attn_status_t mla_fwd_paged(const mla_args* a, void* stream) {
 }
 attn_status_t mla_sparse_fwd(const mla_args* a, void* stream) {
   return mla_entry(a, stream, true);
+}
+
+attn_status_t attn_selftest_wait_timeout(void* stream) {
+  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launch_status(cudaGetLastError());
 }
 
 attn_status_t attn_get_device_error(int32_t* code, void* stream) {

@@ -434,6 +434,15 @@ attn_status_t mla_sparse_fwd(const mla_args* args, void* stream);
 /* word was non-zero, ATTN_OK otherwise.                                     */
 attn_status_t attn_get_device_error(int32_t* code, void* stream);
 
+/* Failure-detection self-test. Launches one CTA on `stream` whose thread    */
+/* waits, with the same bounded wait the kernels use, on an mbarrier that     */
+/* nothing arrives on. The wait gives up after its limit (2 s), raises        */
+/* ATTN_DEVERR_TIMEOUT with site ATTN_SELFTEST_SITE in the device error word, */
+/* and the kernel returns; the context stays usable. Read the word with       */
+/* attn_get_device_error. Returns ATTN_ERR_CUDA if the launch fails.          */
+enum { ATTN_SELFTEST_SITE = 200 };
+attn_status_t attn_selftest_wait_timeout(void* stream);
+
 /* A static description of a status code. */
 const char* attn_status_str(int32_t status);
 
