@@ -64,7 +64,8 @@ def decode_bf16(bits: np.ndarray) -> np.ndarray:
     """bfloat16 is the upper half of an IEEE-754 binary32: widen the 16 bits
     into the high half of a 32-bit word and read it as binary32."""
     b = np.asarray(bits).astype(np.uint16).astype(np.uint32) << 16
-    return b.view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # NaN codes widen to NaN
+        return b.view(np.float32).astype(np.float64)
 
 
 def decode_fp16(bits: np.ndarray) -> np.ndarray:

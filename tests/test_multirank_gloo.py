@@ -34,7 +34,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks_reduce_max_and_rate():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of this (possibly CUDA) process
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     for r in range(world):
