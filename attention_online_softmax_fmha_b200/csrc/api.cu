@@ -4,7 +4,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -25,21 +24,6 @@ namespace {
 // ---------------------------------------------------------------------------
 // Scheduler metadata / paged decode / combine
 // ---------------------------------------------------------------------------
-
-// Runs `configure` (a kernel's function attributes) once per device: the
-// attributes belong to the current device's context, so every device needs
-// its own call. Devices past 63 configure on every launch. Safe under
-// concurrent callers (a repeated call is harmless).
-template <typename F>
-attn_status_t configure_per_device(std::atomic<uint64_t>& done, F&& configure) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
-  const uint64_t bit = dev < 64 ? uint64_t(1) << dev : 0;
-  if (bit && (done.load(std::memory_order_acquire) & bit)) return ATTN_OK;
-  const attn_status_t st = configure();
-  if (st == ATTN_OK && bit) done.fetch_or(bit, std::memory_order_release);
-  return st;
-}
 
 // The failure-detection self-test: one thread waits, with the kernels' own
 // bounded wait, on a barrier nothing arrives on (phase 0 never completes),

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -70,6 +71,21 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 attn_status_t launch_status(cudaError_t e) {
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// Runs `configure` (a kernel's function attributes) once per device: the
+// attributes belong to the current device's context, so every device needs
+// its own call. Devices past 63 configure on every launch. Safe under
+// concurrent callers (a repeated call is harmless).
+template <typename F>
+attn_status_t configure_per_device(std::atomic<uint64_t>& done, F&& configure) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  const uint64_t bit = dev < 64 ? uint64_t(1) << dev : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return ATTN_OK;
+  const attn_status_t st = configure();
+  if (st == ATTN_OK && bit) done.fetch_or(bit, std::memory_order_release);
+  return st;
 }
 
 bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }

@@ -22,16 +22,16 @@ attn_status_t launch_prefill(int grid, const CUtensorMap& mq, const CUtensorMap&
                              const CUtensorMap& mv, const PrefillParams& p, cudaStream_t stream) {
   using C = PrefillCfg<D, kType>;
   auto kernel = prefill_kernel<D, kType, kMask>;
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<uint64_t> configured{0};
+  const attn_status_t cst = configure_per_device(configured, [&]() -> attn_status_t {
     // The warpgroups trade registers with setmaxnreg out of the block's
     // launch allocation; that split is only valid at exactly this count.
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
     if (fa.numRegs != kPrefillLaunchRegs) return ATTN_ERR_UNSUPPORTED;
-    if (set_smem(kernel, C::kSmemBytes) != cudaSuccess) return ATTN_ERR_CUDA;
-    configured = true;
-  }
+    return launch_status(set_smem(kernel, C::kSmemBytes));
+  });
+  if (cst != ATTN_OK) return cst;
   kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
   return launch_status(cudaGetLastError());
 }
