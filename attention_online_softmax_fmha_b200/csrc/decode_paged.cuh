@@ -242,7 +242,8 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
   const int loads_per_tile = P >= kDecTileKeys ? 1 : kDecTileKeys / P;
   const int box_rows = P >= kDecTileKeys ? kDecTileKeys : P;
   int u = seg_begin_units, s = first_seg;
-  while (u < seg_end_units) {
+  bool stop = false;
+  while (u < seg_end_units && !stop) {
     // segment s covers units [seg_prefix(s), seg_prefix(s+1)) (or all of
     // one segment without metadata)
     int sb, se;
@@ -268,7 +269,10 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
       if (it >= kDecStages) {
         bool ok = true;
         if (lane == 0) ok = mbar_wait(&empty[st], ((it / kDecStages) - 1) & 1, abort, 31);
-        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+          stop = true;  // abort: stop issuing, but still drain what is in flight
+          break;
+        }
       }
       if (t >= sg.nct) {
         // appended keys: one 64-row box of the new k / v per 128-byte chunk
@@ -319,7 +323,8 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
     u = min(seg_end_units, se);
     ++s;
   }
-  // drain: the last stages' copies must land before the CTA exits
+  // drain (also after an abort): the last stages' copies must land before
+  // the CTA exits
   if (lane == 0) {
     int zero = 0;
     for (int i = max(0, it - kDecStages); i < it; ++i)
