@@ -222,7 +222,7 @@ attn_status_t run_decode(const attn_paged_args& a, const DecodeShape& ds, cudaSt
   });
   if (cst != ATTN_OK) return cst;
   const int grid = a.meta ? ds.G : ds.S;
-  kernel<<<grid, 160, C::kSmemBytes, stream>>>(mk, mv, mkn, mvn, p);
+  kernel<<<grid, kDecThreads, C::kSmemBytes, stream>>>(mk, mv, mkn, mvn, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (a.meta) {
     const int64_t warps = (int64_t)ds.S * kDecRows;

@@ -13,13 +13,16 @@
 //   warp 4      producer: reads the block-table entries 32 at a time and
 //               issues one TMA box per (page, 64-column chunk) for K and V,
 //               128-byte swizzled, into a 6-stage ring (32 KB per stage).
-//   warps 0-3   consumers: warp w owns keys [16w, 16w + 16) of every tile and
-//               keeps its own online-softmax state (running max, sums, O in
-//               registers). S = Q K^T and O += P V use mma.sync m16n8k16 with
-//               fp32 accumulation. With one consumer warp per SM
-//               sub-partition, a 64-key tile takes about as long to consume
-//               as a bf16 tile takes to load. At the end of a segment piece
-//               the four warp states are merged through shared memory.
+//   warps 0-7   consumers, two warpgroups taking alternate tiles (warpgroup
+//               it % 2 takes the CTA's it-th tile, so each stage of the even
+//               ring always goes to the same warpgroup). Warp w of a
+//               warpgroup owns keys [16w, 16w + 16) of its tiles and keeps its
+//               own online-softmax state (running max, sums, O in registers).
+//               S = Q K^T and O += P V use mma.sync m16n8k16 with fp32
+//               accumulation. Two consumer warps per SM sub-partition hide
+//               each other's per-tile latency chain (wait, ldmatrix, MMA,
+//               shuffles, exp2). At the end of a segment piece the eight warp
+//               states are merged through shared memory.
 // FP8 caches (e4m3 / e5m2, D = 128) arrive as 128-byte rows. S = Q K^T runs
 // on the FP8 codes directly (mma.sync m16n8k32, Q kept in FP8); each warp
 // rewrites its 16 V rows as fp16 (exact for both formats) in a private
@@ -42,7 +45,11 @@ namespace attn {
 
 constexpr int kDecTileKeys = 64;
 constexpr int kDecRows = 16;       // query rows per segment (mma M)
-constexpr int kDecStages = 6;
+constexpr int kDecStages = 6;      // even: stage st always feeds warpgroup st % 2
+constexpr int kDecConsumerWarps = 8;  // two warpgroups
+constexpr int kDecConsumerThreads = 32 * kDecConsumerWarps;
+constexpr int kDecThreads = kDecConsumerThreads + 32;  // + the producer warp
+static_assert(kDecStages % 2 == 0, "alternate tiles keep a stage with one warpgroup");
 
 struct DecodeParams {
   const void* q;
@@ -82,8 +89,8 @@ struct DecodeCfg {
   // FP8: each consumer warp's fp16 copy of its 16 V rows
   static constexpr int kStgWarpBytes = kFp8 ? 16 * D * 2 : 0;
   static constexpr int kStgOff = kQOff + kDecRows * kQStride;
-  static constexpr int kRedOff = kStgOff + 4 * kStgWarpBytes;  // merge buffers
-  static constexpr int kRedBytes = kDecRows * D * 4 + 4 * kDecRows * 4 * 3;
+  static constexpr int kRedOff = kStgOff + kDecConsumerWarps * kStgWarpBytes;  // merge buffers
+  static constexpr int kRedBytes = kDecRows * D * 4 + kDecConsumerWarps * kDecRows * 4 * 3;
   static constexpr int kBarOff = kRedOff + kRedBytes;
   static constexpr int kSmemBytes = kBarOff + 2 * kDecStages * 8 + 64 + 1024;
 };
@@ -235,7 +242,8 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
   const int loads_per_tile = P >= kDecTileKeys ? 1 : kDecTileKeys / P;
   const int box_rows = P >= kDecTileKeys ? kDecTileKeys : P;
   int u = seg_begin_units, s = first_seg;
-  while (u < seg_end_units) {
+  bool stop = false;
+  while (u < seg_end_units && !stop) {
     // segment s covers units [seg_prefix(s), seg_prefix(s+1)) (or all of
     // one segment without metadata)
     int sb, se;
@@ -261,7 +269,10 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
       if (it >= kDecStages) {
         bool ok = true;
         if (lane == 0) ok = mbar_wait(&empty[st], ((it / kDecStages) - 1) & 1, abort, 31);
-        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return;
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+          stop = true;  // abort: stop issuing, but still drain what is in flight
+          break;
+        }
       }
       if (t >= sg.nct) {
         // appended keys: one 64-row box of the new k / v per 128-byte chunk
@@ -312,7 +323,8 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
     u = min(seg_end_units, se);
     ++s;
   }
-  // drain: the last stages' copies must land before the CTA exits
+  // drain (also after an abort): the last stages' copies must land before
+  // the CTA exits
   if (lane == 0) {
     int zero = 0;
     for (int i = max(0, it - kDecStages); i < it; ++i)
@@ -331,15 +343,20 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
   constexpr bool kOutF16 = kType == 1;    // output: fp16 for fp16 input, else bf16
   using C = DecodeCfg<D, kFp8>;
   using InT = typename std::conditional<kOutF16, __half, __nv_bfloat16>::type;
-  const int tid = threadIdx.x;  // 0..127
-  const int warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;  // 0 .. kDecConsumerThreads - 1
+  const int gw = tid >> 5, lane = tid & 31;  // consumer warp 0..7
+  const int wg = gw >> 2, warp = gw & 3;     // warpgroup; key slice of its tiles
   const int qr = lane >> 2;          // fragment row (and row + 8)
   const int qc = (lane & 3) * 2;     // fragment column pair
   uint8_t* qs = smem + C::kQOff;
   float* red_o = reinterpret_cast<float*>(smem + C::kRedOff);  // [16][D]
-  float* red_m = red_o + kDecRows * D;                          // [4 warps][16]
-  float* red_l = red_m + 4 * kDecRows;
-  float* red_r = red_l + 4 * kDecRows;
+  float* red_m = red_o + kDecRows * D;                          // [8 warps][16]
+  float* red_l = red_m + kDecConsumerWarps * kDecRows;
+  float* red_r = red_l + kDecConsumerWarps * kDecRows;
+  // After a failed wait (timeout or abort) a warp skips the rest of its tiles
+  // but still takes every named barrier, so no other consumer warp is left
+  // waiting at one.
+  bool dead = false;
   const int32_t* meta = p.meta;
   const MetaLayout ml(p.num_ctas, p.num_segs);
   int it = 0;
@@ -362,9 +379,9 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
 
     // --- Q rows of the segment -> shared memory (16-bit, or the FP8 codes
     //     as they are; zero padded) ---
-    named_barrier(1, 128);  // previous piece finished with qs / red
+    named_barrier(1, kDecConsumerThreads);  // previous piece finished with qs / red
     constexpr int kQUnit = kFp8 ? 16 : 8;  // elements per 16-byte unit
-    for (int x = tid; x < kDecRows * (D / kQUnit); x += 128) {
+    for (int x = tid; x < kDecRows * (D / kQUnit); x += kDecConsumerThreads) {
       const int r = x / (D / kQUnit), cu = x % (D / kQUnit);
       uint4 v = make_uint4(0, 0, 0, 0);
       if (r < nrows) {
@@ -378,7 +395,7 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       }
       *reinterpret_cast<uint4*>(qs + r * C::kQStride + cu * 16) = v;
     }
-    named_barrier(1, 128);
+    named_barrier(1, kDecConsumerThreads);
     // A fragments of Q: one per 32-byte k-step (16 bf16/fp16 values, or 32
     // FP8 codes read through the same 16-bit ldmatrix view)
     constexpr int kKSteps = D * C::kElt / 32;
@@ -415,12 +432,20 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       vscale = p.v_descale[di];
     }
     // FP8: this warp's fp16 V tile (16 keys)
-    const uint32_t vstg = smem_u32(smem + C::kStgOff + warp * C::kStgWarpBytes);
+    const uint32_t vstg = smem_u32(smem + C::kStgOff + gw * C::kStgWarpBytes);
 
     for (int t = a; t < e; ++t) {
       if (!sg.visible(t)) continue;
       const int st = it % kDecStages;
-      if (!warp_wait(&full[st], (it / kDecStages) & 1, abort, 33)) return;
+      if ((it & 1) != wg || dead) {  // the other warpgroup's tile, or given up
+        ++it;
+        continue;
+      }
+      if (!warp_wait(&full[st], (it / kDecStages) & 1, abort, 33)) {
+        dead = true;
+        ++it;
+        continue;
+      }
       const uint32_t kbase = smem_u32(smem + C::kStageOff + st * C::kStageBytes);
       const uint32_t vbase = kbase + C::kTileBytes;
       // sequence position of this warp's first key, and the end of the valid
@@ -432,7 +457,7 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         // sequence become zeros (P = 0 must not meet a NaN there).
         __syncwarp();  // the previous tile's reads of the copy are done
         const uint8_t* vt = smem + C::kStageOff + st * C::kStageBytes + C::kTileBytes;
-#pragma unroll
+#pragma unroll 2
         for (int x = lane; x < 16 * (D / 16); x += 32) {
           const int kr = x / (D / 16), u = x % (D / 16);
           const int row = warp * 16 + kr;
@@ -545,7 +570,7 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       ++it;
     }
 
-    // --- merge the four warps' states -----------------------------------
+    // --- merge the eight warps' states ----------------------------------
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       l_run[h2] += __shfl_xor_sync(0xffffffffu, l_run[h2], 1);
@@ -554,22 +579,22 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       l_rnd[h2] += __shfl_xor_sync(0xffffffffu, l_rnd[h2], 2);
     }
     if ((lane & 3) == 0) {
-      red_m[warp * kDecRows + qr] = m_run[0];
-      red_m[warp * kDecRows + qr + 8] = m_run[1];
+      red_m[gw * kDecRows + qr] = m_run[0];
+      red_m[gw * kDecRows + qr + 8] = m_run[1];
     }
-    for (int x = tid; x < kDecRows * D; x += 128) red_o[x] = 0.f;
-    named_barrier(1, 128);
+    for (int x = tid; x < kDecRows * D; x += kDecConsumerThreads) red_o[x] = 0.f;
+    named_barrier(1, kDecConsumerThreads);
     float scale_w[2];
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       const int r = qr + h2 * 8;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w * kDecRows + r]);
+      for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, red_m[w * kDecRows + r]);
       scale_w[h2] = (m_run[h2] == -INFINITY) ? 0.f : ex2(m_run[h2] - M);
       if ((lane & 3) == 0) {
-        red_l[warp * kDecRows + r] = l_run[h2] * scale_w[h2];
-        red_r[warp * kDecRows + r] = l_rnd[h2] * scale_w[h2];
+        red_l[gw * kDecRows + r] = l_run[h2] * scale_w[h2];
+        red_r[gw * kDecRows + r] = l_rnd[h2] * scale_w[h2];
       }
     }
 #pragma unroll
@@ -580,7 +605,7 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       atomicAdd(&red_o[(qr + 8) * D + c], o[n][2] * scale_w[1]);
       atomicAdd(&red_o[(qr + 8) * D + c + 1], o[n][3] * scale_w[1]);
     }
-    named_barrier(1, 128);
+    named_barrier(1, kDecConsumerThreads);
 
     // --- write: thread -> (row, 16 columns) --------------------------------
     {
@@ -589,12 +614,12 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         nsplit = meta[ml.seg_nsplit + s];
         if (nsplit > 1) slot = meta[ml.seg_slot + s] + (blockIdx.x - meta[ml.seg_first + s]);
       }
-      constexpr int kPer = D / 8;  // columns per thread (8 threads per row)
+      constexpr int kPer = D / 8;  // columns per thread (8 threads per row, 128 threads)
       const int r = tid >> 3, c0 = (tid & 7) * kPer;
-      if (r < nrows) {
+      if (r < nrows) {  // tid < 128: r < 16 = kDecRows
         float M = -INFINITY, L = 0.f, LR = 0.f;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < kDecConsumerWarps; ++w) {
           M = fmaxf(M, red_m[w * kDecRows + r]);
           L += red_l[w * kDecRows + r];
           LR += red_r[w * kDecRows + r];
@@ -637,7 +662,7 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
 }
 
 template <int D, int kType>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(kDecThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v,
                   const __grid_constant__ CUtensorMap map_kn,
@@ -690,7 +715,7 @@ __global__ void __launch_bounds__(160, 1)
          (p.seqlen_new + kDecTileKeys - 1) / kDecTileKeys;
     if (ue == 0) ue = 1;  // still write O = 0, LSE = -inf for an empty sequence
   }
-  if (threadIdx.x >= 128) {
+  if (threadIdx.x >= kDecConsumerThreads) {
     decode_producer<D, kFp8>(p, &map_k, &map_v, &map_kn, &map_vn, smem, full, empty, abort, ub,
                              ue, s0, seg_prefix);
   } else {
