@@ -400,8 +400,10 @@ def combine(out_partial: np.ndarray, lse_partial: np.ndarray, sink=None):
 
 def mla_paged(q, kv_cache, block_table, cache_seqlens, head_dim_v, scale, causal=False,
               rows=None):
-    """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, 1, 576). K is the
-    whole row, V its first head_dim_v entries."""
+    """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, H_kv, 576). K is
+    the whole row, V its first head_dim_v entries. With H_kv > 1 (MATE
+    "Attention", MLA example: a cache of 2 KV heads) query head h reads KV
+    head floor(h / (H_q / H_kv)), as in GQA."""
     kv = np.asarray(kv_cache, np.float64)
     return attention_paged(q, kv, kv[..., :head_dim_v], block_table, cache_seqlens, scale,
                            causal, (-1, -1), None, rows)
@@ -409,9 +411,11 @@ def mla_paged(q, kv_cache, block_table, cache_seqlens, head_dim_v, scale, causal
 
 def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, scale,
                rows=None, block_size=1, causal=False):
-    """q (B, s_q, H_q, 576); indices (B, s_q, 1, topk) logical positions. Query
-    token (b, i) attends to the listed positions p with 0 <= p < L_b (each
-    listed occurrence counts once); the others are skipped.
+    """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, H_kv, 576);
+    indices (B, s_q, H_kv, topk) logical positions. Query token (b, i) of
+    head h attends, in KV head g = floor(h / (H_q / H_kv)), to the positions
+    listed in indices[b, i, g] with 0 <= p < L_b (each listed occurrence
+    counts once); the others are skipped.
     block_size > 1 (MindSpore "sparse_flash_attention": sparse_block_size, a
     power of two up to 128): each index k >= 0 lists the block of positions
     k * block_size .. k * block_size + block_size - 1 (reading: the index
@@ -422,7 +426,7 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
     q = np.asarray(q, np.float64)
     kv = np.asarray(kv_cache, np.float64)
     B, Sq, Hq, _ = q.shape
-    page = kv.shape[1]
+    page, Hkv = kv.shape[1], kv.shape[2]
     out = np.zeros((B, Sq, Hq, head_dim_v), np.float64)
     lse = np.full((B, Hq, Sq), NEG_INF, np.float64)
     want = None
@@ -435,17 +439,22 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
         for i in range(Sq):
             if want is not None and (b, i) not in want:
                 continue
-            hs = list(range(Hq)) if want is None else sorted(set(want[(b, i)]))
-            idx = np.asarray(indices[b, i, 0], dtype=np.int64)
-            if block_size > 1:
-                idx = idx[idx >= 0]
-                idx = (idx[:, None] * block_size + np.arange(block_size)[None, :]).reshape(-1)
-            idx = idx[(idx >= 0) & (idx < L)]
-            if causal:
-                idx = idx[idx <= i + L - Sq]
-            rows_kv = kv[np.asarray(block_table[b], np.int64)[idx // page], idx % page, 0, :]
-            vis = np.ones((len(hs), idx.size), dtype=bool)
-            o, l = attention_rows(q[b, i, hs, :], rows_kv, rows_kv[:, :head_dim_v], scale, vis)
-            out[b, i, hs, :] = o
-            lse[b, hs, i] = l
+            hs_all = list(range(Hq)) if want is None else sorted(set(want[(b, i)]))
+            for g in range(Hkv):
+                hs = [h for h in hs_all if _kv_head(h, Hq, Hkv) == g]
+                if not hs:
+                    continue
+                idx = np.asarray(indices[b, i, g], dtype=np.int64)
+                if block_size > 1:
+                    idx = idx[idx >= 0]
+                    idx = (idx[:, None] * block_size + np.arange(block_size)[None, :]).reshape(-1)
+                idx = idx[(idx >= 0) & (idx < L)]
+                if causal:
+                    idx = idx[idx <= i + L - Sq]
+                rows_kv = kv[np.asarray(block_table[b], np.int64)[idx // page], idx % page, g, :]
+                vis = np.ones((len(hs), idx.size), dtype=bool)
+                o, l = attention_rows(q[b, i, hs, :], rows_kv, rows_kv[:, :head_dim_v], scale,
+                                      vis)
+                out[b, i, hs, :] = o
+                lse[b, hs, i] = l
     return out, lse

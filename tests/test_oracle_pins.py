@@ -428,6 +428,28 @@ def test_mla_sparse_subset_matches_sdpa_on_gathered_rows():
 # Additive score mask and seqused (padded layout)
 # ---------------------------------------------------------------------------
 
+def test_mla_two_kv_heads_equal_each_group_alone():
+    # H_kv = 2: heads 0..G-1 read KV head 0 (and its index list), heads
+    # G..2G-1 KV head 1; each half equals the one-KV-head problem on its slice
+    lens, page, D, Dv, G, sq, topk = [9, 20], 4, 6, 4, 3, 2, 5
+    ck, _, bt = _paged_case(lens, page, 2, D, "permuted")
+    q = RNG.normal(size=(2, sq, 2 * G, D))
+    idx = np.stack([[[RNG.choice(max(L, 1) + 3, topk, replace=False) - 1 for _ in range(2)]
+                     for _ in range(sq)] for L in lens])
+    do, dl = oracle.mla_paged(q, ck, bt, lens, Dv, 0.5)
+    so, sl = oracle.mla_sparse(q, ck, bt, lens, idx, Dv, 0.5)
+    for g in range(2):
+        hs = slice(g * G, (g + 1) * G)
+        o1, l1 = oracle.mla_paged(q[:, :, hs], ck[:, :, g:g + 1], bt, lens, Dv, 0.5)
+        np.testing.assert_allclose(do[:, :, hs], o1, rtol=1e-13)
+        np.testing.assert_allclose(dl[:, hs], l1, rtol=1e-13)
+        o2, l2 = oracle.mla_sparse(q[:, :, hs], ck[:, :, g:g + 1], bt, lens,
+                                   idx[:, :, g:g + 1], Dv, 0.5)
+        np.testing.assert_allclose(so[:, :, hs], o2, rtol=1e-13)
+        np.testing.assert_allclose(sl[:, hs], l2, rtol=1e-13)
+    assert np.abs(so[:, :, :G] - so[:, :, G:]).max() > 1e-3
+
+
 def test_additive_mask_zero_and_constant_shift():
     """A zero mask changes nothing; a mask constant over a row's keys leaves O
     unchanged (softmax is shift-invariant) and adds the constant to the LSE."""
