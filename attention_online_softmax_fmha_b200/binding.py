@@ -97,7 +97,7 @@ class MlaArgs(ctypes.Structure):
                 ("idx_stride_b", c_i64), ("idx_stride_s", c_i64),
                 ("scale", c_f32), ("causal", c_i32), ("meta", c_vp), ("meta_bytes", c_sz),
                 ("num_ctas", c_i32), ("workspace", c_vp), ("workspace_bytes", c_sz),
-                ("sparse_block_size", c_i32)]
+                ("sparse_block_size", c_i32), ("kv_stride_h", c_i64), ("idx_stride_h", c_i64)]
 
 
 ARG_STRUCTS = {0: VarlenArgs, 1: SchedArgs, 2: PagedArgs, 3: CombineArgs, 4: MlaArgs}
@@ -422,7 +422,8 @@ def mla_args(q, kv_cache, block_table, cache_seqlens, *, head_dim_v=512, scale=N
         q.stride(1), q.stride(2), kv_cache.stride(0), kv_cache.stride(1), out.stride(0),
         out.stride(1), out.stride(2), 0 if indices is None else indices.stride(0),
         0 if indices is None else indices.stride(1), float(scale), int(bool(causal)), _ptr(meta),
-        0 if meta is None else meta.numel() * 4, int(num_ctas), None, 0, int(sparse_block_size))
+        0 if meta is None else meta.numel() * 4, int(num_ctas), None, 0, int(sparse_block_size),
+        kv_cache.stride(2), 0 if indices is None else indices.stride(2))
     if meta is not None:
         nbytes = int(lib().mla_workspace_size(ctypes.byref(a)))
         if workspace is None:
@@ -447,10 +448,10 @@ def mla_sparse_fwd(q, kv_cache, block_table, cache_seqlens, indices, *, stream=N
 
 
 def mla_metadata(inp_cache_seqlens, *, batch, seqlen_q, num_heads_q, page_size, topk=0,
-                 num_ctas=0, stream=None, sparse_block_size=0):
+                 num_ctas=0, stream=None, sparse_block_size=0, num_heads_kv=1):
     """Scheduler metadata for mla_fwd_paged (topk = 0) or mla_sparse_fwd."""
     return sched_metadata(inp_cache_seqlens, batch=batch, seqlen_q=seqlen_q,
-                          num_heads_q=num_heads_q, num_heads_kv=1, head_dim_qk=576,
+                          num_heads_q=num_heads_q, num_heads_kv=num_heads_kv, head_dim_qk=576,
                           head_dim_v=512, page_size=page_size,
                           mode=SCHED_MLA_SPARSE if topk else SCHED_MLA, topk=topk,
                           num_ctas=num_ctas, stream=stream, sparse_block_size=sparse_block_size)

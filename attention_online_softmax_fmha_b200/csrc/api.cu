@@ -77,16 +77,19 @@ attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int h
     ds.sh.segs_per_seq = heads_kv * ds.n_rsub;
     ds.sh.unit_keys = kDecTileKeys;
   } else {
-    if (heads_kv != 1 || !mla_heads_ok(heads_q)) return ATTN_ERR_UNSUPPORTED;
+    // row tiles of each KV head's group of query heads
+    ds.group = heads_q / heads_kv;
+    if (!mla_heads_ok(ds.group)) return ATTN_ERR_UNSUPPORTED;
     if (mode == ATTN_SCHED_MLA_SPARSE && topk <= 0) return ATTN_ERR_INVALID_ARG;
-    if (heads_q >= kMlaRows) {
-      ds.tiles_per_token = heads_q / kMlaRows;
+    if (ds.group >= kMlaRows) {
+      ds.tiles_per_token = ds.group / kMlaRows;
       ds.row_tiles = seqlen_q * ds.tiles_per_token;
     } else {
-      ds.tokens_per_tile = mode == ATTN_SCHED_MLA_SPARSE ? 1 : kMlaRows / heads_q;
+      ds.tokens_per_tile = mode == ATTN_SCHED_MLA_SPARSE ? 1 : kMlaRows / ds.group;
       ds.row_tiles = (seqlen_q + ds.tokens_per_tile - 1) / ds.tokens_per_tile;
     }
-    ds.sh.segs_per_seq = ds.row_tiles;  // both V halves: one cluster of two CTAs
+    // both V halves of a row tile: one cluster of two CTAs
+    ds.sh.segs_per_seq = heads_kv * ds.row_tiles;
     ds.sh.unit_keys = kMlaBN;
   }
   const int64_t S = (int64_t)batch * ds.sh.segs_per_seq;
@@ -255,8 +258,12 @@ attn_status_t check_mla(const mla_args* a, bool sparse) {
       !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
     return ATTN_ERR_INVALID_ARG;
   if (sparse && (a->idx_stride_b <= 0 || a->idx_stride_s <= 0)) return ATTN_ERR_INVALID_ARG;
+  if (a->num_heads_q % a->num_heads_kv) return ATTN_ERR_INVALID_ARG;
+  if (a->num_heads_kv > 1 &&
+      (!stride_ok(a->kv_stride_h, 2) || (sparse && a->idx_stride_h <= 0)))
+    return ATTN_ERR_INVALID_ARG;
   if (a->head_dim_qk != kMlaDqk || a->head_dim_v != kMlaDv) return ATTN_ERR_UNSUPPORTED;
-  if (a->num_heads_kv != 1 || !mla_heads_ok(a->num_heads_q)) return ATTN_ERR_UNSUPPORTED;
+  if (!mla_heads_ok(a->num_heads_q / a->num_heads_kv)) return ATTN_ERR_UNSUPPORTED;
   if (!pow2_in(a->page_size, 16, 256)) return ATTN_ERR_UNSUPPORTED;
   if (!sbs_ok(a->sparse_block_size) || (!sparse && a->sparse_block_size > 1))
     return ATTN_ERR_INVALID_ARG;
@@ -272,15 +279,19 @@ size_t mla_ws_bytes(const DecodeShape& ds) {
 
 template <bool kSparse>
 attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t stream) {
-  const int box_h = a.num_heads_q >= kMlaRows ? kMlaRows : a.num_heads_q;
-  const int box_t = a.num_heads_q >= kMlaRows ? 1 : ds.tokens_per_tile;
+  // Q boxes: the query heads of one KV head (128 at most) x the tile's tokens
+  const int box_h = ds.group >= kMlaRows ? kMlaRows : ds.group;
+  const int box_t = ds.group >= kMlaRows ? 1 : ds.tokens_per_tile;
+  // The cache as (576, page row, block, KV head); with one KV head the last
+  // stride only has to be valid.
+  const uint64_t kv_sh = a.num_heads_kv > 1 ? (uint64_t)a.kv_stride_h
+                                             : a.kv_stride_blk * (uint64_t)a.num_blocks;
   CUtensorMap mq, mkv;
   if (!encode_4d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk, a.num_heads_q,
                  a.seqlen_q, a.batch, a.q_stride_h, a.q_stride_s, a.q_stride_b, 64, box_h, box_t,
                  1) ||
       !encode_4d(&mkv, a.kv_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk, a.page_size,
-                 a.num_blocks, 1, a.kv_stride_tok, a.kv_stride_blk,
-                 a.kv_stride_blk * (uint64_t)a.num_blocks, 64,
+                 a.num_blocks, a.num_heads_kv, a.kv_stride_tok, a.kv_stride_blk, kv_sh, 64,
                  a.page_size >= kMlaBN ? kMlaBN : a.page_size, 1, 1))
     return ATTN_ERR_INVALID_ARG;
   MlaParams p;
@@ -302,11 +313,15 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   p.o_sh = a.o_stride_h;
   p.kv_sblk = a.kv_stride_blk;
   p.kv_stok = a.kv_stride_tok;
+  p.kv_sh = a.num_heads_kv > 1 ? a.kv_stride_h : 0;
   p.idx_sb = a.idx_stride_b;
   p.idx_ss = a.idx_stride_s;
+  p.idx_sh = a.num_heads_kv > 1 ? a.idx_stride_h : 0;
   p.batch = a.batch;
   p.seqlen_q = a.seqlen_q;
   p.heads_q = a.num_heads_q;
+  p.heads_kv = a.num_heads_kv;
+  p.group = ds.group;
   p.page_size = a.page_size;
   p.topk = a.topk;
   p.sbs = a.sparse_block_size > 1 ? a.sparse_block_size : 1;

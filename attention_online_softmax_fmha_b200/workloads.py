@@ -235,10 +235,10 @@ def make_paged(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, num_h
 
 @dataclasses.dataclass
 class MlaInputs:
-    """MLA-absorbed decode: one KV head whose 576-wide row is [512 latent | 64
-    rope]; V is the first 512 of the row."""
+    """MLA-absorbed decode: H_kv latent KV heads (usually 1) whose 576-wide
+    rows are [512 latent | 64 rope]; V is the first 512 of the row."""
     q: torch.Tensor                # (B, s_q, H_q, 576)
-    kv_cache: torch.Tensor         # (num_blocks, page_size, 1, 576)
+    kv_cache: torch.Tensor         # (num_blocks, page_size, H_kv, 576)
     block_table: torch.Tensor
     cache_seqlens: torch.Tensor
     seqlens: List[int]
@@ -247,8 +247,9 @@ class MlaInputs:
     head_dim_v: int
     causal: bool
     scale: float
-    indices: Optional[torch.Tensor]  # int32 (B, s_q, 1, topk) or None
+    indices: Optional[torch.Tensor]  # int32 (B, s_q, H_kv, topk) or None
     topk: int
+    num_heads_kv: int = 1
 
     @property
     def batch(self) -> int:
@@ -278,22 +279,25 @@ def sparse_indices(seqlens: Sequence[int], seqlen_q: int, topk: int, seed: int,
 def make_mla(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, page_size: int = 64,
              head_dim: int = 576, head_dim_v: int = 512, table: str = "permuted",
              causal: bool = False, topk: int = 0, index_kind: str = "uniform",
-             scale: Optional[float] = None, seed: int = 0, device="cpu") -> MlaInputs:
+             scale: Optional[float] = None, num_heads_kv: int = 1, seed: int = 0,
+             device="cpu") -> MlaInputs:
     seqlens = [int(x) for x in seqlens]
     g_cpu = _gen(seed + 7919, "cpu")
     bt, nblocks = _block_table(seqlens, page_size, table, g_cpu)
     g = _gen(seed, device)
     B = len(seqlens)
     q = _values((B, seqlen_q, num_heads_q, head_dim), "bf16", g, device)
-    kv = _values((nblocks, page_size, 1, head_dim), "bf16", g, device)
+    kv = _values((nblocks, page_size, num_heads_kv, head_dim), "bf16", g, device)
     idx = None
     if topk:
-        idx = sparse_indices(seqlens, seqlen_q, topk, seed, index_kind).to(device)
+        # one index list per KV head (the first with the given seed)
+        idx = torch.cat([sparse_indices(seqlens, seqlen_q, topk, seed + 7 * h, index_kind)
+                         for h in range(num_heads_kv)], dim=2).to(device)
     if scale is None:
         scale = 1.0 / math.sqrt(head_dim)
     return MlaInputs(q, kv, bt.to(device), torch.tensor(seqlens, dtype=torch.int32, device=device),
                      seqlens, page_size, num_heads_q, head_dim_v, bool(causal), float(scale), idx,
-                     int(topk))
+                     int(topk), int(num_heads_kv))
 
 
 # The five workloads the benchmark and the full-size parity tests use.
