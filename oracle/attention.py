@@ -458,3 +458,30 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
                 out[b, i, hs, :] = o
                 lse[b, hs, i] = l
     return out, lse
+
+
+def mla_sparse_tnd(q, kv_cache, block_table, cache_seqlens, cu_seqlens_q, indices, head_dim_v,
+                   scale, block_size=1, causal=False):
+    """The sparse MLA attention with packed (TND) queries (MindSpore
+    "sparse_flash_attention", layout_query="TND" with a paged cache): q
+    (T, H_q, 576) holds the query tokens of the B sequences back to back,
+    sequence b owning tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 (the
+    prefix-sum form of actual_seq_lengths_query); indices (T, H_kv, topk).
+    Each sequence is the BSND problem of its own tokens (token i of sequence
+    b is its i-th query row; causal aligns its last token with the cache's
+    last key). Returns out (T, H_q, D_v) and lse (H_q, T)."""
+    q = np.asarray(q, np.float64)
+    T, Hq, _ = q.shape
+    out = np.zeros((T, Hq, head_dim_v), np.float64)
+    lse = np.full((Hq, T), NEG_INF, np.float64)
+    cu = [int(x) for x in cu_seqlens_q]
+    for b in range(len(cu) - 1):
+        t0, t1 = cu[b], cu[b + 1]
+        if t1 <= t0:
+            continue
+        o, l = mla_sparse(q[None, t0:t1], kv_cache, np.asarray(block_table)[b:b + 1],
+                          [int(cache_seqlens[b])], np.asarray(indices)[None, t0:t1],
+                          head_dim_v, scale, block_size=block_size, causal=causal)
+        out[t0:t1] = o[0]
+        lse[:, t0:t1] = l[0]
+    return out, lse

@@ -450,6 +450,47 @@ def test_mla_two_kv_heads_equal_each_group_alone():
     assert np.abs(so[:, :, :G] - so[:, :, G:]).max() > 1e-3
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_mla_sparse_tnd_equal_lengths_is_bsnd_reshaped(causal):
+    # packed (TND) queries of equal-length sequences are the BSND problem
+    # with its batch and token axes merged
+    lens, page, D, Dv, Hq, S, topk = [9, 20, 14], 4, 6, 4, 2, 3, 6
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    q = RNG.normal(size=(3, S, Hq, D))
+    idx = np.stack([[[RNG.choice(L + 2, topk, replace=False) - 1] for _ in range(S)]
+                    for L in lens])
+    ro, rl = oracle.mla_sparse(q, ck, bt, lens, idx, Dv, 0.5, causal=causal)
+    cu = np.arange(4) * S
+    to, tl = oracle.mla_sparse_tnd(q.reshape(3 * S, Hq, D), ck, bt, lens, cu,
+                                   idx.reshape(3 * S, 1, topk), Dv, 0.5, causal=causal)
+    np.testing.assert_array_equal(to, ro.reshape(3 * S, Hq, Dv))
+    np.testing.assert_array_equal(tl, rl.transpose(1, 0, 2).reshape(Hq, 3 * S))
+
+
+def test_mla_sparse_tnd_unequal_lengths_follow_each_sequence():
+    # sequence b's tokens see only sequence b's cache; an empty sequence
+    # contributes no tokens
+    lens, page, D, Dv, Hq, topk = [9, 30, 14], 4, 6, 4, 2, 5
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    nq = [2, 0, 3]
+    cu = np.concatenate([[0], np.cumsum(nq)])
+    q = RNG.normal(size=(5, Hq, D))
+    idx = np.stack([[RNG.choice(lens[b] + 1, topk, replace=False) - 1]
+                    for b in range(3) for _ in range(nq[b])])
+    to, tl = oracle.mla_sparse_tnd(q, ck, bt, lens, cu, idx, Dv, 0.5, causal=True)
+    for b in (0, 2):
+        t0, t1 = cu[b], cu[b + 1]
+        o, l = oracle.mla_sparse(q[None, t0:t1], ck, bt[b:b + 1], [lens[b]], idx[None, t0:t1], Dv,
+                                 0.5, causal=True)
+        np.testing.assert_array_equal(to[t0:t1], o[0])
+        np.testing.assert_array_equal(tl[:, t0:t1], l[0])
+    # the other sequences' caches are not read: changing them changes nothing
+    ck2 = ck.copy()
+    ck2[bt[1][:8]] += 1.0
+    to2, _ = oracle.mla_sparse_tnd(q, ck2, bt, lens, cu, idx, Dv, 0.5, causal=True)
+    np.testing.assert_array_equal(to2, to)
+
+
 def test_additive_mask_zero_and_constant_shift():
     """A zero mask changes nothing; a mask constant over a row's keys leaves O
     unchanged (softmax is shift-invariant) and adds the constant to the LSE."""
