@@ -104,6 +104,11 @@ struct MlaParams {
   int64_t idx_sb, idx_ss, idx_sh;
   int32_t batch, seqlen_q, heads_q, page_size, topk;
   int32_t heads_kv, group;  // latent KV heads; query heads per KV head (H_q / H_kv)
+  // Packed (TND) sparse queries: the query side is one sequence of seqlen_q = T
+  // tokens (batch = 1); token t belongs to KV sequence b with
+  // cu_q[b] <= t < cu_q[b + 1] (batch_kv sequences). nullptr: BSND.
+  const int32_t* cu_q;
+  int32_t batch_kv;
   int32_t sbs;              // sparse: positions per index (sparse_block_size, >= 1)
   int32_t sbs_log2;         // log2(sbs) (sbs is a power of two)
   int32_t tiles_per_token;  // group >= 128: group / 128 (else 1)
@@ -128,7 +133,9 @@ static_assert(sizeof(MlaBarriers) <= 256, "barrier block");
 
 // A segment and its rows.
 struct MlaSeg {
-  int b, len;
+  int b, len;        // query-side batch index; cached keys of the KV sequence
+  int bk;            // KV-side sequence (block table, cache length): b, or TND's
+  int q0, sq;        // first token and token count of the query rows of sequence bk
   int kvg;           // KV head; its query heads are kvg * group .. + group - 1
   int tok0, head0;   // first (token, head within the group) of the row tile
   int rows_valid;    // rows of the tile that exist (the rest are padding)
@@ -141,7 +148,6 @@ DEVI void mla_seg(const MlaParams& p, int s, MlaSeg& g) {
   const int rem = s - g.b * p.segs_per_seq;  // (KV head, row tile) within the sequence
   g.kvg = rem / p.row_tiles;
   const int rt = rem - g.kvg * p.row_tiles;
-  g.len = p.cache_seqlens[g.b];
   if (p.group >= kMlaRows) {
     g.tok0 = rt / p.tiles_per_token;
     g.head0 = (rt % p.tiles_per_token) * kMlaRows;
@@ -151,6 +157,21 @@ DEVI void mla_seg(const MlaParams& p, int s, MlaSeg& g) {
     g.head0 = 0;
     g.rows_valid = kSparse ? p.group : min(kMlaRows, (p.seqlen_q - g.tok0) * p.group);
   }
+  g.bk = g.b;
+  g.q0 = 0;
+  g.sq = p.seqlen_q;
+  if (kSparse && p.cu_q) {
+    // the packed token's sequence: the last b with cu_q[b] <= tok0
+    int lo = 0, hi = p.batch_kv - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.cu_q[mid] <= g.tok0) lo = mid; else hi = mid - 1;
+    }
+    g.bk = lo;
+    g.q0 = p.cu_q[lo];
+    g.sq = p.cu_q[lo + 1] - g.q0;
+  }
+  g.len = p.cache_seqlens[g.bk];
   if (kSparse)
     g.units = (p.topk * p.sbs + kMlaBN - 1) / kMlaBN;
   else
@@ -255,7 +276,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
     }
     if (!__shfl_sync(0xffffffffu, (int)(*abort == 0), 0)) return;
     ++nq;
-    const int32_t* bt = p.block_table + (int64_t)g.b * p.bt_stride;
+    const int32_t* bt = p.block_table + (int64_t)g.bk * p.bt_stride;
     for (int t = a; t < e; ++t, ++it) {
       const int st = it % kMlaStages;
       uint8_t* dst = smem + kMlaKVOff + st * kMlaKVBytes;
@@ -541,7 +562,7 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     const bool valid_row = r < g.rows_valid && tok < p.seqlen_q;
     // dense: visible keys [0, hi]; causal aligns the last token with the last key
     int hi = g.len - 1;
-    if (p.causal) hi = min(hi, tok + g.len - p.seqlen_q);
+    if (p.causal) hi = min(hi, (tok - g.q0) + g.len - g.sq);
     const int* idx_row =
         kSparse ? p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss + g.kvg * p.idx_sh
                 : nullptr;

@@ -26,6 +26,7 @@ dtype conversion); FP8 E4M3 inputs are N(0, 1) converted by torch to
 from __future__ import annotations
 
 import dataclasses
+import itertools
 import math
 from typing import List, Optional, Sequence
 
@@ -298,6 +299,45 @@ def make_mla(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, page_si
     return MlaInputs(q, kv, bt.to(device), torch.tensor(seqlens, dtype=torch.int32, device=device),
                      seqlens, page_size, num_heads_q, head_dim_v, bool(causal), float(scale), idx,
                      int(topk), int(num_heads_kv))
+
+
+@dataclasses.dataclass
+class MlaTndInputs:
+    """Sparse MLA with packed (TND) queries: sequence b owns query tokens
+    cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and reads its own cache."""
+    q: torch.Tensor                # (T, H_q, 576)
+    kv_cache: torch.Tensor         # (num_blocks, page_size, 1, 576)
+    block_table: torch.Tensor
+    cache_seqlens: torch.Tensor
+    cu_seqlens_q: torch.Tensor     # int32 (B + 1)
+    seqlens: List[int]
+    seqlens_q: List[int]
+    page_size: int
+    num_heads_q: int
+    causal: bool
+    scale: float
+    indices: torch.Tensor          # int32 (T, 1, topk)
+    topk: int
+
+
+def make_mla_tnd(*, seqlens: Sequence[int], seqlens_q: Sequence[int], num_heads_q: int,
+                 topk: int, page_size: int = 64, causal: bool = False, seed: int = 0,
+                 device="cpu") -> MlaTndInputs:
+    seqlens = [int(x) for x in seqlens]
+    seqlens_q = [int(x) for x in seqlens_q]
+    g_cpu = _gen(seed + 7919, "cpu")
+    bt, nblocks = _block_table(seqlens, page_size, "permuted", g_cpu)
+    g = _gen(seed, device)
+    T = sum(seqlens_q)
+    q = _values((T, num_heads_q, 576), "bf16", g, device)
+    kv = _values((nblocks, page_size, 1, 576), "bf16", g, device)
+    idx = torch.cat([sparse_indices([L], n, topk, seed + b)[0, :, 0]
+                     for b, (L, n) in enumerate(zip(seqlens, seqlens_q)) if n > 0])
+    cu = torch.tensor([0] + list(itertools.accumulate(seqlens_q)), dtype=torch.int32)
+    return MlaTndInputs(q, kv, bt.to(device),
+                        torch.tensor(seqlens, dtype=torch.int32, device=device), cu.to(device),
+                        seqlens, seqlens_q, page_size, num_heads_q, bool(causal),
+                        1.0 / math.sqrt(576), idx[:, None, :].contiguous().to(device), int(topk))
 
 
 # The five workloads the benchmark and the full-size parity tests use.

@@ -405,6 +405,8 @@ typedef struct {
                               /* sparse_block_size); dense: must be 0 or 1     */
   int64_t kv_stride_h;        /* H_kv > 1: KV-head stride of kv_cache          */
   int64_t idx_stride_h;       /* H_kv > 1, sparse: KV-head stride of indices   */
+  const int32_t* cu_seqlens_q; /* mla_sparse_fwd with packed (TND) queries, or  */
+                              /* NULL; see mla_sparse_fwd                       */
 } mla_args;
 
 /* Bytes of workspace for these arguments (host only; 0 when meta is NULL).  */
@@ -424,6 +426,15 @@ attn_status_t mla_fwd_paged(const mla_args* args, void* stream);
 /* causal = 0: no mask beyond the index set (sparse_mode=0); causal = 1:    */
 /* also p <= i + cache_seqlens[b] - s_q (sparse_mode=3, "rightDownCausal").   */
 /* meta from attn_sched_metadata(mode=ATTN_SCHED_MLA_SPARSE) or NULL.        */
+/* Packed queries (MindSpore "sparse_flash_attention", layout_query="TND"   */
+/*   with a PA_BSND cache): cu_seqlens_q int32 (B+1) prefix sums, the        */
+/*   prefix-sum form of actual_seq_lengths_query. q (T, H_q, 576) with       */
+/*   seqlen_q = T (q/o/idx batch strides unused), indices (T, H_kv, topk),   */
+/*   out (T, H_q, 512), lse (H_q, T). Token t of sequence b (cu[b] <= t <   */
+/*   cu[b+1]) reads sequence b's cache; with causal, its row i = t - cu[b]   */
+/*   sees p <= i + cache_seqlens[b] - (cu[b+1] - cu[b]). The metadata is     */
+/*   made with batch = 1 and seqlen_q = T. Values of cu_seqlens_q are not    */
+/*   validated (cu[B] must equal T).                                         */
 /* ------------------------------------------------------------------------ */
 attn_status_t mla_sparse_fwd(const mla_args* args, void* stream);
 

@@ -207,3 +207,35 @@ def test_sparse_causal_right_down():
                                lens, inp.indices.cpu().numpy(), 512, inp.scale, causal=True)
     assert_close_out(to_f64(out), ro, 1e-2)
     assert_close_lse(lse.cpu().numpy(), rl)
+
+
+def _run_tnd(inp, use_meta, num_ctas=0):
+    T = inp.q.shape[0]
+    meta = None
+    if use_meta:
+        meta = B.mla_metadata(inp.cache_seqlens, batch=1, seqlen_q=T, num_heads_q=inp.num_heads_q,
+                              page_size=inp.page_size, topk=inp.topk, num_ctas=num_ctas)
+    out, lse = B.mla_sparse_fwd(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens,
+                                inp.indices, scale=inp.scale, causal=inp.causal, meta=meta,
+                                num_ctas=num_ctas, cu_seqlens_q=inp.cu_seqlens_q)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    return out, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sparse_packed_tnd_queries(causal):
+    """Packed (TND) queries (MindSpore sparse_flash_attention,
+    layout_query="TND"): sequence b's tokens read only sequence b's cache;
+    one sequence has no query token."""
+    inp = W.make_mla_tnd(seqlens=[20, 300, 3000, 50], seqlens_q=[3, 1, 5, 0], num_heads_q=128,
+                         topk=128, page_size=64, causal=causal, seed=42, device="cuda")
+    ro, rl = oracle.mla_sparse_tnd(to_f64(inp.q), to_f64(inp.kv_cache),
+                                   inp.block_table.cpu().numpy(), inp.seqlens,
+                                   inp.cu_seqlens_q.cpu().numpy(), inp.indices.cpu().numpy(), 512,
+                                   inp.scale, causal=causal)
+    for kw in (dict(use_meta=True, num_ctas=3), dict(use_meta=False)):
+        out, lse = _run_tnd(inp, **kw)
+        assert_close_out(to_f64(out), ro, 1e-2)
+        assert_close_lse(lse.cpu().numpy(), rl)
+
