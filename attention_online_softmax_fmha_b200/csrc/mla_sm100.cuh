@@ -245,7 +245,10 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
     for (; pend > 0; --pend) mbar_arrive(&bars->kv_full[(it - pend) % kMlaStages]);
   };
   int u = ub;
-  while (u < ue) {
+  // After a failed wait the producer stops issuing and falls through to the
+  // drains below, so no copy it issued lands after the CTA exits.
+  bool stop = false;
+  while (u < ue && !stop) {
     int sb, se;
     if (prefix) {
       sb = prefix[s];
@@ -264,8 +267,10 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       continue;
     }
     // Q tile of the segment: this CTA's chunks of the 576 columns
+    bool q_issued = false;
     if (lane == 0) {
       bool ok = nq == 0 || mbar_wait(&bars->q_empty, (nq - 1) & 1, abort, 60);
+      q_issued = ok;
       if (ok) {
         const int box_rows = p.group >= kMlaRows ? kMlaRows : p.group * (kSparse ? 1 : p.tokens_per_tile);
         mbar_expect_tx(&bars->q_full, nch * box_rows * 128);
@@ -274,8 +279,8 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
                       mla_chunk(rank, c) * 64, g.kvg * p.group + g.head0, g.tok0, g.b);
       }
     }
-    if (!__shfl_sync(0xffffffffu, (int)(*abort == 0), 0)) return;
-    ++nq;
+    if (__shfl_sync(0xffffffffu, q_issued ? 1 : 0, 0)) ++nq;
+    if (!__shfl_sync(0xffffffffu, (int)(*abort == 0), 0)) break;
     const int32_t* bt = p.block_table + (int64_t)g.bk * p.bt_stride;
     for (int t = a; t < e; ++t, ++it) {
       const int st = it % kMlaStages;
@@ -293,7 +298,8 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       }
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
         if constexpr (kSparse) flush_gathers();
-        return;
+        stop = true;
+        break;
       }
       if constexpr (!kSparse) {
         // keys [32t, 32t + 32): pages of the block table, one TMA box per
@@ -358,6 +364,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
         }
       }
     }
+    if (stop) break;
     // The segment's last S needs its last tiles before Q may be replaced.
     if constexpr (kSparse) flush_gathers();
     u = min(ue, se);
