@@ -227,9 +227,10 @@ def _run_tnd(inp, use_meta, num_ctas=0):
 def test_sparse_packed_tnd_queries(causal):
     """Packed (TND) queries (MindSpore sparse_flash_attention,
     layout_query="TND"): sequence b's tokens read only sequence b's cache;
-    one sequence has no query token."""
-    inp = W.make_mla_tnd(seqlens=[20, 300, 3000, 50], seqlens_q=[3, 1, 5, 0], num_heads_q=128,
-                         topk=128, page_size=64, causal=causal, seed=42, device="cuda")
+    two sequences (one in the middle) have no query token."""
+    inp = W.make_mla_tnd(seqlens=[20, 300, 3000, 50, 90], seqlens_q=[3, 0, 5, 2, 0],
+                         num_heads_q=128, topk=128, page_size=64, causal=causal, seed=42,
+                         device="cuda")
     ro, rl = oracle.mla_sparse_tnd(to_f64(inp.q), to_f64(inp.kv_cache),
                                    inp.block_table.cpu().numpy(), inp.seqlens,
                                    inp.cu_seqlens_q.cpu().numpy(), inp.indices.cpu().numpy(), 512,
