@@ -98,7 +98,8 @@ class MlaArgs(ctypes.Structure):
                 ("idx_stride_b", c_i64), ("idx_stride_s", c_i64),
                 ("scale", c_f32), ("causal", c_i32), ("meta", c_vp), ("meta_bytes", c_sz),
                 ("num_ctas", c_i32), ("workspace", c_vp), ("workspace_bytes", c_sz),
-                ("sparse_block_size", c_i32)]
+                ("sparse_block_size", c_i32), ("kv_stride_h", c_i64), ("idx_stride_h", c_i64),
+                ("cu_seqlens_q", c_vp)]
 
 
 ARG_STRUCTS = {0: VarlenArgs, 1: SchedArgs, 2: PagedArgs, 3: CombineArgs, 4: MlaArgs}
@@ -413,27 +414,49 @@ def combine(out_partial, lse_partial, *, num_splits_per_seq=None, sink=None, out
 
 def mla_args(q, kv_cache, block_table, cache_seqlens, *, head_dim_v=512, scale=None,
              causal=False, indices=None, meta=None, num_ctas=0, workspace=None, out=None,
-             lse=None, sparse_block_size=0):
+             lse=None, sparse_block_size=0, cu_seqlens_q=None):
+    """BSND: q (B, s_q, H_q, 576), indices (B, s_q, H_kv, topk); out
+    (B, s_q, H_q, 512), lse (B, H_q, s_q). Packed (TND, sparse only, with
+    cu_seqlens_q int32 (B+1)): q (T, H_q, 576), indices (T, H_kv, topk); out
+    (T, H_q, 512), lse (H_q, T)."""
     _rows(q=q, kv_cache=kv_cache, out=out, block_table=block_table, indices=indices)
     _same_dtype(q, kv_cache=kv_cache)
-    _dense(cache_seqlens=cache_seqlens, lse=lse)
-    _int32(block_table=block_table, cache_seqlens=cache_seqlens, indices=indices)
-    B, sq, Hq, Dqk = q.shape
-    if out is None:
-        out = torch.empty(B, sq, Hq, head_dim_v, device=q.device, dtype=torch.bfloat16)
-    if lse is None:
-        lse = torch.empty(B, Hq, sq, device=q.device, dtype=torch.float32)
+    _dense(cache_seqlens=cache_seqlens, lse=lse, cu_seqlens_q=cu_seqlens_q)
+    _int32(block_table=block_table, cache_seqlens=cache_seqlens, indices=indices,
+           cu_seqlens_q=cu_seqlens_q)
+    tnd = cu_seqlens_q is not None
+    if tnd:
+        if q.dim() != 3 or indices is None:
+            raise ValueError("packed queries: q (T, H_q, 576) and sparse indices")
+        B = cache_seqlens.numel()
+        sq, Hq, Dqk = q.shape
+        if out is None:
+            out = torch.empty(sq, Hq, head_dim_v, device=q.device, dtype=torch.bfloat16)
+        if lse is None:
+            lse = torch.empty(Hq, sq, device=q.device, dtype=torch.float32)
+        qs = (0, q.stride(0), q.stride(1))
+        os_ = (0, out.stride(0), out.stride(1))
+        ist = (0, indices.stride(0), indices.stride(1))
+    else:
+        B, sq, Hq, Dqk = q.shape
+        if out is None:
+            out = torch.empty(B, sq, Hq, head_dim_v, device=q.device, dtype=torch.bfloat16)
+        if lse is None:
+            lse = torch.empty(B, Hq, sq, device=q.device, dtype=torch.float32)
+        qs = (q.stride(0), q.stride(1), q.stride(2))
+        os_ = (out.stride(0), out.stride(1), out.stride(2))
+        ist = (0, 0, 0) if indices is None else (indices.stride(0), indices.stride(1),
+                                                 indices.stride(2))
     if scale is None:
         scale = 1.0 / math.sqrt(Dqk)
     topk = 0 if indices is None else indices.shape[-1]
     a = MlaArgs(
         _ptr(q), _ptr(kv_cache), _ptr(block_table), _ptr(cache_seqlens), _ptr(indices),
         _ptr(out), _ptr(lse), B, sq, Hq, kv_cache.shape[2], Dqk, head_dim_v, kv_cache.shape[1],
-        kv_cache.shape[0], block_table.shape[1], topk, block_table.stride(0), q.stride(0),
-        q.stride(1), q.stride(2), kv_cache.stride(0), kv_cache.stride(1), out.stride(0),
-        out.stride(1), out.stride(2), 0 if indices is None else indices.stride(0),
-        0 if indices is None else indices.stride(1), float(scale), int(bool(causal)), _ptr(meta),
-        0 if meta is None else meta.numel() * 4, int(num_ctas), None, 0, int(sparse_block_size))
+        kv_cache.shape[0], block_table.shape[1], topk, block_table.stride(0), *qs,
+        kv_cache.stride(0), kv_cache.stride(1), *os_, ist[0], ist[1], float(scale),
+        int(bool(causal)), _ptr(meta), 0 if meta is None else meta.numel() * 4, int(num_ctas),
+        None, 0, int(sparse_block_size), kv_cache.stride(2), ist[2], _ptr(cu_seqlens_q))
     if meta is not None:
         nbytes = int(lib().mla_workspace_size(ctypes.byref(a)))
         if workspace is None:
@@ -458,10 +481,11 @@ def mla_sparse_fwd(q, kv_cache, block_table, cache_seqlens, indices, *, stream=N
 
 
 def mla_metadata(inp_cache_seqlens, *, batch, seqlen_q, num_heads_q, page_size, topk=0,
-                 num_ctas=0, stream=None, sparse_block_size=0):
-    """Scheduler metadata for mla_fwd_paged (topk = 0) or mla_sparse_fwd."""
+                 num_ctas=0, stream=None, sparse_block_size=0, num_heads_kv=1):
+    """Scheduler metadata for mla_fwd_paged (topk = 0) or mla_sparse_fwd. For
+    packed (TND) queries pass batch=1 and seqlen_q=T."""
     return sched_metadata(inp_cache_seqlens, batch=batch, seqlen_q=seqlen_q,
-                          num_heads_q=num_heads_q, num_heads_kv=1, head_dim_qk=576,
+                          num_heads_q=num_heads_q, num_heads_kv=num_heads_kv, head_dim_qk=576,
                           head_dim_v=512, page_size=page_size,
                           mode=SCHED_MLA_SPARSE if topk else SCHED_MLA, topk=topk,
                           num_ctas=num_ctas, stream=stream, sparse_block_size=sparse_block_size)

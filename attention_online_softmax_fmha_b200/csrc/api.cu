@@ -76,16 +76,19 @@ attn_status_t decode_shape(int mode, int batch, int seqlen_q, int heads_q, int h
     ds.sh.segs_per_seq = heads_kv * ds.n_rsub;
     ds.sh.unit_keys = kDecTileKeys;
   } else {
-    if (heads_kv != 1 || !mla_heads_ok(heads_q)) return ATTN_ERR_UNSUPPORTED;
+    // row tiles of each KV head's group of query heads
+    ds.group = heads_q / heads_kv;
+    if (!mla_heads_ok(ds.group)) return ATTN_ERR_UNSUPPORTED;
     if (mode == ATTN_SCHED_MLA_SPARSE && topk <= 0) return ATTN_ERR_INVALID_ARG;
-    if (heads_q >= kMlaRows) {
-      ds.tiles_per_token = heads_q / kMlaRows;
+    if (ds.group >= kMlaRows) {
+      ds.tiles_per_token = ds.group / kMlaRows;
       ds.row_tiles = seqlen_q * ds.tiles_per_token;
     } else {
-      ds.tokens_per_tile = mode == ATTN_SCHED_MLA_SPARSE ? 1 : kMlaRows / heads_q;
+      ds.tokens_per_tile = mode == ATTN_SCHED_MLA_SPARSE ? 1 : kMlaRows / ds.group;
       ds.row_tiles = (seqlen_q + ds.tokens_per_tile - 1) / ds.tokens_per_tile;
     }
-    ds.sh.segs_per_seq = ds.row_tiles;  // both V halves: one cluster of two CTAs
+    // both V halves of a row tile: one cluster of two CTAs
+    ds.sh.segs_per_seq = heads_kv * ds.row_tiles;
     ds.sh.unit_keys = kMlaBN;
   }
   const int64_t S = (int64_t)batch * ds.sh.segs_per_seq;
@@ -248,14 +251,22 @@ attn_status_t check_mla(const mla_args* a, bool sparse) {
   if (a->block_table_stride < a->max_pages_per_seq) return ATTN_ERR_INVALID_ARG;
   if (!(a->scale > 0.f) || !std::isfinite(a->scale)) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(a->q) || !aligned16(a->kv_cache) || !aligned16(a->out)) return ATTN_ERR_INVALID_ARG;
-  if (!stride_ok(a->q_stride_b, 2) || !stride_ok(a->q_stride_s, 2) ||
-      !stride_ok(a->q_stride_h, 2) || !stride_ok(a->kv_stride_blk, 2) ||
-      !stride_ok(a->kv_stride_tok, 2) || !stride_ok(a->o_stride_b, 2) ||
+  // packed (TND) queries: sparse only; there is no query batch axis
+  const bool tnd = a->cu_seqlens_q != nullptr;
+  if (tnd && !sparse) return ATTN_ERR_UNSUPPORTED;
+  if ((!tnd && (!stride_ok(a->q_stride_b, 2) || !stride_ok(a->o_stride_b, 2))) ||
+      !stride_ok(a->q_stride_s, 2) || !stride_ok(a->q_stride_h, 2) ||
+      !stride_ok(a->kv_stride_blk, 2) || !stride_ok(a->kv_stride_tok, 2) ||
       !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
     return ATTN_ERR_INVALID_ARG;
-  if (sparse && (a->idx_stride_b <= 0 || a->idx_stride_s <= 0)) return ATTN_ERR_INVALID_ARG;
+  if (sparse && ((!tnd && a->idx_stride_b <= 0) || a->idx_stride_s <= 0))
+    return ATTN_ERR_INVALID_ARG;
+  if (a->num_heads_q % a->num_heads_kv) return ATTN_ERR_INVALID_ARG;
+  if (a->num_heads_kv > 1 &&
+      (!stride_ok(a->kv_stride_h, 2) || (sparse && a->idx_stride_h <= 0)))
+    return ATTN_ERR_INVALID_ARG;
   if (a->head_dim_qk != kMlaDqk || a->head_dim_v != kMlaDv) return ATTN_ERR_UNSUPPORTED;
-  if (a->num_heads_kv != 1 || !mla_heads_ok(a->num_heads_q)) return ATTN_ERR_UNSUPPORTED;
+  if (!mla_heads_ok(a->num_heads_q / a->num_heads_kv)) return ATTN_ERR_UNSUPPORTED;
   if (!pow2_in(a->page_size, 16, 256)) return ATTN_ERR_UNSUPPORTED;
   if (!sbs_ok(a->sparse_block_size) || (!sparse && a->sparse_block_size > 1))
     return ATTN_ERR_INVALID_ARG;
@@ -271,15 +282,22 @@ size_t mla_ws_bytes(const DecodeShape& ds) {
 
 template <bool kSparse>
 attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t stream) {
-  const int box_h = a.num_heads_q >= kMlaRows ? kMlaRows : a.num_heads_q;
-  const int box_t = a.num_heads_q >= kMlaRows ? 1 : ds.tokens_per_tile;
+  // Q boxes: the query heads of one KV head (128 at most) x the tile's tokens
+  const int box_h = ds.group >= kMlaRows ? kMlaRows : ds.group;
+  const int box_t = ds.group >= kMlaRows ? 1 : ds.tokens_per_tile;
+  // TND: the query side is one batch of seqlen_q = T packed tokens
+  const bool tnd = a.cu_seqlens_q != nullptr;
+  const int batch_q = tnd ? 1 : a.batch;
+  const uint64_t q_sb = tnd ? (uint64_t)a.q_stride_s * a.seqlen_q : (uint64_t)a.q_stride_b;
+  // The cache as (576, page row, block, KV head); with one KV head the last
+  // stride only has to be valid.
+  const uint64_t kv_sh = a.num_heads_kv > 1 ? (uint64_t)a.kv_stride_h
+                                             : a.kv_stride_blk * (uint64_t)a.num_blocks;
   CUtensorMap mq, mkv;
   if (!encode_4d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk, a.num_heads_q,
-                 a.seqlen_q, a.batch, a.q_stride_h, a.q_stride_s, a.q_stride_b, 64, box_h, box_t,
-                 1) ||
+                 a.seqlen_q, batch_q, a.q_stride_h, a.q_stride_s, q_sb, 64, box_h, box_t, 1) ||
       !encode_4d(&mkv, a.kv_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk, a.page_size,
-                 a.num_blocks, 1, a.kv_stride_tok, a.kv_stride_blk,
-                 a.kv_stride_blk * (uint64_t)a.num_blocks, 64,
+                 a.num_blocks, a.num_heads_kv, a.kv_stride_tok, a.kv_stride_blk, kv_sh, 64,
                  a.page_size >= kMlaBN ? kMlaBN : a.page_size, 1, 1))
     return ATTN_ERR_INVALID_ARG;
   MlaParams p;
@@ -293,19 +311,25 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   p.meta = a.meta;
   p.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv_cache);
   p.bt_stride = a.block_table_stride;
-  p.q_sb = a.q_stride_b;
+  p.q_sb = tnd ? 0 : a.q_stride_b;
   p.q_ss = a.q_stride_s;
   p.q_sh = a.q_stride_h;
-  p.o_sb = a.o_stride_b;
+  p.o_sb = tnd ? 0 : a.o_stride_b;
   p.o_ss = a.o_stride_s;
   p.o_sh = a.o_stride_h;
   p.kv_sblk = a.kv_stride_blk;
   p.kv_stok = a.kv_stride_tok;
-  p.idx_sb = a.idx_stride_b;
+  p.kv_sh = a.num_heads_kv > 1 ? a.kv_stride_h : 0;
+  p.idx_sb = tnd ? 0 : a.idx_stride_b;
   p.idx_ss = a.idx_stride_s;
-  p.batch = a.batch;
+  p.idx_sh = a.num_heads_kv > 1 ? a.idx_stride_h : 0;
+  p.batch = batch_q;
+  p.batch_kv = a.batch;
+  p.cu_q = a.cu_seqlens_q;
   p.seqlen_q = a.seqlen_q;
   p.heads_q = a.num_heads_q;
+  p.heads_kv = a.num_heads_kv;
+  p.group = ds.group;
   p.page_size = a.page_size;
   p.topk = a.topk;
   p.sbs = a.sparse_block_size > 1 ? a.sparse_block_size : 1;
@@ -347,7 +371,9 @@ attn_status_t mla_entry(const mla_args* a, void* stream, bool sparse) {
   if (st != ATTN_OK) return st;
   DecodeShape ds;
   const int mode = sparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
-  st = decode_shape(mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv,
+  // TND: the work is that of one batch of seqlen_q = T tokens
+  const int batch_q = a->cu_seqlens_q ? 1 : a->batch;
+  st = decode_shape(mode, batch_q, a->seqlen_q, a->num_heads_q, a->num_heads_kv,
                     sparse_positions(mode, a->topk, a->sparse_block_size), a->num_ctas, ds);
   if (st != ATTN_OK) return st;
   if (a->meta) {
@@ -497,7 +523,8 @@ size_t mla_workspace_size(const mla_args* a) {
   if (check_mla(a, sparse) != ATTN_OK) return 0;
   DecodeShape ds;
   const int mode = sparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
-  if (decode_shape(mode, a->batch, a->seqlen_q, a->num_heads_q, a->num_heads_kv,
+  if (decode_shape(mode, a->cu_seqlens_q ? 1 : a->batch, a->seqlen_q, a->num_heads_q,
+                   a->num_heads_kv,
                    sparse_positions(mode, a->topk, a->sparse_block_size), a->num_ctas,
                    ds) != ATTN_OK)
     return 0;

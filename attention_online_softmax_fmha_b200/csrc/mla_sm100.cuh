@@ -4,8 +4,11 @@
 // 512; flash_mla_sparse_fwd); MindSpore "sparse_flash_attention"
 // (attention_mode=2: the 512 latent ("nope") and 64 rope parts concatenated
 // along D; sparse_indices of logical positions; PA_BSND cache + block table).
-// One KV head: every query row (token i, head h) scores against the whole
-// 576-wide cached row; V is the row's first 512 entries.
+// Every query row (token i, head h) scores against the whole 576-wide cached
+// row of its KV head g = h / (H_q / H_kv); V is the row's first 512 entries.
+// With H_kv > 1 (the MATE MLA example's cache of 2 KV heads) the row tiles of
+// each KV head are separate segments; a segment reads only its KV head's
+// rows (and, sparse, its KV head's index list).
 //
 // Work decomposition. A cluster of two CTAs owns 128 query rows ("row tile")
 // and streams the keys once for both V halves: CTA rank r holds the score
@@ -18,9 +21,9 @@
 // (its first four 64-column chunks). Half of Q and of each key row per CTA
 // leaves room for a four-stage key ring, and the cache is read once per row
 // tile instead of once per V half.
-//   dense : segment = (sequence, row tile), keys 0 .. L-1 in tiles of 32
+//   dense : segment = (sequence, KV head, row tile), keys 0 .. L-1 in tiles of 32
 //           (causal: key j visible to token i iff j <= i + L - s_q).
-//   sparse: segment = (sequence, token, head tile), keys = that token's
+//   sparse: segment = (sequence, KV head, token, head tile), keys = that token's
 //           listed positions in tiles of 32 entries; entries outside [0, L)
 //           are skipped, and with causal (sparse_mode=3) those past
 //           i + L - s_q too.
@@ -97,14 +100,20 @@ struct MlaParams {
   int64_t bt_stride;
   int64_t q_sb, q_ss, q_sh;
   int64_t o_sb, o_ss, o_sh;
-  int64_t kv_sblk, kv_stok;
-  int64_t idx_sb, idx_ss;
+  int64_t kv_sblk, kv_stok, kv_sh;
+  int64_t idx_sb, idx_ss, idx_sh;
   int32_t batch, seqlen_q, heads_q, page_size, topk;
+  int32_t heads_kv, group;  // latent KV heads; query heads per KV head (H_q / H_kv)
+  // Packed (TND) sparse queries: the query side is one sequence of seqlen_q = T
+  // tokens (batch = 1); token t belongs to KV sequence b with
+  // cu_q[b] <= t < cu_q[b + 1] (batch_kv sequences). nullptr: BSND.
+  const int32_t* cu_q;
+  int32_t batch_kv;
   int32_t sbs;              // sparse: positions per index (sparse_block_size, >= 1)
   int32_t sbs_log2;         // log2(sbs) (sbs is a power of two)
-  int32_t tiles_per_token;  // heads_q >= 128: heads_q / 128 (else 1)
-  int32_t tokens_per_tile;  // heads_q < 128: 128 / heads_q (else 1)
-  int32_t row_tiles;        // dense: row tiles per sequence
+  int32_t tiles_per_token;  // group >= 128: group / 128 (else 1)
+  int32_t tokens_per_tile;  // group < 128: 128 / group (else 1)
+  int32_t row_tiles;        // row tiles per (sequence, KV head)
   int32_t segs_per_seq, num_segs, num_ctas;  // num_ctas: clusters (metadata slots)
   float scale_log2;
   int32_t causal;
@@ -124,8 +133,11 @@ static_assert(sizeof(MlaBarriers) <= 256, "barrier block");
 
 // A segment and its rows.
 struct MlaSeg {
-  int b, len;
-  int tok0, head0;   // first (token, head) of the row tile
+  int b, len;        // query-side batch index; cached keys of the KV sequence
+  int bk;            // KV-side sequence (block table, cache length): b, or TND's
+  int q0, sq;        // first token and token count of the query rows of sequence bk
+  int kvg;           // KV head; its query heads are kvg * group .. + group - 1
+  int tok0, head0;   // first (token, head within the group) of the row tile
   int rows_valid;    // rows of the tile that exist (the rest are padding)
   int units;         // KV tiles of the segment
 };
@@ -133,17 +145,33 @@ struct MlaSeg {
 template <bool kSparse>
 DEVI void mla_seg(const MlaParams& p, int s, MlaSeg& g) {
   g.b = s / p.segs_per_seq;
-  const int rt = s - g.b * p.segs_per_seq;  // row tile index within the sequence
-  g.len = p.cache_seqlens[g.b];
-  if (p.heads_q >= kMlaRows) {
+  const int rem = s - g.b * p.segs_per_seq;  // (KV head, row tile) within the sequence
+  g.kvg = rem / p.row_tiles;
+  const int rt = rem - g.kvg * p.row_tiles;
+  if (p.group >= kMlaRows) {
     g.tok0 = rt / p.tiles_per_token;
     g.head0 = (rt % p.tiles_per_token) * kMlaRows;
     g.rows_valid = kMlaRows;
   } else {
     g.tok0 = kSparse ? rt : rt * p.tokens_per_tile;
     g.head0 = 0;
-    g.rows_valid = kSparse ? p.heads_q : min(kMlaRows, (p.seqlen_q - g.tok0) * p.heads_q);
+    g.rows_valid = kSparse ? p.group : min(kMlaRows, (p.seqlen_q - g.tok0) * p.group);
   }
+  g.bk = g.b;
+  g.q0 = 0;
+  g.sq = p.seqlen_q;
+  if (kSparse && p.cu_q) {
+    // the packed token's sequence: the last b with cu_q[b] <= tok0
+    int lo = 0, hi = p.batch_kv - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.cu_q[mid] <= g.tok0) lo = mid; else hi = mid - 1;
+    }
+    g.bk = lo;
+    g.q0 = p.cu_q[lo];
+    g.sq = p.cu_q[lo + 1] - g.q0;
+  }
+  g.len = p.cache_seqlens[g.bk];
   if (kSparse)
     g.units = (p.topk * p.sbs + kMlaBN - 1) / kMlaBN;
   else
@@ -152,21 +180,21 @@ DEVI void mla_seg(const MlaParams& p, int s, MlaSeg& g) {
 
 // Key position of entry e of token tok's sparse list (-1: skipped): with
 // sparse_block_size bs, index k >= 0 lists positions k*bs .. k*bs + bs - 1.
-DEVI int mla_sparse_pos(const MlaParams& p, int b, int tok, int e) {
+DEVI int mla_sparse_pos(const MlaParams& p, int b, int kvg, int tok, int e) {
   if (e >= (p.topk << p.sbs_log2)) return -1;
   const int blk = e >> p.sbs_log2;
-  const int k = __ldg(p.indices + b * p.idx_sb + (int64_t)tok * p.idx_ss + blk);
+  const int k = __ldg(p.indices + b * p.idx_sb + (int64_t)tok * p.idx_ss + kvg * p.idx_sh + blk);
   return k >= 0 ? (k << p.sbs_log2) + (e & (p.sbs - 1)) : -1;
 }
 
-// Token and head of tile row x.
+// Token and (global) query head of tile row x.
 DEVI void mla_row(const MlaParams& p, const MlaSeg& g, int x, int& tok, int& head) {
-  if (p.heads_q >= kMlaRows) {
+  if (p.group >= kMlaRows) {
     tok = g.tok0;
-    head = g.head0 + x;
+    head = g.kvg * p.group + g.head0 + x;
   } else {
-    tok = g.tok0 + x / p.heads_q;
-    head = x % p.heads_q;
+    tok = g.tok0 + x / p.group;
+    head = g.kvg * p.group + x % p.group;
   }
 }
 
@@ -217,7 +245,10 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
     for (; pend > 0; --pend) mbar_arrive(&bars->kv_full[(it - pend) % kMlaStages]);
   };
   int u = ub;
-  while (u < ue) {
+  // After a failed wait the producer stops issuing and falls through to the
+  // drains below, so no copy it issued lands after the CTA exits.
+  bool stop = false;
+  while (u < ue && !stop) {
     int sb, se;
     if (prefix) {
       sb = prefix[s];
@@ -236,19 +267,21 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       continue;
     }
     // Q tile of the segment: this CTA's chunks of the 576 columns
+    bool q_issued = false;
     if (lane == 0) {
       bool ok = nq == 0 || mbar_wait(&bars->q_empty, (nq - 1) & 1, abort, 60);
+      q_issued = ok;
       if (ok) {
-        const int box_rows = p.heads_q >= kMlaRows ? kMlaRows : p.heads_q * (kSparse ? 1 : p.tokens_per_tile);
+        const int box_rows = p.group >= kMlaRows ? kMlaRows : p.group * (kSparse ? 1 : p.tokens_per_tile);
         mbar_expect_tx(&bars->q_full, nch * box_rows * 128);
         for (int c = 0; c < nch; ++c)
           tma_load_4d(smem + kMlaQOff + c * kMlaQChunkBytes, mq, &bars->q_full,
-                      mla_chunk(rank, c) * 64, g.head0, g.tok0, g.b);
+                      mla_chunk(rank, c) * 64, g.kvg * p.group + g.head0, g.tok0, g.b);
       }
     }
-    if (!__shfl_sync(0xffffffffu, (int)(*abort == 0), 0)) return;
-    ++nq;
-    const int32_t* bt = p.block_table + (int64_t)g.b * p.bt_stride;
+    if (__shfl_sync(0xffffffffu, q_issued ? 1 : 0, 0)) ++nq;
+    if (!__shfl_sync(0xffffffffu, (int)(*abort == 0), 0)) break;
+    const int32_t* bt = p.block_table + (int64_t)g.bk * p.bt_stride;
     for (int t = a; t < e; ++t, ++it) {
       const int st = it % kMlaStages;
       uint8_t* dst = smem + kMlaKVOff + st * kMlaKVBytes;
@@ -265,7 +298,8 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       }
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
         if constexpr (kSparse) flush_gathers();
-        return;
+        stop = true;
+        break;
       }
       if constexpr (!kSparse) {
         // keys [32t, 32t + 32): pages of the block table, one TMA box per
@@ -284,7 +318,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
           if (lane == 0)
             for (int c = 0; c < nch; ++c)
               tma_load_4d(dst + c * kMlaKVChunkBytes + j * box * 128, mkv, &bars->kv_full[st],
-                          mla_chunk(rank, c) * 64, key0 % P, pg, 0);
+                          mla_chunk(rank, c) * 64, key0 % P, pg, g.kvg);
         }
       } else {
         // lane k gathers key t*32 + k: 8 async copies of 16 bytes per chunk
@@ -292,13 +326,16 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
         int pos = -1;
         if (p.sbs_log2 == 0) {  // one key per index: the index itself
           const int e_idx = t * kMlaBN + lane;
-          if (e_idx < p.topk) pos = p.indices[g.b * p.idx_sb + g.tok0 * p.idx_ss + e_idx];
+          if (e_idx < p.topk)
+            pos = p.indices[g.b * p.idx_sb + g.tok0 * p.idx_ss + g.kvg * p.idx_sh + e_idx];
         } else {
-          pos = mla_sparse_pos(p, g.b, g.tok0, t * kMlaBN + lane);
+          pos = mla_sparse_pos(p, g.b, g.kvg, g.tok0, t * kMlaBN + lane);
         }
         const bool valid = pos >= 0 && pos < g.len;
         const __nv_bfloat16* src = nullptr;
-        if (valid) src = p.kv + (int64_t)bt[pos / P] * p.kv_sblk + (int64_t)(pos % P) * p.kv_stok;
+        if (valid)
+          src = p.kv + g.kvg * p.kv_sh + (int64_t)bt[pos / P] * p.kv_sblk +
+                (int64_t)(pos % P) * p.kv_stok;
         const uint32_t dbase = smem_u32(dst) + lane * 128;
         for (int c = 0; c < nch; ++c) {
           const int gc = mla_chunk(rank, c);
@@ -327,6 +364,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
         }
       }
     }
+    if (stop) break;
     // The segment's last S needs its last tiles before Q may be replaced.
     if constexpr (kSparse) flush_gathers();
     u = min(ue, se);
@@ -531,9 +569,10 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     const bool valid_row = r < g.rows_valid && tok < p.seqlen_q;
     // dense: visible keys [0, hi]; causal aligns the last token with the last key
     int hi = g.len - 1;
-    if (p.causal) hi = min(hi, tok + g.len - p.seqlen_q);
+    if (p.causal) hi = min(hi, (tok - g.q0) + g.len - g.sq);
     const int* idx_row =
-        kSparse ? p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss : nullptr;
+        kSparse ? p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss + g.kvg * p.idx_sh
+                : nullptr;
     float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
     bool seen = false;
     // The partial scores of tile g + 1 go to the other CTA as soon as those of
@@ -761,7 +800,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     s_bad = 0;
     if (p.meta) {
       const int mode = kSparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
-      if (!(meta_matches(p.meta, mode, p.batch, p.seqlen_q, p.heads_q, 1, p.page_size,
+      if (!(meta_matches(p.meta, mode, p.batch, p.seqlen_q, p.heads_q, p.heads_kv, p.page_size,
                          p.num_segs, kMlaBN, kMlaDqk, kMlaDv) &&
             p.meta[kMetaNumCtas] == p.num_ctas &&
             (!kSparse || p.meta[kMetaTopk] == p.topk * p.sbs))) {
@@ -809,8 +848,8 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaParams p) {
   const int vh = (gw / kMlaRows) & 1, r = gw % kMlaRows;
   if (s >= p.num_segs) return;
   const int mode = kSparse ? ATTN_SCHED_MLA_SPARSE : ATTN_SCHED_MLA;
-  if (!(meta_matches(p.meta, mode, p.batch, p.seqlen_q, p.heads_q, 1, p.page_size, p.num_segs,
-                     kMlaBN, kMlaDqk, kMlaDv) &&
+  if (!(meta_matches(p.meta, mode, p.batch, p.seqlen_q, p.heads_q, p.heads_kv, p.page_size,
+                     p.num_segs, kMlaBN, kMlaDqk, kMlaDv) &&
         p.meta[kMetaNumCtas] == p.num_ctas))
     return;
   const MetaLayout ml(p.num_ctas, p.num_segs);

@@ -26,6 +26,7 @@ dtype conversion); FP8 E4M3 inputs are N(0, 1) converted by torch to
 from __future__ import annotations
 
 import dataclasses
+import itertools
 import math
 from typing import List, Optional, Sequence
 
@@ -235,10 +236,10 @@ def make_paged(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, num_h
 
 @dataclasses.dataclass
 class MlaInputs:
-    """MLA-absorbed decode: one KV head whose 576-wide row is [512 latent | 64
-    rope]; V is the first 512 of the row."""
+    """MLA-absorbed decode: H_kv latent KV heads (usually 1) whose 576-wide
+    rows are [512 latent | 64 rope]; V is the first 512 of the row."""
     q: torch.Tensor                # (B, s_q, H_q, 576)
-    kv_cache: torch.Tensor         # (num_blocks, page_size, 1, 576)
+    kv_cache: torch.Tensor         # (num_blocks, page_size, H_kv, 576)
     block_table: torch.Tensor
     cache_seqlens: torch.Tensor
     seqlens: List[int]
@@ -247,8 +248,9 @@ class MlaInputs:
     head_dim_v: int
     causal: bool
     scale: float
-    indices: Optional[torch.Tensor]  # int32 (B, s_q, 1, topk) or None
+    indices: Optional[torch.Tensor]  # int32 (B, s_q, H_kv, topk) or None
     topk: int
+    num_heads_kv: int = 1
 
     @property
     def batch(self) -> int:
@@ -278,22 +280,64 @@ def sparse_indices(seqlens: Sequence[int], seqlen_q: int, topk: int, seed: int,
 def make_mla(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, page_size: int = 64,
              head_dim: int = 576, head_dim_v: int = 512, table: str = "permuted",
              causal: bool = False, topk: int = 0, index_kind: str = "uniform",
-             scale: Optional[float] = None, seed: int = 0, device="cpu") -> MlaInputs:
+             scale: Optional[float] = None, num_heads_kv: int = 1, seed: int = 0,
+             device="cpu") -> MlaInputs:
     seqlens = [int(x) for x in seqlens]
     g_cpu = _gen(seed + 7919, "cpu")
     bt, nblocks = _block_table(seqlens, page_size, table, g_cpu)
     g = _gen(seed, device)
     B = len(seqlens)
     q = _values((B, seqlen_q, num_heads_q, head_dim), "bf16", g, device)
-    kv = _values((nblocks, page_size, 1, head_dim), "bf16", g, device)
+    kv = _values((nblocks, page_size, num_heads_kv, head_dim), "bf16", g, device)
     idx = None
     if topk:
-        idx = sparse_indices(seqlens, seqlen_q, topk, seed, index_kind).to(device)
+        # one index list per KV head (the first with the given seed)
+        idx = torch.cat([sparse_indices(seqlens, seqlen_q, topk, seed + 7 * h, index_kind)
+                         for h in range(num_heads_kv)], dim=2).to(device)
     if scale is None:
         scale = 1.0 / math.sqrt(head_dim)
     return MlaInputs(q, kv, bt.to(device), torch.tensor(seqlens, dtype=torch.int32, device=device),
                      seqlens, page_size, num_heads_q, head_dim_v, bool(causal), float(scale), idx,
-                     int(topk))
+                     int(topk), int(num_heads_kv))
+
+
+@dataclasses.dataclass
+class MlaTndInputs:
+    """Sparse MLA with packed (TND) queries: sequence b owns query tokens
+    cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and reads its own cache."""
+    q: torch.Tensor                # (T, H_q, 576)
+    kv_cache: torch.Tensor         # (num_blocks, page_size, 1, 576)
+    block_table: torch.Tensor
+    cache_seqlens: torch.Tensor
+    cu_seqlens_q: torch.Tensor     # int32 (B + 1)
+    seqlens: List[int]
+    seqlens_q: List[int]
+    page_size: int
+    num_heads_q: int
+    causal: bool
+    scale: float
+    indices: torch.Tensor          # int32 (T, 1, topk)
+    topk: int
+
+
+def make_mla_tnd(*, seqlens: Sequence[int], seqlens_q: Sequence[int], num_heads_q: int,
+                 topk: int, page_size: int = 64, causal: bool = False, seed: int = 0,
+                 device="cpu") -> MlaTndInputs:
+    seqlens = [int(x) for x in seqlens]
+    seqlens_q = [int(x) for x in seqlens_q]
+    g_cpu = _gen(seed + 7919, "cpu")
+    bt, nblocks = _block_table(seqlens, page_size, "permuted", g_cpu)
+    g = _gen(seed, device)
+    T = sum(seqlens_q)
+    q = _values((T, num_heads_q, 576), "bf16", g, device)
+    kv = _values((nblocks, page_size, 1, 576), "bf16", g, device)
+    idx = torch.cat([sparse_indices([L], n, topk, seed + b)[0, :, 0]
+                     for b, (L, n) in enumerate(zip(seqlens, seqlens_q)) if n > 0])
+    cu = torch.tensor([0] + list(itertools.accumulate(seqlens_q)), dtype=torch.int32)
+    return MlaTndInputs(q, kv, bt.to(device),
+                        torch.tensor(seqlens, dtype=torch.int32, device=device), cu.to(device),
+                        seqlens, seqlens_q, page_size, num_heads_q, bool(causal),
+                        1.0 / math.sqrt(576), idx[:, None, :].contiguous().to(device), int(topk))
 
 
 # The five workloads the benchmark and the full-size parity tests use.

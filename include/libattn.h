@@ -358,21 +358,22 @@ attn_status_t attn_combine(const attn_combine_args* args, void* stream);
 /* with 576-wide rows and head_dim_v=512); MindSpore "sparse_flash_attention"*/
 /* (attention_mode=2: nope (512) and rope (64) parts concatenated along D).  */
 /*                                                                          */
-/* q (B, s_q, H_q, 576) bf16; kv_cache (num_blocks, page_size, 1, 576) bf16, */
-/* each row [512 latent | 64 rope]; K is the whole row, V its first          */
-/* head_dim_v (= 512) entries. block_table, cache_seqlens as in              */
-/* attn_fwd_paged_kvcache. out (B, s_q, H_q, 512) bf16; lse (B, H_q, s_q)    */
-/* fp32 nullable. meta from attn_sched_metadata(mode=ATTN_SCHED_MLA) or      */
-/* NULL; workspace from mla_workspace_size().                                */
-/* Supported now: H_kv = 1, H_q * s_q a multiple of 64 up to 1024,           */
-/*   page_size a multiple of 16; H_kv > 1 returns UNSUPPORTED.               */
+/* q (B, s_q, H_q, 576) bf16; kv_cache (num_blocks, page_size, H_kv, 576)   */
+/* bf16, each row [512 latent | 64 rope]; K is the whole row, V its first    */
+/* head_dim_v (= 512) entries. Query head h reads KV head h / (H_q / H_kv)  */
+/* (the MATE example's cache has 2 KV heads). block_table, cache_seqlens as  */
+/* in attn_fwd_paged_kvcache. out (B, s_q, H_q, 512) bf16; lse (B, H_q, s_q) */
+/* fp32 nullable. meta from attn_sched_metadata(mode=ATTN_SCHED_MLA, same    */
+/* H_q and H_kv) or NULL; workspace from mla_workspace_size().               */
+/* Supported now: H_q / H_kv a power of two up to 128 or a multiple of 128;  */
+/*   page_size a power of two in [16, 256].                                  */
 /* ------------------------------------------------------------------------ */
 typedef struct {
   const void* q;
   const void* kv_cache;
   const int32_t* block_table;
   const int32_t* cache_seqlens;
-  const int32_t* indices;     /* mla_sparse_fwd only: (B, s_q, 1, topk)     */
+  const int32_t* indices;     /* mla_sparse_fwd only: (B, s_q, H_kv, topk)  */
   void* out;
   float* lse;
   int32_t batch;
@@ -402,6 +403,10 @@ typedef struct {
                               /* index k >= 0 lists positions k*bs .. k*bs+bs-1 */
                               /* (MindSpore sparse_flash_attention             */
                               /* sparse_block_size); dense: must be 0 or 1     */
+  int64_t kv_stride_h;        /* H_kv > 1: KV-head stride of kv_cache          */
+  int64_t idx_stride_h;       /* H_kv > 1, sparse: KV-head stride of indices   */
+  const int32_t* cu_seqlens_q; /* mla_sparse_fwd with packed (TND) queries, or  */
+                              /* NULL; see mla_sparse_fwd                       */
 } mla_args;
 
 /* Bytes of workspace for these arguments (host only; 0 when meta is NULL).  */
@@ -421,6 +426,15 @@ attn_status_t mla_fwd_paged(const mla_args* args, void* stream);
 /* causal = 0: no mask beyond the index set (sparse_mode=0); causal = 1:    */
 /* also p <= i + cache_seqlens[b] - s_q (sparse_mode=3, "rightDownCausal").   */
 /* meta from attn_sched_metadata(mode=ATTN_SCHED_MLA_SPARSE) or NULL.        */
+/* Packed queries (MindSpore "sparse_flash_attention", layout_query="TND"   */
+/*   with a PA_BSND cache): cu_seqlens_q int32 (B+1) prefix sums, the        */
+/*   prefix-sum form of actual_seq_lengths_query. q (T, H_q, 576) with       */
+/*   seqlen_q = T (q/o/idx batch strides unused), indices (T, H_kv, topk),   */
+/*   out (T, H_q, 512), lse (H_q, T). Token t of sequence b (cu[b] <= t <   */
+/*   cu[b+1]) reads sequence b's cache; with causal, its row i = t - cu[b]   */
+/*   sees p <= i + cache_seqlens[b] - (cu[b+1] - cu[b]). The metadata is     */
+/*   made with batch = 1 and seqlen_q = T. Values of cu_seqlens_q are not    */
+/*   validated (cu[B] must equal T).                                         */
 /* ------------------------------------------------------------------------ */
 attn_status_t mla_sparse_fwd(const mla_args* args, void* stream);
 

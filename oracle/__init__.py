@@ -6,5 +6,6 @@ library. It shares no code with the CUDA path.
 """
 from .attention import *  # noqa: F401,F403
 from .attention import (attention_rows, attention_varlen, attention_padded, attention_paged,
-                        combine, decode, mla_paged, mla_sparse, visible_mask, visible_range,
+                        combine, decode, mla_paged, mla_sparse, mla_sparse_tnd, visible_mask,
+                        visible_range,
                         gather_pages)

@@ -401,8 +401,10 @@ def combine(out_partial: np.ndarray, lse_partial: np.ndarray, sink=None):
 
 def mla_paged(q, kv_cache, block_table, cache_seqlens, head_dim_v, scale, causal=False,
               rows=None):
-    """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, 1, 576). K is the
-    whole row, V its first head_dim_v entries."""
+    """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, H_kv, 576). K is
+    the whole row, V its first head_dim_v entries. With H_kv > 1 (MATE
+    "Attention", MLA example: a cache of 2 KV heads) query head h reads KV
+    head floor(h / (H_q / H_kv)), as in GQA."""
     kv = np.asarray(kv_cache, np.float64)
     return attention_paged(q, kv, kv[..., :head_dim_v], block_table, cache_seqlens, scale,
                            causal, (-1, -1), None, rows)
@@ -410,9 +412,11 @@ def mla_paged(q, kv_cache, block_table, cache_seqlens, head_dim_v, scale, causal
 
 def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, scale,
                rows=None, block_size=1, causal=False):
-    """q (B, s_q, H_q, 576); indices (B, s_q, 1, topk) logical positions. Query
-    token (b, i) attends to the listed positions p with 0 <= p < L_b (each
-    listed occurrence counts once); the others are skipped.
+    """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, H_kv, 576);
+    indices (B, s_q, H_kv, topk) logical positions. Query token (b, i) of
+    head h attends, in KV head g = floor(h / (H_q / H_kv)), to the positions
+    listed in indices[b, i, g] with 0 <= p < L_b (each listed occurrence
+    counts once); the others are skipped.
     block_size > 1 (MindSpore "sparse_flash_attention": sparse_block_size, a
     power of two up to 128): each index k >= 0 lists the block of positions
     k * block_size .. k * block_size + block_size - 1 (reading: the index
@@ -423,7 +427,7 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
     q = np.asarray(q, np.float64)
     kv = np.asarray(kv_cache, np.float64)
     B, Sq, Hq, _ = q.shape
-    page = kv.shape[1]
+    page, Hkv = kv.shape[1], kv.shape[2]
     out = np.zeros((B, Sq, Hq, head_dim_v), np.float64)
     lse = np.full((B, Hq, Sq), NEG_INF, np.float64)
     want = None
@@ -436,17 +440,49 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
         for i in range(Sq):
             if want is not None and (b, i) not in want:
                 continue
-            hs = list(range(Hq)) if want is None else sorted(set(want[(b, i)]))
-            idx = np.asarray(indices[b, i, 0], dtype=np.int64)
-            if block_size > 1:
-                idx = idx[idx >= 0]
-                idx = (idx[:, None] * block_size + np.arange(block_size)[None, :]).reshape(-1)
-            idx = idx[(idx >= 0) & (idx < L)]
-            if causal:
-                idx = idx[idx <= i + L - Sq]
-            rows_kv = kv[np.asarray(block_table[b], np.int64)[idx // page], idx % page, 0, :]
-            vis = np.ones((len(hs), idx.size), dtype=bool)
-            o, l = attention_rows(q[b, i, hs, :], rows_kv, rows_kv[:, :head_dim_v], scale, vis)
-            out[b, i, hs, :] = o
-            lse[b, hs, i] = l
+            hs_all = list(range(Hq)) if want is None else sorted(set(want[(b, i)]))
+            for g in range(Hkv):
+                hs = [h for h in hs_all if _kv_head(h, Hq, Hkv) == g]
+                if not hs:
+                    continue
+                idx = np.asarray(indices[b, i, g], dtype=np.int64)
+                if block_size > 1:
+                    idx = idx[idx >= 0]
+                    idx = (idx[:, None] * block_size + np.arange(block_size)[None, :]).reshape(-1)
+                idx = idx[(idx >= 0) & (idx < L)]
+                if causal:
+                    idx = idx[idx <= i + L - Sq]
+                rows_kv = kv[np.asarray(block_table[b], np.int64)[idx // page], idx % page, g, :]
+                vis = np.ones((len(hs), idx.size), dtype=bool)
+                o, l = attention_rows(q[b, i, hs, :], rows_kv, rows_kv[:, :head_dim_v], scale,
+                                      vis)
+                out[b, i, hs, :] = o
+                lse[b, hs, i] = l
+    return out, lse
+
+
+def mla_sparse_tnd(q, kv_cache, block_table, cache_seqlens, cu_seqlens_q, indices, head_dim_v,
+                   scale, block_size=1, causal=False):
+    """The sparse MLA attention with packed (TND) queries (MindSpore
+    "sparse_flash_attention", layout_query="TND" with a paged cache): q
+    (T, H_q, 576) holds the query tokens of the B sequences back to back,
+    sequence b owning tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 (the
+    prefix-sum form of actual_seq_lengths_query); indices (T, H_kv, topk).
+    Each sequence is the BSND problem of its own tokens (token i of sequence
+    b is its i-th query row; causal aligns its last token with the cache's
+    last key). Returns out (T, H_q, D_v) and lse (H_q, T)."""
+    q = np.asarray(q, np.float64)
+    T, Hq, _ = q.shape
+    out = np.zeros((T, Hq, head_dim_v), np.float64)
+    lse = np.full((Hq, T), NEG_INF, np.float64)
+    cu = [int(x) for x in cu_seqlens_q]
+    for b in range(len(cu) - 1):
+        t0, t1 = cu[b], cu[b + 1]
+        if t1 <= t0:
+            continue
+        o, l = mla_sparse(q[None, t0:t1], kv_cache, np.asarray(block_table)[b:b + 1],
+                          [int(cache_seqlens[b])], np.asarray(indices)[None, t0:t1],
+                          head_dim_v, scale, block_size=block_size, causal=causal)
+        out[t0:t1] = o[0]
+        lse[:, t0:t1] = l[0]
     return out, lse

@@ -133,6 +133,19 @@ def test_sched_rejects_appended_keys_outside_gqa_decode(L):
     assert L.attn_sched_metadata(ctypes.byref(a), None) == B.INVALID_ARG
 
 
+def test_mla_packed_queries_are_sparse_only(L):
+    a = B.MlaArgs()
+    base = dict(q=0x1000, kv_cache=0x2000, block_table=0x3000, cache_seqlens=0x4000,
+                out=0x5000, batch=2, seqlen_q=9, num_heads_q=128, num_heads_kv=1,
+                head_dim_qk=576, head_dim_v=512, page_size=64, num_blocks=8,
+                max_pages_per_seq=4, block_table_stride=4, q_stride_s=128 * 576,
+                q_stride_h=576, kv_stride_blk=64 * 576, kv_stride_tok=576,
+                o_stride_s=128 * 512, o_stride_h=512, scale=0.04, cu_seqlens_q=0x6000)
+    for k, v in base.items():
+        setattr(a, k, v)
+    assert L.mla_fwd_paged(ctypes.byref(a), None) == B.UNSUPPORTED  # dense: BSND only
+
+
 def test_null_struct_is_invalid(L):
     for fn in ["attn_fwd_varlen", "attn_sched_metadata", "attn_fwd_paged_kvcache",
                "attn_combine", "mla_fwd_paged", "mla_sparse_fwd"]:

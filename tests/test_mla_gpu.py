@@ -26,7 +26,7 @@ def run(inp, use_meta=True, num_ctas=0):
     if use_meta:
         meta = B.mla_metadata(inp.cache_seqlens, batch=inp.batch, seqlen_q=inp.q.shape[1],
                               num_heads_q=inp.num_heads_q, page_size=inp.page_size, topk=topk,
-                              num_ctas=num_ctas)
+                              num_ctas=num_ctas, num_heads_kv=inp.num_heads_kv)
     kw = dict(scale=inp.scale, causal=inp.causal, meta=meta, num_ctas=num_ctas)
     if inp.indices is None:
         out, lse = B.mla_fwd_paged(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, **kw)
@@ -70,23 +70,40 @@ def test_dense_without_metadata_causal_and_page16():
 
 def test_mate_example_shapes():
     # The MATE MLA example: q (1, 32, 8, 576), a 4-page cache of 16-token
-    # pages, block_table all zeros, cache_seqlens [32], head_dim_v 512. Its
-    # cache has 2 KV heads, which is rejected; with one KV head it runs (the
-    # all-zero table repeats page 0).
+    # pages with 2 KV heads, block_table all zeros (page 0 repeats),
+    # cache_seqlens [32], head_dim_v 512; with and without metadata.
     g = torch.Generator(device="cuda").manual_seed(0)
     q = torch.randn(1, 32, 8, 576, generator=g, device="cuda").to(torch.bfloat16)
     bt = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
     cs = torch.tensor([32], dtype=torch.int32, device="cuda")
     kv2 = torch.randn(4, 16, 2, 576, generator=g, device="cuda").to(torch.bfloat16)
-    with pytest.raises(B.AttnError) as e:
-        B.mla_fwd_paged(q, kv2, bt, cs, head_dim_v=512)
-    assert e.value.status == B.UNSUPPORTED
-    kv1 = kv2[:, :, :1].contiguous()
-    out, lse = B.mla_fwd_paged(q, kv1, bt, cs, head_dim_v=512)
-    torch.cuda.synchronize()
-    ro, rl = oracle.mla_paged(to_f64(q), to_f64(kv1), bt.cpu().numpy(), [32], 512, 1 / 24.0)
-    assert_close_out(to_f64(out), ro, 1e-2)
-    assert_close_lse(lse.cpu().numpy(), rl)
+    ro, rl = oracle.mla_paged(to_f64(q), to_f64(kv2), bt.cpu().numpy(), [32], 512, 1 / 24.0)
+    meta = B.mla_metadata(cs, batch=1, seqlen_q=32, num_heads_q=8, page_size=16, num_ctas=3,
+                          num_heads_kv=2)
+    for kw in (dict(), dict(meta=meta, num_ctas=3)):
+        out, lse = B.mla_fwd_paged(q, kv2, bt, cs, head_dim_v=512, **kw)
+        torch.cuda.synchronize()
+        assert B.device_error() == 0
+        assert_close_out(to_f64(out), ro, 1e-2)
+        assert_close_lse(lse.cpu().numpy(), rl)
+
+
+@pytest.mark.parametrize("Hq,Hkv,sq", [(256, 2, 1), (64, 4, 3)])
+def test_dense_several_kv_heads(Hq, Hkv, sq):
+    # 128 query heads per KV head (one row tile per token), and 16 (eight
+    # tokens per row tile); split and unsplit
+    inp = W.make_mla(seqlens=[7, 100, 700], seqlen_q=sq, num_heads_q=Hq, num_heads_kv=Hkv,
+                     page_size=32, causal=sq > 1, seed=40, device="cuda")
+    check(inp, num_ctas=5)
+    check(inp, use_meta=False)
+
+
+def test_sparse_several_kv_heads():
+    inp = W.make_mla(seqlens=[20, 300, 3000], seqlen_q=2, num_heads_q=128, num_heads_kv=2,
+                     page_size=64, topk=128, seed=41, device="cuda")
+    assert not torch.equal(inp.indices[:, :, 0], inp.indices[:, :, 1])
+    check(inp, num_ctas=3)
+    check(inp, use_meta=False)
 
 
 @pytest.mark.parametrize("num_ctas", [3, 0])
@@ -190,3 +207,36 @@ def test_sparse_causal_right_down():
                                lens, inp.indices.cpu().numpy(), 512, inp.scale, causal=True)
     assert_close_out(to_f64(out), ro, 1e-2)
     assert_close_lse(lse.cpu().numpy(), rl)
+
+
+def _run_tnd(inp, use_meta, num_ctas=0):
+    T = inp.q.shape[0]
+    meta = None
+    if use_meta:
+        meta = B.mla_metadata(inp.cache_seqlens, batch=1, seqlen_q=T, num_heads_q=inp.num_heads_q,
+                              page_size=inp.page_size, topk=inp.topk, num_ctas=num_ctas)
+    out, lse = B.mla_sparse_fwd(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens,
+                                inp.indices, scale=inp.scale, causal=inp.causal, meta=meta,
+                                num_ctas=num_ctas, cu_seqlens_q=inp.cu_seqlens_q)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    return out, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sparse_packed_tnd_queries(causal):
+    """Packed (TND) queries (MindSpore sparse_flash_attention,
+    layout_query="TND"): sequence b's tokens read only sequence b's cache;
+    two sequences (one in the middle) have no query token."""
+    inp = W.make_mla_tnd(seqlens=[20, 300, 3000, 50, 90], seqlens_q=[3, 0, 5, 2, 0],
+                         num_heads_q=128, topk=128, page_size=64, causal=causal, seed=42,
+                         device="cuda")
+    ro, rl = oracle.mla_sparse_tnd(to_f64(inp.q), to_f64(inp.kv_cache),
+                                   inp.block_table.cpu().numpy(), inp.seqlens,
+                                   inp.cu_seqlens_q.cpu().numpy(), inp.indices.cpu().numpy(), 512,
+                                   inp.scale, causal=causal)
+    for kw in (dict(use_meta=True, num_ctas=3), dict(use_meta=False)):
+        out, lse = _run_tnd(inp, **kw)
+        assert_close_out(to_f64(out), ro, 1e-2)
+        assert_close_lse(lse.cpu().numpy(), rl)
+

@@ -428,6 +428,69 @@ def test_mla_sparse_subset_matches_sdpa_on_gathered_rows():
 # Additive score mask and seqused (padded layout)
 # ---------------------------------------------------------------------------
 
+def test_mla_two_kv_heads_equal_each_group_alone():
+    # H_kv = 2: heads 0..G-1 read KV head 0 (and its index list), heads
+    # G..2G-1 KV head 1; each half equals the one-KV-head problem on its slice
+    lens, page, D, Dv, G, sq, topk = [9, 20], 4, 6, 4, 3, 2, 5
+    ck, _, bt = _paged_case(lens, page, 2, D, "permuted")
+    q = RNG.normal(size=(2, sq, 2 * G, D))
+    idx = np.stack([[[RNG.choice(max(L, 1) + 3, topk, replace=False) - 1 for _ in range(2)]
+                     for _ in range(sq)] for L in lens])
+    do, dl = oracle.mla_paged(q, ck, bt, lens, Dv, 0.5)
+    so, sl = oracle.mla_sparse(q, ck, bt, lens, idx, Dv, 0.5)
+    for g in range(2):
+        hs = slice(g * G, (g + 1) * G)
+        o1, l1 = oracle.mla_paged(q[:, :, hs], ck[:, :, g:g + 1], bt, lens, Dv, 0.5)
+        np.testing.assert_allclose(do[:, :, hs], o1, rtol=1e-13)
+        np.testing.assert_allclose(dl[:, hs], l1, rtol=1e-13)
+        o2, l2 = oracle.mla_sparse(q[:, :, hs], ck[:, :, g:g + 1], bt, lens,
+                                   idx[:, :, g:g + 1], Dv, 0.5)
+        np.testing.assert_allclose(so[:, :, hs], o2, rtol=1e-13)
+        np.testing.assert_allclose(sl[:, hs], l2, rtol=1e-13)
+    assert np.abs(so[:, :, :G] - so[:, :, G:]).max() > 1e-3
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_mla_sparse_tnd_equal_lengths_is_bsnd_reshaped(causal):
+    # packed (TND) queries of equal-length sequences are the BSND problem
+    # with its batch and token axes merged
+    lens, page, D, Dv, Hq, S, topk = [9, 20, 14], 4, 6, 4, 2, 3, 6
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    q = RNG.normal(size=(3, S, Hq, D))
+    idx = np.stack([[[RNG.choice(L + 2, topk, replace=False) - 1] for _ in range(S)]
+                    for L in lens])
+    ro, rl = oracle.mla_sparse(q, ck, bt, lens, idx, Dv, 0.5, causal=causal)
+    cu = np.arange(4) * S
+    to, tl = oracle.mla_sparse_tnd(q.reshape(3 * S, Hq, D), ck, bt, lens, cu,
+                                   idx.reshape(3 * S, 1, topk), Dv, 0.5, causal=causal)
+    np.testing.assert_array_equal(to, ro.reshape(3 * S, Hq, Dv))
+    np.testing.assert_array_equal(tl, rl.transpose(1, 0, 2).reshape(Hq, 3 * S))
+
+
+def test_mla_sparse_tnd_unequal_lengths_follow_each_sequence():
+    # sequence b's tokens see only sequence b's cache; an empty sequence
+    # contributes no tokens
+    lens, page, D, Dv, Hq, topk = [9, 30, 14], 4, 6, 4, 2, 5
+    ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
+    nq = [2, 0, 3]
+    cu = np.concatenate([[0], np.cumsum(nq)])
+    q = RNG.normal(size=(5, Hq, D))
+    idx = np.stack([[RNG.choice(lens[b] + 1, topk, replace=False) - 1]
+                    for b in range(3) for _ in range(nq[b])])
+    to, tl = oracle.mla_sparse_tnd(q, ck, bt, lens, cu, idx, Dv, 0.5, causal=True)
+    for b in (0, 2):
+        t0, t1 = cu[b], cu[b + 1]
+        o, l = oracle.mla_sparse(q[None, t0:t1], ck, bt[b:b + 1], [lens[b]], idx[None, t0:t1], Dv,
+                                 0.5, causal=True)
+        np.testing.assert_array_equal(to[t0:t1], o[0])
+        np.testing.assert_array_equal(tl[:, t0:t1], l[0])
+    # the other sequences' caches are not read: changing them changes nothing
+    ck2 = ck.copy()
+    ck2[bt[1][:8]] += 1.0
+    to2, _ = oracle.mla_sparse_tnd(q, ck2, bt, lens, cu, idx, Dv, 0.5, causal=True)
+    np.testing.assert_array_equal(to2, to)
+
+
 def test_additive_mask_zero_and_constant_shift():
     """A zero mask changes nothing; a mask constant over a row's keys leaves O
     unchanged (softmax is shift-invariant) and adds the constant to the LSE."""
