@@ -39,6 +39,10 @@ from attention_online_softmax_fmha_b200 import workloads as W  # noqa: E402
 
 METRIC = "prefill TFLOP/s & decode KV GB/s on 1 B200; % of tensor/HBM roofline"
 HEADLINE = "varlen_causal_gqa"
+# Timed beside the headline in a default run, each with its own roofline: the
+# decode half of the metric, the other prefill configurations and MLA.
+DEFAULT_EXTRA = ["paged_decode", "paged_decode_fp8", "window_sink", "window_sink_fp8",
+                 "mla_dense", "mla_sparse"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -227,7 +231,8 @@ def prefill_workload(name: str, seed: int, device):
            "visible_pairs_per_head": pairs, "additive_mask": inp.mask is not None}
     return dict(step=step, e2e_step=e2e_step, work=flops / 1e12, unit="TFLOP/s", bound=bound,
                 kernel=f"prefill_kernel<{D},{ {'bf16': 0, 'fp16': 1, 'e4m3': 2, 'e5m2': 3}[inp.dtype] }>", launches_per_step=1, h2d=h2d, d2h=d2h, cfg=cfg,
-                dtype=inp.dtype, inp=inp, per_unit=f"2*(D_qk+D_v)*H_q FLOP per visible pair, "
+                dtype=inp.dtype, inp=inp, outputs=(out, lse),
+                per_unit=f"2*(D_qk+D_v)*H_q FLOP per visible pair, "
                 f"{pairs} visible pairs per head")
 
 
@@ -287,7 +292,7 @@ def paged_workload(name: str, seed: int, device):
                 kernel="decode_kernel<128,%d>" % (2 if fp8 else 0), launches_per_step=3,
                 h2d=sum(t.numel() * t.element_size() for t in host_small),
                 d2h=sum(t.numel() * t.element_size() for t in host_out), cfg=cfg,
-                dtype=inp.dtype, inp=inp, keep=(meta, ws, out, lse),
+                dtype=inp.dtype, inp=inp, keep=(meta, ws, out, lse), outputs=(out, lse),
                 per_unit=f"(D_k + D_v) * {es} B per cached token per KV head + Q/O/LSE/table; "
                 f"{nbytes} B per step")
 
@@ -348,7 +353,7 @@ def mla_workload(name: str, seed: int, device):
                 kernel=f"mla_kernel<{int(sparse)}>", launches_per_step=3,
                 h2d=sum(t.numel() * t.element_size() for t in host_small),
                 d2h=sum(t.numel() * t.element_size() for t in host_out), cfg=cfg, dtype="bf16",
-                inp=inp, keep=(meta, ws, out, lse), gbytes=nbytes / 1e9,
+                inp=inp, keep=(meta, ws, out, lse), outputs=(out, lse), gbytes=nbytes / 1e9,
                 per_unit=f"2*(576+512)*H_q FLOP per visible (token, key) pair; "
                 f"{pairs_tok} pairs, {nbytes} bytes per step")
 
@@ -417,7 +422,12 @@ def cpu_baseline(name: str, seed: int, budget_s: float = 15.0):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
         cores = 1
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+    try:
+        host_cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        host_cores = os.cpu_count()
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores,
+            "host_cores": host_cores, "host_cpu_count": os.cpu_count(), "kind": "oracle",
             "sample": f"{n} of {len(heads)} (sequence, head) pairs, all query rows, "
                       f"{dt:.1f} s fp64 numpy"}
 
@@ -472,7 +482,12 @@ def run_ours(args, rank, world, device):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
     peaks, peak_kind = load_peaks()
     traffic = load_traffic()
-    names = (args.only or list(WORKLOADS)) if args.all else [args.workload]
+    if args.all:
+        names = list(args.only or WORKLOADS)
+    elif args.headline_only or args.workload != HEADLINE:
+        names = [args.workload]
+    else:
+        names = [args.workload] + DEFAULT_EXTRA
     if args.workload not in names:
         names.insert(0, args.workload)
     results = {}
@@ -541,6 +556,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
     ap.add_argument("--only", nargs="*", default=None, help="with --all: a subset of workloads")
     ap.add_argument("--all", action="store_true", help="also run every other workload")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time the headline workload alone (no decode / MLA / FP8 rows)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clock-window", type=float, default=0.5,
