@@ -186,6 +186,28 @@ DEVI void row_key_range(const PrefillParams& p, int i, int len_q, int len_k, int
   if (p.window_right >= 0) hi = min(hi, i + delta + p.window_right);
 }
 
+// bf16 inputs: a query tile with a row that sees fewer than kShortRow keys
+// runs P V twice, on P rounded to bf16 and on the rounding remainder (also
+// bf16), so P carries about 16 significant bits. With few keys the bf16
+// rounding of P does not average out: for two keys it moves O by up to
+// 2^-9 * |v_1 - v_0| / 4, which, on top of the final rounding of O to bf16,
+// can exceed 1e-2. Rows with many keys need no remainder.
+constexpr int kShortRow = 128;
+
+// Whether Q tile w of unit u holds a row with fewer than kShortRow visible
+// keys. The count of a row is concave in the row index (the upper bound is a
+// minimum of increasing lines, the lower bound a maximum of them), so its
+// minimum over the tile is at the tile's first or last row.
+DEVI bool prefill_short_tile(const PrefillParams& p, const PrefillUnit& u, int w) {
+  const int i0 = u.m * kPrefillUnit + w * kPrefillBM;
+  if (i0 >= u.len_q) return false;
+  const int i1 = min(i0 + kPrefillBM, u.len_q) - 1;
+  int lo0, hi0, lo1, hi1;
+  row_key_range(p, i0, u.len_q, u.len_k, lo0, hi0);
+  row_key_range(p, i1, u.len_q, u.len_k, lo1, hi1);
+  return min(hi0 - lo0, hi1 - lo1) + 1 < kShortRow;
+}
+
 // ---------------------------------------------------------------------------
 // Producer warp (one thread)
 // ---------------------------------------------------------------------------
@@ -278,9 +300,10 @@ DEVI void prefill_issue_pv(uint32_t d_tmem, uint32_t a_tmem, uint64_t dv, uint32
 }
 
 // O_w += P_w V for the key tile with global index g: the head of P as soon as
-// the softmax has released it, then the tail.
+// the softmax has released it, then the tail; with `split`, then the rounding
+// remainder of P (TMEM columns 64 .. 127 of the tile's S buffer).
 DEVI bool prefill_pv(PrefillBarriers* bars, int w, int g, uint32_t t_o, uint32_t t_p, uint64_t dv,
-                     uint32_t idesc, bool first) {
+                     uint32_t idesc, bool first, bool split) {
   volatile int* abort = &bars->abort;
   constexpr int kHead = kSplitKeys / 16;
   if constexpr (kHead > 0) {
@@ -291,10 +314,16 @@ DEVI bool prefill_pv(PrefillBarriers* bars, int w, int g, uint32_t t_o, uint32_t
   if (!warp_wait(&bars->p_full[w], g & 1, abort, 11)) return false;
   tc_fence_after();
   prefill_issue_pv<kHead, kPrefillBN / 16>(t_o, t_p, dv, idesc, first);
+  if (split) {
+    // a rolled loop: the MMA warp runs on few registers
+#pragma unroll 1
+    for (int kk = 0; kk < kPrefillBN / 16; ++kk)
+      mma_f16_ts_w(t_o, t_p + kPrefillBN / 2 + kk * 8, dv + kk * (16 * 128 >> 4), idesc, 1u);
+  }
   return true;
 }
 
-template <int D, int kType>
+template <int D, int kType, bool kMask>
 DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* bars,
                       uint32_t tmem) {
   using C = PrefillCfg<D, kType>;
@@ -328,6 +357,8 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
     if (n <= 0) continue;
     if (!warp_wait(&bars->q_full, nq & 1, abort, 10)) goto drain;
     ++nq;
+    const bool split0 = kType == 0 && !kMask && prefill_short_tile(p, u, 0);
+    const bool split1 = kType == 0 && !kMask && prefill_short_tile(p, u, 1);
     // Order per key tile j: PV0_{j-1}, S0_j, PV1_{j-1}, S1_j. S_w needs the
     // S_w/P_w buffer that PV_w_{j-1} reads; the tensor pipe runs in order.
     for (int j = 0; j <= n; ++j) {
@@ -342,7 +373,7 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
         if (j == 1 && units > 0 && !warp_wait(&bars->o_empty[0], (units - 1) & 1, abort, 13))
           goto drain;
         if (!prefill_pv(bars, 0, g - 1, tO0, tS0, dv_base + sp * (kPVBytes >> 4), idesc_pv,
-                        j == 1))
+                        j == 1, split0))
           goto drain;
         if (j == n) tc_commit_w(&bars->o_full[0]);
       } else {
@@ -356,7 +387,7 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
         if (j == 1 && units > 0 && !warp_wait(&bars->o_empty[1], (units - 1) & 1, abort, 13))
           goto drain;
         if (!prefill_pv(bars, 1, g - 1, tO1, tS1, dv_base + sp * (kPVBytes >> 4), idesc_pv,
-                        j == 1))
+                        j == 1, split1))
           goto drain;
         if (j == n) tc_commit_w(&bars->o_full[1]);
         tc_commit_w(&pv_empty[sp]);
@@ -455,9 +486,14 @@ struct PrefillRow {
 // P = 2^(s * scale * log2e - m) rounded to the MMA's input type (to nearest
 // even), written over S 32 keys (16 packed words) at a time, the head
 // released first; the row sums (kRnd: also the sum of the rounded P).
+// split (bf16, kRnd instance): the rounding remainder P - bf16(P), itself
+// rounded to bf16, goes to TMEM columns 64 .. 127 of the buffer; O is then
+// normalised by the fp32 sum, which the two parts together match to about
+// 2^-16.
 template <int kType, bool kRnd>
 DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float sl2,
-                           const uint32_t* s, PrefillRow& row) {
+                           uint32_t* s, PrefillRow& row, bool split) {
+  constexpr bool kSplit = kRnd && kType == 0;  // the remainder pass may run
   constexpr bool kFp16 = kType != 0;  // P in fp16 (fp16 and FP8 inputs)
   const float m_use = (row.m_run == -INFINITY) ? 0.f : row.m_run;
   const uint64_t negm = f2pack(-m_use, -m_use);
@@ -489,8 +525,23 @@ DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float 
       acc_e[c & 3] = add2(acc_e[c & 3], f2pack(p0, p1));
       pk[c] = pack2<kFp16>(p0, p1);
       if constexpr (kRnd) acc_packed<kFp16>(acc_r[c & 1], acc_r[2 + (c & 1)], pk[c]);
+      if constexpr (kSplit) {  // keep P itself: S of this element is no longer needed
+        s[e] = __float_as_uint(p0);
+        s[e + 1] = __float_as_uint(p1);
+      }
     }
     tmem_store<16>(s_tmem + ch * 16, pk);
+    if (kSplit && split) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int e = ch * 32 + 2 * c;
+        // the bf16 halves of pk[c] widened exactly; P minus them is exact
+        const float r0 = __uint_as_float(s[e]) - __uint_as_float(pk[c] << 16);
+        const float r1 = __uint_as_float(s[e + 1]) - __uint_as_float(pk[c] & 0xffff0000u);
+        pk[c] = pack_bf16x2(r0, r1);
+      }
+      tmem_store<16>(s_tmem + kPrefillBN / 2 + ch * 16, pk);
+    }
     if (ch == kSplitKeys / 32 - 1) {
       // The head of P: the P V MMA starts on it.
       tmem_store_wait();
@@ -503,7 +554,8 @@ DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float 
     float e0, e1;
     f2unpack(e, e0, e1);
     row.l_run += e0 + e1;
-    row.l_rnd += kRnd ? (acc_r[0] + acc_r[1]) + (acc_r[2] + acc_r[3]) : e0 + e1;
+    row.l_rnd += (kRnd && !(kSplit && split)) ? (acc_r[0] + acc_r[1]) + (acc_r[2] + acc_r[3])
+                                              : e0 + e1;
   }
   tmem_store_wait();
   tc_fence_before();
@@ -516,7 +568,7 @@ DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float 
 template <int D, int kType, bool kMask>
 DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t o_tmem, int w,
                                int j, int g, int k0, float sl2, PrefillRow& row,
-                               const float* mrow, int len_k) {
+                               const float* mrow, int len_k, bool split) {
   volatile int* abort = &bars->abort;
   if (!warp_wait(&bars->s_full[w], g & 1, abort, 20 + w)) return false;
   tc_fence_after();
@@ -606,10 +658,10 @@ DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t 
   // difference matters only for rows with few visible keys, whose keys all
   // lie in first or partially masked tiles; other tiles add their fp32 sum to
   // both (their rounding errors average out over the row's many keys).
-  if (j == 0 || kMask || __any_sync(0xffffffffu, partial))
-    prefill_exp_tile<kType, true>(bars, s_tmem, w, sl2, s, row);
+  if (j == 0 || kMask || split || __any_sync(0xffffffffu, partial))
+    prefill_exp_tile<kType, true>(bars, s_tmem, w, sl2, s, row, split);
   else
-    prefill_exp_tile<kType, false>(bars, s_tmem, w, sl2, s, row);
+    prefill_exp_tile<kType, false>(bars, s_tmem, w, sl2, s, row, false);
   return true;
 }
 
@@ -659,10 +711,11 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
     row.seen = false;
     const float* mrow =
         (kMask && valid) ? p.mask + u.b * p.m_sb + u.h * p.m_sh + (int64_t)i * p.m_ss : nullptr;
+    const bool split = kType == 0 && !kMask && prefill_short_tile(p, u, w);
     for (int j = 0; j < n; ++j, ++sj)
       if (!prefill_softmax_tile<D, kType, kMask>(bars, s_tmem, o_tmem, w, j, sj,
                                                  (u.kt0 + j) * kPrefillBN, sl2, row, mrow,
-                                                 u.len_k))
+                                                 u.len_k, split))
         return;
     // Epilogue: wait for the last P V, read O, release O, normalise, store.
     if (!warp_wait(&bars->o_full[w], units & 1, abort, 22 + w)) return;
@@ -759,7 +812,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (warp == 8) {
       if (elect_lane0()) prefill_producer<D, kType>(p, &map_q, &map_k, &map_v, smem, bars);
     } else if (warp == 9) {
-      prefill_mma<D, kType>(p, smem, bars, tmem);  // whole warp, one lane issues
+      prefill_mma<D, kType, kMask>(p, smem, bars, tmem);  // whole warp, one lane issues
     } else if constexpr (C::kFp8) {
       prefill_convert<D, kType>(p, smem, bars);
     }

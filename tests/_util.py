@@ -21,14 +21,34 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return oracle.decode(bits, fmt)
 
 
-def assert_close_out(got, want, atol, what="out"):
+def round_bf16(x):
+    """float64 values rounded to the nearest bf16 value (8 significant bits),
+    ties to even; the normal range only (|x| >= 2^-126), which is all the
+    outputs compared here need."""
+    m, e = np.frexp(np.asarray(x, np.float64))   # x = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0), e - 8)   # np.rint rounds half to even
+
+
+def assert_close_out(got, want, atol, what="out", rounded=True):
+    """Every element within atol of the fp64 oracle, or (rounded) equal to the
+    oracle's value correctly rounded to bf16. The output is bf16 by definition
+    (MATE "Attention", FMHA dtype notes), and its own rounding moves an element
+    by up to half a bf16 unit: 2^-7 = 0.0078 for |O| in [2, 4), 0.0156 in
+    [4, 8). Where that alone reaches the tolerance, the correctly rounded
+    value is the best any kernel can return, and it is accepted."""
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
     assert got.shape == want.shape, (got.shape, want.shape)
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     err = np.abs(got - want)
-    i = np.unravel_index(np.argmax(err), err.shape)
-    assert err.max() <= atol, f"{what}: max abs err {err.max():.3e} at {i} (got {got[i]}, want {want[i]})"
+    bad = err > atol
+    if rounded:
+        bad &= got != round_bf16(want)
+    if bad.any():
+        e = np.where(bad, err, 0.0)
+        i = np.unravel_index(np.argmax(e), e.shape)
+        raise AssertionError(f"{what}: max abs err {err[i]:.3e} at {i} (got {got[i]}, "
+                             f"want {want[i]}), {int(bad.sum())} elements beyond {atol}")
     return float(err.max())
 
 
