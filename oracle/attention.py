@@ -400,18 +400,23 @@ def combine(out_partial: np.ndarray, lse_partial: np.ndarray, sink=None):
 # ---------------------------------------------------------------------------
 
 def mla_paged(q, kv_cache, block_table, cache_seqlens, head_dim_v, scale, causal=False,
-              rows=None):
+              rows=None, q_descale=None, k_descale=None, v_descale=None):
     """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, H_kv, 576). K is
     the whole row, V its first head_dim_v entries. With H_kv > 1 (MATE
     "Attention", MLA example: a cache of 2 KV heads) query head h reads KV
-    head floor(h / (H_q / H_kv)), as in GQA."""
+    head floor(h / (H_q / H_kv)), as in GQA.
+    FP8 (MATE "Attention", FMHA FP8 paragraph, applied to the MLA cache): q,
+    K and V of sequence b and KV head g are multiplied by q_descale[b, g],
+    k_descale[b, g] and v_descale[b, g] (all three given or none); K and V are
+    the same cached row, each with its own descale."""
     kv = np.asarray(kv_cache, np.float64)
     return attention_paged(q, kv, kv[..., :head_dim_v], block_table, cache_seqlens, scale,
-                           causal, (-1, -1), None, rows)
+                           causal, (-1, -1), None, rows, q_descale, k_descale, v_descale)
 
 
 def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, scale,
-               rows=None, block_size=1, causal=False):
+               rows=None, block_size=1, causal=False, q_descale=None, k_descale=None,
+               v_descale=None):
     """q (B, s_q, H_q, 576); kv_cache (num_blocks, page_size, H_kv, 576);
     indices (B, s_q, H_kv, topk) logical positions. Query token (b, i) of
     head h attends, in KV head g = floor(h / (H_q / H_kv)), to the positions
@@ -423,6 +428,7 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
     counts blocks); negative indices are skipped.
     causal (sparse_mode=3, "rightDownCausal"): a listed position p is also
     required to satisfy p <= i + L_b - s_q (bottom-right alignment).
+    q_descale, k_descale, v_descale (B, H_kv): FP8 descales as in mla_paged.
     Returns out (B, s_q, H_q, D_v) and lse (B, H_q, s_q)."""
     q = np.asarray(q, np.float64)
     kv = np.asarray(kv_cache, np.float64)
@@ -453,16 +459,20 @@ def mla_sparse(q, kv_cache, block_table, cache_seqlens, indices, head_dim_v, sca
                 if causal:
                     idx = idx[idx <= i + L - Sq]
                 rows_kv = kv[np.asarray(block_table[b], np.int64)[idx // page], idx % page, g, :]
+                qs, ks, vs = q[b, i, hs, :], rows_kv, rows_kv[:, :head_dim_v]
+                if q_descale is not None:
+                    dq, dk, dv = (float(d[b][g]) for d in (q_descale, k_descale, v_descale))
+                    qs, ks, vs = qs * dq, ks * dk, vs * dv
                 vis = np.ones((len(hs), idx.size), dtype=bool)
-                o, l = attention_rows(q[b, i, hs, :], rows_kv, rows_kv[:, :head_dim_v], scale,
-                                      vis)
+                o, l = attention_rows(qs, ks, vs, scale, vis)
                 out[b, i, hs, :] = o
                 lse[b, hs, i] = l
     return out, lse
 
 
 def mla_sparse_tnd(q, kv_cache, block_table, cache_seqlens, cu_seqlens_q, indices, head_dim_v,
-                   scale, block_size=1, causal=False):
+                   scale, block_size=1, causal=False, q_descale=None, k_descale=None,
+                   v_descale=None):
     """The sparse MLA attention with packed (TND) queries (MindSpore
     "sparse_flash_attention", layout_query="TND" with a paged cache): q
     (T, H_q, 576) holds the query tokens of the B sequences back to back,
@@ -470,7 +480,8 @@ def mla_sparse_tnd(q, kv_cache, block_table, cache_seqlens, cu_seqlens_q, indice
     prefix-sum form of actual_seq_lengths_query); indices (T, H_kv, topk).
     Each sequence is the BSND problem of its own tokens (token i of sequence
     b is its i-th query row; causal aligns its last token with the cache's
-    last key). Returns out (T, H_q, D_v) and lse (H_q, T)."""
+    last key). q/k/v_descale (B, H_kv): FP8 descales of each sequence, as in
+    mla_paged. Returns out (T, H_q, D_v) and lse (H_q, T)."""
     q = np.asarray(q, np.float64)
     T, Hq, _ = q.shape
     out = np.zeros((T, Hq, head_dim_v), np.float64)
@@ -480,9 +491,14 @@ def mla_sparse_tnd(q, kv_cache, block_table, cache_seqlens, cu_seqlens_q, indice
         t0, t1 = cu[b], cu[b + 1]
         if t1 <= t0:
             continue
+        desc = {}
+        if q_descale is not None:
+            desc = dict(q_descale=np.asarray(q_descale)[b:b + 1],
+                        k_descale=np.asarray(k_descale)[b:b + 1],
+                        v_descale=np.asarray(v_descale)[b:b + 1])
         o, l = mla_sparse(q[None, t0:t1], kv_cache, np.asarray(block_table)[b:b + 1],
                           [int(cache_seqlens[b])], np.asarray(indices)[None, t0:t1],
-                          head_dim_v, scale, block_size=block_size, causal=causal)
+                          head_dim_v, scale, block_size=block_size, causal=causal, **desc)
         out[t0:t1] = o[0]
         lse[:, t0:t1] = l[0]
     return out, lse

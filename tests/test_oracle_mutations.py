@@ -38,6 +38,10 @@ MUTATIONS = [
      "idx[:, None] + np.arange(block_size)"),
     ("sparse causal not bottom-right", "idx = idx[idx <= i + L - Sq]", "idx = idx[idx <= i]"),
     ("additive mask dropped", "s = s + np.asarray(bias, dtype=np.float64)", "s = s"),
+    ("MLA K and V descales swapped", "None, rows, q_descale, k_descale, v_descale)",
+     "None, rows, q_descale, v_descale, k_descale)"),
+    ("sparse MLA V scaled by the K descale", "qs, ks, vs = qs * dq, ks * dk, vs * dv",
+     "qs, ks, vs = qs * dq, ks * dk, vs * dk"),
 ]
 
 

@@ -397,6 +397,52 @@ def test_mla_dense_equals_sdpa_with_latent_values():
             np.testing.assert_allclose(out[b, i], ref, rtol=1e-12)
 
 
+def _e4m3_values(shape):
+    """Random e4m3 codes (NaN codes excluded) decoded to float64."""
+    codes = RNG.integers(0, 256, size=shape).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38
+    return oracle.decode(codes, "e4m3")
+
+
+def test_mla_fp8_descales_match_sdpa_on_scaled_rows():
+    # K = row * k_descale and V = row[:Dv] * v_descale of the same cached row:
+    # a transposed descale (K's on V) or a dropped one fails here.
+    lens, page, Hq, Hkv, D, Dv = [7, 12], 4, 4, 2, 10, 6
+    _, _, bt = _paged_case(lens, page, Hkv, D, "permuted")
+    ck = _e4m3_values((int(bt.max()) + 1, page, Hkv, D))
+    q = _e4m3_values((2, 2, Hq, D))
+    qd, kd, vd = (RNG.uniform(0.5, 2, size=(2, Hkv)) for _ in range(3))
+    out, lse = oracle.mla_paged(q, ck, bt, lens, Dv, 0.3, q_descale=qd, k_descale=kd,
+                                v_descale=vd)
+    for b, L in enumerate(lens):
+        rows = oracle.gather_pages(ck, bt[b], L)
+        for h in range(Hq):
+            g = h // (Hq // Hkv)
+            kk, vv = rows[:, g, :] * kd[b, g], rows[:, g, :Dv] * vd[b, g]
+            qq = q[b, :, h, :] * qd[b, g]
+            ref = _sdpa(qq[None], kk[None], vv[None], 0.3)[0]
+            np.testing.assert_allclose(out[b, :, h], ref, rtol=1e-12, atol=1e-14)
+            s = 0.3 * qq @ kk.T
+            np.testing.assert_allclose(lse[b, h], torch.logsumexp(torch.as_tensor(s), -1).numpy(),
+                                       rtol=1e-12)
+
+
+def test_mla_sparse_fp8_descales_match_sdpa_on_gathered_rows():
+    lens, page, Hq, D, Dv = [20], 4, 2, 8, 5
+    pages = -(-20 // page)
+    ck = _e4m3_values((pages, page, 1, D))
+    bt = RNG.permutation(pages)[None]
+    q = _e4m3_values((1, 1, Hq, D))
+    sel = np.array([1, 4, 5, 11, 17, 19])
+    qd, kd, vd = (RNG.uniform(0.5, 2, size=(1, 1)) for _ in range(3))
+    out, _ = oracle.mla_sparse(q, ck, bt, lens, sel.reshape(1, 1, 1, -1), Dv, 0.5,
+                               q_descale=qd, k_descale=kd, v_descale=vd)
+    rows = oracle.gather_pages(ck, bt[0], 20)[sel, 0, :]
+    ref = _sdpa(q[0, 0][:, None, :] * qd[0, 0], np.repeat(rows[None] * kd[0, 0], Hq, 0),
+                np.repeat(rows[None, :, :Dv] * vd[0, 0], Hq, 0), 0.5)[:, 0, :]
+    np.testing.assert_allclose(out[0, 0], ref, rtol=1e-12)
+
+
 def test_mla_sparse_all_positions_equals_dense_and_skips_invalid():
     lens, page, Hq, D, Dv, topk = [7, 12], 4, 3, 10, 6, 16
     ck, _, bt = _paged_case(lens, page, 1, D, "permuted")
