@@ -99,7 +99,8 @@ class MlaArgs(ctypes.Structure):
                 ("scale", c_f32), ("causal", c_i32), ("meta", c_vp), ("meta_bytes", c_sz),
                 ("num_ctas", c_i32), ("workspace", c_vp), ("workspace_bytes", c_sz),
                 ("sparse_block_size", c_i32), ("kv_stride_h", c_i64), ("idx_stride_h", c_i64),
-                ("cu_seqlens_q", c_vp)]
+                ("cu_seqlens_q", c_vp), ("dtype", c_i32), ("q_descale", c_vp),
+                ("k_descale", c_vp), ("v_descale", c_vp)]
 
 
 ARG_STRUCTS = {0: VarlenArgs, 1: SchedArgs, 2: PagedArgs, 3: CombineArgs, 4: MlaArgs}
@@ -414,14 +415,17 @@ def combine(out_partial, lse_partial, *, num_splits_per_seq=None, sink=None, out
 
 def mla_args(q, kv_cache, block_table, cache_seqlens, *, head_dim_v=512, scale=None,
              causal=False, indices=None, meta=None, num_ctas=0, workspace=None, out=None,
-             lse=None, sparse_block_size=0, cu_seqlens_q=None):
+             lse=None, sparse_block_size=0, cu_seqlens_q=None, q_descale=None, k_descale=None,
+             v_descale=None):
     """BSND: q (B, s_q, H_q, 576), indices (B, s_q, H_kv, topk); out
     (B, s_q, H_q, 512), lse (B, H_q, s_q). Packed (TND, sparse only, with
     cu_seqlens_q int32 (B+1)): q (T, H_q, 576), indices (T, H_kv, topk); out
-    (T, H_q, 512), lse (H_q, T)."""
+    (T, H_q, 512), lse (H_q, T). q and kv_cache are both bf16 or both
+    float8_e4m3fn; e4m3 takes fp32 (B, H_kv) descales (all three or none)."""
     _rows(q=q, kv_cache=kv_cache, out=out, block_table=block_table, indices=indices)
     _same_dtype(q, kv_cache=kv_cache)
-    _dense(cache_seqlens=cache_seqlens, lse=lse, cu_seqlens_q=cu_seqlens_q)
+    _dense(cache_seqlens=cache_seqlens, lse=lse, cu_seqlens_q=cu_seqlens_q,
+           q_descale=q_descale, k_descale=k_descale, v_descale=v_descale)
     _int32(block_table=block_table, cache_seqlens=cache_seqlens, indices=indices,
            cu_seqlens_q=cu_seqlens_q)
     tnd = cu_seqlens_q is not None
@@ -456,7 +460,8 @@ def mla_args(q, kv_cache, block_table, cache_seqlens, *, head_dim_v=512, scale=N
         kv_cache.shape[0], block_table.shape[1], topk, block_table.stride(0), *qs,
         kv_cache.stride(0), kv_cache.stride(1), *os_, ist[0], ist[1], float(scale),
         int(bool(causal)), _ptr(meta), 0 if meta is None else meta.numel() * 4, int(num_ctas),
-        None, 0, int(sparse_block_size), kv_cache.stride(2), ist[2], _ptr(cu_seqlens_q))
+        None, 0, int(sparse_block_size), kv_cache.stride(2), ist[2], _ptr(cu_seqlens_q),
+        _TORCH_DTYPE.get(q.dtype, -1), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale))
     if meta is not None:
         nbytes = int(lib().mla_workspace_size(ctypes.byref(a)))
         if workspace is None:

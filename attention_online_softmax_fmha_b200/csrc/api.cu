@@ -251,19 +251,24 @@ attn_status_t check_mla(const mla_args* a, bool sparse) {
   if (a->block_table_stride < a->max_pages_per_seq) return ATTN_ERR_INVALID_ARG;
   if (!(a->scale > 0.f) || !std::isfinite(a->scale)) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(a->q) || !aligned16(a->kv_cache) || !aligned16(a->out)) return ATTN_ERR_INVALID_ARG;
+  if (a->dtype != ATTN_DTYPE_BF16 && a->dtype != ATTN_DTYPE_E4M3) return ATTN_ERR_UNSUPPORTED;
+  const bool fp8 = a->dtype == ATTN_DTYPE_E4M3;
+  const int ne = (a->q_descale != nullptr) + (a->k_descale != nullptr) + (a->v_descale != nullptr);
+  if (ne != 0 && (ne != 3 || !fp8)) return ATTN_ERR_INVALID_ARG;
+  const int es = fp8 ? 1 : 2;  // bytes per q / cache element
   // packed (TND) queries: sparse only; there is no query batch axis
   const bool tnd = a->cu_seqlens_q != nullptr;
   if (tnd && !sparse) return ATTN_ERR_UNSUPPORTED;
-  if ((!tnd && (!stride_ok(a->q_stride_b, 2) || !stride_ok(a->o_stride_b, 2))) ||
-      !stride_ok(a->q_stride_s, 2) || !stride_ok(a->q_stride_h, 2) ||
-      !stride_ok(a->kv_stride_blk, 2) || !stride_ok(a->kv_stride_tok, 2) ||
+  if ((!tnd && (!stride_ok(a->q_stride_b, es) || !stride_ok(a->o_stride_b, 2))) ||
+      !stride_ok(a->q_stride_s, es) || !stride_ok(a->q_stride_h, es) ||
+      !stride_ok(a->kv_stride_blk, es) || !stride_ok(a->kv_stride_tok, es) ||
       !stride_ok(a->o_stride_s, 2) || !stride_ok(a->o_stride_h, 2))
     return ATTN_ERR_INVALID_ARG;
   if (sparse && ((!tnd && a->idx_stride_b <= 0) || a->idx_stride_s <= 0))
     return ATTN_ERR_INVALID_ARG;
   if (a->num_heads_q % a->num_heads_kv) return ATTN_ERR_INVALID_ARG;
   if (a->num_heads_kv > 1 &&
-      (!stride_ok(a->kv_stride_h, 2) || (sparse && a->idx_stride_h <= 0)))
+      (!stride_ok(a->kv_stride_h, es) || (sparse && a->idx_stride_h <= 0)))
     return ATTN_ERR_INVALID_ARG;
   if (a->head_dim_qk != kMlaDqk || a->head_dim_v != kMlaDv) return ATTN_ERR_UNSUPPORTED;
   if (!mla_heads_ok(a->num_heads_q / a->num_heads_kv)) return ATTN_ERR_UNSUPPORTED;
@@ -280,8 +285,14 @@ size_t mla_ws_bytes(const DecodeShape& ds) {
          256;
 }
 
-template <bool kSparse>
+template <bool kSparse, bool kFp8>
 attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t stream) {
+  using C = MlaCfg<kFp8>;
+  // a TMA box column is 128 bytes: 64 bf16 or 128 e4m3 values
+  const CUtensorMapDataType dt =
+      kFp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int es = kFp8 ? 1 : 2;
+  const uint32_t box_c = kFp8 ? 128 : 64;
   // Q boxes: the query heads of one KV head (128 at most) x the tile's tokens
   const int box_h = ds.group >= kMlaRows ? kMlaRows : ds.group;
   const int box_t = ds.group >= kMlaRows ? 1 : ds.tokens_per_tile;
@@ -294,10 +305,10 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   const uint64_t kv_sh = a.num_heads_kv > 1 ? (uint64_t)a.kv_stride_h
                                              : a.kv_stride_blk * (uint64_t)a.num_blocks;
   CUtensorMap mq, mkv;
-  if (!encode_4d(&mq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk, a.num_heads_q,
-                 a.seqlen_q, batch_q, a.q_stride_h, a.q_stride_s, q_sb, 64, box_h, box_t, 1) ||
-      !encode_4d(&mkv, a.kv_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kMlaDqk, a.page_size,
-                 a.num_blocks, a.num_heads_kv, a.kv_stride_tok, a.kv_stride_blk, kv_sh, 64,
+  if (!encode_4d(&mq, a.q, dt, es, kMlaDqk, a.num_heads_q, a.seqlen_q, batch_q, a.q_stride_h,
+                 a.q_stride_s, q_sb, box_c, box_h, box_t, 1) ||
+      !encode_4d(&mkv, a.kv_cache, dt, es, kMlaDqk, a.page_size, a.num_blocks, a.num_heads_kv,
+                 a.kv_stride_tok, a.kv_stride_blk, kv_sh, box_c,
                  a.page_size >= kMlaBN ? kMlaBN : a.page_size, 1, 1))
     return ATTN_ERR_INVALID_ARG;
   MlaParams p;
@@ -309,7 +320,10 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   p.cache_seqlens = a.cache_seqlens;
   p.indices = a.indices;
   p.meta = a.meta;
-  p.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv_cache);
+  p.kv = a.kv_cache;
+  p.q_descale = a.q_descale;
+  p.k_descale = a.k_descale;
+  p.v_descale = a.v_descale;
   p.bt_stride = a.block_table_stride;
   p.q_sb = tnd ? 0 : a.q_stride_b;
   p.q_ss = a.q_stride_s;
@@ -348,15 +362,15 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
     p.ws_o = reinterpret_cast<float*>(a.workspace);
     p.ws_lse = p.ws_o + slots * 2 * kMlaRows * kMlaDvHalf;
   }
-  auto kernel = mla_kernel<kSparse>;
+  auto kernel = mla_kernel<kSparse, kFp8>;
   static std::atomic<uint64_t> configured{0};
   const attn_status_t cst = configure_per_device(configured, [&] {
-    return launch_status(set_smem(kernel, kMlaSmemBytes));
+    return launch_status(set_smem(kernel, C::kSmemBytes));
   });
   if (cst != ATTN_OK) return cst;
   // Clusters of two CTAs (the kernel's __cluster_dims__): one per segment, or
   // one per metadata slot.
-  kernel<<<2 * (a.meta ? ds.G : ds.S), 192, kMlaSmemBytes, stream>>>(mq, mkv, p);
+  kernel<<<2 * (a.meta ? ds.G : ds.S), C::kThreads, C::kSmemBytes, stream>>>(mq, mkv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (a.meta) {
     const int64_t warps = (int64_t)ds.S * 2 * kMlaRows;
@@ -383,7 +397,9 @@ attn_status_t mla_entry(const mla_args* a, void* stream, bool sparse) {
     if (!aligned16(a->workspace)) return ATTN_ERR_INVALID_ARG;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return sparse ? run_mla<true>(*a, ds, s) : run_mla<false>(*a, ds, s);
+  if (a->dtype == ATTN_DTYPE_E4M3)
+    return sparse ? run_mla<true, true>(*a, ds, s) : run_mla<false, true>(*a, ds, s);
+  return sparse ? run_mla<true, false>(*a, ds, s) : run_mla<false, false>(*a, ds, s);
 }
 
 }  // namespace

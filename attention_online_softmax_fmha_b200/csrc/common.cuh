@@ -313,6 +313,18 @@ DEVI float sum2(uint32_t packed) {
   return __uint_as_float(packed << 16) + __uint_as_float(packed & 0xffff0000u);
 }
 
+// Two FP8 values (low byte first) to two fp16 values, exactly (every e4m3
+// and every e5m2 value is an fp16 value). kType: 2 = e4m3, 3 = e5m2.
+template <int kType>
+DEVI uint32_t fp8x2_to_f16x2(unsigned short v) {
+  uint32_t h;
+  if constexpr (kType == 3)
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(v));
+  else
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
+  return h;
+}
+
 DEVI void store_out(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 DEVI void store_out(__half* p, float v) { *p = __float2half_rn(v); }
 

@@ -63,28 +63,63 @@ constexpr int kMlaSBufs = 3;       // S buffers in TMEM
 constexpr int kMlaSAhead = 3;
 static_assert(kMlaSAhead >= 2 && kMlaSAhead <= kMlaSBufs, "S lookahead");
 constexpr int kMlaXsBufs = 2;      // partial-S exchange buffers in shared memory
-constexpr int kMlaMaxChunks = 5;   // 64-column chunks per CTA (rank 0: 5, rank 1: 4)
 constexpr int kGatherLag = 1;      // sparse: tiles of gathers in flight before a stage is signalled
 static_assert(kGatherLag < kMlaStages, "gather lag");
 constexpr int kMlaQChunkBytes = kMlaRows * 128;                // 16 KB
 constexpr int kMlaKVChunkBytes = kMlaBN * 128;                 // 4 KB
-constexpr int kMlaQBytes = kMlaMaxChunks * kMlaQChunkBytes;    // 80 KB
-constexpr int kMlaKVBytes = kMlaMaxChunks * kMlaKVChunkBytes;  // 20 KB
 constexpr int kMlaXsBytes = kMlaRows * kMlaBN * 4;             // one partial S tile, 16 KB
-constexpr int kMlaQOff = 0;
-constexpr int kMlaXsOff = kMlaQOff + kMlaQBytes;               // partial S received here
-constexpr int kMlaXoOff = kMlaXsOff + kMlaXsBufs * kMlaXsBytes;  // and staged here to send
-constexpr int kMlaKVOff = kMlaXoOff + kMlaXsBufs * kMlaXsBytes;
-constexpr int kMlaBarOff = kMlaKVOff + kMlaStages * kMlaKVBytes;
-constexpr int kMlaSmemBytes = kMlaBarOff + 256;
-static_assert(kMlaSmemBytes <= 232448, "shared memory per CTA");
 constexpr uint32_t kMlaTmemCols = 512;
 constexpr uint32_t kMlaTmemS = 0;      // three S buffers of 32 columns
 constexpr uint32_t kMlaTmemO = 256;    // 256 columns of O
 
-// Global 64-column chunk of the 576-wide row held in local chunk c of rank r.
-DEVI int mla_chunk(int rank, int c) { return rank == 0 ? (c < 4 ? c : 8) : 4 + c; }
-DEVI int mla_nchunks(int rank) { return rank == 0 ? 5 : 4; }
+// Shared-memory layout of the bf16 (kFp8 = false) and the e4m3 kernel. A
+// chunk is one 128-byte column of a TMA box: 64 bf16 or 128 e4m3 values.
+// e4m3 rows also need an fp16 copy of the tile's V half for P V (FP8 has no
+// fp16 partner type in one MMA, and P stays fp16), made by two extra warps.
+template <bool kFp8>
+struct MlaCfg {
+  static constexpr int kMaxChunks = kFp8 ? 3 : 5;          // chunks per CTA (rank 0)
+  static constexpr int kQBytes = kMaxChunks * kMlaQChunkBytes;
+  static constexpr int kKVBytes = kMaxChunks * kMlaKVChunkBytes;
+  static constexpr int kQOff = 0;
+  static constexpr int kXsOff = kQOff + kQBytes;                      // partial S received here
+  static constexpr int kXoOff = kXsOff + kMlaXsBufs * kMlaXsBytes;    // and staged here to send
+  static constexpr int kKVOff = kXoOff + kMlaXsBufs * kMlaXsBytes;
+  static constexpr int kVHStages = kFp8 ? 2 : 0;
+  static constexpr int kVHBytes = 4 * kMlaKVChunkBytes;  // fp16 V half: 4 chunks of 64 columns
+  static constexpr int kVHOff = kKVOff + kMlaStages * kKVBytes;
+  static constexpr int kBarOff = kVHOff + kVHStages * kVHBytes;
+  static constexpr int kSmemBytes = kBarOff + 256;
+  static constexpr int kThreads = kFp8 ? 256 : 192;  // + two conversion warps
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
+
+// Columns held by each CTA. bf16: rank 0 the nope columns 0..255 and the rope
+// (chunks 0-3 and 8 of 64 columns), rank 1 the nope columns 256..511. e4m3
+// (128 columns per chunk): rank 0 columns 0..255 and a box at column 448,
+// of which only the second half (the rope, 512..575) is used; rank 1 columns
+// 256..511. Either way a CTA's first 256 columns are its V half.
+template <bool kFp8>
+DEVI int mla_nchunks(int rank) { return kFp8 ? (rank == 0 ? 3 : 2) : (rank == 0 ? 5 : 4); }
+// First element column of local chunk c of rank r.
+template <bool kFp8>
+DEVI int mla_col(int rank, int c) {
+  if constexpr (kFp8) return rank == 0 ? (c < 2 ? 128 * c : 448) : 256 + 128 * c;
+  return 64 * (rank == 0 ? (c < 4 ? c : 8) : 4 + c);
+}
+// 32-byte K steps of this CTA's partial score, and the (chunk, step within
+// the chunk) of step k: e4m3 rank 0 skips the first half of its last box.
+template <bool kFp8>
+DEVI int mla_ksteps(int rank) { return kFp8 ? (rank == 0 ? 10 : 8) : 4 * mla_nchunks<false>(rank); }
+template <bool kFp8>
+DEVI void mla_kstep(int k, int& chunk, int& sub) {
+  chunk = k >> 2;
+  sub = k & 3;
+  if (kFp8 && k >= 8) {
+    chunk = 2;
+    sub = k - 6;
+  }
+}
 
 struct MlaParams {
   const void* q;
@@ -96,7 +131,10 @@ struct MlaParams {
   const int32_t* meta;
   float* ws_o;    // [slot][V half][128][256]
   float* ws_lse;  // [slot][128]
-  const __nv_bfloat16* kv;
+  const void* kv;
+  const float* q_descale;  // FP8: (B, H_kv) each, or nullptr (all 1)
+  const float* k_descale;
+  const float* v_descale;
   int64_t bt_stride;
   int64_t q_sb, q_ss, q_sh;
   int64_t o_sb, o_ss, o_sh;
@@ -122,6 +160,7 @@ struct MlaParams {
 struct MlaBarriers {
   uint64_t q_full, q_empty;
   uint64_t kv_full[kMlaStages], kv_empty[kMlaStages];
+  uint64_t vh_full[2], vh_empty[2];  // FP8: the fp16 copies of V
   uint64_t s_full[kMlaSBufs], p_full[2];
   uint64_t xs_full[kMlaXsBufs];  // the other CTA's partial S tile has landed here
   uint64_t o_full, o_empty;
@@ -222,12 +261,14 @@ DEVI void mla_range(const MlaParams& p, int& ub, int& ue, int& s0, const int32_t
 // ---------------------------------------------------------------------------
 // Producer warp
 // ---------------------------------------------------------------------------
-template <bool kSparse>
+template <bool kSparse, bool kFp8>
 DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensorMap* mkv,
                        uint8_t* smem, MlaBarriers* bars, int rank) {
+  using C = MlaCfg<kFp8>;
+  constexpr int kEsize = kFp8 ? 1 : 2;
   volatile int* abort = &bars->abort;
   const int lane = threadIdx.x & 31;
-  const int nch = mla_nchunks(rank);
+  const int nch = mla_nchunks<kFp8>(rank);
   if (lane == 0) {
     tma_prefetch_desc(mq);
     if (!kSparse) tma_prefetch_desc(mkv);
@@ -275,8 +316,8 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
         const int box_rows = p.group >= kMlaRows ? kMlaRows : p.group * (kSparse ? 1 : p.tokens_per_tile);
         mbar_expect_tx(&bars->q_full, nch * box_rows * 128);
         for (int c = 0; c < nch; ++c)
-          tma_load_4d(smem + kMlaQOff + c * kMlaQChunkBytes, mq, &bars->q_full,
-                      mla_chunk(rank, c) * 64, g.kvg * p.group + g.head0, g.tok0, g.b);
+          tma_load_4d(smem + C::kQOff + c * kMlaQChunkBytes, mq, &bars->q_full,
+                      mla_col<kFp8>(rank, c), g.kvg * p.group + g.head0, g.tok0, g.b);
       }
     }
     if (__shfl_sync(0xffffffffu, q_issued ? 1 : 0, 0)) ++nq;
@@ -284,7 +325,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
     const int32_t* bt = p.block_table + (int64_t)g.bk * p.bt_stride;
     for (int t = a; t < e; ++t, ++it) {
       const int st = it % kMlaStages;
-      uint8_t* dst = smem + kMlaKVOff + st * kMlaKVBytes;
+      uint8_t* dst = smem + C::kKVOff + st * C::kKVBytes;
       bool ok = true;
       if (it >= kMlaStages) {
         const uint32_t parity = ((it / kMlaStages) - 1) & 1;
@@ -318,7 +359,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
           if (lane == 0)
             for (int c = 0; c < nch; ++c)
               tma_load_4d(dst + c * kMlaKVChunkBytes + j * box * 128, mkv, &bars->kv_full[st],
-                          mla_chunk(rank, c) * 64, key0 % P, pg, g.kvg);
+                          mla_col<kFp8>(rank, c), key0 % P, pg, g.kvg);
         }
       } else {
         // lane k gathers key t*32 + k: 8 async copies of 16 bytes per chunk
@@ -332,19 +373,20 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
           pos = mla_sparse_pos(p, g.b, g.kvg, g.tok0, t * kMlaBN + lane);
         }
         const bool valid = pos >= 0 && pos < g.len;
-        const __nv_bfloat16* src = nullptr;
+        const uint8_t* src = nullptr;  // the cached row, in bytes
         if (valid)
-          src = p.kv + g.kvg * p.kv_sh + (int64_t)bt[pos / P] * p.kv_sblk +
-                (int64_t)(pos % P) * p.kv_stok;
+          src = static_cast<const uint8_t*>(p.kv) +
+                (g.kvg * p.kv_sh + (int64_t)bt[pos / P] * p.kv_sblk +
+                 (int64_t)(pos % P) * p.kv_stok) * kEsize;
         const uint32_t dbase = smem_u32(dst) + lane * 128;
         for (int c = 0; c < nch; ++c) {
-          const int gc = mla_chunk(rank, c);
+          const int gcol = mla_col<kFp8>(rank, c) * kEsize;  // byte column of the chunk
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
             const uint32_t d = dbase + c * kMlaKVChunkBytes + ((x ^ (lane & 7)) << 4);
             if (valid) {
               asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d),
-                           "l"(src + gc * 64 + x * 8)
+                           "l"(src + gcol + x * 16)
                            : "memory");
             } else {
               asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(d), "r"(0) : "memory");
@@ -388,35 +430,49 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
 // ---------------------------------------------------------------------------
 // S of the tile with global index g (this CTA's partial scores): waits for
 // its key stage, writes S buffer g % 3; after the segment's last S, releases Q.
+// e4m3: S runs on the FP8 codes (kind::f8f6f4); P V reads the fp16 copy of V,
+// so the stage is released here (with the conversion warps' arrivals).
+template <bool kFp8>
 DEVI bool mla_issue_s(MlaBarriers* bars, int g, uint64_t dq, uint64_t dkv, uint32_t tmem, int nk,
                       bool last) {
-  constexpr uint32_t idesc_s = make_idesc(128, kMlaBN, 1, 0, 0);
+  // kind::f16 format 1 = bf16; kind::f8f6f4 format 0 = e4m3
+  constexpr uint32_t idesc_s = make_idesc(128, kMlaBN, kFp8 ? 0 : 1, 0, 0);
   const int st = g % kMlaStages;
   if (!warp_wait(&bars->kv_full[st], (g / kMlaStages) & 1, &bars->abort, 71)) return false;
   tc_fence_after();
   const uint32_t sbuf = tmem + kMlaTmemS + (g % kMlaSBufs) * kMlaBN;
-  const uint64_t kst = dkv + st * (kMlaKVBytes >> 4);
+  const uint64_t kst = dkv + st * (MlaCfg<kFp8>::kKVBytes >> 4);
 #pragma unroll 4
   for (int k = 0; k < nk; ++k) {
-    const uint32_t qo = (k >> 2) * (kMlaQChunkBytes >> 4) + (k & 3) * 2;
-    const uint32_t ko = (k >> 2) * (kMlaKVChunkBytes >> 4) + (k & 3) * 2;
-    mma_f16_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
+    int ch, sub;
+    mla_kstep<kFp8>(k, ch, sub);
+    const uint32_t qo = ch * (kMlaQChunkBytes >> 4) + sub * 2;
+    const uint32_t ko = ch * (kMlaKVChunkBytes >> 4) + sub * 2;
+    if constexpr (kFp8)
+      mma_f8_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
+    else
+      mma_f16_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
   }
   tc_commit_w(&bars->s_full[g % kMlaSBufs]);
+  if constexpr (kFp8) tc_commit_w(&bars->kv_empty[st]);
   if (last) tc_commit_w(&bars->q_empty);
   return true;
 }
 
-template <bool kSparse>
+template <bool kSparse, bool kFp8>
 DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem, int rank) {
+  using C = MlaCfg<kFp8>;
   volatile int* abort = &bars->abort;
-  const int nk = mla_nchunks(rank) * 4;  // 16-column K steps of the partial score
-  constexpr uint32_t idesc_pv = make_idesc(128, kMlaDvHalf, 1, 0, 1);
-  const uint64_t dq = sdesc_sw128(smem_u32(smem + kMlaQOff), 16, 1024);
-  const uint64_t dkv = sdesc_sw128(smem_u32(smem + kMlaKVOff), 16, 1024);
-  // This CTA's V half: local chunks 0..3 of the key tile, MN-major (leading
-  // byte offset = chunk stride, stride byte offset = 8 keys x 128 bytes).
-  const uint64_t dv = sdesc_sw128(smem_u32(smem + kMlaKVOff), kMlaKVChunkBytes, 1024);
+  const int nk = mla_ksteps<kFp8>(rank);  // 32-byte K steps of the partial score
+  // P V: bf16 P and V, or (e4m3 rows) fp16 P and the fp16 copy of V
+  constexpr uint32_t idesc_pv = make_idesc(128, kMlaDvHalf, kFp8 ? 0 : 1, 0, 1);
+  const uint64_t dq = sdesc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+  const uint64_t dkv = sdesc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
+  // This CTA's V half: local chunks 0..3 of the bf16 key tile (or of the
+  // fp16 copy), MN-major (leading byte offset = chunk stride, stride byte
+  // offset = 8 keys x 128 bytes).
+  const uint64_t dv = sdesc_sw128(smem_u32(smem + (kFp8 ? C::kVHOff : C::kKVOff)),
+                                  kMlaKVChunkBytes, 1024);
   int ub, ue, s;
   const int32_t* prefix;
   mla_range<kSparse>(p, ub, ue, s, prefix);
@@ -448,23 +504,32 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
     // in an earlier P V: the pipe runs in order). The softmax thus finds
     // S_{g+1} ready while it finishes tile g.
     for (int j = 0; j < kMlaSAhead && j < n; ++j)
-      if (!mla_issue_s(bars, it + j, dq, dkv, tmem, nk, j == n - 1)) goto drain;
+      if (!mla_issue_s<kFp8>(bars, it + j, dq, dkv, tmem, nk, j == n - 1)) goto drain;
     for (int j = 0; j < n; ++j) {
       const int gi = it + j, sp = gi % kMlaStages;
       if (!warp_wait(&bars->p_full[gi & 1], (gi >> 1) & 1, abort, 72)) goto drain;
       if (j == 0 && pieces > 0 && !warp_wait(&bars->o_empty, (pieces - 1) & 1, abort, 73))
         goto drain;
+      uint64_t vst;
+      if constexpr (kFp8) {
+        if (!warp_wait(&bars->vh_full[gi & 1], (gi >> 1) & 1, abort, 75)) goto drain;
+        vst = dv + (gi & 1) * (C::kVHBytes >> 4);
+      } else {
+        vst = dv + sp * (C::kKVBytes >> 4);
+      }
       tc_fence_after();
       const uint32_t pbuf = tmem + kMlaTmemS + (gi % kMlaSBufs) * kMlaBN;
-      const uint64_t vst = dv + sp * (kMlaKVBytes >> 4);
 #pragma unroll
       for (int kk = 0; kk < kMlaBN / 16; ++kk)
         mma_f16_ts_w(tmem + kMlaTmemO, pbuf + kk * 8, vst + kk * (16 * 128 >> 4), idesc_pv,
                      (j > 0 || kk > 0) ? 1u : 0u);
-      tc_commit_w(&bars->kv_empty[sp]);
+      if constexpr (kFp8)
+        tc_commit_w(&bars->vh_empty[gi & 1]);
+      else
+        tc_commit_w(&bars->kv_empty[sp]);
       tc_commit_w(&bars->o_full);
       if (j + kMlaSAhead < n &&
-          !mla_issue_s(bars, gi + kMlaSAhead, dq, dkv, tmem, nk, j + kMlaSAhead == n - 1))
+          !mla_issue_s<kFp8>(bars, gi + kMlaSAhead, dq, dkv, tmem, nk, j + kMlaSAhead == n - 1))
         goto drain;
     }
     it += n;
@@ -480,6 +545,77 @@ drain : {
 }
 
 // ---------------------------------------------------------------------------
+// e4m3 rows only: conversion warps (warps 6, 7). Each key tile's V half (the
+// CTA's first two 128-column chunks of e4m3 codes) is rewritten as fp16, which
+// holds every e4m3 value exactly, in the layout the P V MMA reads (four
+// 64-column chunks, 128-byte swizzled); keys past the end of the cache become
+// zeros so that P = 0 never meets a NaN code. The FP8 stage is then released
+// (with the S MMA's commit) and the fp16 copy handed to the MMA warp.
+// ---------------------------------------------------------------------------
+template <bool kSparse>
+DEVI void mla_convert(const MlaParams& p, uint8_t* smem, MlaBarriers* bars) {
+  using C = MlaCfg<true>;
+  volatile int* abort = &bars->abort;
+  const int t = threadIdx.x - 192;  // 0..63
+  int ub, ue, s;
+  const int32_t* prefix;
+  mla_range<kSparse>(p, ub, ue, s, prefix);
+  int it = 0;
+  int u = ub;
+  while (u < ue) {
+    int sb, se;
+    if (prefix) {
+      sb = prefix[s];
+      se = prefix[s + 1];
+      if (se <= u) { ++s; continue; }
+    } else {
+      sb = u;
+      se = ue;
+    }
+    MlaSeg g;
+    mla_seg<kSparse>(p, s, g);
+    const int a = u - sb, e = min(ue, se) - sb;
+    for (int j = 0; j < e - a; ++j, ++it) {
+      const int st = it % kMlaStages, hb = it & 1;
+      if (!mbar_wait(&bars->kv_full[st], (it / kMlaStages) & 1, abort, 76)) return;
+      if (it >= 2 && !mbar_wait(&bars->vh_empty[hb], ((it >> 1) - 1) & 1, abort, 77)) return;
+      // keys of the tile that exist (sparse: skipped entries are zeros already)
+      const int nvalid = kSparse ? kMlaBN : g.len - (a + j) * kMlaBN;
+      const uint8_t* src = smem + C::kKVOff + st * C::kKVBytes;
+      uint8_t* dst = smem + C::kVHOff + hb * C::kVHBytes;
+#pragma unroll 2
+      for (int x = t; x < kMlaBN * 16; x += 64) {
+        // key row, source chunk (0, 1) and its 16-byte unit: e4m3 columns
+        // 128 * c + 16 * unit .. + 15
+        const int row = x >> 4, c = (x >> 3) & 1, unit = x & 7;
+        uint4 v = *reinterpret_cast<const uint4*>(src + c * kMlaKVChunkBytes + row * 128 +
+                                                  ((unit ^ (row & 7)) << 4));
+        if (row >= nvalid) v = make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          h[2 * q] = fp8x2_to_f16x2<2>((unsigned short)(w[q] & 0xffff));
+          h[2 * q + 1] = fp8x2_to_f16x2<2>((unsigned short)(w[q] >> 16));
+        }
+        // fp16 columns 128 c + 16 unit .. + 15: chunk 2c + unit / 4, units
+        // 2 (unit % 4) and + 1 of that chunk's 128-byte row
+        const int dchunk = 2 * c + (unit >> 2), du = (unit & 3) * 2;
+        uint8_t* drow = dst + dchunk * kMlaKVChunkBytes + row * 128;
+        *reinterpret_cast<uint4*>(drow + ((du ^ (row & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(drow + (((du + 1) ^ (row & 7)) << 4)) =
+            make_uint4(h[4], h[5], h[6], h[7]);
+      }
+      fence_proxy_async_smem();  // the fp16 tile is read by the tensor core
+      mbar_arrive(&bars->vh_full[hb]);
+      mbar_arrive(&bars->kv_empty[st]);
+    }
+    u = min(ue, se);
+    ++s;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Softmax warpgroup
 // ---------------------------------------------------------------------------
 // Loads this CTA's partial scores of the tile with global index g into sv
@@ -489,8 +625,10 @@ drain : {
 // CTA's tile g - 1, which the other CTA sent after reading its tile g - 2
 // (the buffer's last use there), so the buffer is free; and the barrier is at
 // most one phase ahead of its waiter.
+template <bool kFp8>
 DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint32_t lane, int r,
                            int rank, int g, uint32_t* sv) {
+  using C = MlaCfg<kFp8>;
   const int sb = g % kMlaSBufs, b = g % kMlaXsBufs;
   if (!warp_wait(&bars->s_full[sb], (g / kMlaSBufs) & 1, &bars->abort, 80)) return false;
   tc_fence_after();
@@ -503,7 +641,7 @@ DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint
   const bool leader = (threadIdx.x & 31) == 0;
   if (leader) bulk_wait_read<1>();
   __syncwarp();
-  uint8_t* stage = smem + kMlaXoOff + b * kMlaXsBytes + r * 128;
+  uint8_t* stage = smem + C::kXoOff + b * kMlaXsBytes + r * 128;
 #pragma unroll
   for (int k = 0; k < 8; ++k)
     *reinterpret_cast<uint4*>(stage + ((k ^ (r & 7)) << 4)) =
@@ -514,16 +652,17 @@ DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint
     const uint32_t bar = mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1);
     const uint32_t off = b * kMlaXsBytes + warp_row0 * 128;
     mbar_arrive_expect_tx_remote(bar, 32 * 128);
-    bulk_copy_to_cluster(mapa_shared(smem_u32(smem + kMlaXsOff + off), rank ^ 1),
-                         smem_u32(smem + kMlaXoOff + off), 32 * 128, bar);
+    bulk_copy_to_cluster(mapa_shared(smem_u32(smem + C::kXsOff + off), rank ^ 1),
+                         smem_u32(smem + C::kXoOff + off), 32 * 128, bar);
     bulk_commit();
   }
   return true;
 }
 
-template <bool kSparse>
+template <bool kSparse, bool kFp8>
 DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem,
                       int rank) {
+  using C = MlaCfg<kFp8>;
   volatile int* abort = &bars->abort;
   const int r = threadIdx.x;  // 0..127
   const uint32_t lane = (uint32_t)(r & ~31) << 16;
@@ -533,7 +672,6 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
   const int32_t* prefix;
   mla_range<kSparse>(p, ub, ue, s, prefix);
   int it = 0;
-  const float sl2 = p.scale_log2;
   if (!p.meta && ue == 0) {
     // empty sequence without metadata: O = 0, LSE = -inf
     MlaSeg g;
@@ -573,13 +711,21 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     const int* idx_row =
         kSparse ? p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss + g.kvg * p.idx_sh
                 : nullptr;
+    // FP8: S and O use the dequantised rows (MATE FMHA dtype notes): the q and
+    // k descales of (sequence, KV head) scale the scores, the v descale O.
+    float sl2 = p.scale_log2, v_scale = 1.f;
+    if (kFp8 && p.q_descale != nullptr) {
+      const int di = g.bk * p.heads_kv + g.kvg;
+      sl2 *= p.q_descale[di] * p.k_descale[di];
+      v_scale = p.v_descale[di];
+    }
     float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
     bool seen = false;
     // The partial scores of tile g + 1 go to the other CTA as soon as those of
     // tile g have arrived here: they are in flight while tile g is
     // exponentiated.
     uint32_t sv[kMlaBN];
-    if (n > 0 && !mla_send_partial(bars, smem, tmem, lane, r, rank, it, sv)) return;
+    if (n > 0 && !mla_send_partial<kFp8>(bars, smem, tmem, lane, r, rank, it, sv)) return;
     for (int j = 0; j < n; ++j) {
       const int gi = it + j;
       const int t = a + j;
@@ -588,7 +734,7 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
         // The other CTA's partials of this tile.
         const int b = gi % kMlaXsBufs;
         if (!warp_wait_cluster(&bars->xs_full[b], (gi / kMlaXsBufs) & 1, abort, 83)) return;
-        const uint8_t* src = smem + kMlaXsOff + b * kMlaXsBytes + r * 128;
+        const uint8_t* src = smem + C::kXsOff + b * kMlaXsBytes + r * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint4 v = *reinterpret_cast<const uint4*>(src + ((k ^ (r & 7)) << 4));
@@ -598,7 +744,8 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
           sv[4 * k + 3] = __float_as_uint(__uint_as_float(sv[4 * k + 3]) + __uint_as_float(v.w));
         }
       }
-      if (j + 1 < n && !mla_send_partial(bars, smem, tmem, lane, r, rank, gi + 1, sv_next)) return;
+      if (j + 1 < n && !mla_send_partial<kFp8>(bars, smem, tmem, lane, r, rank, gi + 1, sv_next))
+        return;
       if constexpr (kSparse) {
         // Key position of entry e (see mla_sparse_pos); visible iff
         // 0 <= pos <= hi (hi = L - 1, or with sparse_mode=3, "rightDownCausal",
@@ -633,10 +780,11 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
         }
         // Rows of the tile past the end of the cache hold whatever the page
         // has there: zero this V half of them so P = 0 never meets a NaN. S
-        // of this tile has been computed already.
+        // of this tile has been computed already. (e4m3: the conversion warps
+        // zero them in the fp16 copy.)
         const int nvalid = g.len - k0;
-        if (nvalid < kMlaBN) {
-          uint8_t* kvs = smem + kMlaKVOff + (gi % kMlaStages) * kMlaKVBytes;
+        if (!kFp8 && nvalid < kMlaBN) {
+          uint8_t* kvs = smem + C::kKVOff + (gi % kMlaStages) * C::kKVBytes;
           const int bad = kMlaBN - nvalid;
           for (int x = r; x < 4 * bad * 8; x += 128) {
             const int c = x / (bad * 8), rem = x % (bad * 8);
@@ -683,12 +831,19 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       for (int c = 0; c < kMlaBN / 2; ++c) {
         const float p0 = ex2(fmaf(__uint_as_float(sv[2 * c]), sl2, -m_use));
         const float p1 = ex2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -m_use));
-        // bf16 P rounded to nearest (ties away from zero; P >= 0); O is
-        // normalised by the sum of the same rounded values
-        const uint32_t r0 = __float_as_uint(p0) + 0x8000u, r1 = __float_as_uint(p1) + 0x8000u;
-        pk[c] = __byte_perm(r0, r1, 0x7632);
         le += p0 + p1;
-        lr += __uint_as_float(r0 & 0xffff0000u) + __uint_as_float(r1 & 0xffff0000u);
+        if constexpr (kFp8) {
+          // fp16 P (to nearest even); O is normalised by the sum of the same
+          // rounded values
+          pk[c] = pack_f16x2(p0, p1);
+          lr += sum2<true>(pk[c]);
+        } else {
+          // bf16 P rounded to nearest (ties away from zero; P >= 0); O is
+          // normalised by the sum of the same rounded values
+          const uint32_t r0 = __float_as_uint(p0) + 0x8000u, r1 = __float_as_uint(p1) + 0x8000u;
+          pk[c] = __byte_perm(r0, r1, 0x7632);
+          lr += __uint_as_float(r0 & 0xffff0000u) + __uint_as_float(r1 & 0xffff0000u);
+        }
       }
       l_run += le;
       l_rnd += lr;
@@ -714,7 +869,7 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     }
     if (!seen) l_run = l_rnd = 0.f;
     const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-    const float inv = (l_rnd > 0.f && seen) ? 1.f / l_rnd : 0.f;
+    const float inv = (l_rnd > 0.f && seen) ? v_scale / l_rnd : 0.f;
     const float lse = (l_run > 0.f && seen) ? (m_use + log2f(l_run)) * kLn2 : -INFINITY;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + g.b * p.o_sb +
                           (int64_t)tok * p.o_ss + (int64_t)head * p.o_sh + rank * kMlaDvHalf;
@@ -764,10 +919,11 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
   }
 }
 
-template <bool kSparse>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+template <bool kSparse, bool kFp8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThreads, 1)
     mla_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
                const MlaParams p) {
+  using C = MlaCfg<kFp8>;
   // 128-byte swizzled TMA tiles need 1024-byte aligned shared memory; both
   // CTAs of the cluster share the layout, so both leave here or neither.
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -775,7 +931,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (threadIdx.x == 0) raise_error(ATTN_DEVERR_SMEM_ALIGN, 2);
     return;
   }
-  MlaBarriers* bars = reinterpret_cast<MlaBarriers*>(smem + kMlaBarOff);
+  MlaBarriers* bars = reinterpret_cast<MlaBarriers*>(smem + C::kBarOff);
   const int warp = threadIdx.x >> 5;
   const int rank = (int)cluster_ctarank();
   if (threadIdx.x == 0) {
@@ -783,7 +939,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     mbar_init(&bars->q_empty, 1);
     for (int i = 0; i < kMlaStages; ++i) {
       mbar_init(&bars->kv_full[i], kSparse ? 32 : 1);
-      mbar_init(&bars->kv_empty[i], 1);
+      // e4m3: released by the S MMA's commit and the 64 conversion threads
+      mbar_init(&bars->kv_empty[i], kFp8 ? 1 + 64 : 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->vh_full[i], 64);
+      mbar_init(&bars->vh_empty[i], 1);
     }
     for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->s_full[i], 1);
     for (int i = 0; i < kMlaXsBufs; ++i)
@@ -821,11 +982,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const uint32_t tmem = bars->tmem_base;
   if (!s_bad) {
     if (warp < 4)
-      mla_softmax<kSparse>(p, smem, bars, tmem, rank);
+      mla_softmax<kSparse, kFp8>(p, smem, bars, tmem, rank);
     else if (warp == 4)
-      mla_producer<kSparse>(p, &map_q, &map_kv, smem, bars, rank);
-    else
-      mla_mma<kSparse>(p, smem, bars, tmem, rank);
+      mla_producer<kSparse, kFp8>(p, &map_q, &map_kv, smem, bars, rank);
+    else if (warp == 5)
+      mla_mma<kSparse, kFp8>(p, smem, bars, tmem, rank);
+    else if constexpr (kFp8)
+      mla_convert<kSparse>(p, smem, bars);
   }
   // The partial-score copies this CTA sent have landed in the other CTA.
   if (warp < 4 && (threadIdx.x & 31) == 0) bulk_wait_all();

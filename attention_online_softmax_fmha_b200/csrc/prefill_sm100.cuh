@@ -416,16 +416,6 @@ drain : {
 // the P V MMA reads (two 64-column chunks, 128-byte swizzled); the e4m3 stage
 // is then released to the producer and the fp16 stage handed to the MMA.
 // ---------------------------------------------------------------------------
-// Two FP8 values (low byte first) to two fp16 values, exactly.
-template <int kType>
-DEVI uint32_t fp8x2_to_f16x2(unsigned short v) {
-  uint32_t h;
-  if constexpr (kType == 3)
-    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(v));
-  else
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
-  return h;
-}
 
 template <int D, int kType>
 DEVI void prefill_convert(const PrefillParams& p, uint8_t* smem, PrefillBarriers* bars) {

@@ -251,6 +251,10 @@ class MlaInputs:
     indices: Optional[torch.Tensor]  # int32 (B, s_q, H_kv, topk) or None
     topk: int
     num_heads_kv: int = 1
+    dtype: str = "bf16"              # "bf16", or "e4m3" for q and the cache
+    q_descale: Optional[torch.Tensor] = None   # e4m3: fp32 (B, H_kv) in [0.5, 2]
+    k_descale: Optional[torch.Tensor] = None
+    v_descale: Optional[torch.Tensor] = None
 
     @property
     def batch(self) -> int:
@@ -280,15 +284,21 @@ def sparse_indices(seqlens: Sequence[int], seqlen_q: int, topk: int, seed: int,
 def make_mla(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, page_size: int = 64,
              head_dim: int = 576, head_dim_v: int = 512, table: str = "permuted",
              causal: bool = False, topk: int = 0, index_kind: str = "uniform",
-             scale: Optional[float] = None, num_heads_kv: int = 1, seed: int = 0,
-             device="cpu") -> MlaInputs:
+             scale: Optional[float] = None, num_heads_kv: int = 1, dtype: str = "bf16",
+             seed: int = 0, device="cpu") -> MlaInputs:
+    """MLA inputs; dtype "e4m3" draws q and the cache as N(0, 1) converted to
+    e4m3 and descales U[0.5, 2] per (sequence, KV head)."""
     seqlens = [int(x) for x in seqlens]
     g_cpu = _gen(seed + 7919, "cpu")
     bt, nblocks = _block_table(seqlens, page_size, table, g_cpu)
     g = _gen(seed, device)
     B = len(seqlens)
-    q = _values((B, seqlen_q, num_heads_q, head_dim), "bf16", g, device)
-    kv = _values((nblocks, page_size, num_heads_kv, head_dim), "bf16", g, device)
+    q = _values((B, seqlen_q, num_heads_q, head_dim), dtype, g, device)
+    kv = _values((nblocks, page_size, num_heads_kv, head_dim), dtype, g, device)
+    desc = [None] * 3
+    if dtype in _FP8:
+        desc = [torch.rand(B, num_heads_kv, generator=g, device=device) * 1.5 + 0.5
+                for _ in range(3)]
     idx = None
     if topk:
         # one index list per KV head (the first with the given seed)
@@ -298,7 +308,7 @@ def make_mla(*, seqlens: Sequence[int], seqlen_q: int, num_heads_q: int, page_si
         scale = 1.0 / math.sqrt(head_dim)
     return MlaInputs(q, kv, bt.to(device), torch.tensor(seqlens, dtype=torch.int32, device=device),
                      seqlens, page_size, num_heads_q, head_dim_v, bool(causal), float(scale), idx,
-                     int(topk), int(num_heads_kv))
+                     int(topk), int(num_heads_kv), dtype, *desc)
 
 
 @dataclasses.dataclass
@@ -373,6 +383,12 @@ CONFIGS = {
                       page_size=64),
     "mla_sparse": dict(kind="mla", lengths=(64, 4096, 65536), seqlen_q=2, num_heads_q=128,
                        page_size=64, topk=2048),
+    # the MLA workloads against an e4m3 latent cache (and e4m3 q) with
+    # per-(sequence, KV head) descales
+    "mla_dense_fp8": dict(kind="mla", lengths=(64, 4096, 65536), seqlen_q=2, num_heads_q=128,
+                          page_size=64, dtype="e4m3"),
+    "mla_sparse_fp8": dict(kind="mla", lengths=(64, 4096, 65536), seqlen_q=2, num_heads_q=128,
+                           page_size=64, topk=2048, dtype="e4m3"),
     # 8-sequence versions of the MLA workloads, for profiler captures
     "mla_dense_small": dict(kind="mla", lengths=(8, 4096, 65536), seqlen_q=2, num_heads_q=128,
                             page_size=64),

@@ -42,7 +42,7 @@ HEADLINE = "varlen_causal_gqa"
 # Timed beside the headline in a default run, each with its own roofline: the
 # decode half of the metric, the other prefill configurations and MLA.
 DEFAULT_EXTRA = ["paged_decode", "paged_decode_fp8", "window_sink", "window_sink_fp8",
-                 "mla_dense", "mla_sparse"]
+                 "mla_dense", "mla_sparse", "mla_dense_fp8", "mla_sparse_fp8"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -312,7 +312,10 @@ def mla_workload(name: str, seed: int, device):
     sa.meta_bytes = meta.numel() * 4
     ma, out, lse, ws = B.mla_args(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens,
                                   scale=inp.scale, causal=inp.causal, indices=inp.indices,
-                                  meta=meta)
+                                  meta=meta, q_descale=inp.q_descale, k_descale=inp.k_descale,
+                                  v_descale=inp.v_descale)
+    fp8 = inp.dtype == "e4m3"
+    es = inp.kv_cache.element_size()
     fn = L.mla_sparse_fwd if sparse else L.mla_fwd_paged
     if sparse:
         idx = inp.indices.cpu()
@@ -323,7 +326,8 @@ def mla_workload(name: str, seed: int, device):
         pairs_tok = sum(inp.seqlens) * sq
         kv_rows = sum(inp.seqlens)
     flops = 2.0 * (576 + 512) * Hq * pairs_tok
-    nbytes = kv_rows * 576 * 2 + inp.q.numel() * 2 + out.numel() * 2 + lse.numel() * 4
+    nbytes = (kv_rows * 576 * es + inp.q.numel() * es + out.numel() * 2 + lse.numel() * 4
+              + (3 * inp.batch * 4 if fp8 else 0))
 
     def step(stream):
         st = L.attn_sched_metadata(ctypes.byref(sa), stream.cuda_stream)
@@ -333,7 +337,8 @@ def mla_workload(name: str, seed: int, device):
         if st != B.OK:
             raise B.AttnError(name, st)
 
-    small = [inp.q, inp.block_table, inp.cache_seqlens] + ([inp.indices] if sparse else [])
+    small = [inp.q, inp.block_table, inp.cache_seqlens] + ([inp.indices] if sparse else []) + (
+        [inp.q_descale, inp.k_descale, inp.v_descale] if fp8 else [])
     host_small = [t.cpu().pin_memory() for t in small]
     host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory(),
                 torch.empty(lse.shape, dtype=lse.dtype).pin_memory()]
@@ -347,12 +352,12 @@ def mla_workload(name: str, seed: int, device):
 
     cfg = {"workload": name, "batch": inp.batch, "seqlen_q": sq, "num_heads_q": Hq,
            "num_heads_kv": 1, "head_dim_qk": 576, "head_dim_v": 512, "page_size": inp.page_size,
-           "cache_seqlens": "uniform[4096,65536]", "topk": topk or None, "dtype": "bf16",
+           "cache_seqlens": "uniform[4096,65536]", "topk": topk or None, "dtype": inp.dtype,
            "kv_bytes_per_step": nbytes}
     return dict(step=step, e2e_step=e2e_step, work=flops / 1e12, unit="TFLOP/s", bound="tensor",
-                kernel=f"mla_kernel<{int(sparse)}>", launches_per_step=3,
+                kernel=f"mla_kernel<{int(sparse)},{int(fp8)}>", launches_per_step=3,
                 h2d=sum(t.numel() * t.element_size() for t in host_small),
-                d2h=sum(t.numel() * t.element_size() for t in host_out), cfg=cfg, dtype="bf16",
+                d2h=sum(t.numel() * t.element_size() for t in host_out), cfg=cfg, dtype=inp.dtype,
                 inp=inp, keep=(meta, ws, out, lse), outputs=(out, lse), gbytes=nbytes / 1e9,
                 per_unit=f"2*(576+512)*H_q FLOP per visible (token, key) pair; "
                 f"{pairs_tok} pairs, {nbytes} bytes per step")
@@ -370,6 +375,8 @@ WORKLOADS = {
     "paged_decode_fp8": paged_workload,
     "mla_dense": mla_workload,
     "mla_sparse": mla_workload,
+    "mla_dense_fp8": mla_workload,
+    "mla_sparse_fp8": mla_workload,
     "mla_dense_small": mla_workload,
     "mla_sparse_small": mla_workload,
 }

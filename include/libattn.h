@@ -367,6 +367,12 @@ attn_status_t attn_combine(const attn_combine_args* args, void* stream);
 /* H_q and H_kv) or NULL; workspace from mla_workspace_size().               */
 /* Supported now: H_q / H_kv a power of two up to 128 or a multiple of 128;  */
 /*   page_size a power of two in [16, 256].                                  */
+/* FP8 (MATE "Attention", FMHA dtype notes and FP8 paragraph, applied to the */
+/*   latent cache): dtype = ATTN_DTYPE_E4M3 makes q and kv_cache e4m3 codes  */
+/*   (strides still in elements, i.e. bytes); q_descale, k_descale and       */
+/*   v_descale fp32 (B, H_kv) are all given (K = row * k_descale,            */
+/*   V = row[:512] * v_descale, q * q_descale) or all NULL (= 1). The output */
+/*   stays bf16. dtype = ATTN_DTYPE_BF16 (0) takes no descales.              */
 /* ------------------------------------------------------------------------ */
 typedef struct {
   const void* q;
@@ -407,6 +413,10 @@ typedef struct {
   int64_t idx_stride_h;       /* H_kv > 1, sparse: KV-head stride of indices   */
   const int32_t* cu_seqlens_q; /* mla_sparse_fwd with packed (TND) queries, or  */
                               /* NULL; see mla_sparse_fwd                       */
+  int32_t dtype;              /* ATTN_DTYPE_BF16 or ATTN_DTYPE_E4M3 (q and cache) */
+  const float* q_descale;     /* e4m3: (B, H_kv) each, all given or all NULL   */
+  const float* k_descale;     /*   (TND: B is the number of sequences)         */
+  const float* v_descale;
 } mla_args;
 
 /* Bytes of workspace for these arguments (host only; 0 when meta is NULL).  */

@@ -1,6 +1,6 @@
 """MLA-absorbed decode (mla_fwd_paged) and its top-k sparse variant
 (mla_sparse_fwd) on the GPU against the fp64 oracle: bf16 outputs within
-1e-2 max-abs, LSE within 1e-3."""
+1e-2 max-abs (5e-2 for e4m3 q and cache with descales), LSE within 1e-3."""
 import numpy as np
 import pytest
 import torch
@@ -27,7 +27,8 @@ def run(inp, use_meta=True, num_ctas=0):
         meta = B.mla_metadata(inp.cache_seqlens, batch=inp.batch, seqlen_q=inp.q.shape[1],
                               num_heads_q=inp.num_heads_q, page_size=inp.page_size, topk=topk,
                               num_ctas=num_ctas, num_heads_kv=inp.num_heads_kv)
-    kw = dict(scale=inp.scale, causal=inp.causal, meta=meta, num_ctas=num_ctas)
+    kw = dict(scale=inp.scale, causal=inp.causal, meta=meta, num_ctas=num_ctas,
+              q_descale=inp.q_descale, k_descale=inp.k_descale, v_descale=inp.v_descale)
     if inp.indices is None:
         out, lse = B.mla_fwd_paged(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, **kw)
     else:
@@ -38,16 +39,27 @@ def run(inp, use_meta=True, num_ctas=0):
     return out, lse
 
 
+def _desc(inp):
+    if inp.q_descale is None:
+        return {}
+    return dict(q_descale=inp.q_descale.cpu().numpy(), k_descale=inp.k_descale.cpu().numpy(),
+                v_descale=inp.v_descale.cpu().numpy())
+
+
+def _atol(inp):
+    return 5e-2 if inp.dtype == "e4m3" else 1e-2
+
+
 def check(inp, **kw):
     out, lse = run(inp, **kw)
     q, kv = to_f64(inp.q), to_f64(inp.kv_cache)
     bt = inp.block_table.cpu().numpy()
     if inp.indices is None:
-        ro, rl = oracle.mla_paged(q, kv, bt, inp.seqlens, 512, inp.scale, inp.causal)
+        ro, rl = oracle.mla_paged(q, kv, bt, inp.seqlens, 512, inp.scale, inp.causal, **_desc(inp))
     else:
         ro, rl = oracle.mla_sparse(q, kv, bt, inp.seqlens, inp.indices.cpu().numpy(), 512,
-                                   inp.scale)
-    assert_close_out(to_f64(out), ro, 1e-2)
+                                   inp.scale, **_desc(inp))
+    assert_close_out(to_f64(out), ro, _atol(inp))
     assert_close_lse(lse.cpu().numpy(), rl)
 
 
@@ -139,12 +151,13 @@ def _sampled(name, topk):
         pages = inp.block_table[b, :npg].long()
         kv = to_f64(inp.kv_cache[pages])
         q = to_f64(inp.q[b:b + 1])
+        desc = {k: v[b:b + 1] for k, v in _desc(inp).items()}
         if topk:
             ro, rl = oracle.mla_sparse(q, kv, np.arange(npg)[None], [L],
-                                       inp.indices[b:b + 1].cpu().numpy(), 512, inp.scale)
+                                       inp.indices[b:b + 1].cpu().numpy(), 512, inp.scale, **desc)
         else:
-            ro, rl = oracle.mla_paged(q, kv, np.arange(npg)[None], [L], 512, inp.scale)
-        assert_close_out(o[b:b + 1], ro, 1e-2)
+            ro, rl = oracle.mla_paged(q, kv, np.arange(npg)[None], [L], 512, inp.scale, **desc)
+        assert_close_out(o[b:b + 1], ro, _atol(inp))
         assert_close_lse(l[b:b + 1], rl)
 
 
@@ -157,6 +170,67 @@ def test_full_size_dense_sampled():
 def test_full_size_sparse_sampled():
     """The top-2048 sparse variant at full size; 3 sequences checked."""
     _sampled("mla_sparse", 2048)
+
+
+# ---------------------------------------------------------------------------
+# e4m3 q and latent cache with (B, H_kv) descales: S on the FP8 codes, P V in
+# fp16 on an exact fp16 copy of V. Tolerance 5e-2.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("num_ctas", [1, 5, 0])
+def test_fp8_dense_split_counts(num_ctas):
+    inp = W.make_mla(seqlens=LENS, seqlen_q=2, num_heads_q=128, page_size=64, dtype="e4m3",
+                     seed=50, device="cuda")
+    check(inp, num_ctas=num_ctas)
+
+
+def test_fp8_dense_without_metadata_causal_page16_several_kv_heads():
+    inp = W.make_mla(seqlens=[5, 77, 300], seqlen_q=3, num_heads_q=64, num_heads_kv=4,
+                     page_size=16, causal=True, dtype="e4m3", seed=51, device="cuda")
+    check(inp, use_meta=False)
+    check(inp, num_ctas=4)
+
+
+def test_fp8_without_descales_equals_unit_descales():
+    inp = W.make_mla(seqlens=[33, 200], seqlen_q=2, num_heads_q=128, dtype="e4m3", seed=52,
+                     device="cuda")
+    out1, lse1 = run(inp, num_ctas=3)
+    ones = torch.ones_like(inp.q_descale)
+    inp.q_descale, inp.k_descale, inp.v_descale = ones, ones, ones.clone()
+    out2, lse2 = run(inp, num_ctas=3)
+    plain = dict(scale=inp.scale, meta=B.mla_metadata(inp.cache_seqlens, batch=2, seqlen_q=2,
+                                                      num_heads_q=128, page_size=64, num_ctas=3),
+                 num_ctas=3)
+    out3, lse3 = B.mla_fwd_paged(inp.q, inp.kv_cache, inp.block_table, inp.cache_seqlens, **plain)
+    torch.cuda.synchronize()
+    assert torch.equal(out2, out3) and torch.equal(lse2, lse3)
+    assert not torch.equal(out1, out2)
+    check(inp, num_ctas=3)
+
+
+@pytest.mark.parametrize("num_ctas", [3, 0])
+def test_fp8_sparse_against_oracle(num_ctas):
+    inp = W.make_mla(seqlens=[20, 300, 3000], seqlen_q=2, num_heads_q=128, page_size=64,
+                     topk=256, dtype="e4m3", seed=53, device="cuda")
+    inp.indices[0, 1, 0, 5] = 19999
+    inp.indices[2, 0, 0, 7] = -5
+    check(inp, num_ctas=num_ctas)
+    check(inp, use_meta=False)
+
+
+def test_fp8_sparse_several_kv_heads():
+    inp = W.make_mla(seqlens=[20, 300, 3000], seqlen_q=2, num_heads_q=128, num_heads_kv=2,
+                     page_size=64, topk=128, dtype="e4m3", seed=54, device="cuda")
+    check(inp, num_ctas=3)
+
+
+def test_fp8_full_size_dense_sampled():
+    """The e4m3 MLA dense workload at full size; 3 sequences checked."""
+    _sampled("mla_dense_fp8", 0)
+
+
+def test_fp8_full_size_sparse_sampled():
+    _sampled("mla_sparse_fp8", 2048)
 
 
 @pytest.mark.parametrize("bs,num_ctas", [(4, 3), (64, 0)])
