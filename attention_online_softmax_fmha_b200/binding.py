@@ -46,7 +46,8 @@ class VarlenArgs(ctypes.Structure):
                 ("window_left", c_i32), ("window_right", c_i32),
                 ("sink", c_vp), ("q_descale", c_vp), ("k_descale", c_vp), ("v_descale", c_vp),
                 ("seqused_q", c_vp), ("seqused_k", c_vp), ("mask", c_vp),
-                ("mask_stride_b", c_i64), ("mask_stride_h", c_i64), ("mask_stride_s", c_i64)]
+                ("mask_stride_b", c_i64), ("mask_stride_h", c_i64), ("mask_stride_s", c_i64),
+                ("work_counter", c_vp)]
 
 
 class SchedArgs(ctypes.Structure):
@@ -226,11 +227,14 @@ def out_dtype_for(dtype: torch.dtype) -> torch.dtype:
 def varlen_args(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=None,
                 max_seqlen_k=None, scale=None, causal=False, window=(-1, -1), sink=None,
                 q_descale=None, k_descale=None, v_descale=None, out=None, lse=None,
-                seqused_q=None, seqused_k=None, mask=None):
+                seqused_q=None, seqused_k=None, mask=None, work_counter=None):
     """Build the argument struct (and allocate out/lse if not given).
 
     mask: fp32 tensor indexed [b, h, i, j] (a 4-D view; size-1 axes broadcast
-    with stride 0); seqused_q/k: int32 (B,) for the padded layout."""
+    with stride 0); seqused_q/k: int32 (B,) for the padded layout.
+    work_counter: an int32 tensor of one element for the dynamic unit
+    schedule (allocated here if not given; kept alive by the struct); False:
+    the static schedule."""
     varlen = cu_seqlens_q is not None
     _rows(q=q, k=k, v=v, out=out, lse=lse)
     _same_dtype(q, k=k, v=v)
@@ -280,6 +284,12 @@ def varlen_args(q, k, v, *, cu_seqlens_q=None, cu_seqlens_k=None, max_seqlen_q=N
         _TORCH_DTYPE.get(q.dtype, -1), float(scale), int(bool(causal)), int(window[0]),
         int(window[1]), _ptr(sink), _ptr(q_descale), _ptr(k_descale), _ptr(v_descale),
         _ptr(seqused_q), _ptr(seqused_k), _ptr(mask), msb, msh, mss)
+    if work_counter is None:
+        work_counter = torch.empty(1, dtype=torch.int32, device=q.device)
+    if work_counter is not False:
+        _int32(work_counter=work_counter)
+        a.work_counter = work_counter.data_ptr()
+        a._keep = work_counter  # the struct holds its address
     return a, out, lse
 
 
@@ -287,6 +297,8 @@ def fwd_varlen(q, k, v, *, stream=None, **kw):
     """Attention forward (attn_fwd_varlen). Returns (out, lse)."""
     a, out, lse = varlen_args(q, k, v, **kw)
     _check("attn_fwd_varlen", lib().attn_fwd_varlen(ctypes.byref(a), _stream(stream)))
+    if stream is not None and getattr(a, "_keep", None) is not None and hasattr(stream, "cuda_stream"):
+        a._keep.record_stream(stream)  # freed only after the work queued there
     return out, lse
 
 

@@ -32,6 +32,9 @@ attn_status_t launch_prefill(int grid, const CUtensorMap& mq, const CUtensorMap&
     return launch_status(set_smem(kernel, C::kSmemBytes));
   });
   if (cst != ATTN_OK) return cst;
+  if (p.work_counter &&
+      cudaMemsetAsync(p.work_counter, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
   return launch_status(cudaGetLastError());
 }
@@ -95,6 +98,7 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   p.causal = a.causal;
   p.window_left = a.window_left;
   p.window_right = a.window_right;
+  p.work_counter = a.work_counter;
 
   const int sms = device_sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
@@ -135,6 +139,7 @@ attn_status_t check_varlen(const attn_varlen_args* a) {
   if (a->head_dim_qk != 64 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
   if (fp8 && a->head_dim_qk != 128) return ATTN_ERR_UNSUPPORTED;
   if (varlen && (a->seqused_q || a->seqused_k)) return ATTN_ERR_INVALID_ARG;  // padded only
+  if (reinterpret_cast<uintptr_t>(a->work_counter) & 3u) return ATTN_ERR_INVALID_ARG;
   if (a->mask) {
     if (a->mask_stride_b < 0 || a->mask_stride_h < 0 || a->mask_stride_s < 0)
       return ATTN_ERR_INVALID_ARG;

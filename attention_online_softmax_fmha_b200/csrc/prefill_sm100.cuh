@@ -9,8 +9,13 @@
 // sparse_mode=3 "rightDownCausal").
 //
 // Design: one CTA per SM, persistent over work units of 256 query rows (two
-// 128-row tiles Q0, Q1 of one sequence and head; heaviest units first). Both
-// tiles stream the same K/V tiles of 128 keys.
+// 128-row tiles Q0, Q1 of one sequence and head). Units are numbered
+// heaviest first (last row block of every sequence and head first); with a
+// work counter each CTA takes the next number when it starts a unit, so
+// CTAs that drew short units take more of them, otherwise every
+// gridDim-th number. The producer takes the numbers and hands them to the
+// other roles through a small ring in shared memory. Both tiles stream the
+// same K/V tiles of 128 keys.
 //   warpgroup 0, 1   softmax of Q0 / Q1: thread r owns query row r of its
 //                    tile (= TMEM lane r). Online softmax in the log2 domain;
 //                    O in TMEM is rescaled only when a row's max grows by more
@@ -62,6 +67,7 @@ struct PrefillParams {
   int32_t causal;
   int32_t window_left;
   int32_t window_right;
+  int32_t* work_counter;  // next unit number (zeroed before the launch), or nullptr
 };
 
 constexpr int kPrefillBM = 128;               // query rows per tile
@@ -118,7 +124,12 @@ struct PrefillCfg {
   static constexpr uint32_t kTmemO0 = 256, kTmemO1 = 256 + D;
 };
 
+// Unit numbers in flight from the producer to the other roles.
+constexpr int kUnitRing = 4;
+
 struct PrefillBarriers {
+  uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
+  int32_t unit_idx[kUnitRing];  // a unit number, or -1 after the CTA's last unit
   uint64_t q_full, q_empty;
   uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t vh_full[4], vh_empty[4];
@@ -176,6 +187,17 @@ DEVI bool prefill_unit(const PrefillParams& p, int t, PrefillUnit& u) {
   return true;
 }
 
+// Takes the k-th unit number of this CTA from the ring (warp-collective; each
+// consuming warp releases the slot once). Returns false if the wait gave up.
+DEVI bool take_unit(PrefillBarriers* bars, int k, int& t, int site) {
+  const int slot = k % kUnitRing;
+  if (!warp_wait(&bars->unit_full[slot], (k / kUnitRing) & 1, &bars->abort, site)) return false;
+  t = *reinterpret_cast<volatile int32_t*>(&bars->unit_idx[slot]);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&bars->unit_empty[slot]);
+  return true;
+}
+
 // Inclusive visible key range of query row i.
 DEVI void row_key_range(const PrefillParams& p, int i, int len_q, int len_k, int& lo, int& hi) {
   const int delta = len_k - len_q;
@@ -219,10 +241,25 @@ DEVI void prefill_producer(const PrefillParams& p, const CUtensorMap* mq, const 
   tma_prefetch_desc(mq);
   tma_prefetch_desc(mk);
   tma_prefetch_desc(mv);
-  int it = 0, nq = 0;
-  for (int t = blockIdx.x; t < p.total_units; t += gridDim.x) {
+  int it = 0, nq = 0, k = 0;
+  for (int fetched = 0;; ++fetched) {
+    // The next unit number: from the counter, or every gridDim-th. Numbers
+    // past a sequence's end are passed over; the roles get the rest, then -1.
+    const int t = p.work_counter ? atomicAdd(p.work_counter, 1)
+                                 : blockIdx.x + fetched * (int)gridDim.x;
+    const bool end = t >= p.total_units;
     PrefillUnit u;
-    if (!prefill_unit(p, t, u)) continue;
+    if (!end && !prefill_unit(p, t, u)) continue;
+    {
+      const int slot = k % kUnitRing;
+      if (k >= kUnitRing &&
+          !mbar_wait(&bars->unit_empty[slot], ((k / kUnitRing) - 1) & 1, abort, 5))
+        goto drain;
+      bars->unit_idx[slot] = end ? -1 : t;
+      mbar_arrive(&bars->unit_full[slot]);  // release: the number is visible to the waiters
+      ++k;
+    }
+    if (end) break;
     const int n = u.kt1 - u.kt0;
     if (n <= 0) continue;
     const int hk = u.h / p.group;
@@ -350,9 +387,12 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
   const uint32_t tO0 = tmem + C::kTmemO0, tO1 = tmem + C::kTmemO1;
   int it = 0, nq = 0, units = 0;
 
-  for (int t = blockIdx.x; t < p.total_units; t += gridDim.x) {
+  for (int k = 0;; ++k) {
+    int t;
+    if (!take_unit(bars, k, t, 9)) goto drain;
+    if (t < 0) break;
     PrefillUnit u;
-    if (!prefill_unit(p, t, u)) continue;
+    prefill_unit(p, t, u);
     const int n = u.kt1 - u.kt0;
     if (n <= 0) continue;
     if (!warp_wait(&bars->q_full, nq & 1, abort, 10)) goto drain;
@@ -424,9 +464,12 @@ DEVI void prefill_convert(const PrefillParams& p, uint8_t* smem, PrefillBarriers
   volatile int* abort = &bars->abort;
   const int t = threadIdx.x - 320;  // 0..63
   int it = 0;
-  for (int wu = blockIdx.x; wu < p.total_units; wu += gridDim.x) {
+  for (int k = 0;; ++k) {
+    int wu;
+    if (!take_unit(bars, k, wu, 52)) return;
+    if (wu < 0) break;
     PrefillUnit u;
-    if (!prefill_unit(p, wu, u)) continue;
+    prefill_unit(p, wu, u);
     const int n = u.kt1 - u.kt0;
     for (int j = 0; j < n; ++j, ++it) {
       const int sv = it % C::kVStages, sh = it % C::kVHStages;
@@ -665,9 +708,12 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
   const uint32_t s_tmem = tmem + (w ? C::kTmemS1 : C::kTmemS0) + lane;
   const uint32_t o_tmem = tmem + (w ? C::kTmemO1 : C::kTmemO0) + lane;
   int sj = 0, units = 0;
-  for (int t = blockIdx.x; t < p.total_units; t += gridDim.x) {
+  for (int k = 0;; ++k) {
+    int t;
+    if (!take_unit(bars, k, t, 24 + w)) return;
+    if (t < 0) break;
     PrefillUnit u;
-    if (!prefill_unit(p, t, u)) continue;
+    prefill_unit(p, t, u);
     const int n = u.kt1 - u.kt0;
     const int i = u.m * kPrefillUnit + w * kPrefillBM + r;
     const bool valid = i < u.len_q;
@@ -760,6 +806,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < kUnitRing; ++i) {
+      mbar_init(&bars->unit_full[i], 1);
+      // released by the MMA warp, the 8 softmax warps and (FP8) the 2 conversion warps
+      mbar_init(&bars->unit_empty[i], 9 + (C::kFp8 ? 2 : 0));
+    }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < C::kKStages; ++s) {

@@ -154,6 +154,14 @@ typedef struct {
   const int32_t* seqused_k;  /* padded layout only; nullable                  */
   const float* mask;         /* additive score mask; nullable                 */
   int64_t mask_stride_b, mask_stride_h, mask_stride_s;
+  int32_t* work_counter;     /* 4 bytes of device memory, or NULL. Given, the  */
+                             /* persistent CTAs take work units (256 query     */
+                             /* rows of one sequence and head, longest-running */
+                             /* first) from this counter as they finish the    */
+                             /* last; NULL: each CTA takes every gridDim-th    */
+                             /* unit. The call zeroes it on `stream` before    */
+                             /* the launch; calls in flight at the same time   */
+                             /* must not share one counter.                    */
 } attn_varlen_args;
 
 attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream);
