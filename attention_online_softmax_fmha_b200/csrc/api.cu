@@ -616,17 +616,45 @@ static __device__ __align__(256) unsigned char g_paged_scratch[kStaticScratchByt
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once
-// per device; host code must not use the array's name as an address).
+// The driver's cuCtxGetCurrent, fetched through the runtime (the library does
+// not link libcuda directly).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the scratch array on the current device (host code must
+// not use the array's name as an address). It is looked up once per device
+// and context: after a device reset the runtime creates a new primary context
+// and loads the library's module again, so the array moves, and the address
+// is looked up anew.
 void* static_scratch_address() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (get_ctx == nullptr) return nullptr;
+  // null until the runtime has made the device's context current on this thread
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (g_scratch_addr[dev] == nullptr || ctx == nullptr || g_scratch_ctx[dev] != ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress((void**)&ptr, g_paged_scratch) != cudaSuccess) return nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
     g_scratch_addr[dev] = ptr;
+    g_scratch_ctx[dev] = ctx;
   }
   return g_scratch_addr[dev];
 }

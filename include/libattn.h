@@ -316,7 +316,9 @@ attn_status_t attn_fwd_paged_kvcache(const attn_paged_args* args, void* stream);
 /* allocated or freed.                                                       */
 /*                                                                          */
 /* The first call on a device looks up the array's device address (a        */
-/* runtime call); make that first call before any stream capture. All calls */
+/* runtime call); make that first call before any stream capture. A device   */
+/* reset moves the array; the first call after it looks the address up      */
+/* again, so make that call before any capture as well. All calls           */
 /* share the one array and it keeps the last call's contents: calls that may */
 /* overlap on the GPU (other streams, other host threads) race on it and     */
 /* must be serialised by the caller. Nothing in the array needs to start at */
