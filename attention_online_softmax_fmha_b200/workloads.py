@@ -394,6 +394,14 @@ CONFIGS = {
                             page_size=64),
     "mla_sparse_small": dict(kind="mla", lengths=(8, 4096, 65536), seqlen_q=2,
                              num_heads_q=128, page_size=64, topk=2048),
+    # reduced-batch FP8 versions, for profiler captures
+    "paged_decode_fp8_small": dict(kind="paged", lengths=(16, 1024, 32768), seqlen_q=1,
+                                   num_heads_q=32, num_heads_kv=8, head_dim=128, page_size=64,
+                                   dtype="e4m3"),
+    "mla_dense_fp8_small": dict(kind="mla", lengths=(8, 4096, 65536), seqlen_q=2,
+                                num_heads_q=128, page_size=64, dtype="e4m3"),
+    "mla_sparse_fp8_small": dict(kind="mla", lengths=(8, 4096, 65536), seqlen_q=2,
+                                 num_heads_q=128, page_size=64, topk=2048, dtype="e4m3"),
 }
 
 

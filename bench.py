@@ -377,6 +377,9 @@ WORKLOADS = {
     "mla_sparse": mla_workload,
     "mla_dense_fp8": mla_workload,
     "mla_sparse_fp8": mla_workload,
+    "paged_decode_fp8_small": paged_workload,
+    "mla_dense_fp8_small": mla_workload,
+    "mla_sparse_fp8_small": mla_workload,
     "mla_dense_small": mla_workload,
     "mla_sparse_small": mla_workload,
 }
