@@ -523,9 +523,9 @@ struct PrefillRow {
 // rounded to bf16, goes to TMEM columns 64 .. 127 of the buffer; O is then
 // normalised by the fp32 sum, which the two parts together match to about
 // 2^-16.
-template <int kType, bool kRnd>
-DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float sl2,
-                           uint32_t* s, PrefillRow& row, bool split) {
+template <int kType, bool kRnd, class Sig>
+DEVI void prefill_exp_tile(const Sig& sig, uint32_t s_tmem, float sl2, uint32_t* s,
+                           PrefillRow& row, bool split) {
   constexpr bool kSplit = kRnd && kType == 0;  // the remainder pass may run
   constexpr bool kFp16 = kType != 0;  // P in fp16 (fp16 and FP8 inputs)
   const float m_use = (row.m_run == -INFINITY) ? 0.f : row.m_run;
@@ -579,7 +579,7 @@ DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float 
       // The head of P: the P V MMA starts on it.
       tmem_store_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_head[w]);
+      sig.p_head();
     }
   }
   {
@@ -592,18 +592,30 @@ DEVI void prefill_exp_tile(PrefillBarriers* bars, uint32_t s_tmem, int w, float 
   }
   tmem_store_wait();
   tc_fence_before();
-  mbar_arrive(&bars->p_full[w]);
+  sig.p_full();
 }
+
+// The softmax's hand-offs with the MMA warp of the one-CTA kernel: S of tile
+// w is ready (a commit on this CTA's barrier); the head / all of P is in TMEM
+// (every thread arrives).
+struct PrefillSig {
+  PrefillBarriers* bars;
+  int w;
+  DEVI bool wait_s(int g) const {
+    return warp_wait(&bars->s_full[w], g & 1, &bars->abort, 20 + w);
+  }
+  DEVI void p_head() const { mbar_arrive(&bars->p_head[w]); }
+  DEVI void p_full() const { mbar_arrive(&bars->p_full[w]); }
+};
 
 // One S tile of keys [k0, k0 + 128) of this thread's row: mask, row max,
 // lazy O rescale, P = 2^(s * scale * log2e - m) written over S (head first),
 // row sums. Returns false if a wait gave up.
-template <int D, int kType, bool kMask>
-DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t o_tmem, int w,
-                               int j, int g, int k0, float sl2, PrefillRow& row,
-                               const float* mrow, int len_k, bool split) {
-  volatile int* abort = &bars->abort;
-  if (!warp_wait(&bars->s_full[w], g & 1, abort, 20 + w)) return false;
+template <int D, int kType, bool kMask, class Sig>
+DEVI bool prefill_softmax_tile(const Sig& sig, uint32_t s_tmem, uint32_t o_tmem, int j, int g,
+                               int k0, float sl2, PrefillRow& row, const float* mrow, int len_k,
+                               bool split) {
+  if (!sig.wait_s(g)) return false;
   tc_fence_after();
   uint32_t s[kPrefillBN];
   tmem_load128(s_tmem, s);
@@ -692,9 +704,9 @@ DEVI bool prefill_softmax_tile(PrefillBarriers* bars, uint32_t s_tmem, uint32_t 
   // lie in first or partially masked tiles; other tiles add their fp32 sum to
   // both (their rounding errors average out over the row's many keys).
   if (j == 0 || kMask || split || __any_sync(0xffffffffu, partial))
-    prefill_exp_tile<kType, true>(bars, s_tmem, w, sl2, s, row, split);
+    prefill_exp_tile<kType, true>(sig, s_tmem, sl2, s, row, split);
   else
-    prefill_exp_tile<kType, false>(bars, s_tmem, w, sl2, s, row, false);
+    prefill_exp_tile<kType, false>(sig, s_tmem, sl2, s, row, false);
   return true;
 }
 
@@ -749,7 +761,7 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
         (kMask && valid) ? p.mask + u.b * p.m_sb + u.h * p.m_sh + (int64_t)i * p.m_ss : nullptr;
     const bool split = kType == 0 && !kMask && prefill_short_tile(p, u, w);
     for (int j = 0; j < n; ++j, ++sj)
-      if (!prefill_softmax_tile<D, kType, kMask>(bars, s_tmem, o_tmem, w, j, sj,
+      if (!prefill_softmax_tile<D, kType, kMask>(PrefillSig{bars, w}, s_tmem, o_tmem, j, sj,
                                                  (u.kt0 + j) * kPrefillBN, sl2, row, mrow,
                                                  u.len_k, split))
         return;
