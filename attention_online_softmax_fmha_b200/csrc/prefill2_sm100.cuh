@@ -166,6 +166,7 @@ struct P2Unit {
 // Unit t: rows m*512 .. m*512 + 511 of (sequence b, head h), numbered as in
 // prefill_unit (last row block of every sequence and head first). False for a
 // unit past its sequence's end.
+template <bool kUnion>
 DEVI bool p2_unit(const PrefillParams& p, int t, P2Unit& u) {
   const int bh = p.batch * p.num_heads_q;
   const int mr = t / bh;
@@ -205,6 +206,14 @@ DEVI bool p2_unit(const PrefillParams& p, int t, P2Unit& u) {
     u.K1 = max(u.K1, u.kt1[w]);
   }
   if (u.K1 == 0) u.K0 = 0;
+  if (kUnion) {
+#pragma unroll
+    for (int w = 0; w < 2; ++w)
+      if (u.kt1[w] > u.kt0[w]) {
+        u.kt0[w] = u.K0;
+        u.kt1[w] = u.K1;
+      }
+  }
   return true;
 }
 
@@ -236,6 +245,7 @@ DEVI bool p2_take_unit(P2Barriers* bars, int k, int& t, int site) {
 // ---------------------------------------------------------------------------
 // Producer (one thread per CTA)
 // ---------------------------------------------------------------------------
+template <bool kUnion>
 DEVI void p2_producer(const PrefillParams& p, const CUtensorMap* mq, const CUtensorMap* mk,
                       const CUtensorMap* mv, uint8_t* smem, P2Barriers* bars, int rank) {
   volatile int* abort = &bars->abort;
@@ -253,7 +263,7 @@ DEVI void p2_producer(const PrefillParams& p, const CUtensorMap* mq, const CUten
     if (rank == 0) {
       // The leader takes the next number and hands it to both CTAs' roles.
       t = p.work_counter ? atomicAdd(p.work_counter, 1) : cluster + fetched * nclusters;
-      if (t < p.total_units && !p2_unit(p, t, u)) continue;
+      if (t < p.total_units && !p2_unit<kUnion>(p, t, u)) continue;
       if (t >= p.total_units) t = -1;
       const int slot = k % kUnitRing;
       if (k >= kUnitRing &&
@@ -268,7 +278,7 @@ DEVI void p2_producer(const PrefillParams& p, const CUtensorMap* mq, const CUten
       if (!mbar_wait_cluster(&bars->unit_full[slot], (k / kUnitRing) & 1, abort, 6)) goto drain;
       t = *reinterpret_cast<volatile int32_t*>(&bars->unit_idx[slot]);
       mbar_arrive_remote(leader_addr(&bars->unit_empty[slot]));
-      if (t >= 0) p2_unit(p, t, u);
+      if (t >= 0) p2_unit<kUnion>(p, t, u);
     }
     ++k;
     if (t < 0) break;
@@ -356,6 +366,7 @@ DEVI bool p2_pv(P2Barriers* bars, int w, int np, uint32_t t_o, uint32_t t_p, uin
   return true;
 }
 
+template <bool kUnion>
 DEVI void p2_mma(const PrefillParams& p, uint8_t* smem, P2Barriers* bars, uint32_t tmem) {
   volatile int* abort = &bars->abort;
   constexpr uint32_t idesc_qk = make_idesc(256, kPrefillBN, 1, 0, 0);
@@ -372,7 +383,7 @@ DEVI void p2_mma(const PrefillParams& p, uint8_t* smem, P2Barriers* bars, uint32
     if (!p2_take_unit(bars, k, t, 9)) goto drain;
     if (t < 0) break;
     P2Unit u;
-    p2_unit(p, t, u);
+    p2_unit<kUnion>(p, t, u);
     if (u.K1 <= u.K0) continue;
     if (!warp_wait_cluster(&bars->q_full, nq & 1, abort, 10)) goto drain;
     ++nq;
@@ -454,6 +465,7 @@ struct P2Sig {
   }
 };
 
+template <bool kUnion>
 DEVI void p2_softmax(const PrefillParams& p, P2Barriers* bars, uint32_t tmem, int w, int rank) {
   using OutT = __nv_bfloat16;
   volatile int* abort = &bars->abort;
@@ -469,7 +481,7 @@ DEVI void p2_softmax(const PrefillParams& p, P2Barriers* bars, uint32_t tmem, in
     if (!p2_take_unit(bars, k, t, 24 + w)) return;
     if (t < 0) break;
     P2Unit u;
-    p2_unit(p, t, u);
+    p2_unit<kUnion>(p, t, u);
     const int n = u.kt1[w] - u.kt0[w];
     const int i = u.m * kP2Unit + w * 2 * kPrefillBM + rank * kPrefillBM + r;
     const bool valid = i < u.len_q;
@@ -527,6 +539,7 @@ DEVI void p2_softmax(const PrefillParams& p, P2Barriers* bars, uint32_t tmem, in
   }
 }
 
+template <bool kUnion>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPrefillThreads, 1)
     prefill2_kernel(const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k,
@@ -582,13 +595,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPrefillThreads, 1)
 
   if (warp < 8) {
     regs_inc<kPrefillSoftmaxRegs>();
-    p2_softmax(p, bars, tmem, warp >> 2, rank);
+    p2_softmax<kUnion>(p, bars, tmem, warp >> 2, rank);
   } else {
     regs_dec<kPrefillOtherRegs>();
     if (warp == 8) {
-      if (elect_lane0()) p2_producer(p, &map_q, &map_k, &map_v, smem, bars, rank);
+      if (elect_lane0()) p2_producer<kUnion>(p, &map_q, &map_k, &map_v, smem, bars, rank);
     } else if (warp == 9 && rank == 0) {
-      p2_mma(p, smem, bars, tmem);  // whole warp, one lane issues
+      p2_mma<kUnion>(p, smem, bars, tmem);  // whole warp, one lane issues
     }
   }
 

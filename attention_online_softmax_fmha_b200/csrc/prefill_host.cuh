@@ -61,13 +61,18 @@ attn_status_t launch_prefill2(int sms, const attn_varlen_args& a, const CUtensor
   const int64_t total = (int64_t)p.num_units_q * a.batch * a.num_heads_q;
   if (total > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
   p.total_units = (int32_t)total;
-  auto kernel = prefill2_kernel;
+  const char* ue = std::getenv("ATTN_P2_UNION");
+  auto kernel = (ue && ue[0] == '1') ? prefill2_kernel<true> : prefill2_kernel<false>;
   static std::atomic<uint64_t> configured{0};
   const attn_status_t cst = configure_per_device(configured, [&]() -> attn_status_t {
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
-    if (fa.numRegs != kPrefillLaunchRegs) return ATTN_ERR_UNSUPPORTED;
-    return launch_status(set_smem(kernel, kP2SmemBytes));
+    for (auto kf : {prefill2_kernel<true>, prefill2_kernel<false>}) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kf) != cudaSuccess) return ATTN_ERR_CUDA;
+      if (fa.numRegs != kPrefillLaunchRegs) return ATTN_ERR_UNSUPPORTED;
+      const attn_status_t st = launch_status(set_smem(kf, kP2SmemBytes));
+      if (st != ATTN_OK) return st;
+    }
+    return ATTN_OK;
   });
   if (cst != ATTN_OK) return cst;
   if (p.work_counter &&
