@@ -45,11 +45,9 @@ namespace attn {
 
 constexpr int kDecTileKeys = 64;
 constexpr int kDecRows = 16;       // query rows per segment (mma M)
-constexpr int kDecStages = 6;      // even: stage st always feeds warpgroup st % 2
 constexpr int kDecConsumerWarps = 8;  // two warpgroups
 constexpr int kDecConsumerThreads = 32 * kDecConsumerWarps;
 constexpr int kDecThreads = kDecConsumerThreads + 32;  // + the producer warp
-static_assert(kDecStages % 2 == 0, "alternate tiles keep a stage with one warpgroup");
 
 struct DecodeParams {
   const void* q;
@@ -83,16 +81,22 @@ struct DecodeCfg {
   static constexpr int kChunks = D / kChunkCols;
   static constexpr int kTileBytes = kDecTileKeys * D * kElt;  // K or V tile
   static constexpr int kStageBytes = 2 * kTileBytes;
+  // Stages in flight: about 190 KB of K/V per SM either way, enough bytes in
+  // flight to cover the memory latency at the SM's share of HBM bandwidth.
+  // Even: stage st always feeds warpgroup st % 2.
+  static constexpr int kStages = kFp8 ? 10 : 6;
+  static_assert(kStages % 2 == 0, "alternate tiles keep a stage with one warpgroup");
   static constexpr int kQStride = D * 2 + 16;                  // padded 16-bit Q row (bytes)
   static constexpr int kStageOff = 0;
-  static constexpr int kQOff = kDecStages * kStageBytes;
+  static constexpr int kQOff = kStages * kStageBytes;
   // FP8: each consumer warp's fp16 copy of its 16 V rows
   static constexpr int kStgWarpBytes = kFp8 ? 16 * D * 2 : 0;
   static constexpr int kStgOff = kQOff + kDecRows * kQStride;
   static constexpr int kRedOff = kStgOff + kDecConsumerWarps * kStgWarpBytes;  // merge buffers
   static constexpr int kRedBytes = kDecRows * D * 4 + kDecConsumerWarps * kDecRows * 4 * 3;
   static constexpr int kBarOff = kRedOff + kRedBytes;
-  static constexpr int kSmemBytes = kBarOff + 2 * kDecStages * 8 + 64 + 1024;
+  static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8 + 64 + 1024;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 struct DecodeSeg {
@@ -265,10 +269,10 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
     int win0 = -(1 << 30), win_val = 0;
     for (int t = a; t < e; ++t) {
       if (!sg.visible(t)) continue;  // no visible key: skipped by all roles
-      const int st = it % kDecStages;
-      if (it >= kDecStages) {
+      const int st = it % C::kStages;
+      if (it >= C::kStages) {
         bool ok = true;
-        if (lane == 0) ok = mbar_wait(&empty[st], ((it / kDecStages) - 1) & 1, abort, 31);
+        if (lane == 0) ok = mbar_wait(&empty[st], ((it / C::kStages) - 1) & 1, abort, 31);
         if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
           stop = true;  // abort: stop issuing, but still drain what is in flight
           break;
@@ -327,8 +331,8 @@ DEVI void decode_producer(const DecodeParams& p, const CUtensorMap* mk, const CU
   // the CTA exits
   if (lane == 0) {
     int zero = 0;
-    for (int i = max(0, it - kDecStages); i < it; ++i)
-      mbar_wait(&full[i % kDecStages], (i / kDecStages) & 1, &zero, 32);
+    for (int i = max(0, it - C::kStages); i < it; ++i)
+      mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1, &zero, 32);
   }
 }
 
@@ -436,12 +440,12 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
 
     for (int t = a; t < e; ++t) {
       if (!sg.visible(t)) continue;
-      const int st = it % kDecStages;
+      const int st = it % C::kStages;
       if ((it & 1) != wg || dead) {  // the other warpgroup's tile, or given up
         ++it;
         continue;
       }
-      if (!warp_wait(&full[st], (it / kDecStages) & 1, abort, 33)) {
+      if (!warp_wait(&full[st], (it / C::kStages) & 1, abort, 33)) {
         dead = true;
         ++it;
         continue;
@@ -673,11 +677,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* empty = full + kDecStages;
-  int* abort = reinterpret_cast<int*>(empty + kDecStages);
+  uint64_t* empty = full + C::kStages;
+  int* abort = reinterpret_cast<int*>(empty + C::kStages);
   __shared__ int s_bad;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kDecStages; ++i) {
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 4);
     }
