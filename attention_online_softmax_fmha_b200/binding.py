@@ -199,6 +199,16 @@ def _check(fn: str, status: int):
         raise AttnError(fn, status)
 
 
+def _keep_for(stream, *tensors):
+    """Buffers allocated here and used by work queued on another stream than
+    torch's current one are released only after that work (record_stream)."""
+    if stream is None or not hasattr(stream, "cuda_stream"):
+        return
+    for t in tensors:
+        if t is not None and t is not False:
+            t.record_stream(stream)
+
+
 def device_error(stream=None) -> int:
     """Read and clear the device error word (synchronises the stream)."""
     code = c_i32(0)
@@ -297,8 +307,7 @@ def fwd_varlen(q, k, v, *, stream=None, **kw):
     """Attention forward (attn_fwd_varlen). Returns (out, lse)."""
     a, out, lse = varlen_args(q, k, v, **kw)
     _check("attn_fwd_varlen", lib().attn_fwd_varlen(ctypes.byref(a), _stream(stream)))
-    if stream is not None and getattr(a, "_keep", None) is not None and hasattr(stream, "cuda_stream"):
-        a._keep.record_stream(stream)  # freed only after the work queued there
+    _keep_for(stream, getattr(a, "_keep", None))
     return out, lse
 
 
@@ -386,6 +395,7 @@ def fwd_paged_kvcache(q, k_cache, v_cache, block_table, cache_seqlens, *, stream
     a, out, lse, ws = paged_args(q, k_cache, v_cache, block_table, cache_seqlens, **kw)
     _check("attn_fwd_paged_kvcache", lib().attn_fwd_paged_kvcache(ctypes.byref(a),
                                                                  _stream(stream)))
+    _keep_for(stream, ws)
     return out, lse
 
 
@@ -487,6 +497,7 @@ def mla_fwd_paged(q, kv_cache, block_table, cache_seqlens, *, stream=None, **kw)
     """MLA-absorbed decode over a paged latent cache. Returns (out, lse)."""
     a, out, lse, ws = mla_args(q, kv_cache, block_table, cache_seqlens, **kw)
     _check("mla_fwd_paged", lib().mla_fwd_paged(ctypes.byref(a), _stream(stream)))
+    _keep_for(stream, ws)
     return out, lse
 
 
@@ -494,6 +505,7 @@ def mla_sparse_fwd(q, kv_cache, block_table, cache_seqlens, indices, *, stream=N
     """MLA decode over top-k index sets. Returns (out, lse)."""
     a, out, lse, ws = mla_args(q, kv_cache, block_table, cache_seqlens, indices=indices, **kw)
     _check("mla_sparse_fwd", lib().mla_sparse_fwd(ctypes.byref(a), _stream(stream)))
+    _keep_for(stream, ws)
     return out, lse
 
 
