@@ -8,10 +8,7 @@
 #include <cstdint>
 #include <cstring>
 
-#include <cstdlib>
-
 #include "host.cuh"
-#include "prefill2_sm100.cuh"
 #include "prefill_sm100.cuh"
 
 namespace attn {
@@ -40,53 +37,6 @@ attn_status_t launch_prefill(int grid, const CUtensorMap& mq, const CUtensorMap&
     return ATTN_ERR_CUDA;
   kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
   return launch_status(cudaGetLastError());
-}
-
-// The two-CTA kernel (bf16, D = 128, no mask): units of 512 rows, K and V
-// boxes of half a tile per CTA.
-attn_status_t launch_prefill2(int sms, const attn_varlen_args& a, const CUtensorMap& mq,
-                              PrefillParams p, cudaStream_t stream) {
-  const bool varlen = a.cu_seqlens_q != nullptr;
-  const uint64_t rows_k = varlen ? (uint64_t)a.total_k : (uint64_t)a.max_seqlen_k;
-  const uint64_t nb = varlen ? 1 : (uint64_t)a.batch;
-  const uint64_t ksb = varlen ? rows_k * a.k_stride_s : a.k_stride_b;
-  const uint64_t vsb = varlen ? rows_k * a.v_stride_s : a.v_stride_b;
-  CUtensorMap mk, mv;
-  if (!encode_4d(&mk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, a.num_heads_kv, rows_k, nb,
-                 a.k_stride_h, a.k_stride_s, ksb, 64, 1, 64, 1) ||
-      !encode_4d(&mv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 128, a.num_heads_kv, rows_k, nb,
-                 a.v_stride_h, a.v_stride_s, vsb, 64, 1, kPrefillBN, 1))
-    return ATTN_ERR_INVALID_ARG;
-  p.num_units_q = (a.max_seqlen_q + kP2Unit - 1) / kP2Unit;
-  const int64_t total = (int64_t)p.num_units_q * a.batch * a.num_heads_q;
-  if (total > INT32_MAX) return ATTN_ERR_UNSUPPORTED;
-  p.total_units = (int32_t)total;
-  const char* ue = std::getenv("ATTN_P2_UNION");
-  auto kernel = (ue && ue[0] == '1') ? prefill2_kernel<true> : prefill2_kernel<false>;
-  static std::atomic<uint64_t> configured{0};
-  const attn_status_t cst = configure_per_device(configured, [&]() -> attn_status_t {
-    for (auto kf : {prefill2_kernel<true>, prefill2_kernel<false>}) {
-      cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, kf) != cudaSuccess) return ATTN_ERR_CUDA;
-      if (fa.numRegs != kPrefillLaunchRegs) return ATTN_ERR_UNSUPPORTED;
-      const attn_status_t st = launch_status(set_smem(kf, kP2SmemBytes));
-      if (st != ATTN_OK) return st;
-    }
-    return ATTN_OK;
-  });
-  if (cst != ATTN_OK) return cst;
-  if (p.work_counter &&
-      cudaMemsetAsync(p.work_counter, 0, sizeof(int32_t), stream) != cudaSuccess)
-    return ATTN_ERR_CUDA;
-  const int clusters = (int)std::min<int64_t>(total, std::max(1, sms / 2));
-  kernel<<<2 * clusters, kPrefillThreads, kP2SmemBytes, stream>>>(mq, mk, mv, p);
-  return launch_status(cudaGetLastError());
-}
-
-// The one-CTA kernel only, for comparison runs (ATTN_PREFILL_ONE_CTA=1).
-bool prefill_one_cta_forced() {
-  const char* e = std::getenv("ATTN_PREFILL_ONE_CTA");
-  return e != nullptr && e[0] == '1';
 }
 
 template <int D, int kType>
@@ -152,9 +102,6 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
 
   const int sms = device_sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
-  if constexpr (D == 128 && kType == 0) {
-    if (!a.mask && !prefill_one_cta_forced()) return launch_prefill2(sms, a, mq, p, stream);
-  }
   const int grid = (int)std::min<int64_t>(total, sms);
   // The additive-mask path is a separate instantiation, so the common path
   // carries none of its registers.

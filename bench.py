@@ -72,8 +72,7 @@ def load_traffic():
 # The sources each kernel family is built from: its device code, its
 # launch code and the shared device and host helpers.
 _FAMILY_SOURCES = {
-    "prefill_kernel": ["prefill_sm100.cuh", "prefill2_sm100.cuh", "prefill_host.cuh"],
-    "prefill2_kernel": ["prefill_sm100.cuh", "prefill2_sm100.cuh", "prefill_host.cuh"],
+    "prefill_kernel": ["prefill_sm100.cuh", "prefill_host.cuh"],
     "decode_kernel": ["decode_paged.cuh", "sched.cuh", "combine.cuh", "api.cu"],
     "mla_kernel": ["mla_sm100.cuh", "sched.cuh", "combine.cuh", "api.cu"],
 }
@@ -230,9 +229,7 @@ def prefill_workload(name: str, seed: int, device):
            "head_dim": D, "causal": inp.causal, "window": list(inp.window),
            "sink": inp.sink is not None, "dtype": inp.dtype, "total_q_tokens": sum(inp.seqlens_q),
            "visible_pairs_per_head": pairs, "additive_mask": inp.mask is not None}
-    # bf16, D = 128 without a mask runs on CTA pairs (prefill2_kernel)
-    kernel = ("prefill2_kernel" if D == 128 and inp.dtype == "bf16" and inp.mask is None
-              else f"prefill_kernel<{D},{ {'bf16': 0, 'fp16': 1, 'e4m3': 2, 'e5m2': 3}[inp.dtype] }>")
+    kernel = f"prefill_kernel<{D},{ {'bf16': 0, 'fp16': 1, 'e4m3': 2, 'e5m2': 3}[inp.dtype] }>"
     return dict(step=step, e2e_step=e2e_step, work=flops / 1e12, unit="TFLOP/s", bound=bound,
                 kernel=kernel, launches_per_step=1, h2d=h2d, d2h=d2h, cfg=cfg,
                 dtype=inp.dtype, inp=inp, outputs=(out, lse),
