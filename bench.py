@@ -508,15 +508,18 @@ def run_ours(args, rank, world, device):
             torch.distributed.barrier()
         torch.cuda.synchronize()
         with ClockSampler(torch.cuda.current_device()) as clk:
-            # The timed region is milliseconds long, shorter than the sampling
-            # period: keep the GPU busy with the same step for a short window
-            # on both sides so the samples describe the clocks it ran at.
+            # Sampling runs through the warm-up and the timed steps. The timed
+            # region is milliseconds long, shorter than the sampling period, so
+            # the same step keeps the GPU busy for a short window right after
+            # it, and those samples describe the clocks under this load. The
+            # window comes after the timed steps, not before: a second of load
+            # ahead of them would put the GPU at its power cap for the timed
+            # steps, and the roofline divides by the burst peak.
             if args.clock_window > 0:
                 clk.wait_first(3.0)
-                load_for(wl["step"], stream, args.clock_window)
             times = time_steps(wl["step"], args.steps, args.warmup, stream, flush)
             if args.clock_window > 0:
-                load_for(wl["step"], stream, args.clock_window / 2)
+                load_for(wl["step"], stream, args.clock_window)
         torch.cuda.synchronize()
         if world > 1:
             torch.distributed.barrier()
