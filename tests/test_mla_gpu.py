@@ -314,3 +314,24 @@ def test_sparse_packed_tnd_queries(causal):
         assert_close_out(to_f64(out), ro, 1e-2)
         assert_close_lse(lse.cpu().numpy(), rl)
 
+
+
+def test_sparse_gathers_from_an_unevenly_strided_cache():
+    """A cache whose blocks are not one evenly strided list of rows (padding
+    after every block) takes the per-lane copy gathers instead of the TMA
+    row gathers; both give the oracle's result."""
+    inp = W.make_mla(seqlens=[20, 300, 3000], seqlen_q=2, num_heads_q=128, page_size=64,
+                     topk=256, seed=55, device="cuda")
+    inp.indices[1, 0, 0, 3] = 5000        # beyond the cache: skipped
+    nb, P = inp.kv_cache.shape[0], inp.kv_cache.shape[1]
+    blk = P * 576 + 64                    # 64 elements of padding after each block
+    store = torch.full((nb * blk,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    view = store.as_strided((nb, P, 1, 576), (blk, 576, 576, 1))
+    view.copy_(inp.kv_cache)
+    padded = W.MlaInputs(inp.q, view, inp.block_table, inp.cache_seqlens, inp.seqlens,
+                         inp.page_size, inp.num_heads_q, 512, False, inp.scale, inp.indices,
+                         inp.topk)
+    out_p, lse_p = run(padded, num_ctas=3)
+    out_c, lse_c = run(inp, num_ctas=3)
+    assert torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
+    check(inp, num_ctas=3)
