@@ -165,7 +165,8 @@ struct MlaBarriers {
   uint64_t kv_full[kMlaStages], kv_empty[kMlaStages];
   uint64_t vh_full[2], vh_empty[2];  // FP8: the fp16 copies of V
   uint64_t s_full[kMlaSBufs], p_full[2];
-  uint64_t xs_full[kMlaXsBufs];  // the other CTA's partial S tile has landed here
+  uint64_t xs_full[kMlaXsBufs];   // the other CTA's partial S tile has landed here
+  uint64_t xs_empty[kMlaXsBufs];  // the other CTA has read the tile this CTA sent it
   uint64_t o_full, o_empty;
   uint64_t mma_drain;
   uint32_t tmem_base;
@@ -656,10 +657,11 @@ DEVI void mla_convert(const MlaParams& p, uint8_t* smem, MlaBarriers* bars) {
 // to spread the banks) into the other CTA's buffer g % 2, completing on that
 // CTA's barrier, where each warp's leader has announced the warp's 4 KB. No
 // staging copy and no proxy fence: the receiver reads the buffer with plain
-// loads once the barrier's phase is complete. This CTA sends tile g only
-// after it has received the other CTA's tile g - 1, which the other CTA sent
-// after reading its tile g - 2 (the buffer's last use there), so the buffer
-// is free; and the barrier is at most one phase ahead of its waiter.
+// loads once the barrier's phase is complete, then releases it (one arrival
+// per warp, with release semantics, on this CTA's xs_empty), and this CTA
+// writes tile g into buffer g % 2 only after that release of tile g - 2.
+// Tile g is sent only after the other CTA's tile g - 1 has arrived, so the
+// full barrier is at most one phase ahead of its waiter.
 DEVI void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
                       uint32_t cluster_bar) {
   asm volatile(
@@ -677,6 +679,9 @@ DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint
   if (!warp_wait(&bars->s_full[sb], (g / kMlaSBufs) & 1, &bars->abort, 80)) return false;
   tc_fence_after();
   tmem_load<32>(tmem + kMlaTmemS + sb * kMlaBN + lane, sv);
+  if (g >= kMlaXsBufs &&
+      !warp_wait_cluster(&bars->xs_empty[b], ((g / kMlaXsBufs) - 1) & 1, &bars->abort, 84))
+    return false;
   const uint32_t bar = mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1);
   if ((threadIdx.x & 31) == 0) mbar_arrive_expect_tx_remote(bar, 32 * 128);
   const uint32_t dst = mapa_shared(smem_u32(smem + C::kXsOff + b * kMlaXsBytes + r * 128), rank ^ 1);
@@ -771,6 +776,11 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
           sv[4 * k + 2] = __float_as_uint(__uint_as_float(sv[4 * k + 2]) + __uint_as_float(v.z));
           sv[4 * k + 3] = __float_as_uint(__uint_as_float(sv[4 * k + 3]) + __uint_as_float(v.w));
         }
+        // This warp's rows of the buffer have been read: the other CTA may
+        // write its next tile there.
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0)
+          mbar_arrive_remote(mapa_shared(smem_u32(&bars->xs_empty[b]), rank ^ 1));
       }
       if (j + 1 < n && !mla_send_partial<kFp8>(bars, smem, tmem, lane, r, rank, gi + 1, sv_next))
         return;
@@ -994,8 +1004,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThrea
       mbar_init(&bars->vh_empty[i], 1);
     }
     for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->s_full[i], 1);
-    for (int i = 0; i < kMlaXsBufs; ++i)
-      mbar_init(&bars->xs_full[i], 4);  // one bulk copy from each softmax warp of the other CTA
+    for (int i = 0; i < kMlaXsBufs; ++i) {
+      mbar_init(&bars->xs_full[i], 4);   // each softmax warp of the other CTA: 4 KB
+      mbar_init(&bars->xs_empty[i], 4);  // each softmax warp of the other CTA has read
+    }
     for (int i = 0; i < 2; ++i) mbar_init(&bars->p_full[i], 128);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_empty, 128);

@@ -73,8 +73,8 @@ def load_traffic():
 # launch code and the shared device and host helpers.
 _FAMILY_SOURCES = {
     "prefill_kernel": ["prefill_sm100.cuh", "prefill_host.cuh"],
-    "decode_kernel": ["decode_paged.cuh", "sched.cuh", "combine.cuh", "api.cu"],
-    "mla_kernel": ["mla_sm100.cuh", "sched.cuh", "combine.cuh", "api.cu"],
+    "decode_kernel": ["decode_paged.cuh", "sched.cuh", "combine.cuh", "sched_host.cuh", "api.cu"],
+    "mla_kernel": ["mla_sm100.cuh", "sched.cuh", "combine.cuh", "sched_host.cuh", "mla_host.cuh"],
 }
 
 
