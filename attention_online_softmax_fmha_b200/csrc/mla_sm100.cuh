@@ -65,6 +65,9 @@ constexpr int kMlaSBufs = 3;       // S buffers in TMEM
 // leaves one tile less of slack for the loads.
 constexpr int kMlaSAhead = 3;
 static_assert(kMlaSAhead >= 2 && kMlaSAhead <= kMlaSBufs, "S lookahead");
+// The O barriers (one per S buffer) rely on S of tile g being issued after P V
+// of tile g - kMlaSBufs.
+static_assert(kMlaSAhead == kMlaSBufs, "O barrier phases");
 constexpr int kMlaXsBufs = 2;      // partial-S exchange buffers in shared memory
 constexpr int kGatherLag = 1;      // sparse: tiles of gathers in flight before a stage is signalled
 static_assert(kGatherLag < kMlaStages, "gather lag");
@@ -167,7 +170,11 @@ struct MlaBarriers {
   uint64_t s_full[kMlaSBufs], p_full[2];
   uint64_t xs_full[kMlaXsBufs];   // the other CTA's partial S tile has landed here
   uint64_t xs_empty[kMlaXsBufs];  // the other CTA has read the tile this CTA sent it
-  uint64_t o_full, o_empty;
+  // o_full[k]: P V of every tile g with g % 3 == k has completed. One barrier
+  // per S buffer: S of tile g is issued after P V of tile g - 3, so a waiter
+  // for P V of tile x knows P V of tile x - 3 (the same barrier's previous
+  // phase) is done, and the barrier is never two phases past the awaited one.
+  uint64_t o_full[kMlaSBufs], o_empty;
   uint64_t mma_drain;
   uint32_t tmem_base;
   int32_t abort;
@@ -560,7 +567,7 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
         tc_commit_w(&bars->vh_empty[gi & 1]);
       else
         tc_commit_w(&bars->kv_empty[sp]);
-      tc_commit_w(&bars->o_full);
+      tc_commit_w(&bars->o_full[gi % kMlaSBufs]);
       if (j + kMlaSAhead < n &&
           !mla_issue_s<kFp8>(bars, gi + kMlaSAhead, dq, dkv, tmem, nk, j + kMlaSAhead == n - 1))
         goto drain;
@@ -866,10 +873,11 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       }
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O may be rescaled once P V of the previous tile (global index
-        // gi - 1) has landed. o_full completes once per P V; P V gi - 2 has
-        // completed (S gi was issued after it) and P V gi is issued only after
-        // this tile's P, so the barrier is at most this one phase behind.
-        if (!warp_wait(&bars->o_full, (gi - 1) & 1, abort, 81)) return;
+        // gi - 1) has landed: phase (gi - 1) / 3 of o_full[(gi - 1) % 3]. Its
+        // previous phase (P V gi - 4) is done, since S gi was issued after P V
+        // gi - 3, and its next one needs P of tile gi + 2, not yet made.
+        const int pv = gi - 1;
+        if (!warp_wait(&bars->o_full[pv % kMlaSBufs], (pv / kMlaSBufs) & 1, abort, 81)) return;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < kMlaDvHalf; c += 32) {
@@ -919,8 +927,10 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       if (ns > 1) slot = p.meta[ml.seg_slot + s] + ((blockIdx.x >> 1) - p.meta[ml.seg_first + s]);
     }
     if (n > 0) {
-      // the segment's last P V (global index it + n - 1; it now counts it)
-      if (!warp_wait(&bars->o_full, (it - 1) & 1, abort, 82)) return;
+      // the segment's last P V (global index it + n - 1; it now counts it);
+      // its barrier's previous phase is done, as for the rescale
+      const int pv = it - 1;
+      if (!warp_wait(&bars->o_full[pv % kMlaSBufs], (pv / kMlaSBufs) & 1, abort, 82)) return;
       tc_fence_after();
     }
     if (!seen) l_run = l_rnd = 0.f;
@@ -1009,7 +1019,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThrea
       mbar_init(&bars->xs_empty[i], 4);  // each softmax warp of the other CTA has read
     }
     for (int i = 0; i < 2; ++i) mbar_init(&bars->p_full[i], 128);
-    mbar_init(&bars->o_full, 1);
+    for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->o_full[i], 1);
     mbar_init(&bars->o_empty, 128);
     mbar_init(&bars->mma_drain, 1);
     bars->abort = 0;
