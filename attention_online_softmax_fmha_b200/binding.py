@@ -24,7 +24,7 @@ c_i32, c_i64, c_f32, c_vp, c_sz = (ctypes.c_int32, ctypes.c_int64, ctypes.c_floa
 OK, INVALID_ARG, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA_ERROR, DEVICE_ERROR = range(6)
 DTYPE_BF16, DTYPE_FP16, DTYPE_E4M3, DTYPE_E5M2, DTYPE_FP32 = range(5)
 SCHED_MHA, SCHED_MLA, SCHED_MLA_SPARSE = range(3)
-DEVERR_TIMEOUT, DEVERR_META_MISMATCH, DEVERR_SMEM_ALIGN = 1, 2, 3
+DEVERR_TIMEOUT, DEVERR_META_MISMATCH, DEVERR_SMEM_ALIGN, DEVERR_UNITS_OVERFLOW = 1, 2, 3, 4
 SELFTEST_SITE = 200
 
 _TORCH_DTYPE = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16,

@@ -93,7 +93,8 @@ struct DecodeCfg {
   static constexpr int kStgWarpBytes = kFp8 ? 16 * D * 2 : 0;
   static constexpr int kStgOff = kQOff + kDecRows * kQStride;
   static constexpr int kRedOff = kStgOff + kDecConsumerWarps * kStgWarpBytes;  // merge buffers
-  static constexpr int kRedBytes = kDecRows * D * 4 + kDecConsumerWarps * kDecRows * 4 * 3;
+  // two O buffers (one per warpgroup), then m, l and the rounded l per warp
+  static constexpr int kRedBytes = 2 * kDecRows * D * 4 + kDecConsumerWarps * kDecRows * 4 * 3;
   static constexpr int kBarOff = kRedOff + kRedBytes;
   static constexpr int kSmemBytes = kBarOff + 2 * kStages * 8 + 64 + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -353,8 +354,8 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
   const int qr = lane >> 2;          // fragment row (and row + 8)
   const int qc = (lane & 3) * 2;     // fragment column pair
   uint8_t* qs = smem + C::kQOff;
-  float* red_o = reinterpret_cast<float*>(smem + C::kRedOff);  // [16][D]
-  float* red_m = red_o + kDecRows * D;                          // [8 warps][16]
+  float* red_o = reinterpret_cast<float*>(smem + C::kRedOff);  // [2 warpgroups][16][D]
+  float* red_m = red_o + 2 * kDecRows * D;                      // [8 warps][16]
   float* red_l = red_m + kDecConsumerWarps * kDecRows;
   float* red_r = red_l + kDecConsumerWarps * kDecRows;
   // After a failed wait (timeout or abort) a warp skips the rest of its tiles
@@ -586,7 +587,6 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
       red_m[gw * kDecRows + qr] = m_run[0];
       red_m[gw * kDecRows + qr + 8] = m_run[1];
     }
-    for (int x = tid; x < kDecRows * D; x += kDecConsumerThreads) red_o[x] = 0.f;
     named_barrier(1, kDecConsumerThreads);
     float scale_w[2];
 #pragma unroll
@@ -601,15 +601,35 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         red_r[gw * kDecRows + r] = l_rnd[h2] * scale_w[h2];
       }
     }
+    // O: the warps of each warpgroup add into that warpgroup's buffer one
+    // after another in warp order, then the second buffer is added to the
+    // first: a fixed order of the sums, so repeated runs agree bit for bit.
+    {
+      float* acc = red_o + wg * kDecRows * D;
+      for (int w = 0; w < 4; ++w) {
+        if (warp == w) {
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      const int c = n * 8 + qc;
-      atomicAdd(&red_o[qr * D + c], o[n][0] * scale_w[0]);
-      atomicAdd(&red_o[qr * D + c + 1], o[n][1] * scale_w[0]);
-      atomicAdd(&red_o[(qr + 8) * D + c], o[n][2] * scale_w[1]);
-      atomicAdd(&red_o[(qr + 8) * D + c + 1], o[n][3] * scale_w[1]);
+          for (int n = 0; n < D / 8; ++n) {
+            const int c = n * 8 + qc;
+            float2* r0 = reinterpret_cast<float2*>(&acc[qr * D + c]);
+            float2* r1 = reinterpret_cast<float2*>(&acc[(qr + 8) * D + c]);
+            float2 v0 = make_float2(o[n][0] * scale_w[0], o[n][1] * scale_w[0]);
+            float2 v1 = make_float2(o[n][2] * scale_w[1], o[n][3] * scale_w[1]);
+            if (w > 0) {
+              const float2 a0 = *r0, a1 = *r1;
+              v0.x += a0.x; v0.y += a0.y;
+              v1.x += a1.x; v1.y += a1.y;
+            }
+            *r0 = v0;
+            *r1 = v1;
+          }
+        }
+        named_barrier(1, kDecConsumerThreads);
+      }
+      for (int x = tid; x < kDecRows * D; x += kDecConsumerThreads)
+        red_o[x] += red_o[kDecRows * D + x];
+      named_barrier(1, kDecConsumerThreads);
     }
-    named_barrier(1, kDecConsumerThreads);
 
     // --- write: thread -> (row, 16 columns) --------------------------------
     {

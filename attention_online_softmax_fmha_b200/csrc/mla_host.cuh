@@ -66,33 +66,6 @@ size_t mla_ws_bytes(const DecodeShape& ds) {
          256;
 }
 
-// A 2-D (rows, cols) bf16 map with a one-row box of 64 columns and 128-byte
-// swizzle, for TMA 4-row gathers.
-bool encode_rows_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
-                    uint64_t row_stride_elems) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {row_stride_elems * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// Sparse bf16 MLA gathers whole cached rows with TMA when the cache is one
-// evenly strided list of rows: row (block * page + token) * H_kv + head at
-// a fixed stride. Returns that row count, or 0 (per-lane copies instead).
-int64_t mla_gather_rows(const mla_args& a) {
-  const int64_t H = a.num_heads_kv;
-  const int64_t R = H > 1 ? a.kv_stride_h : a.kv_stride_tok;  // elements per row
-  if (R < kMlaDqk || !stride_ok(R, 2)) return 0;
-  if (a.kv_stride_tok != H * R || a.kv_stride_blk != (int64_t)a.page_size * H * R) return 0;
-  const int64_t rows = (int64_t)a.num_blocks * a.page_size * H;
-  return rows < INT32_MAX ? rows : 0;
-}
-
 template <bool kSparse, bool kFp8>
 attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t stream) {
   using C = MlaCfg<kFp8>;
@@ -128,17 +101,6 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   p.cache_seqlens = a.cache_seqlens;
   p.indices = a.indices;
   p.meta = a.meta;
-  CUtensorMap mrows = mkv;  // unused unless the sparse gathers use TMA
-  p.gather_rows = 0;
-  if (kSparse && !kFp8) {
-    const int64_t rows = mla_gather_rows(a);
-    if (rows > 0) {
-      const int64_t R = a.num_heads_kv > 1 ? a.kv_stride_h : a.kv_stride_tok;
-      if (!encode_rows_2d(&mrows, a.kv_cache, kMlaDqk, (uint64_t)rows, (uint64_t)R))
-        return ATTN_ERR_INVALID_ARG;
-      p.gather_rows = (int32_t)rows;
-    }
-  }
   p.kv = a.kv_cache;
   p.q_descale = a.q_descale;
   p.k_descale = a.k_descale;
@@ -189,7 +151,7 @@ attn_status_t run_mla(const mla_args& a, const DecodeShape& ds, cudaStream_t str
   if (cst != ATTN_OK) return cst;
   // Clusters of two CTAs (the kernel's __cluster_dims__): one per segment, or
   // one per metadata slot.
-  kernel<<<2 * (a.meta ? ds.G : ds.S), C::kThreads, C::kSmemBytes, stream>>>(mq, mkv, mrows, p);
+  kernel<<<2 * (a.meta ? ds.G : ds.S), C::kThreads, C::kSmemBytes, stream>>>(mq, mkv, p);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   if (a.meta) {
     const int64_t warps = (int64_t)ds.S * 2 * kMlaRows;

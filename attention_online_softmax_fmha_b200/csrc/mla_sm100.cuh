@@ -15,9 +15,9 @@
 // dimensions of its V half (rank 0: nope 0..255 and the 64 rope dimensions,
 // rank 1: nope 256..511) of Q and of every key, computes the partial scores
 // S_r = Q_r K_r^T on its tensor core, and the two halves swap partials through
-// distributed shared memory (asynchronous remote stores, st.async, into the
-// other CTA, completing on its barrier), so both see S = S_0 + S_1 (the same
-// sum in the same order: identical P). Each CTA then accumulates O for its 256 V columns
+// distributed shared memory (one bulk copy per warp into the other CTA,
+// completing on its barrier), so both see S = S_0 + S_1 (the same sum in the
+// same order: identical P). Each CTA then accumulates O for its 256 V columns
 // (its first four 64-column chunks). Half of Q and of each key row per CTA
 // leaves room for a four-stage key ring, and the cache is read once per row
 // tile instead of once per V half.
@@ -34,10 +34,7 @@
 //   warps 0-3  softmax: thread r owns query row r (= TMEM lane r).
 //   warp 4     producer: Q tile (TMA, resident), key tiles of 32 keys into a
 //              4-stage ring: dense by TMA boxes through the block table;
-//              sparse (bf16, cache rows evenly strided) by TMA 4-row gathers
-//              (tile::gather4) over a (row, 576) view of the cache, a skipped
-//              entry reading row 0, whose V half the softmax then zeroes;
-//              otherwise by per-lane 16-byte async copies of the gathered rows
+//              sparse by per-lane 16-byte async copies of the gathered rows
 //              (each lane one key, zeros for skipped keys), completed and
 //              fenced before the stage is handed over.
 //   warp 5     TMEM owner and MMA issuer (whole warp, one elected lane):
@@ -88,8 +85,9 @@ struct MlaCfg {
   static constexpr int kQBytes = kMaxChunks * kMlaQChunkBytes;
   static constexpr int kKVBytes = kMaxChunks * kMlaKVChunkBytes;
   static constexpr int kQOff = 0;
-  static constexpr int kXsOff = kQOff + kQBytes;  // the other CTA's partial S lands here
-  static constexpr int kKVOff = kXsOff + kMlaXsBufs * kMlaXsBytes;
+  static constexpr int kXsOff = kQOff + kQBytes;                      // partial S received here
+  static constexpr int kXoOff = kXsOff + kMlaXsBufs * kMlaXsBytes;    // and staged here to send
+  static constexpr int kKVOff = kXoOff + kMlaXsBufs * kMlaXsBytes;
   static constexpr int kVHStages = kFp8 ? 2 : 0;
   static constexpr int kVHBytes = 4 * kMlaKVChunkBytes;  // fp16 V half: 4 chunks of 64 columns
   static constexpr int kVHOff = kKVOff + kMlaStages * kKVBytes;
@@ -152,7 +150,6 @@ struct MlaParams {
   // cu_q[b] <= t < cu_q[b + 1] (batch_kv sequences). nullptr: BSND.
   const int32_t* cu_q;
   int32_t batch_kv;
-  int32_t gather_rows;      // sparse, bf16: rows of the (row, 576) view for TMA gathers, 0: copies
   int32_t sbs;              // sparse: positions per index (sparse_block_size, >= 1)
   int32_t sbs_log2;         // log2(sbs) (sbs is a power of two)
   int32_t tiles_per_token;  // group >= 128: group / 128 (else 1)
@@ -168,8 +165,7 @@ struct MlaBarriers {
   uint64_t kv_full[kMlaStages], kv_empty[kMlaStages];
   uint64_t vh_full[2], vh_empty[2];  // FP8: the fp16 copies of V
   uint64_t s_full[kMlaSBufs], p_full[2];
-  uint64_t xs_full[kMlaXsBufs];   // the other CTA's partial S tile has landed here
-  uint64_t xs_empty[kMlaXsBufs];  // the other CTA has read the tile this CTA sent it
+  uint64_t xs_full[kMlaXsBufs];  // the other CTA's partial S tile has landed here
   // o_full[k]: P V of every tile g with g % 3 == k has completed. One barrier
   // per S buffer: S of tile g is issued after P V of tile g - 3, so a waiter
   // for P V of tile x knows P V of tile x - 3 (the same barrier's previous
@@ -272,21 +268,9 @@ DEVI void mla_range(const MlaParams& p, int& ub, int& ue, int& s0, const int32_t
 // ---------------------------------------------------------------------------
 // Producer warp
 // ---------------------------------------------------------------------------
-// Four rows (y0..y3) of a 2-D tensor map, columns [x, x + box), into four
-// consecutive 128-byte rows of shared memory (no multicast).
-DEVI void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y0, int y1,
-                      int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
-      "r"(smem_u32(bar))
-      : "memory");
-}
-
 template <bool kSparse, bool kFp8>
 DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensorMap* mkv,
-                       const CUtensorMap* mrows, uint8_t* smem, MlaBarriers* bars, int rank) {
+                       uint8_t* smem, MlaBarriers* bars, int rank) {
   using C = MlaCfg<kFp8>;
   constexpr int kEsize = kFp8 ? 1 : 2;
   volatile int* abort = &bars->abort;
@@ -396,23 +380,6 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
           pos = mla_sparse_pos(p, g.b, g.kvg, g.tok0, t * kMlaBN + lane);
         }
         const bool valid = pos >= 0 && pos < g.len;
-        if (p.gather_rows > 0) {
-          // Row of the (row, 576) view: (block * page + row in page) * H_kv + KV head.
-          const int row = valid ? ((bt[pos / P] * P + pos % P) * p.heads_kv + g.kvg) : 0;
-          if (lane == 0) mbar_expect_tx(&bars->kv_full[st], nch * kMlaBN * 128);
-#pragma unroll
-          for (int q4 = 0; q4 < kMlaBN / 4; ++q4) {
-            const int r0 = __shfl_sync(0xffffffffu, row, 4 * q4);
-            const int r1 = __shfl_sync(0xffffffffu, row, 4 * q4 + 1);
-            const int r2 = __shfl_sync(0xffffffffu, row, 4 * q4 + 2);
-            const int r3 = __shfl_sync(0xffffffffu, row, 4 * q4 + 3);
-            if (lane == 0)
-              for (int c = 0; c < nch; ++c)
-                tma_gather4(dst + c * kMlaKVChunkBytes + 4 * q4 * 128, mrows, &bars->kv_full[st],
-                            mla_col<kFp8>(rank, c), r0, r1, r2, r3);
-          }
-          continue;
-        }
         const uint8_t* src = nullptr;  // the cached row, in bytes
         if (valid)
           src = static_cast<const uint8_t*>(p.kv) +
@@ -452,7 +419,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
     u = min(ue, se);
     ++s;
   }
-  if (!kSparse || p.gather_rows > 0) {
+  if constexpr (!kSparse) {
     if (lane == 0) {  // the last stages' copies must land before the CTA exits
       int zero = 0;
       for (int i = max(0, it - kMlaStages); i < it; ++i)
@@ -659,25 +626,12 @@ DEVI void mla_convert(const MlaParams& p, uint8_t* smem, MlaBarriers* bars) {
 // Softmax warpgroup
 // ---------------------------------------------------------------------------
 // Loads this CTA's partial scores of the tile with global index g into sv
-// and sends them to the other CTA of the cluster: each thread stores its row
-// with asynchronous remote stores (st.async, 16-byte pieces permuted by row
-// to spread the banks) into the other CTA's buffer g % 2, completing on that
-// CTA's barrier, where each warp's leader has announced the warp's 4 KB. No
-// staging copy and no proxy fence: the receiver reads the buffer with plain
-// loads once the barrier's phase is complete, then releases it (one arrival
-// per warp, with release semantics, on this CTA's xs_empty), and this CTA
-// writes tile g into buffer g % 2 only after that release of tile g - 2.
-// Tile g is sent only after the other CTA's tile g - 1 has arrived, so the
-// full barrier is at most one phase ahead of its waiter.
-DEVI void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                      uint32_t cluster_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::
-          "r"(cluster_addr),
-      "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
-      : "memory");
-}
-
+// and sends them to the other CTA of the cluster: 16-byte pieces permuted by
+// row (to spread the banks) into its buffer g % 2, then one arrival per row
+// on its barrier. This CTA sends tile g only after it has received the other
+// CTA's tile g - 1, which the other CTA sent after reading its tile g - 2
+// (the buffer's last use there), so the buffer is free; and the barrier is at
+// most one phase ahead of its waiter.
 template <bool kFp8>
 DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint32_t lane, int r,
                            int rank, int g, uint32_t* sv) {
@@ -686,16 +640,29 @@ DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint
   if (!warp_wait(&bars->s_full[sb], (g / kMlaSBufs) & 1, &bars->abort, 80)) return false;
   tc_fence_after();
   tmem_load<32>(tmem + kMlaTmemS + sb * kMlaBN + lane, sv);
-  if (g >= kMlaXsBufs &&
-      !warp_wait_cluster(&bars->xs_empty[b], ((g / kMlaXsBufs) - 1) & 1, &bars->abort, 84))
-    return false;
-  const uint32_t bar = mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1);
-  if ((threadIdx.x & 31) == 0) mbar_arrive_expect_tx_remote(bar, 32 * 128);
-  const uint32_t dst = mapa_shared(smem_u32(smem + C::kXsOff + b * kMlaXsBytes + r * 128), rank ^ 1);
+  // Stage this warp's 32 rows (16-byte pieces permuted by row to spread the
+  // banks) and send them with one bulk copy into the other CTA's buffer b,
+  // completing on its barrier. Staging buffer b was last the source of the
+  // copy two tiles ago: that copy must have read it.
+  const int warp_row0 = r & ~31;
+  const bool leader = (threadIdx.x & 31) == 0;
+  if (leader) bulk_wait_read<1>();
+  __syncwarp();
+  uint8_t* stage = smem + C::kXoOff + b * kMlaXsBytes + r * 128;
 #pragma unroll
   for (int k = 0; k < 8; ++k)
-    st_async_v4(dst + ((k ^ (r & 7)) << 4), sv[4 * k], sv[4 * k + 1], sv[4 * k + 2], sv[4 * k + 3],
-                bar);
+    *reinterpret_cast<uint4*>(stage + ((k ^ (r & 7)) << 4)) =
+        make_uint4(sv[4 * k], sv[4 * k + 1], sv[4 * k + 2], sv[4 * k + 3]);
+  fence_proxy_async_smem();  // the copy reads through the async proxy
+  __syncwarp();
+  if (leader) {
+    const uint32_t bar = mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1);
+    const uint32_t off = b * kMlaXsBytes + warp_row0 * 128;
+    mbar_arrive_expect_tx_remote(bar, 32 * 128);
+    bulk_copy_to_cluster(mapa_shared(smem_u32(smem + C::kXsOff + off), rank ^ 1),
+                         smem_u32(smem + C::kXoOff + off), 32 * 128, bar);
+    bulk_commit();
+  }
   return true;
 }
 
@@ -783,11 +750,6 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
           sv[4 * k + 2] = __float_as_uint(__uint_as_float(sv[4 * k + 2]) + __uint_as_float(v.z));
           sv[4 * k + 3] = __float_as_uint(__uint_as_float(sv[4 * k + 3]) + __uint_as_float(v.w));
         }
-        // This warp's rows of the buffer have been read: the other CTA may
-        // write its next tile there.
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0)
-          mbar_arrive_remote(mapa_shared(smem_u32(&bars->xs_empty[b]), rank ^ 1));
       }
       if (j + 1 < n && !mla_send_partial<kFp8>(bars, smem, tmem, lane, r, rank, gi + 1, sv_next))
         return;
@@ -814,24 +776,6 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
               pos = k >= 0 ? (k << p.sbs_log2) + (e & (p.sbs - 1)) : -1;
             }
             if (!(pos >= 0 && pos <= hi)) sv[c] = __float_as_uint(-INFINITY);
-          }
-        }
-        if (!kFp8 && p.gather_rows > 0) {
-          // Skipped entries were gathered from row 0 of the cache, whatever it
-          // holds: zero their V half so P = 0 never meets a NaN there. Key r
-          // of the tile by thread r; every row of the tile is token tok0.
-          if (r < kMlaBN) {
-            const int pos = mla_sparse_pos(p, g.b, g.kvg, g.tok0, t * kMlaBN + r);
-            if (!(pos >= 0 && pos < g.len)) {
-              uint8_t* krow = smem + C::kKVOff + (gi % kMlaStages) * C::kKVBytes + r * 128;
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-#pragma unroll
-                for (int x = 0; x < 8; ++x)
-                  *reinterpret_cast<uint4*>(krow + c * kMlaKVChunkBytes + x * 16) =
-                      make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
           }
         }
       } else {
@@ -988,7 +932,7 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
 template <bool kSparse, bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThreads, 1)
     mla_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
-               const __grid_constant__ CUtensorMap map_rows, const MlaParams p) {
+               const MlaParams p) {
   using C = MlaCfg<kFp8>;
   // 128-byte swizzled TMA tiles need 1024-byte aligned shared memory; both
   // CTAs of the cluster share the layout, so both leave here or neither.
@@ -1004,8 +948,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThrea
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
     for (int i = 0; i < kMlaStages; ++i) {
-      // sparse copies: one arrival per producer lane; TMA: the expect_tx arrival
-      mbar_init(&bars->kv_full[i], (kSparse && p.gather_rows == 0) ? 32 : 1);
+      mbar_init(&bars->kv_full[i], kSparse ? 32 : 1);
       // e4m3: released by the S MMA's commit and the 64 conversion threads
       mbar_init(&bars->kv_empty[i], kFp8 ? 1 + 64 : 1);
     }
@@ -1014,10 +957,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThrea
       mbar_init(&bars->vh_empty[i], 1);
     }
     for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->s_full[i], 1);
-    for (int i = 0; i < kMlaXsBufs; ++i) {
-      mbar_init(&bars->xs_full[i], 4);   // each softmax warp of the other CTA: 4 KB
-      mbar_init(&bars->xs_empty[i], 4);  // each softmax warp of the other CTA has read
-    }
+    for (int i = 0; i < kMlaXsBufs; ++i)
+      mbar_init(&bars->xs_full[i], 4);  // one bulk copy from each softmax warp of the other CTA
     for (int i = 0; i < 2; ++i) mbar_init(&bars->p_full[i], 128);
     for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->o_full[i], 1);
     mbar_init(&bars->o_empty, 128);
@@ -1053,12 +994,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThrea
     if (warp < 4)
       mla_softmax<kSparse, kFp8>(p, smem, bars, tmem, rank);
     else if (warp == 4)
-      mla_producer<kSparse, kFp8>(p, &map_q, &map_kv, &map_rows, smem, bars, rank);
+      mla_producer<kSparse, kFp8>(p, &map_q, &map_kv, smem, bars, rank);
     else if (warp == 5)
       mla_mma<kSparse, kFp8>(p, smem, bars, tmem, rank);
     else if constexpr (kFp8)
       mla_convert<kSparse>(p, smem, bars);
   }
+  // The partial-score copies this CTA sent have landed in the other CTA.
+  if (warp < 4 && (threadIdx.x & 31) == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   // No remote arrival or store into this CTA's shared memory after this.

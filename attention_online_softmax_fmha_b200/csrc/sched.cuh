@@ -68,7 +68,7 @@ struct SchedShape {
 // last (partial) tile.
 DEVI int32_t sched_units(const SchedShape& sh, int32_t len) {
   if (sh.mode == ATTN_SCHED_MLA_SPARSE) return (sh.topk + sh.unit_keys - 1) / sh.unit_keys;
-  const int32_t cached = len > 0 ? (len + sh.unit_keys - 1) / sh.unit_keys : 0;
+  const int32_t cached = len > 0 ? (len - 1) / sh.unit_keys + 1 : 0;  // no overflow at 2^31 - 1
   return cached + (sh.new_keys + sh.unit_keys - 1) / sh.unit_keys;
 }
 
@@ -124,12 +124,28 @@ __global__ void __launch_bounds__(1024, 1) sched_kernel(const SchedParams p) {
   int32_t* seg_slot = p.meta + ml.seg_slot;
   const int tid = threadIdx.x;
 
-  // 1. units per segment, then their exclusive prefix sums
+  // 1. units per segment, then their exclusive prefix sums. The sums are
+  //    int32: a problem with more units than that is refused (an invalid
+  //    header, which the main kernels reject, and a device error).
+  __shared__ unsigned long long sh_units;
+  if (tid == 0) sh_units = 0;
+  __syncthreads();
+  unsigned long long mine = 0;
   for (int s = tid; s < p.S; s += blockDim.x) {
     const int b = s / p.sh.segs_per_seq;
-    seg_begin[s] = sched_units(p.sh, p.cache_seqlens[b]);
+    const int32_t n = sched_units(p.sh, p.cache_seqlens[b]);
+    seg_begin[s] = n;
+    mine += (unsigned long long)max(n, 0);
   }
+  atomicAdd(&sh_units, mine);
   __syncthreads();
+  if (sh_units > (unsigned long long)INT32_MAX) {
+    if (tid == 0) {
+      p.meta[kMetaMagic] = 0;
+      raise_error(ATTN_DEVERR_UNITS_OVERFLOW, 50);
+    }
+    return;
+  }
   int32_t total;
   block_exclusive_scan(seg_begin, p.S, sh_warp, total);
   if (tid == 0) seg_begin[p.S] = total;

@@ -70,7 +70,11 @@ enum {
   ATTN_DEVERR_NONE = 0,
   ATTN_DEVERR_TIMEOUT = 1,        /* a bounded pipeline wait gave up            */
   ATTN_DEVERR_META_MISMATCH = 2,  /* scheduler metadata built for other args    */
-  ATTN_DEVERR_SMEM_ALIGN = 3      /* dynamic shared memory not 1024-byte aligned */
+  ATTN_DEVERR_SMEM_ALIGN = 3,     /* dynamic shared memory not 1024-byte aligned */
+  ATTN_DEVERR_UNITS_OVERFLOW = 4  /* attn_sched_metadata: total work units of the
+                                     problem above 2^31 - 1 (the metadata is left
+                                     invalid, so the main call raises
+                                     ATTN_DEVERR_META_MISMATCH if this word is clear) */
 };
 
 typedef enum {
@@ -183,6 +187,11 @@ attn_status_t attn_fwd_varlen(const attn_varlen_args* args, void* stream);
 /* num_ctas = 0 picks the device's SM count. The MLA modes schedule over     */
 /* clusters of two CTAs: their slots number max(1, num_ctas / 2), and the    */
 /* MLA kernels launch two CTAs per slot.                                     */
+/* Limits: batch x segments per sequence at most 2^24 (ATTN_ERR_UNSUPPORTED  */
+/* on the host); the problem's total units (keys in tiles of 64 for GQA,     */
+/* 32 for MLA, per segment) at most 2^31 - 1, checked on the device:         */
+/* above it the header is left invalid and ATTN_DEVERR_UNITS_OVERFLOW is     */
+/* raised.                                                                   */
 /* ------------------------------------------------------------------------ */
 enum { ATTN_SCHED_MHA = 0, ATTN_SCHED_MLA = 1, ATTN_SCHED_MLA_SPARSE = 2 };
 

@@ -258,3 +258,37 @@ def test_combine_against_oracle(with_counts):
                                 sink.double().numpy()[None, :])
         assert_close_out(o[b], ro, 1e-2)
         assert_close_lse(l[b], rl.T)
+
+
+def test_unit_count_overflow_is_reported():
+    """Sixteen sequences of 2^31 - 1 cached keys and eight KV heads: 128
+    segments of 2^25 tiles each, 2^32 units in all, past the int32 prefix
+    sums. Only the scheduler runs (it reads cache_seqlens alone); it leaves
+    the header invalid and raises the overflow code."""
+    lens = torch.full((16,), 2**31 - 1, dtype=torch.int32, device="cuda")
+    meta = B.sched_metadata(lens, batch=16, seqlen_q=1, num_heads_q=8, num_heads_kv=8,
+                            head_dim_qk=128, head_dim_v=128, page_size=64, num_ctas=5)
+    torch.cuda.synchronize()
+    word = B.device_error()
+    assert word & 0xff == B.DEVERR_UNITS_OVERFLOW and word >> 8 == 50, hex(word)
+    assert int(meta[0]) == 0  # no valid magic: a main call would refuse it
+    # below the limit: seven sequences, 56 segments, 56 * 2^25 < 2^31
+    meta = B.sched_metadata(lens[:7], batch=7, seqlen_q=1, num_heads_q=8, num_heads_kv=8,
+                            head_dim_qk=128, head_dim_v=128, page_size=64, num_ctas=5)
+    torch.cuda.synchronize()
+    assert B.device_error() == 0
+    assert int(meta[0]) != 0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_repeated_runs_are_bitwise_identical(dtype):
+    """The split and every sum's order are fixed by the metadata, so repeated
+    runs agree bit for bit; a race between the producer and the two consumer
+    warpgroups shows up as a difference."""
+    inp = W.make_paged(seqlens=[1, 63, 64, 65, 700, 3000, 9000], seqlen_q=1, num_heads_q=32,
+                       num_heads_kv=8, head_dim=128, page_size=64, sink=True, dtype=dtype,
+                       seed=93, device="cuda")
+    ref_o, ref_l, _ = run_paged(inp, num_ctas=11)
+    for _ in range(15):
+        o, l, _ = run_paged(inp, num_ctas=11)
+        assert torch.equal(o, ref_o) and torch.equal(l, ref_l)

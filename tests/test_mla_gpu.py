@@ -317,9 +317,9 @@ def test_sparse_packed_tnd_queries(causal):
 
 
 def test_sparse_gathers_from_an_unevenly_strided_cache():
-    """A cache whose blocks are not one evenly strided list of rows (padding
-    after every block) takes the per-lane copy gathers instead of the TMA
-    row gathers; both give the oracle's result."""
+    """A cache with NaN padding after every block (block stride above
+    page_size x 576) gives bit for bit the packed cache's result: the sparse
+    gathers follow the block stride and never read the padding."""
     inp = W.make_mla(seqlens=[20, 300, 3000], seqlen_q=2, num_heads_q=128, page_size=64,
                      topk=256, seed=55, device="cuda")
     inp.indices[1, 0, 0, 3] = 5000        # beyond the cache: skipped
@@ -334,4 +334,24 @@ def test_sparse_gathers_from_an_unevenly_strided_cache():
     out_p, lse_p = run(padded, num_ctas=3)
     out_c, lse_c = run(inp, num_ctas=3)
     assert torch.equal(out_p, out_c) and torch.equal(lse_p, lse_c)
+    check(inp, num_ctas=3)
+
+
+@pytest.mark.parametrize("dtype,topk", [("e4m3", 256), ("bf16", 256), ("e4m3", 0), ("bf16", 0)])
+def test_repeated_runs_are_bitwise_identical(dtype, topk):
+    """The kernels are deterministic (fixed split, fixed order of every sum),
+    so repeated runs must agree bit for bit; a race between the roles (a
+    stage, an exchange buffer or the O accumulator read too early) shows up as
+    a difference. 24 runs each without metadata and with 3 clusters; the first
+    run is checked against the oracle."""
+    inp = W.make_mla(seqlens=[20, 300, 3000], seqlen_q=2, num_heads_q=128, page_size=64,
+                     topk=topk, dtype=dtype, seed=56, device="cuda")
+    if topk:
+        inp.indices[0, 1, 0, 5] = 19999
+        inp.indices[2, 0, 0, 7] = -5
+    for kw in (dict(use_meta=False), dict(num_ctas=3)):
+        ref_o, ref_l = run(inp, **kw)
+        for _ in range(23):
+            o, l = run(inp, **kw)
+            assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
     check(inp, num_ctas=3)
