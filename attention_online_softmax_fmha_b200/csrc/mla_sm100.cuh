@@ -18,9 +18,9 @@
 // distributed shared memory (one bulk copy per warp into the other CTA,
 // completing on its barrier), so both see S = S_0 + S_1 (the same sum in the
 // same order: identical P). Each CTA then accumulates O for its 256 V columns
-// (its first four 64-column chunks). Half of Q and of each key row per CTA
-// leaves room for a four-stage key ring, and the cache is read once per row
-// tile instead of once per V half.
+// (its first four 64-column chunks). Q sits in TMEM (the S MMAs read A from
+// there), which leaves shared memory for a deep key ring, and the cache is
+// read once per row tile instead of once per V half.
 //   dense : segment = (sequence, KV head, row tile), keys 0 .. L-1 in tiles of 32
 //           (causal: key j visible to token i iff j <= i + L - s_q).
 //   sparse: segment = (sequence, KV head, token, head tile), keys = that token's
@@ -30,17 +30,22 @@
 // Segments are split over persistent clusters by the scheduler metadata (a
 // metadata "CTA" is a cluster); split segments go through the combine kernel.
 //
-// Roles (192 threads per CTA):
-//   warps 0-3  softmax: thread r owns query row r (= TMEM lane r).
-//   warp 4     producer: Q tile (TMA, resident), key tiles of 32 keys into a
-//              4-stage ring: dense by TMA boxes through the block table;
-//              sparse by per-lane 16-byte async copies of the gathered rows
-//              (each lane one key, zeros for skipped keys), completed and
-//              fenced before the stage is handed over.
-//   warp 5     TMEM owner and MMA issuer (whole warp, one elected lane):
-//              S_j = Q K_j^T (M=128, N=32) into one of three TMEM S buffers
-//              (issued three tiles ahead); O += P_j V_j (M=128, N=256, K=32)
-//              with P from TMEM.
+// Roles (320 threads per CTA; e4m3 rows 384):
+//   warps 0-3  softmax: thread r owns query row r (= TMEM lane r). Adds the
+//              other CTA's partial scores to its own, writes P over S.
+//   warp 4     producer: Q chunks (TMA) through two staging buffers, key
+//              tiles of 32 keys into a 6-stage (e4m3: 8-stage) ring: dense by
+//              TMA boxes through the block table; sparse by per-lane 16-byte
+//              async copies of the gathered rows (each lane one key, zeros for
+//              skipped keys), completed and fenced before the stage is handed
+//              over.
+//   warp 5     TMEM owner and MMA issuer (whole warp, one elected lane): Q
+//              chunks into TMEM (tcgen05.cp); S_j = Q K_j^T (M=128, N=32, A
+//              from TMEM) into one of three TMEM S buffers (issued three tiles
+//              ahead); O += P_j V_j (M=128, N=256, K=32) with P from TMEM.
+//   warps 6-7  e4m3 rows only: the fp16 copy of each tile's V half.
+//   last 4     sender: loads each S tile and sends it to the other CTA, so
+//              the softmax never waits on the exchange's copy.
 #pragma once
 
 #include "combine.cuh"
@@ -54,7 +59,7 @@ constexpr int kMlaDv = 512;
 constexpr int kMlaDvHalf = 256;
 constexpr int kMlaBN = 32;         // keys per tile
 constexpr int kMlaRows = 128;      // query rows per row tile
-constexpr int kMlaStages = 4;
+constexpr int kMlaMaxStages = 8;  // key stages of the deepest ring (MlaCfg::kStages)
 constexpr int kMlaSBufs = 3;       // S buffers in TMEM
 // S of tile g + kMlaSAhead is issued after P V of tile g. The softmax needs
 // S one tile ahead (it sends tile g + 1's partials before finishing tile g),
@@ -67,13 +72,14 @@ static_assert(kMlaSAhead >= 2 && kMlaSAhead <= kMlaSBufs, "S lookahead");
 static_assert(kMlaSAhead == kMlaSBufs, "O barrier phases");
 constexpr int kMlaXsBufs = 2;      // partial-S exchange buffers in shared memory
 constexpr int kGatherLag = 1;      // sparse: tiles of gathers in flight before a stage is signalled
-static_assert(kGatherLag < kMlaStages, "gather lag");
 constexpr int kMlaQChunkBytes = kMlaRows * 128;                // 16 KB
 constexpr int kMlaKVChunkBytes = kMlaBN * 128;                 // 4 KB
 constexpr int kMlaXsBytes = kMlaRows * kMlaBN * 4;             // one partial S tile, 16 KB
 constexpr uint32_t kMlaTmemCols = 512;
 constexpr uint32_t kMlaTmemS = 0;      // three S buffers of 32 columns
+constexpr uint32_t kMlaTmemQ = 96;     // Q: 32 columns per 128-byte chunk, 5 chunks at most
 constexpr uint32_t kMlaTmemO = 256;    // 256 columns of O
+constexpr int kMlaQStages = 2;         // Q staging buffers of one chunk (128 rows x 128 bytes)
 
 // Shared-memory layout of the bf16 (kFp8 = false) and the e4m3 kernel. A
 // chunk is one 128-byte column of a TMA box: 64 bf16 or 128 e4m3 values.
@@ -82,19 +88,25 @@ constexpr uint32_t kMlaTmemO = 256;    // 256 columns of O
 template <bool kFp8>
 struct MlaCfg {
   static constexpr int kMaxChunks = kFp8 ? 3 : 5;          // chunks per CTA (rank 0)
-  static constexpr int kQBytes = kMaxChunks * kMlaQChunkBytes;
   static constexpr int kKVBytes = kMaxChunks * kMlaKVChunkBytes;
-  static constexpr int kQOff = 0;
-  static constexpr int kXsOff = kQOff + kQBytes;                      // partial S received here
-  static constexpr int kXoOff = kXsOff + kMlaXsBufs * kMlaXsBytes;    // and staged here to send
+  // Q passes through two one-chunk staging buffers into TMEM, where the S
+  // MMAs read it; the shared memory this frees holds more key stages.
+  static constexpr int kQSOff = 0;
+  static constexpr int kXsOff = kQSOff + kMlaQStages * kMlaQChunkBytes;  // partial S received here
+  static constexpr int kXoOff = kXsOff + kMlaXsBufs * kMlaXsBytes;       // and staged here to send
   static constexpr int kKVOff = kXoOff + kMlaXsBufs * kMlaXsBytes;
+  static constexpr int kStages = kFp8 ? 8 : 6;
   static constexpr int kVHStages = kFp8 ? 2 : 0;
   static constexpr int kVHBytes = 4 * kMlaKVChunkBytes;  // fp16 V half: 4 chunks of 64 columns
-  static constexpr int kVHOff = kKVOff + kMlaStages * kKVBytes;
+  static constexpr int kVHOff = kKVOff + kStages * kKVBytes;
   static constexpr int kBarOff = kVHOff + kVHStages * kVHBytes;
-  static constexpr int kSmemBytes = kBarOff + 256;
-  static constexpr int kThreads = kFp8 ? 256 : 192;  // + two conversion warps
+  static constexpr int kSmemBytes = kBarOff + 512;
+  // softmax 0-3, producer 4, MMA 5, (e4m3: conversion 6-7), sender warpgroup
+  static constexpr int kSendWarp0 = kFp8 ? 8 : 6;
+  static constexpr int kThreads = (kSendWarp0 + 4) * 32;
+  static_assert(kStages <= kMlaMaxStages && kGatherLag < kStages, "key ring");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  static_assert(kMlaTmemQ + 32 * kMaxChunks <= kMlaTmemO, "TMEM columns");
 };
 
 // Columns held by each CTA. bf16: rank 0 the nope columns 0..255 and the rope
@@ -161,11 +173,14 @@ struct MlaParams {
 };
 
 struct MlaBarriers {
-  uint64_t q_full, q_empty;
-  uint64_t kv_full[kMlaStages], kv_empty[kMlaStages];
+  uint64_t qs_full[kMlaQStages], qs_empty[kMlaQStages];  // Q chunk staging buffers
+  uint64_t q_done;  // the segment's last S has completed: TMEM Q may be replaced
+  uint64_t kv_full[kMlaMaxStages], kv_empty[kMlaMaxStages];
   uint64_t vh_full[2], vh_empty[2];  // FP8: the fp16 copies of V
   uint64_t s_full[kMlaSBufs], p_full[2];
-  uint64_t xs_full[kMlaXsBufs];  // the other CTA's partial S tile has landed here
+  uint64_t xs_full[kMlaXsBufs];   // the other CTA's partial S tile has landed here
+  uint64_t xs_empty[kMlaXsBufs];  // the other CTA has read the tile this CTA sent it
+  uint64_t s_read[kMlaSBufs];     // the sender has loaded S buffer k: P may overwrite it
   // o_full[k]: P V of every tile g with g % 3 == k has completed. One barrier
   // per S buffer: S of tile g is issued after P V of tile g - 3, so a waiter
   // for P V of tile x knows P V of tile x - 3 (the same barrier's previous
@@ -175,7 +190,7 @@ struct MlaBarriers {
   uint32_t tmem_base;
   int32_t abort;
 };
-static_assert(sizeof(MlaBarriers) <= 256, "barrier block");
+static_assert(sizeof(MlaBarriers) <= 512, "barrier block");
 
 // A segment and its rows.
 struct MlaSeg {
@@ -283,14 +298,14 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
   int ub, ue, s;
   const int32_t* prefix;
   mla_range<kSparse>(p, ub, ue, s, prefix);
-  int it = 0, nq = 0;
+  int it = 0, nqc = 0;  // key tiles and Q chunks issued
   const int P = p.page_size;
   // Sparse gathers issued and not yet signalled: tiles it - pend .. it - 1.
   int pend = 0;
   auto flush_gathers = [&]() {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     fence_proxy_async_smem();
-    for (; pend > 0; --pend) mbar_arrive(&bars->kv_full[(it - pend) % kMlaStages]);
+    for (; pend > 0; --pend) mbar_arrive(&bars->kv_full[(it - pend) % C::kStages]);
   };
   int u = ub;
   // After a failed wait the producer stops issuing and falls through to the
@@ -314,28 +329,33 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       ++s;
       continue;
     }
-    // Q tile of the segment: this CTA's chunks of the 576 columns
-    bool q_issued = false;
-    if (lane == 0) {
-      bool ok = nq == 0 || mbar_wait(&bars->q_empty, (nq - 1) & 1, abort, 60);
-      q_issued = ok;
-      if (ok) {
-        const int box_rows = p.group >= kMlaRows ? kMlaRows : p.group * (kSparse ? 1 : p.tokens_per_tile);
-        mbar_expect_tx(&bars->q_full, nch * box_rows * 128);
-        for (int c = 0; c < nch; ++c)
-          tma_load_4d(smem + C::kQOff + c * kMlaQChunkBytes, mq, &bars->q_full,
+    // Q tile of the segment: this CTA's chunks of the 576 columns, one at a
+    // time through the staging buffers (the MMA warp copies each into TMEM).
+    const int box_rows =
+        p.group >= kMlaRows ? kMlaRows : p.group * (kSparse ? 1 : p.tokens_per_tile);
+    for (int c = 0; c < nch && !stop; ++c) {
+      const int qb = nqc % kMlaQStages;
+      bool ok = true;
+      if (lane == 0) {
+        ok = nqc < kMlaQStages ||
+             mbar_wait(&bars->qs_empty[qb], ((nqc / kMlaQStages) - 1) & 1, abort, 60);
+        if (ok) {
+          mbar_expect_tx(&bars->qs_full[qb], box_rows * 128);
+          tma_load_4d(smem + C::kQSOff + qb * kMlaQChunkBytes, mq, &bars->qs_full[qb],
                       mla_col<kFp8>(rank, c), g.kvg * p.group + g.head0, g.tok0, g.b);
+        }
       }
+      if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) ++nqc;
+      else stop = true;
     }
-    if (__shfl_sync(0xffffffffu, q_issued ? 1 : 0, 0)) ++nq;
-    if (!__shfl_sync(0xffffffffu, (int)(*abort == 0), 0)) break;
+    if (stop) break;
     const int32_t* bt = p.block_table + (int64_t)g.bk * p.bt_stride;
     for (int t = a; t < e; ++t, ++it) {
-      const int st = it % kMlaStages;
+      const int st = it % C::kStages;
       uint8_t* dst = smem + C::kKVOff + st * C::kKVBytes;
       bool ok = true;
-      if (it >= kMlaStages) {
-        const uint32_t parity = ((it / kMlaStages) - 1) & 1;
+      if (it >= C::kStages) {
+        const uint32_t parity = ((it / C::kStages) - 1) & 1;
         if constexpr (kSparse) {
           // About to block on a stage: signal every gathered tile first (the
           // MMA warp may need them to free that stage).
@@ -408,13 +428,14 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
         if (pend > kGatherLag) {
           asm volatile("cp.async.wait_group %0;" ::"n"(kGatherLag) : "memory");
           fence_proxy_async_smem();
-          mbar_arrive(&bars->kv_full[(it - kGatherLag) % kMlaStages]);
+          mbar_arrive(&bars->kv_full[(it - kGatherLag) % C::kStages]);
           --pend;
         }
       }
     }
     if (stop) break;
-    // The segment's last S needs its last tiles before Q may be replaced.
+    // The segment's last S needs its last tiles before TMEM Q may be replaced
+    // (and the next segment's Q chunks wait for that).
     if constexpr (kSparse) flush_gathers();
     u = min(ue, se);
     ++s;
@@ -422,30 +443,43 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
   if constexpr (!kSparse) {
     if (lane == 0) {  // the last stages' copies must land before the CTA exits
       int zero = 0;
-      for (int i = max(0, it - kMlaStages); i < it; ++i)
-        mbar_wait(&bars->kv_full[i % kMlaStages], (i / kMlaStages) & 1, &zero, 62);
+      for (int i = max(0, it - C::kStages); i < it; ++i)
+        mbar_wait(&bars->kv_full[i % C::kStages], (i / C::kStages) & 1, &zero, 62);
     }
   }
-  if (lane == 0 && nq > 0) {
+  if (lane == 0) {  // and the last Q chunks
     int zero = 0;
-    mbar_wait(&bars->q_full, (nq - 1) & 1, &zero, 63);
+    for (int i = max(0, nqc - kMlaQStages); i < nqc; ++i)
+      mbar_wait(&bars->qs_full[i % kMlaQStages], (i / kMlaQStages) & 1, &zero, 63);
   }
 }
 
 // ---------------------------------------------------------------------------
 // MMA warp (whole warp; one elected lane issues)
 // ---------------------------------------------------------------------------
-// S of the tile with global index g (this CTA's partial scores): waits for
-// its key stage, writes S buffer g % 3; after the segment's last S, releases Q.
+// Shared memory to TMEM: 128 rows of 32 bytes (row i to lane i, 8 columns
+// from taddr's), the source given by a shared-memory matrix descriptor. Runs
+// in order with the MMAs this thread issues after it; one elected lane.
+DEVI void tc_cp_128x256b_w(uint32_t taddr, uint64_t sdesc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::1.128x256b [%0], %1;\n\t}" ::"r"(taddr),
+      "l"(sdesc)
+      : "memory");
+}
+
+// S of the tile with global index g (this CTA's partial scores), A = Q from
+// TMEM: waits for its key stage, writes S buffer g % 3; the segment's last S
+// also signals q_done (TMEM Q may then be replaced).
 // e4m3: S runs on the FP8 codes (kind::f8f6f4); P V reads the fp16 copy of V,
 // so the stage is released here (with the conversion warps' arrivals).
 template <bool kFp8>
-DEVI bool mla_issue_s(MlaBarriers* bars, int g, uint64_t dq, uint64_t dkv, uint32_t tmem, int nk,
-                      bool last) {
+DEVI bool mla_issue_s(MlaBarriers* bars, int g, uint64_t dkv, uint32_t tmem, int nk, bool last) {
   // kind::f16 format 1 = bf16; kind::f8f6f4 format 0 = e4m3
   constexpr uint32_t idesc_s = make_idesc(128, kMlaBN, kFp8 ? 0 : 1, 0, 0);
-  const int st = g % kMlaStages;
-  if (!warp_wait(&bars->kv_full[st], (g / kMlaStages) & 1, &bars->abort, 71)) return false;
+  constexpr int kStages = MlaCfg<kFp8>::kStages;
+  const int st = g % kStages;
+  if (!warp_wait(&bars->kv_full[st], (g / kStages) & 1, &bars->abort, 71)) return false;
   tc_fence_after();
   const uint32_t sbuf = tmem + kMlaTmemS + (g % kMlaSBufs) * kMlaBN;
   const uint64_t kst = dkv + st * (MlaCfg<kFp8>::kKVBytes >> 4);
@@ -453,16 +487,17 @@ DEVI bool mla_issue_s(MlaBarriers* bars, int g, uint64_t dq, uint64_t dkv, uint3
   for (int k = 0; k < nk; ++k) {
     int ch, sub;
     mla_kstep<kFp8>(k, ch, sub);
-    const uint32_t qo = ch * (kMlaQChunkBytes >> 4) + sub * 2;
+    // 32 bytes of each Q row per K step: 8 TMEM columns
+    const uint32_t qa = tmem + kMlaTmemQ + ch * 32 + sub * 8;
     const uint32_t ko = ch * (kMlaKVChunkBytes >> 4) + sub * 2;
     if constexpr (kFp8)
-      mma_f8_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
+      mma_f8_ts_w(sbuf, qa, kst + ko, idesc_s, k > 0 ? 1u : 0u);
     else
-      mma_f16_ss_w(sbuf, dq + qo, kst + ko, idesc_s, k > 0 ? 1u : 0u);
+      mma_f16_ts_w(sbuf, qa, kst + ko, idesc_s, k > 0 ? 1u : 0u);
   }
   tc_commit_w(&bars->s_full[g % kMlaSBufs]);
   if constexpr (kFp8) tc_commit_w(&bars->kv_empty[st]);
-  if (last) tc_commit_w(&bars->q_empty);
+  if (last) tc_commit_w(&bars->q_done);
   return true;
 }
 
@@ -473,7 +508,9 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
   const int nk = mla_ksteps<kFp8>(rank);  // 32-byte K steps of the partial score
   // P V: bf16 P and V, or (e4m3 rows) fp16 P and the fp16 copy of V
   constexpr uint32_t idesc_pv = make_idesc(128, kMlaDvHalf, kFp8 ? 0 : 1, 0, 1);
-  const uint64_t dq = sdesc_sw128(smem_u32(smem + C::kQOff), 16, 1024);
+  // Q staging buffers, 128-byte swizzled K-major: 32-byte K steps
+  const uint64_t dqs = sdesc_sw128(smem_u32(smem + C::kQSOff), 16, 1024);
+  const int nch = mla_nchunks<kFp8>(rank);
   const uint64_t dkv = sdesc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
   // This CTA's V half: local chunks 0..3 of the bf16 key tile (or of the
   // fp16 copy), MN-major (leading byte offset = chunk stride, stride byte
@@ -483,7 +520,7 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
   int ub, ue, s;
   const int32_t* prefix;
   mla_range<kSparse>(p, ub, ue, s, prefix);
-  int it = 0, nq = 0, pieces = 0;
+  int it = 0, nqc = 0, nseg = 0, pieces = 0;
   int u = ub;
   while (u < ue) {
     int sb, se;
@@ -504,16 +541,30 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
       ++s;
       continue;
     }
-    if (!warp_wait(&bars->q_full, nq & 1, abort, 70)) goto drain;
-    ++nq;
+    // Q into TMEM once the previous segment's S MMAs have read the old one:
+    // each staged chunk as 4 copies of 128 rows x 32 bytes (lane = row, 8
+    // columns each, the layout of an A operand in TMEM), then the staging
+    // buffer goes back to the producer.
+    if (nseg > 0 && !warp_wait(&bars->q_done, (nseg - 1) & 1, abort, 70)) goto drain;
+    ++nseg;
+    for (int c = 0; c < nch; ++c, ++nqc) {
+      const int qb = nqc % kMlaQStages;
+      if (!warp_wait(&bars->qs_full[qb], (nqc / kMlaQStages) & 1, abort, 78)) goto drain;
+      tc_fence_after();
+#pragma unroll
+      for (int sub = 0; sub < 4; ++sub)
+        tc_cp_128x256b_w(tmem + kMlaTmemQ + c * 32 + sub * 8,
+                         dqs + qb * (kMlaQChunkBytes >> 4) + sub * 2);
+      tc_commit_w(&bars->qs_empty[qb]);
+    }
     // S of the first kMlaSAhead tiles, then per tile g: PV_g, S_{g+kMlaSAhead}
     // (into buffer (g + kMlaSAhead) % 3, whose last P the tensor core has read
     // in an earlier P V: the pipe runs in order). The softmax thus finds
     // S_{g+1} ready while it finishes tile g.
     for (int j = 0; j < kMlaSAhead && j < n; ++j)
-      if (!mla_issue_s<kFp8>(bars, it + j, dq, dkv, tmem, nk, j == n - 1)) goto drain;
+      if (!mla_issue_s<kFp8>(bars, it + j, dkv, tmem, nk, j == n - 1)) goto drain;
     for (int j = 0; j < n; ++j) {
-      const int gi = it + j, sp = gi % kMlaStages;
+      const int gi = it + j, sp = gi % C::kStages;
       if (!warp_wait(&bars->p_full[gi & 1], (gi >> 1) & 1, abort, 72)) goto drain;
       if (j == 0 && pieces > 0 && !warp_wait(&bars->o_empty, (pieces - 1) & 1, abort, 73))
         goto drain;
@@ -536,7 +587,7 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
         tc_commit_w(&bars->kv_empty[sp]);
       tc_commit_w(&bars->o_full[gi % kMlaSBufs]);
       if (j + kMlaSAhead < n &&
-          !mla_issue_s<kFp8>(bars, gi + kMlaSAhead, dq, dkv, tmem, nk, j + kMlaSAhead == n - 1))
+          !mla_issue_s<kFp8>(bars, gi + kMlaSAhead, dkv, tmem, nk, j + kMlaSAhead == n - 1))
         goto drain;
     }
     it += n;
@@ -583,8 +634,8 @@ DEVI void mla_convert(const MlaParams& p, uint8_t* smem, MlaBarriers* bars) {
     mla_seg<kSparse>(p, s, g);
     const int a = u - sb, e = min(ue, se) - sb;
     for (int j = 0; j < e - a; ++j, ++it) {
-      const int st = it % kMlaStages, hb = it & 1;
-      if (!mbar_wait(&bars->kv_full[st], (it / kMlaStages) & 1, abort, 76)) return;
+      const int st = it % C::kStages, hb = it & 1;
+      if (!mbar_wait(&bars->kv_full[st], (it / C::kStages) & 1, abort, 76)) return;
       if (it >= 2 && !mbar_wait(&bars->vh_empty[hb], ((it >> 1) - 1) & 1, abort, 77)) return;
       // keys of the tile that exist (sparse: skipped entries are zeros already)
       const int nvalid = kSparse ? kMlaBN : g.len - (a + j) * kMlaBN;
@@ -625,47 +676,98 @@ DEVI void mla_convert(const MlaParams& p, uint8_t* smem, MlaBarriers* bars) {
 // ---------------------------------------------------------------------------
 // Softmax warpgroup
 // ---------------------------------------------------------------------------
-// Loads this CTA's partial scores of the tile with global index g into sv
-// and sends them to the other CTA of the cluster: 16-byte pieces permuted by
-// row (to spread the banks) into its buffer g % 2, then one arrival per row
-// on its barrier. This CTA sends tile g only after it has received the other
-// CTA's tile g - 1, which the other CTA sent after reading its tile g - 2
-// (the buffer's last use there), so the buffer is free; and the barrier is at
-// most one phase ahead of its waiter.
-template <bool kFp8>
-DEVI bool mla_send_partial(MlaBarriers* bars, uint8_t* smem, uint32_t tmem, uint32_t lane, int r,
-                           int rank, int g, uint32_t* sv) {
-  using C = MlaCfg<kFp8>;
-  const int sb = g % kMlaSBufs, b = g % kMlaXsBufs;
-  if (!warp_wait(&bars->s_full[sb], (g / kMlaSBufs) & 1, &bars->abort, 80)) return false;
-  tc_fence_after();
-  tmem_load<32>(tmem + kMlaTmemS + sb * kMlaBN + lane, sv);
-  // Stage this warp's 32 rows (16-byte pieces permuted by row to spread the
-  // banks) and send them with one bulk copy into the other CTA's buffer b,
-  // completing on its barrier. Staging buffer b was last the source of the
-  // copy two tiles ago: that copy must have read it.
-  const int warp_row0 = r & ~31;
-  const bool leader = (threadIdx.x & 31) == 0;
-  if (leader) bulk_wait_read<1>();
-  __syncwarp();
-  uint8_t* stage = smem + C::kXoOff + b * kMlaXsBytes + r * 128;
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    *reinterpret_cast<uint4*>(stage + ((k ^ (r & 7)) << 4)) =
-        make_uint4(sv[4 * k], sv[4 * k + 1], sv[4 * k + 2], sv[4 * k + 3]);
-  fence_proxy_async_smem();  // the copy reads through the async proxy
-  __syncwarp();
-  if (leader) {
-    const uint32_t bar = mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1);
-    const uint32_t off = b * kMlaXsBytes + warp_row0 * 128;
-    mbar_arrive_expect_tx_remote(bar, 32 * 128);
-    bulk_copy_to_cluster(mapa_shared(smem_u32(smem + C::kXsOff + off), rank ^ 1),
-                         smem_u32(smem + C::kXoOff + off), 32 * 128, bar);
-    bulk_commit();
-  }
-  return true;
+// ---------------------------------------------------------------------------
+// Sender warpgroup
+// ---------------------------------------------------------------------------
+// Remote arrivals with relaxed semantics. A release at cluster scope here
+// cost about a thousand cycles per tile on the softmax's critical path.
+// expect_tx publishes nothing (the bulk copy's complete_tx carries the data);
+// the release of a receive buffer follows loads whose values the thread has
+// already consumed (the adds before it), and a warp issues in order, so the
+// loads have returned before the arrival leaves.
+DEVI void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+DEVI void mbar_expect_tx_remote_relaxed(uint32_t cluster_addr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(
+                   cluster_addr),
+               "r"(bytes)
+               : "memory");
 }
 
+// For every tile, in the MMA warp's order: loads this CTA's partial scores
+// (thread = row = TMEM lane) and tells the softmax the S buffer may take P
+// (s_read), then sends the rows to the other CTA's receive buffer g % 2:
+// each warp stages its 32 rows (16-byte pieces permuted by row to spread the
+// banks), fences them for the async proxy and sends one 4 KB bulk copy that
+// completes on that CTA's barrier. Before writing buffer b it waits until the
+// other CTA's softmax has read the tile sent there before (xs_empty), and
+// staging buffer b until the copy two tiles ago has read it. The softmax
+// threads thus never wait on the exchange's staging, fence or copy.
+template <bool kSparse, bool kFp8>
+DEVI void mla_sender(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem,
+                     int rank, int quarter) {
+  using C = MlaCfg<kFp8>;
+  volatile int* abort = &bars->abort;
+  const int r = quarter * 32 + (threadIdx.x & 31);  // row = TMEM lane
+  const uint32_t lane = (uint32_t)(quarter * 32) << 16;
+  const bool leader = (threadIdx.x & 31) == 0;
+  int ub, ue, s;
+  const int32_t* prefix;
+  mla_range<kSparse>(p, ub, ue, s, prefix);
+  int g = 0;
+  int u = ub;
+  while (u < ue) {
+    int sb, se;
+    if (prefix) {
+      sb = prefix[s];
+      se = prefix[s + 1];
+      if (se <= u) { ++s; continue; }
+    } else {
+      sb = u;
+      se = ue;
+    }
+    const int n = max(0, min(ue, se) - u);
+    for (int j = 0; j < n; ++j, ++g) {
+      const int sbuf = g % kMlaSBufs, b = g % kMlaXsBufs;
+      uint32_t sv[kMlaBN];
+      if (!warp_wait(&bars->s_full[sbuf], (g / kMlaSBufs) & 1, abort, 80)) return;
+      tc_fence_after();
+      tmem_load<32>(tmem + kMlaTmemS + sbuf * kMlaBN + lane, sv);
+      tc_fence_before();
+      __syncwarp();
+      if (leader) mbar_arrive(&bars->s_read[sbuf]);
+      if (g >= kMlaXsBufs &&
+          !warp_wait_cluster(&bars->xs_empty[b], ((g / kMlaXsBufs) - 1) & 1, abort, 84))
+        return;
+      const int warp_row0 = r & ~31;
+      if (leader) bulk_wait_read<1>();
+      __syncwarp();
+      uint8_t* stage = smem + C::kXoOff + b * kMlaXsBytes + r * 128;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<uint4*>(stage + ((k ^ (r & 7)) << 4)) =
+            make_uint4(sv[4 * k], sv[4 * k + 1], sv[4 * k + 2], sv[4 * k + 3]);
+      fence_proxy_async_smem();  // the copy reads through the async proxy
+      __syncwarp();
+      if (leader) {
+        const uint32_t bar = mapa_shared(smem_u32(&bars->xs_full[b]), rank ^ 1);
+        const uint32_t off = b * kMlaXsBytes + warp_row0 * 128;
+        mbar_expect_tx_remote_relaxed(bar, 32 * 128);
+        bulk_copy_to_cluster(mapa_shared(smem_u32(smem + C::kXsOff + off), rank ^ 1),
+                             smem_u32(smem + C::kXoOff + off), 32 * 128, bar);
+        bulk_commit();
+      }
+    }
+    u = min(ue, se);
+    ++s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Softmax warpgroup
+// ---------------------------------------------------------------------------
 template <bool kSparse, bool kFp8>
 DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem,
                       int rank) {
@@ -728,18 +830,16 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     }
     float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
     bool seen = false;
-    // The partial scores of tile g + 1 go to the other CTA as soon as those of
-    // tile g have arrived here: they are in flight while tile g is
-    // exponentiated.
     uint32_t sv[kMlaBN];
-    if (n > 0 && !mla_send_partial<kFp8>(bars, smem, tmem, lane, r, rank, it, sv)) return;
     for (int j = 0; j < n; ++j) {
       const int gi = it + j;
       const int t = a + j;
-      uint32_t sv_next[kMlaBN];
       {
-        // The other CTA's partials of this tile.
-        const int b = gi % kMlaXsBufs;
+        // This CTA's partial scores of the tile, plus the other CTA's.
+        const int b = gi % kMlaXsBufs, sbuf = gi % kMlaSBufs;
+        if (!warp_wait(&bars->s_full[sbuf], (gi / kMlaSBufs) & 1, abort, 86)) return;
+        tc_fence_after();
+        tmem_load<32>(tmem + kMlaTmemS + sbuf * kMlaBN + lane, sv);
         if (!warp_wait_cluster(&bars->xs_full[b], (gi / kMlaXsBufs) & 1, abort, 83)) return;
         const uint8_t* src = smem + C::kXsOff + b * kMlaXsBytes + r * 128;
 #pragma unroll
@@ -750,9 +850,12 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
           sv[4 * k + 2] = __float_as_uint(__uint_as_float(sv[4 * k + 2]) + __uint_as_float(v.z));
           sv[4 * k + 3] = __float_as_uint(__uint_as_float(sv[4 * k + 3]) + __uint_as_float(v.w));
         }
+        // This warp's rows of the buffer have been read: the other CTA may
+        // send its next tile there.
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0)
+          mbar_arrive_remote_relaxed(mapa_shared(smem_u32(&bars->xs_empty[b]), rank ^ 1));
       }
-      if (j + 1 < n && !mla_send_partial<kFp8>(bars, smem, tmem, lane, r, rank, gi + 1, sv_next))
-        return;
       if constexpr (kSparse) {
         // Key position of entry e (see mla_sparse_pos); visible iff
         // 0 <= pos <= hi (hi = L - 1, or with sparse_mode=3, "rightDownCausal",
@@ -791,7 +894,7 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
         // zero them in the fp16 copy.)
         const int nvalid = g.len - k0;
         if (!kFp8 && nvalid < kMlaBN) {
-          uint8_t* kvs = smem + C::kKVOff + (gi % kMlaStages) * C::kKVBytes;
+          uint8_t* kvs = smem + C::kKVOff + (gi % C::kStages) * C::kKVBytes;
           const int bad = kMlaBN - nvalid;
           for (int x = r; x < 4 * bad * 8; x += 128) {
             const int c = x / (bad * 8), rem = x % (bad * 8);
@@ -855,12 +958,13 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       }
       l_run += le;
       l_rnd += lr;
+      // P replaces S in the buffer once the sender has loaded S from it
+      if (!warp_wait(&bars->s_read[gi % kMlaSBufs], (gi / kMlaSBufs) & 1, abort, 87)) return;
+      tc_fence_after();
       tmem_store<16>(tmem + kMlaTmemS + (gi % kMlaSBufs) * kMlaBN + lane, pk);
       tmem_store_wait();
       tc_fence_before();
       mbar_arrive(&bars->p_full[gi & 1]);
-#pragma unroll
-      for (int c = 0; c < kMlaBN; ++c) sv[c] = sv_next[c];
     }
     it += n;
 
@@ -945,9 +1049,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThrea
   const int warp = threadIdx.x >> 5;
   const int rank = (int)cluster_ctarank();
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
-    for (int i = 0; i < kMlaStages; ++i) {
+    for (int i = 0; i < kMlaQStages; ++i) {
+      mbar_init(&bars->qs_full[i], 1);
+      mbar_init(&bars->qs_empty[i], 1);
+    }
+    mbar_init(&bars->q_done, 1);
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&bars->kv_full[i], kSparse ? 32 : 1);
       // e4m3: released by the S MMA's commit and the 64 conversion threads
       mbar_init(&bars->kv_empty[i], kFp8 ? 1 + 64 : 1);
@@ -957,8 +1064,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThrea
       mbar_init(&bars->vh_empty[i], 1);
     }
     for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->s_full[i], 1);
-    for (int i = 0; i < kMlaXsBufs; ++i)
-      mbar_init(&bars->xs_full[i], 4);  // one bulk copy from each softmax warp of the other CTA
+    for (int i = 0; i < kMlaXsBufs; ++i) {
+      mbar_init(&bars->xs_full[i], 4);   // one bulk copy from each sender warp of the other CTA
+      mbar_init(&bars->xs_empty[i], 4);  // each softmax warp of the other CTA has read
+    }
+    for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->s_read[i], 4);  // each sender warp
     for (int i = 0; i < 2; ++i) mbar_init(&bars->p_full[i], 128);
     for (int i = 0; i < kMlaSBufs; ++i) mbar_init(&bars->o_full[i], 1);
     mbar_init(&bars->o_empty, 128);
@@ -997,11 +1107,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MlaCfg<kFp8>::kThrea
       mla_producer<kSparse, kFp8>(p, &map_q, &map_kv, smem, bars, rank);
     else if (warp == 5)
       mla_mma<kSparse, kFp8>(p, smem, bars, tmem, rank);
+    else if (warp >= C::kSendWarp0)
+      mla_sender<kSparse, kFp8>(p, smem, bars, tmem, rank, warp & 3);
     else if constexpr (kFp8)
       mla_convert<kSparse>(p, smem, bars);
   }
   // The partial-score copies this CTA sent have landed in the other CTA.
-  if (warp < 4 && (threadIdx.x & 31) == 0) bulk_wait_all();
+  if (warp >= C::kSendWarp0 && (threadIdx.x & 31) == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   // No remote arrival or store into this CTA's shared memory after this.
