@@ -12,8 +12,9 @@
 //
 // Work decomposition. A cluster of two CTAs owns 128 query rows ("row tile")
 // and streams the keys once for both V halves: CTA rank r holds the score
-// dimensions of its V half (rank 0: nope 0..255 and the 64 rope dimensions,
-// rank 1: nope 256..511) of Q and of every key, computes the partial scores
+// dimensions of its V half (rank r: nope 256r .. 256r + 255) and a share of
+// the 64 rope dimensions (dense: 32 each; sparse: all on rank 0) of Q and of
+// every key, computes the partial scores
 // S_r = Q_r K_r^T on its tensor core, and the two halves swap partials through
 // distributed shared memory (one bulk copy per warp into the other CTA,
 // completing on its barrier), so both see S = S_0 + S_1 (the same sum in the
@@ -109,30 +110,42 @@ struct MlaCfg {
   static_assert(kMlaTmemQ + 32 * kMaxChunks <= kMlaTmemO, "TMEM columns");
 };
 
-// Columns held by each CTA. bf16: rank 0 the nope columns 0..255 and the rope
-// (chunks 0-3 and 8 of 64 columns), rank 1 the nope columns 256..511. e4m3
-// (128 columns per chunk): rank 0 columns 0..255 and a box at column 448,
-// of which only the second half (the rope, 512..575) is used; rank 1 columns
-// 256..511. Either way a CTA's first 256 columns are its V half.
-template <bool kFp8>
-DEVI int mla_nchunks(int rank) { return kFp8 ? (rank == 0 ? 3 : 2) : (rank == 0 ? 5 : 4); }
+// Columns held by each CTA. A CTA's first 256 columns are its V half: rank r
+// holds the nope (latent) columns 256r .. 256r + 255. The 64 rope columns
+// (512..575) sit in one more box: bf16 chunk 4 (64 columns at 512); e4m3
+// chunk 2 (the box at 448, whose second half is the rope). Dense kernels
+// split the rope, 32 columns to each CTA (both load its box), so the two
+// CTAs' S MMAs take 18 (e4m3: 9) K steps each; sparse kernels, bound by the
+// gathered bytes rather than the MMAs, leave it all to rank 0 (20 and 16
+// steps; e4m3 10 and 8) and rank 1 loads no rope box.
+template <bool kFp8, bool kSplitRope>
+DEVI int mla_nchunks(int rank) {
+  return (kSplitRope || rank == 0) ? (kFp8 ? 3 : 5) : (kFp8 ? 2 : 4);
+}
 // First element column of local chunk c of rank r.
 template <bool kFp8>
 DEVI int mla_col(int rank, int c) {
-  if constexpr (kFp8) return rank == 0 ? (c < 2 ? 128 * c : 448) : 256 + 128 * c;
-  return 64 * (rank == 0 ? (c < 4 ? c : 8) : 4 + c);
+  if constexpr (kFp8) return c < 2 ? 256 * rank + 128 * c : 448;
+  return c < 4 ? 64 * (4 * rank + c) : 512;
 }
 // 32-byte K steps of this CTA's partial score, and the (chunk, step within
-// the chunk) of step k: e4m3 rank 0 skips the first half of its last box.
+// the chunk) of step k. The rope steps start at step 2 of the e4m3 box (its
+// first half is latent columns 448..511, counted by rank 1) and, with a split
+// rope, rank 1 takes the second half of the rope.
+template <bool kFp8, bool kSplitRope>
+DEVI int mla_ksteps(int rank) {
+  return kSplitRope ? (kFp8 ? 9 : 18) : (kFp8 ? (rank == 0 ? 10 : 8) : (rank == 0 ? 20 : 16));
+}
 template <bool kFp8>
-DEVI int mla_ksteps(int rank) { return kFp8 ? (rank == 0 ? 10 : 8) : 4 * mla_nchunks<false>(rank); }
-template <bool kFp8>
-DEVI void mla_kstep(int k, int& chunk, int& sub) {
+DEVI void mla_kstep(int k, int rope_off, int& chunk, int& sub) {
   chunk = k >> 2;
   sub = k & 3;
   if (kFp8 && k >= 8) {
     chunk = 2;
-    sub = k - 6;
+    sub = 2 + (k - 8) + rope_off;
+  } else if (!kFp8 && k >= 16) {
+    chunk = 4;
+    sub = (k - 16) + rope_off;
   }
 }
 
@@ -247,6 +260,17 @@ DEVI int mla_sparse_pos(const MlaParams& p, int b, int kvg, int tok, int e) {
   const int k = __ldg(p.indices + b * p.idx_sb + (int64_t)tok * p.idx_ss + kvg * p.idx_sh + blk);
   return k >= 0 ? (k << p.sbs_log2) + (e & (p.sbs - 1)) : -1;
 }
+// The same in two steps, so that the index load can be issued a tile early
+// and stay in flight until its value is used: the raw index word of entry e
+// (-1 past the list), then the position it gives.
+DEVI int mla_sparse_raw(const MlaParams& p, int b, int kvg, int tok, int e) {
+  if (e >= (p.topk << p.sbs_log2)) return -1;
+  return __ldg(p.indices + b * p.idx_sb + (int64_t)tok * p.idx_ss + kvg * p.idx_sh +
+               (e >> p.sbs_log2));
+}
+DEVI int mla_pos_of(const MlaParams& p, int k, int e) {
+  return k >= 0 ? (k << p.sbs_log2) + (e & (p.sbs - 1)) : -1;
+}
 
 // Token and (global) query head of tile row x.
 DEVI void mla_row(const MlaParams& p, const MlaSeg& g, int x, int& tok, int& head) {
@@ -290,7 +314,7 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
   constexpr int kEsize = kFp8 ? 1 : 2;
   volatile int* abort = &bars->abort;
   const int lane = threadIdx.x & 31;
-  const int nch = mla_nchunks<kFp8>(rank);
+  const int nch = mla_nchunks<kFp8, !kSparse>(rank);
   if (lane == 0) {
     tma_prefetch_desc(mq);
     if (!kSparse) tma_prefetch_desc(mkv);
@@ -350,6 +374,15 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
     }
     if (stop) break;
     const int32_t* bt = p.block_table + (int64_t)g.bk * p.bt_stride;
+    // sparse: this lane's index word is loaded two tiles ahead and its cache
+    // block one tile ahead, so no dependent global load sits between a stage
+    // becoming free and the gathers into it.
+    int pos_c = -1, blk_c = 0, raw_n = -1;  // tile t's position and block; tile t + 1's index
+    if constexpr (kSparse) {
+      pos_c = mla_sparse_pos(p, g.b, g.kvg, g.tok0, a * kMlaBN + lane);
+      if (pos_c >= 0 && pos_c < g.len) blk_c = __ldg(bt + pos_c / P);
+      if (a + 1 < e) raw_n = mla_sparse_raw(p, g.b, g.kvg, g.tok0, (a + 1) * kMlaBN + lane);
+    }
     for (int t = a; t < e; ++t, ++it) {
       const int st = it % C::kStages;
       uint8_t* dst = smem + C::kKVOff + st * C::kKVBytes;
@@ -391,20 +424,17 @@ DEVI void mla_producer(const MlaParams& p, const CUtensorMap* mq, const CUtensor
       } else {
         // lane k gathers key t*32 + k: 8 async copies of 16 bytes per chunk
         // into the 128-byte-swizzled layout, or zeros if the entry is skipped.
-        int pos = -1;
-        if (p.sbs_log2 == 0) {  // one key per index: the index itself
-          const int e_idx = t * kMlaBN + lane;
-          if (e_idx < p.topk)
-            pos = p.indices[g.b * p.idx_sb + g.tok0 * p.idx_ss + g.kvg * p.idx_sh + e_idx];
-        } else {
-          pos = mla_sparse_pos(p, g.b, g.kvg, g.tok0, t * kMlaBN + lane);
-        }
+        const int pos = pos_c, blk = blk_c;
         const bool valid = pos >= 0 && pos < g.len;
+        // ahead: the position and block of tile t + 1, the index of tile t + 2
+        pos_c = mla_pos_of(p, raw_n, (t + 1) * kMlaBN + lane);
+        blk_c = (pos_c >= 0 && pos_c < g.len) ? __ldg(bt + pos_c / P) : 0;
+        raw_n = t + 2 < e ? mla_sparse_raw(p, g.b, g.kvg, g.tok0, (t + 2) * kMlaBN + lane) : -1;
         const uint8_t* src = nullptr;  // the cached row, in bytes
         if (valid)
           src = static_cast<const uint8_t*>(p.kv) +
-                (g.kvg * p.kv_sh + (int64_t)bt[pos / P] * p.kv_sblk +
-                 (int64_t)(pos % P) * p.kv_stok) * kEsize;
+                (g.kvg * p.kv_sh + (int64_t)blk * p.kv_sblk + (int64_t)(pos % P) * p.kv_stok) *
+                    kEsize;
         const uint32_t dbase = smem_u32(dst) + lane * 128;
         for (int c = 0; c < nch; ++c) {
           const int gcol = mla_col<kFp8>(rank, c) * kEsize;  // byte column of the chunk
@@ -474,7 +504,8 @@ DEVI void tc_cp_128x256b_w(uint32_t taddr, uint64_t sdesc) {
 // e4m3: S runs on the FP8 codes (kind::f8f6f4); P V reads the fp16 copy of V,
 // so the stage is released here (with the conversion warps' arrivals).
 template <bool kFp8>
-DEVI bool mla_issue_s(MlaBarriers* bars, int g, uint64_t dkv, uint32_t tmem, int nk, bool last) {
+DEVI bool mla_issue_s(MlaBarriers* bars, int g, uint64_t dkv, uint32_t tmem, int nk, int rope_off,
+                      bool last) {
   // kind::f16 format 1 = bf16; kind::f8f6f4 format 0 = e4m3
   constexpr uint32_t idesc_s = make_idesc(128, kMlaBN, kFp8 ? 0 : 1, 0, 0);
   constexpr int kStages = MlaCfg<kFp8>::kStages;
@@ -486,7 +517,7 @@ DEVI bool mla_issue_s(MlaBarriers* bars, int g, uint64_t dkv, uint32_t tmem, int
 #pragma unroll 4
   for (int k = 0; k < nk; ++k) {
     int ch, sub;
-    mla_kstep<kFp8>(k, ch, sub);
+    mla_kstep<kFp8>(k, rope_off, ch, sub);
     // 32 bytes of each Q row per K step: 8 TMEM columns
     const uint32_t qa = tmem + kMlaTmemQ + ch * 32 + sub * 8;
     const uint32_t ko = ch * (kMlaKVChunkBytes >> 4) + sub * 2;
@@ -505,12 +536,14 @@ template <bool kSparse, bool kFp8>
 DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t tmem, int rank) {
   using C = MlaCfg<kFp8>;
   volatile int* abort = &bars->abort;
-  const int nk = mla_ksteps<kFp8>(rank);  // 32-byte K steps of the partial score
+  const int nk = mla_ksteps<kFp8, !kSparse>(rank);  // 32-byte K steps of the partial score
+  // with a split rope, rank 1 takes its second half (2 bf16 or 1 e4m3 K steps on)
+  const int rope_off = (!kSparse && rank == 1) ? (kFp8 ? 1 : 2) : 0;
   // P V: bf16 P and V, or (e4m3 rows) fp16 P and the fp16 copy of V
   constexpr uint32_t idesc_pv = make_idesc(128, kMlaDvHalf, kFp8 ? 0 : 1, 0, 1);
   // Q staging buffers, 128-byte swizzled K-major: 32-byte K steps
   const uint64_t dqs = sdesc_sw128(smem_u32(smem + C::kQSOff), 16, 1024);
-  const int nch = mla_nchunks<kFp8>(rank);
+  const int nch = mla_nchunks<kFp8, !kSparse>(rank);
   const uint64_t dkv = sdesc_sw128(smem_u32(smem + C::kKVOff), 16, 1024);
   // This CTA's V half: local chunks 0..3 of the bf16 key tile (or of the
   // fp16 copy), MN-major (leading byte offset = chunk stride, stride byte
@@ -562,7 +595,7 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
     // in an earlier P V: the pipe runs in order). The softmax thus finds
     // S_{g+1} ready while it finishes tile g.
     for (int j = 0; j < kMlaSAhead && j < n; ++j)
-      if (!mla_issue_s<kFp8>(bars, it + j, dkv, tmem, nk, j == n - 1)) goto drain;
+      if (!mla_issue_s<kFp8>(bars, it + j, dkv, tmem, nk, rope_off, j == n - 1)) goto drain;
     for (int j = 0; j < n; ++j) {
       const int gi = it + j, sp = gi % C::kStages;
       if (!warp_wait(&bars->p_full[gi & 1], (gi >> 1) & 1, abort, 72)) goto drain;
@@ -587,7 +620,8 @@ DEVI void mla_mma(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint32_t
         tc_commit_w(&bars->kv_empty[sp]);
       tc_commit_w(&bars->o_full[gi % kMlaSBufs]);
       if (j + kMlaSAhead < n &&
-          !mla_issue_s<kFp8>(bars, gi + kMlaSAhead, dkv, tmem, nk, j + kMlaSAhead == n - 1))
+          !mla_issue_s<kFp8>(bars, gi + kMlaSAhead, dkv, tmem, nk, rope_off,
+                             j + kMlaSAhead == n - 1))
         goto drain;
     }
     it += n;
@@ -817,9 +851,14 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
     // dense: visible keys [0, hi]; causal aligns the last token with the last key
     int hi = g.len - 1;
     if (p.causal) hi = min(hi, (tok - g.q0) + g.len - g.sq);
-    const int* idx_row =
-        kSparse ? p.indices + g.b * p.idx_sb + (int64_t)tok * p.idx_ss + g.kvg * p.idx_sh
-                : nullptr;
+    // sparse: every row of the tile is token tok0, so key visibility is the
+    // same for all rows; lane c of each warp evaluates key c of a tile and
+    // the warp shares the result by ballot. The index is loaded one tile ahead.
+    int hi0 = g.len - 1;
+    if (kSparse && p.causal) hi0 = min(hi0, (g.tok0 - g.q0) + g.len - g.sq);
+    const int lane_c = threadIdx.x & 31;
+    int raw_next = -1;
+    if (kSparse && n > 0) raw_next = mla_sparse_raw(p, g.b, g.kvg, g.tok0, a * kMlaBN + lane_c);
     // FP8: S and O use the dequantised rows (MATE FMHA dtype notes): the q and
     // k descales of (sequence, KV head) scale the scores, the v descale O.
     float sl2 = p.scale_log2, v_scale = 1.f;
@@ -859,28 +898,13 @@ DEVI void mla_softmax(const MlaParams& p, uint8_t* smem, MlaBarriers* bars, uint
       if constexpr (kSparse) {
         // Key position of entry e (see mla_sparse_pos); visible iff
         // 0 <= pos <= hi (hi = L - 1, or with sparse_mode=3, "rightDownCausal",
-        // also tok + L - s_q). One key per index: the index row is read with
-        // contiguous loads.
-        const int n_e = valid_row ? (p.topk << p.sbs_log2) : 0;
-        if (p.sbs_log2 == 0) {
-          const int* idx = idx_row + t * kMlaBN;
+        // also tok + L - s_q).
+        const int pos = mla_pos_of(p, raw_next, t * kMlaBN + lane_c);
+        if (j + 1 < n) raw_next = mla_sparse_raw(p, g.b, g.kvg, g.tok0, (t + 1) * kMlaBN + lane_c);
+        const uint32_t vis = __ballot_sync(0xffffffffu, pos >= 0 && pos <= hi0);
 #pragma unroll
-          for (int c = 0; c < kMlaBN; ++c) {
-            const int pos = (t * kMlaBN + c < n_e) ? __ldg(idx + c) : -1;
-            if (!(pos >= 0 && pos <= hi)) sv[c] = __float_as_uint(-INFINITY);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kMlaBN; ++c) {
-            const int e = t * kMlaBN + c;
-            int pos = -1;
-            if (e < n_e) {
-              const int k = __ldg(idx_row + (e >> p.sbs_log2));
-              pos = k >= 0 ? (k << p.sbs_log2) + (e & (p.sbs - 1)) : -1;
-            }
-            if (!(pos >= 0 && pos <= hi)) sv[c] = __float_as_uint(-INFINITY);
-          }
-        }
+        for (int c = 0; c < kMlaBN; ++c)
+          if (!valid_row || !((vis >> c) & 1u)) sv[c] = __float_as_uint(-INFINITY);
       } else {
         const int k0 = t * kMlaBN;
         if (k0 + kMlaBN - 1 > hi) {
