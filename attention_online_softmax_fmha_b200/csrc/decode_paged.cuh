@@ -534,12 +534,16 @@ DEVI void decode_consumer(const DecodeParams& p, uint8_t* smem, uint64_t* full, 
         l_run[h2] *= alpha[h2];
         l_rnd[h2] *= alpha[h2];
       }
+      // O is rescaled only when some row of the warp raised its max (the
+      // product by 1 would change nothing).
+      if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        o[n][0] *= alpha[0];
-        o[n][1] *= alpha[0];
-        o[n][2] *= alpha[1];
-        o[n][3] *= alpha[1];
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][0] *= alpha[0];
+          o[n][1] *= alpha[0];
+          o[n][2] *= alpha[1];
+          o[n][3] *= alpha[1];
+        }
       }
       // P (rounded to the input type) as the A operand of P V
       uint32_t pa[4];
