@@ -22,7 +22,8 @@
 //               accumulation. Two consumer warps per SM sub-partition hide
 //               each other's per-tile latency chain (wait, ldmatrix, MMA,
 //               shuffles, exp2). At the end of a segment piece the eight warp
-//               states are merged through shared memory.
+//               states are merged through shared memory in a fixed order, so
+//               repeated runs agree bit for bit.
 // FP8 caches (e4m3 / e5m2, D = 128) arrive as 128-byte rows. S = Q K^T runs
 // on the FP8 codes directly (mma.sync m16n8k32, Q kept in FP8); each warp
 // rewrites its 16 V rows as fp16 (exact for both formats) in a private

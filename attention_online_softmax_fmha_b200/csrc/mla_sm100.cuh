@@ -62,10 +62,10 @@ constexpr int kMlaBN = 32;         // keys per tile
 constexpr int kMlaRows = 128;      // query rows per row tile
 constexpr int kMlaMaxStages = 8;  // key stages of the deepest ring (MlaCfg::kStages)
 constexpr int kMlaSBufs = 3;       // S buffers in TMEM
-// S of tile g + kMlaSAhead is issued after P V of tile g. The softmax needs
-// S one tile ahead (it sends tile g + 1's partials before finishing tile g),
-// so at least 2; each tile further ahead keeps one more key stage busy and
-// leaves one tile less of slack for the loads.
+// S of tile g + kMlaSAhead is issued after P V of tile g. The sender needs S
+// ahead of the softmax (the other CTA waits for its partials), so at least
+// 2; each tile further ahead keeps one more key stage busy and leaves one
+// tile less of slack for the loads.
 constexpr int kMlaSAhead = 3;
 static_assert(kMlaSAhead >= 2 && kMlaSAhead <= kMlaSBufs, "S lookahead");
 // The O barriers (one per S buffer) rely on S of tile g being issued after P V
@@ -88,7 +88,7 @@ constexpr int kMlaQStages = 2;         // Q staging buffers of one chunk (128 ro
 // fp16 partner type in one MMA, and P stays fp16), made by two extra warps.
 template <bool kFp8>
 struct MlaCfg {
-  static constexpr int kMaxChunks = kFp8 ? 3 : 5;          // chunks per CTA (rank 0)
+  static constexpr int kMaxChunks = kFp8 ? 3 : 5;          // chunks per CTA (at most)
   static constexpr int kKVBytes = kMaxChunks * kMlaKVChunkBytes;
   // Q passes through two one-chunk staging buffers into TMEM, where the S
   // MMAs read it; the shared memory this frees holds more key stages.
