@@ -137,7 +137,9 @@ __global__ void __launch_bounds__(1024, 1) sched_kernel(const SchedParams p) {
     seg_begin[s] = n;
     mine += (unsigned long long)max(n, 0);
   }
-  atomicAdd(&sh_units, mine);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  if ((tid & 31) == 0) atomicAdd(&sh_units, mine);
   __syncthreads();
   if (sh_units > (unsigned long long)INT32_MAX) {
     if (tid == 0) {
