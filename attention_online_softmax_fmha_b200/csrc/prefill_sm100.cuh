@@ -115,7 +115,7 @@ struct PrefillCfg {
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kVHOff = kVOff + kVStages * kTileBytes;
   static constexpr int kBarOff = kVHOff + kVHStages * kVHBytes;
-  static constexpr int kBarBytes = 512;
+  static constexpr int kBarBytes = 1024;
   static constexpr int kSmemBytes = kBarOff + kBarBytes;
   // The dynamic shared memory base is 1024-byte aligned (the kernel checks).
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -127,9 +127,20 @@ struct PrefillCfg {
 // Unit numbers in flight from the producer to the other roles.
 constexpr int kUnitRing = 4;
 
+struct PrefillUnit {
+  int b, h, m;
+  int len_q, len_k;
+  int row_q, row_k;  // first packed row of this sequence (0 for padded)
+  int bcoord;        // batch coordinate of the tensor maps (0 for varlen)
+  int kt0, kt1;      // key tiles [kt0, kt1)
+};
+
 struct PrefillBarriers {
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   int32_t unit_idx[kUnitRing];  // a unit number, or -1 after the CTA's last unit
+  // The producer's decoding of each unit in the ring, so that no other role
+  // reads the sequence offsets from global memory between two units.
+  PrefillUnit units[kUnitRing];
   uint64_t q_full, q_empty;
   uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t vh_full[4], vh_empty[4];
@@ -138,15 +149,8 @@ struct PrefillBarriers {
   uint32_t tmem_base;
   int32_t abort;
 };
-static_assert(sizeof(PrefillBarriers) <= 512, "barrier block");
+static_assert(sizeof(PrefillBarriers) <= 1024, "barrier block");
 
-struct PrefillUnit {
-  int b, h, m;
-  int len_q, len_k;
-  int row_q, row_k;  // first packed row of this sequence (0 for padded)
-  int bcoord;        // batch coordinate of the tensor maps (0 for varlen)
-  int kt0, kt1;      // key tiles [kt0, kt1)
-};
 
 // Maps a linear work index to a unit; returns false for units past the end
 // of their sequence. Every role calls this with the same index and gets the
@@ -187,12 +191,19 @@ DEVI bool prefill_unit(const PrefillParams& p, int t, PrefillUnit& u) {
   return true;
 }
 
-// Takes the k-th unit number of this CTA from the ring (warp-collective; each
-// consuming warp releases the slot once). Returns false if the wait gave up.
-DEVI bool take_unit(PrefillBarriers* bars, int k, int& t, int site) {
+// Takes the k-th unit number of this CTA, and its decoding, from the ring
+// (warp-collective; each consuming warp releases the slot once). Returns
+// false if the wait gave up.
+DEVI bool take_unit(PrefillBarriers* bars, int k, int& t, PrefillUnit& u, int site) {
   const int slot = k % kUnitRing;
   if (!warp_wait(&bars->unit_full[slot], (k / kUnitRing) & 1, &bars->abort, site)) return false;
   t = *reinterpret_cast<volatile int32_t*>(&bars->unit_idx[slot]);
+  if (t >= 0) {
+    const volatile int* src = reinterpret_cast<const volatile int*>(&bars->units[slot]);
+    int* dst = reinterpret_cast<int*>(&u);
+#pragma unroll
+    for (int x = 0; x < (int)(sizeof(PrefillUnit) / sizeof(int)); ++x) dst[x] = src[x];
+  }
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(&bars->unit_empty[slot]);
   return true;
@@ -256,7 +267,8 @@ DEVI void prefill_producer(const PrefillParams& p, const CUtensorMap* mq, const 
           !mbar_wait(&bars->unit_empty[slot], ((k / kUnitRing) - 1) & 1, abort, 5))
         goto drain;
       bars->unit_idx[slot] = end ? -1 : t;
-      mbar_arrive(&bars->unit_full[slot]);  // release: the number is visible to the waiters
+      if (!end) bars->units[slot] = u;
+      mbar_arrive(&bars->unit_full[slot]);  // release: the unit is visible to the waiters
       ++k;
     }
     if (end) break;
@@ -389,10 +401,9 @@ DEVI void prefill_mma(const PrefillParams& p, uint8_t* smem, PrefillBarriers* ba
 
   for (int k = 0;; ++k) {
     int t;
-    if (!take_unit(bars, k, t, 9)) goto drain;
-    if (t < 0) break;
     PrefillUnit u;
-    prefill_unit(p, t, u);
+    if (!take_unit(bars, k, t, u, 9)) goto drain;
+    if (t < 0) break;
     const int n = u.kt1 - u.kt0;
     if (n <= 0) continue;
     if (!warp_wait(&bars->q_full, nq & 1, abort, 10)) goto drain;
@@ -466,10 +477,9 @@ DEVI void prefill_convert(const PrefillParams& p, uint8_t* smem, PrefillBarriers
   int it = 0;
   for (int k = 0;; ++k) {
     int wu;
-    if (!take_unit(bars, k, wu, 52)) return;
-    if (wu < 0) break;
     PrefillUnit u;
-    prefill_unit(p, wu, u);
+    if (!take_unit(bars, k, wu, u, 52)) return;
+    if (wu < 0) break;
     const int n = u.kt1 - u.kt0;
     for (int j = 0; j < n; ++j, ++it) {
       const int sv = it % C::kVStages, sh = it % C::kVHStages;
@@ -722,10 +732,9 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
   int sj = 0, units = 0;
   for (int k = 0;; ++k) {
     int t;
-    if (!take_unit(bars, k, t, 24 + w)) return;
-    if (t < 0) break;
     PrefillUnit u;
-    prefill_unit(p, t, u);
+    if (!take_unit(bars, k, t, u, 24 + w)) return;
+    if (t < 0) break;
     const int n = u.kt1 - u.kt0;
     const int i = u.m * kPrefillUnit + w * kPrefillBM + r;
     const bool valid = i < u.len_q;
@@ -785,15 +794,26 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
     const float denom = row.l_rnd + (has_sink ? ex2(sink2 - m_use) : 0.f);
     const float inv = (denom > 0.f && row.seen) ? v_scale / denom : 0.f;
     if (valid) {
+      constexpr bool kOutF16 = kType == 1;
+      auto word = [&](int c) {
+        return pack2<kOutF16>(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
+      };
+      // Each thread writes its own row: 32-byte stores where the row allows
+      // (half the store transactions of 16-byte ones), else 16-byte ones.
+      if ((reinterpret_cast<uintptr_t>(orow) & 31u) == 0) {
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        uint4 v;
-        constexpr bool kOutF16 = kType == 1;
-        v.x = pack2<kOutF16>(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-        v.y = pack2<kOutF16>(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-        v.z = pack2<kOutF16>(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-        v.w = pack2<kOutF16>(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-        reinterpret_cast<uint4*>(orow)[c] = v;
+        for (int c = 0; c < D / 16; ++c)
+          asm volatile(
+              "st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(orow + 16 * c),
+              "r"(word(8 * c)), "r"(word(8 * c + 1)), "r"(word(8 * c + 2)), "r"(word(8 * c + 3)),
+              "r"(word(8 * c + 4)), "r"(word(8 * c + 5)), "r"(word(8 * c + 6)),
+              "r"(word(8 * c + 7))
+              : "memory");
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c)
+          reinterpret_cast<uint4*>(orow)[c] =
+              make_uint4(word(4 * c), word(4 * c + 1), word(4 * c + 2), word(4 * c + 3));
       }
       if (lrow) *lrow = row.l_run > 0.f ? (m_use + log2f(row.l_run)) * kLn2 : -INFINITY;
     }
