@@ -19,7 +19,8 @@ namespace {
 // ---------------------------------------------------------------------------
 template <int D, int kType, bool kMask>
 attn_status_t launch_prefill(int grid, const CUtensorMap& mq, const CUtensorMap& mk,
-                             const CUtensorMap& mv, const PrefillParams& p, cudaStream_t stream) {
+                             const CUtensorMap& mv, const CUtensorMap& mo, const PrefillParams& p,
+                             cudaStream_t stream) {
   using C = PrefillCfg<D, kType>;
   auto kernel = prefill_kernel<D, kType, kMask>;
   static std::atomic<uint64_t> configured{0};
@@ -35,7 +36,7 @@ attn_status_t launch_prefill(int grid, const CUtensorMap& mq, const CUtensorMap&
   if (p.work_counter &&
       cudaMemsetAsync(p.work_counter, 0, sizeof(int32_t), stream) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+  kernel<<<grid, kPrefillThreads, C::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
   return launch_status(cudaGetLastError());
 }
 
@@ -54,13 +55,20 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   const uint64_t qsb = varlen ? rows_q * a.q_stride_s : a.q_stride_b;
   const uint64_t ksb = varlen ? rows_k * a.k_stride_s : a.k_stride_b;
   const uint64_t vsb = varlen ? rows_k * a.v_stride_s : a.v_stride_b;
-  CUtensorMap mq, mk, mv;
+  // The output (TMA stores of whole 128-row tiles): bf16, or fp16 for fp16
+  // inputs; 64-column boxes.
+  const CUtensorMapDataType dto =
+      kType == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint64_t osb = varlen ? rows_q * a.o_stride_s : a.o_stride_b;
+  CUtensorMap mq, mk, mv, mo;
   if (!encode_4d(&mq, a.q, dt, es, D, a.num_heads_q, rows_q, nb, a.q_stride_h, a.q_stride_s, qsb,
                  bx, 1, 128, 1) ||
       !encode_4d(&mk, a.k, dt, es, D, a.num_heads_kv, rows_k, nb, a.k_stride_h, a.k_stride_s, ksb,
                  bx, 1, kPrefillBN, 1) ||
       !encode_4d(&mv, a.v, dt, es, D, a.num_heads_kv, rows_k, nb, a.v_stride_h, a.v_stride_s, vsb,
-                 bx, 1, kPrefillBN, 1))
+                 bx, 1, kPrefillBN, 1) ||
+      !encode_4d(&mo, a.out, dto, 2, D, a.num_heads_q, rows_q, nb, a.o_stride_h, a.o_stride_s, osb,
+                 64, 1, kPrefillBM, 1))
     return ATTN_ERR_INVALID_ARG;
 
   PrefillParams p;
@@ -105,8 +113,8 @@ attn_status_t run_prefill(const attn_varlen_args& a, cudaStream_t stream) {
   const int grid = (int)std::min<int64_t>(total, sms);
   // The additive-mask path is a separate instantiation, so the common path
   // carries none of its registers.
-  return a.mask ? launch_prefill<D, kType, true>(grid, mq, mk, mv, p, stream)
-                : launch_prefill<D, kType, false>(grid, mq, mk, mv, p, stream);
+  return a.mask ? launch_prefill<D, kType, true>(grid, mq, mk, mv, mo, p, stream)
+                : launch_prefill<D, kType, false>(grid, mq, mk, mv, mo, p, stream);
 }
 
 attn_status_t check_varlen(const attn_varlen_args* a) {

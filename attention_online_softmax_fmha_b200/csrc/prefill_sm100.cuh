@@ -104,7 +104,7 @@ struct PrefillCfg {
   static constexpr int kChunks = D * kInBytes / 128;     // 128-byte column chunks
   // K and V tiles have separate rings: K is released as soon as both S MMAs
   // have read it, V after both P V MMAs (FP8: after the conversion).
-  static constexpr int kKStages = kFp8 ? 4 : ((D == 64) ? 4 : 3);
+  static constexpr int kKStages = kFp8 ? 4 : ((D == 64) ? 4 : 2);
   static constexpr int kVStages = (D == 64) ? 4 : 2;
   static constexpr int kVHStages = kFp8 ? 2 : 0;         // fp16 copies of V (FP8)
   static constexpr int kChunkBytes = 128 * 128;          // 128 rows x 128 bytes
@@ -114,7 +114,12 @@ struct PrefillCfg {
   static constexpr int kKOff = 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kKStages * kTileBytes;
   static constexpr int kVHOff = kVOff + kVStages * kTileBytes;
-  static constexpr int kBarOff = kVHOff + kVHStages * kVHBytes;
+  // The output staging tile: 128 rows of D 16-bit values in 64-column chunks,
+  // the box layout of the output tensor map (TMA store).
+  static constexpr int kOutChunks = D / 64;
+  static constexpr int kOStageOff = kVHOff + kVHStages * kVHBytes;
+  static constexpr int kOStageBytes = kOutChunks * kChunkBytes;
+  static constexpr int kBarOff = kOStageOff + kOStageBytes;
   static constexpr int kBarBytes = 1024;
   static constexpr int kSmemBytes = kBarOff + kBarBytes;
   // The dynamic shared memory base is 1024-byte aligned (the kernel checks).
@@ -145,6 +150,13 @@ struct PrefillBarriers {
   uint64_t k_full[4], v_full[4], k_empty[4], v_empty[4];
   uint64_t vh_full[4], vh_empty[4];
   uint64_t s_full[2], p_head[2], p_full[2], o_full[2], o_empty[2];
+  // The output staging tile, used by the two softmax warpgroups in turn
+  // (use u = 2 * unit + warpgroup): full once all 128 rows are written,
+  // free once the TMA store has read it.
+  uint64_t ostage_full, ostage_free;
+  // What the staged tile is: whether to store it, and its box coordinates
+  // (written by the warpgroup's first thread before it arrives).
+  int32_t ostage_store, ostage_c1, ostage_c2, ostage_c3;
   uint64_t mma_drain;
   uint32_t tmem_base;
   int32_t abort;
@@ -518,6 +530,15 @@ DEVI void prefill_convert(const PrefillParams& p, uint8_t* smem, PrefillBarriers
 // (= TMEM lane r). The two warpgroups run offset by about half a tile, so one
 // exponentiates while the other waits for its next S.
 // ---------------------------------------------------------------------------
+// TMA store of one box from shared memory (the tensor map's swizzled layout).
+DEVI void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 struct PrefillRow {
   float m_run;  // running max (log2 domain, includes the sink)
   float l_run;  // sum of the fp32 P (for the LSE)
@@ -721,7 +742,8 @@ DEVI bool prefill_softmax_tile(const Sig& sig, uint32_t s_tmem, uint32_t o_tmem,
 }
 
 template <int D, int kType, bool kMask>
-DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_t tmem, int w) {
+DEVI void prefill_softmax(const PrefillParams& p, const CUtensorMap* mo, uint8_t* smem,
+                          PrefillBarriers* bars, uint32_t tmem, int w) {
   using C = PrefillCfg<D, kType>;
   using OutT = typename std::conditional<kType == 1, __half, __nv_bfloat16>::type;
   volatile int* abort = &bars->abort;
@@ -730,6 +752,49 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
   const uint32_t s_tmem = tmem + (w ? C::kTmemS1 : C::kTmemS0) + lane;
   const uint32_t o_tmem = tmem + (w ? C::kTmemO1 : C::kTmemO0) + lane;
   int sj = 0, units = 0;
+  // The output goes out through the staging tile, one warpgroup at a time
+  // (use number ouse = 2 * unit + w): a tile whose 128 rows all belong to
+  // the sequence is written there and stored by TMA (one thread, in the
+  // background); other rows are stored directly. Every unit takes its turn,
+  // so the two warpgroups alternate.
+  int ouse = w;
+  auto turn_begin = [&]() -> bool {
+    return ouse < 1 || warp_wait(&bars->ostage_free, (ouse - 1) & 1, abort, 26 + w);
+  };
+  auto turn_end = [&](bool staged, const PrefillUnit& u, int i0) -> bool {
+    if (staged) fence_proxy_async_smem();  // the TMA store reads through the async proxy
+    if constexpr (!C::kFp8) {
+      // 16-bit inputs: the store warp issues the TMA store and passes the turn on
+      if (r == 0) {
+        bars->ostage_store = staged ? 1 : 0;
+        bars->ostage_c1 = u.h;
+        bars->ostage_c2 = u.row_q + i0;
+        bars->ostage_c3 = u.bcoord;
+      }
+      mbar_arrive(&bars->ostage_full);
+      ouse += 2;
+      return true;
+    }
+    mbar_arrive(&bars->ostage_full);
+    bool ok = true;
+    if (r < 32) {  // warp 0 of the warpgroup; its lane 0 stores and passes the turn on
+      if (r == 0) {
+        ok = mbar_wait(&bars->ostage_full, ouse & 1, abort, 28 + w);
+        if (ok && staged) {
+#pragma unroll
+          for (int c = 0; c < C::kOutChunks; ++c)
+            tma_store_4d(mo, smem + C::kOStageOff + c * C::kChunkBytes, c * 64, u.h, u.row_q + i0,
+                         u.bcoord);
+          bulk_commit();
+          bulk_wait_read<0>();  // the staging tile has been read
+        }
+        if (ok) mbar_arrive(&bars->ostage_free);
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    ouse += 2;
+    return ok;
+  };
   for (int k = 0;; ++k) {
     int t;
     PrefillUnit u;
@@ -742,12 +807,14 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
                  (int64_t)(u.row_q + i) * p.o_ss + (int64_t)u.h * p.o_sh;
     float* lrow = p.lse ? p.lse + u.b * p.lse_sb + u.h * p.lse_sh + (u.row_q + i) : nullptr;
     if (n <= 0) {
+      if (!turn_begin()) return;
       if (valid) {
         const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
         if (lrow) *lrow = -INFINITY;
       }
+      if (!turn_end(false, u, 0)) return;
       continue;
     }
     float sl2 = p.scale_log2;
@@ -793,38 +860,80 @@ DEVI void prefill_softmax(const PrefillParams& p, PrefillBarriers* bars, uint32_
     const float m_use = (row.m_run == -INFINITY) ? 0.f : row.m_run;
     const float denom = row.l_rnd + (has_sink ? ex2(sink2 - m_use) : 0.f);
     const float inv = (denom > 0.f && row.seen) ? v_scale / denom : 0.f;
+    constexpr bool kOutF16 = kType == 1;
+    auto word = [&](int c) {
+      return pack2<kOutF16>(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
+    };
+    const int i0 = i - r;
+    const bool staged = i0 + kPrefillBM <= u.len_q;
+    if (!turn_begin()) return;
+    if (staged) {
+      // row r into the staging tile: 64-column chunks, 16-byte pieces
+      // permuted by row (the 128-byte swizzle of the tensor map)
+      uint8_t* srow = smem + C::kOStageOff + r * 128;
+#pragma unroll
+      for (int c = 0; c < C::kOutChunks; ++c)
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+          *reinterpret_cast<uint4*>(srow + c * C::kChunkBytes + ((x ^ (r & 7)) << 4)) =
+              make_uint4(word(32 * c + 4 * x), word(32 * c + 4 * x + 1),
+                         word(32 * c + 4 * x + 2), word(32 * c + 4 * x + 3));
+    } else if (valid) {
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c)
+        reinterpret_cast<uint4*>(orow)[c] =
+            make_uint4(word(4 * c), word(4 * c + 1), word(4 * c + 2), word(4 * c + 3));
+    }
+    if (!turn_end(staged, u, i0)) return;
     if (valid) {
-      constexpr bool kOutF16 = kType == 1;
-      auto word = [&](int c) {
-        return pack2<kOutF16>(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
-      };
-      // Each thread writes its own row: 32-byte stores where the row allows
-      // (half the store transactions of 16-byte ones), else 16-byte ones.
-      if ((reinterpret_cast<uintptr_t>(orow) & 31u) == 0) {
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c)
-          asm volatile(
-              "st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(orow + 16 * c),
-              "r"(word(8 * c)), "r"(word(8 * c + 1)), "r"(word(8 * c + 2)), "r"(word(8 * c + 3)),
-              "r"(word(8 * c + 4)), "r"(word(8 * c + 5)), "r"(word(8 * c + 6)),
-              "r"(word(8 * c + 7))
-              : "memory");
-      } else {
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-          reinterpret_cast<uint4*>(orow)[c] =
-              make_uint4(word(4 * c), word(4 * c + 1), word(4 * c + 2), word(4 * c + 3));
-      }
       if (lrow) *lrow = row.l_run > 0.f ? (m_use + log2f(row.l_run)) * kLn2 : -INFINITY;
     }
   }
+  if (r == 0) bulk_wait_all();  // this warpgroup's output stores have completed
+}
+
+// 16-bit inputs only: the output store warp (warp 10, one thread). For every
+// unit, in the softmax warpgroups' order of turns (warpgroup 0, then 1), it
+// waits for the staged tile, stores it with TMA when it is a whole tile,
+// waits until the stores have read the staging tile and passes the turn on.
+// The softmax warps never wait on the store.
+template <int D, int kType>
+DEVI void prefill_store(const PrefillParams& p, const CUtensorMap* mo, uint8_t* smem,
+                        PrefillBarriers* bars) {
+  using C = PrefillCfg<D, kType>;
+  volatile int* abort = &bars->abort;
+  int ouse = 0;
+  for (int k = 0;; ++k) {
+    const int slot = k % kUnitRing;
+    if (!mbar_wait(&bars->unit_full[slot], (k / kUnitRing) & 1, abort, 29)) break;
+    const int t = *reinterpret_cast<volatile int32_t*>(&bars->unit_idx[slot]);
+    mbar_arrive(&bars->unit_empty[slot]);
+    if (t < 0) break;
+    bool ok = true;
+    for (int w = 0; w < 2 && ok; ++w, ++ouse) {
+      ok = mbar_wait(&bars->ostage_full, ouse & 1, abort, 30);
+      if (!ok) break;
+      if (*reinterpret_cast<volatile int32_t*>(&bars->ostage_store)) {
+        const int c1 = bars->ostage_c1, c2 = bars->ostage_c2, c3 = bars->ostage_c3;
+#pragma unroll
+        for (int c = 0; c < C::kOutChunks; ++c)
+          tma_store_4d(mo, smem + C::kOStageOff + c * C::kChunkBytes, c * 64, c1, c2, c3);
+        bulk_commit();
+        bulk_wait_read<0>();  // the staging tile has been read
+      }
+      mbar_arrive(&bars->ostage_free);
+    }
+    if (!ok) break;
+  }
+  bulk_wait_all();
 }
 
 template <int D, int kType, bool kMask>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_k,
-                   const __grid_constant__ CUtensorMap map_v, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap map_v,
+                   const __grid_constant__ CUtensorMap map_o, const PrefillParams p) {
   using C = PrefillCfg<D, kType>;
   // 128-byte swizzled TMA tiles need 1024-byte aligned shared memory. The
   // layout leaves no slack for aligning at run time (the tiles take 224 KB),
@@ -840,8 +949,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(&bars->unit_full[i], 1);
-      // released by the MMA warp, the 8 softmax warps and (FP8) the 2 conversion warps
-      mbar_init(&bars->unit_empty[i], 9 + (C::kFp8 ? 2 : 0));
+      // released by the MMA warp, the 8 softmax warps and the 2 conversion
+      // warps (FP8) or the output store warp (16-bit inputs)
+      mbar_init(&bars->unit_empty[i], 9 + (C::kFp8 ? 2 : 1));
     }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
@@ -864,6 +974,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(&bars->o_full[w], 1);
       mbar_init(&bars->o_empty[w], 128);
     }
+    mbar_init(&bars->ostage_full, 128);
+    mbar_init(&bars->ostage_free, 1);
     mbar_init(&bars->mma_drain, 1);
     bars->abort = 0;
     fence_barrier_init();
@@ -879,7 +991,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   if (warp < 8) {
     regs_inc<kPrefillSoftmaxRegs>();
-    prefill_softmax<D, kType, kMask>(p, bars, tmem, warp >> 2);
+    prefill_softmax<D, kType, kMask>(p, &map_o, smem, bars, tmem, warp >> 2);
   } else {
     regs_dec<kPrefillOtherRegs>();
     if (warp == 8) {
@@ -888,6 +1000,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       prefill_mma<D, kType, kMask>(p, smem, bars, tmem);  // whole warp, one lane issues
     } else if constexpr (C::kFp8) {
       prefill_convert<D, kType>(p, smem, bars);
+    } else if (warp == 10) {
+      if (elect_lane0()) prefill_store<D, kType>(p, &map_o, smem, bars);
     }
   }
 
