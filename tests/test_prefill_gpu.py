@@ -271,3 +271,24 @@ def test_repeated_runs_are_bitwise_identical(dtype):
     for _ in range(15):
         o, l = B_fwd(inp.q, inp.k, inp.v, **kw)
         assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
+
+
+def test_strided_output_view():
+    """Output written through a strided view (padding after every head's D
+    values and a padding head after every row): equal bit for bit to the
+    packed output, and the padding is untouched. Whole 128-row tiles go out
+    by TMA store through a tensor map of the view's strides, ragged tiles by
+    direct stores; both must follow the strides."""
+    lens = [300, 128, 513]
+    inp = W.make_prefill(seqlens_q=lens, num_heads_q=8, num_heads_kv=2, head_dim=128,
+                         varlen=True, causal=True, seed=97, device="cuda")
+    kw = dict(scale=inp.scale, causal=True, cu_seqlens_q=inp.cu_seqlens_q,
+              cu_seqlens_k=inp.cu_seqlens_k, max_seqlen_q=max(lens), max_seqlen_k=max(lens))
+    ref_o, ref_l = B_fwd(inp.q, inp.k, inp.v, **kw)
+    T = inp.q.shape[0]
+    big = torch.full((T, 9, 192), float("nan"), dtype=torch.bfloat16, device="cuda")
+    view = big[:, :8, :128]
+    o, l = B_fwd(inp.q, inp.k, inp.v, out=view, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(view, ref_o) and torch.equal(l, ref_l)
+    assert torch.isnan(big[:, :8, 128:]).all() and torch.isnan(big[:, 8:, :]).all()
