@@ -13,9 +13,9 @@
 // heaviest first (last row block of every sequence and head first); with a
 // work counter each CTA takes the next number when it starts a unit, so
 // CTAs that drew short units take more of them, otherwise every
-// gridDim-th number. The producer takes the numbers and hands them to the
-// other roles through a small ring in shared memory. Both tiles stream the
-// same K/V tiles of 128 keys.
+// gridDim-th number. The producer takes the numbers, decodes the units and
+// hands both to the other roles through a small ring in shared memory. Both
+// tiles stream the same K/V tiles of 128 keys.
 //   warpgroup 0, 1   softmax of Q0 / Q1: thread r owns query row r of its
 //                    tile (= TMEM lane r). Online softmax in the log2 domain;
 //                    O in TMEM is rescaled only when a row's max grows by more
@@ -28,8 +28,11 @@
 //                    runs. S_w = Q_w K^T lands in TMEM; P_w (bf16) overwrites
 //                    it and is the TMEM A operand of O_w += P_w V, started on
 //                    the first 96 keys while the last 32 are exponentiated.
-//   warps 10, 11     FP8 only: convert each e4m3 V tile to fp16 for P V;
-//                    otherwise idle (they complete the register warpgroup).
+//   warps 10, 11     FP8: convert each e4m3 V tile to fp16 for P V. 16-bit
+//                    inputs: warp 10 issues the output TMA stores, warp 11
+//                    is idle (they complete the register warpgroup).
+// Output: whole 128-row tiles go through a shared-memory staging tile and a
+// TMA store, ragged tiles are stored directly by their threads.
 // Registers move from warpgroup 2 to the softmax warpgroups with setmaxnreg;
 // the host checks the kernel's register count before launching.
 // Every mbarrier wait is bounded; a timeout raises ATTN_DEVERR_TIMEOUT and the
