@@ -648,7 +648,7 @@ struct PrefillSig {
 template <int D, int kType, bool kMask, class Sig>
 DEVI bool prefill_softmax_tile(const Sig& sig, uint32_t s_tmem, uint32_t o_tmem, int j, int g,
                                int k0, float sl2, PrefillRow& row, const float* mrow, int len_k,
-                               bool split) {
+                               bool few, bool split) {
   if (!sig.wait_s(g)) return false;
   tc_fence_after();
   uint32_t s[kPrefillBN];
@@ -734,10 +734,12 @@ DEVI bool prefill_softmax_tile(const Sig& sig, uint32_t s_tmem, uint32_t o_tmem,
   // O is normalised by the sum of the rounded P the MMA consumes (the
   // weights then stay a convex combination and the rounding error scales
   // with the spread of V, not with |O|); the LSE uses the fp32 sum. The
-  // difference matters only for rows with few visible keys, whose keys all
-  // lie in first or partially masked tiles; other tiles add their fp32 sum to
-  // both (their rounding errors average out over the row's many keys).
-  if (j == 0 || kMask || split || __any_sync(0xffffffffu, partial))
+  // difference matters only for rows with few visible keys (fewer than
+  // kShortRow): tiles that hold such a row, first tiles and masked tiles add
+  // the rounded sum; other tiles, diagonal and window-edge tiles of long rows
+  // included, add their fp32 sum to both (their rounding errors average out
+  // over the row's many keys).
+  if (j == 0 || kMask || few)
     prefill_exp_tile<kType, true>(sig, s_tmem, sl2, s, row, split);
   else
     prefill_exp_tile<kType, false>(sig, s_tmem, sl2, s, row, false);
@@ -838,11 +840,12 @@ DEVI void prefill_softmax(const PrefillParams& p, const CUtensorMap* mo, uint8_t
     row.seen = false;
     const float* mrow =
         (kMask && valid) ? p.mask + u.b * p.m_sb + u.h * p.m_sh + (int64_t)i * p.m_ss : nullptr;
-    const bool split = kType == 0 && !kMask && prefill_short_tile(p, u, w);
+    const bool few = !kMask && prefill_short_tile(p, u, w);
+    const bool split = kType == 0 && few;
     for (int j = 0; j < n; ++j, ++sj)
       if (!prefill_softmax_tile<D, kType, kMask>(PrefillSig{bars, w}, s_tmem, o_tmem, j, sj,
                                                  (u.kt0 + j) * kPrefillBN, sl2, row, mrow,
-                                                 u.len_k, split))
+                                                 u.len_k, few, split))
         return;
     // Epilogue: wait for the last P V, read O, release O, normalise, store.
     if (!warp_wait(&bars->o_full[w], units & 1, abort, 22 + w)) return;
