@@ -38,6 +38,21 @@ def test_every_declared_function_is_exported(L):
         assert hasattr(L, n)
 
 
+def test_enum_values_match_the_header():
+    """The binding's status, device-error and scheduler-mode constants are the
+    header's enum values."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    vals = {k: int(v) for k, v in re.findall(r"\b(ATTN_\w+)\s*=\s*(\d+)", src)}
+    pairs = {"ATTN_OK": B.OK, "ATTN_ERR_DEVICE": B.DEVICE_ERROR,
+             "ATTN_DEVERR_TIMEOUT": B.DEVERR_TIMEOUT,
+             "ATTN_DEVERR_META_MISMATCH": B.DEVERR_META_MISMATCH,
+             "ATTN_DEVERR_SMEM_ALIGN": B.DEVERR_SMEM_ALIGN,
+             "ATTN_DEVERR_UNITS_OVERFLOW": B.DEVERR_UNITS_OVERFLOW,
+             "ATTN_SCHED_MHA": B.SCHED_MHA, "ATTN_SELFTEST_SITE": B.SELFTEST_SITE}
+    for name, value in pairs.items():
+        assert vals[name] == value, name
+
+
 def test_struct_mirrors_match(L):
     for which, cls in B.ARG_STRUCTS.items():
         assert L.attn_args_sizeof(which) == ctypes.sizeof(cls), cls.__name__
